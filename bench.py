@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA core on B200.
+
+Workload (one step = one pass of the prefill hot path over one batch): B=1 sequence of
+T=4096 tokens, H=32 heads, head_dim 128, 64-token chunks, BF16-exact inputs widened to
+FP32, initial state N(0, 0.1): kda_gate (g_raw -> gate), kda_beta (b_logit -> beta) and
+kda_chunk_prefill (q, k, v, gate, beta, state -> core, state). Inputs are resident in
+HBM; L2 is flushed (a 512 MB write) before every timed step, outside the timed events.
+Multi-GPU: each rank runs its own independent sequence (weak scaling, no collective).
+
+Also reported: the dominant kernel's roofline (CUDA events around each launch), a decode
+leg (256 sequences x 1 token, kda_decode_fused, state GB/s), an end-to-end leg through
+the same C-ABI calls from pinned host buffers (copies inside the timed region), and the
+FP64 oracle timed on the host cores (`cpu_baseline`). `--impl reference` times the oracle
+alone (it is this project's reference implementation) and prints its own line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (% tensor-core roofline); decode state GB/s (% of HBM peak)"
+B, T, H, D = 1, 4096, 32, 128
+CONFIG = {"workload": "kda_chunk_prefill B1 T4096 H32 D128 chunk64 (gate+beta+chunked core), FP32 I/O",
+          "global_batch": B, "seq_len": T, "heads": H, "head_dim": D, "chunk": 64,
+          "l2": "flushed before every timed step (512 MB write)"}
+# Algorithmic work per token-head: q, k, v, gate, core at D FP32 values each + beta.
+BYTES_PER_TOKEN_HEAD = 5 * D * 4 + 4
+FLOPS_PER_TOKEN_HEAD = 139_000  # L, M, WY/UT solve, W.S, Q.S, M.U, K^T.U at C=64, D=128 (triangles as half)
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _src_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f).get(kernel_key)
+    if not j or j.get("src_sha") != _src_sha(j["src"]):
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(1.0)  # nvidia-smi start-up; the first sample lands before the warm-up
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r.split(",") for r in (getattr(self, "out", "") or "").strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _oracle_baseline(T_sample):
+    """The FP64 oracle (as it stands) on the first T_sample tokens of the workload: gate,
+    sigmoid and the token recurrence for all 32 heads, on all host cores."""
+    import oracle
+    from synth import core_inputs
+    ci = core_inputs(1, T_sample, H, D, seed=1, bf16_inputs=True, s0_std=0.1)
+    cores = oracle.default_threads()
+    oracle.build()
+    t0 = time.perf_counter()
+    g = oracle.gate(ci.g_raw.float(), ci.dt_bias, ci.a_log, H, D)
+    beta = oracle.sigmoid(ci.b_logit)
+    oracle.recurrence(ci.q, ci.k, ci.v, g, beta, ci.s0, 1.0, cores)
+    dt = time.perf_counter() - t0
+    return T_sample / dt, dt, cores
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    T_sample = 512
+    times = []
+    for i in range(args.warmup + args.steps):
+        tps, dt, cores = _oracle_baseline(T_sample)
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1000.0 * sum(times) / len(times)
+    value = T_sample / (ms / 1000.0)
+    sample = f"oracle on the first {T_sample} tokens of the T=4096 sequence, all 32 heads, per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": CONFIG,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill-impl", default="tc", choices=["tc", "simt"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import torch
+    import torch.distributed as dist
+    import kda_gated_delta_gate_b200 as kda
+    from synth import core_inputs, pad_rows, t_pad
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    kda.lib()
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    d = kda.dims(H, D)
+    Tp = t_pad(T)
+
+    # ---- inputs resident in HBM (each rank its own sequence: seed differs by rank)
+    ci = core_inputs(B, T, H, D, seed=1 + 1000 * rank, bf16_inputs=True, s0_std=0.1)
+    q = pad_rows(ci.q, Tp, 0.0).to(dev)
+    k = pad_rows(ci.k, Tp, 0.0).to(dev)
+    v = pad_rows(ci.v, Tp, 0.0).to(dev)
+    g_raw = pad_rows(ci.g_raw, Tp, 0.0).to(dev)
+    b_logit = pad_rows(ci.b_logit, Tp, 0.0).to(dev)
+    dt_bias, a_log = ci.dt_bias.to(dev), ci.a_log.to(dev)
+    gate = torch.empty((B * Tp, H, D), device=dev)
+    beta = torch.empty((B * Tp, H), device=dev)
+    core = torch.empty((B * Tp, H, D), device=dev)
+    state = ci.s0[0].to(dev).clone()
+    ptrs = kda.ptr_array([state], device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def step(kev=None):
+        kda.kda_gate(g_raw, dt_bias, a_log, gate, B * T, d, s)
+        kda.kda_beta(b_logit, beta, B * T * H, s)
+        if kev:
+            kev[0].record(stream)
+        kda.kda_chunk_prefill(q, k, v, gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl)
+        if kev:
+            kev[1].record(stream)
+        return 3
+
+    launches = 0
+    with Clocks(local) as clk:
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            ev_s[i][0].record(stream)
+            launches += step(ev_k[i])
+            ev_s[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev_s) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev_k) / args.steps
+    if world > 1:
+        t = torch.tensor([step_ms, kern_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, kern_ms = t.tolist()
+
+    hbm, tc_peak, peak_kind = _peaks()
+    alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
+    alg_flops = B * T * H * FLOPS_PER_TOKEN_HEAD
+    achieved_gbs = alg_bytes / (kern_ms * 1e-3) / 1e9
+    achieved_tf = alg_flops / (kern_ms * 1e-3) / 1e12
+
+    # ---- decode leg: 256 sequences x 1 token, fused stateful row (state GB/s)
+    dec = _decode_leg(kda, torch, dev, s, stream, flush, hbm)
+
+    # ---- end-to-end leg: the same C-ABI calls from pinned host buffers, copies timed
+    e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world)
+
+    result = None
+    if rank == 0:
+        tokens_per_s = world * B * T / (step_ms * 1e-3)
+        cpu = None
+        if not args.no_cpu_baseline:
+            tps, dt, cores = _oracle_baseline(1024)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"FP64 oracle (gate, sigmoid, token recurrence, 32 heads) on the first 1024 tokens "
+                             f"of the workload; {dt:.1f} s wall"}
+        result = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": dict(CONFIG, parallelism=f"dp{world}",
+                                                                                     prefill_impl=args.prefill_impl),
+            "roofline": {"kernel": "kda_chunk_prefill", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved_gbs / hbm, "peak_kind": peak_kind,
+                         "traffic": _traffic("chunk_prefill_" + args.prefill_impl),
+                         "kernel_ms": kern_ms, "alg_bytes_per_launch": alg_bytes,
+                         "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                                    "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
+            "decode": dec,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _decode_leg(kda, torch, dev, s, stream, flush, hbm):
+    from synth import decode_inputs
+    N = 256
+    di = decode_inputs(N, H, D, seed=3, device="cpu")
+    dd = kda.dims(H, D)
+    x, cw, gr = di.x.to(dev), di.conv_w.to(dev), di.g_raw.to(dev)
+    dtb, al, bl, og, ow = di.dt_bias.to(dev), di.a_log.to(dev), di.b_logit.to(dev), di.out_gate.to(dev), di.o_norm.to(dev)
+    cs = [di.conv_state[n].to(dev).clone() for n in range(N)]
+    hs = [di.s0[n].to(dev).clone() for n in range(N)]
+    cp, hp = kda.ptr_array(cs, device=dev), kda.ptr_array(hs, device=dev)
+    out = torch.empty((N, H * D), dtype=torch.bfloat16, device=dev)
+    times = []
+    for i in range(25):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        kda.kda_decode_fused(x, cp, cw, gr, dtb, al, bl, hp, og, ow, out, None, None, N, dd, s)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 5:
+            times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    state_bytes = N * H * D * D * 4 * 2
+    all_bytes = state_bytes + N * (3 * H * D * 2 + 3 * H * D * 3 * 2 * 2 + H * D * 2 * 3 + H * 4)
+    return {"workload": "kda_decode_fused 256 seqs x 1 token, H32 D128 (conv+gate+beta+recurrence+o_norm)",
+            "ms": ms, "tokens_per_s": N / (ms * 1e-3), "state_gbs": state_bytes / (ms * 1e-3) / 1e9,
+            "all_gbs": all_bytes / (ms * 1e-3) / 1e9, "hbm_peak_gbs": hbm,
+            "frac_hbm": all_bytes / (ms * 1e-3) / 1e9 / hbm}
+
+
+def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world):
+    from synth import pad_rows
+    host = {n: pad_rows(getattr(ci, n), Tp, 0.0).pin_memory() for n in ("q", "k", "v", "g_raw", "b_logit")}
+    host["s0"] = ci.s0[0].clone().pin_memory()
+    dv = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    dt_bias, a_log = ci.dt_bias.to(dev), ci.a_log.to(dev)
+    gate = torch.empty((B * Tp, H, D), device=dev)
+    beta = torch.empty((B * Tp, H), device=dev)
+    core = torch.empty((B * Tp, H, D), device=dev)
+    core_h = torch.empty_like(core, device="cpu").pin_memory()
+    s_h = torch.empty_like(host["s0"]).pin_memory()
+    ptrs = kda.ptr_array([dv["s0"]], device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = core_h.numel() * 4 + s_h.numel() * 4
+
+    def one():
+        for n, t in host.items():
+            dv[n].copy_(t, non_blocking=True)
+        kda.kda_gate(dv["g_raw"], dt_bias, a_log, gate, B * T, d, s)
+        kda.kda_beta(dv["b_logit"], beta, B * T * H, s)
+        kda.kda_chunk_prefill(dv["q"], dv["k"], dv["v"], gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl)
+        core_h.copy_(core, non_blocking=True)
+        s_h.copy_(dv["s0"], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(3, args.steps // 2)
+    a.record(stream)
+    for _ in range(n):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    return {"value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,218 @@
+/*
+ * kda.h — C ABI of the B200 (sm_100a) KDA core library, libkda.so.
+ *
+ * The KDA core of a GLM-5.3-Next linear-attention block: per head and token, a
+ * per-channel bounded log-decay gate, a sigmoid beta, a delta-rule update of a
+ * head_dim x head_dim FP32 state and the read-out o = scale * S^T q; run as a chunked
+ * prefill (64-token chunks, padded, guarded past T) or as a one-token / K-token decode.
+ *
+ * Sources (page title, section):
+ *   Glm5NextKdaWorkspace — the stage buffers, their shapes and precisions;
+ *   Glm5NextKdaLayer     — decode, decode_k (snapshots), prefill, prefill_with_pad_fill;
+ *   Glm5NextLayer        — prefill_gdn_full_batched (equal-length streams, a device array
+ *                          of one state pointer per stream);
+ *   Glm5NextKdaWeights   — weight layouts: Linear [out, in] BF16, conv [conv_dim, 4],
+ *                          dt_bias [heads*head_dim] F32 (per channel), a_log [heads] F32
+ *                          (per head), o_norm [head_dim] BF16.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller unless a comment says "host".
+ *     Nothing is allocated on these calls (the workspace is sized once, at creation).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls are asynchronous: they enqueue kernels and return.
+ *   - Return value: KDA_OK, or an error code from the list below. Argument errors are
+ *     found on the host before anything is launched; on such an error nothing runs.
+ *     KDA_ERR_CUDA reports a launch error (cudaGetLastError after the launch).
+ *     Errors found on the device (a bounded wait that gave up) are latched into a
+ *     device status word that kda_device_status() reads.
+ *   - BF16 tensors are passed as their 16-bit patterns (kda_bf16).
+ *   - Row-major layouts. "[T_pad, H, D]" means T_pad rows of H*D contiguous values.
+ *   - Every FP32 / BF16 tensor pointer must be 16-byte aligned (vector loads/stores);
+ *     otherwise KDA_ERR_MISALIGNED.
+ *   - Dimensions: head_dim D in {64, 128}; chunk = 64; heads H >= 1.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null pointer, negative or zero size, bad count      */
+    KDA_ERR_ALIAS = 2,        /* two buffers that must not overlap do (g_raw/out_gate) */
+    KDA_ERR_CAPACITY = 3,     /* T beyond the workspace's max_tokens                  */
+    KDA_ERR_UNSUPPORTED = 4,  /* head_dim not 64/128, chunk not 64, K too large        */
+    KDA_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed                  */
+    KDA_ERR_TIMEOUT = 6,      /* device-side bounded wait gave up (latched)            */
+    KDA_ERR_MISALIGNED = 7    /* a tensor pointer is not 16-byte aligned               */
+};
+
+typedef uint16_t kda_bf16;
+
+/* Model dimensions, passed by host pointer to every call. */
+typedef struct kda_dims {
+    int heads;      /* H                                                   */
+    int head_dim;   /* D = dk = dv (64 or 128)                             */
+    int chunk;      /* prefill chunk length; must be 64                    */
+    float scale;    /* read-out scale: o = scale * S^T q (1.0 by default)  */
+    float l2_eps;   /* q/k L2 norm: x / sqrt(sum x^2 + l2_eps)             */
+    float rms_eps;  /* o_norm: x / sqrt(mean x^2 + rms_eps)                */
+} kda_dims;
+
+/* Library version (major*100 + minor). */
+KDA_API int kda_version(void);
+
+/* Short text for a status code (static storage, never NULL). */
+KDA_API const char *kda_status_string(int status);
+
+/* T rounded up to whole chunks: the row count of every prefill buffer ("T_pad",
+ * Glm5NextKdaWorkspace: prefill buffers padded to a whole number of chunks). */
+KDA_API size_t kda_t_pad(size_t T, int chunk);
+
+/* Read (host *out) and optionally clear the current device's latched status word.
+ * Synchronises the device. Returns KDA_OK or KDA_ERR_CUDA. */
+KDA_API int kda_device_status(int *out, int clear);
+
+/* ---------------------------------------------------------------------------------
+ * kda_gate — the bounded log-decay gate (Glm5NextKdaWorkspace, field `gate`, from
+ * field `g_raw`; Glm5NextKdaWeights, `dt_bias` per channel, `a_log` per head):
+ *     gate[t, h, d] = -exp(a_log[h]) * softplus(g_raw[t, h*D + d] + dt_bias[h*D + d])
+ *   g_raw   [n_rows, H*D] BF16
+ *   dt_bias [H*D] F32,  a_log [H] F32
+ *   gate    [n_rows, H, D] F32, written for rows 0..n_rows-1 only (a padded caller passes
+ *           the valid row count; the tail is left as it is).
+ */
+KDA_API int kda_gate(const kda_bf16 *g_raw, const float *dt_bias, const float *a_log, float *gate,
+             int n_rows, const kda_dims *dims, void *stream);
+
+/* kda_beta — beta = sigmoid(b_logit), elementwise, n values (Glm5NextKdaWorkspace,
+ * field `beta`: sigmoid(b_proj(h)) in FP32). b_logit and beta may be the same buffer. */
+KDA_API int kda_beta(const float *b_logit, float *beta, int n, void *stream);
+
+/* ---------------------------------------------------------------------------------
+ * kda_chunk_prefill — the chunked KDA core over B equal-length streams of T tokens
+ * (Glm5NextKdaLayer `prefill` / `prefill_with_pad_fill`; Glm5NextLayer
+ * `prefill_gdn_full_batched`). Stream b occupies rows [b*T_pad, b*T_pad + T_pad) of
+ * every token-major buffer, T_pad = kda_t_pad(T, 64); rows >= T of each stream are
+ * padding: they are never read into the state or the valid outputs, whatever they hold
+ * (the in-kernel guard that prefill_with_pad_fill's poison tail tests).
+ *   q, k, v   [B*T_pad, H, D] F32; q and k are used as given (already L2-normalised)
+ *   gate      [B*T_pad, H, D] F32 log-decay (kda_gate's output)
+ *   beta      [B*T_pad, H]    F32 (kda_beta's output)
+ *   h_state   DEVICE array of B device pointers, each to that stream's [H, D, D] F32
+ *             state (row = key channel, column = value channel); read as the carried
+ *             state and overwritten with the state after exactly T tokens.
+ *   core      [B*T_pad, H, D] F32 output o = scale * S^T q for rows < T (pad rows are
+ *             not written).
+ * The per-(stream, head) states must not overlap each other or any input.
+ */
+KDA_API int kda_chunk_prefill(const float *q, const float *k, const float *v, const float *gate,
+                      const float *beta, float *const *h_state, float *core, int B, int T,
+                      const kda_dims *dims, void *stream);
+
+/* kda_chunk_prefill_simt — the same contract as kda_chunk_prefill, computed by the
+ * plain FP32 CUDA-core kernel (no tensor cores). Kept as a second implementation. */
+KDA_API int kda_chunk_prefill_simt(const float *q, const float *k, const float *v, const float *gate,
+                           const float *beta, float *const *h_state, float *core, int B, int T,
+                           const kda_dims *dims, void *stream);
+
+/* ---------------------------------------------------------------------------------
+ * kda_recurrent_decode — one token for each of N independent sequences, from
+ * pre-normalised q/k (Glm5NextKdaLayer `decode`: kda_recurrent takes q/k as given):
+ *     S' = diag(exp(gate)) S;  u = beta (v - S'^T k);  S = S' + k u^T;  o = scale S^T q
+ *   q, k, v, gate [N, H, D] F32;  beta [N, H] F32
+ *   h_state   DEVICE array of N device pointers to [H, D, D] F32 states, updated in place
+ *   o         [N, H, D] F32
+ */
+KDA_API int kda_recurrent_decode(const float *q, const float *k, const float *v, const float *gate,
+                         const float *beta, float *const *h_state, float *o, int N,
+                         const kda_dims *dims, void *stream);
+
+/* ---------------------------------------------------------------------------------
+ * kda_decode_fused — the whole stateful row of the block decode for N sequences, one
+ * token each, in one kernel per (sequence, head) (Glm5NextKdaLayer `decode`: the conv
+ * fuses SiLU and L2, the recurrence reads the pre-normalised BF16 q/k, then o_norm):
+ *   conv:  y[c] = sum_{j<3} w[c,j] * state[c,j] + w[c,3] * x[c]; SiLU; per-head L2 of the
+ *          q and k channels (one BF16 rounding); state <- (state[c,1], state[c,2], x[c])
+ *   gate:  as kda_gate;  beta = sigmoid(b_logit)
+ *   core:  one recurrence step as kda_recurrent_decode
+ *   o_norm: out = core / sqrt(mean_d core^2 + rms_eps) * w_o[d] * sigmoid(out_gate) (BF16)
+ * Arguments:
+ *   x          [N, 3*H*D] BF16: the q|k|v projection rows (before the conv)
+ *   conv_state DEVICE array of N device pointers to [3*H*D, 3] BF16 (oldest -> newest),
+ *              updated in place
+ *   conv_w     [3*H*D, 4] BF16 (tap 3 multiplies the current token)
+ *   g_raw      [N, H*D] BF16;  dt_bias [H*D] F32;  a_log [H] F32;  b_logit [N, H] F32
+ *   h_state    DEVICE array of N device pointers to [H, D, D] F32 states, in place
+ *   out_gate   [N, H*D] BF16 (must not overlap g_raw: KDA_ERR_ALIAS)
+ *   o_norm_w   [D] BF16
+ *   o_norm_out [N, H*D] BF16 output
+ *   conv_out   [N, 3*H*D] BF16 output of the front end, or NULL
+ *   core       [N, H, D] F32 output before o_norm, or NULL
+ */
+KDA_API int kda_decode_fused(const kda_bf16 *x, kda_bf16 *const *conv_state, const kda_bf16 *conv_w,
+                     const kda_bf16 *g_raw, const float *dt_bias, const float *a_log,
+                     const float *b_logit, float *const *h_state, const kda_bf16 *out_gate,
+                     const kda_bf16 *o_norm_w, kda_bf16 *o_norm_out, kda_bf16 *conv_out,
+                     float *core, int N, const kda_dims *dims, void *stream);
+
+/* kda_decode_k — K rows of ONE sequence (Glm5NextKdaLayer `decode_k`): the stateful
+ * row of kda_decode_fused applied K times in order, the state carried in registers.
+ * Bit-identical to K serial kda_decode_fused calls with N = 1 (the same device code
+ * runs each row). Arguments as kda_decode_fused with N replaced by K rows of one
+ * sequence, and conv_state / h_state single device pointers. Snapshots:
+ *   n_snap     0 or K-1
+ *   h_snap     HOST array of n_snap device pointers to [H, D, D] F32, or NULL if n_snap = 0
+ *   conv_snap  HOST array of n_snap device pointers to [3*H*D, 3] BF16, or NULL
+ * snapshot t receives the (recurrent, conv) state AFTER row t, t = 0..K-2.
+ * 1 <= K <= 32 (KDA_ERR_UNSUPPORTED beyond).
+ */
+KDA_API int kda_decode_k(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w,
+                 const kda_bf16 *g_raw, const float *dt_bias, const float *a_log,
+                 const float *b_logit, float *h_state, const kda_bf16 *out_gate,
+                 const kda_bf16 *o_norm_w, kda_bf16 *o_norm_out, kda_bf16 *conv_out, float *core,
+                 int K, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
+                 const kda_dims *dims, void *stream);
+
+/* ---------------------------------------------------------------------------------
+ * kda_front_conv_silu_l2 — prefill front end for one sequence of T tokens
+ * (Glm5NextKdaWorkspace, fields `conv_out` and `q_f32`/`k_f32`/`v_f32`):
+ *   conv (as kda_decode_fused, from the carried conv state) + SiLU -> BF16 conv_out;
+ *   then l2_norm_bf16 in place on the q|k channels (per head, on the BF16 values);
+ *   then, if the F32 pointers are not NULL, q/k/v widened to [T_pad, H*D] F32 with rows
+ *   T..T_pad-1 set to pad_fill (Glm5NextKdaLayer `prefill_with_pad_fill`).
+ *   x          [T, 3*H*D] BF16 (qkv_proj)
+ *   conv_state [3*H*D, 3] BF16, carried: replaced by the last three inputs of (state || x)
+ *   conv_w     [3*H*D, 4] BF16
+ *   conv_out   [T, 3*H*D] BF16 output
+ *   q_f32, k_f32, v_f32  [T_pad, H*D] F32 outputs, all three or none (NULL)
+ */
+KDA_API int kda_front_conv_silu_l2(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w,
+                           kda_bf16 *conv_out, float *q_f32, float *k_f32, float *v_f32,
+                           float pad_fill, int T, const kda_dims *dims, void *stream);
+
+/* kda_back_gated_rmsnorm — the sigmoid-gated RMSNorm over head_dim (Glm5NextKdaWorkspace,
+ * field `o_norm_out`; Glm5NextKdaWeights, field `o_norm`):
+ *     out[t, h*D+d] = core[t,h,d] / sqrt(mean_d core[t,h,:]^2 + rms_eps) * w[d]
+ *                     * sigmoid(out_gate[t, h*D+d])                       -> BF16
+ *   core [T, H, D] F32;  out_gate [T, H*D] BF16;  w [D] BF16;  out [T, H*D] BF16
+ */
+KDA_API int kda_back_gated_rmsnorm(const float *core, const kda_bf16 *out_gate, const kda_bf16 *w,
+                           kda_bf16 *out, int T, const kda_dims *dims, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,176 @@
+"""Python binding of libkda.so, the B200 KDA core library (C ABI: include/kda.h).
+
+Argument marshalling only: every function here passes device pointers, sizes and the
+current CUDA stream to the C entry point of the same name; all computation happens in
+the library's sm_100a kernels. PyTorch supplies device memory and streams.
+
+There is no fallback: if libkda.so is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Iterable, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "kda.h")
+
+KDA_OK = 0
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_ALIAS", 3: "KDA_ERR_CAPACITY",
+          4: "KDA_ERR_UNSUPPORTED", 5: "KDA_ERR_CUDA", 6: "KDA_ERR_TIMEOUT", 7: "KDA_ERR_MISALIGNED"}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class KdaDims(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("scale", ctypes.c_float), ("l2_eps", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+
+
+def dims(heads: int, head_dim: int, chunk: int = 64, scale: float = 1.0, l2_eps: float = 1e-6,
+         rms_eps: float = 1e-6) -> KdaDims:
+    return KdaDims(heads, head_dim, chunk, scale, l2_eps, rms_eps)
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_DIMS = ctypes.POINTER(KdaDims)
+
+_SIGS = {
+    "kda_version": ([], _I),
+    "kda_status_string": ([_I], ctypes.c_char_p),
+    "kda_t_pad": ([ctypes.c_size_t, _I], ctypes.c_size_t),
+    "kda_device_status": ([ctypes.POINTER(_I), _I], _I),
+    "kda_gate": ([_VP, _VP, _VP, _VP, _I, _DIMS, _VP], _I),
+    "kda_beta": ([_VP, _VP, _I, _VP], _I),
+    "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
+    "kda_chunk_prefill_simt": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
+    "kda_recurrent_decode": ([_VP] * 7 + [_I, _DIMS, _VP], _I),
+    "kda_decode_fused": ([_VP] * 13 + [_I, _DIMS, _VP], _I),
+    "kda_decode_k": ([_VP] * 13 + [_I, _VP, _VP, _I, _DIMS, _VP], _I),
+    "kda_front_conv_silu_l2": ([_VP] * 7 + [_F, _I, _DIMS, _VP], _I),
+    "kda_back_gated_rmsnorm": ([_VP] * 4 + [_I, _DIMS, _VP], _I),
+}
+
+
+def lib():
+    """Load libkda.so (built in-tree by kda_gated_delta_gate_b200.build). Raises if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kda_gated_delta_gate_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list:
+    """Every function name include/kda.h declares."""
+    with open(HEADER_PATH) as f:
+        return re.findall(r"^KDA_API\s+[\w\s\*]*?\b(kda_\w+)\s*\(", f.read(), flags=re.M)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _call(name: str, *args) -> int:
+    rc = getattr(lib(), name)(*args)
+    if rc != KDA_OK:
+        raise KdaError(name, rc)
+    return rc
+
+
+def ptr_array(tensors: Sequence, device="cuda"):
+    """Device int64 tensor holding the data pointers of `tensors` (a `T* const*` argument)."""
+    import torch
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def host_ptr_array(tensors: Iterable):
+    ts = list(tensors)
+    return (ctypes.c_void_p * max(1, len(ts)))(*[t.data_ptr() for t in ts])
+
+
+def t_pad(T: int, chunk: int = 64) -> int:
+    return int(lib().kda_t_pad(T, chunk))
+
+
+def device_status(clear: bool = True) -> int:
+    out = ctypes.c_int(0)
+    _call("kda_device_status", ctypes.byref(out), 1 if clear else 0)
+    return out.value
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def kda_gate(g_raw, dt_bias, a_log, gate, n_rows: int, d: KdaDims, stream=None):
+    return _call("kda_gate", _p(g_raw), _p(dt_bias), _p(a_log), _p(gate), n_rows, ctypes.byref(d), _stream(stream))
+
+
+def kda_beta(b_logit, beta, n: int, stream=None):
+    return _call("kda_beta", _p(b_logit), _p(beta), n, _stream(stream))
+
+
+def kda_chunk_prefill(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None,
+                      impl: str = "tc"):
+    name = "kda_chunk_prefill" if impl == "tc" else "kda_chunk_prefill_simt"
+    return _call(name, _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core), B, T,
+                 ctypes.byref(d), _stream(stream))
+
+
+def kda_recurrent_decode(q, k, v, gate, beta, h_state_ptrs, o, N: int, d: KdaDims, stream=None):
+    return _call("kda_recurrent_decode", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(o), N,
+                 ctypes.byref(d), _stream(stream))
+
+
+def kda_decode_fused(x, conv_state_ptrs, conv_w, g_raw, dt_bias, a_log, b_logit, h_state_ptrs, out_gate,
+                     o_norm_w, o_norm_out, conv_out, core, N: int, d: KdaDims, stream=None):
+    return _call("kda_decode_fused", _p(x), _p(conv_state_ptrs), _p(conv_w), _p(g_raw), _p(dt_bias), _p(a_log),
+                 _p(b_logit), _p(h_state_ptrs), _p(out_gate), _p(o_norm_w), _p(o_norm_out), _p(conv_out), _p(core),
+                 N, ctypes.byref(d), _stream(stream))
+
+
+def kda_decode_k(x, conv_state, conv_w, g_raw, dt_bias, a_log, b_logit, h_state, out_gate, o_norm_w, o_norm_out,
+                 conv_out, core, K: int, h_snaps: Sequence, conv_snaps: Sequence, d: KdaDims, stream=None):
+    n = len(h_snaps)
+    hs = host_ptr_array(h_snaps) if n else None
+    cs = host_ptr_array(conv_snaps) if n else None
+    return _call("kda_decode_k", _p(x), _p(conv_state), _p(conv_w), _p(g_raw), _p(dt_bias), _p(a_log), _p(b_logit),
+                 _p(h_state), _p(out_gate), _p(o_norm_w), _p(o_norm_out), _p(conv_out), _p(core), K,
+                 ctypes.cast(hs, _VP) if hs is not None else None, ctypes.cast(cs, _VP) if cs is not None else None,
+                 n, ctypes.byref(d), _stream(stream))
+
+
+def kda_front_conv_silu_l2(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32, pad_fill: float, T: int,
+                           d: KdaDims, stream=None):
+    return _call("kda_front_conv_silu_l2", _p(x), _p(conv_state), _p(conv_w), _p(conv_out), _p(q_f32), _p(k_f32),
+                 _p(v_f32), float(pad_fill), T, ctypes.byref(d), _stream(stream))
+
+
+def kda_back_gated_rmsnorm(core, out_gate, w, out, T: int, d: KdaDims, stream=None):
+    return _call("kda_back_gated_rmsnorm", _p(core), _p(out_gate), _p(w), _p(out), T, ctypes.byref(d),
+                 _stream(stream))

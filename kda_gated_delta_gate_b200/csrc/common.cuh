@@ -1,0 +1,75 @@
+// Shared device/host helpers of libkda (sm_100a). Internal: not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+constexpr int kChunk = 64;
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Round-to-nearest-even FP32 -> BF16 (the CUDA intrinsic; NaN stays NaN).
+__device__ __forceinline__ uint16_t f32_to_bf16(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
+}
+
+// softplus in the overflow-free form max(x,0) + log1p(exp(-|x|)).
+__device__ __forceinline__ float softplus_f32(float x) {
+    return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+
+__device__ __forceinline__ float sigmoid_f32(float x) {
+    return 1.0f / (1.0f + expf(-x));
+}
+
+// The bounded log-decay gate: -exp(a_log[h]) * softplus(g_raw + dt_bias).
+__device__ __forceinline__ float kda_gate_f32(float g_raw, float dt_bias, float neg_exp_alog) {
+    return neg_exp_alog * softplus_f32(g_raw + dt_bias);
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlaps(const void *a, size_t abytes, const void *b, size_t bbytes) {
+    const char *x = static_cast<const char *>(a), *y = static_cast<const char *>(b);
+    return x < y + bbytes && y < x + abytes;
+}
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+// Basic validation shared by every entry point. Returns KDA_OK or an error code.
+inline int check_dims(const kda_dims *d) {
+    if (!d) return KDA_ERR_INVALID_ARG;
+    if (d->heads < 1) return KDA_ERR_INVALID_ARG;
+    if (d->head_dim != 64 && d->head_dim != 128) return KDA_ERR_UNSUPPORTED;
+    if (d->chunk != kChunk) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+// Device address of this device's latched status word (kda_api.cu).
+int *device_status_ptr();
+
+}  // namespace kda
+
+#define KDA_TRY(expr)                        \
+    do {                                     \
+        int _kda_rc = (expr);                \
+        if (_kda_rc != KDA_OK) return _kda_rc; \
+    } while (0)
+
+namespace kda {
+// Chunked prefill implementations (kda_chunk_simt.cu, kda_chunk_tc.cu).
+int chunk_prefill_check(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                        float *const *h_state, float *core, int B, int T, const kda_dims *dims);
+int chunk_prefill_simt(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                       float *const *h_state, float *core, int B, int T, const kda_dims *dims, cudaStream_t s);
+}  // namespace kda

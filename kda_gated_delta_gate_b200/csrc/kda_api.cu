@@ -1,0 +1,73 @@
+// Library-wide C-ABI entry points: version, status text, T_pad, latched device status.
+#include <atomic>
+
+#include "common.cuh"
+
+namespace kda {
+
+// One status word per device (a __device__ variable exists once per device context).
+// Kernels that run bounded waits write a KDA_ERR_* code here instead of trapping.
+__device__ int g_device_status;
+
+int *device_status_ptr() {
+    static std::atomic<int *> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+    if (dev < 64) {
+        int *p = cache[dev].load(std::memory_order_relaxed);
+        if (p) return p;
+    }
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return nullptr;
+    if (dev < 64) cache[dev].store(static_cast<int *>(addr), std::memory_order_relaxed);
+    return static_cast<int *>(addr);
+}
+
+}  // namespace kda
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+const char *kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_ALIAS: return "buffers that must not overlap do";
+        case KDA_ERR_CAPACITY: return "token count beyond the workspace capacity";
+        case KDA_ERR_UNSUPPORTED: return "unsupported dimensions";
+        case KDA_ERR_CUDA: return "CUDA runtime error";
+        case KDA_ERR_TIMEOUT: return "device-side wait timed out";
+        case KDA_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+size_t kda_t_pad(size_t T, int chunk) {
+    if (chunk <= 0) return 0;
+    const size_t c = static_cast<size_t>(chunk);
+    return (T + c - 1) / c * c;
+}
+
+int kda_device_status(int *out, int clear) {
+    if (!out) return KDA_ERR_INVALID_ARG;
+    int *p = kda::device_status_ptr();
+    if (!p) return KDA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaMemcpy(out, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+}  // extern "C"
+
+extern "C" int kda_chunk_prefill(const float *q, const float *k, const float *v, const float *gate,
+                                 const float *beta, float *const *h_state, float *core, int B, int T,
+                                 const kda_dims *dims, void *stream) {
+    KDA_TRY(kda::chunk_prefill_check(q, k, v, gate, beta, h_state, core, B, T, dims));
+    if (B == 0 || T == 0) return KDA_OK;
+    return kda::chunk_prefill_simt(q, k, v, gate, beta, h_state, core, B, T, dims, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,95 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/kda.h declares,
+and rejects bad arguments on the host before anything reaches the device."""
+import ctypes
+
+import pytest
+
+import kda_gated_delta_gate_b200 as kda
+
+BOGUS = 0x10000  # never dereferenced: every case below fails validation first
+
+
+@pytest.fixture(scope="module")
+def L():
+    from kda_gated_delta_gate_b200 import build
+    build.build()
+    return kda.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = kda.header_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(kda._SIGS), "binding and header disagree"
+
+
+def test_version_status_tpad(L):
+    assert L.kda_version() >= 100
+    for s in range(8):
+        assert L.kda_status_string(s)
+    assert L.kda_status_string(99) == b"unknown status"
+    assert [kda.t_pad(t) for t in (0, 1, 63, 64, 65, 65500, 4096)] == [0, 64, 64, 64, 128, 65536, 4096]
+
+
+def _d(**kw):
+    base = dict(heads=2, head_dim=64)
+    base.update(kw)
+    return kda.dims(**base)
+
+
+def test_gate_argument_checks(L):
+    rc = L.kda_gate(None, BOGUS, BOGUS, BOGUS, 4, ctypes.byref(_d()), None)
+    assert rc == 1
+    assert L.kda_gate(BOGUS, BOGUS, BOGUS, BOGUS, 4, ctypes.byref(_d(head_dim=96)), None) == 4
+    assert L.kda_gate(BOGUS, BOGUS, BOGUS, BOGUS, 4, ctypes.byref(_d(chunk=32)), None) == 4
+    assert L.kda_gate(BOGUS + 2, BOGUS, BOGUS, BOGUS, 4, ctypes.byref(_d()), None) == 7
+    assert L.kda_gate(BOGUS, BOGUS, BOGUS, BOGUS, -1, ctypes.byref(_d()), None) == 1
+    assert L.kda_gate(BOGUS, BOGUS, BOGUS, BOGUS, 0, ctypes.byref(_d()), None) == 0  # empty: nothing runs
+    assert L.kda_gate(BOGUS, BOGUS, BOGUS, BOGUS, 4, None, None) == 1
+
+
+def test_prefill_argument_checks(L):
+    d = ctypes.byref(_d())
+    args = [BOGUS] * 7
+    assert L.kda_chunk_prefill(*args, 1, 0, d, None) == 0  # T = 0: nothing to do
+    assert L.kda_chunk_prefill(*args, 0, 10, d, None) == 0  # B = 0
+    assert L.kda_chunk_prefill(*args, -1, 10, d, None) == 1
+    bad = list(args)
+    bad[5] = None
+    assert L.kda_chunk_prefill(*bad, 1, 10, d, None) == 1
+    bad = list(args)
+    bad[6] = BOGUS + 4
+    assert L.kda_chunk_prefill(*bad, 1, 10, d, None) == 7
+    assert L.kda_chunk_prefill_simt(*args, 1, 10, ctypes.byref(_d(head_dim=32)), None) == 4
+
+
+def test_decode_alias_and_snapshot_checks(L):
+    d = ctypes.byref(_d())
+    g_raw = BOGUS
+    out_gate = BOGUS + 64  # overlaps g_raw's [N, H*D] BF16 range
+    rc = L.kda_decode_fused(BOGUS, BOGUS, BOGUS, g_raw, BOGUS, BOGUS, BOGUS, BOGUS, out_gate, BOGUS, BOGUS,
+                            None, None, 2, d, None)
+    assert rc == 2
+    far = BOGUS + (1 << 20)
+    common = [BOGUS, BOGUS, BOGUS, g_raw, BOGUS, BOGUS, BOGUS, BOGUS, far, BOGUS, BOGUS, None, None]
+    assert L.kda_decode_k(*common, 0, None, None, 0, d, None) == 1          # K < 1
+    assert L.kda_decode_k(*common, 40, None, None, 0, d, None) == 4         # K > 32
+    assert L.kda_decode_k(*common, 4, None, None, 2, d, None) == 1          # n_snap not 0 or K-1
+    assert L.kda_decode_k(*common, 4, None, None, 3, d, None) == 1          # snapshots missing
+    assert L.kda_recurrent_decode(*([BOGUS] * 7), -3, d, None) == 1
+
+
+def test_front_back_argument_checks(L):
+    d = ctypes.byref(_d())
+    assert L.kda_front_conv_silu_l2(BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, None, None, 0.0, 8, d, None) == 1
+    assert L.kda_front_conv_silu_l2(BOGUS, BOGUS, BOGUS, BOGUS, None, None, None, 0.0, 0, d, None) == 0
+    assert L.kda_back_gated_rmsnorm(BOGUS, BOGUS, BOGUS, BOGUS + 8, 8, d, None) == 7
+    assert L.kda_back_gated_rmsnorm(None, BOGUS, BOGUS, BOGUS, 8, d, None) == 1
+
+
+def test_binding_raises_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(kda, "_lib", None)
+    monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "libkda.so"))
+    with pytest.raises(ImportError):
+        kda.lib()
