@@ -60,3 +60,19 @@ def build(verbose: bool = False) -> str:
 
 if __name__ == "__main__":
     print(build(verbose="-v" in sys.argv))
+
+
+PROBE_SRC = os.path.join(ROOT, "tests", "cuda", "umma_probe.cu")
+PROBE_LIB = os.path.join(ROOT, "_build", "libumma_probe.so")
+
+
+def build_probe() -> str:
+    """Test-only library exercising the tcgen05 building blocks (tests/cuda/umma_probe.cu)."""
+    os.makedirs(os.path.dirname(PROBE_LIB), exist_ok=True)
+    deps = [PROBE_SRC, os.path.join(CSRC, "umma.cuh")]
+    if not os.path.exists(PROBE_LIB) or os.path.getmtime(PROBE_LIB) < max(os.path.getmtime(d) for d in deps):
+        cmd = [NVCC, *ARCH, *FLAGS, "-shared", "--cudart", "static", "-o", PROBE_LIB, PROBE_SRC]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed for the probe:\n{r.stdout}\n{r.stderr}")
+    return PROBE_LIB
