@@ -193,6 +193,7 @@ def main():
     core = torch.empty((B * Tp, H, D), device=dev)
     state = ci.s0[0].to(dev).clone()
     ptrs = kda.ptr_array([state], device=dev)
+    scratch = torch.empty(max(16, kda.kda_chunk_prefill_scratch_bytes(B, T, d)), dtype=torch.uint8, device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -202,7 +203,7 @@ def main():
         kda.kda_beta(b_logit, beta, B * T * H, s)
         if kev:
             kev[0].record(stream)
-        kda.kda_chunk_prefill(q, k, v, gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl)
+        kda.kda_chunk_prefill(q, k, v, gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl, scratch=scratch)
         if kev:
             kev[1].record(stream)
         return 3
@@ -241,7 +242,7 @@ def main():
     dec = _decode_leg(kda, torch, dev, s, stream, flush, hbm)
 
     # ---- end-to-end leg: the same C-ABI calls from pinned host buffers, copies timed
-    e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world)
+    e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch)
 
     result = None
     if rank == 0:
@@ -306,7 +307,7 @@ def _decode_leg(kda, torch, dev, s, stream, flush, hbm):
             "frac_hbm": all_bytes / (ms * 1e-3) / 1e9 / hbm}
 
 
-def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world):
+def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
     from synth import pad_rows
     host = {n: pad_rows(getattr(ci, n), Tp, 0.0).pin_memory() for n in ("q", "k", "v", "g_raw", "b_logit")}
     host["s0"] = ci.s0[0].clone().pin_memory()
@@ -326,7 +327,8 @@ def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world):
             dv[n].copy_(t, non_blocking=True)
         kda.kda_gate(dv["g_raw"], dt_bias, a_log, gate, B * T, d, s)
         kda.kda_beta(dv["b_logit"], beta, B * T * H, s)
-        kda.kda_chunk_prefill(dv["q"], dv["k"], dv["v"], gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl)
+        kda.kda_chunk_prefill(dv["q"], dv["k"], dv["v"], gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl,
+                              scratch=scratch)
         core_h.copy_(core, non_blocking=True)
         s_h.copy_(dv["s0"], non_blocking=True)
 

@@ -115,11 +115,19 @@ KDA_API int kda_beta(const float *b_logit, float *beta, int n, void *stream);
  *             state and overwritten with the state after exactly T tokens.
  *   core      [B*T_pad, H, D] F32 output o = scale * S^T q for rows < T (pad rows are
  *             not written).
- * The per-(stream, head) states must not overlap each other or any input.
+ *   scratch   caller-owned device scratch of at least kda_chunk_prefill_scratch_bytes(B, T,
+ *             dims) bytes, 16-byte aligned (per-chunk operand tiles passed between the two
+ *             kernels of the call); contents on entry do not matter. KDA_ERR_CAPACITY if
+ *             scratch_bytes is too small.
+ * Computed with tcgen05 tensor cores in split-BF16 precision (about 2^-16 relative per
+ * product). The per-(stream, head) states must not overlap each other or any input.
  */
 KDA_API int kda_chunk_prefill(const float *q, const float *k, const float *v, const float *gate,
-                      const float *beta, float *const *h_state, float *core, int B, int T,
-                      const kda_dims *dims, void *stream);
+                              const float *beta, float *const *h_state, float *core, int B, int T,
+                              void *scratch, size_t scratch_bytes, const kda_dims *dims, void *stream);
+
+/* Scratch bytes kda_chunk_prefill needs for B streams of T tokens (0 if B or T is 0). */
+KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dims);
 
 /* kda_chunk_prefill_simt — the same contract as kda_chunk_prefill, computed by the
  * plain FP32 CUDA-core kernel (no tensor cores). Kept as a second implementation. */

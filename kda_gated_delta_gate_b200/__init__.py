@@ -51,7 +51,8 @@ _SIGS = {
     "kda_device_status": ([ctypes.POINTER(_I), _I], _I),
     "kda_gate": ([_VP, _VP, _VP, _VP, _I, _DIMS, _VP], _I),
     "kda_beta": ([_VP, _VP, _I, _VP], _I),
-    "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
+    "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
+    "kda_chunk_prefill_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_prefill_simt": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_recurrent_decode": ([_VP] * 7 + [_I, _DIMS, _VP], _I),
     "kda_decode_fused": ([_VP] * 13 + [_I, _DIMS, _VP], _I),
@@ -135,11 +136,24 @@ def kda_beta(b_logit, beta, n: int, stream=None):
     return _call("kda_beta", _p(b_logit), _p(beta), n, _stream(stream))
 
 
+def kda_chunk_prefill_scratch_bytes(B: int, T: int, d: KdaDims) -> int:
+    return int(lib().kda_chunk_prefill_scratch_bytes(B, T, ctypes.byref(d)))
+
+
 def kda_chunk_prefill(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None,
-                      impl: str = "tc"):
-    name = "kda_chunk_prefill" if impl == "tc" else "kda_chunk_prefill_simt"
-    return _call(name, _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core), B, T,
-                 ctypes.byref(d), _stream(stream))
+                      impl: str = "tc", scratch=None):
+    """impl "tc": the tensor-core path (needs `scratch`, a device buffer of at least
+    kda_chunk_prefill_scratch_bytes bytes; one is allocated here if None). impl "simt": the
+    CUDA-core path (no scratch)."""
+    if impl == "simt":
+        return _call("kda_chunk_prefill_simt", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core),
+                     B, T, ctypes.byref(d), _stream(stream))
+    nbytes = kda_chunk_prefill_scratch_bytes(B, T, d)
+    if scratch is None:
+        import torch
+        scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    return _call("kda_chunk_prefill", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core), B, T,
+                 _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
 
 
 def kda_recurrent_decode(q, k, v, gate, beta, h_state_ptrs, o, N: int, d: KdaDims, stream=None):

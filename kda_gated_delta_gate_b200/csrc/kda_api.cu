@@ -64,10 +64,19 @@ int kda_device_status(int *out, int clear) {
 
 }  // extern "C"
 
+extern "C" size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dims) {
+    if (kda::check_dims(dims) != KDA_OK) return 0;
+    return kda::chunk_prefill_scratch_bytes(B, T, dims->heads);
+}
+
 extern "C" int kda_chunk_prefill(const float *q, const float *k, const float *v, const float *gate,
-                                 const float *beta, float *const *h_state, float *core, int B, int T,
-                                 const kda_dims *dims, void *stream) {
+                                 const float *beta, float *const *h_state, float *core, int B, int T, void *scratch,
+                                 size_t scratch_bytes, const kda_dims *dims, void *stream) {
     KDA_TRY(kda::chunk_prefill_check(q, k, v, gate, beta, h_state, core, B, T, dims));
     if (B == 0 || T == 0) return KDA_OK;
-    return kda::chunk_prefill_simt(q, k, v, gate, beta, h_state, core, B, T, dims, static_cast<cudaStream_t>(stream));
+    if (!scratch) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(scratch)) return KDA_ERR_MISALIGNED;
+    if (scratch_bytes < kda::chunk_prefill_scratch_bytes(B, T, dims->heads)) return KDA_ERR_CAPACITY;
+    return kda::chunk_prefill_tc(q, k, v, gate, beta, h_state, core, B, T, dims, scratch,
+                                 static_cast<cudaStream_t>(stream));
 }

@@ -127,3 +127,21 @@ extern "C" __attribute__((visibility("default"))) int probe_run(int i, const flo
         default: return -1;
     }
 }
+
+// A bounded wait that is never satisfied: nothing arrives on the barrier, so mbar_wait must
+// give up after `cycles` SM clocks and the kernel records that in *status (1) and returns.
+__global__ void timeout_kernel(int *status, long long cycles) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = mbar_wait(&bar, 0, cycles);
+    if (threadIdx.x == 0) *status = ok ? 0 : 1;
+}
+
+extern "C" __attribute__((visibility("default"))) int probe_timeout(int *status, long long cycles) {
+    timeout_kernel<<<1, 32>>>(status, cycles);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}

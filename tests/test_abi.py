@@ -52,15 +52,21 @@ def test_gate_argument_checks(L):
 def test_prefill_argument_checks(L):
     d = ctypes.byref(_d())
     args = [BOGUS] * 7
-    assert L.kda_chunk_prefill(*args, 1, 0, d, None) == 0  # T = 0: nothing to do
-    assert L.kda_chunk_prefill(*args, 0, 10, d, None) == 0  # B = 0
-    assert L.kda_chunk_prefill(*args, -1, 10, d, None) == 1
+    need = L.kda_chunk_prefill_scratch_bytes(2, 100, d)
+    assert need == 2 * 2 * 2 * 32768  # B * H * chunks * one [Tb; M'] tile pair
+    assert L.kda_chunk_prefill_scratch_bytes(0, 100, d) == 0
+    assert L.kda_chunk_prefill(*args, 1, 0, BOGUS, 0, d, None) == 0  # T = 0: nothing to do
+    assert L.kda_chunk_prefill(*args, 0, 10, BOGUS, 0, d, None) == 0  # B = 0
+    assert L.kda_chunk_prefill(*args, -1, 10, BOGUS, need, d, None) == 1
+    assert L.kda_chunk_prefill(*args, 2, 100, BOGUS, need - 16, d, None) == 3  # scratch too small
+    assert L.kda_chunk_prefill(*args, 2, 100, None, need, d, None) == 1
+    assert L.kda_chunk_prefill(*args, 2, 100, BOGUS + 8, need, d, None) == 7
     bad = list(args)
     bad[5] = None
-    assert L.kda_chunk_prefill(*bad, 1, 10, d, None) == 1
+    assert L.kda_chunk_prefill(*bad, 1, 10, BOGUS, need, d, None) == 1
     bad = list(args)
     bad[6] = BOGUS + 4
-    assert L.kda_chunk_prefill(*bad, 1, 10, d, None) == 7
+    assert L.kda_chunk_prefill(*bad, 1, 10, BOGUS, need, d, None) == 7
     assert L.kda_chunk_prefill_simt(*args, 1, 10, ctypes.byref(_d(head_dim=32)), None) == 4
 
 

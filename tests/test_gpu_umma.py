@@ -46,3 +46,20 @@ def test_umma_shapes_and_layouts(probe):
         if st.item() != 0 or not np.isfinite(err) or err > 1e-5:
             failures.append((i, M, N, K, amn, bmn, st.item(), float(err)))
     assert not failures, failures
+
+
+def test_bounded_wait_gives_up_and_context_survives(probe):
+    """Failure detection without a GPU fault: a wait on a barrier nothing arrives on returns
+    after its limit (about 1 ms here), the kernel reports it in a status word the host reads,
+    and the context stays usable for the next launch."""
+    probe.probe_timeout.argtypes = [ctypes.c_void_p, ctypes.c_longlong]
+    st = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    assert probe.probe_timeout(st.data_ptr(), 2_000_000) == 0
+    torch.cuda.synchronize()
+    assert st.item() == 1
+    A = torch.ones((128, 128), device="cuda")
+    D = torch.empty((128, 16), device="cuda")
+    s2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert probe.probe_run(0, A.data_ptr(), A.data_ptr(), D.data_ptr(), s2.data_ptr()) == 0
+    torch.cuda.synchronize()
+    assert s2.item() == 0 and torch.all(D == 128.0)
