@@ -42,21 +42,23 @@ constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 1.9 GHz
 
 // ================================================================ phase 1: intra-chunk
 
+constexpr int kIntraThreads = 512;
+
 template <int D>
 struct Intra {
     static constexpr int P = D + 8;   // fp32 row stride of [C][D] tiles (bank-spread, 16-B aligned)
     static constexpr int PC = C + 1;  // row stride of [C][C] tiles
     static constexpr int NZ = 48;     // rows of the block-local backward factors (blocks 0..2)
-    static constexpr size_t floats = 3 * C * P + NZ * P + 3 * C * PC + 3 * D + C + 3 * 256;
+    static constexpr size_t floats = 3 * C * P + NZ * P + 3 * C * PC + 4 * D + C + 3 * 256;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kIntraThreads, 1)
 intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
              const float *__restrict__ beta, uint8_t *__restrict__ scratch, int T, int T_pad, int H) {
     using I = Intra<D>;
-    constexpr int P = I::P, PC = I::PC;
+    constexpr int P = I::P, PC = I::PC, NT = kIntraThreads;
     extern __shared__ float smem[];
     float *sK = smem;              // k, then X (rows 16..63): k_i prod_{s=16a}^{i} a_s
     float *sQ = sK + C * P;        // q, then Y (rows 16..63): q_i prod_{s=16a}^{i} a_s
@@ -65,8 +67,8 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     float *sL = sZ + I::NZ * P;    // L' (unscaled), then M'
     float *sM = sL + C * PC;       // M
     float *sT = sM + C * PC;       // T, then Tb
-    float *sSig = sT + C * PC;     // [3][D]: block-1 product, block-2 product, both
-    float *sB = sSig + 3 * D;      // beta
+    float *sF = sT + C * PC;       // [4][D]: whole-block decay products
+    float *sB = sF + 4 * D;        // beta
     float *sTmp = sB + C;          // [3][256]
 
     const int tid = threadIdx.x;
@@ -76,7 +78,7 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     const size_t rs = static_cast<size_t>(H) * D;
 
     // ---- load k, q and a = e^g (pad guard: rows >= n are k = q = 0, a = 1)
-    for (int e = tid; e < C * D / 4; e += kThreads) {
+    for (int e = tid; e < C * D / 4; e += NT) {
         const int i = e / (D / 4), c = 4 * (e % (D / 4));
         float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv, av = make_float4(1.f, 1.f, 1.f, 1.f);
         if (i < n) {
@@ -94,30 +96,36 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     __syncthreads();
 
     // ---- diagonal 16x16 blocks: thread (block a, j pair, channel group) walks i upward with
-    //      the running product G = k_j prod_{s=j+1}^{i} a_s; the 8 channel groups of one j
-    //      are 8 adjacent lanes and reduce with shuffles.
+    //      the running product G = k_j prod_{s=j+1}^{i} a_s over its channels; the 16 channel
+    //      groups of one j are 16 adjacent lanes and reduce with shuffles. Channel group cg
+    //      holds float4 columns cg, cg + 16, ... (conflict-free 16-byte loads).
     {
-        constexpr int CPT = D / 8;
-        const int a = tid >> 6, jp = (tid >> 3) & 7, cg = tid & 7;
-        const unsigned gmask = 0xFFu << (tid & 24);
+        constexpr int NV = D / 64;  // float4 per thread per row (2 for D = 128, 1 for D = 64)
+        const int cg = tid & 15, jp = (tid >> 4) & 7, a = tid >> 7;
+        const unsigned gmask = 0xFFFFu << (tid & 16);
 #pragma unroll 1
         for (int pass = 0; pass < 2; ++pass) {
             const int j = 16 * a + (pass == 0 ? jp : 15 - jp);
-            float G[CPT];
+            float4 G[NV];
 #pragma unroll
-            for (int cc = 0; cc < CPT; ++cc) G[cc] = sK[j * P + cg + 8 * cc];
+            for (int w = 0; w < NV; ++w) G[w] = *reinterpret_cast<const float4 *>(sK + j * P + 4 * (cg + 16 * w));
 #pragma unroll 1
             for (int i = j; i < 16 * a + 16; ++i) {
                 float ls = 0.f, ms = 0.f;
 #pragma unroll
-                for (int cc = 0; cc < CPT; ++cc) {
-                    const int c = cg + 8 * cc;
-                    if (i > j) G[cc] *= sA[i * P + c];
-                    ls = fmaf(sK[i * P + c], G[cc], ls);
-                    ms = fmaf(sQ[i * P + c], G[cc], ms);
+                for (int w = 0; w < NV; ++w) {
+                    const int c = 4 * (cg + 16 * w);
+                    if (i > j) {
+                        const float4 av = *reinterpret_cast<const float4 *>(sA + i * P + c);
+                        G[w].x *= av.x; G[w].y *= av.y; G[w].z *= av.z; G[w].w *= av.w;
+                    }
+                    const float4 kv = *reinterpret_cast<const float4 *>(sK + i * P + c);
+                    const float4 qv = *reinterpret_cast<const float4 *>(sQ + i * P + c);
+                    ls = fmaf(kv.x, G[w].x, fmaf(kv.y, G[w].y, fmaf(kv.z, G[w].z, fmaf(kv.w, G[w].w, ls))));
+                    ms = fmaf(qv.x, G[w].x, fmaf(qv.y, G[w].y, fmaf(qv.z, G[w].z, fmaf(qv.w, G[w].w, ms))));
                 }
 #pragma unroll
-                for (int o = 1; o < 8; o <<= 1) {
+                for (int o = 1; o < 16; o <<= 1) {
                     ls += __shfl_xor_sync(gmask, ls, o);
                     ms += __shfl_xor_sync(gmask, ms, o);
                 }
@@ -130,79 +138,104 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     }
     __syncthreads();
 
-    // ---- block-local factors, one thread per channel: Z (backward, blocks 0..2), then X, Y
-    //      (forward, blocks 1..3, in place over k and q) and the per-block decay products.
-    if (tid < D) {
-        const int c = tid;
-#pragma unroll 1
-        for (int bb = 0; bb < 3; ++bb) {
-            float f = 1.f;
-            for (int j = 16 * bb + 15; j >= 16 * bb; --j) {
+    // ---- block-local factors, thread (channel c, block a): Z (backward within blocks 0..2),
+    //      the whole-block products F, then X, Y (forward within blocks 1..3, in place).
+    if (tid < 4 * D) {
+        const int c = tid % D, a = tid / D;
+        float f = 1.f;
+        if (a < 3) {
+            for (int j = 16 * a + 15; j >= 16 * a; --j) {
                 sZ[j * P + c] = sK[j * P + c] * f;
                 f *= sA[j * P + c];
             }
+        } else {
+            for (int j = 16 * a + 15; j >= 16 * a; --j) f *= sA[j * P + c];
         }
-        float F[4];
-#pragma unroll 1
-        for (int aa = 0; aa < 4; ++aa) {
-            float f = 1.f;
-            for (int i = 16 * aa; i < 16 * aa + 16; ++i) {
-                f *= sA[i * P + c];
-                if (aa > 0) {
-                    sK[i * P + c] *= f;
-                    sQ[i * P + c] *= f;
-                }
-            }
-            F[aa] = f;
+        sF[a * D + c] = f;
+    }
+    __syncthreads();
+    if (tid < 3 * D) {
+        const int c = tid % D, a = 1 + tid / D;
+        float f = 1.f;
+        for (int i = 16 * a; i < 16 * a + 16; ++i) {
+            f *= sA[i * P + c];
+            sK[i * P + c] *= f;
+            sQ[i * P + c] *= f;
         }
-        sSig[c] = F[1];
-        sSig[D + c] = F[2];
-        sSig[2 * D + c] = F[1] * F[2];
     }
     __syncthreads();
 
-    // ---- off-diagonal blocks (a > b): L'[i][j] = sum_c X_ic sigma_ab,c Z_jc (same with Y for M),
-    //      sigma_ab = the decay of the whole blocks strictly between b and a (1 if adjacent).
-    if (tid < 96) {
-        const int p = tid >> 4;
-        const int pa[6] = {1, 2, 2, 3, 3, 3}, pb[6] = {0, 0, 1, 0, 1, 2};
-        const int a = pa[p], bb = pb[p];
-        const int sig = (a == 2 && bb == 0) ? 0 : (a == 3 && bb == 1) ? 1 : (a == 3 && bb == 0) ? 2 : -1;
-        const int i0 = 16 * a + 4 * ((tid & 15) >> 2), j0 = 16 * bb + 4 * (tid & 3);
+    // ---- off-diagonal blocks (a > b): L'[i][j] = sum_c X_ic sigma_ab,c Z_jc (Y for M), with
+    //      sigma_ab the decay of the whole blocks strictly between b and a (1 when adjacent).
+    //      Thread = (4x4 tile, channel quarter); the 4 quarters are adjacent lanes.
+    if (tid < 384) {
+        const int qtr = tid & 3, tile = tid >> 2;
+        const int p = tile >> 4;
+        const int pa = p == 0 ? 1 : (p < 3 ? 2 : 3);
+        const int pb = p == 0 ? 0 : (p == 1 ? 0 : (p == 2 ? 1 : p - 3));
+        const int i0 = 16 * pa + 4 * ((tile & 15) >> 2), j0 = 16 * pb + 4 * (tile & 3);
         float l[4][4], m[4][4];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int s = 0; s < 4; ++s) { l[r][s] = 0.f; m[r][s] = 0.f; }
+            for (int s2 = 0; s2 < 4; ++s2) { l[r][s2] = 0.f; m[r][s2] = 0.f; }
 #pragma unroll 2
-        for (int c = 0; c < D; ++c) {
-            const float sg = sig >= 0 ? sSig[sig * D + c] : 1.f;
-            float z[4], x[4], y[4];
+        for (int cq = 0; cq < D / 16; ++cq) {
+            const int c = 4 * (qtr + 4 * cq);
+            float4 sg = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (pa - pb >= 2) {
+                sg = *reinterpret_cast<const float4 *>(sF + 1 * D + c);
+                if (pa - pb == 3) {
+                    const float4 f2 = *reinterpret_cast<const float4 *>(sF + 2 * D + c);
+                    sg.x *= f2.x; sg.y *= f2.y; sg.z *= f2.z; sg.w *= f2.w;
+                } else if (pa == 3) {
+                    sg = *reinterpret_cast<const float4 *>(sF + 2 * D + c);
+                }
+            }
+            float4 z[4], x[4], y[4];
 #pragma unroll
-            for (int s = 0; s < 4; ++s) z[s] = sZ[(j0 + s) * P + c] * sg;
+            for (int s2 = 0; s2 < 4; ++s2) {
+                z[s2] = *reinterpret_cast<const float4 *>(sZ + (j0 + s2) * P + c);
+                z[s2].x *= sg.x; z[s2].y *= sg.y; z[s2].z *= sg.z; z[s2].w *= sg.w;
+            }
 #pragma unroll
-            for (int r = 0; r < 4; ++r) { x[r] = sK[(i0 + r) * P + c]; y[r] = sQ[(i0 + r) * P + c]; }
+            for (int r = 0; r < 4; ++r) {
+                x[r] = *reinterpret_cast<const float4 *>(sK + (i0 + r) * P + c);
+                y[r] = *reinterpret_cast<const float4 *>(sQ + (i0 + r) * P + c);
+            }
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    l[r][s] = fmaf(x[r], z[s], l[r][s]);
-                    m[r][s] = fmaf(y[r], z[s], m[r][s]);
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    l[r][s2] = fmaf(x[r].x, z[s2].x, fmaf(x[r].y, z[s2].y, fmaf(x[r].z, z[s2].z, fmaf(x[r].w, z[s2].w, l[r][s2]))));
+                    m[r][s2] = fmaf(y[r].x, z[s2].x, fmaf(y[r].y, z[s2].y, fmaf(y[r].z, z[s2].z, fmaf(y[r].w, z[s2].w, m[r][s2]))));
                 }
         }
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                sL[(i0 + r) * PC + j0 + s] = l[r][s];
-                sM[(i0 + r) * PC + j0 + s] = m[r][s];
+            for (int s2 = 0; s2 < 4; ++s2) {
+#pragma unroll
+                for (int o = 1; o < 4; o <<= 1) {
+                    l[r][s2] += __shfl_xor_sync(0xffffffffu, l[r][s2], o);
+                    m[r][s2] += __shfl_xor_sync(0xffffffffu, m[r][s2], o);
+                }
             }
+        if (qtr == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    sL[(i0 + r) * PC + j0 + s2] = l[r][s2];
+                    sM[(i0 + r) * PC + j0 + s2] = m[r][s2];
+                }
+        }
     }
     __syncthreads();
 
     // ---- L = diag(beta) L' (strict lower). T = (I + L)^-1: 16x16 diagonal blocks by
     //      substitution, then off-diagonal blocks T_ab = -T_aa sum_{b<=c<a} L_ac T_cb.
-    for (int e = tid; e < C * C; e += kThreads) {
+    for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, j = e % C;
         if (i > j) sL[i * PC + j] *= sB[i];
     }
@@ -229,7 +262,7 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
 #pragma unroll 1
     for (int dist = 1; dist < 4; ++dist) {
         const int npairs = 4 - dist;
-        for (int e = tid; e < npairs * 256; e += kThreads) {
+        for (int e = tid; e < npairs * 256; e += NT) {
             const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
             const int bb = pr, aa = pr + dist;
             float acc = 0.f;
@@ -240,7 +273,7 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
             sTmp[pr * 256 + i * 16 + j] = acc;
         }
         __syncthreads();
-        for (int e = tid; e < npairs * 256; e += kThreads) {
+        for (int e = tid; e < npairs * 256; e += NT) {
             const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
             const int bb = pr, aa = pr + dist;
             float acc = 0.f;
@@ -252,12 +285,12 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
         __syncthreads();
     }
     // ---- Tb = T diag(beta) (lower incl. diagonal), then M' = M Tb (lower triangular) into sL
-    for (int e = tid; e < C * C; e += kThreads) {
+    for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, j = e % C;
         if (j <= i) sT[i * PC + j] *= sB[j];
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += kThreads) {
+    for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, l = e % C;
         float acc = 0.f;
         for (int j = l; j <= i; ++j) acc = fmaf(sM[i * PC + j], sT[j * PC + l], acc);
@@ -266,23 +299,20 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     __syncthreads();
     // ---- write [Tb; M'] as BF16 hi and lo K-major swizzled tiles (128 rows x 64 columns)
     uint8_t *dst = scratch + ((static_cast<size_t>(b) * H + h) * (T_pad / C) + ch) * kA2Bytes;
-    for (int e = tid; e < 128 * 8; e += kThreads) {
+    for (int e = tid; e < 128 * 8; e += NT) {
         const int row = e >> 3, c0 = 8 * (e & 7);
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int col = c0 + u;
+            x[u] = row < 64 ? (col <= row ? sT[row * PC + col] : 0.f) : sL[(row - 64) * PC + col];
+        }
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            float v2[2];
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-                const int col = c0 + 2 * u + w;
-                float val;
-                if (row < 64) val = col <= row ? sT[row * PC + col] : 0.f;
-                else val = sL[(row - 64) * PC + col];
-                v2[w] = val;
-            }
             uint16_t h0, l0, h1, l1;
-            split_bf16(v2[0], h0, l0);
-            split_bf16(v2[1], h1, l1);
+            split_bf16(x[2 * u], h0, l0);
+            split_bf16(x[2 * u + 1], h1, l1);
             hw[u] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
             lw[u] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
         }
@@ -296,17 +326,49 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
 
 template <int D, int DVS>
 struct State {
-    static constexpr int A1 = 2 * 128 * D * 2;  // [K o A; Q o A] hi + lo, K-major, K = D
-    static constexpr int A2 = kA2Bytes;          // [Tb; M'] hi + lo
-    static constexpr int A3 = 2 * C * D * 2;     // (K o e^{Gamma_C - Gamma}) hi + lo, MN-major
-    static constexpr int B1 = 2 * DVS * D * 2;   // S0^T hi + lo, K-major (N = DVS, K = D)
-    static constexpr int B2 = 2 * DVS * C * 2;   // R^T, then U^T: hi + lo, K-major (N = DVS, K = 64)
+    static constexpr int NB = DVS < 64 ? 64 : DVS;  // MN-major B tiles span whole 64-wide atoms
+    static constexpr int A1 = 2 * 128 * D * 2;      // [K o A; Q o A] hi + lo, K-major, K = D
+    static constexpr int A2 = kA2Bytes;             // [Tb; M'] hi + lo
+    static constexpr int A3 = 2 * C * D * 2;        // K o e^{Gamma_C - Gamma} hi + lo, MN-major (M = D, K = 64)
+    static constexpr int B1 = 2 * NB * D * 2;       // S0 hi + lo, MN-major (N = value columns, K = D keys)
+    static constexpr int B2 = 2 * NB * C * 2;       // R, then U: hi + lo, MN-major (N = value columns, K = 64)
+    static constexpr int VP = DVS + 4;              // V row stride (floats): 16-byte skew per row
+    static constexpr int VS = C * VP * 4;           // V rows of the slice, FP32 (prefetched)
+    // operand build: thread = (8-channel group, token segment); the channel groups of one
+    // token are adjacent lanes, so a warp's 16-byte stores cover whole swizzled rows
+    static constexpr int CG = D / 8, SEGS = kThreads / CG, TPS = C / SEGS;
+    static constexpr int SEG = SEGS * D * 4;        // per-segment decay sums
     static constexpr int OFF_A1 = 0, OFF_A2 = OFF_A1 + A1, OFF_A3 = OFF_A2 + A2, OFF_B1 = OFF_A3 + A3,
-                         OFF_B2 = OFF_B1 + B1, OFF_MISC = OFF_B2 + B2;
-    static constexpr int MISC = 4096;
+                         OFF_B2 = OFF_B1 + B1, OFF_V = OFF_B2 + B2, OFF_SEG = OFF_V + VS, OFF_MISC = OFF_SEG + SEG;
+    static constexpr int MISC = 1024;
     static constexpr int bytes = OFF_MISC + MISC + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
 };
+
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Split 8 FP32 values into BF16 hi and lo, packed as two 16-byte chunks (paired conversions).
+__device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) split_bf16x2(x[2 * u], x[2 * u + 1], h[u], l[u]);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void st_pair(uint8_t *tile, int half_bytes, uint32_t off, const float (&x)[8]) {
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4 *>(tile + off) = hi;
+    *reinterpret_cast<uint4 *>(tile + half_bytes + off) = lo;
+}
 
 template <int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -314,17 +376,17 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
              const float *__restrict__ gate, const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state,
              float *__restrict__ core, int T, int T_pad, int H, float scale, int *__restrict__ status) {
     using S = State<D, DVS>;
-    constexpr int TPC = kThreads / D;   // threads per channel in the operand build (2 or 4)
-    constexpr int TOK = C / TPC;        // tokens per thread (32 or 16)
-    constexpr int HALF = DVS / 2;       // value columns per thread in the epilogues
+    constexpr int SEGS = S::SEGS, TPS = S::TPS;
+    constexpr int HALF = DVS / 2;  // value columns per thread in the epilogues
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = sm + S::OFF_A1, *sA2 = sm + S::OFF_A2, *sA3 = sm + S::OFF_A3, *sB1 = sm + S::OFF_B1,
             *sB2 = sm + S::OFF_B2;
+    float *sV = reinterpret_cast<float *>(sm + S::OFF_V);              // [C][VP]
+    float *sSeg = reinterpret_cast<float *>(sm + S::OFF_SEG);          // [SEGS][D]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);  // 0: A2 copy, 1..3: MMA groups
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 64);
-    float *sGseg = reinterpret_cast<float *>(sm + S::OFF_MISC + 128);  // [TPC][D] segment totals
-    float *sAC = sGseg + 4 * D;                                        // [D] A_C = e^{Gamma_C}
+    float *sAC = reinterpret_cast<float *>(sm + S::OFF_MISC + 128);   // [D] A_C = e^{Gamma_C}
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -348,15 +410,56 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
     const uint32_t tD1 = tmem, tD2 = tmem + DVS, tD3 = tmem + 2 * DVS;
     bool ok = true;
 
-    // Epilogue thread roles. For an M = 128 accumulator, warp w reads TMEM lanes 32(w%4)..+31
-    // (rows), columns [ (w/4) * HALF, + HALF ). For D3 with D = 64 (M = 64) the rows are
-    // 16 (w%4) + lane for lanes < 16.
+    // Epilogue roles: for an M = 128 accumulator warp w reads TMEM lanes 32(w%4)..+31 (rows),
+    // value columns [(w/4) HALF, + HALF). D3 with D = 64 (M = 64) has rows 16 (w%4) + lane, lane < 16.
     const int quad = warp & 3, colh = warp >> 2;
-    const int erow = 32 * quad + lane;  // accumulator row of this thread (M = 128 layout)
-    const int ccol = colh * HALF;       // first value column of this thread (within the slice)
-    const int srow = (D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1);  // key row of D3
+    const int erow = 32 * quad + lane;
+    const int ccol = colh * HALF;
+    const int srow = (D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1);
 
-    // FP32 master state slice: key row srow, columns [ccol, ccol + HALF)
+    // Operand-build role: 8 channels [8 cg, 8 cg + 8) x TPS tokens of segment sgm.
+    const int cg = tid % S::CG, sgm = tid / S::CG;
+    const int cb = 8 * cg, tok0 = sgm * TPS;
+    float G[TPS][8], K8[TPS][8], Q8[TPS][8];  // this thread's g, k, q of the next chunk
+    auto load_chunk = [&](int chn) {
+        const int nn = min(C, T - chn * C);
+        const size_t r0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(chn) * C;
+#pragma unroll
+        for (int t = 0; t < TPS; ++t) {
+            const int i = tok0 + t;
+            float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, k0 = g0, k1 = g0, q0 = g0, q1 = g0;
+            if (i < nn) {
+                const size_t off = (r0 + i) * rs + static_cast<size_t>(h) * D + cb;
+                g0 = *reinterpret_cast<const float4 *>(gate + off);
+                g1 = *reinterpret_cast<const float4 *>(gate + off + 4);
+                k0 = *reinterpret_cast<const float4 *>(k + off);
+                k1 = *reinterpret_cast<const float4 *>(k + off + 4);
+                q0 = *reinterpret_cast<const float4 *>(q + off);
+                q1 = *reinterpret_cast<const float4 *>(q + off + 4);
+            }
+            G[t][0] = g0.x; G[t][1] = g0.y; G[t][2] = g0.z; G[t][3] = g0.w;
+            G[t][4] = g1.x; G[t][5] = g1.y; G[t][6] = g1.z; G[t][7] = g1.w;
+            K8[t][0] = k0.x; K8[t][1] = k0.y; K8[t][2] = k0.z; K8[t][3] = k0.w;
+            K8[t][4] = k1.x; K8[t][5] = k1.y; K8[t][6] = k1.z; K8[t][7] = k1.w;
+            Q8[t][0] = q0.x; Q8[t][1] = q0.y; Q8[t][2] = q0.z; Q8[t][3] = q0.w;
+            Q8[t][4] = q1.x; Q8[t][5] = q1.y; Q8[t][6] = q1.z; Q8[t][7] = q1.w;
+        }
+    };
+
+    // V rows of the slice for epilogue 1, prefetched one chunk ahead into shared memory: the
+    // thread that reads row erow, columns [ccol, ccol + HALF) is the thread that copies them.
+    auto prefetch_v = [&](int chn) {
+        if (quad < 2) {
+            const int nn = min(C, T - chn * C);
+            const size_t r0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(chn) * C;
+            const float *src = v + (r0 + (erow < nn ? erow : 0)) * rs + static_cast<size_t>(h) * D + c0 + ccol;
+#pragma unroll
+            for (int j = 0; j < HALF; j += 4) cp_async16(sV + erow * S::VP + ccol + j, src + j, erow < nn ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+
+    // FP32 master state slice: key row srow, value columns [ccol, ccol + HALF)
     float st[HALF];
     if (srow >= 0) {
 #pragma unroll
@@ -365,20 +468,21 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
             st[j] = x.x; st[j + 1] = x.y; st[j + 2] = x.z; st[j + 3] = x.w;
         }
     }
-    // S0^T into B1: element (n = value column, k = key row)
+    // S0 into B1 (MN-major: element (n = value column, k = key row)), 16-byte chunks
     auto write_state_operand = [&]() {
         if (srow >= 0) {
 #pragma unroll
-            for (int j = 0; j < HALF; ++j) {
-                uint16_t hi, lo;
-                split_bf16(st[j], hi, lo);
-                const uint32_t off = kmaj_off(ccol + j, srow, DVS);
-                *reinterpret_cast<uint16_t *>(sB1 + off) = hi;
-                *reinterpret_cast<uint16_t *>(sB1 + S::B1 / 2 + off) = lo;
+            for (int j = 0; j < HALF; j += 8) {
+                float x[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) x[u] = st[j + u];
+                st_pair(sB1, S::B1 / 2, mnmaj_off(ccol + j, srow, D), x);
             }
         }
     };
     write_state_operand();
+    load_chunk(0);
+    prefetch_v(0);
 
 #pragma unroll 1
     for (int ch = 0; ch < nch; ++ch) {
@@ -397,120 +501,114 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
                 "l"(src), "r"(kA2Bytes), "r"(smem_u32(&bars[0]))
                 : "memory");
         }
-        // ---- operands from q, k, g: thread (channel c, token segment sg)
+        // ---- operand build: cumulative decay over the segments (sums exchanged through shared
+        //      memory), then running products of a = e^g inside the segment.
         {
-            const int c = tid % D, sg = tid / D, t0 = sg * TOK;
-            float g[TOK];
+            float seg[8];
 #pragma unroll
-            for (int t = 0; t < TOK; ++t) {
-                const int i = t0 + t;
-                g[t] = i < n ? gate[(row0 + i) * rs + static_cast<size_t>(h) * D + c] : 0.f;
+            for (int u = 0; u < 8; ++u) {
+                float sum = 0.f;
+#pragma unroll
+                for (int t = 0; t < TPS; ++t) sum += G[t][u];
+                seg[u] = sum;
             }
-            // segment sums -> exclusive prefix over segments
-            float tot = 0.f;
-#pragma unroll
-            for (int t = 0; t < TOK; ++t) tot += g[t];
-            sGseg[sg * D + c] = tot;
+            *reinterpret_cast<float4 *>(sSeg + sgm * D + cb) = make_float4(seg[0], seg[1], seg[2], seg[3]);
+            *reinterpret_cast<float4 *>(sSeg + sgm * D + cb + 4) = make_float4(seg[4], seg[5], seg[6], seg[7]);
             __syncthreads();
-            float pre = 0.f, all = 0.f;
+            float pre[8], tot[8];
 #pragma unroll
-            for (int s2 = 0; s2 < TPC; ++s2) {
-                const float x = sGseg[s2 * D + c];
-                if (s2 < sg) pre += x;
-                all += x;
-            }
-            if (sg == 0) sAC[c] = expf(all);
-            // e^{Gamma_i} by a forward running product (K o A, Q o A), then e^{Gamma_C - Gamma_i}
-            // by a backward one (K o e^{Gamma_C - Gamma}); only a = e^g and k stay in registers.
-            float av[TOK], kk[TOK];
-            float f = expf(pre);
+            for (int u = 0; u < 8; ++u) { pre[u] = 0.f; tot[u] = 0.f; }
+#pragma unroll 4
+            for (int s2 = 0; s2 < SEGS; ++s2) {
+                const float4 x0 = *reinterpret_cast<const float4 *>(sSeg + s2 * D + cb);
+                const float4 x1 = *reinterpret_cast<const float4 *>(sSeg + s2 * D + cb + 4);
+                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-            for (int t = 0; t < TOK; ++t) {
-                const int i = t0 + t;
-                av[t] = expf(g[t]);
-                f *= av[t];
-                float kv = 0.f, qv = 0.f;
-                if (i < n) {
-                    const size_t off = (row0 + i) * rs + static_cast<size_t>(h) * D + c;
-                    kv = k[off];
-                    qv = q[off];
+                for (int u = 0; u < 8; ++u) {
+                    if (s2 < sgm) pre[u] += xs[u];
+                    tot[u] += xs[u];
                 }
-                kk[t] = kv;
-                uint16_t hi, lo;
-                split_bf16(kv * f, hi, lo);
-                uint32_t off = kmaj_off(i, c, 128);
-                *reinterpret_cast<uint16_t *>(sA1 + off) = hi;
-                *reinterpret_cast<uint16_t *>(sA1 + S::A1 / 2 + off) = lo;
-                split_bf16(qv * f, hi, lo);
-                off = kmaj_off(64 + i, c, 128);
-                *reinterpret_cast<uint16_t *>(sA1 + off) = hi;
-                *reinterpret_cast<uint16_t *>(sA1 + S::A1 / 2 + off) = lo;
             }
-            // Gamma_C - Gamma_{t0+TOK-1} = the sum of the later segments
-            float fb = expf(all - pre - tot);
+            float f[8], fb[8];
 #pragma unroll
-            for (int t = TOK - 1; t >= 0; --t) {
-                uint16_t hi, lo;
-                split_bf16(kk[t] * fb, hi, lo);
-                const uint32_t off = mnmaj_off(c, t0 + t, C);
-                *reinterpret_cast<uint16_t *>(sA3 + off) = hi;
-                *reinterpret_cast<uint16_t *>(sA3 + S::A3 / 2 + off) = lo;
-                fb *= av[t];
+            for (int u = 0; u < 8; ++u) {
+                f[u] = __expf(pre[u]);                    // e^{Gamma before the segment}
+                fb[u] = __expf(tot[u] - pre[u] - seg[u]);  // e^{Gamma_C - Gamma at the segment's last token}
+            }
+            if (sgm == 0) {
+                *reinterpret_cast<float4 *>(sAC + cb) = make_float4(__expf(tot[0]), __expf(tot[1]), __expf(tot[2]), __expf(tot[3]));
+                *reinterpret_cast<float4 *>(sAC + cb + 4) = make_float4(__expf(tot[4]), __expf(tot[5]), __expf(tot[6]), __expf(tot[7]));
+            }
+#pragma unroll
+            for (int t = 0; t < TPS; ++t) {
+                const int i = tok0 + t;
+                float xk[8], xq[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    G[t][u] = __expf(G[t][u]);  // a = e^g from here on
+                    f[u] *= G[t][u];
+                    xk[u] = K8[t][u] * f[u];
+                    xq[u] = Q8[t][u] * f[u];
+                }
+                st_pair(sA1, S::A1 / 2, kmaj_off(i, cb, 128), xk);
+                st_pair(sA1, S::A1 / 2, kmaj_off(64 + i, cb, 128), xq);
+            }
+#pragma unroll
+            for (int t = TPS - 1; t >= 0; --t) {
+                float xb[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    xb[u] = K8[t][u] * fb[u];
+                    fb[u] *= G[t][u];
+                }
+                st_pair(sA3, S::A3 / 2, mnmaj_off(cb, tok0 + t, C), xb);
             }
         }
+        // prefetch the next chunk's g, k, q while this chunk's MMAs run
+        if (ch + 1 < nch) load_chunk(ch + 1);
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
         tc_fence_after();
         // ---- MMA1: D1 = [K o A; Q o A] . S0
         if (tid == 0 && ok) {
-            constexpr uint32_t id = idesc_bf16(128, DVS, false, false);
+            constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
             const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
             int acc = 0;
 #pragma unroll 1
             for (int ks = 0; ks < D / 16; ++ks) {
                 const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + S::A1 / 2, 128, 0, ks);
-                const uint64_t bh = kmaj_desc(b0, DVS, 0, ks), bl = kmaj_desc(b0 + S::B1 / 2, DVS, 0, ks);
+                const uint64_t bh = mnmaj_desc(b0, D, 0, ks), bl = mnmaj_desc(b0 + S::B1 / 2, D, 0, ks);
                 mma_bf16(tD1, ah, bh, id, acc); acc = 1;
                 mma_bf16(tD1, ah, bl, id, 1);
                 mma_bf16(tD1, al, bh, id, 1);
             }
             mma_commit(&bars[1]);
         }
-        // e1: V rows of this thread for R (rows 0..63, quads 0 and 1), or the Q half of D1
-        // kept for the output (rows 64..127, quads 2 and 3)
+        // e1: the Q half of D1 kept for the output (rows 64..127, quads 2 and 3)
         float e1[HALF];
-        if (quad < 2) {
-            const int i = erow;
-#pragma unroll
-            for (int j = 0; j < HALF; j += 4) {
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < n) x = *reinterpret_cast<const float4 *>(v + (row0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j);
-                e1[j] = x.x; e1[j + 1] = x.y; e1[j + 2] = x.z; e1[j + 3] = x.w;
-            }
-        }
+        cp_async_wait_all();  // this thread's V rows of this chunk are in sV
         ok = ok && mbar_wait(&bars[1], par, kWaitCycles);
         tc_fence_after();
-        // ---- epilogue 1: R = V - D1[0:64] -> R^T into B2
+        // ---- epilogue 1: R = V - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
             float x[8];
             tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
             tmem_ld_wait();
             if (quad < 2) {
+                const float4 v0 = *reinterpret_cast<const float4 *>(sV + erow * S::VP + ccol + j);
+                const float4 v1 = *reinterpret_cast<const float4 *>(sV + erow * S::VP + ccol + j + 4);
+                const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    uint16_t hi, lo;
-                    split_bf16(e1[j + u] - x[u], hi, lo);
-                    const uint32_t off = kmaj_off(ccol + j + u, erow, DVS);
-                    *reinterpret_cast<uint16_t *>(sB2 + off) = hi;
-                    *reinterpret_cast<uint16_t *>(sB2 + S::B2 / 2 + off) = lo;
-                }
+                for (int u = 0; u < 8; ++u) x[u] = vv[u] - x[u];
+                st_pair(sB2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
             } else {
 #pragma unroll
                 for (int u = 0; u < 8; ++u) e1[j + u] = x[u];
             }
         }
+        if (ch + 1 < nch) prefetch_v(ch + 1);  // this thread is done with its V rows of this chunk
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
@@ -518,13 +616,13 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         // ---- MMA2: D2 = [Tb; M'] . R  (after the bulk copy of the tile has landed)
         if (tid == 0 && ok) ok = mbar_wait(&bars[0], par, kWaitCycles);
         if (tid == 0 && ok) {
-            constexpr uint32_t id = idesc_bf16(128, DVS, false, false);
+            constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
             const uint32_t a0 = smem_u32(sA2), b0 = smem_u32(sB2);
             int acc = 0;
 #pragma unroll 1
             for (int ks = 0; ks < C / 16; ++ks) {
                 const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + kTileBytes, 128, 0, ks);
-                const uint64_t bh = kmaj_desc(b0, DVS, 0, ks), bl = kmaj_desc(b0 + S::B2 / 2, DVS, 0, ks);
+                const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
                 mma_bf16(tD2, ah, bh, id, acc); acc = 1;
                 mma_bf16(tD2, ah, bl, id, 1);
                 mma_bf16(tD2, al, bh, id, 1);
@@ -533,21 +631,14 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         }
         ok = ok && mbar_wait(&bars[2], par, kWaitCycles);
         tc_fence_after();
-        // ---- epilogue 2: U = D2[0:64] -> U^T into B2 (R^T is consumed); O = scale (D1q + D2q)
+        // ---- epilogue 2: U = D2[0:64] -> B2 (R is consumed); O = scale (D1[64:] + D2[64:])
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
             float x[8];
             tmem_ld8(tmem_lane_base(tD2, warp) + ccol + j, x);
             tmem_ld_wait();
             if (quad < 2) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    uint16_t hi, lo;
-                    split_bf16(x[u], hi, lo);
-                    const uint32_t off = kmaj_off(ccol + j + u, erow, DVS);
-                    *reinterpret_cast<uint16_t *>(sB2 + off) = hi;
-                    *reinterpret_cast<uint16_t *>(sB2 + S::B2 / 2 + off) = lo;
-                }
+                st_pair(sB2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
             } else {
                 const int i = erow - 64;
                 if (i < n) {
@@ -567,13 +658,13 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         tc_fence_after();
         // ---- MMA3: D3 = (K o e^{Gamma_C - Gamma})^T . U
         if (tid == 0 && ok) {
-            constexpr uint32_t id = idesc_bf16(D, DVS, true, false);
+            constexpr uint32_t id = idesc_bf16(D, DVS, true, true);
             const uint32_t a0 = smem_u32(sA3), b0 = smem_u32(sB2);
             int acc = 0;
 #pragma unroll 1
             for (int ks = 0; ks < C / 16; ++ks) {
                 const uint64_t ah = mnmaj_desc(a0, C, 0, ks), al = mnmaj_desc(a0 + S::A3 / 2, C, 0, ks);
-                const uint64_t bh = kmaj_desc(b0, DVS, 0, ks), bl = kmaj_desc(b0 + S::B2 / 2, DVS, 0, ks);
+                const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
                 mma_bf16(tD3, ah, bh, id, acc); acc = 1;
                 mma_bf16(tD3, ah, bl, id, 1);
                 mma_bf16(tD3, al, bh, id, 1);
@@ -582,7 +673,7 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         }
         ok = ok && mbar_wait(&bars[3], par, kWaitCycles);
         tc_fence_after();
-        // ---- epilogue 3: S = A_C o S0 + D3 (FP32 in registers), S^T split into B1
+        // ---- epilogue 3: S = A_C o S0 + D3 (FP32 in registers), S into B1
         {
             const float ac = srow >= 0 ? sAC[srow] : 0.f;
 #pragma unroll
@@ -635,7 +726,7 @@ int launch_tc(const float *q, const float *k, const float *v, const float *gate,
         KDA_TRY(set_smem(state_kernel<D, DVS>, State<D, DVS>::bytes));
         attrs = true;
     }
-    intra_kernel<D><<<dim3(T_pad / C, H, B), kThreads, Intra<D>::bytes, s>>>(
+    intra_kernel<D><<<dim3(T_pad / C, H, B), kIntraThreads, Intra<D>::bytes, s>>>(
         k, q, gate, beta, static_cast<uint8_t *>(scratch), T, T_pad, H);
     KDA_TRY(launch_status());
     state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(
