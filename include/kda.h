@@ -129,6 +129,32 @@ KDA_API int kda_chunk_prefill(const float *q, const float *k, const float *v, co
 /* Scratch bytes kda_chunk_prefill needs for B streams of T tokens (0 if B or T is 0). */
 KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dims);
 
+/* kda_chunk_prefill_noalloc — kda_chunk_prefill for callers that cannot allocate device
+ * memory (the pages have no counterpart: this is a deployment variant). Some callers cannot
+ * call cudaMalloc at all: an engine that hands all free HBM to its KV-cache / state pools at
+ * start-up has no room left for a scratch buffer, and a plug-in inside a host framework that
+ * owns the memory budget may not allocate behind its back. This entry point allocates
+ * nothing and takes no scratch argument: it uses one file-scope device array of
+ * kda_chunk_prefill_noalloc_max_scratch_bytes() bytes (32 MiB), which every GPU that loads
+ * the library holds until the process exits.
+ *   - Arguments, layouts and results are exactly those of kda_chunk_prefill.
+ *   - Requests needing more scratch than that (kda_chunk_prefill_scratch_bytes(B, T, dims)
+ *     above the maximum, i.e. B * heads * ceil(T / 64) > 1024 chunk tiles) are rejected with
+ *     KDA_ERR_CAPACITY before anything runs.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents. Nothing in it
+ *     needs to start at zero (each call writes every tile it later reads), but calls that
+ *     overlap on the GPU (different streams, or different host threads) race on it:
+ *     serialise them.
+ */
+KDA_API int kda_chunk_prefill_noalloc(const float *q, const float *k, const float *v, const float *gate,
+                                      const float *beta, float *const *h_state, float *core, int B, int T,
+                                      const kda_dims *dims, void *stream);
+
+/* Size in bytes of the device array kda_chunk_prefill_noalloc uses (32 MiB). */
+KDA_API size_t kda_chunk_prefill_noalloc_max_scratch_bytes(void);
+
 /* kda_chunk_prefill_simt — the same contract as kda_chunk_prefill, computed by the
  * plain FP32 CUDA-core kernel (no tensor cores). Kept as a second implementation. */
 KDA_API int kda_chunk_prefill_simt(const float *q, const float *k, const float *v, const float *gate,

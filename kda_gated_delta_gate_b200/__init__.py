@@ -54,6 +54,8 @@ _SIGS = {
     "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_prefill_simt": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
+    "kda_chunk_prefill_noalloc": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
+    "kda_chunk_prefill_noalloc_max_scratch_bytes": ([], ctypes.c_size_t),
     "kda_recurrent_decode": ([_VP] * 7 + [_I, _DIMS, _VP], _I),
     "kda_decode_fused": ([_VP] * 13 + [_I, _DIMS, _VP], _I),
     "kda_decode_k": ([_VP] * 13 + [_I, _VP, _VP, _I, _DIMS, _VP], _I),
@@ -154,6 +156,13 @@ def kda_chunk_prefill(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d
         scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     return _call("kda_chunk_prefill", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core), B, T,
                  _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+
+
+def kda_chunk_prefill_noalloc(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None):
+    """kda_chunk_prefill without a scratch argument, for callers that cannot allocate: the
+    library's own 32 MiB device array is used (calls must not overlap on the GPU)."""
+    return _call("kda_chunk_prefill_noalloc", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core),
+                 B, T, ctypes.byref(d), _stream(stream))
 
 
 def kda_recurrent_decode(q, k, v, gate, beta, h_state_ptrs, o, N: int, d: KdaDims, stream=None):
