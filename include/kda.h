@@ -116,9 +116,9 @@ KDA_API int kda_beta(const float *b_logit, float *beta, int n, void *stream);
  *   core      [B*T_pad, H, D] F32 output o = scale * S^T q for rows < T (pad rows are
  *             not written).
  *   scratch   caller-owned device scratch of at least kda_chunk_prefill_scratch_bytes(B, T,
- *             dims) bytes, 16-byte aligned (per-chunk operand tiles passed between the two
- *             kernels of the call); contents on entry do not matter. KDA_ERR_CAPACITY if
- *             scratch_bytes is too small.
+ *             dims) bytes (129 KB per (stream, head, chunk) at head_dim 128), 16-byte aligned:
+ *             the per-chunk operand tiles passed between the two kernels of the call; contents
+ *             on entry do not matter. KDA_ERR_CAPACITY if scratch_bytes is too small.
  * Computed with tcgen05 tensor cores in split-BF16 precision (about 2^-16 relative per
  * product). The per-(stream, head) states must not overlap each other or any input.
  */
@@ -139,8 +139,8 @@ KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dim
  * the library holds until the process exits.
  *   - Arguments, layouts and results are exactly those of kda_chunk_prefill.
  *   - Requests needing more scratch than that (kda_chunk_prefill_scratch_bytes(B, T, dims)
- *     above the maximum, i.e. B * heads * ceil(T / 64) > 1024 chunk tiles) are rejected with
- *     KDA_ERR_CAPACITY before anything runs.
+ *     above the maximum; for head_dim 128, B * heads * ceil(T / 64) > 254 chunks) are
+ *     rejected with KDA_ERR_CAPACITY before anything runs.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *     with that device current; make that first call before any stream capture.
  *   - Every call shares the one array and it keeps the last call's contents. Nothing in it

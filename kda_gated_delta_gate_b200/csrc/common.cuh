@@ -72,7 +72,7 @@ int chunk_prefill_check(const float *q, const float *k, const float *v, const fl
                         float *const *h_state, float *core, int B, int T, const kda_dims *dims);
 int chunk_prefill_simt(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                        float *const *h_state, float *core, int B, int T, const kda_dims *dims, cudaStream_t s);
-size_t chunk_prefill_scratch_bytes(int B, int T, int H);
+size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D);
 int chunk_prefill_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                      float *const *h_state, float *core, int B, int T, const kda_dims *dims, void *scratch,
                      cudaStream_t s);

@@ -66,7 +66,7 @@ int kda_device_status(int *out, int clear) {
 
 extern "C" size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dims) {
     if (kda::check_dims(dims) != KDA_OK) return 0;
-    return kda::chunk_prefill_scratch_bytes(B, T, dims->heads);
+    return kda::chunk_prefill_scratch_bytes(B, T, dims->heads, dims->head_dim);
 }
 
 extern "C" int kda_chunk_prefill(const float *q, const float *k, const float *v, const float *gate,
@@ -76,7 +76,7 @@ extern "C" int kda_chunk_prefill(const float *q, const float *k, const float *v,
     if (B == 0 || T == 0) return KDA_OK;
     if (!scratch) return KDA_ERR_INVALID_ARG;
     if (!kda::aligned16(scratch)) return KDA_ERR_MISALIGNED;
-    if (scratch_bytes < kda::chunk_prefill_scratch_bytes(B, T, dims->heads)) return KDA_ERR_CAPACITY;
+    if (scratch_bytes < kda::chunk_prefill_scratch_bytes(B, T, dims->heads, dims->head_dim)) return KDA_ERR_CAPACITY;
     return kda::chunk_prefill_tc(q, k, v, gate, beta, h_state, core, B, T, dims, scratch,
                                  static_cast<cudaStream_t>(stream));
 }

@@ -48,7 +48,8 @@ extern "C" int kda_chunk_prefill_noalloc(const float *q, const float *k, const f
                                          const kda_dims *dims, void *stream) {
     KDA_TRY(kda::chunk_prefill_check(q, k, v, gate, beta, h_state, core, B, T, dims));
     if (B == 0 || T == 0) return KDA_OK;
-    if (kda::chunk_prefill_scratch_bytes(B, T, dims->heads) > kda::kNoAllocScratchBytes) return KDA_ERR_CAPACITY;
+    if (kda::chunk_prefill_scratch_bytes(B, T, dims->heads, dims->head_dim) > kda::kNoAllocScratchBytes)
+        return KDA_ERR_CAPACITY;
     void *scratch = nullptr;
     KDA_TRY(kda::scratch_address(&scratch));
     return kda::chunk_prefill_tc(q, k, v, gate, beta, h_state, core, B, T, dims, scratch,

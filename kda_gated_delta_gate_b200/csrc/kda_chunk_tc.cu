@@ -26,6 +26,8 @@
 //    O = scale (D1[64:128] + D2[64:128]);  S = A_C o S0 + D3 (FP32 master copy in registers).
 // Rows >= T of the last chunk are loaded as zeros (k = q = v = 0, g = 0, beta = 0): the pad
 // guard. They add nothing to L, M, R, U or the state, and their outputs are not written.
+#include <algorithm>
+
 #include "common.cuh"
 #include "umma.cuh"
 
@@ -38,7 +40,40 @@ constexpr int C = kChunk;          // 64
 constexpr int kThreads = 256;
 constexpr int kTileBytes = 16384;  // one 128 x 64 BF16 K-major tile
 constexpr int kA2Bytes = 2 * kTileBytes;
+
+// Per (stream, head, chunk) the intra kernel writes one pack of state-independent operands,
+// each a BF16 hi tile followed by its lo tile, laid out exactly as the state kernel's shared
+// memory wants them (so a bulk copy moves each):
+//   A1 [K o A; Q o A]           128 x D, K-major          (A = e^Gamma)
+//   A2 [Tb; M']                 128 x 64, K-major
+//   A3 K o e^{Gamma_C - Gamma}  D (M) x 64 (K), MN-major
+//   AC e^{Gamma_C}              D FP32 (1 KB slot)
+template <int D>
+struct Pack {
+    static constexpr int A1 = 2 * 128 * D * 2;
+    static constexpr int A2 = kA2Bytes;
+    static constexpr int A3 = 2 * C * D * 2;
+    static constexpr int AC = 1024;
+    static constexpr int OFF_A1 = 0, OFF_A2 = A1, OFF_A3 = A1 + A2, OFF_AC = A1 + A2 + A3;
+    static constexpr int bytes = A1 + A2 + A3 + AC;
+};
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 1.9 GHz
+
+// Split 8 FP32 values into BF16 hi and lo, packed as two 16-byte chunks (paired conversions).
+__device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) split_bf16x2(x[2 * u], x[2 * u + 1], h[u], l[u]);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void st_pair(uint8_t *tile, int half_bytes, uint32_t off, const float (&x)[8]) {
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4 *>(tile + off) = hi;
+    *reinterpret_cast<uint4 *>(tile + half_bytes + off) = lo;
+}
 
 // ================================================================ phase 1: intra-chunk
 
@@ -48,22 +83,25 @@ template <int D>
 struct Intra {
     static constexpr int P = D + 8;   // fp32 row stride of [C][D] tiles (bank-spread, 16-B aligned)
     static constexpr int PC = C + 1;  // row stride of [C][C] tiles
-    static constexpr int NZ = 48;     // rows of the block-local backward factors (blocks 0..2)
+    static constexpr int NZ = 64;     // rows of the block-local backward factors
     static constexpr size_t floats = 3 * C * P + NZ * P + 3 * C * PC + 4 * D + C + 3 * 256;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
+// The exact CUDA-core intra-chunk computation of one (stream b, head h, chunk ch): every decay
+// factor is a product of per-token factors <= 1, whatever g holds. It writes the whole operand
+// pack. Used for the chunks whose in-block decay is too strong for the tensor-core path.
 template <int D>
-__global__ void __launch_bounds__(kIntraThreads, 1)
-intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
-             const float *__restrict__ beta, uint8_t *__restrict__ scratch, int T, int T_pad, int H) {
+__device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, const float *__restrict__ q,
+                                                const float *__restrict__ gate, const float *__restrict__ beta,
+                                                uint8_t *__restrict__ scratch, int T, int T_pad, int H, int b,
+                                                int h, int ch, float *smem) {
     using I = Intra<D>;
     constexpr int P = I::P, PC = I::PC, NT = kIntraThreads;
-    extern __shared__ float smem[];
-    float *sK = smem;              // k, then X (rows 16..63): k_i prod_{s=16a}^{i} a_s
-    float *sQ = sK + C * P;        // q, then Y (rows 16..63): q_i prod_{s=16a}^{i} a_s
+    float *sK = smem;              // k, then X: k_i prod_{s=16a}^{i} a_s  (a = block of i)
+    float *sQ = sK + C * P;        // q, then Y: q_i prod_{s=16a}^{i} a_s
     float *sA = sQ + C * P;        // a = e^g
-    float *sZ = sA + C * P;        // Z (rows 0..47): k_j prod_{s=j+1}^{16b+15} a_s
+    float *sZ = sA + C * P;        // Z: k_j prod_{s=j+1}^{16b+15} a_s
     float *sL = sZ + I::NZ * P;    // L' (unscaled), then M'
     float *sM = sL + C * PC;       // M
     float *sT = sM + C * PC;       // T, then Tb
@@ -72,7 +110,6 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     float *sTmp = sB + C;          // [3][256]
 
     const int tid = threadIdx.x;
-    const int ch = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int n = min(C, T - ch * C);
     const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
     const size_t rs = static_cast<size_t>(H) * D;
@@ -143,19 +180,15 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     if (tid < 4 * D) {
         const int c = tid % D, a = tid / D;
         float f = 1.f;
-        if (a < 3) {
-            for (int j = 16 * a + 15; j >= 16 * a; --j) {
-                sZ[j * P + c] = sK[j * P + c] * f;
-                f *= sA[j * P + c];
-            }
-        } else {
-            for (int j = 16 * a + 15; j >= 16 * a; --j) f *= sA[j * P + c];
+        for (int j = 16 * a + 15; j >= 16 * a; --j) {
+            sZ[j * P + c] = sK[j * P + c] * f;
+            f *= sA[j * P + c];
         }
         sF[a * D + c] = f;
     }
     __syncthreads();
-    if (tid < 3 * D) {
-        const int c = tid % D, a = 1 + tid / D;
+    if (tid < 4 * D) {
+        const int c = tid % D, a = tid / D;
         float f = 1.f;
         for (int i = 16 * a; i < 16 * a + 16; ++i) {
             f *= sA[i * P + c];
@@ -233,6 +266,42 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     }
     __syncthreads();
 
+    // ---- the state kernel's operands for this chunk: K o A = X P_a, Q o A = Y P_a and
+    //      K o e^{Gamma_C - Gamma} = Z S_a, with P_a / S_a the decay of all blocks before / after
+    //      block a; 16-byte chunks of 8 channels written straight into the pack.
+    using PK = Pack<D>;
+    uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * (T_pad / C) + ch) * PK::bytes;
+    for (int e = tid; e < C * (D / 8); e += NT) {
+        const int i = e / (D / 8), cb = 8 * (e % (D / 8)), a = i >> 4;
+        float xk[8], xq[8], xb[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c = cb + u;
+            float pre = 1.f, suf = 1.f;
+            for (int bb = 0; bb < a; ++bb) pre *= sF[bb * D + c];
+            for (int bb = a + 1; bb < 4; ++bb) suf *= sF[bb * D + c];
+            xk[u] = sK[i * P + c] * pre;
+            xq[u] = sQ[i * P + c] * pre;
+            xb[u] = sZ[i * P + c] * suf;
+        }
+        uint4 hi, lo;
+        split8(xk, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
+        split8(xq, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
+        split8(xb, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
+    }
+    if (tid < D) {
+        float acv = 1.f;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) acv *= sF[bb * D + tid];
+        reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = acv;
+    }
+
     // ---- L = diag(beta) L' (strict lower). T = (I + L)^-1: 16x16 diagonal blocks by
     //      substitution, then off-diagonal blocks T_ab = -T_aa sum_{b<=c<a} L_ac T_cb.
     for (int e = tid; e < C * C; e += NT) {
@@ -298,7 +367,7 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     }
     __syncthreads();
     // ---- write [Tb; M'] as BF16 hi and lo K-major swizzled tiles (128 rows x 64 columns)
-    uint8_t *dst = scratch + ((static_cast<size_t>(b) * H + h) * (T_pad / C) + ch) * kA2Bytes;
+    uint8_t *dst = pack + PK::OFF_A2;
     for (int e = tid; e < 128 * 8; e += NT) {
         const int row = e >> 3, c0 = 8 * (e & 7);
         float x[8];
@@ -322,24 +391,355 @@ intra_kernel(const float *__restrict__ k, const float *__restrict__ q, const flo
     }
 }
 
+// All chunks through the CUDA-core body (grid = chunks x heads x streams).
+template <int D>
+__global__ void __launch_bounds__(kIntraThreads, 1)
+intra_simt_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
+                  const float *__restrict__ beta, uint8_t *__restrict__ scratch, int T, int T_pad, int H) {
+    extern __shared__ float smem[];
+    intra_simt_body<D>(k, q, gate, beta, scratch, T, T_pad, H, blockIdx.z, blockIdx.y, blockIdx.x, smem);
+}
+
+// Only the chunks the tensor-core kernel listed (count and packed (b, h, ch) entries in scratch).
+template <int D>
+__global__ void __launch_bounds__(kIntraThreads, 1)
+intra_fix_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
+                 const float *__restrict__ beta, uint8_t *__restrict__ scratch, const int *__restrict__ list,
+                 int T, int T_pad, int H) {
+    extern __shared__ float smem[];
+    const int count = list[0];
+    const int nch = T_pad / C;
+    for (int e = blockIdx.x; e < count; e += gridDim.x) {
+        const int id = list[1 + e];
+        const int ch = id % nch, h = (id / nch) % H, b = id / (nch * H);
+        intra_simt_body<D>(k, q, gate, beta, scratch, T, T_pad, H, b, h, ch, smem);
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- intra-chunk on tensor cores
+//
+// L' and M for all pairs of the chunk in one tcgen05 MMA. Each 16-token block a gets the
+// reference point m_a = 16a + 7 (its middle). With Gamma the in-chunk cumulative decay,
+//   A rows  i (block a):      k_i e^{Gamma_i - Gamma_{m_a}}   (and q_i ... for rows 64 + i)
+//   B rows  (a', j), j <= 16a'+15:  k_j e^{Gamma_{m_a'} - Gamma_j}
+// so D[i][(a, j)] = sum_c k_ic k_jc e^{Gamma_ic - Gamma_jc} = L'[i][j] exactly for every j <= i
+// (the reference cancels). B holds the 16, 32, 48, 64 rows of a' = 0..3 at column offsets
+// 0, 16, 48, 96 (160 rows). Factors above 1 come only from decay inside one block (at most
+// 8 tokens); a chunk whose |Gamma_i - Gamma_{m_a}| exceeds kRefBound for some channel is
+// handed to the CUDA-core body instead (listed in scratch, run by intra_fix_kernel).
+
+constexpr float kRefBound = 80.0f;  // e^80 and e^-80 are comfortably inside BF16/FP32 range
+
+template <int D>
+struct IntraTC {
+    static constexpr int NB = 160;                  // B rows
+    static constexpr int A_BYTES = 2 * 128 * D * 2;  // A hi + lo (K-major, K = D)
+    static constexpr int B_BYTES = 2 * NB * D * 2;   // B hi + lo
+    static constexpr int GP = D + 4;                // Gamma row stride (floats)
+    static constexpr int PC = C + 1;
+    static constexpr int LMT = 3 * C * PC * 4;     // L, M, T (FP32); Gamma lives here first
+    static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_LMT = A_BYTES + B_BYTES, OFF_TAB = OFF_LMT + LMT;
+    static constexpr int TAB = 14 * D * 4;          // per-channel reference factors
+    static constexpr int OFF_MISC = OFF_TAB + TAB;  // beta[C], tmp[768], barrier, tmem slot, flags
+    static constexpr int MISC = (C + 768) * 4 + 256;
+    static constexpr int bytes = OFF_MISC + MISC + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kIntraThreads, 1)
+intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
+                const float *__restrict__ beta, uint8_t *__restrict__ scratch, int *__restrict__ list, int T,
+                int T_pad, int H, int *__restrict__ status) {
+    using I = IntraTC<D>;
+    using PK = Pack<D>;
+    constexpr int NT = kIntraThreads, GP = I::GP, PC = I::PC;
+    constexpr int CG = D / 8;                 // 8-channel groups
+    constexpr int UPT = C * CG / NT;          // (token, group) units per thread: 2 (D=128) or 1
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = sm + I::OFF_A, *sBt = sm + I::OFF_B;
+    float *sG = reinterpret_cast<float *>(sm + I::OFF_LMT);  // Gamma [C][GP], before L/M/T
+    float *sL = reinterpret_cast<float *>(sm + I::OFF_LMT);  // L' then M'
+    float *sM = sL + C * PC;
+    float *sT = sM + C * PC;
+    float *sTab = reinterpret_cast<float *>(sm + I::OFF_TAB);
+    float *sB = reinterpret_cast<float *>(sm + I::OFF_MISC);
+    float *sTmp = sB + C;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + (C + 768) * 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
+    // reference tables, [entry][D]: 0..3 e^{Gamma_{m_a}}, 4..7 e^{Gamma_C - Gamma_{m_a}},
+    // 8..13 e^{Gamma_{m_a} - Gamma_{m_b}} for (a,b) = (1,0),(2,0),(2,1),(3,0),(3,1),(3,2)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ch = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n = min(C, T - ch * C);
+    const int nch = T_pad / C;
+    const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
+    const size_t rs = static_cast<size_t>(H) * D;
+    uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * nch + ch) * PK::bytes;
+
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    // ---- load: unit (token i, 8-channel group); g goes to shared memory for the scan
+    float kk[UPT][8], qq[UPT][8];
+#pragma unroll
+    for (int u = 0; u < UPT; ++u) {
+        const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
+        float4 k0 = make_float4(0.f, 0.f, 0.f, 0.f), k1 = k0, q0 = k0, q1 = k0, g0 = k0, g1 = k0;
+        if (i < n) {
+            const size_t off = (row0 + i) * rs + static_cast<size_t>(h) * D + cb;
+            k0 = *reinterpret_cast<const float4 *>(k + off);
+            k1 = *reinterpret_cast<const float4 *>(k + off + 4);
+            q0 = *reinterpret_cast<const float4 *>(q + off);
+            q1 = *reinterpret_cast<const float4 *>(q + off + 4);
+            g0 = *reinterpret_cast<const float4 *>(gate + off);
+            g1 = *reinterpret_cast<const float4 *>(gate + off + 4);
+        }
+        kk[u][0] = k0.x; kk[u][1] = k0.y; kk[u][2] = k0.z; kk[u][3] = k0.w;
+        kk[u][4] = k1.x; kk[u][5] = k1.y; kk[u][6] = k1.z; kk[u][7] = k1.w;
+        qq[u][0] = q0.x; qq[u][1] = q0.y; qq[u][2] = q0.z; qq[u][3] = q0.w;
+        qq[u][4] = q1.x; qq[u][5] = q1.y; qq[u][6] = q1.z; qq[u][7] = q1.w;
+        *reinterpret_cast<float4 *>(sG + i * GP + cb) = g0;
+        *reinterpret_cast<float4 *>(sG + i * GP + cb + 4) = g1;
+    }
+    if (tid < C) sB[tid] = tid < n ? beta[(row0 + tid) * H + h] : 0.f;
+    __syncthreads();
+    // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, quarter of 16 tokens)
+    {
+        constexpr int QT = NT / D;  // 4 (D=128) or 8 (D=64) token ranges
+        constexpr int TPQ = C / QT;
+        const int c = tid % D, qr = tid / D;
+        float acc = 0.f;
+        for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) { acc += sG[i * GP + c]; sG[i * GP + c] = acc; }
+        sTmp[qr * D + c] = acc;
+        __syncthreads();
+        float pre = 0.f;
+        for (int r = 0; r < qr; ++r) pre += sTmp[r * D + c];
+        if (qr > 0)
+            for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * GP + c] += pre;
+        __syncthreads();
+    }
+    if (tid < D) {
+        const int c = tid;
+        const float gm[4] = {sG[7 * GP + c], sG[23 * GP + c], sG[39 * GP + c], sG[55 * GP + c]};
+        const float gc = sG[63 * GP + c];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            sTab[a * D + c] = __expf(gm[a]);
+            sTab[(4 + a) * D + c] = __expf(gc - gm[a]);
+        }
+        sTab[8 * D + c] = __expf(gm[1] - gm[0]);
+        sTab[9 * D + c] = __expf(gm[2] - gm[0]);
+        sTab[10 * D + c] = __expf(gm[2] - gm[1]);
+        sTab[11 * D + c] = __expf(gm[3] - gm[0]);
+        sTab[12 * D + c] = __expf(gm[3] - gm[1]);
+        sTab[13 * D + c] = __expf(gm[3] - gm[2]);
+    }
+    __syncthreads();
+    // ---- operands: A (mid-block reference), B (all references), and the state kernel's pack
+    bool safe = true;
+#pragma unroll
+    for (int u = 0; u < UPT; ++u) {
+        const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
+        float ef[8], ei[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const float r = sG[i * GP + cb + w] - sG[(16 * a + 7) * GP + cb + w];
+            safe = safe && fabsf(r) <= kRefBound;
+            ef[w] = __expf(r);
+            ei[w] = __expf(-r);
+        }
+        float x[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
+        st_pair(sA, I::A_BYTES / 2, kmaj_off(i, cb, 128), x);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w];
+        st_pair(sA, I::A_BYTES / 2, kmaj_off(64 + i, cb, 128), x);
+        // B rows for every reference block a2 >= a (column offsets 0, 16, 48, 96)
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2) {
+            if (a2 < a) continue;
+            const int off2 = 8 * a2 * (a2 + 1);
+            const int tix = a2 == a ? -1 : (a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13))));
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * (tix < 0 ? 1.f : sTab[tix * D + cb + w]);
+            st_pair(sBt, I::B_BYTES / 2, kmaj_off(off2 + i, cb, I::NB), x);
+        }
+        // the state kernel's operands: K o e^Gamma, Q o e^Gamma, K o e^{Gamma_C - Gamma}
+        uint4 hi, lo;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w] * sTab[a * D + cb + w];
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w] * sTab[a * D + cb + w];
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * sTab[(4 + a) * D + cb + w];
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
+    }
+    if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
+    fence_async_smem();
+    tc_fence_before();
+    safe = __syncthreads_and(safe) != 0;
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    if (safe) {
+        // ---- D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127)
+        if (tid == 0) {
+            constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
+#pragma unroll 1
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
+                const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
+                mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
+                mma_bf16(tmem, ah, bl, id, 1);
+                mma_bf16(tmem, al, bh, id, 1);
+            }
+            mma_commit(bar);
+        }
+        ok = mbar_wait(bar, 0, kWaitCycles);
+        tc_fence_after();
+        // ---- read back: warp (quad, part); row r = 32 quad + lane (i = r % 64, block a = i / 16)
+        //      needs columns [off_a, off_a + 16(a+1)); the quad's window is [0, 48) for rows in
+        //      blocks 0-1 and [48, 160) for blocks 2-3, split over the 4 warps of the quad.
+        {
+            const int quad = warp & 3, part = warp >> 2;
+            const int r = 32 * quad + lane, i = r & 63, a = i >> 4;
+            const int off_a = 8 * a * (a + 1);
+            const int w0 = (quad & 1) ? 48 : 0, wlen = (quad & 1) ? 112 : 48;
+            float *dstm = r < 64 ? sL : sM;
+            for (int c8 = part * 8; c8 < wlen; c8 += 32) {
+                float x[8];
+                tmem_ld8(tmem_lane_base(tmem, warp) + w0 + c8, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    const int j = w0 + c8 + w - off_a;
+                    if (j >= 0 && j <= i) dstm[i * PC + j] = x[w];
+                }
+            }
+        }
+        tc_fence_before();
+    }
+    ok = __syncthreads_and(ok) != 0;
+    if (!safe || !ok) {
+        // the CUDA-core body redoes this chunk (it rewrites the whole pack)
+        if (tid == 0) {
+            if (!ok) atomicExch(status, KDA_ERR_TIMEOUT);
+            const int slot = atomicAdd(list, 1);
+            list[1 + slot] = (b * H + h) * nch + ch;
+        }
+    } else {
+        // ---- L = diag(beta) L' (strict lower). T = (I + L)^-1 as in the CUDA-core body.
+        for (int e = tid; e < C * C; e += NT) {
+            const int i = e / C, j = e % C;
+            if (i > j) sL[i * PC + j] *= sB[i];
+        }
+        __syncthreads();
+        if (tid < 64) {
+            const int a = tid / 16, j = tid % 16, base = 16 * a;
+            float t[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float val = (i == j) ? 1.f : 0.f;
+                if (i > j) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m2 = 0; m2 < 16; ++m2)
+                        if (m2 >= j && m2 < i) acc = fmaf(sL[(base + i) * PC + base + m2], t[m2], acc);
+                    val = -acc;
+                }
+                t[i] = val;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sT[(base + i) * PC + base + j] = t[i];
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int dist = 1; dist < 4; ++dist) {
+            const int npairs = 4 - dist;
+            for (int e = tid; e < npairs * 256; e += NT) {
+                const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
+                const int bb = pr, aa = pr + dist;
+                float acc = 0.f;
+                for (int cb2 = bb; cb2 < aa; ++cb2)
+#pragma unroll
+                    for (int m2 = 0; m2 < 16; ++m2)
+                        acc = fmaf(sL[(16 * aa + i) * PC + 16 * cb2 + m2], sT[(16 * cb2 + m2) * PC + 16 * bb + j], acc);
+                sTmp[pr * 256 + i * 16 + j] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < npairs * 256; e += NT) {
+                const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
+                const int bb = pr, aa = pr + dist;
+                float acc = 0.f;
+#pragma unroll
+                for (int m2 = 0; m2 < 16; ++m2)
+                    acc = fmaf(sT[(16 * aa + i) * PC + 16 * aa + m2], sTmp[pr * 256 + m2 * 16 + j], acc);
+                sT[(16 * aa + i) * PC + 16 * bb + j] = -acc;
+            }
+            __syncthreads();
+        }
+        for (int e = tid; e < C * C; e += NT) {
+            const int i = e / C, j = e % C;
+            if (j <= i) sT[i * PC + j] *= sB[j];
+        }
+        __syncthreads();
+        for (int e = tid; e < C * C; e += NT) {
+            const int i = e / C, l = e % C;
+            float acc = 0.f;
+            for (int j = l; j <= i; ++j) acc = fmaf(sM[i * PC + j], sT[j * PC + l], acc);
+            sL[i * PC + l] = acc;
+        }
+        __syncthreads();
+        uint8_t *dst = pack + PK::OFF_A2;
+        for (int e = tid; e < 128 * 8; e += NT) {
+            const int row = e >> 3, c0 = 8 * (e & 7);
+            float x[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const int col = c0 + w;
+                x[w] = row < 64 ? (col <= row ? sT[row * PC + col] : 0.f) : sL[(row - 64) * PC + col];
+            }
+            uint4 hi, lo;
+            split8(x, hi, lo);
+            const uint32_t off = kmaj_off(row, c0, 128);
+            *reinterpret_cast<uint4 *>(dst + off) = hi;
+            *reinterpret_cast<uint4 *>(dst + kTileBytes + off) = lo;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
 // ================================================================ phase 2: state pass
 
 template <int D, int DVS>
 struct State {
+    using PK = Pack<D>;
     static constexpr int NB = DVS < 64 ? 64 : DVS;  // MN-major B tiles span whole 64-wide atoms
-    static constexpr int A1 = 2 * 128 * D * 2;      // [K o A; Q o A] hi + lo, K-major, K = D
-    static constexpr int A2 = kA2Bytes;             // [Tb; M'] hi + lo
-    static constexpr int A3 = 2 * C * D * 2;        // K o e^{Gamma_C - Gamma} hi + lo, MN-major (M = D, K = 64)
     static constexpr int B1 = 2 * NB * D * 2;       // S0 hi + lo, MN-major (N = value columns, K = D keys)
     static constexpr int B2 = 2 * NB * C * 2;       // R, then U: hi + lo, MN-major (N = value columns, K = 64)
     static constexpr int VP = DVS + 4;              // V row stride (floats): 16-byte skew per row
     static constexpr int VS = C * VP * 4;           // V rows of the slice, FP32 (prefetched)
-    // operand build: thread = (8-channel group, token segment); the channel groups of one
-    // token are adjacent lanes, so a warp's 16-byte stores cover whole swizzled rows
-    static constexpr int CG = D / 8, SEGS = kThreads / CG, TPS = C / SEGS;
-    static constexpr int SEG = SEGS * D * 4;        // per-segment decay sums
-    static constexpr int OFF_A1 = 0, OFF_A2 = OFF_A1 + A1, OFF_A3 = OFF_A2 + A2, OFF_B1 = OFF_A3 + A3,
-                         OFF_B2 = OFF_B1 + B1, OFF_V = OFF_B2 + B2, OFF_SEG = OFF_V + VS, OFF_MISC = OFF_SEG + SEG;
+    // A1, A2, A3 at the front, in the pack's own order and sizes
+    static constexpr int OFF_A1 = 0, OFF_A2 = PK::A1, OFF_A3 = PK::A1 + PK::A2, OFF_B1 = OFF_A3 + PK::A3,
+                         OFF_B2 = OFF_B1 + B1, OFF_V = OFF_B2 + B2, OFF_MISC = OFF_V + VS;
     static constexpr int MISC = 1024;
     static constexpr int bytes = OFF_MISC + MISC + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
@@ -354,39 +754,30 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uin
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Split 8 FP32 values into BF16 hi and lo, packed as two 16-byte chunks (paired conversions).
-__device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) split_bf16x2(x[2 * u], x[2 * u + 1], h[u], l[u]);
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-__device__ __forceinline__ void st_pair(uint8_t *tile, int half_bytes, uint32_t off, const float (&x)[8]) {
-    uint4 hi, lo;
-    split8(x, hi, lo);
-    *reinterpret_cast<uint4 *>(tile + off) = hi;
-    *reinterpret_cast<uint4 *>(tile + half_bytes + off) = lo;
+// Issue a bulk global -> shared copy of `bytes` (multiple of 16) completing on `bar`.
+__device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
 template <int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
-state_kernel(const float *__restrict__ q, const float *__restrict__ k, const float *__restrict__ v,
-             const float *__restrict__ gate, const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state,
+state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state,
              float *__restrict__ core, int T, int T_pad, int H, float scale, int *__restrict__ status) {
     using S = State<D, DVS>;
-    constexpr int SEGS = S::SEGS, TPS = S::TPS;
+    using PK = Pack<D>;
     constexpr int HALF = DVS / 2;  // value columns per thread in the epilogues
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = sm + S::OFF_A1, *sA2 = sm + S::OFF_A2, *sA3 = sm + S::OFF_A3, *sB1 = sm + S::OFF_B1,
             *sB2 = sm + S::OFF_B2;
     float *sV = reinterpret_cast<float *>(sm + S::OFF_V);              // [C][VP]
-    float *sSeg = reinterpret_cast<float *>(sm + S::OFF_SEG);          // [SEGS][D]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);  // 0: A2 copy, 1..3: MMA groups
+    // barriers: 0/4/5 bulk copies of A1/A2/A3, 1..3 the three MMA groups
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 64);
-    float *sAC = reinterpret_cast<float *>(sm + S::OFF_MISC + 128);   // [D] A_C = e^{Gamma_C}
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -394,10 +785,14 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
     const size_t rs = static_cast<size_t>(H) * D;
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
     const int nch = T_pad / C;
+    const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
+        bulk_copy(sA1, packs + PK::OFF_A1, PK::A1, &bars[0]);
+        bulk_copy(sA2, packs + PK::OFF_A2, PK::A2, &bars[4]);
+        bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[5]);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -416,35 +811,6 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
     const int erow = 32 * quad + lane;
     const int ccol = colh * HALF;
     const int srow = (D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1);
-
-    // Operand-build role: 8 channels [8 cg, 8 cg + 8) x TPS tokens of segment sgm.
-    const int cg = tid % S::CG, sgm = tid / S::CG;
-    const int cb = 8 * cg, tok0 = sgm * TPS;
-    float G[TPS][8], K8[TPS][8], Q8[TPS][8];  // this thread's g, k, q of the next chunk
-    auto load_chunk = [&](int chn) {
-        const int nn = min(C, T - chn * C);
-        const size_t r0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(chn) * C;
-#pragma unroll
-        for (int t = 0; t < TPS; ++t) {
-            const int i = tok0 + t;
-            float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, k0 = g0, k1 = g0, q0 = g0, q1 = g0;
-            if (i < nn) {
-                const size_t off = (r0 + i) * rs + static_cast<size_t>(h) * D + cb;
-                g0 = *reinterpret_cast<const float4 *>(gate + off);
-                g1 = *reinterpret_cast<const float4 *>(gate + off + 4);
-                k0 = *reinterpret_cast<const float4 *>(k + off);
-                k1 = *reinterpret_cast<const float4 *>(k + off + 4);
-                q0 = *reinterpret_cast<const float4 *>(q + off);
-                q1 = *reinterpret_cast<const float4 *>(q + off + 4);
-            }
-            G[t][0] = g0.x; G[t][1] = g0.y; G[t][2] = g0.z; G[t][3] = g0.w;
-            G[t][4] = g1.x; G[t][5] = g1.y; G[t][6] = g1.z; G[t][7] = g1.w;
-            K8[t][0] = k0.x; K8[t][1] = k0.y; K8[t][2] = k0.z; K8[t][3] = k0.w;
-            K8[t][4] = k1.x; K8[t][5] = k1.y; K8[t][6] = k1.z; K8[t][7] = k1.w;
-            Q8[t][0] = q0.x; Q8[t][1] = q0.y; Q8[t][2] = q0.z; Q8[t][3] = q0.w;
-            Q8[t][4] = q1.x; Q8[t][5] = q1.y; Q8[t][6] = q1.z; Q8[t][7] = q1.w;
-        }
-    };
 
     // V rows of the slice for epilogue 1, prefetched one chunk ahead into shared memory: the
     // thread that reads row erow, columns [ccol, ccol + HALF) is the thread that copies them.
@@ -481,103 +847,32 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         }
     };
     write_state_operand();
-    load_chunk(0);
     prefetch_v(0);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
 #pragma unroll 1
     for (int ch = 0; ch < nch; ++ch) {
         const int n = min(C, T - ch * C);
         const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
         const uint32_t par = ch & 1;
-        // ---- bulk copy of this chunk's [Tb; M'] tile (the previous MMA2 finished reading A2)
-        if (tid == 0) {
-            const uint8_t *src = scratch + ((static_cast<size_t>(b) * H + h) * nch + ch) * kA2Bytes;
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bars[0])),
-                         "r"(kA2Bytes)
-                         : "memory");
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                    smem_u32(sA2)),
-                "l"(src), "r"(kA2Bytes), "r"(smem_u32(&bars[0]))
-                : "memory");
-        }
-        // ---- operand build: cumulative decay over the segments (sums exchanged through shared
-        //      memory), then running products of a = e^g inside the segment.
-        {
-            float seg[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                float sum = 0.f;
-#pragma unroll
-                for (int t = 0; t < TPS; ++t) sum += G[t][u];
-                seg[u] = sum;
-            }
-            *reinterpret_cast<float4 *>(sSeg + sgm * D + cb) = make_float4(seg[0], seg[1], seg[2], seg[3]);
-            *reinterpret_cast<float4 *>(sSeg + sgm * D + cb + 4) = make_float4(seg[4], seg[5], seg[6], seg[7]);
-            __syncthreads();
-            float pre[8], tot[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) { pre[u] = 0.f; tot[u] = 0.f; }
-#pragma unroll 4
-            for (int s2 = 0; s2 < SEGS; ++s2) {
-                const float4 x0 = *reinterpret_cast<const float4 *>(sSeg + s2 * D + cb);
-                const float4 x1 = *reinterpret_cast<const float4 *>(sSeg + s2 * D + cb + 4);
-                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    if (s2 < sgm) pre[u] += xs[u];
-                    tot[u] += xs[u];
-                }
-            }
-            float f[8], fb[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                f[u] = __expf(pre[u]);                    // e^{Gamma before the segment}
-                fb[u] = __expf(tot[u] - pre[u] - seg[u]);  // e^{Gamma_C - Gamma at the segment's last token}
-            }
-            if (sgm == 0) {
-                *reinterpret_cast<float4 *>(sAC + cb) = make_float4(__expf(tot[0]), __expf(tot[1]), __expf(tot[2]), __expf(tot[3]));
-                *reinterpret_cast<float4 *>(sAC + cb + 4) = make_float4(__expf(tot[4]), __expf(tot[5]), __expf(tot[6]), __expf(tot[7]));
-            }
-#pragma unroll
-            for (int t = 0; t < TPS; ++t) {
-                const int i = tok0 + t;
-                float xk[8], xq[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    G[t][u] = __expf(G[t][u]);  // a = e^g from here on
-                    f[u] *= G[t][u];
-                    xk[u] = K8[t][u] * f[u];
-                    xq[u] = Q8[t][u] * f[u];
-                }
-                st_pair(sA1, S::A1 / 2, kmaj_off(i, cb, 128), xk);
-                st_pair(sA1, S::A1 / 2, kmaj_off(64 + i, cb, 128), xq);
-            }
-#pragma unroll
-            for (int t = TPS - 1; t >= 0; --t) {
-                float xb[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    xb[u] = K8[t][u] * fb[u];
-                    fb[u] *= G[t][u];
-                }
-                st_pair(sA3, S::A3 / 2, mnmaj_off(cb, tok0 + t, C), xb);
-            }
-        }
-        // prefetch the next chunk's g, k, q while this chunk's MMAs run
-        if (ch + 1 < nch) load_chunk(ch + 1);
-        fence_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;
-        tc_fence_after();
-        // ---- MMA1: D1 = [K o A; Q o A] . S0
+        const uint8_t *next = packs + static_cast<size_t>(ch + 1) * PK::bytes;
+        const bool more = ch + 1 < nch;
+        // e^{Gamma_C} of this thread's key row, read early (used in epilogue 3)
+        const float ac = srow >= 0 ? reinterpret_cast<const float *>(packs + static_cast<size_t>(ch) * PK::bytes +
+                                                                    PK::OFF_AC)[srow]
+                                   : 0.f;
+        // ---- MMA1: D1 = [K o A; Q o A] . S0   (A1 copied for this chunk)
+        if (tid == 0 && ok) ok = mbar_wait(&bars[0], par, kWaitCycles);
         if (tid == 0 && ok) {
             constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
             const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
             int acc = 0;
-#pragma unroll 1
+#pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + S::A1 / 2, 128, 0, ks);
+                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + PK::A1 / 2, 128, 0, ks);
                 const uint64_t bh = mnmaj_desc(b0, D, 0, ks), bl = mnmaj_desc(b0 + S::B1 / 2, D, 0, ks);
                 mma_bf16(tD1, ah, bh, id, acc); acc = 1;
                 mma_bf16(tD1, ah, bl, id, 1);
@@ -590,6 +885,7 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         cp_async_wait_all();  // this thread's V rows of this chunk are in sV
         ok = ok && mbar_wait(&bars[1], par, kWaitCycles);
         tc_fence_after();
+        if (tid == 0 && ok && more) bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);  // A1 is free again
         // ---- epilogue 1: R = V - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
@@ -608,18 +904,18 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
                 for (int u = 0; u < 8; ++u) e1[j + u] = x[u];
             }
         }
-        if (ch + 1 < nch) prefetch_v(ch + 1);  // this thread is done with its V rows of this chunk
+        if (more) prefetch_v(ch + 1);  // this thread is done with its V rows of this chunk
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
         tc_fence_after();
-        // ---- MMA2: D2 = [Tb; M'] . R  (after the bulk copy of the tile has landed)
-        if (tid == 0 && ok) ok = mbar_wait(&bars[0], par, kWaitCycles);
+        // ---- MMA2: D2 = [Tb; M'] . R
+        if (tid == 0 && ok) ok = mbar_wait(&bars[4], par, kWaitCycles);
         if (tid == 0 && ok) {
             constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
             const uint32_t a0 = smem_u32(sA2), b0 = smem_u32(sB2);
             int acc = 0;
-#pragma unroll 1
+#pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
                 const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + kTileBytes, 128, 0, ks);
                 const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
@@ -631,6 +927,7 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         }
         ok = ok && mbar_wait(&bars[2], par, kWaitCycles);
         tc_fence_after();
+        if (tid == 0 && ok && more) bulk_copy(sA2, next + PK::OFF_A2, PK::A2, &bars[4]);  // A2 is free again
         // ---- epilogue 2: U = D2[0:64] -> B2 (R is consumed); O = scale (D1[64:] + D2[64:])
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
@@ -657,13 +954,14 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         ok = __syncthreads_and(ok) != 0;
         tc_fence_after();
         // ---- MMA3: D3 = (K o e^{Gamma_C - Gamma})^T . U
+        if (tid == 0 && ok) ok = mbar_wait(&bars[5], par, kWaitCycles);
         if (tid == 0 && ok) {
             constexpr uint32_t id = idesc_bf16(D, DVS, true, true);
             const uint32_t a0 = smem_u32(sA3), b0 = smem_u32(sB2);
             int acc = 0;
-#pragma unroll 1
+#pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t ah = mnmaj_desc(a0, C, 0, ks), al = mnmaj_desc(a0 + S::A3 / 2, C, 0, ks);
+                const uint64_t ah = mnmaj_desc(a0, C, 0, ks), al = mnmaj_desc(a0 + PK::A3 / 2, C, 0, ks);
                 const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
                 mma_bf16(tD3, ah, bh, id, acc); acc = 1;
                 mma_bf16(tD3, ah, bl, id, 1);
@@ -673,18 +971,16 @@ state_kernel(const float *__restrict__ q, const float *__restrict__ k, const flo
         }
         ok = ok && mbar_wait(&bars[3], par, kWaitCycles);
         tc_fence_after();
+        if (tid == 0 && ok && more) bulk_copy(sA3, next + PK::OFF_A3, PK::A3, &bars[5]);  // A3 is free again
         // ---- epilogue 3: S = A_C o S0 + D3 (FP32 in registers), S into B1
-        {
-            const float ac = srow >= 0 ? sAC[srow] : 0.f;
 #pragma unroll
-            for (int j = 0; j < HALF; j += 8) {
-                float x[8];
-                tmem_ld8(tmem_lane_base(tD3, warp) + ccol + j, x);
-                tmem_ld_wait();
-                if (srow >= 0) {
+        for (int j = 0; j < HALF; j += 8) {
+            float x[8];
+            tmem_ld8(tmem_lane_base(tD3, warp) + ccol + j, x);
+            tmem_ld_wait();
+            if (srow >= 0) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) st[j + u] = fmaf(ac, st[j + u], x[u]);
-                }
+                for (int u = 0; u < 8; ++u) st[j + u] = fmaf(ac, st[j + u], x[u]);
             }
         }
         write_state_operand();
@@ -714,31 +1010,53 @@ int set_smem(K kernel, int bytes) {
                : KDA_ERR_CUDA;
 }
 
+// Scratch layout: the operand packs, then a 256-byte slot with the count of chunks the
+// tensor-core intra kernel handed to the CUDA-core body, then their (b, h, chunk) ids.
+template <int D>
+size_t packs_bytes(int B, int H, int nch) { return static_cast<size_t>(B) * H * nch * Pack<D>::bytes; }
+
 template <int D, int DVS>
 int launch_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
               float *const *h_state, float *core, int B, int T, int H, float scale, void *scratch, cudaStream_t s) {
     const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C));
+    const int nch = T_pad / C;
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
     static bool attrs = false;
     if (!attrs) {
-        KDA_TRY(set_smem(intra_kernel<D>, static_cast<int>(Intra<D>::bytes)));
+        KDA_TRY(set_smem(intra_tc_kernel<D>, IntraTC<D>::bytes));
+        KDA_TRY(set_smem(intra_fix_kernel<D>, static_cast<int>(Intra<D>::bytes)));
         KDA_TRY(set_smem(state_kernel<D, DVS>, State<D, DVS>::bytes));
         attrs = true;
     }
-    intra_kernel<D><<<dim3(T_pad / C, H, B), kIntraThreads, Intra<D>::bytes, s>>>(
-        k, q, gate, beta, static_cast<uint8_t *>(scratch), T, T_pad, H);
+    uint8_t *sc = static_cast<uint8_t *>(scratch);
+    int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(B, H, nch));
+    if (cudaMemsetAsync(list, 0, sizeof(int), s) != cudaSuccess) return KDA_ERR_CUDA;
+    intra_tc_kernel<D><<<dim3(nch, H, B), kIntraThreads, IntraTC<D>::bytes, s>>>(k, q, gate, beta, sc, list, T, T_pad,
+                                                                                 H, status);
+    KDA_TRY(launch_status());
+    int sms = 148;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int fix_grid = static_cast<int>(std::min<long long>(static_cast<long long>(B) * H * nch, sms));
+    intra_fix_kernel<D><<<fix_grid, kIntraThreads, Intra<D>::bytes, s>>>(k, q, gate, beta, sc, list, T, T_pad, H);
     KDA_TRY(launch_status());
     state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(
-        q, k, v, gate, static_cast<const uint8_t *>(scratch), h_state, core, T, T_pad, H, scale, status);
+        v, sc, h_state, core, T, T_pad, H, scale, status);
     return launch_status();
 }
 
 }  // namespace
 
-size_t chunk_prefill_scratch_bytes(int B, int T, int H) {
+size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D) {
     if (B <= 0 || T <= 0 || H <= 0) return 0;
-    return static_cast<size_t>(B) * H * (kda_t_pad(static_cast<size_t>(T), C) / C) * kA2Bytes;
+    const int nch = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C) / C);
+    const size_t packs = D == 64 ? packs_bytes<64>(B, H, nch) : packs_bytes<128>(B, H, nch);
+    const size_t list = (4 + 4 * static_cast<size_t>(B) * H * nch + 255) / 256 * 256;
+    return packs + list;
 }
 
 int chunk_prefill_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,

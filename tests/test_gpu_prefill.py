@@ -103,6 +103,20 @@ def test_poison_pad_tail(impl):
     _check(ci, outs[1][0], outs[1][1])
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_prefill_extreme_decay_takes_exact_path(D):
+    """One head with a decay of hundreds of nats per token in some channels (beyond what the
+    tensor-core intra path accepts inside a 16-token block): those chunks are recomputed by the
+    exact CUDA-core path; all heads still match the oracle."""
+    ci = core_inputs(1, 200, 3, D, seed=31, s0_std=0.1)
+    ci.a_log[1] = 3.0                      # exp(3) = 20 on head 1
+    ci.dt_bias[1 * D + 5] = 20.0           # softplus ~ 20: g ~ -400 per token on one channel
+    ci.dt_bias[1 * D + 9] = 6.0
+    for impl in IMPLS:
+        core, S, _ = gpu_prefill(ci, impl=impl)
+        _check(ci, core, S)
+
+
 def test_tc_and_simt_agree():
     ci = core_inputs(2, 333, 4, 128, seed=12, s0_std=0.1)
     a, Sa, _ = gpu_prefill(ci, impl="tc")
