@@ -245,6 +245,77 @@ KDA_API int kda_front_conv_silu_l2(const kda_bf16 *x, kda_bf16 *conv_state, cons
 KDA_API int kda_back_gated_rmsnorm(const float *core, const kda_bf16 *out_gate, const kda_bf16 *w,
                            kda_bf16 *out, int T, const kda_dims *dims, void *stream);
 
+/* ---------------------------------------------------------------------------------
+ * kda_gemm_bf16 — C[M x N] = A[M x K] . W[N x K]^T with BF16 A and W (torch Linear
+ * layout [out, in], Glm5NextKdaWeights) and FP32 accumulation on the tensor cores; C is
+ * BF16 (out_f32 = 0) or FP32 (out_f32 = 1). Row strides lda, ldw, ldc in elements (ldc lets a
+ * projection write into a column range of a wider row, e.g. the packed q|k|v rows).
+ * K a multiple of 64; A and W 16-byte aligned with lda/ldw multiples of 8 (TMA tiles). M and N
+ * are free (tiles are masked); C rows are written with 16-byte stores when C is 16-byte aligned
+ * and ldc a multiple of 8 (BF16) / 4 (FP32), element by element otherwise.
+ */
+KDA_API int kda_gemm_bf16(const kda_bf16 *A, int lda, const kda_bf16 *W, int ldw, void *C, int ldc, int M, int N,
+                          int K, int out_f32, void *stream);
+
+/* ---------------------------------------------------------------------------------
+ * Block prefill: one KDA block over T tokens of one sequence (Glm5NextKdaLayer `prefill` /
+ * `prefill_with_pad_fill`), stage by stage into a workspace (Glm5NextKdaWorkspace) that is
+ * allocated once for max_tokens. Weights are device pointers in the layouts of
+ * Glm5NextKdaWeights; hidden, rank and H*D multiples of 64.
+ */
+typedef struct kda_block_weights {
+    const kda_bf16 *q_proj, *k_proj, *v_proj; /* [H*D, hidden] each                     */
+    const kda_bf16 *conv;                     /* [3*H*D, 4] depthwise conv (q|k|v)       */
+    const kda_bf16 *f_a;                      /* [rank, hidden]                          */
+    const kda_bf16 *f_b;                      /* [H*D, rank]                             */
+    const float *dt_bias;                     /* [H*D] F32, per channel                  */
+    const float *a_log;                       /* [H] F32, per head                       */
+    const kda_bf16 *b_proj;                   /* [H, hidden]                             */
+    const kda_bf16 *g_a;                      /* [rank, hidden]                          */
+    const kda_bf16 *g_b;                      /* [H*D, rank]                             */
+    const kda_bf16 *o_norm;                   /* [D]                                     */
+    const kda_bf16 *o_proj;                   /* [hidden, H*D]                           */
+    int hidden, rank;
+} kda_block_weights;
+
+/* Workspace stage buffers (kda_workspace_buffer): shapes for T tokens, T_pad = kda_t_pad(T, 64). */
+enum {
+    KDA_BUF_QKV_PROJ = 0,   /* [T, 3*H*D] BF16  q|k|v projections                  */
+    KDA_BUF_CONV_OUT,       /* [T, 3*H*D] BF16  after conv + SiLU, q|k normalised  */
+    KDA_BUF_Q_F32,          /* [T_pad, H*D] F32                                    */
+    KDA_BUF_K_F32,          /* [T_pad, H*D] F32                                    */
+    KDA_BUF_V_F32,          /* [T_pad, H*D] F32                                    */
+    KDA_BUF_GATE,           /* [T_pad, H, D] F32 log-decay                         */
+    KDA_BUF_BETA,           /* [T_pad, H] F32                                      */
+    KDA_BUF_CORE,           /* [T_pad, H, D] F32 KDA output before o_norm          */
+    KDA_BUF_G_RAW,          /* [T, H*D] BF16  f_b(f_a(h))                           */
+    KDA_BUF_OUT_GATE,       /* [T, H*D] BF16  g_b(g_a(h))                           */
+    KDA_BUF_O_NORM_OUT,     /* [T, H*D] BF16                                       */
+    KDA_BUF_FINAL_OUT,      /* [T, hidden] BF16  block output                      */
+    KDA_BUF_F_A_OUT,        /* [T, rank] BF16                                      */
+    KDA_BUF_G_A_OUT,        /* [T, rank] BF16                                      */
+    KDA_BUF_PREFILL_SCRATCH,/* chunked-prefill scratch                             */
+    KDA_BUF_COUNT
+};
+
+typedef struct kda_workspace kda_workspace;
+
+/* Allocate the workspace for up to max_tokens tokens (the only allocating call). */
+KDA_API int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_tokens,
+                                 kda_workspace **out);
+KDA_API int kda_workspace_destroy(kda_workspace *ws);
+KDA_API size_t kda_workspace_max_tokens(const kda_workspace *ws);
+/* Device pointer and size of one stage buffer (the buffers are public so each stage can be
+ * compared on its own, as the workspace page intends). */
+KDA_API int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr, size_t *bytes);
+
+/* kda_block_prefill — hidden [T, hidden] BF16 (device); h_state [H, D, D] F32 and conv_state
+ * [3*H*D, 3] BF16 are carried and updated in place; pad_fill primes the q/k/v tails
+ * (Glm5NextKdaLayer `prefill_with_pad_fill`; 0 for `prefill`). The block output lands in
+ * KDA_BUF_FINAL_OUT. KDA_ERR_CAPACITY if T > max_tokens. Allocates nothing. */
+KDA_API int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T, float *h_state,
+                              kda_bf16 *conv_state, float pad_fill, kda_workspace *ws, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,6 +38,16 @@ def dims(heads: int, head_dim: int, chunk: int = 64, scale: float = 1.0, l2_eps:
     return KdaDims(heads, head_dim, chunk, scale, l2_eps, rms_eps)
 
 
+class KdaBlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q_proj", "k_proj", "v_proj", "conv", "f_a", "f_b", "dt_bias",
+                                                  "a_log", "b_proj", "g_a", "g_b", "o_norm", "o_proj")] + \
+               [("hidden", ctypes.c_int), ("rank", ctypes.c_int)]
+
+
+# workspace stage buffers (include/kda.h, KDA_BUF_*)
+BUFFERS = ("qkv_proj", "conv_out", "q_f32", "k_f32", "v_f32", "gate", "beta", "core", "g_raw", "out_gate",
+           "o_norm_out", "final_out", "f_a_out", "g_a_out", "prefill_scratch")
+
 _lib = None
 _VP = ctypes.c_void_p
 _I = ctypes.c_int
@@ -61,6 +71,12 @@ _SIGS = {
     "kda_decode_k": ([_VP] * 13 + [_I, _VP, _VP, _I, _DIMS, _VP], _I),
     "kda_front_conv_silu_l2": ([_VP] * 7 + [_F, _I, _DIMS, _VP], _I),
     "kda_back_gated_rmsnorm": ([_VP] * 4 + [_I, _DIMS, _VP], _I),
+    "kda_gemm_bf16": ([_VP, _I, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP], _I),
+    "kda_workspace_create": ([_DIMS, _I, _I, ctypes.c_size_t, ctypes.POINTER(_VP)], _I),
+    "kda_workspace_destroy": ([_VP], _I),
+    "kda_workspace_max_tokens": ([_VP], ctypes.c_size_t),
+    "kda_workspace_buffer": ([_VP, _I, ctypes.POINTER(_VP), ctypes.POINTER(ctypes.c_size_t)], _I),
+    "kda_block_prefill": ([_VP, _VP, _I, _VP, _VP, _F, _VP, _VP], _I),
 }
 
 
@@ -197,3 +213,83 @@ def kda_front_conv_silu_l2(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32,
 def kda_back_gated_rmsnorm(core, out_gate, w, out, T: int, d: KdaDims, stream=None):
     return _call("kda_back_gated_rmsnorm", _p(core), _p(out_gate), _p(w), _p(out), T, ctypes.byref(d),
                  _stream(stream))
+
+
+def kda_gemm_bf16(A, W, C, M: int, N: int, K: int, *, lda=None, ldw=None, ldc=None, stream=None):
+    """C[M x N] = A[M x K] . W[N x K]^T (BF16 in, FP32 accumulate); C's dtype picks the output."""
+    import torch
+    out_f32 = 1 if C.dtype == torch.float32 else 0
+    return _call("kda_gemm_bf16", _p(A), lda if lda is not None else A.stride(0), _p(W),
+                 ldw if ldw is not None else W.stride(0), _p(C), ldc if ldc is not None else C.stride(0), M, N, K,
+                 out_f32, _stream(stream))
+
+
+def block_weights_struct(w) -> KdaBlockWeights:
+    """KdaBlockWeights from an object with device tensors q_proj, ..., o_proj and ints hidden, rank."""
+    return KdaBlockWeights(*[_p(getattr(w, n)) for n in ("q_proj", "k_proj", "v_proj", "conv", "f_a", "f_b",
+                                                          "dt_bias", "a_log", "b_proj", "g_a", "g_b", "o_norm",
+                                                          "o_proj")], w.hidden, w.rank)
+
+
+class Workspace:
+    """The block prefill's stage buffers, allocated once for max_tokens (kda_workspace_create)."""
+
+    def __init__(self, d: KdaDims, hidden: int, rank: int, max_tokens: int):
+        self.dims = d
+        self._h = ctypes.c_void_p()
+        _call("kda_workspace_create", ctypes.byref(d), hidden, rank, max_tokens, ctypes.byref(self._h))
+
+    @property
+    def handle(self):
+        return self._h
+
+    def buffer(self, name: str):
+        """(device pointer, bytes) of a stage buffer."""
+        ptr, nb = ctypes.c_void_p(), ctypes.c_size_t()
+        _call("kda_workspace_buffer", self._h, BUFFERS.index(name), ctypes.byref(ptr), ctypes.byref(nb))
+        return ptr.value, nb.value
+
+    def view(self, name: str, shape, dtype):
+        """A torch view of (the front of) a stage buffer; the workspace must outlive it."""
+        import torch
+        ptr, nb = self.buffer(name)
+        n = 1
+        for x in shape:
+            n *= x
+        es = torch.empty((), dtype=dtype).element_size()
+        assert n * es <= nb
+        return _device_view(ptr, shape, dtype)
+
+    def close(self):
+        if self._h:
+            lib().kda_workspace_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _device_view(ptr: int, shape, dtype):
+    """Wrap device memory owned by the library as a torch tensor (no copy, no ownership)."""
+    import torch
+
+    class _Holder:
+        def __init__(self, p, nbytes):
+            self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1", "data": (p, False),
+                                             "version": 3, "strides": None}
+
+    n = 1
+    for x in shape:
+        n *= x
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    raw = torch.as_tensor(_Holder(ptr, nbytes), device="cuda")
+    return raw.view(dtype).view(tuple(shape))
+
+
+def kda_block_prefill(weights: KdaBlockWeights, hidden, T: int, h_state, conv_state, pad_fill: float,
+                      ws: Workspace, stream=None):
+    return _call("kda_block_prefill", ctypes.byref(weights), _p(hidden), T, _p(h_state), _p(conv_state),
+                 float(pad_fill), ws.handle, _stream(stream))

@@ -1,0 +1,148 @@
+// One KDA block prefill (Glm5NextKdaLayer `prefill` / `prefill_with_pad_fill`), stage by stage
+// into the workspace buffers of Glm5NextKdaWorkspace, with the weights of Glm5NextKdaWeights:
+//   q, k, v = h W^T           -> qkv_proj [T, 3*H*D] BF16 (three GEMMs writing the packed row)
+//   conv + SiLU + q|k L2      -> conv_out, q_f32/k_f32/v_f32 [T_pad, H*D] (tails = pad_fill)
+//   g_raw = f_b(f_a(h))       -> gate (kda_gate)
+//   beta = sigmoid(b_proj(h)) (FP32 logits)
+//   chunked core              -> core [T_pad, H, D], recurrent state carried in place
+//   out_gate = g_b(g_a(h));  o_norm_out = gated RMSNorm(core, out_gate);  final_out = o_proj
+// The workspace is allocated once (kda_workspace_create) for at most max_tokens tokens; the
+// prefill call itself allocates nothing.
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+
+namespace kda {
+namespace {
+// Writes the call's state pointer into the workspace's one-entry device pointer array (a kernel
+// argument, so no host synchronisation is involved).
+__global__ void store_ptr_kernel(float **slot, float *p) { *slot = p; }
+}  // namespace
+int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
+              int out_f32, cudaStream_t s);
+}
+
+struct kda_workspace {
+    kda_dims dims;
+    int hidden, rank;
+    size_t max_tokens, t_pad_max;
+    void *buf[KDA_BUF_COUNT];
+    size_t bytes[KDA_BUF_COUNT];
+    float **state_slot;  // device array holding the one state pointer of the call
+};
+
+extern "C" {
+
+int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_tokens, kda_workspace **out) {
+    if (!out) return KDA_ERR_INVALID_ARG;
+    *out = nullptr;
+    KDA_TRY(kda::check_dims(dims));
+    if (hidden <= 0 || rank <= 0 || max_tokens == 0) return KDA_ERR_INVALID_ARG;
+    if (hidden % 64 || rank % 64 || (dims->heads * dims->head_dim) % 64) return KDA_ERR_UNSUPPORTED;
+    kda_workspace *ws = new (std::nothrow) kda_workspace();
+    if (!ws) return KDA_ERR_CUDA;
+    ws->dims = *dims;
+    ws->hidden = hidden;
+    ws->rank = rank;
+    ws->max_tokens = max_tokens;
+    ws->t_pad_max = kda_t_pad(max_tokens, dims->chunk);
+    const size_t T = max_tokens, Tp = ws->t_pad_max;
+    const size_t qkv = static_cast<size_t>(dims->heads) * dims->head_dim, H = dims->heads;
+    const size_t sizes[KDA_BUF_COUNT] = {
+        T * 3 * qkv * 2,   // QKV_PROJ
+        T * 3 * qkv * 2,   // CONV_OUT
+        Tp * qkv * 4,      // Q_F32
+        Tp * qkv * 4,      // K_F32
+        Tp * qkv * 4,      // V_F32
+        Tp * qkv * 4,      // GATE
+        Tp * H * 4,        // BETA
+        Tp * qkv * 4,      // CORE
+        T * qkv * 2,       // G_RAW
+        T * qkv * 2,       // OUT_GATE
+        T * qkv * 2,       // O_NORM_OUT
+        T * hidden * 2,    // FINAL_OUT
+        T * rank * 2,      // F_A_OUT
+        T * rank * 2,      // G_A_OUT
+        kda_chunk_prefill_scratch_bytes(1, static_cast<int>(T), dims),  // PREFILL_SCRATCH
+    };
+    for (int i = 0; i < KDA_BUF_COUNT; ++i) {
+        ws->bytes[i] = sizes[i];
+        if (cudaMalloc(&ws->buf[i], sizes[i] ? sizes[i] : 16) != cudaSuccess) {
+            kda_workspace_destroy(ws);
+            return KDA_ERR_CUDA;
+        }
+    }
+    if (cudaMalloc(reinterpret_cast<void **>(&ws->state_slot), sizeof(float *)) != cudaSuccess) {
+        kda_workspace_destroy(ws);
+        return KDA_ERR_CUDA;
+    }
+    *out = ws;
+    return KDA_OK;
+}
+
+int kda_workspace_destroy(kda_workspace *ws) {
+    if (!ws) return KDA_OK;
+    for (int i = 0; i < KDA_BUF_COUNT; ++i)
+        if (ws->buf[i]) cudaFree(ws->buf[i]);
+    if (ws->state_slot) cudaFree(ws->state_slot);
+    delete ws;
+    return KDA_OK;
+}
+
+size_t kda_workspace_max_tokens(const kda_workspace *ws) { return ws ? ws->max_tokens : 0; }
+
+int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr, size_t *bytes) {
+    if (!ws || !ptr || which < 0 || which >= KDA_BUF_COUNT) return KDA_ERR_INVALID_ARG;
+    *ptr = ws->buf[which];
+    if (bytes) *bytes = ws->bytes[which];
+    return KDA_OK;
+}
+
+int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T, float *h_state,
+                      kda_bf16 *conv_state, float pad_fill, kda_workspace *ws, void *stream) {
+    if (!w || !hidden || !h_state || !conv_state || !ws || T < 0) return KDA_ERR_INVALID_ARG;
+    if (T == 0) return KDA_OK;
+    if (static_cast<size_t>(T) > ws->max_tokens) return KDA_ERR_CAPACITY;
+    if (w->hidden != ws->hidden || w->rank != ws->rank) return KDA_ERR_INVALID_ARG;
+    if (!w->q_proj || !w->k_proj || !w->v_proj || !w->conv || !w->f_a || !w->f_b || !w->dt_bias || !w->a_log ||
+        !w->b_proj || !w->g_a || !w->g_b || !w->o_norm || !w->o_proj)
+        return KDA_ERR_INVALID_ARG;
+    const kda_dims *d = &ws->dims;
+    auto s = static_cast<cudaStream_t>(stream);
+    const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
+    const int Tp = static_cast<int>(kda_t_pad(static_cast<size_t>(T), d->chunk));
+    auto B = [&](int i) { return ws->buf[i]; };
+    auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+
+    // q | k | v projections straight into the packed qkv_proj rows
+    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, T, qkv, Hd, 0, s));
+    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, T, qkv, Hd, 0, s));
+    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, T, qkv, Hd, 0, s));
+    KDA_TRY(kda_front_conv_silu_l2(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_Q_F32),
+                                   f32(KDA_BUF_K_F32), f32(KDA_BUF_V_F32), pad_fill, T, d, stream));
+    // forget gate: g_raw = f_b(f_a(h)) -> gate
+    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, T, R, Hd, 0, s));
+    KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, T, qkv, R, 0, s));
+    KDA_TRY(kda_gate(bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log, f32(KDA_BUF_GATE), T, d, stream));
+    // beta = sigmoid(b_proj(h)), FP32 logits
+    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, T, H, Hd, 1, s));
+    KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), T * H, stream));
+    // chunked core from the carried state
+    kda::store_ptr_kernel<<<1, 1, 0, s>>>(ws->state_slot, h_state);
+    KDA_TRY(kda::launch_status());
+    KDA_TRY(kda_chunk_prefill(f32(KDA_BUF_Q_F32), f32(KDA_BUF_K_F32), f32(KDA_BUF_V_F32), f32(KDA_BUF_GATE),
+                              f32(KDA_BUF_BETA), ws->state_slot, f32(KDA_BUF_CORE), 1, T, B(KDA_BUF_PREFILL_SCRATCH),
+                              ws->bytes[KDA_BUF_PREFILL_SCRATCH], d, stream));
+    // output gate, gated RMSNorm, output projection
+    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, T, R, Hd, 0, s));
+    KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0, s));
+    KDA_TRY(kda_back_gated_rmsnorm(f32(KDA_BUF_CORE), bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT), T, d,
+                                   stream));
+    KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), Hd, T, Hd, qkv, 0, s));
+    (void)Tp;
+    return KDA_OK;
+}
+
+}  // extern "C"

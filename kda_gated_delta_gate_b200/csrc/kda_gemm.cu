@@ -1,0 +1,280 @@
+// BF16 projection GEMM on tcgen05: C[M x N] = A[M x K] . W[N x K]^T (torch Linear layout,
+// Glm5NextKdaWeights: every projection is a [out, in] BF16 matrix), FP32 accumulation in
+// TMEM, BF16 or FP32 output with a row stride (so q/k/v projections can write straight into
+// the packed q|k|v rows of Glm5NextKdaWorkspace `qkv_proj`).
+//
+// Persistent, warp-specialised kernel (192 threads, one CTA per SM):
+//   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 W tiles, 128-byte swizzle, 4-stage
+//               ring of shared-memory buffers (full / empty mbarriers). No multicast.
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128, N = BN, K = 16) into
+//               one of two accumulators and commits to the stage's `empty` barrier.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator rows (TMEM lanes = rows), convert, store;
+//               then release the accumulator so the MMAs of the next tile overlap this one.
+// Every wait is bounded; a wait that gives up sets a shared abort flag so all roles leave
+// their loops, records KDA_ERR_TIMEOUT in the device status word, and TMEM is freed.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace kda {
+namespace {
+
+using namespace umma;
+
+constexpr int BM = 128, BK = 64, STAGES = 4, kGemmThreads = 192;
+constexpr long long kGemmWait = 4000000000LL;
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int A_STAGE = BM * BK * 2;
+    static constexpr int B_STAGE = BN * BK * 2;
+    static constexpr int STAGE = A_STAGE + B_STAGE;
+    static constexpr int OFF_BARS = STAGES * STAGE;
+    static constexpr int bytes = OFF_BARS + 256 + 1024;
+    static constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
+};
+
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *tm, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// Wait for a phase, giving up when another role aborted or the clock budget ran out.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort, int *status) {
+    const uint32_t addr = smem_u32(bar);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(addr, parity)) {
+        if (*abort) return false;
+        if (clock64() - t0 > kGemmWait) {
+            *abort = 1;
+            atomicExch(status, KDA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, void *__restrict__ Cout,
+            int ldc, int M, int N, int K, int out_f32, int vec, int *__restrict__ status) {
+    using G = GemmCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + G::OFF_BARS);
+    uint64_t *empty = full + STAGES;
+    uint64_t *accf = empty + STAGES;
+    uint64_t *acce = accf + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN, ntiles = tiles_m * tiles_n;
+    const int nk = K / BK;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 4); }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, G::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---- TMA producer
+            int it = 0;
+            for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+                const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!wait_or_abort(&empty[s], ph ^ 1, abort, status)) goto done;
+                    uint8_t *sa = sm + s * G::STAGE;
+                    mbar_expect_tx(&full[s], G::STAGE);
+                    tma_load_2d(sa, &tmA, kb * BK, m0, &full[s]);
+                    tma_load_2d(sa + G::A_STAGE, &tmW, kb * BK, n0, &full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ---- MMA issuer
+            constexpr uint32_t id = idesc_bf16(BM, BN, false, false);
+            int it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+                const int acc = tc & 1;
+                const uint32_t aph = (tc >> 1) & 1;
+                if (!wait_or_abort(&acce[acc], aph ^ 1, abort, status)) goto done;
+                tc_fence_after();
+                const uint32_t dcol = tmem + acc * BN;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!wait_or_abort(&full[s], ph, abort, status)) goto done;
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sm + s * G::STAGE), b0 = a0 + G::A_STAGE;
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks)
+                        mma_bf16(dcol, kmaj_desc(a0, BM, 0, ks), kmaj_desc(b0, BN, 0, ks), id,
+                                 (kb > 0 || ks > 0) ? 1u : 0u);
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&accf[acc]);
+            }
+        }
+    } else {  // ---- epilogue warps 2..5: TMEM lanes 32 (warp % 4) .. + 31
+        const int quad = warp & 3;
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+            const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+            const int acc = tc & 1;
+            const uint32_t aph = (tc >> 1) & 1;
+            if (!wait_or_abort(&accf[acc], aph, abort, status)) goto done;
+            tc_fence_after();
+            const int row = m0 + 32 * quad + lane;
+            const uint32_t src = tmem_lane_base(tmem, warp) + acc * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float x[16];
+                tmem_ld16(src + c, x);
+                tmem_ld_wait();
+                if (row < M && n0 + c < N && !(vec && n0 + c + 16 <= N)) {
+                    // ragged column tail or unaligned rows: element stores
+                    for (int u = 0; u < 16 && n0 + c + u < N; ++u) {
+                        if (out_f32) static_cast<float *>(Cout)[static_cast<size_t>(row) * ldc + n0 + c + u] = x[u];
+                        else static_cast<__nv_bfloat16 *>(Cout)[static_cast<size_t>(row) * ldc + n0 + c + u] = __float2bfloat16_rn(x[u]);
+                    }
+                } else if (row < M && n0 + c < N) {
+                    if (out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(Cout) + static_cast<size_t>(row) * ldc + n0 + c);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) dst[u] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+                    } else {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(x[2 * u], x[2 * u + 1]);
+                            w[u] = *reinterpret_cast<const uint32_t *>(&p);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(Cout) + static_cast<size_t>(row) * ldc + n0 + c);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[acc]);
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, G::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D BF16 tensor map over `rows` x `cols` (row stride ld elements), box 64 (K) x box_rows.
+int make_map(CUtensorMap *tm, const void *base, int rows, int cols, int ld, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return KDA_ERR_CUDA;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KDA_OK : KDA_ERR_INVALID_ARG;
+}
+
+int sm_count() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+template <int BN>
+int launch_gemm(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
+                int out_f32, cudaStream_t s) {
+    using G = GemmCfg<BN>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::bytes) !=
+            cudaSuccess)
+            return KDA_ERR_CUDA;
+        attr = true;
+    }
+    CUtensorMap ta, tw;
+    KDA_TRY(make_map(&ta, A, M, K, lda, BM));
+    KDA_TRY(make_map(&tw, W, N, K, ldw, BN));
+    int *status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
+    const long long ntiles = static_cast<long long>((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = static_cast<int>(std::min<long long>(ntiles, sm_count()));
+    // 16-element vector stores need 16-byte aligned rows
+    const int vec = aligned16(Cout) && (ldc % (out_f32 ? 4 : 8)) == 0;
+    gemm_kernel<BN><<<grid, kGemmThreads, G::bytes, s>>>(ta, tw, Cout, ldc, M, N, K, out_f32, vec, status);
+    return launch_status();
+}
+
+}  // namespace
+
+int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
+              int out_f32, cudaStream_t s) {
+    if (N > 128) return launch_gemm<256>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    if (N > 64) return launch_gemm<128>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    if (N > 32) return launch_gemm<64>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    return launch_gemm<32>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+}
+
+}  // namespace kda
+
+extern "C" int kda_gemm_bf16(const kda_bf16 *A, int lda, const kda_bf16 *W, int ldw, void *C, int ldc, int M, int N,
+                             int K, int out_f32, void *stream) {
+    if (!A || !W || !C || M < 0 || N < 0 || K < 0) return KDA_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return KDA_OK;
+    if (K == 0 || K % 64 != 0) return KDA_ERR_UNSUPPORTED;
+    if (lda < K || ldw < K || ldc < N) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(A) || !kda::aligned16(W) || (lda % 8) || (ldw % 8)) return KDA_ERR_MISALIGNED;
+    return kda::gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, static_cast<cudaStream_t>(stream));
+}
