@@ -157,6 +157,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefill-impl", default="tc", choices=["tc", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-block", action="store_true", help="skip the block-prefill leg")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -244,15 +245,18 @@ def main():
     # ---- end-to-end leg: the same C-ABI calls from pinned host buffers, copies timed
     e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch)
 
+    # ---- the full block (projections + front end + core + back end) and its dominant GEMM
+    blk = None if args.no_block else _block_leg(kda, torch, dev, s, stream, flush, tc_peak)
+
     result = None
     if rank == 0:
         tokens_per_s = world * B * T / (step_ms * 1e-3)
         cpu = None
         if not args.no_cpu_baseline:
-            tps, dt, cores = _oracle_baseline(1024)
+            tps, dt, cores = _oracle_baseline(T)
             cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                   "sample": f"FP64 oracle (gate, sigmoid, token recurrence, 32 heads) on the first 1024 tokens "
-                             f"of the workload; {dt:.1f} s wall"}
+                   "sample": f"FP64 oracle (gate, sigmoid, token recurrence, 32 heads) over the whole {T}-token "
+                             f"workload once; {dt:.2f} s wall on {cores} threads"}
         result = {
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -265,6 +269,7 @@ def main():
                          "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                                     "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
             "decode": dec,
+            "block_prefill": blk,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "gpu_launches": launches,
@@ -305,6 +310,49 @@ def _decode_leg(kda, torch, dev, s, stream, flush, hbm):
             "ms": ms, "tokens_per_s": N / (ms * 1e-3), "state_gbs": state_bytes / (ms * 1e-3) / 1e9,
             "all_gbs": all_bytes / (ms * 1e-3) / 1e9, "hbm_peak_gbs": hbm,
             "frac_hbm": all_bytes / (ms * 1e-3) / 1e9 / hbm}
+
+
+def _block_leg(kda, torch, dev, s, stream, flush, tc_peak):
+    """KDA block prefill, hidden 4096, H 32, D 128, rank 128, T 8192 (BF16 weights N(0, 0.02)),
+    and the q_proj-sized GEMM (8192 x 4096 x 4096) alone."""
+    import types
+    from synth import block_hidden, block_weights
+    hidden, Hh, Dd, rank, Tb = 4096, 32, 128, 128, 8192
+    Wt = block_weights(hidden, Hh, Dd, rank, seed=2, device=dev)
+    hid = block_hidden(Tb, hidden, seed=2, device=dev)
+    dw = types.SimpleNamespace(q_proj=Wt.w_q, k_proj=Wt.w_k, v_proj=Wt.w_v, conv=Wt.conv_w, f_a=Wt.f_a, f_b=Wt.f_b,
+                               dt_bias=Wt.dt_bias, a_log=Wt.a_log, b_proj=Wt.b_proj, g_a=Wt.g_a, g_b=Wt.g_b,
+                               o_norm=Wt.o_norm, o_proj=Wt.o_proj, hidden=hidden, rank=rank)
+    st = kda.block_weights_struct(dw)
+    ws = kda.Workspace(kda.dims(Hh, Dd), hidden, rank, max_tokens=Tb)
+    hs = torch.zeros((Hh, Dd, Dd), device=dev)
+    cs = torch.zeros((3 * Hh * Dd, 3), dtype=torch.bfloat16, device=dev)
+
+    def timed(fn, reps=6, warm=3):
+        ts = []
+        for i in range(warm + reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= warm:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    ms = timed(lambda: kda.kda_block_prefill(st, hid, Tb, hs, cs, 0.0, ws, s))
+    qkv, cd = Hh * Dd, 3 * Hh * Dd
+    flops = 2.0 * Tb * hidden * (3 * qkv + 2 * rank + Hh) + 2.0 * Tb * rank * 2 * qkv + 2.0 * Tb * qkv * hidden
+    C = torch.empty((Tb, hidden), dtype=torch.bfloat16, device=dev)
+    gms = timed(lambda: kda.kda_gemm_bf16(hid, Wt.w_q, C, Tb, hidden, hidden, stream=s))
+    gflop = 2.0 * Tb * hidden * hidden
+    ws.close()
+    return {"workload": "kda_block_prefill hidden 4096 H32 D128 rank 128 T8192 (9 GEMMs + conv + gate + core + o_norm)",
+            "ms": ms, "tokens_per_s": Tb / (ms * 1e-3), "proj_flops": flops,
+            "tflops_all": flops / (ms * 1e-3) / 1e12,
+            "gemm": {"shape": "8192x4096x4096 bf16->bf16", "ms": gms, "tflops": gflop / (gms * 1e-3) / 1e12,
+                     "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak}}
 
 
 def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):

@@ -542,20 +542,25 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
         sTab[13 * D + c] = __expf(gm[3] - gm[2]);
     }
     __syncthreads();
-    // ---- operands: A (mid-block reference), B (all references), and the state kernel's pack
+    // ---- operands of the L/M MMA: A (mid-block reference) and B (all references), in shared memory
     bool safe = true;
+    auto ld8 = [](const float *p, float (&x)[8]) {
+        const float4 a0 = *reinterpret_cast<const float4 *>(p), a1 = *reinterpret_cast<const float4 *>(p + 4);
+        x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w; x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
+    };
 #pragma unroll
     for (int u = 0; u < UPT; ++u) {
         const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
-        float ef[8], ei[8];
+        float gi[8], gm[8], ef[8], ei[8], x[8];
+        ld8(sG + i * GP + cb, gi);
+        ld8(sG + (16 * a + 7) * GP + cb, gm);
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            const float r = sG[i * GP + cb + w] - sG[(16 * a + 7) * GP + cb + w];
+            const float r = gi[w] - gm[w];
             safe = safe && fabsf(r) <= kRefBound;
             ef[w] = __expf(r);
             ei[w] = __expf(-r);
         }
-        float x[8];
 #pragma unroll
         for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
         st_pair(sA, I::A_BYTES / 2, kmaj_off(i, cb, 128), x);
@@ -567,51 +572,76 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
         for (int a2 = 0; a2 < 4; ++a2) {
             if (a2 < a) continue;
             const int off2 = 8 * a2 * (a2 + 1);
-            const int tix = a2 == a ? -1 : (a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13))));
+            if (a2 == a) {
 #pragma unroll
-            for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * (tix < 0 ? 1.f : sTab[tix * D + cb + w]);
+                for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w];
+            } else {
+                const int tix = a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13)));
+                float tb[8];
+                ld8(sTab + tix * D + cb, tb);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * tb[w];
+            }
             st_pair(sBt, I::B_BYTES / 2, kmaj_off(off2 + i, cb, I::NB), x);
         }
-        // the state kernel's operands: K o e^Gamma, Q o e^Gamma, K o e^{Gamma_C - Gamma}
-        uint4 hi, lo;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w] * sTab[a * D + cb + w];
-        split8(x, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w] * sTab[a * D + cb + w];
-        split8(x, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * sTab[(4 + a) * D + cb + w];
-        split8(x, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
     }
-    if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
     fence_async_smem();
     tc_fence_before();
     safe = __syncthreads_and(safe) != 0;
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // ---- D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127), issued now so that the
+    //      operand pack below is written while the tensor core works
+    if (safe && tid == 0) {
+        constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
+            const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
+            mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
+            mma_bf16(tmem, ah, bl, id, 1);
+            mma_bf16(tmem, al, bh, id, 1);
+        }
+        mma_commit(bar);
+    }
+    // ---- the state kernel's operands: K o e^Gamma, Q o e^Gamma, K o e^{Gamma_C - Gamma}
+    //      (written for unsafe chunks too; the CUDA-core body then rewrites the whole pack)
+#pragma unroll
+    for (int u = 0; u < UPT; ++u) {
+        const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
+        float gi[8], gm[8], em[8], ecm[8], x[8];
+        ld8(sG + i * GP + cb, gi);
+        ld8(sG + (16 * a + 7) * GP + cb, gm);
+        ld8(sTab + a * D + cb, em);
+        ld8(sTab + (4 + a) * D + cb, ecm);
+        float ef[8], ei[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            ef[w] = __expf(gi[w] - gm[w]) * em[w];    // e^{Gamma_i}
+            ei[w] = __expf(gm[w] - gi[w]) * ecm[w];   // e^{Gamma_C - Gamma_i}
+        }
+        uint4 hi, lo;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w];
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w];
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
+    }
+    if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
+    __syncthreads();  // every read of Gamma is done: L'/M are about to overwrite its space
     bool ok = true;
     if (safe) {
-        // ---- D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127)
-        if (tid == 0) {
-            constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
-            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
-#pragma unroll 1
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
-                const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
-                mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
-                mma_bf16(tmem, ah, bl, id, 1);
-                mma_bf16(tmem, al, bh, id, 1);
-            }
-            mma_commit(bar);
-        }
         ok = mbar_wait(bar, 0, kWaitCycles);
         tc_fence_after();
         // ---- read back: warp (quad, part); row r = 32 quad + lane (i = r % 64, block a = i / 16)
@@ -700,28 +730,74 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
             if (j <= i) sT[i * PC + j] *= sB[j];
         }
         __syncthreads();
-        for (int e = tid; e < C * C; e += NT) {
-            const int i = e / C, l = e % C;
-            float acc = 0.f;
-            for (int j = l; j <= i; ++j) acc = fmaf(sM[i * PC + j], sT[j * PC + l], acc);
-            sL[i * PC + l] = acc;
-        }
-        __syncthreads();
-        uint8_t *dst = pack + PK::OFF_A2;
-        for (int e = tid; e < 128 * 8; e += NT) {
-            const int row = e >> 3, c0 = 8 * (e & 7);
-            float x[8];
+        // ---- M' = M Tb on the tensor cores (M = 64, N = 64, K = 64): A = M (K-major),
+        //      B = Tb (MN-major: element (l, j) = Tb[j][l]); operands reuse the A region.
+        uint8_t *sA2a = sA, *sA2b = sA + 16384;
+        {
+            const int r = tid >> 3, c0 = 8 * (tid & 7);  // one 8-column chunk of one row per thread
+            float xm[8], xt[8];
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
-                const int col = c0 + w;
-                x[w] = row < 64 ? (col <= row ? sT[row * PC + col] : 0.f) : sL[(row - 64) * PC + col];
+                const int c = c0 + w;
+                xm[w] = c <= r ? sM[r * PC + c] : 0.f;
+                xt[w] = c <= r ? sT[r * PC + c] : 0.f;
             }
+            st_pair(sA2a, 8192, kmaj_off(r, c0, 64), xm);
+            st_pair(sA2b, 8192, mnmaj_off(c0, r, 64), xt);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t tM = tmem + I::NB;  // columns 160..223
+        if (tid == 0) {
+            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
+            const uint32_t a0 = smem_u32(sA2a), b0 = smem_u32(sA2b);
+#pragma unroll
+            for (int ks = 0; ks < C / 16; ++ks) {
+                const uint64_t ah = kmaj_desc(a0, 64, 0, ks), al = kmaj_desc(a0 + 8192, 64, 0, ks);
+                const uint64_t bh = mnmaj_desc(b0, 64, 0, ks), bl = mnmaj_desc(b0 + 8192, 64, 0, ks);
+                mma_bf16(tM, ah, bh, id, ks > 0 ? 1u : 0u);
+                mma_bf16(tM, ah, bl, id, 1);
+                mma_bf16(tM, al, bh, id, 1);
+            }
+            mma_commit(bar);
+        }
+        // rows 0..63 of [Tb; M']: Tb, written while M' is computed
+        uint8_t *dst = pack + PK::OFF_A2;
+        {
+            const int row = tid >> 3, c0 = 8 * (tid & 7);
+            float x[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = c0 + w <= row ? sT[row * PC + c0 + w] : 0.f;
             uint4 hi, lo;
             split8(x, hi, lo);
             const uint32_t off = kmaj_off(row, c0, 128);
             *reinterpret_cast<uint4 *>(dst + off) = hi;
             *reinterpret_cast<uint4 *>(dst + kTileBytes + off) = lo;
         }
+        // rows 64..127: M' from TMEM (M = 64 layout: row 16 q + lane in lanes < 16 of quad q)
+        const bool ok2 = mbar_wait(bar, 1, kWaitCycles);
+        tc_fence_after();
+        if (!ok2 && tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
+        {
+            const int quad = warp & 3, part = warp >> 2;
+            const int row = 16 * quad + lane;
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                float x[8];
+                tmem_ld8(tmem_lane_base(tM, warp) + 16 * part + 8 * h8, x);
+                tmem_ld_wait();
+                if (lane < 16 && ok2) {
+                    uint4 hi, lo;
+                    split8(x, hi, lo);
+                    const uint32_t off = kmaj_off(64 + row, 16 * part + 8 * h8, 128);
+                    *reinterpret_cast<uint4 *>(dst + off) = hi;
+                    *reinterpret_cast<uint4 *>(dst + kTileBytes + off) = lo;
+                }
+            }
+        }
+        tc_fence_before();
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
