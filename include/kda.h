@@ -166,7 +166,9 @@ KDA_API int kda_chunk_prefill_simt(const float *q, const float *k, const float *
  * pre-normalised q/k (Glm5NextKdaLayer `decode`: kda_recurrent takes q/k as given):
  *     S' = diag(exp(gate)) S;  u = beta (v - S'^T k);  S = S' + k u^T;  o = scale S^T q
  *   q, k, v, gate [N, H, D] F32;  beta [N, H] F32
- *   h_state   DEVICE array of N device pointers to [H, D, D] F32 states, updated in place
+ *   h_state   DEVICE array of N device pointers to [H, D, D] F32 states, updated in place;
+ *             each 16-byte aligned (a misaligned one is skipped and latches
+ *             KDA_ERR_MISALIGNED in kda_device_status)
  *   o         [N, H, D] F32
  */
 KDA_API int kda_recurrent_decode(const float *q, const float *k, const float *v, const float *gate,
@@ -188,7 +190,8 @@ KDA_API int kda_recurrent_decode(const float *q, const float *k, const float *v,
  *              updated in place
  *   conv_w     [3*H*D, 4] BF16 (tap 3 multiplies the current token)
  *   g_raw      [N, H*D] BF16;  dt_bias [H*D] F32;  a_log [H] F32;  b_logit [N, H] F32
- *   h_state    DEVICE array of N device pointers to [H, D, D] F32 states, in place
+ *   h_state    DEVICE array of N device pointers to [H, D, D] F32 states, in place, each
+ *              16-byte aligned (a misaligned one is skipped and latches KDA_ERR_MISALIGNED)
  *   out_gate   [N, H*D] BF16 (must not overlap g_raw: KDA_ERR_ALIAS)
  *   o_norm_w   [D] BF16
  *   o_norm_out [N, H*D] BF16 output
@@ -202,7 +205,7 @@ KDA_API int kda_decode_fused(const kda_bf16 *x, kda_bf16 *const *conv_state, con
                      float *core, int N, const kda_dims *dims, void *stream);
 
 /* kda_decode_k — K rows of ONE sequence (Glm5NextKdaLayer `decode_k`): the stateful
- * row of kda_decode_fused applied K times in order, the state carried in registers.
+ * row of kda_decode_fused applied K times in order, the state kept in shared memory.
  * Bit-identical to K serial kda_decode_fused calls with N = 1 (the same device code
  * runs each row). Arguments as kda_decode_fused with N replaced by K rows of one
  * sequence, and conv_state / h_state single device pointers. Snapshots:

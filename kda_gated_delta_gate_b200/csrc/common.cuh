@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kda.h"
 
 namespace kda {
@@ -52,6 +54,24 @@ inline int check_dims(const kda_dims *d) {
     if (d->heads < 1) return KDA_ERR_INVALID_ARG;
     if (d->head_dim != 64 && d->head_dim != 128) return KDA_ERR_UNSUPPORTED;
     if (d->chunk != kChunk) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+// Opt a kernel in to `bytes` of dynamic shared memory, once per device (the attribute belongs
+// to the device's context; `done` has one bit per device already set). With max_carveout the
+// kernel also asks for the largest shared-memory carve-out, so that several of its CTAs fit.
+template <typename K>
+int smem_opt_in(K kernel, int bytes, std::atomic<unsigned long long> &done, bool max_carveout = false) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev > 63) return KDA_ERR_CUDA;
+    const unsigned long long bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return KDA_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (max_carveout &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    done.fetch_or(bit, std::memory_order_acq_rel);
     return KDA_OK;
 }
 

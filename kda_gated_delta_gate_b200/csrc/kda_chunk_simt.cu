@@ -281,13 +281,8 @@ template <int D, int DVS>
 int launch_simt(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                 float *const *h_state, float *core, int B, int T, int H, float scale, cudaStream_t s) {
     using SM = SimtSmem<D, DVS>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(chunk_simt_kernel<D, DVS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(SM::bytes)) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    KDA_TRY(smem_opt_in(chunk_simt_kernel<D, DVS>, static_cast<int>(SM::bytes), attr_done));
     const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C));
     dim3 grid(D / DVS, H, B);
     chunk_simt_kernel<D, DVS><<<grid, kThreads, SM::bytes, s>>>(q, k, v, gate, beta, h_state, core, T, T_pad, H, scale);

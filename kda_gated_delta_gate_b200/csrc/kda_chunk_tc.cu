@@ -6,26 +6,24 @@
 // channel (Gamma_C its last row), A = e^Gamma:
 //   L[i][j] = beta_i sum_c k_ic k_jc e^{Gamma_ic - Gamma_jc}  (i > j);  T = (I + L)^-1
 //   M[i][j] =        sum_c q_ic k_jc e^{Gamma_ic - Gamma_jc}  (i >= j)
-//   Tb = T diag(beta);  M' = M Tb
-//   R = V - (K o A) S0;  U = Tb R;  O = scale ((Q o A) S0 + M' R)
+//   W = T diag(beta) (K o A);  U~ = T diag(beta) V              (the WY / UT form)
+//   U = U~ - W S0;  O = scale ((Q o A) S0 + M U)
 //   S = diag(A_C) S0 + (K o e^{Gamma_C - Gamma})^T U
-// which is the gated delta rule unrolled over the chunk (U = (I + L)^-1 diag(beta)(V - (K o A) S0)
-// and M U = M' R).
+// which is the gated delta rule unrolled over the chunk (U = (I + L)^-1 diag(beta)(V - (K o A) S0)).
 //
 // Two kernels:
-//  intra (one CTA per chunk-head, all in parallel, CUDA cores): L, M, T, Tb, M'. The decay
-//    factors come from a = e^g by running products inside 16-token blocks, and across blocks
-//    as products of per-block factors, so every factor is <= 1 and nothing overflows. It writes
-//    [Tb; M'] (128 x 64) as a BF16 hi/lo pair of 128-byte-swizzled K-major operand tiles.
-//  state (one CTA per (stream, head, value slice), chunks in order): builds [K o A; Q o A] and
-//    K o e^{Gamma_C - Gamma} from q, k, g, bulk-copies the [Tb; M'] tile, and runs three
-//    tcgen05 MMAs per chunk, each in split-BF16 precision (x = hi + lo; hi.hi + hi.lo + lo.hi):
-//      D1 = [K o A; Q o A] . S0        (M = 128, N = DVS, K = D)
-//      D2 = [Tb; M'] . R               (M = 128, N = DVS, K = 64)  with R = V - D1[0:64]
-//      D3 = (K o e^{Gamma_C-Gamma})^T . U  (M = D,  N = DVS, K = 64)  with U = D2[0:64]
-//    O = scale (D1[64:128] + D2[64:128]);  S = A_C o S0 + D3 (FP32 master copy in registers).
+//  intra (one CTA per chunk-head, all in parallel): L and M in one tcgen05 MMA, T on CUDA
+//    cores, then W | U~ in a second MMA. It writes a pack of state-independent operands,
+//    laid out as the state kernel's shared memory wants them (so one bulk copy moves each).
+//  state (one CTA per (stream, head, value slice), chunks in order): two dependent tcgen05
+//    MMA groups per chunk, each in split-BF16 precision (x = hi + lo; hi.hi + hi.lo + lo.hi):
+//      D1  = [W; Q o A] . S0                 (M = 128, N = DVS, K = D)
+//      U   = U~ - D1[0:64]                   (epilogue, into shared memory)
+//      D3  = (K o e^{Gamma_C - Gamma})^T . U (M = D, N = DVS, K = 64)
+//      D1 += [0; M] . U                      (so D1[64:128] = (Q o A) S0 + M U)
+//    O = scale D1[64:128];  S = A_C o S0 + D3 (FP32 master copy in registers).
 // Rows >= T of the last chunk are loaded as zeros (k = q = v = 0, g = 0, beta = 0): the pad
-// guard. They add nothing to L, M, R, U or the state, and their outputs are not written.
+// guard. They add nothing to L, M, W, U~ or the state, and their outputs are not written.
 #include <algorithm>
 
 #include "common.cuh"
@@ -39,23 +37,27 @@ using namespace umma;
 constexpr int C = kChunk;          // 64
 constexpr int kThreads = 256;
 constexpr int kTileBytes = 16384;  // one 128 x 64 BF16 K-major tile
-constexpr int kA2Bytes = 2 * kTileBytes;
 
 // Per (stream, head, chunk) the intra kernel writes one pack of state-independent operands,
-// each a BF16 hi tile followed by its lo tile, laid out exactly as the state kernel's shared
-// memory wants them (so a bulk copy moves each):
-//   A1 [K o A; Q o A]           128 x D, K-major          (A = e^Gamma)
-//   A2 [Tb; M']                 128 x 64, K-major
-//   A3 K o e^{Gamma_C - Gamma}  D (M) x 64 (K), MN-major
-//   AC e^{Gamma_C}              D FP32 (1 KB slot)
+// each BF16 operand as a hi tile followed by its lo tile, laid out exactly as the state
+// kernel's shared memory wants them (so a bulk copy moves each):
+//   A1 [W; Q o A]                 128 x D, K-major          (A = e^Gamma)
+//   AM M (lower, with diagonal)   64 x 64, K-major          (rows 64..127 of the [0; M] tile)
+//   A3 K o e^{Gamma_C - Gamma}    D (M) x 64 (K), MN-major
+//   UT U~ in FP32, D/32 groups of 32 value columns, [group][64 rows][UP] (UP = 36: a 16-byte
+//      skew per row, so the state kernel's per-row 16-byte reads are conflict-free)
+//   AC e^{Gamma_C}                D FP32 (1 KB slot)
 template <int D>
 struct Pack {
     static constexpr int A1 = 2 * 128 * D * 2;
-    static constexpr int A2 = kA2Bytes;
+    static constexpr int AM = 2 * C * C * 2;
     static constexpr int A3 = 2 * C * D * 2;
+    static constexpr int UP = 36;
+    static constexpr int UG_BYTES = C * UP * 4;
+    static constexpr int UT = (D / 32) * UG_BYTES;
     static constexpr int AC = 1024;
-    static constexpr int OFF_A1 = 0, OFF_A2 = A1, OFF_A3 = A1 + A2, OFF_AC = A1 + A2 + A3;
-    static constexpr int bytes = A1 + A2 + A3 + AC;
+    static constexpr int OFF_A1 = 0, OFF_AM = A1, OFF_A3 = OFF_AM + AM, OFF_UT = OFF_A3 + A3, OFF_AC = OFF_UT + UT;
+    static constexpr int bytes = OFF_AC + AC;
 };
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 1.9 GHz
 
@@ -78,13 +80,87 @@ __device__ __forceinline__ void st_pair(uint8_t *tile, int half_bytes, uint32_t 
 // ================================================================ phase 1: intra-chunk
 
 constexpr int kIntraThreads = 512;
+constexpr int kLPC = C + 1;  // row stride of the FP32 [C][C] tiles L and M (conflict-free column writes)
+constexpr int kTPC = C + 4;  // row stride of T (16-byte aligned rows for vector reads)
+
+// T = (I + L)^-1 for the strictly lower 64 x 64 L in sL (row stride kLPC; only i > j is read);
+// T's lower triangle and diagonal land in sT (row stride kTPC), together with zeros in the
+// blocks above the diagonal that the combination steps read. Blocked, each step parallel:
+//   16 x 16 diagonal blocks by substitution (one thread per column);
+//   32 x 32 halves:  T_21 = -T_22 (L_21 T_11)  from their 16 x 16 blocks;
+//   the whole:       T_21 = -T_22 (L_21 T_11)  from the two 32 x 32 halves.
+// The products run 4 columns per thread (16-byte reads of the right operand). All
+// kIntraThreads threads call it; sTmp holds 1024 floats (16-byte aligned).
+__device__ __forceinline__ void invert_unit_lower64(const float *__restrict__ sL, float *__restrict__ sT,
+                                                    float *__restrict__ sTmp) {
+    constexpr int PC = kLPC, PT = kTPC;
+    const int tid = threadIdx.x;
+    auto fma4 = [](float a, const float4 &b, float4 &acc) {
+        acc.x = fmaf(a, b.x, acc.x); acc.y = fmaf(a, b.y, acc.y); acc.z = fmaf(a, b.z, acc.z); acc.w = fmaf(a, b.w, acc.w);
+    };
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < 64) {
+        const int base = 16 * (tid >> 4), j = tid & 15;
+        float t[16];  // column j of the block's inverse; t[m] = 0 above the diagonal
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < i; ++m) acc = fmaf(sL[(base + i) * PC + base + m], t[m], acc);
+            t[i] = i == j ? 1.f : (i < j ? 0.f : -acc);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sT[(base + i) * PT + base + j] = t[i];
+    }
+    __syncthreads();
+    if (tid < 128) {  // X_h = L_{2h+1,2h} T_{2h,2h}, row i, columns 4c..4c+3
+        const int hh = tid >> 6, i = (tid >> 2) & 15, c4 = 4 * (tid & 3), b0 = 32 * hh;
+        float4 x = zero4;
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+            fma4(sL[(b0 + 16 + i) * PC + b0 + m], *reinterpret_cast<const float4 *>(sT + (b0 + m) * PT + b0 + c4), x);
+        *reinterpret_cast<float4 *>(sTmp + hh * 256 + i * 16 + c4) = x;
+        *reinterpret_cast<float4 *>(sT + (b0 + i) * PT + b0 + 16 + c4) = zero4;  // block above the diagonal
+    }
+    __syncthreads();
+    if (tid < 128) {  // T_{2h+1,2h} = -T_{2h+1,2h+1} X_h
+        const int hh = tid >> 6, i = (tid >> 2) & 15, c4 = 4 * (tid & 3), b0 = 32 * hh;
+        float4 x = zero4;
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+            fma4(sT[(b0 + 16 + i) * PT + b0 + 16 + m], *reinterpret_cast<const float4 *>(sTmp + hh * 256 + m * 16 + c4), x);
+        *reinterpret_cast<float4 *>(sT + (b0 + 16 + i) * PT + b0 + c4) = make_float4(-x.x, -x.y, -x.z, -x.w);
+    } else if (tid < 384) {  // the upper-right 32 x 32 block
+        const int e = tid - 128;
+        *reinterpret_cast<float4 *>(sT + (e >> 3) * PT + 32 + 4 * (e & 7)) = zero4;
+    }
+    __syncthreads();
+    if (tid < 256) {  // Y = L_LU T_UU, row i, columns 4c..4c+3
+        const int i = tid >> 3, c4 = 4 * (tid & 7);
+        float4 y = zero4;
+#pragma unroll
+        for (int m = 0; m < 32; ++m) fma4(sL[(32 + i) * PC + m], *reinterpret_cast<const float4 *>(sT + m * PT + c4), y);
+        *reinterpret_cast<float4 *>(sTmp + i * 32 + c4) = y;
+    }
+    __syncthreads();
+    if (tid < 256) {  // T_LU = -T_LL Y
+        const int i = tid >> 3, c4 = 4 * (tid & 7);
+        float4 y = zero4;
+#pragma unroll
+        for (int m = 0; m < 32; ++m)
+            fma4(sT[(32 + i) * PT + 32 + m], *reinterpret_cast<const float4 *>(sTmp + m * 32 + c4), y);
+        *reinterpret_cast<float4 *>(sT + (32 + i) * PT + c4) = make_float4(-y.x, -y.y, -y.z, -y.w);
+    }
+    __syncthreads();
+}
 
 template <int D>
 struct Intra {
     static constexpr int P = D + 8;   // fp32 row stride of [C][D] tiles (bank-spread, 16-B aligned)
-    static constexpr int PC = C + 1;  // row stride of [C][C] tiles
+    static constexpr int PC = kLPC;   // row stride of [C][C] tiles
     static constexpr int NZ = 64;     // rows of the block-local backward factors
-    static constexpr size_t floats = 3 * C * P + NZ * P + 3 * C * PC + 4 * D + C + 3 * 256;
+    static constexpr int PT = kTPC;   // row stride of T
+    static constexpr size_t floats = 3 * C * P + NZ * P + 2 * C * PC + C * PT + 4 * D + C + 1024;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -93,21 +169,22 @@ struct Intra {
 // pack. Used for the chunks whose in-block decay is too strong for the tensor-core path.
 template <int D>
 __device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, const float *__restrict__ q,
-                                                const float *__restrict__ gate, const float *__restrict__ beta,
+                                                const float *__restrict__ v, const float *__restrict__ gate,
+                                                const float *__restrict__ beta,
                                                 uint8_t *__restrict__ scratch, int T, int T_pad, int H, int b,
                                                 int h, int ch, float *smem) {
     using I = Intra<D>;
     constexpr int P = I::P, PC = I::PC, NT = kIntraThreads;
     float *sK = smem;              // k, then X: k_i prod_{s=16a}^{i} a_s  (a = block of i)
     float *sQ = sK + C * P;        // q, then Y: q_i prod_{s=16a}^{i} a_s
-    float *sA = sQ + C * P;        // a = e^g
+    float *sA = sQ + C * P;        // a = e^g, then v
     float *sZ = sA + C * P;        // Z: k_j prod_{s=j+1}^{16b+15} a_s
     float *sL = sZ + I::NZ * P;    // L' (unscaled), then M'
     float *sM = sL + C * PC;       // M
-    float *sT = sM + C * PC;       // T, then Tb
-    float *sF = sT + C * PC;       // [4][D]: whole-block decay products
+    float *sT = sM + C * PC;       // T, then Tb (row stride PT)
+    float *sF = sT + C * I::PT;    // [4][D]: whole-block decay products
     float *sB = sF + 4 * D;        // beta
-    float *sTmp = sB + C;          // [3][256]
+    float *sTmp = sB + C;          // [1024]
 
     const int tid = threadIdx.x;
     const int n = min(C, T - ch * C);
@@ -266,34 +343,39 @@ __device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, con
     }
     __syncthreads();
 
-    // ---- the state kernel's operands for this chunk: K o A = X P_a, Q o A = Y P_a and
-    //      K o e^{Gamma_C - Gamma} = Z S_a, with P_a / S_a the decay of all blocks before / after
-    //      block a; 16-byte chunks of 8 channels written straight into the pack.
+    // ---- the chunk's operands: K o A = X P_a (kept in sK for W), Q o A = Y P_a (pack), and
+    //      K o e^{Gamma_C - Gamma} = Z S_a (pack), with P_a / S_a the decay of all blocks before /
+    //      after block a; 16-byte chunks of 8 channels. v replaces a = e^g in sA (pad rows 0).
     using PK = Pack<D>;
     uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * (T_pad / C) + ch) * PK::bytes;
     for (int e = tid; e < C * (D / 8); e += NT) {
         const int i = e / (D / 8), cb = 8 * (e % (D / 8)), a = i >> 4;
-        float xk[8], xq[8], xb[8];
+        float xq[8], xb[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int c = cb + u;
             float pre = 1.f, suf = 1.f;
             for (int bb = 0; bb < a; ++bb) pre *= sF[bb * D + c];
             for (int bb = a + 1; bb < 4; ++bb) suf *= sF[bb * D + c];
-            xk[u] = sK[i * P + c] * pre;
+            sK[i * P + c] *= pre;
             xq[u] = sQ[i * P + c] * pre;
             xb[u] = sZ[i * P + c] * suf;
         }
         uint4 hi, lo;
-        split8(xk, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
         split8(xq, hi, lo);
         *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
         *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
         split8(xb, hi, lo);
         *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
         *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+        if (i < n) {
+            const float *src = v + (row0 + i) * rs + static_cast<size_t>(h) * D + cb;
+            v0 = *reinterpret_cast<const float4 *>(src);
+            v1 = *reinterpret_cast<const float4 *>(src + 4);
+        }
+        *reinterpret_cast<float4 *>(sA + i * P + cb) = v0;
+        *reinterpret_cast<float4 *>(sA + i * P + cb + 4) = v1;
     }
     if (tid < D) {
         float acv = 1.f;
@@ -301,118 +383,68 @@ __device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, con
         for (int bb = 0; bb < 4; ++bb) acv *= sF[bb * D + tid];
         reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = acv;
     }
-
-    // ---- L = diag(beta) L' (strict lower). T = (I + L)^-1: 16x16 diagonal blocks by
-    //      substitution, then off-diagonal blocks T_ab = -T_aa sum_{b<=c<a} L_ac T_cb.
+    // ---- M into the pack (64 x 64 K-major, zero above the diagonal); L = diag(beta) L'
+    {
+        const int r = tid >> 3, c0 = 8 * (tid & 7);
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = c0 + u <= r ? sM[r * PC + c0 + u] : 0.f;
+        uint4 hi, lo;
+        split8(x, hi, lo);
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + kmaj_off(r, c0, 64)) = hi;
+        *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + PK::AM / 2 + kmaj_off(r, c0, 64)) = lo;
+    }
     for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, j = e % C;
         if (i > j) sL[i * PC + j] *= sB[i];
     }
     __syncthreads();
-    if (tid < 64) {
-        const int a = tid / 16, j = tid % 16, base = 16 * a;
-        float t[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float val = (i == j) ? 1.f : 0.f;
-            if (i > j) {
-                float acc = 0.f;
-#pragma unroll
-                for (int m2 = 0; m2 < 16; ++m2)
-                    if (m2 >= j && m2 < i) acc = fmaf(sL[(base + i) * PC + base + m2], t[m2], acc);
-                val = -acc;
-            }
-            t[i] = val;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sT[(base + i) * PC + base + j] = t[i];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int dist = 1; dist < 4; ++dist) {
-        const int npairs = 4 - dist;
-        for (int e = tid; e < npairs * 256; e += NT) {
-            const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
-            const int bb = pr, aa = pr + dist;
-            float acc = 0.f;
-            for (int cb = bb; cb < aa; ++cb)
-#pragma unroll
-                for (int m2 = 0; m2 < 16; ++m2)
-                    acc = fmaf(sL[(16 * aa + i) * PC + 16 * cb + m2], sT[(16 * cb + m2) * PC + 16 * bb + j], acc);
-            sTmp[pr * 256 + i * 16 + j] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < npairs * 256; e += NT) {
-            const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
-            const int bb = pr, aa = pr + dist;
-            float acc = 0.f;
-#pragma unroll
-            for (int m2 = 0; m2 < 16; ++m2)
-                acc = fmaf(sT[(16 * aa + i) * PC + 16 * aa + m2], sTmp[pr * 256 + m2 * 16 + j], acc);
-            sT[(16 * aa + i) * PC + 16 * bb + j] = -acc;
-        }
-        __syncthreads();
-    }
-    // ---- Tb = T diag(beta) (lower incl. diagonal), then M' = M Tb (lower triangular) into sL
+    invert_unit_lower64(sL, sT, sTmp);
+    // ---- Tb = T diag(beta) in place (lower triangle and diagonal)
     for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, j = e % C;
-        if (j <= i) sT[i * PC + j] *= sB[j];
+        if (j <= i) sT[i * I::PT + j] *= sB[j];
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += NT) {
-        const int i = e / C, l = e % C;
-        float acc = 0.f;
-        for (int j = l; j <= i; ++j) acc = fmaf(sM[i * PC + j], sT[j * PC + l], acc);
-        sL[i * PC + l] = acc;  // zero when l > i (empty sum)
-    }
-    __syncthreads();
-    // ---- write [Tb; M'] as BF16 hi and lo K-major swizzled tiles (128 rows x 64 columns)
-    uint8_t *dst = pack + PK::OFF_A2;
-    for (int e = tid; e < 128 * 8; e += NT) {
-        const int row = e >> 3, c0 = 8 * (e & 7);
-        float x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int col = c0 + u;
-            x[u] = row < 64 ? (col <= row ? sT[row * PC + col] : 0.f) : sL[(row - 64) * PC + col];
+    // ---- W = Tb (K o A) -> A1 rows 0..63 (BF16 hi/lo);  U~ = Tb V -> UT (FP32)
+    for (int e = tid; e < 2 * C * (D / 8); e += NT) {
+        const int wv = e / (C * (D / 8)), r = e % (C * (D / 8));
+        const int i = r / (D / 8), cb = 8 * (r % (D / 8));
+        const float *src = wv == 0 ? sK : sA;
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j <= i; ++j) {
+            const float t = sT[i * I::PT + j];
+            const float4 s0 = *reinterpret_cast<const float4 *>(src + j * P + cb);
+            const float4 s1 = *reinterpret_cast<const float4 *>(src + j * P + cb + 4);
+            x[0] = fmaf(t, s0.x, x[0]); x[1] = fmaf(t, s0.y, x[1]); x[2] = fmaf(t, s0.z, x[2]); x[3] = fmaf(t, s0.w, x[3]);
+            x[4] = fmaf(t, s1.x, x[4]); x[5] = fmaf(t, s1.y, x[5]); x[6] = fmaf(t, s1.z, x[6]); x[7] = fmaf(t, s1.w, x[7]);
         }
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uint16_t h0, l0, h1, l1;
-            split_bf16(x[2 * u], h0, l0);
-            split_bf16(x[2 * u + 1], h1, l1);
-            hw[u] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-            lw[u] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+        if (wv == 0) {
+            uint4 hi, lo;
+            split8(x, hi, lo);
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
+        } else {
+            float *dst = reinterpret_cast<float *>(pack + PK::OFF_UT + (cb >> 5) * PK::UG_BYTES) + i * PK::UP + (cb & 31);
+            *reinterpret_cast<float4 *>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
         }
-        const uint32_t off = kmaj_off(row, c0, 128);
-        *reinterpret_cast<uint4 *>(dst + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4 *>(dst + kTileBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-}
-
-// All chunks through the CUDA-core body (grid = chunks x heads x streams).
-template <int D>
-__global__ void __launch_bounds__(kIntraThreads, 1)
-intra_simt_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
-                  const float *__restrict__ beta, uint8_t *__restrict__ scratch, int T, int T_pad, int H) {
-    extern __shared__ float smem[];
-    intra_simt_body<D>(k, q, gate, beta, scratch, T, T_pad, H, blockIdx.z, blockIdx.y, blockIdx.x, smem);
 }
 
 // Only the chunks the tensor-core kernel listed (count and packed (b, h, ch) entries in scratch).
 template <int D>
 __global__ void __launch_bounds__(kIntraThreads, 1)
-intra_fix_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
-                 const float *__restrict__ beta, uint8_t *__restrict__ scratch, const int *__restrict__ list,
-                 int T, int T_pad, int H) {
+intra_fix_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ v,
+                 const float *__restrict__ gate, const float *__restrict__ beta, uint8_t *__restrict__ scratch,
+                 const int *__restrict__ list, int T, int T_pad, int H) {
     extern __shared__ float smem[];
     const int count = list[0];
     const int nch = T_pad / C;
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
         const int id = list[1 + e];
         const int ch = id % nch, h = (id / nch) % H, b = id / (nch * H);
-        intra_simt_body<D>(k, q, gate, beta, scratch, T, T_pad, H, b, h, ch, smem);
+        intra_simt_body<D>(k, q, v, gate, beta, scratch, T, T_pad, H, b, h, ch, smem);
         __syncthreads();
     }
 }
@@ -433,50 +465,78 @@ constexpr float kRefBound = 80.0f;  // e^80 and e^-80 are comfortably inside BF1
 
 template <int D>
 struct IntraTC {
-    static constexpr int NB = 160;                  // B rows
-    static constexpr int A_BYTES = 2 * 128 * D * 2;  // A hi + lo (K-major, K = D)
-    static constexpr int B_BYTES = 2 * NB * D * 2;   // B hi + lo
-    static constexpr int GP = D + 4;                // Gamma row stride (floats)
-    static constexpr int PC = C + 1;
-    static constexpr int LMT = 3 * C * PC * 4;     // L, M, T (FP32); Gamma lives here first
-    static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_LMT = A_BYTES + B_BYTES, OFF_TAB = OFF_LMT + LMT;
-    static constexpr int TAB = 14 * D * 4;          // per-channel reference factors
-    static constexpr int OFF_MISC = OFF_TAB + TAB;  // beta[C], tmp[768], barrier, tmem slot, flags
-    static constexpr int MISC = (C + 768) * 4 + 256;
+    static constexpr int NB = 160;                   // B rows of the L/M MMA
+    static constexpr int A_BYTES = 2 * 128 * D * 2;  // L/M A operand (hi + lo, K = D); then the
+                                                     // W | U~ B operand [K o A | V] (N = 2D, K = 64)
+    static constexpr int B_BYTES = 2 * NB * D * 2;   // L/M B operand; then L, M, T and the Tb operand;
+                                                     // then the staged W | U~ results
+    static constexpr int PC = kLPC, PT = kTPC;
+    static constexpr int LMT = (2 * C * PC + C * PT) * 4;
+    static constexpr int OFF_TB = (LMT + 1023) / 1024 * 1024;  // Tb, 64 x 64 K-major, hi + lo
+    static constexpr int W_STAGE = 2 * C * D * 2;              // W rows 0..63 of A1, hi + lo panels
+    static constexpr int STAGE = W_STAGE + Pack<D>::UT;
+    static constexpr int R2a = B_BYTES > OFF_TB + 2 * 8192 ? B_BYTES : OFF_TB + 2 * 8192;
+    static constexpr int R2 = R2a > STAGE ? R2a : STAGE;
+    static constexpr int GP = D + 4;                 // Gamma row stride (floats)
+    static constexpr int G_BYTES = C * GP * 4;
+    static constexpr int TAB = 14 * D * 4;           // per-channel reference factors
+    static constexpr int MISC = (C + 1024) * 4 + 256;  // beta[C], tmp[1024], barrier, tmem slot
+    static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_G = OFF_B + R2, OFF_TAB = OFF_G + G_BYTES,
+                         OFF_MISC = OFF_TAB + TAB;
     static constexpr int bytes = OFF_MISC + MISC + 1024;
 };
 
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// One thread: bulk shared -> global copy (bytes a multiple of 16), in this thread's bulk group.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Persistent: gridDim.x CTAs walk the (stream, head, chunk) items; each item's q, k, g and
+// beta are fetched while the previous item finishes (g by cp.async into shared memory, q and k
+// into registers, v into L2), and its W | U~ results leave through shared memory in bulk copies.
 template <int D>
 __global__ void __launch_bounds__(kIntraThreads, 1)
-intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ gate,
-                const float *__restrict__ beta, uint8_t *__restrict__ scratch, int *__restrict__ list, int T,
-                int T_pad, int H, int *__restrict__ status) {
+intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ v,
+                const float *__restrict__ gate, const float *__restrict__ beta, uint8_t *__restrict__ scratch,
+                int *__restrict__ list, int B, int T, int T_pad, int H, int *__restrict__ status) {
     using I = IntraTC<D>;
     using PK = Pack<D>;
-    constexpr int NT = kIntraThreads, GP = I::GP, PC = I::PC;
-    constexpr int CG = D / 8;                 // 8-channel groups
-    constexpr int UPT = C * CG / NT;          // (token, group) units per thread: 2 (D=128) or 1
+    constexpr int NT = kIntraThreads, GP = I::GP, PC = I::PC, PT = I::PT;
+    constexpr int CG = D / 8;         // 8-channel groups
+    constexpr int UPT = C * CG / NT;  // (token, group) units per thread: 2 (D=128) or 1
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = sm + I::OFF_A, *sBt = sm + I::OFF_B;
-    float *sG = reinterpret_cast<float *>(sm + I::OFF_LMT);  // Gamma [C][GP], before L/M/T
-    float *sL = reinterpret_cast<float *>(sm + I::OFF_LMT);  // L' then M'
+    uint8_t *sA = sm + I::OFF_A, *sBt = sm + I::OFF_B, *sTb = sm + I::OFF_B + I::OFF_TB;
+    float *sL = reinterpret_cast<float *>(sm + I::OFF_B);  // after the L/M MMA: L, M, T
     float *sM = sL + C * PC;
     float *sT = sM + C * PC;
+    uint8_t *sW = sm + I::OFF_B;                            // after the W | U~ MMA: staged results
+    float *sUt = reinterpret_cast<float *>(sm + I::OFF_B + I::W_STAGE);
+    float *sG = reinterpret_cast<float *>(sm + I::OFF_G);
     float *sTab = reinterpret_cast<float *>(sm + I::OFF_TAB);
     float *sB = reinterpret_cast<float *>(sm + I::OFF_MISC);
     float *sTmp = sB + C;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + (C + 768) * 4);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + (C + 1024) * 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
     // reference tables, [entry][D]: 0..3 e^{Gamma_{m_a}}, 4..7 e^{Gamma_C - Gamma_{m_a}},
     // 8..13 e^{Gamma_{m_a} - Gamma_{m_b}} for (a,b) = (1,0),(2,0),(2,1),(3,0),(3,1),(3,2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ch = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int n = min(C, T - ch * C);
     const int nch = T_pad / C;
-    const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
+    const int total = B * H * nch;
     const size_t rs = static_cast<size_t>(H) * D;
-    uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * nch + ch) * PK::bytes;
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
@@ -486,319 +546,342 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
         mbar_init(bar, 1);
         fence_mbar_init();
     }
-    // ---- load: unit (token i, 8-channel group); g goes to shared memory for the scan
-    float kk[UPT][8], qq[UPT][8];
-#pragma unroll
-    for (int u = 0; u < UPT; ++u) {
-        const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
-        float4 k0 = make_float4(0.f, 0.f, 0.f, 0.f), k1 = k0, q0 = k0, q1 = k0, g0 = k0, g1 = k0;
-        if (i < n) {
-            const size_t off = (row0 + i) * rs + static_cast<size_t>(h) * D + cb;
-            k0 = *reinterpret_cast<const float4 *>(k + off);
-            k1 = *reinterpret_cast<const float4 *>(k + off + 4);
-            q0 = *reinterpret_cast<const float4 *>(q + off);
-            q1 = *reinterpret_cast<const float4 *>(q + off + 4);
-            g0 = *reinterpret_cast<const float4 *>(gate + off);
-            g1 = *reinterpret_cast<const float4 *>(gate + off + 4);
-        }
-        kk[u][0] = k0.x; kk[u][1] = k0.y; kk[u][2] = k0.z; kk[u][3] = k0.w;
-        kk[u][4] = k1.x; kk[u][5] = k1.y; kk[u][6] = k1.z; kk[u][7] = k1.w;
-        qq[u][0] = q0.x; qq[u][1] = q0.y; qq[u][2] = q0.z; qq[u][3] = q0.w;
-        qq[u][4] = q1.x; qq[u][5] = q1.y; qq[u][6] = q1.z; qq[u][7] = q1.w;
-        *reinterpret_cast<float4 *>(sG + i * GP + cb) = g0;
-        *reinterpret_cast<float4 *>(sG + i * GP + cb + 4) = g1;
-    }
-    if (tid < C) sB[tid] = tid < n ? beta[(row0 + tid) * H + h] : 0.f;
-    __syncthreads();
-    // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, quarter of 16 tokens)
-    {
-        constexpr int QT = NT / D;  // 4 (D=128) or 8 (D=64) token ranges
-        constexpr int TPQ = C / QT;
-        const int c = tid % D, qr = tid / D;
-        float acc = 0.f;
-        for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) { acc += sG[i * GP + c]; sG[i * GP + c] = acc; }
-        sTmp[qr * D + c] = acc;
-        __syncthreads();
-        float pre = 0.f;
-        for (int r = 0; r < qr; ++r) pre += sTmp[r * D + c];
-        if (qr > 0)
-            for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * GP + c] += pre;
-        __syncthreads();
-    }
-    if (tid < D) {
-        const int c = tid;
-        const float gm[4] = {sG[7 * GP + c], sG[23 * GP + c], sG[39 * GP + c], sG[55 * GP + c]};
-        const float gc = sG[63 * GP + c];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            sTab[a * D + c] = __expf(gm[a]);
-            sTab[(4 + a) * D + c] = __expf(gc - gm[a]);
-        }
-        sTab[8 * D + c] = __expf(gm[1] - gm[0]);
-        sTab[9 * D + c] = __expf(gm[2] - gm[0]);
-        sTab[10 * D + c] = __expf(gm[2] - gm[1]);
-        sTab[11 * D + c] = __expf(gm[3] - gm[0]);
-        sTab[12 * D + c] = __expf(gm[3] - gm[1]);
-        sTab[13 * D + c] = __expf(gm[3] - gm[2]);
-    }
-    __syncthreads();
-    // ---- operands of the L/M MMA: A (mid-block reference) and B (all references), in shared memory
-    bool safe = true;
     auto ld8 = [](const float *p, float (&x)[8]) {
         const float4 a0 = *reinterpret_cast<const float4 *>(p), a1 = *reinterpret_cast<const float4 *>(p + 4);
         x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w; x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
     };
+    // ---- fetch one item's inputs: k, q into registers; g into shared memory (cp.async, zeros
+    //      for rows past T); v only into L2; beta into a register of threads < C
+    float kk[UPT][8], qq[UPT][8], bnext = 0.f;
+    auto fetch = [&](int it) {
+        const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
+        const int n = min(C, T - ch * C);
+        const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
 #pragma unroll
-    for (int u = 0; u < UPT; ++u) {
-        const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
-        float gi[8], gm[8], ef[8], ei[8], x[8];
-        ld8(sG + i * GP + cb, gi);
-        ld8(sG + (16 * a + 7) * GP + cb, gm);
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const float r = gi[w] - gm[w];
-            safe = safe && fabsf(r) <= kRefBound;
-            ef[w] = __expf(r);
-            ei[w] = __expf(-r);
-        }
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
-        st_pair(sA, I::A_BYTES / 2, kmaj_off(i, cb, 128), x);
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w];
-        st_pair(sA, I::A_BYTES / 2, kmaj_off(64 + i, cb, 128), x);
-        // B rows for every reference block a2 >= a (column offsets 0, 16, 48, 96)
-#pragma unroll
-        for (int a2 = 0; a2 < 4; ++a2) {
-            if (a2 < a) continue;
-            const int off2 = 8 * a2 * (a2 + 1);
-            if (a2 == a) {
-#pragma unroll
-                for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w];
-            } else {
-                const int tix = a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13)));
-                float tb[8];
-                ld8(sTab + tix * D + cb, tb);
-#pragma unroll
-                for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * tb[w];
+        for (int u = 0; u < UPT; ++u) {
+            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
+            const bool in = i < n;
+            const size_t off = (row0 + (in ? i : 0)) * rs + static_cast<size_t>(h) * D + cb;
+            float4 k0 = make_float4(0.f, 0.f, 0.f, 0.f), k1 = k0, q0 = k0, q1 = k0;
+            if (in) {
+                k0 = *reinterpret_cast<const float4 *>(k + off);
+                k1 = *reinterpret_cast<const float4 *>(k + off + 4);
+                q0 = *reinterpret_cast<const float4 *>(q + off);
+                q1 = *reinterpret_cast<const float4 *>(q + off + 4);
+                if ((cb & 31) == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(v + off));
             }
-            st_pair(sBt, I::B_BYTES / 2, kmaj_off(off2 + i, cb, I::NB), x);
+            cp_async16(sG + i * GP + cb, gate + off, in ? 16u : 0u);
+            cp_async16(sG + i * GP + cb + 4, gate + off + 4, in ? 16u : 0u);
+            kk[u][0] = k0.x; kk[u][1] = k0.y; kk[u][2] = k0.z; kk[u][3] = k0.w;
+            kk[u][4] = k1.x; kk[u][5] = k1.y; kk[u][6] = k1.z; kk[u][7] = k1.w;
+            qq[u][0] = q0.x; qq[u][1] = q0.y; qq[u][2] = q0.z; qq[u][3] = q0.w;
+            qq[u][4] = q1.x; qq[u][5] = q1.y; qq[u][6] = q1.z; qq[u][7] = q1.w;
         }
-    }
-    fence_async_smem();
+        cp_async_commit();
+        if (tid < C) bnext = tid < n ? beta[(row0 + tid) * H + h] : 0.f;
+    };
+    if (blockIdx.x < total) fetch(blockIdx.x);
     tc_fence_before();
-    safe = __syncthreads_and(safe) != 0;
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // ---- D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127), issued now so that the
-    //      operand pack below is written while the tensor core works
-    if (safe && tid == 0) {
-        constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
-            const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
-            mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
-            mma_bf16(tmem, ah, bl, id, 1);
-            mma_bf16(tmem, al, bh, id, 1);
-        }
-        mma_commit(bar);
-    }
-    // ---- the state kernel's operands: K o e^Gamma, Q o e^Gamma, K o e^{Gamma_C - Gamma}
-    //      (written for unsafe chunks too; the CUDA-core body then rewrites the whole pack)
-#pragma unroll
-    for (int u = 0; u < UPT; ++u) {
-        const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
-        float gi[8], gm[8], em[8], ecm[8], x[8];
-        ld8(sG + i * GP + cb, gi);
-        ld8(sG + (16 * a + 7) * GP + cb, gm);
-        ld8(sTab + a * D + cb, em);
-        ld8(sTab + (4 + a) * D + cb, ecm);
-        float ef[8], ei[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            ef[w] = __expf(gi[w] - gm[w]) * em[w];    // e^{Gamma_i}
-            ei[w] = __expf(gm[w] - gi[w]) * ecm[w];   // e^{Gamma_C - Gamma_i}
-        }
-        uint4 hi, lo;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
-        split8(x, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(i, cb, 128)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(i, cb, 128)) = lo;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w];
-        split8(x, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w];
-        split8(x, hi, lo);
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
-        *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
-    }
-    if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
-    __syncthreads();  // every read of Gamma is done: L'/M are about to overwrite its space
-    bool ok = true;
-    if (safe) {
-        ok = mbar_wait(bar, 0, kWaitCycles);
-        tc_fence_after();
-        // ---- read back: warp (quad, part); row r = 32 quad + lane (i = r % 64, block a = i / 16)
-        //      needs columns [off_a, off_a + 16(a+1)); the quad's window is [0, 48) for rows in
-        //      blocks 0-1 and [48, 160) for blocks 2-3, split over the 4 warps of the quad.
-        {
-            const int quad = warp & 3, part = warp >> 2;
-            const int r = 32 * quad + lane, i = r & 63, a = i >> 4;
-            const int off_a = 8 * a * (a + 1);
-            const int w0 = (quad & 1) ? 48 : 0, wlen = (quad & 1) ? 112 : 48;
-            float *dstm = r < 64 ? sL : sM;
-            for (int c8 = part * 8; c8 < wlen; c8 += 32) {
-                float x[8];
-                tmem_ld8(tmem_lane_base(tmem, warp) + w0 + c8, x);
-                tmem_ld_wait();
-#pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    const int j = w0 + c8 + w - off_a;
-                    if (j >= 0 && j <= i) dstm[i * PC + j] = x[w];
-                }
-            }
-        }
-        tc_fence_before();
-    }
-    ok = __syncthreads_and(ok) != 0;
-    if (!safe || !ok) {
-        // the CUDA-core body redoes this chunk (it rewrites the whole pack)
-        if (tid == 0) {
-            if (!ok) atomicExch(status, KDA_ERR_TIMEOUT);
-            const int slot = atomicAdd(list, 1);
-            list[1 + slot] = (b * H + h) * nch + ch;
-        }
-    } else {
-        // ---- L = diag(beta) L' (strict lower). T = (I + L)^-1 as in the CUDA-core body.
-        for (int e = tid; e < C * C; e += NT) {
-            const int i = e / C, j = e % C;
-            if (i > j) sL[i * PC + j] *= sB[i];
-        }
-        __syncthreads();
-        if (tid < 64) {
-            const int a = tid / 16, j = tid % 16, base = 16 * a;
-            float t[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float val = (i == j) ? 1.f : 0.f;
-                if (i > j) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int m2 = 0; m2 < 16; ++m2)
-                        if (m2 >= j && m2 < i) acc = fmaf(sL[(base + i) * PC + base + m2], t[m2], acc);
-                    val = -acc;
-                }
-                t[i] = val;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sT[(base + i) * PC + base + j] = t[i];
-        }
-        __syncthreads();
+    bool dead = false;  // a tensor-core wait timed out: hand every remaining item to the CUDA-core body
+
 #pragma unroll 1
-        for (int dist = 1; dist < 4; ++dist) {
-            const int npairs = 4 - dist;
-            for (int e = tid; e < npairs * 256; e += NT) {
-                const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
-                const int bb = pr, aa = pr + dist;
-                float acc = 0.f;
-                for (int cb2 = bb; cb2 < aa; ++cb2)
-#pragma unroll
-                    for (int m2 = 0; m2 < 16; ++m2)
-                        acc = fmaf(sL[(16 * aa + i) * PC + 16 * cb2 + m2], sT[(16 * cb2 + m2) * PC + 16 * bb + j], acc);
-                sTmp[pr * 256 + i * 16 + j] = acc;
-            }
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const int ch = item % nch, h = (item / nch) % H, b = item / (nch * H);
+        const int n = min(C, T - ch * C);
+        const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
+        uint8_t *pack = scratch + static_cast<size_t>(item) * PK::bytes;
+        cp_async_wait_all();
+        if (tid < C) sB[tid] = bnext;
+        if (tid == 0) bulk_wait_read();  // the previous item's staged results have left
+        __syncthreads();
+        // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, range of tokens)
+        {
+            constexpr int QT = NT / D;  // 4 (D=128) or 8 (D=64) token ranges
+            constexpr int TPQ = C / QT;
+            const int c = tid % D, qr = tid / D;
+            float acc = 0.f;
+            for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) { acc += sG[i * GP + c]; sG[i * GP + c] = acc; }
+            sTmp[qr * D + c] = acc;
             __syncthreads();
-            for (int e = tid; e < npairs * 256; e += NT) {
-                const int pr = e / 256, i = (e % 256) / 16, j = e % 16;
-                const int bb = pr, aa = pr + dist;
-                float acc = 0.f;
-#pragma unroll
-                for (int m2 = 0; m2 < 16; ++m2)
-                    acc = fmaf(sT[(16 * aa + i) * PC + 16 * aa + m2], sTmp[pr * 256 + m2 * 16 + j], acc);
-                sT[(16 * aa + i) * PC + 16 * bb + j] = -acc;
-            }
+            float pre = 0.f;
+            for (int r = 0; r < qr; ++r) pre += sTmp[r * D + c];
+            if (qr > 0)
+                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * GP + c] += pre;
             __syncthreads();
         }
-        for (int e = tid; e < C * C; e += NT) {
-            const int i = e / C, j = e % C;
-            if (j <= i) sT[i * PC + j] *= sB[j];
+        if (tid < D) {
+            const int c = tid;
+            const float gm[4] = {sG[7 * GP + c], sG[23 * GP + c], sG[39 * GP + c], sG[55 * GP + c]};
+            const float gc = sG[63 * GP + c];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                sTab[a * D + c] = __expf(gm[a]);
+                sTab[(4 + a) * D + c] = __expf(gc - gm[a]);
+            }
+            sTab[8 * D + c] = __expf(gm[1] - gm[0]);
+            sTab[9 * D + c] = __expf(gm[2] - gm[0]);
+            sTab[10 * D + c] = __expf(gm[2] - gm[1]);
+            sTab[11 * D + c] = __expf(gm[3] - gm[0]);
+            sTab[12 * D + c] = __expf(gm[3] - gm[1]);
+            sTab[13 * D + c] = __expf(gm[3] - gm[2]);
         }
         __syncthreads();
-        // ---- M' = M Tb on the tensor cores (M = 64, N = 64, K = 64): A = M (K-major),
-        //      B = Tb (MN-major: element (l, j) = Tb[j][l]); operands reuse the A region.
-        uint8_t *sA2a = sA, *sA2b = sA + 16384;
-        {
-            const int r = tid >> 3, c0 = 8 * (tid & 7);  // one 8-column chunk of one row per thread
-            float xm[8], xt[8];
+        // ---- operands of the L/M MMA: A (mid-block reference) and B (all references)
+        bool safe = !dead;
+#pragma unroll
+        for (int u = 0; u < UPT; ++u) {
+            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
+            float gi[8], gm[8], ef[8], ei[8], x[8];
+            ld8(sG + i * GP + cb, gi);
+            ld8(sG + (16 * a + 7) * GP + cb, gm);
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
-                const int c = c0 + w;
-                xm[w] = c <= r ? sM[r * PC + c] : 0.f;
-                xt[w] = c <= r ? sT[r * PC + c] : 0.f;
+                const float r = gi[w] - gm[w];
+                safe = safe && fabsf(r) <= kRefBound;
+                ef[w] = __expf(r);
+                ei[w] = __expf(-r);
             }
-            st_pair(sA2a, 8192, kmaj_off(r, c0, 64), xm);
-            st_pair(sA2b, 8192, mnmaj_off(c0, r, 64), xt);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
+            st_pair(sA, I::A_BYTES / 2, kmaj_off(i, cb, 128), x);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w];
+            st_pair(sA, I::A_BYTES / 2, kmaj_off(64 + i, cb, 128), x);
+            // B rows for every reference block a2 >= a (column offsets 0, 16, 48, 96)
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2) {
+                if (a2 < a) continue;
+                const int off2 = 8 * a2 * (a2 + 1);
+                if (a2 == a) {
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w];
+                } else {
+                    const int tix = a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13)));
+                    float tb[8];
+                    ld8(sTab + tix * D + cb, tb);
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * tb[w];
+                }
+                st_pair(sBt, I::B_BYTES / 2, kmaj_off(off2 + i, cb, I::NB), x);
+            }
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        safe = __syncthreads_and(safe) != 0;
         tc_fence_after();
-        const uint32_t tM = tmem + I::NB;  // columns 160..223
-        if (tid == 0) {
-            constexpr uint32_t id = idesc_bf16(64, 64, false, true);
-            const uint32_t a0 = smem_u32(sA2a), b0 = smem_u32(sA2b);
+        // ---- D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127), issued now so that the
+        //      operand pack below is written while the tensor core works
+        if (safe && tid == 0) {
+            constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
 #pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 64, 0, ks), al = kmaj_desc(a0 + 8192, 64, 0, ks);
-                const uint64_t bh = mnmaj_desc(b0, 64, 0, ks), bl = mnmaj_desc(b0 + 8192, 64, 0, ks);
-                mma_bf16(tM, ah, bh, id, ks > 0 ? 1u : 0u);
-                mma_bf16(tM, ah, bl, id, 1);
-                mma_bf16(tM, al, bh, id, 1);
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
+                const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
+                mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
+                mma_bf16(tmem, ah, bl, id, 1);
+                mma_bf16(tmem, al, bh, id, 1);
             }
             mma_commit(bar);
         }
-        // rows 0..63 of [Tb; M']: Tb, written while M' is computed
-        uint8_t *dst = pack + PK::OFF_A2;
-        {
-            const int row = tid >> 3, c0 = 8 * (tid & 7);
-            float x[8];
+        // ---- state-independent operands of the pack: Q o e^Gamma (A1 rows 64..127),
+        //      K o e^{Gamma_C - Gamma} (A3), e^{Gamma_C}; K o e^Gamma stays in registers (kk)
+        //      (written for unsafe chunks too; the CUDA-core body then rewrites the whole pack)
 #pragma unroll
-            for (int w = 0; w < 8; ++w) x[w] = c0 + w <= row ? sT[row * PC + c0 + w] : 0.f;
+        for (int u = 0; u < UPT; ++u) {
+            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
+            float gi[8], gm[8], em[8], ecm[8], x[8];
+            ld8(sG + i * GP + cb, gi);
+            ld8(sG + (16 * a + 7) * GP + cb, gm);
+            ld8(sTab + a * D + cb, em);
+            ld8(sTab + (4 + a) * D + cb, ecm);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const float ef = __expf(gi[w] - gm[w]) * em[w];   // e^{Gamma_i}
+                const float ei = __expf(gm[w] - gi[w]) * ecm[w];  // e^{Gamma_C - Gamma_i}
+                x[w] = qq[u][w] * ef;
+                qq[u][w] = kk[u][w] * ei;
+                kk[u][w] *= ef;
+            }
             uint4 hi, lo;
             split8(x, hi, lo);
-            const uint32_t off = kmaj_off(row, c0, 128);
-            *reinterpret_cast<uint4 *>(dst + off) = hi;
-            *reinterpret_cast<uint4 *>(dst + kTileBytes + off) = lo;
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
+            split8(qq[u], hi, lo);
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
         }
-        // rows 64..127: M' from TMEM (M = 64 layout: row 16 q + lane in lanes < 16 of quad q)
-        const bool ok2 = mbar_wait(bar, 1, kWaitCycles);
-        tc_fence_after();
-        if (!ok2 && tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
-        {
-            const int quad = warp & 3, part = warp >> 2;
-            const int row = 16 * quad + lane;
+        if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
+        // v rows of this thread's units (L2 hits by now), for the W | U~ operand
+        float vv[UPT][8];
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                float x[8];
-                tmem_ld8(tmem_lane_base(tM, warp) + 16 * part + 8 * h8, x);
-                tmem_ld_wait();
-                if (lane < 16 && ok2) {
-                    uint4 hi, lo;
-                    split8(x, hi, lo);
-                    const uint32_t off = kmaj_off(64 + row, 16 * part + 8 * h8, 128);
-                    *reinterpret_cast<uint4 *>(dst + off) = hi;
-                    *reinterpret_cast<uint4 *>(dst + kTileBytes + off) = lo;
+        for (int u = 0; u < UPT; ++u) {
+            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
+            float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+            if (i < n) {
+                const float *src = v + (row0 + i) * rs + static_cast<size_t>(h) * D + cb;
+                v0 = *reinterpret_cast<const float4 *>(src);
+                v1 = *reinterpret_cast<const float4 *>(src + 4);
+            }
+            vv[u][0] = v0.x; vv[u][1] = v0.y; vv[u][2] = v0.z; vv[u][3] = v0.w;
+            vv[u][4] = v1.x; vv[u][5] = v1.y; vv[u][6] = v1.z; vv[u][7] = v1.w;
+        }
+        bool ok = true;
+        if (safe) {
+            ok = mbar_wait(bar, 0, kWaitCycles);
+            tc_fence_after();
+            // ---- read back: warp (quad, part); row r = 32 quad + lane (i = r % 64, block a = i / 16)
+            //      needs columns [off_a, off_a + 16(a+1)); the quad's window is [0, 48) for rows in
+            //      blocks 0-1 and [48, 160) for blocks 2-3, split over the 4 warps of the quad.
+            //      L = diag(beta) L' (strictly lower) and M (lower with diagonal) go to shared memory.
+            if (ok) {
+                const int quad = warp & 3, part = warp >> 2;
+                const int r = 32 * quad + lane, i = r & 63, a = i >> 4;
+                const int off_a = 8 * a * (a + 1);
+                const int w0 = (quad & 1) ? 48 : 0, wlen = (quad & 1) ? 112 : 48;
+                const bool is_l = r < 64;
+                float *dstm = is_l ? sL : sM;
+                const float bi = is_l ? sB[i] : 1.f;
+                for (int c8 = part * 8; c8 < wlen; c8 += 32) {
+                    float x[8];
+                    tmem_ld8(tmem_lane_base(tmem, warp) + w0 + c8, x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const int j = w0 + c8 + w - off_a;
+                        if (j >= 0 && (is_l ? j < i : j <= i)) dstm[i * PC + j] = x[w] * bi;
+                    }
                 }
             }
+            tc_fence_before();
         }
-        tc_fence_before();
+        ok = __syncthreads_and(ok) != 0;
+        const bool run = safe && ok;
+        if (run) {
+            // ---- the W | U~ B operand in the (now free) A region: [K o A | V], MN-major (n = channel
+            //      0..D-1 for K o A, D..2D-1 for V; k = token)
+#pragma unroll
+            for (int u = 0; u < UPT; ++u) {
+                const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
+                st_pair(sA, I::A_BYTES / 2, mnmaj_off(cb, i, C), kk[u]);
+                st_pair(sA, I::A_BYTES / 2, mnmaj_off(D + cb, i, C), vv[u]);
+            }
+            // ---- M into the pack (64 x 64 K-major, zero above the diagonal)
+            const int r = tid >> 3, c0 = 8 * (tid & 7);
+            float x[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = c0 + w <= r ? sM[r * PC + c0 + w] : 0.f;
+            uint4 hi, lo;
+            split8(x, hi, lo);
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + kmaj_off(r, c0, 64)) = hi;
+            *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + PK::AM / 2 + kmaj_off(r, c0, 64)) = lo;
+        }
+        // ---- the next item's inputs, fetched while this one finishes (Gamma's space and the
+        //      k, q registers are free; this item's beta is in sB)
+        if (item + static_cast<int>(gridDim.x) < total) fetch(item + gridDim.x);
+        bool done = false;
+        if (run) {
+            invert_unit_lower64(sL, sT, sTmp);
+            // ---- Tb = T diag(beta) as the A operand (64 x 64 K-major, zero above the diagonal)
+            {
+                const int r = tid >> 3, c0 = 8 * (tid & 7);
+                float tr[8], bc[8], x[8];
+                ld8(sT + r * PT + c0, tr);
+                ld8(sB + c0, bc);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) x[w] = c0 + w <= r ? tr[w] * bc[w] : 0.f;
+                st_pair(sTb, 8192, kmaj_off(r, c0, 64), x);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            // ---- [W | U~] = Tb . [K o A | V]  (M = 64, N = 2D, K = 64) into TMEM columns 0..2D-1
+            if (tid == 0) {
+                constexpr uint32_t id = idesc_bf16(64, 2 * D, false, true);
+                const uint32_t a0 = smem_u32(sTb), b0 = smem_u32(sA);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks) {
+                    const uint64_t ah = kmaj_desc(a0, 64, 0, ks), al = kmaj_desc(a0 + 8192, 64, 0, ks);
+                    const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + I::A_BYTES / 2, C, 0, ks);
+                    mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
+                    mma_bf16(tmem, ah, bl, id, 1);
+                    mma_bf16(tmem, al, bh, id, 1);
+                }
+                mma_commit(bar);
+            }
+            bool ok2 = mbar_wait(bar, 1, kWaitCycles);
+            tc_fence_after();
+            ok2 = __syncthreads_and(ok2) != 0;
+            if (ok2) {
+                // M = 64 layout: row 16 quad + lane in lanes < 16 of the quad; warp part p takes
+                // columns [p 2D/4, (p+1) 2D/4): W for columns < D, U~ above. Staged in shared
+                // memory (the B region: L, M, T and Tb are dead) in the pack's own layout.
+                const int quad = warp & 3, part = warp >> 2;
+                const int row = 16 * quad + lane;
+                constexpr int CW = 2 * D / 4;
+#pragma unroll
+                for (int c16 = 0; c16 < CW; c16 += 16) {
+                    const int col = part * CW + c16;
+                    float x[16];
+                    tmem_ld16(tmem_lane_base(tmem, warp) + col, x);
+                    tmem_ld_wait();
+                    if (lane < 16) {
+#pragma unroll
+                        for (int hlf = 0; hlf < 2; ++hlf) {
+                            const int cc = col + 8 * hlf;
+                            const float(&x8)[8] = *reinterpret_cast<const float(*)[8]>(x + 8 * hlf);
+                            if (cc < D) {
+                                // rows 0..63 of A1 panel p = cc / 64: the first 8 KB of the panel
+                                const uint32_t off = (cc >> 6) * 8192 + kmaj_off(row, cc & 63, 64);
+                                uint4 hi, lo;
+                                split8(x8, hi, lo);
+                                *reinterpret_cast<uint4 *>(sW + off) = hi;
+                                *reinterpret_cast<uint4 *>(sW + I::W_STAGE / 2 + off) = lo;
+                            } else {
+                                const int c = cc - D;
+                                float *dst = sUt + (c >> 5) * (PK::UG_BYTES / 4) + row * PK::UP + (c & 31);
+                                *reinterpret_cast<float4 *>(dst) = make_float4(x8[0], x8[1], x8[2], x8[3]);
+                                *reinterpret_cast<float4 *>(dst + 4) = make_float4(x8[4], x8[5], x8[6], x8[7]);
+                            }
+                        }
+                    }
+                }
+                fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    // W hi and lo: rows 0..63 of each 64-column panel of A1 (8 KB each); U~ whole
+#pragma unroll
+                    for (int p = 0; p < D / 64; ++p) {
+                        bulk_store(pack + PK::OFF_A1 + p * 16384, sW + p * 8192, 8192);
+                        bulk_store(pack + PK::OFF_A1 + PK::A1 / 2 + p * 16384, sW + I::W_STAGE / 2 + p * 8192, 8192);
+                    }
+                    bulk_store(pack + PK::OFF_UT, sUt, PK::UT);
+                    bulk_commit();
+                }
+                done = true;
+            } else {
+                if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
+                mbar_wait(bar, 1, kWaitCycles);  // bounded: the MMA may still be reading shared memory
+                dead = true;
+            }
+            tc_fence_before();
+        } else if (safe && !ok) {
+            if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
+            mbar_wait(bar, 0, kWaitCycles);
+            dead = true;
+        }
+        if (!done && tid == 0) {
+            // the CUDA-core body redoes this chunk (it rewrites the whole pack)
+            const int slot = atomicAdd(list, 1);
+            list[1 + slot] = item;
+        }
+        __syncthreads();
     }
+    if (tid == 0) bulk_wait_all();  // every staged result is in global memory
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
@@ -809,26 +892,25 @@ template <int D, int DVS>
 struct State {
     using PK = Pack<D>;
     static constexpr int NB = DVS < 64 ? 64 : DVS;  // MN-major B tiles span whole 64-wide atoms
+    static constexpr int A2 = 2 * kTileBytes;       // [0; M]: 128 x 64 K-major hi + lo, rows 0..63 zero
     static constexpr int B1 = 2 * NB * D * 2;       // S0 hi + lo, MN-major (N = value columns, K = D keys)
-    static constexpr int B2 = 2 * NB * C * 2;       // R, then U: hi + lo, MN-major (N = value columns, K = 64)
-    static constexpr int VP = DVS + 4;              // V row stride (floats): 16-byte skew per row
-    static constexpr int VS = C * VP * 4;           // V rows of the slice, FP32 (prefetched)
-    // A1, A2, A3 at the front, in the pack's own order and sizes
-    static constexpr int OFF_A1 = 0, OFF_A2 = PK::A1, OFF_A3 = PK::A1 + PK::A2, OFF_B1 = OFF_A3 + PK::A3,
-                         OFF_B2 = OFF_B1 + B1, OFF_V = OFF_B2 + B2, OFF_MISC = OFF_V + VS;
+    static constexpr int B2 = 2 * NB * C * 2;       // U hi + lo, MN-major (N = value columns, K = 64)
+    static constexpr int US = (DVS / 32) * PK::UG_BYTES;  // the slice's U~ groups
+    static constexpr int OFF_A1 = 0, OFF_A2 = PK::A1, OFF_A3 = OFF_A2 + A2, OFF_B1 = OFF_A3 + PK::A3,
+                         OFF_B2 = OFF_B1 + B1, OFF_U = OFF_B2 + B2, OFF_MISC = OFF_U + US;
     static constexpr int MISC = 1024;
     static constexpr int bytes = OFF_MISC + MISC + 1024;  // + alignment slack
-    static constexpr uint32_t TMEM_COLS = 3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512);
+    static constexpr uint32_t TMEM_COLS = 2 * DVS <= 32 ? 32 : (2 * DVS <= 64 ? 64 : 128);
 };
 
-// 16-byte asynchronous global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-                 "r"(src_bytes)
+// A bulk global -> shared copy completing on `bar`, whose expected bytes were already
+// announced by the caller (several copies on one barrier).
+__device__ __forceinline__ void bulk_copy_nx(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Issue a bulk global -> shared copy of `bytes` (multiple of 16) completing on `bar`.
 __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
@@ -841,8 +923,8 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
 
 template <int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
-state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state,
-             float *__restrict__ core, int T, int T_pad, int H, float scale, int *__restrict__ status) {
+state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core, int T,
+             int T_pad, int H, float scale, int *__restrict__ status) {
     using S = State<D, DVS>;
     using PK = Pack<D>;
     constexpr int HALF = DVS / 2;  // value columns per thread in the epilogues
@@ -850,8 +932,8 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = sm + S::OFF_A1, *sA2 = sm + S::OFF_A2, *sA3 = sm + S::OFF_A3, *sB1 = sm + S::OFF_B1,
             *sB2 = sm + S::OFF_B2;
-    float *sV = reinterpret_cast<float *>(sm + S::OFF_V);              // [C][VP]
-    // barriers: 0/4/5 bulk copies of A1/A2/A3, 1..3 the three MMA groups
+    const float *sU = reinterpret_cast<const float *>(sm + S::OFF_U);  // [DVS/32][64][UP]
+    // barriers: copies 0 A1, 1 M, 2 A3, 3 U~; MMA groups 4 (D1), 5 (D3 and D1 += [0; M] U)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 64);
 
@@ -862,23 +944,37 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
     const int nch = T_pad / C;
     const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
+    const size_t u_off = PK::OFF_UT + static_cast<size_t>(c0 / 32) * PK::UG_BYTES;
 
+    auto copy_m = [&](const uint8_t *pk) {  // M's hi and lo halves into rows 64..127 of A2
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bars[1])),
+                     "r"(static_cast<uint32_t>(PK::AM))
+                     : "memory");
+        bulk_copy_nx(sA2 + 8192, pk + PK::OFF_AM, PK::AM / 2, &bars[1]);
+        bulk_copy_nx(sA2 + kTileBytes + 8192, pk + PK::OFF_AM + PK::AM / 2, PK::AM / 2, &bars[1]);
+    };
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         bulk_copy(sA1, packs + PK::OFF_A1, PK::A1, &bars[0]);
-        bulk_copy(sA2, packs + PK::OFF_A2, PK::A2, &bars[4]);
-        bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[5]);
+        copy_m(packs);
+        bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[2]);
+        bulk_copy(const_cast<float *>(sU), packs + u_off, S::US, &bars[3]);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
         tmem_relinquish();
     }
+    // rows 0..63 of both halves of A2 stay zero: D1 += [0; M] U adds nothing to rows 0..63
+    for (int e = tid; e < 2 * 8192 / 16; e += kThreads) {
+        const int half = e / (8192 / 16), off = (e % (8192 / 16)) * 16;
+        *reinterpret_cast<uint4 *>(sA2 + half * kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tD1 = tmem, tD2 = tmem + DVS, tD3 = tmem + 2 * DVS;
+    const uint32_t tD1 = tmem, tD3 = tmem + DVS;
     bool ok = true;
 
     // Epilogue roles: for an M = 128 accumulator warp w reads TMEM lanes 32(w%4)..+31 (rows),
@@ -887,19 +983,6 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
     const int erow = 32 * quad + lane;
     const int ccol = colh * HALF;
     const int srow = (D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1);
-
-    // V rows of the slice for epilogue 1, prefetched one chunk ahead into shared memory: the
-    // thread that reads row erow, columns [ccol, ccol + HALF) is the thread that copies them.
-    auto prefetch_v = [&](int chn) {
-        if (quad < 2) {
-            const int nn = min(C, T - chn * C);
-            const size_t r0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(chn) * C;
-            const float *src = v + (r0 + (erow < nn ? erow : 0)) * rs + static_cast<size_t>(h) * D + c0 + ccol;
-#pragma unroll
-            for (int j = 0; j < HALF; j += 4) cp_async16(sV + erow * S::VP + ccol + j, src + j, erow < nn ? 16u : 0u);
-        }
-        cp_async_commit();
-    };
 
     // FP32 master state slice: key row srow, value columns [ccol, ccol + HALF)
     float st[HALF];
@@ -923,7 +1006,6 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
         }
     };
     write_state_operand();
-    prefetch_v(0);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -936,119 +1018,77 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
         const uint32_t par = ch & 1;
         const uint8_t *next = packs + static_cast<size_t>(ch + 1) * PK::bytes;
         const bool more = ch + 1 < nch;
-        // e^{Gamma_C} of this thread's key row, read early (used in epilogue 3)
+        // e^{Gamma_C} of this thread's key row, read early (used in epilogue 2)
         const float ac = srow >= 0 ? reinterpret_cast<const float *>(packs + static_cast<size_t>(ch) * PK::bytes +
                                                                     PK::OFF_AC)[srow]
                                    : 0.f;
-        // ---- MMA1: D1 = [K o A; Q o A] . S0   (A1 copied for this chunk)
+        // ---- MMA group 1: D1 = [W; Q o A] . S0
         if (tid == 0 && ok) ok = mbar_wait(&bars[0], par, kWaitCycles);
         if (tid == 0 && ok) {
             constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
             const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
-            int acc = 0;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + PK::A1 / 2, 128, 0, ks);
                 const uint64_t bh = mnmaj_desc(b0, D, 0, ks), bl = mnmaj_desc(b0 + S::B1 / 2, D, 0, ks);
-                mma_bf16(tD1, ah, bh, id, acc); acc = 1;
+                mma_bf16(tD1, ah, bh, id, ks > 0 ? 1u : 0u);
                 mma_bf16(tD1, ah, bl, id, 1);
                 mma_bf16(tD1, al, bh, id, 1);
             }
-            mma_commit(&bars[1]);
+            mma_commit(&bars[4]);
         }
-        // e1: the Q half of D1 kept for the output (rows 64..127, quads 2 and 3)
-        float e1[HALF];
-        cp_async_wait_all();  // this thread's V rows of this chunk are in sV
-        ok = ok && mbar_wait(&bars[1], par, kWaitCycles);
+        ok = ok && mbar_wait(&bars[4], par, kWaitCycles);
+        ok = ok && mbar_wait(&bars[3], par, kWaitCycles);  // U~ of this chunk
         tc_fence_after();
         if (tid == 0 && ok && more) bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);  // A1 is free again
-        // ---- epilogue 1: R = V - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
+        // ---- epilogue 1: U = U~ - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
+        if (quad < 2) {
 #pragma unroll
-        for (int j = 0; j < HALF; j += 8) {
-            float x[8];
-            tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
-            tmem_ld_wait();
-            if (quad < 2) {
-                const float4 v0 = *reinterpret_cast<const float4 *>(sV + erow * S::VP + ccol + j);
-                const float4 v1 = *reinterpret_cast<const float4 *>(sV + erow * S::VP + ccol + j + 4);
-                const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-                for (int u = 0; u < 8; ++u) x[u] = vv[u] - x[u];
-                st_pair(sB2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
-            } else {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) e1[j + u] = x[u];
-            }
-        }
-        if (more) prefetch_v(ch + 1);  // this thread is done with its V rows of this chunk
-        fence_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;
-        tc_fence_after();
-        // ---- MMA2: D2 = [Tb; M'] . R
-        if (tid == 0 && ok) ok = mbar_wait(&bars[4], par, kWaitCycles);
-        if (tid == 0 && ok) {
-            constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
-            const uint32_t a0 = smem_u32(sA2), b0 = smem_u32(sB2);
-            int acc = 0;
-#pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + kTileBytes, 128, 0, ks);
-                const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
-                mma_bf16(tD2, ah, bh, id, acc); acc = 1;
-                mma_bf16(tD2, ah, bl, id, 1);
-                mma_bf16(tD2, al, bh, id, 1);
-            }
-            mma_commit(&bars[2]);
-        }
-        ok = ok && mbar_wait(&bars[2], par, kWaitCycles);
-        tc_fence_after();
-        if (tid == 0 && ok && more) bulk_copy(sA2, next + PK::OFF_A2, PK::A2, &bars[4]);  // A2 is free again
-        // ---- epilogue 2: U = D2[0:64] -> B2 (R is consumed); O = scale (D1[64:] + D2[64:])
-#pragma unroll
-        for (int j = 0; j < HALF; j += 8) {
-            float x[8];
-            tmem_ld8(tmem_lane_base(tD2, warp) + ccol + j, x);
-            tmem_ld_wait();
-            if (quad < 2) {
-                st_pair(sB2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
-            } else {
-                const int i = erow - 64;
-                if (i < n) {
-                    float *dst = core + (row0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
-                    float4 o0 = make_float4(scale * (e1[j] + x[0]), scale * (e1[j + 1] + x[1]),
-                                            scale * (e1[j + 2] + x[2]), scale * (e1[j + 3] + x[3]));
-                    float4 o1 = make_float4(scale * (e1[j + 4] + x[4]), scale * (e1[j + 5] + x[5]),
-                                            scale * (e1[j + 6] + x[6]), scale * (e1[j + 7] + x[7]));
-                    *reinterpret_cast<float4 *>(dst) = o0;
-                    *reinterpret_cast<float4 *>(dst + 4) = o1;
-                }
+            for (int j = 0; j < HALF; j += 8) {
+                float x[8];
+                tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
+                tmem_ld_wait();
+                const int c = ccol + j;  // column within the slice
+                const float *ur = sU + (c >> 5) * (PK::UG_BYTES / 4) + erow * PK::UP + (c & 31);
+                const float4 u0 = *reinterpret_cast<const float4 *>(ur);
+                const float4 u1 = *reinterpret_cast<const float4 *>(ur + 4);
+                x[0] = u0.x - x[0]; x[1] = u0.y - x[1]; x[2] = u0.z - x[2]; x[3] = u0.w - x[3];
+                x[4] = u1.x - x[4]; x[5] = u1.y - x[5]; x[6] = u1.z - x[6]; x[7] = u1.w - x[7];
+                st_pair(sB2, S::B2 / 2, mnmaj_off(c, erow, C), x);
             }
         }
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
         tc_fence_after();
-        // ---- MMA3: D3 = (K o e^{Gamma_C - Gamma})^T . U
-        if (tid == 0 && ok) ok = mbar_wait(&bars[5], par, kWaitCycles);
+        if (tid == 0 && ok && more) bulk_copy(const_cast<float *>(sU), next + u_off, S::US, &bars[3]);
+        // ---- MMA group 2: D3 = (K o e^{Gamma_C - Gamma})^T . U;  D1 += [0; M] . U
+        if (tid == 0 && ok) ok = mbar_wait(&bars[1], par, kWaitCycles) && mbar_wait(&bars[2], par, kWaitCycles);
         if (tid == 0 && ok) {
-            constexpr uint32_t id = idesc_bf16(D, DVS, true, true);
-            const uint32_t a0 = smem_u32(sA3), b0 = smem_u32(sB2);
-            int acc = 0;
+            constexpr uint32_t id3 = idesc_bf16(D, DVS, true, true);
+            constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
+            const uint32_t a3 = smem_u32(sA3), a2 = smem_u32(sA2), b0 = smem_u32(sB2);
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t ah = mnmaj_desc(a0, C, 0, ks), al = mnmaj_desc(a0 + PK::A3 / 2, C, 0, ks);
                 const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
-                mma_bf16(tD3, ah, bh, id, acc); acc = 1;
-                mma_bf16(tD3, ah, bl, id, 1);
-                mma_bf16(tD3, al, bh, id, 1);
+                const uint64_t ah = mnmaj_desc(a3, C, 0, ks), al = mnmaj_desc(a3 + PK::A3 / 2, C, 0, ks);
+                mma_bf16(tD3, ah, bh, id3, ks > 0 ? 1u : 0u);
+                mma_bf16(tD3, ah, bl, id3, 1);
+                mma_bf16(tD3, al, bh, id3, 1);
+                const uint64_t mh = kmaj_desc(a2, 128, 0, ks), ml = kmaj_desc(a2 + kTileBytes, 128, 0, ks);
+                mma_bf16(tD1, mh, bh, idm, 1);
+                mma_bf16(tD1, mh, bl, idm, 1);
+                mma_bf16(tD1, ml, bh, idm, 1);
             }
-            mma_commit(&bars[3]);
+            mma_commit(&bars[5]);
         }
-        ok = ok && mbar_wait(&bars[3], par, kWaitCycles);
+        ok = ok && mbar_wait(&bars[5], par, kWaitCycles);
         tc_fence_after();
-        if (tid == 0 && ok && more) bulk_copy(sA3, next + PK::OFF_A3, PK::A3, &bars[5]);  // A3 is free again
-        // ---- epilogue 3: S = A_C o S0 + D3 (FP32 in registers), S into B1
+        if (tid == 0 && ok && more) {  // M and A3 are free again
+            copy_m(next);
+            bulk_copy(sA3, next + PK::OFF_A3, PK::A3, &bars[2]);
+        }
+        // ---- epilogue 2: S = A_C o S0 + D3 (FP32 in registers), S into B1;  O = scale D1[64:128]
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
             float x[8];
@@ -1060,6 +1100,22 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
             }
         }
         write_state_operand();
+        if (quad >= 2) {
+            const int i = erow - 64;
+#pragma unroll
+            for (int j = 0; j < HALF; j += 8) {
+                float x[8];
+                tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
+                tmem_ld_wait();
+                if (i < n) {
+                    float *dst = core + (row0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
+                    *reinterpret_cast<float4 *>(dst) =
+                        make_float4(scale * x[0], scale * x[1], scale * x[2], scale * x[3]);
+                    *reinterpret_cast<float4 *>(dst + 4) =
+                        make_float4(scale * x[4], scale * x[5], scale * x[6], scale * x[7]);
+                }
+            }
+        }
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
@@ -1079,13 +1135,6 @@ state_kernel(const float *__restrict__ v, const uint8_t *__restrict__ scratch, f
     if (warp == 0) tmem_dealloc(tmem, S::TMEM_COLS);
 }
 
-template <typename K>
-int set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-               ? KDA_OK
-               : KDA_ERR_CUDA;
-}
-
 // Scratch layout: the operand packs, then a 256-byte slot with the count of chunks the
 // tensor-core intra kernel handed to the CUDA-core body, then their (b, h, chunk) ids.
 template <int D>
@@ -1098,30 +1147,29 @@ int launch_tc(const float *q, const float *k, const float *v, const float *gate,
     const int nch = T_pad / C;
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
-    static bool attrs = false;
-    if (!attrs) {
-        KDA_TRY(set_smem(intra_tc_kernel<D>, IntraTC<D>::bytes));
-        KDA_TRY(set_smem(intra_fix_kernel<D>, static_cast<int>(Intra<D>::bytes)));
-        KDA_TRY(set_smem(state_kernel<D, DVS>, State<D, DVS>::bytes));
-        attrs = true;
-    }
+    static std::atomic<unsigned long long> attr_intra{0}, attr_fix{0}, attr_state{0};
+    KDA_TRY(smem_opt_in(intra_tc_kernel<D>, IntraTC<D>::bytes, attr_intra));
+    KDA_TRY(smem_opt_in(intra_fix_kernel<D>, static_cast<int>(Intra<D>::bytes), attr_fix));
+    KDA_TRY(smem_opt_in(state_kernel<D, DVS>, State<D, DVS>::bytes, attr_state));
     uint8_t *sc = static_cast<uint8_t *>(scratch);
     int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(B, H, nch));
     if (cudaMemsetAsync(list, 0, sizeof(int), s) != cudaSuccess) return KDA_ERR_CUDA;
-    intra_tc_kernel<D><<<dim3(nch, H, B), kIntraThreads, IntraTC<D>::bytes, s>>>(k, q, gate, beta, sc, list, T, T_pad,
-                                                                                 H, status);
-    KDA_TRY(launch_status());
     int sms = 148;
     {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    const int fix_grid = static_cast<int>(std::min<long long>(static_cast<long long>(B) * H * nch, sms));
-    intra_fix_kernel<D><<<fix_grid, kIntraThreads, Intra<D>::bytes, s>>>(k, q, gate, beta, sc, list, T, T_pad, H);
+    const long long items = static_cast<long long>(B) * H * nch;
+    const int intra_grid = static_cast<int>(std::min<long long>(items, sms));
+    intra_tc_kernel<D><<<intra_grid, kIntraThreads, IntraTC<D>::bytes, s>>>(k, q, v, gate, beta, sc, list, B, T, T_pad,
+                                                                            H, status);
+    KDA_TRY(launch_status());
+    const int fix_grid = intra_grid;
+    intra_fix_kernel<D><<<fix_grid, kIntraThreads, Intra<D>::bytes, s>>>(k, q, v, gate, beta, sc, list, T, T_pad, H);
     KDA_TRY(launch_status());
     state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(
-        v, sc, h_state, core, T, T_pad, H, scale, status);
+        sc, h_state, core, T, T_pad, H, scale, status);
     return launch_status();
 }
 

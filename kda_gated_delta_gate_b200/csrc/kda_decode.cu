@@ -11,34 +11,46 @@
 // intrinsics (__fmul_rn / __fadd_rn / __fmaf_rn), which the compiler may not re-associate
 // or contract differently — this is what makes decode_k bit-identical to K decodes.
 //
-// State thread layout (256 threads): D/4 threads per row, each holding a float4 column
-// group; RG = 256/(D/4) row groups; thread (rg, c4) owns rows rg, rg+RG, ... (RPT rows).
-// A warp therefore loads whole 512-byte (D=128) rows: coalesced 16-byte accesses.
+// The state comes in through shared memory: one bulk copy brings the head's 64 KB in (issued
+// first, so the row's small inputs load under it). The updated state goes straight from
+// registers to global memory (coalesced 128-byte rows), so a CTA's slot frees as soon as its
+// stores are issued; only decode_k keeps the state in shared memory between its rows. Low
+// register use lets three CTAs share an SM, so three heads' state streams overlap on every
+// SM. Thread layout (256 threads): thread t owns value column j = t % D and the row group
+// t / D (RG = 256 / D groups of D / RG consecutive key rows); a warp reads 32 consecutive
+// floats of one row, so shared-memory accesses are conflict-free.
 #include "common.cuh"
+#include "umma.cuh"
 
 namespace kda {
 namespace {
 
+using umma::fence_mbar_init;
+using umma::mbar_init;
+using umma::smem_u32;
+
 constexpr int kThreads = 256;
+constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 1.9 GHz
 
 template <int D>
 struct Lay {
-    static constexpr int TPR = D / 4;
-    static constexpr int RG = kThreads / TPR;
-    static constexpr int RPT = D / RG;
-    static constexpr int NW = D / 32;  // warps spanned by threads 0..D-1
+    static constexpr int RG = kThreads / D;  // row groups: 2 (D = 128) or 4 (D = 64)
+    static constexpr int RPG = D / RG;       // rows per group
+    static constexpr int NW = D / 32;        // warps spanned by threads 0..D-1
 };
 
+template <int D>
 struct __align__(16) Smem {
-    float q[128], k[128], v[128], a[128], u[128], o[128];
-    float red[2][16][128];
+    float S[D * D];  // the head's state, row i = key channel i
+    float q[D], k[D], v[D], a[D], u[D], o[D];
+    float red[2][Lay<D>::RG][D];
     float wsum[2][8];
-    float bcast[4];
+    uint64_t bar;
 };
 
 // Sum of (x, y) over threads 0..D-1 in a fixed tree (same order on every call).
 template <int D>
-__device__ __forceinline__ float2 sum2_first_d(float x, float y, Smem &sm) {
+__device__ __forceinline__ float2 sum2_first_d(float x, float y, Smem<D> &sm) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -54,64 +66,84 @@ __device__ __forceinline__ float2 sum2_first_d(float x, float y, Smem &sm) {
     return make_float2(sx, sy);
 }
 
-template <int D>
-__device__ __forceinline__ void load_state(float4 (&st)[Lay<D>::RPT], const float *S) {
-    const int rg = threadIdx.x / Lay<D>::TPR, c4 = threadIdx.x % Lay<D>::TPR;
-#pragma unroll
-    for (int r = 0; r < Lay<D>::RPT; ++r)
-        st[r] = __ldcs(reinterpret_cast<const float4 *>(S + (rg + Lay<D>::RG * r) * D) + c4);
+// L2 policy for data touched once (the state streams).
+__device__ __forceinline__ uint64_t evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
 }
 
+// One thread: bulk-copy the state (D*D floats) from global memory into sm.S, completing on sm.bar.
 template <int D>
-__device__ __forceinline__ void store_state(const float4 (&st)[Lay<D>::RPT], float *S, bool streaming) {
-    const int rg = threadIdx.x / Lay<D>::TPR, c4 = threadIdx.x % Lay<D>::TPR;
-#pragma unroll
-    for (int r = 0; r < Lay<D>::RPT; ++r) {
-        float4 *p = reinterpret_cast<float4 *>(S + (rg + Lay<D>::RG * r) * D) + c4;
-        if (streaming) __stcs(p, st[r]); else *p = st[r];
-    }
+__device__ __forceinline__ void state_load_issue(Smem<D> &sm, const float *S) {
+    constexpr uint32_t bytes = D * D * 4;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&sm.bar)), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(sm.S)),
+        "l"(S), "r"(bytes), "r"(smem_u32(&sm.bar)), "l"(evict_first_policy())
+        : "memory");
 }
 
-// One recurrence step on the register-resident state, with q,k,v,a(=exp g) in smem:
+// Every thread: wait (bounded) for the state copy; false on timeout.
+template <int D>
+__device__ __forceinline__ bool state_load_wait(Smem<D> &sm) {
+    return umma::mbar_wait(&sm.bar, 0, kWaitCycles);
+}
+
+// One recurrence step on the shared-memory state, with q,k,v,a(=exp g) in shared memory:
 //   S' = diag(a) S;  y_k = S'^T k, y_q = S'^T q;  u = beta (v - y_k);  S = S' + k u^T;
 //   o = scale (y_q + (k.q) u)   (= scale S^T q after the update).   o lands in sm.o.
+// The decayed value S'[i][j] is formed twice (once per pass) by the same rounded product.
+// Pass 2 writes the new state to shared memory (keep), to global memory (g, streaming), to
+// a snapshot (snap, plain stores), in any combination.
 template <int D>
-__device__ __forceinline__ void state_step(float4 (&st)[Lay<D>::RPT], Smem &sm, float beta, float kq, float scale) {
+__device__ __forceinline__ void state_step(Smem<D> &sm, float beta, float kq, float scale, bool keep, float *g,
+                                           float *snap) {
     using L = Lay<D>;
-    const int tid = threadIdx.x, rg = tid / L::TPR, c4 = tid % L::TPR;
-    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
-#pragma unroll
-    for (int r = 0; r < L::RPT; ++r) {
-        const int row = rg + L::RG * r;
-        const float a = sm.a[row], kr = sm.k[row], qr = sm.q[row];
-        float4 s = st[r];
-        s.x = __fmul_rn(s.x, a); s.y = __fmul_rn(s.y, a); s.z = __fmul_rn(s.z, a); s.w = __fmul_rn(s.w, a);
-        st[r] = s;
-        pk.x = __fmaf_rn(s.x, kr, pk.x); pk.y = __fmaf_rn(s.y, kr, pk.y);
-        pk.z = __fmaf_rn(s.z, kr, pk.z); pk.w = __fmaf_rn(s.w, kr, pk.w);
-        pq.x = __fmaf_rn(s.x, qr, pq.x); pq.y = __fmaf_rn(s.y, qr, pq.y);
-        pq.z = __fmaf_rn(s.z, qr, pq.z); pq.w = __fmaf_rn(s.w, qr, pq.w);
+    const int tid = threadIdx.x, j = tid % D, grp = tid / D, r0 = grp * L::RPG;
+    float pk = 0.f, pq = 0.f;
+#pragma unroll 16
+    for (int r = 0; r < L::RPG; ++r) {
+        const int i = r0 + r;
+        const float s = __fmul_rn(sm.S[i * D + j], sm.a[i]);
+        pk = __fmaf_rn(s, sm.k[i], pk);
+        pq = __fmaf_rn(s, sm.q[i], pq);
     }
-    *reinterpret_cast<float4 *>(&sm.red[0][rg][4 * c4]) = pk;
-    *reinterpret_cast<float4 *>(&sm.red[1][rg][4 * c4]) = pq;
+    sm.red[0][grp][j] = pk;
+    sm.red[1][grp][j] = pq;
     __syncthreads();
     if (tid < D) {
         float yk = sm.red[0][0][tid], yq = sm.red[1][0][tid];
 #pragma unroll
-        for (int g = 1; g < L::RG; ++g) { yk = __fadd_rn(yk, sm.red[0][g][tid]); yq = __fadd_rn(yq, sm.red[1][g][tid]); }
+        for (int gg = 1; gg < L::RG; ++gg) { yk = __fadd_rn(yk, sm.red[0][gg][tid]); yq = __fadd_rn(yq, sm.red[1][gg][tid]); }
         const float u = __fmul_rn(beta, __fsub_rn(sm.v[tid], yk));
         sm.u[tid] = u;
         sm.o[tid] = __fmul_rn(scale, __fmaf_rn(kq, u, yq));
     }
     __syncthreads();
-    const float4 u4 = *reinterpret_cast<const float4 *>(&sm.u[4 * c4]);
-#pragma unroll
-    for (int r = 0; r < L::RPT; ++r) {
-        const float kr = sm.k[rg + L::RG * r];
-        float4 s = st[r];
-        s.x = __fmaf_rn(kr, u4.x, s.x); s.y = __fmaf_rn(kr, u4.y, s.y);
-        s.z = __fmaf_rn(kr, u4.z, s.z); s.w = __fmaf_rn(kr, u4.w, s.w);
-        st[r] = s;
+    const float u = sm.u[j];
+    if (!keep) {
+#pragma unroll 16
+        for (int r = 0; r < L::RPG; ++r) {
+            const int i = r0 + r;
+            __stcs(g + i * D + j, __fmaf_rn(sm.k[i], u, __fmul_rn(sm.S[i * D + j], sm.a[i])));
+        }
+    } else if (snap) {
+#pragma unroll 16
+        for (int r = 0; r < L::RPG; ++r) {
+            const int i = r0 + r;
+            const float x = __fmaf_rn(sm.k[i], u, __fmul_rn(sm.S[i * D + j], sm.a[i]));
+            sm.S[i * D + j] = x;
+            snap[i * D + j] = x;
+        }
+    } else {
+#pragma unroll 16
+        for (int r = 0; r < L::RPG; ++r) {
+            const int i = r0 + r;
+            sm.S[i * D + j] = __fmaf_rn(sm.k[i], u, __fmul_rn(sm.S[i * D + j], sm.a[i]));
+        }
     }
 }
 
@@ -119,19 +151,54 @@ __device__ __forceinline__ float sigmoid_rn(float x) {
     return __frcp_rn(__fadd_rn(1.0f, expf(-x)));
 }
 
+// Thread 0: initialise the copy barrier and start the state copy. The barrier's initialisation
+// is made visible to the other threads by the first __syncthreads that follows.
+template <int D>
+__device__ __forceinline__ void state_begin(Smem<D> &sm, const float *S) {
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar, 1);
+        fence_mbar_init();
+        state_load_issue<D>(sm, S);
+    }
+}
+
+// Every thread: wait for the state copy. On a timeout the status is latched, the copy is
+// waited for once more (bounded), and false is returned to every thread of the block.
+template <int D>
+__device__ __forceinline__ bool state_ready(Smem<D> &sm, int *status) {
+    bool ok = state_load_wait<D>(sm);
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok) {
+        if (threadIdx.x == 0) {
+            atomicExch(status, KDA_ERR_TIMEOUT);
+            state_load_wait<D>(sm);
+        }
+        __syncthreads();
+    }
+    return ok;
+}
+
+__device__ __forceinline__ bool misaligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
 // ----------------------------------------------------------------------------- core-only decode
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
 recurrent_decode_kernel(const float *__restrict__ q, const float *__restrict__ k, const float *__restrict__ v,
                         const float *__restrict__ gate, const float *__restrict__ beta,
-                        float *const *__restrict__ h_state, float *__restrict__ o, int H, float scale) {
-    __shared__ Smem sm;
+                        float *const *__restrict__ h_state, float *__restrict__ o, int H, float scale,
+                        int *__restrict__ status) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    Smem<D> &sm = *reinterpret_cast<Smem<D> *>(smem_raw);
     const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
     float *S = h_state[n] + static_cast<size_t>(h) * D * D;
-    float4 st[Lay<D>::RPT];
-    load_state<D>(st, S);
+    if (misaligned16(S)) {  // the bulk copies need 16-byte alignment: skip this head
+        if (tid == 0) atomicExch(status, KDA_ERR_MISALIGNED);
+        return;
+    }
+    state_begin<D>(sm, S);
     const size_t row = (static_cast<size_t>(n) * H + h) * D;
+    const float bt = beta[static_cast<size_t>(n) * H + h];
     float qk = 0.f;
     if (tid < D) {
         const float qd = q[row + tid], kd = k[row + tid];
@@ -140,9 +207,9 @@ recurrent_decode_kernel(const float *__restrict__ q, const float *__restrict__ k
         qk = __fmul_rn(qd, kd);
     }
     const float kq = sum2_first_d<D>(tid < D ? qk : 0.f, 0.f, sm).x;
-    state_step<D>(st, sm, beta[static_cast<size_t>(n) * H + h], kq, scale);
+    if (!state_ready<D>(sm, status)) return;
+    state_step<D>(sm, bt, kq, scale, false, S, nullptr);
     if (tid < D) o[row + tid] = sm.o[tid];
-    store_state<D>(st, S, true);
 }
 
 // ----------------------------------------------------------------------------- fused stateful row
@@ -161,6 +228,7 @@ struct RowParams {
     const uint16_t *out_gate, *o_norm_w;
     uint16_t *o_norm_out, *conv_out;
     float *core;
+    int *status;
     int H, K, n_snap;
     float scale, l2_eps, rms_eps;
     float *h_snap[kMaxSnap];
@@ -168,14 +236,18 @@ struct RowParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) decode_rows_kernel(const RowParams p) {
-    __shared__ Smem sm;
+__global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParams p) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    Smem<D> &sm = *reinterpret_cast<Smem<D> *>(smem_raw);
     const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, H = p.H;
     const int qkv = H * D;
     float *S = (p.h_one ? p.h_one : p.h_arr[n]) + static_cast<size_t>(h) * D * D;
+    if (misaligned16(S)) {  // the bulk copies need 16-byte alignment: skip this head
+        if (tid == 0) atomicExch(p.status, KDA_ERR_MISALIGNED);
+        return;
+    }
+    state_begin<D>(sm, S);
     uint16_t *cst = p.conv_one ? p.conv_one : p.conv_arr[n];
-    float4 st[Lay<D>::RPT];
-    load_state<D>(st, S);
 
     // This thread's conv channels: q and k channel d (tid < D) or v channel d (D <= tid < 2D).
     const bool qk_thread = tid < D, v_thread = tid >= D && tid < 2 * D;
@@ -198,18 +270,26 @@ __global__ void __launch_bounds__(kThreads, 2) decode_rows_kernel(const RowParam
     const float nea = -expf(p.a_log[h]);
     const float dtb = qk_thread ? p.dt_bias[h * D + d] : 0.f;
     const float ow = qk_thread ? bf16_to_f32(p.o_norm_w[d]) : 0.f;
+    bool ok = true;
 
     for (int t = 0; t < p.K; ++t) {
         const size_t row = static_cast<size_t>(n) * p.K + t;
+        // every global input of the row, loaded up front (they do not depend on the state)
+        float x0 = 0.f, x1 = 0.f, graw = 0.f, og = 0.f;
+        if (qk_thread || v_thread) x0 = bf16_to_f32(p.x[row * 3 * qkv + c0]);
+        if (qk_thread) {
+            x1 = bf16_to_f32(p.x[row * 3 * qkv + c1]);
+            graw = bf16_to_f32(p.g_raw[row * qkv + h * D + d]);
+            og = bf16_to_f32(p.out_gate[row * qkv + h * D + d]);
+        }
+        const float blog = p.b_logit[row * H + h];
         // conv step + SiLU (fixed-order FP32), new conv state in registers
         float y0 = 0.f, y1 = 0.f;
         if (qk_thread || v_thread) {
-            const float x0 = bf16_to_f32(p.x[row * 3 * qkv + c0]);
             y0 = __fmaf_rn(w0[3], x0, __fmaf_rn(w0[2], s0[2], __fmaf_rn(w0[1], s0[1], __fmul_rn(w0[0], s0[0]))));
             y0 = __fmul_rn(y0, sigmoid_rn(y0));
             s0[0] = s0[1]; s0[1] = s0[2]; s0[2] = x0;
             if (qk_thread) {
-                const float x1 = bf16_to_f32(p.x[row * 3 * qkv + c1]);
                 y1 = __fmaf_rn(w1[3], x1, __fmaf_rn(w1[2], s1[2], __fmaf_rn(w1[1], s1[1], __fmul_rn(w1[0], s1[0]))));
                 y1 = __fmul_rn(y1, sigmoid_rn(y1));
                 s1[0] = s1[1]; s1[1] = s1[2]; s1[2] = x1;
@@ -224,29 +304,33 @@ __global__ void __launch_bounds__(kThreads, 2) decode_rows_kernel(const RowParam
             qv = bf16_to_f32(qb); kv = bf16_to_f32(kb);
             sm.q[d] = qv; sm.k[d] = kv;
             if (p.conv_out) { p.conv_out[row * 3 * qkv + c0] = qb; p.conv_out[row * 3 * qkv + c1] = kb; }
-            // gate for key channel d, and beta
-            const float g = kda_gate_f32(bf16_to_f32(p.g_raw[row * qkv + h * D + d]), dtb, nea);
-            sm.a[d] = expf(g);
+            // gate for key channel d
+            sm.a[d] = expf(kda_gate_f32(graw, dtb, nea));
         } else if (v_thread) {
             const uint16_t vb = f32_to_bf16(y0);
             sm.v[d] = bf16_to_f32(vb);
             if (p.conv_out) p.conv_out[row * 3 * qkv + c0] = vb;
         }
-        const float beta = sigmoid_rn(p.b_logit[row * H + h]);
+        const float beta = sigmoid_rn(blog);
         const float kq = sum2_first_d<D>(qk_thread ? __fmul_rn(qv, kv) : 0.f, 0.f, sm).x;
-        state_step<D>(st, sm, beta, kq, p.scale);
+        if (t == 0) {
+            ok = state_ready<D>(sm, p.status);
+            if (!ok) break;  // block-uniform
+        }
+        // the last row streams the state out; earlier rows keep it (and write their snapshot)
+        const bool last = t == p.K - 1;
+        float *snap = !last && t < p.n_snap ? p.h_snap[t] + static_cast<size_t>(h) * D * D : nullptr;
+        state_step<D>(sm, beta, kq, p.scale, !last, S, snap);  // sm.o is complete when it returns
         // o_norm: sigmoid-gated RMSNorm over the head's D outputs
         const float ov = qk_thread ? sm.o[d] : 0.f;
         const float ms = sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm).x;
         if (qk_thread) {
             const float rs = rsqrtf(__fadd_rn(__fmul_rn(ms, 1.0f / D), p.rms_eps));
-            const float og = bf16_to_f32(p.out_gate[row * qkv + h * D + d]);
             const float yv = __fmul_rn(__fmul_rn(__fmul_rn(ov, rs), ow), sigmoid_rn(og));
             p.o_norm_out[row * qkv + h * D + d] = f32_to_bf16(yv);
             if (p.core) p.core[row * qkv + h * D + d] = ov;
         }
         if (t < p.n_snap) {
-            store_state<D>(st, p.h_snap[t] + static_cast<size_t>(h) * D * D, false);
             uint16_t *cs = p.conv_snap[t];
             if (qk_thread || v_thread) {
 #pragma unroll
@@ -257,9 +341,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_rows_kernel(const RowParam
                 }
             }
         }
-        __syncthreads();  // smem rows are rewritten by the next row
     }
-    store_state<D>(st, S, true);
+    if (!ok) return;
     if (qk_thread || v_thread) {
 #pragma unroll
         for (int j = 0; j < 3; ++j) cst[c0 * 3 + j] = f32_to_bf16(s0[j]);
@@ -270,10 +353,29 @@ __global__ void __launch_bounds__(kThreads, 2) decode_rows_kernel(const RowParam
     }
 }
 
-int launch_rows(const RowParams &p, int N, int D, cudaStream_t s) {
-    dim3 grid(p.H, N);
-    if (D == 128) decode_rows_kernel<128><<<grid, kThreads, 0, s>>>(p);
-    else decode_rows_kernel<64><<<grid, kThreads, 0, s>>>(p);
+template <int D>
+int launch_rows_d(const RowParams &p, int N, cudaStream_t s) {
+    static std::atomic<unsigned long long> attr_done{0};
+    KDA_TRY(smem_opt_in(decode_rows_kernel<D>, static_cast<int>(sizeof(Smem<D>)), attr_done, true));
+    decode_rows_kernel<D><<<dim3(p.H, N), kThreads, sizeof(Smem<D>), s>>>(p);
+    return launch_status();
+}
+
+int launch_rows(RowParams &p, int N, int D, cudaStream_t s) {
+    p.status = device_status_ptr();
+    if (!p.status) return KDA_ERR_CUDA;
+    return D == 128 ? launch_rows_d<128>(p, N, s) : launch_rows_d<64>(p, N, s);
+}
+
+template <int D>
+int launch_recurrent(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                     float *const *h_state, float *o, int N, int H, float scale, cudaStream_t s) {
+    int *status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
+    static std::atomic<unsigned long long> attr_done{0};
+    KDA_TRY(smem_opt_in(recurrent_decode_kernel<D>, static_cast<int>(sizeof(Smem<D>)), attr_done, true));
+    recurrent_decode_kernel<D><<<dim3(H, N), kThreads, sizeof(Smem<D>), s>>>(q, k, v, gate, beta, h_state, o, H,
+                                                                               scale, status);
     return launch_status();
 }
 
@@ -290,13 +392,10 @@ int kda_recurrent_decode(const float *q, const float *k, const float *v, const f
         return KDA_ERR_MISALIGNED;
     if (N == 0) return KDA_OK;
     if (N > 65535) return KDA_ERR_UNSUPPORTED;
-    dim3 grid(dims->heads, N);
     auto s = static_cast<cudaStream_t>(stream);
     if (dims->head_dim == 128)
-        kda::recurrent_decode_kernel<128><<<grid, kda::kThreads, 0, s>>>(q, k, v, gate, beta, h_state, o, dims->heads, dims->scale);
-    else
-        kda::recurrent_decode_kernel<64><<<grid, kda::kThreads, 0, s>>>(q, k, v, gate, beta, h_state, o, dims->heads, dims->scale);
-    return kda::launch_status();
+        return kda::launch_recurrent<128>(q, k, v, gate, beta, h_state, o, N, dims->heads, dims->scale, s);
+    return kda::launch_recurrent<64>(q, k, v, gate, beta, h_state, o, N, dims->heads, dims->scale, s);
 }
 
 static int fill_row_params(kda::RowParams &p, const kda_bf16 *x, const kda_bf16 *conv_w, const kda_bf16 *g_raw,

@@ -237,13 +237,8 @@ template <int BN>
 int launch_gemm(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
                 int out_f32, cudaStream_t s) {
     using G = GemmCfg<BN>;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::bytes) !=
-            cudaSuccess)
-            return KDA_ERR_CUDA;
-        attr = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    KDA_TRY(smem_opt_in(gemm_kernel<BN>, G::bytes, attr_done));
     CUtensorMap ta, tw;
     KDA_TRY(make_map(&ta, A, M, K, lda, BM));
     KDA_TRY(make_map(&tw, W, N, K, ldw, BN));

@@ -53,8 +53,10 @@ def test_prefill_argument_checks(L):
     d = ctypes.byref(_d())
     args = [BOGUS] * 7
     need = L.kda_chunk_prefill_scratch_bytes(2, 100, d)
-    # B * H * chunks operand packs (D = 64) + the list of chunks handed to the CUDA-core path
-    assert need == 2 * 2 * 2 * (32768 + 32768 + 16384 + 1024) + 256
+    # B * H * chunks operand packs (D = 64: [W; Q o A], M, K o e^{Gamma_C - Gamma} as BF16 hi/lo
+    # tiles, U~ in FP32 with a 4-float row skew, e^{Gamma_C}) + the list of chunks handed to the
+    # CUDA-core path
+    assert need == 2 * 2 * 2 * (32768 + 16384 + 16384 + 2 * 64 * 36 * 4 + 1024) + 256
     assert L.kda_chunk_prefill_scratch_bytes(0, 100, d) == 0
     assert L.kda_chunk_prefill(*args, 1, 0, BOGUS, 0, d, None) == 0  # T = 0: nothing to do
     assert L.kda_chunk_prefill(*args, 0, 10, BOGUS, 0, d, None) == 0  # B = 0

@@ -137,3 +137,30 @@ def test_decode_k_without_snapshots_and_k1():
                          None, 1, [], [], d)
     torch.cuda.synchronize()
     assert torch.equal(out, out_b) and torch.equal(h_a, h_b) and torch.equal(c_a, c_b)
+
+
+def test_misaligned_state_pointer_is_skipped():
+    """A state pointer 4 bytes off a 16-byte boundary (the state copies need 16): that
+    sequence's heads are left untouched and KDA_ERR_MISALIGNED is latched; the aligned
+    sequence in the same call is still updated correctly."""
+    N, H, D = 2, 2, 64
+    ci = core_inputs(N, 1, H, D, seed=5, s0_std=0.1)
+    d = kda.dims(H, D)
+    gate = torch.empty((N, H, D), device="cuda")
+    kda.kda_gate(ci.g_raw.reshape(N, H * D).cuda(), ci.dt_bias.cuda(), ci.a_log.cuda(), gate, N, d)
+    beta = ci.b_logit.reshape(N, H).cuda().contiguous()
+    kda.kda_beta(beta, beta, beta.numel())
+    good = ci.s0[0].cuda().clone()
+    buf = torch.zeros(H * D * D + 4, device="cuda")
+    bad = buf[1:1 + H * D * D].view(H, D, D)
+    bad.copy_(ci.s0[1].cuda())
+    before = bad.clone()
+    o = torch.empty((N, H, D), device="cuda")
+    kda.kda_recurrent_decode(ci.q.reshape(N, H, D).cuda(), ci.k.reshape(N, H, D).cuda(),
+                             ci.v.reshape(N, H, D).cuda(), gate, beta, kda.ptr_array([good, bad]), o, N, d)
+    torch.cuda.synchronize()
+    assert kda.device_status(clear=True) == 7  # KDA_ERR_MISALIGNED
+    assert torch.equal(bad, before)
+    o_ref, S_ref = oracle_prefill(ci)
+    assert rel_l2(np64(o[0]), o_ref[0, 0]) <= TOL
+    assert rel_l2(np64(good), S_ref[0]) <= TOL

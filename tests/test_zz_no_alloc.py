@@ -41,7 +41,7 @@ def _run(fn, ci, d, q, k, v, gate, beta):
 
 
 def test_noalloc_matches_scratch_entry_point_twice(cuda_ok):
-    args = _inputs(2, 448, 16, 128, seed=21)  # 2 x 16 x 7 chunk packs of 129 KB: 28.2 MiB of scratch
+    args = _inputs(2, 384, 16, 128, seed=21)  # 2 x 16 x 6 chunk packs of 149 KB: 27.9 MiB of scratch
     ref_core, ref_S = _run(kda.kda_chunk_prefill, *args)
     for _ in range(2):
         core, S = _run(kda.kda_chunk_prefill_noalloc, *args)
