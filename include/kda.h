@@ -116,7 +116,7 @@ KDA_API int kda_beta(const float *b_logit, float *beta, int n, void *stream);
  *   core      [B*T_pad, H, D] F32 output o = scale * S^T q for rows < T (pad rows are
  *             not written).
  *   scratch   caller-owned device scratch of at least kda_chunk_prefill_scratch_bytes(B, T,
- *             dims) bytes (129 KB per (stream, head, chunk) at head_dim 128), 16-byte aligned:
+ *             dims) bytes (149 KB per (stream, head, chunk) at head_dim 128), 16-byte aligned:
  *             the per-chunk operand tiles passed between the two kernels of the call; contents
  *             on entry do not matter. KDA_ERR_CAPACITY if scratch_bytes is too small.
  * Computed with tcgen05 tensor cores in split-BF16 precision (about 2^-16 relative per
@@ -129,6 +129,22 @@ KDA_API int kda_chunk_prefill(const float *q, const float *k, const float *v, co
 /* Scratch bytes kda_chunk_prefill needs for B streams of T tokens (0 if B or T is 0). */
 KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dims);
 
+/* kda_chunk_prefill_fused — kda_chunk_prefill reading the front end's BF16 output and the
+ * raw gate directly (Glm5NextKdaWorkspace `conv_out` and `g_raw`: the fused-input mode, in
+ * which the FP32 q/k/v/gate buffers are never written or read):
+ *   qkv       [B*T_pad, 3*H*D] BF16 rows q | k | v after conv + SiLU + per-head L2 (the
+ *             layout kda_front_conv_silu_l2 writes to conv_out); only rows < T are read
+ *   g_raw     [B*T_pad, H*D] BF16; dt_bias [H*D] F32; a_log [H] F32: the gate
+ *             g = -exp(a_log[h]) softplus(g_raw + dt_bias) (as kda_gate) is formed in the
+ *             kernel; only rows < T are read
+ *   beta      [B*T_pad, H] F32 (kda_beta's output)
+ *   h_state, core, B, T, scratch, scratch_bytes, dims: as kda_chunk_prefill (same scratch size).
+ * The result equals kda_chunk_prefill on the widened inputs and kda_gate's output. */
+KDA_API int kda_chunk_prefill_fused(const kda_bf16 *qkv, const kda_bf16 *g_raw, const float *dt_bias,
+                                    const float *a_log, const float *beta, float *const *h_state, float *core,
+                                    int B, int T, void *scratch, size_t scratch_bytes, const kda_dims *dims,
+                                    void *stream);
+
 /* kda_chunk_prefill_noalloc — kda_chunk_prefill for callers that cannot allocate device
  * memory (the pages have no counterpart: this is a deployment variant). Some callers cannot
  * call cudaMalloc at all: an engine that hands all free HBM to its KV-cache / state pools at
@@ -139,7 +155,7 @@ KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dim
  * the library holds until the process exits.
  *   - Arguments, layouts and results are exactly those of kda_chunk_prefill.
  *   - Requests needing more scratch than that (kda_chunk_prefill_scratch_bytes(B, T, dims)
- *     above the maximum; for head_dim 128, B * heads * ceil(T / 64) > 254 chunks) are
+ *     above the maximum; for head_dim 128, B * heads * ceil(T / 64) > 219 chunks) are
  *     rejected with KDA_ERR_CAPACITY before anything runs.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *     with that device current; make that first call before any stream capture.
@@ -285,10 +301,10 @@ typedef struct kda_block_weights {
 enum {
     KDA_BUF_QKV_PROJ = 0,   /* [T, 3*H*D] BF16  q|k|v projections                  */
     KDA_BUF_CONV_OUT,       /* [T, 3*H*D] BF16  after conv + SiLU, q|k normalised  */
-    KDA_BUF_Q_F32,          /* [T_pad, H*D] F32                                    */
-    KDA_BUF_K_F32,          /* [T_pad, H*D] F32                                    */
-    KDA_BUF_V_F32,          /* [T_pad, H*D] F32                                    */
-    KDA_BUF_GATE,           /* [T_pad, H, D] F32 log-decay                         */
+    KDA_BUF_Q_F32,          /* 0 bytes: the block's core reads conv_out directly   */
+    KDA_BUF_K_F32,          /* 0 bytes (as above)                                  */
+    KDA_BUF_V_F32,          /* 0 bytes (as above)                                  */
+    KDA_BUF_GATE,           /* 0 bytes: the gate is formed inside the core         */
     KDA_BUF_BETA,           /* [T_pad, H] F32                                      */
     KDA_BUF_CORE,           /* [T_pad, H, D] F32 KDA output before o_norm          */
     KDA_BUF_G_RAW,          /* [T, H*D] BF16  f_b(f_a(h))                           */
@@ -313,9 +329,11 @@ KDA_API size_t kda_workspace_max_tokens(const kda_workspace *ws);
 KDA_API int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr, size_t *bytes);
 
 /* kda_block_prefill — hidden [T, hidden] BF16 (device); h_state [H, D, D] F32 and conv_state
- * [3*H*D, 3] BF16 are carried and updated in place; pad_fill primes the q/k/v tails
- * (Glm5NextKdaLayer `prefill_with_pad_fill`; 0 for `prefill`). The block output lands in
- * KDA_BUF_FINAL_OUT. KDA_ERR_CAPACITY if T > max_tokens. Allocates nothing. */
+ * [3*H*D, 3] BF16 are carried and updated in place. The chunked core runs in the fused-input
+ * mode (kda_chunk_prefill_fused on conv_out and g_raw), which never reads a row past T, so
+ * pad_fill (Glm5NextKdaLayer `prefill_with_pad_fill`; 0 for `prefill`) cannot change the
+ * result; it is accepted for that signature. The block output lands in KDA_BUF_FINAL_OUT.
+ * KDA_ERR_CAPACITY if T > max_tokens. Allocates nothing. */
 KDA_API int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T, float *h_state,
                               kda_bf16 *conv_state, float pad_fill, kda_workspace *ws, void *stream);
 

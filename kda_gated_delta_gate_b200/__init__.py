@@ -63,6 +63,7 @@ _SIGS = {
     "kda_beta": ([_VP, _VP, _I, _VP], _I),
     "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
+    "kda_chunk_prefill_fused": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_simt": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_chunk_prefill_noalloc": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_chunk_prefill_noalloc_max_scratch_bytes": ([], ctypes.c_size_t),
@@ -172,6 +173,19 @@ def kda_chunk_prefill(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d
         scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     return _call("kda_chunk_prefill", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core), B, T,
                  _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+
+
+def kda_chunk_prefill_fused(qkv, g_raw, dt_bias, a_log, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims,
+                            stream=None, scratch=None):
+    """The chunked prefill on the front end's BF16 q|k|v rows and the raw BF16 gate input
+    (the gate is formed in the kernel). `scratch` as for kda_chunk_prefill."""
+    if scratch is None:
+        import torch
+        need = kda_chunk_prefill_scratch_bytes(B, T, d)
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+    return _call("kda_chunk_prefill_fused", _p(qkv), _p(g_raw), _p(dt_bias), _p(a_log), _p(beta), _p(h_state_ptrs),
+                 _p(core), B, T, _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d),
+                 _stream(stream))
 
 
 def kda_chunk_prefill_noalloc(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None):

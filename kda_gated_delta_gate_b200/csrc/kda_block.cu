@@ -1,10 +1,11 @@
 // One KDA block prefill (Glm5NextKdaLayer `prefill` / `prefill_with_pad_fill`), stage by stage
 // into the workspace buffers of Glm5NextKdaWorkspace, with the weights of Glm5NextKdaWeights:
 //   q, k, v = h W^T           -> qkv_proj [T, 3*H*D] BF16 (three GEMMs writing the packed row)
-//   conv + SiLU + q|k L2      -> conv_out, q_f32/k_f32/v_f32 [T_pad, H*D] (tails = pad_fill)
-//   g_raw = f_b(f_a(h))       -> gate (kda_gate)
+//   conv + SiLU + q|k L2      -> conv_out [T, 3*H*D] BF16 (conv state carried in place)
+//   g_raw = f_b(f_a(h))       -> g_raw [T, H*D] BF16
 //   beta = sigmoid(b_proj(h)) (FP32 logits)
-//   chunked core              -> core [T_pad, H, D], recurrent state carried in place
+//   chunked core, fused-input mode: reads conv_out and g_raw directly (the gate is formed in
+//   the kernel; rows past T are never read)  -> core [T_pad, H, D], recurrent state in place
 //   out_gate = g_b(g_a(h));  o_norm_out = gated RMSNorm(core, out_gate);  final_out = o_proj
 // The workspace is allocated once (kda_workspace_create) for at most max_tokens tokens; the
 // prefill call itself allocates nothing.
@@ -52,10 +53,10 @@ int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_
     const size_t sizes[KDA_BUF_COUNT] = {
         T * 3 * qkv * 2,   // QKV_PROJ
         T * 3 * qkv * 2,   // CONV_OUT
-        Tp * qkv * 4,      // Q_F32
-        Tp * qkv * 4,      // K_F32
-        Tp * qkv * 4,      // V_F32
-        Tp * qkv * 4,      // GATE
+        0,                 // Q_F32 (the fused-input core does not widen q, k, v or the gate)
+        0,                 // K_F32
+        0,                 // V_F32
+        0,                 // GATE
         Tp * H * 4,        // BETA
         Tp * qkv * 4,      // CORE
         T * qkv * 2,       // G_RAW
@@ -120,21 +121,20 @@ int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T,
     KDA_TRY(kda::gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, T, qkv, Hd, 0, s));
     KDA_TRY(kda::gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, T, qkv, Hd, 0, s));
     KDA_TRY(kda::gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, T, qkv, Hd, 0, s));
-    KDA_TRY(kda_front_conv_silu_l2(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_Q_F32),
-                                   f32(KDA_BUF_K_F32), f32(KDA_BUF_V_F32), pad_fill, T, d, stream));
-    // forget gate: g_raw = f_b(f_a(h)) -> gate
+    KDA_TRY(kda_front_conv_silu_l2(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), nullptr, nullptr,
+                                   nullptr, pad_fill, T, d, stream));
+    // forget-gate input: g_raw = f_b(f_a(h)) (the gate itself is formed inside the chunked core)
     KDA_TRY(kda::gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, T, R, Hd, 0, s));
     KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, T, qkv, R, 0, s));
-    KDA_TRY(kda_gate(bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log, f32(KDA_BUF_GATE), T, d, stream));
     // beta = sigmoid(b_proj(h)), FP32 logits
     KDA_TRY(kda::gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, T, H, Hd, 1, s));
     KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), T * H, stream));
-    // chunked core from the carried state
+    // chunked core from the carried state, on the BF16 conv_out rows and g_raw
     kda::store_ptr_kernel<<<1, 1, 0, s>>>(ws->state_slot, h_state);
     KDA_TRY(kda::launch_status());
-    KDA_TRY(kda_chunk_prefill(f32(KDA_BUF_Q_F32), f32(KDA_BUF_K_F32), f32(KDA_BUF_V_F32), f32(KDA_BUF_GATE),
-                              f32(KDA_BUF_BETA), ws->state_slot, f32(KDA_BUF_CORE), 1, T, B(KDA_BUF_PREFILL_SCRATCH),
-                              ws->bytes[KDA_BUF_PREFILL_SCRATCH], d, stream));
+    KDA_TRY(kda_chunk_prefill_fused(bf(KDA_BUF_CONV_OUT), bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log, f32(KDA_BUF_BETA),
+                                    ws->state_slot, f32(KDA_BUF_CORE), 1, T, B(KDA_BUF_PREFILL_SCRATCH),
+                                    ws->bytes[KDA_BUF_PREFILL_SCRATCH], d, stream));
     // output gate, gated RMSNorm, output projection
     KDA_TRY(kda::gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, T, R, Hd, 0, s));
     KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0, s));

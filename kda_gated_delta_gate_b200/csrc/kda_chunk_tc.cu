@@ -27,6 +27,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "tma.cuh"
 #include "umma.cuh"
 
 namespace kda {
@@ -59,6 +60,66 @@ struct Pack {
     static constexpr int OFF_A1 = 0, OFF_AM = A1, OFF_A3 = OFF_AM + AM, OFF_UT = OFF_A3 + A3, OFF_AC = OFF_UT + UT;
     static constexpr int bytes = OFF_AC + AC;
 };
+// The chunked path's inputs. FP32 mode: q, k, v, gate [B*T_pad, H, D]. Fused mode: qkv, the
+// BF16 conv_out rows [B*T_pad, 3*H*D] (q | k | v after conv + SiLU + L2), and the BF16 g_raw
+// rows [B*T_pad, H*D] with dt_bias and a_log: the gate is formed in the kernel. beta
+// [B*T_pad, H] FP32 in both.
+struct PrefillIn {
+    const float *q, *k, *v, *gate;
+    const uint16_t *qkv, *g_raw;
+    const float *dt_bias, *a_log, *beta;
+};
+
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t u, float &lo, float &hi) {
+    lo = __uint_as_float(u << 16);
+    hi = __uint_as_float(u & 0xFFFF0000u);
+}
+
+// Channels [c, c + 8) of global token row `row`, head h: q (part 0), k (1) or v (2), as FP32.
+template <int D, bool FUSED>
+__device__ __forceinline__ void load8_in(const PrefillIn &in, int part, size_t row, int H, int h, int c,
+                                         float (&x)[8]) {
+    if constexpr (FUSED) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(in.qkv + row * (3 * static_cast<size_t>(H) * D) +
+                                                         static_cast<size_t>(part * H + h) * D + c);
+        bf16x2_to_f32(u.x, x[0], x[1]); bf16x2_to_f32(u.y, x[2], x[3]);
+        bf16x2_to_f32(u.z, x[4], x[5]); bf16x2_to_f32(u.w, x[6], x[7]);
+    } else {
+        const float *p = (part == 0 ? in.q : (part == 1 ? in.k : in.v)) + row * (static_cast<size_t>(H) * D) +
+                         static_cast<size_t>(h) * D + c;
+        const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+}
+
+// Channels [c, c + 4): q / k / v as above, or the log-decay g (part 3; formed from g_raw in fused mode).
+template <int D, bool FUSED>
+__device__ __forceinline__ float4 load4_in(const PrefillIn &in, int part, size_t row, int H, int h, int c) {
+    if constexpr (FUSED) {
+        if (part == 3) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(in.g_raw + row * (static_cast<size_t>(H) * D) +
+                                                             static_cast<size_t>(h) * D + c);
+            const float nea = -expf(in.a_log[h]);
+            const float *dt = in.dt_bias + static_cast<size_t>(h) * D + c;
+            float r0, r1, r2, r3;
+            bf16x2_to_f32(u.x, r0, r1);
+            bf16x2_to_f32(u.y, r2, r3);
+            return make_float4(kda_gate_f32(r0, dt[0], nea), kda_gate_f32(r1, dt[1], nea),
+                               kda_gate_f32(r2, dt[2], nea), kda_gate_f32(r3, dt[3], nea));
+        }
+        const uint2 u = *reinterpret_cast<const uint2 *>(in.qkv + row * (3 * static_cast<size_t>(H) * D) +
+                                                         static_cast<size_t>(part * H + h) * D + c);
+        float4 r;
+        bf16x2_to_f32(u.x, r.x, r.y);
+        bf16x2_to_f32(u.y, r.z, r.w);
+        return r;
+    } else {
+        const float *p = (part == 0 ? in.q : (part == 1 ? in.k : (part == 2 ? in.v : in.gate))) +
+                         row * (static_cast<size_t>(H) * D) + static_cast<size_t>(h) * D + c;
+        return *reinterpret_cast<const float4 *>(p);
+    }
+}
+
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 1.9 GHz
 
 // Split 8 FP32 values into BF16 hi and lo, packed as two 16-byte chunks (paired conversions).
@@ -167,12 +228,9 @@ struct Intra {
 // The exact CUDA-core intra-chunk computation of one (stream b, head h, chunk ch): every decay
 // factor is a product of per-token factors <= 1, whatever g holds. It writes the whole operand
 // pack. Used for the chunks whose in-block decay is too strong for the tensor-core path.
-template <int D>
-__device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, const float *__restrict__ q,
-                                                const float *__restrict__ v, const float *__restrict__ gate,
-                                                const float *__restrict__ beta,
-                                                uint8_t *__restrict__ scratch, int T, int T_pad, int H, int b,
-                                                int h, int ch, float *smem) {
+template <int D, bool FUSED>
+__device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__restrict__ scratch, int T, int T_pad,
+                                                int H, int b, int h, int ch, float *smem) {
     using I = Intra<D>;
     constexpr int P = I::P, PC = I::PC, NT = kIntraThreads;
     float *sK = smem;              // k, then X: k_i prod_{s=16a}^{i} a_s  (a = block of i)
@@ -189,24 +247,22 @@ __device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, con
     const int tid = threadIdx.x;
     const int n = min(C, T - ch * C);
     const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
-    const size_t rs = static_cast<size_t>(H) * D;
 
     // ---- load k, q and a = e^g (pad guard: rows >= n are k = q = 0, a = 1)
     for (int e = tid; e < C * D / 4; e += NT) {
         const int i = e / (D / 4), c = 4 * (e % (D / 4));
         float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv, av = make_float4(1.f, 1.f, 1.f, 1.f);
         if (i < n) {
-            const size_t off = (row0 + i) * rs + static_cast<size_t>(h) * D + c;
-            kv = *reinterpret_cast<const float4 *>(k + off);
-            qv = *reinterpret_cast<const float4 *>(q + off);
-            const float4 g = *reinterpret_cast<const float4 *>(gate + off);
+            kv = load4_in<D, FUSED>(in, 1, row0 + i, H, h, c);
+            qv = load4_in<D, FUSED>(in, 0, row0 + i, H, h, c);
+            const float4 g = load4_in<D, FUSED>(in, 3, row0 + i, H, h, c);
             av = make_float4(expf(g.x), expf(g.y), expf(g.z), expf(g.w));
         }
         *reinterpret_cast<float4 *>(sK + i * P + c) = kv;
         *reinterpret_cast<float4 *>(sQ + i * P + c) = qv;
         *reinterpret_cast<float4 *>(sA + i * P + c) = av;
     }
-    if (tid < C) sB[tid] = tid < n ? beta[(row0 + tid) * H + h] : 0.f;
+    if (tid < C) sB[tid] = tid < n ? in.beta[(row0 + tid) * H + h] : 0.f;
     __syncthreads();
 
     // ---- diagonal 16x16 blocks: thread (block a, j pair, channel group) walks i upward with
@@ -370,9 +426,8 @@ __device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, con
         *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
         float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
         if (i < n) {
-            const float *src = v + (row0 + i) * rs + static_cast<size_t>(h) * D + cb;
-            v0 = *reinterpret_cast<const float4 *>(src);
-            v1 = *reinterpret_cast<const float4 *>(src + 4);
+            v0 = load4_in<D, FUSED>(in, 2, row0 + i, H, h, cb);
+            v1 = load4_in<D, FUSED>(in, 2, row0 + i, H, h, cb + 4);
         }
         *reinterpret_cast<float4 *>(sA + i * P + cb) = v0;
         *reinterpret_cast<float4 *>(sA + i * P + cb + 4) = v1;
@@ -433,18 +488,17 @@ __device__ __forceinline__ void intra_simt_body(const float *__restrict__ k, con
 }
 
 // Only the chunks the tensor-core kernel listed (count and packed (b, h, ch) entries in scratch).
-template <int D>
+template <int D, bool FUSED>
 __global__ void __launch_bounds__(kIntraThreads, 1)
-intra_fix_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ v,
-                 const float *__restrict__ gate, const float *__restrict__ beta, uint8_t *__restrict__ scratch,
-                 const int *__restrict__ list, int T, int T_pad, int H) {
+intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *__restrict__ list, int T, int T_pad,
+                 int H) {
     extern __shared__ float smem[];
     const int count = list[0];
     const int nch = T_pad / C;
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
         const int id = list[1 + e];
         const int ch = id % nch, h = (id / nch) % H, b = id / (nch * H);
-        intra_simt_body<D>(k, q, v, gate, beta, scratch, T, T_pad, H, b, h, ch, smem);
+        intra_simt_body<D, FUSED>(in, scratch, T, T_pad, H, b, h, ch, smem);
         __syncthreads();
     }
 }
@@ -477,22 +531,14 @@ struct IntraTC {
     static constexpr int STAGE = W_STAGE + Pack<D>::UT;
     static constexpr int R2a = B_BYTES > OFF_TB + 2 * 8192 ? B_BYTES : OFF_TB + 2 * 8192;
     static constexpr int R2 = R2a > STAGE ? R2a : STAGE;
-    static constexpr int GP = D + 4;                 // Gamma row stride (floats)
+    static constexpr int GP = D;                     // g, then Gamma, then v: dense [C][D] rows (TMA boxes)
     static constexpr int G_BYTES = C * GP * 4;
     static constexpr int TAB = 14 * D * 4;           // per-channel reference factors
-    static constexpr int MISC = (C + 1024) * 4 + 256;  // beta[C], tmp[1024], barrier, tmem slot
+    static constexpr int MISC = (C + 1024) * 4 + 256;  // beta[C], tmp[1024], barriers, tmem slot
     static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_G = OFF_B + R2, OFF_TAB = OFF_G + G_BYTES,
                          OFF_MISC = OFF_TAB + TAB;
     static constexpr int bytes = OFF_MISC + MISC + 1024;
 };
-
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // One thread: bulk shared -> global copy (bytes a multiple of 16), in this thread's bulk group.
 __device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
@@ -505,13 +551,15 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Persistent: gridDim.x CTAs walk the (stream, head, chunk) items; each item's q, k, g and
-// beta are fetched while the previous item finishes (g by cp.async into shared memory, q and k
-// into registers, v into L2), and its W | U~ results leave through shared memory in bulk copies.
-template <int D>
+// beta are fetched while the previous item finishes (g by a TMA box into shared memory, q and
+// k into registers, v into L2); v itself arrives by a TMA box once g's space is free again,
+// and the W | U~ results leave through shared memory in bulk copies. The g and v boxes come
+// from 3-D maps whose row extent is T, so rows past T arrive as zeros (the pad guard).
+template <int D, bool FUSED>
 __global__ void __launch_bounds__(kIntraThreads, 1)
-intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const float *__restrict__ v,
-                const float *__restrict__ gate, const float *__restrict__ beta, uint8_t *__restrict__ scratch,
-                int *__restrict__ list, int B, int T, int T_pad, int H, int *__restrict__ status) {
+intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmV, const PrefillIn in,
+                uint8_t *__restrict__ scratch, int *__restrict__ list, int B, int T, int T_pad, int H,
+                int *__restrict__ status) {
     using I = IntraTC<D>;
     using PK = Pack<D>;
     constexpr int NT = kIntraThreads, GP = I::GP, PC = I::PC, PT = I::PT;
@@ -529,13 +577,19 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
     float *sTab = reinterpret_cast<float *>(sm + I::OFF_TAB);
     float *sB = reinterpret_cast<float *>(sm + I::OFF_MISC);
     float *sTmp = sB + C;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + (C + 1024) * 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + (C + 1024) * 4);  // MMA commits
+    uint64_t *gbar = bar + 1, *vbar = bar + 2;                                          // g, v boxes
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 3);
     // reference tables, [entry][D]: 0..3 e^{Gamma_{m_a}}, 4..7 e^{Gamma_C - Gamma_{m_a}},
     // 8..13 e^{Gamma_{m_a} - Gamma_{m_b}} for (a,b) = (1,0),(2,0),(2,1),(3,0),(3,1),(3,2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nch = T_pad / C;
     const int total = B * H * nch;
+    constexpr uint32_t kBox = C * D * (FUSED ? 2 : 4);  // one g (g_raw) or v box
+    // g's box: FP32 g at the start of its space, or BF16 g_raw in the upper half (the gate is
+    // then formed in place, FP32, dense)
+    void *gdst = reinterpret_cast<uint8_t *>(sG) + (FUSED ? C * D * 2 : 0);
+    const int vx0 = FUSED ? 2 * H * D : 0;  // v's column in the box source
     const size_t rs = static_cast<size_t>(H) * D;
 
     if (warp == 0) {
@@ -544,14 +598,17 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
     }
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(gbar, 1);
+        mbar_init(vbar, 1);
         fence_mbar_init();
     }
     auto ld8 = [](const float *p, float (&x)[8]) {
         const float4 a0 = *reinterpret_cast<const float4 *>(p), a1 = *reinterpret_cast<const float4 *>(p + 4);
         x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w; x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
     };
-    // ---- fetch one item's inputs: k, q into registers; g into shared memory (cp.async, zeros
-    //      for rows past T); v only into L2; beta into a register of threads < C
+    // ---- fetch one item's inputs: k, q into registers (zeros past T); g by one TMA box into
+    //      shared memory (thread 0; the caller made the space free); v only into L2; beta into
+    //      a register of threads < C
     float kk[UPT][8], qq[UPT][8], bnext = 0.f;
     auto fetch = [&](int it) {
         const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
@@ -560,48 +617,78 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
 #pragma unroll
         for (int u = 0; u < UPT; ++u) {
             const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
-            const bool in = i < n;
-            const size_t off = (row0 + (in ? i : 0)) * rs + static_cast<size_t>(h) * D + cb;
-            float4 k0 = make_float4(0.f, 0.f, 0.f, 0.f), k1 = k0, q0 = k0, q1 = k0;
-            if (in) {
-                k0 = *reinterpret_cast<const float4 *>(k + off);
-                k1 = *reinterpret_cast<const float4 *>(k + off + 4);
-                q0 = *reinterpret_cast<const float4 *>(q + off);
-                q1 = *reinterpret_cast<const float4 *>(q + off + 4);
-                if ((cb & 31) == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(v + off));
+            if (i < n) {
+                load8_in<D, FUSED>(in, 1, row0 + i, H, h, cb, kk[u]);
+                load8_in<D, FUSED>(in, 0, row0 + i, H, h, cb, qq[u]);
+                if ((cb & (FUSED ? 63 : 31)) == 0) {
+                    const void *vp = FUSED ? static_cast<const void *>(in.qkv + (row0 + i) * (3 * rs) + 2 * rs +
+                                                                      static_cast<size_t>(h) * D + cb)
+                                           : static_cast<const void *>(in.v + (row0 + i) * rs +
+                                                                      static_cast<size_t>(h) * D + cb);
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(vp));
+                }
+            } else {
+#pragma unroll
+                for (int w = 0; w < 8; ++w) { kk[u][w] = 0.f; qq[u][w] = 0.f; }
             }
-            cp_async16(sG + i * GP + cb, gate + off, in ? 16u : 0u);
-            cp_async16(sG + i * GP + cb + 4, gate + off + 4, in ? 16u : 0u);
-            kk[u][0] = k0.x; kk[u][1] = k0.y; kk[u][2] = k0.z; kk[u][3] = k0.w;
-            kk[u][4] = k1.x; kk[u][5] = k1.y; kk[u][6] = k1.z; kk[u][7] = k1.w;
-            qq[u][0] = q0.x; qq[u][1] = q0.y; qq[u][2] = q0.z; qq[u][3] = q0.w;
-            qq[u][4] = q1.x; qq[u][5] = q1.y; qq[u][6] = q1.z; qq[u][7] = q1.w;
         }
-        cp_async_commit();
-        if (tid < C) bnext = tid < n ? beta[(row0 + tid) * H + h] : 0.f;
+        if (tid == 0) {
+            mbar_expect_tx(gbar, kBox);
+            tma_load_3d(gdst, &tmG, h * D, ch * C, b, gbar);
+        }
+        if (tid < C) bnext = tid < n ? in.beta[(row0 + tid) * H + h] : 0.f;
     };
-    if (blockIdx.x < total) fetch(blockIdx.x);
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();  // barriers initialised
     tc_fence_after();
+    if (blockIdx.x < total) fetch(blockIdx.x);
     const uint32_t tmem = *tmem_slot;
-    bool dead = false;  // a tensor-core wait timed out: hand every remaining item to the CUDA-core body
+    bool dead = false;  // a wait timed out: hand every remaining item to the CUDA-core body
+    uint32_t iter = 0;  // items done by this CTA: the parity of the g and v boxes
 
 #pragma unroll 1
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    for (int item = blockIdx.x; item < total; item += gridDim.x, ++iter) {
         const int ch = item % nch, h = (item / nch) % H, b = item / (nch * H);
-        const int n = min(C, T - ch * C);
-        const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
         uint8_t *pack = scratch + static_cast<size_t>(item) * PK::bytes;
-        cp_async_wait_all();
+        if (dead) {  // block-uniform
+            if (tid == 0) list[1 + atomicAdd(list, 1)] = item;
+            continue;
+        }
+        const uint32_t par = iter & 1;
+        bool okg = mbar_wait(gbar, par, kWaitCycles);
         if (tid < C) sB[tid] = bnext;
         if (tid == 0) bulk_wait_read();  // the previous item's staged results have left
-        __syncthreads();
+        okg = __syncthreads_and(okg) != 0;
+        if (!okg) {
+            if (tid == 0) {
+                atomicExch(status, KDA_ERR_TIMEOUT);
+                mbar_wait(gbar, par, kWaitCycles);
+                list[1 + atomicAdd(list, 1)] = item;
+            }
+            dead = true;
+            __syncthreads();
+            continue;
+        }
         // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, range of tokens)
         {
             constexpr int QT = NT / D;  // 4 (D=128) or 8 (D=64) token ranges
             constexpr int TPQ = C / QT;
             const int c = tid % D, qr = tid / D;
+            if constexpr (FUSED) {
+                // g = -exp(a_log) softplus(g_raw + dt_bias) (0 past T), FP32 over g_raw's box
+                const uint16_t *gr = reinterpret_cast<const uint16_t *>(gdst);
+                const int n = min(C, T - ch * C);
+                float x[TPQ];
+#pragma unroll
+                for (int r = 0; r < TPQ; ++r) x[r] = bf16_to_f32(gr[(qr * TPQ + r) * D + c]);
+                const float nea = -expf(in.a_log[h]), dtb = in.dt_bias[static_cast<size_t>(h) * D + c];
+                __syncthreads();
+#pragma unroll
+                for (int r = 0; r < TPQ; ++r) {
+                    const int i = qr * TPQ + r;
+                    sG[i * GP + c] = i < n ? kda_gate_f32(x[r], dtb, nea) : 0.f;
+                }
+            }
             float acc = 0.f;
             for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) { acc += sG[i * GP + c]; sG[i * GP + c] = acc; }
             sTmp[qr * D + c] = acc;
@@ -629,8 +716,12 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
             sTab[13 * D + c] = __expf(gm[3] - gm[2]);
         }
         __syncthreads();
-        // ---- operands of the L/M MMA: A (mid-block reference) and B (all references)
-        bool safe = !dead;
+        // ---- one pass over this thread's (token, 8-channel group) units builds the operands of
+        //      the L/M MMA in shared memory, A (mid-block reference) and B (all references),
+        //      and writes the state-independent pack operands: Q o e^Gamma (A1 rows 64..127) and
+        //      K o e^{Gamma_C - Gamma} (A3); K o e^Gamma stays in registers (kk) for W | U~.
+        //      (The pack is written for unsafe chunks too; the CUDA-core body then rewrites it.)
+        bool safe = true;
 #pragma unroll
         for (int u = 0; u < UPT; ++u) {
             const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
@@ -667,44 +758,18 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
                 }
                 st_pair(sBt, I::B_BYTES / 2, kmaj_off(off2 + i, cb, I::NB), x);
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        safe = __syncthreads_and(safe) != 0;
-        tc_fence_after();
-        // ---- D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127), issued now so that the
-        //      operand pack below is written while the tensor core works
-        if (safe && tid == 0) {
-            constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
-            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
-                const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
-                mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
-                mma_bf16(tmem, ah, bl, id, 1);
-                mma_bf16(tmem, al, bh, id, 1);
-            }
-            mma_commit(bar);
-        }
-        // ---- state-independent operands of the pack: Q o e^Gamma (A1 rows 64..127),
-        //      K o e^{Gamma_C - Gamma} (A3), e^{Gamma_C}; K o e^Gamma stays in registers (kk)
-        //      (written for unsafe chunks too; the CUDA-core body then rewrites the whole pack)
-#pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
-            float gi[8], gm[8], em[8], ecm[8], x[8];
-            ld8(sG + i * GP + cb, gi);
-            ld8(sG + (16 * a + 7) * GP + cb, gm);
+            // pack operands: e^{Gamma_i} = ef e^{Gamma_m}, e^{Gamma_C - Gamma_i} = ei e^{Gamma_C - Gamma_m}
+            float em[8];
             ld8(sTab + a * D + cb, em);
-            ld8(sTab + (4 + a) * D + cb, ecm);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) ef[w] *= em[w];
+            ld8(sTab + (4 + a) * D + cb, em);
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
-                const float ef = __expf(gi[w] - gm[w]) * em[w];   // e^{Gamma_i}
-                const float ei = __expf(gm[w] - gi[w]) * ecm[w];  // e^{Gamma_C - Gamma_i}
-                x[w] = qq[u][w] * ef;
-                qq[u][w] = kk[u][w] * ei;
-                kk[u][w] *= ef;
+                ei[w] *= em[w];
+                x[w] = qq[u][w] * ef[w];
+                qq[u][w] = kk[u][w] * ei[w];
+                kk[u][w] *= ef[w];
             }
             uint4 hi, lo;
             split8(x, hi, lo);
@@ -715,19 +780,28 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
             *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
         }
         if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
-        // v rows of this thread's units (L2 hits by now), for the W | U~ operand
-        float vv[UPT][8];
+        fence_async_smem();
+        tc_fence_before();
+        safe = __syncthreads_and(safe) != 0;
+        tc_fence_after();
+        // ---- v by one TMA box into g's space (Gamma is no longer read), for the W | U~ operand;
+        //      D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127)
+        if (tid == 0) {
+            mbar_expect_tx(vbar, kBox);
+            tma_load_3d(sG, &tmV, vx0 + h * D, ch * C, b, vbar);
+            if (safe) {
+                constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
+                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
 #pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
-            float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-            if (i < n) {
-                const float *src = v + (row0 + i) * rs + static_cast<size_t>(h) * D + cb;
-                v0 = *reinterpret_cast<const float4 *>(src);
-                v1 = *reinterpret_cast<const float4 *>(src + 4);
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
+                    const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
+                    mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
+                    mma_bf16(tmem, ah, bl, id, 1);
+                    mma_bf16(tmem, al, bh, id, 1);
+                }
+                mma_commit(bar);
             }
-            vv[u][0] = v0.x; vv[u][1] = v0.y; vv[u][2] = v0.z; vv[u][3] = v0.w;
-            vv[u][4] = v1.x; vv[u][5] = v1.y; vv[u][6] = v1.z; vv[u][7] = v1.w;
         }
         bool ok = true;
         if (safe) {
@@ -758,6 +832,7 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
             }
             tc_fence_before();
         }
+        ok = ok && mbar_wait(vbar, par, kWaitCycles);
         ok = __syncthreads_and(ok) != 0;
         const bool run = safe && ok;
         if (run) {
@@ -766,8 +841,16 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
+                float x[8];
+                if constexpr (FUSED) {
+                    const uint4 w4 = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(sG) + i * D + cb);
+                    bf16x2_to_f32(w4.x, x[0], x[1]); bf16x2_to_f32(w4.y, x[2], x[3]);
+                    bf16x2_to_f32(w4.z, x[4], x[5]); bf16x2_to_f32(w4.w, x[6], x[7]);
+                } else {
+                    ld8(sG + i * GP + cb, x);
+                }
                 st_pair(sA, I::A_BYTES / 2, mnmaj_off(cb, i, C), kk[u]);
-                st_pair(sA, I::A_BYTES / 2, mnmaj_off(D + cb, i, C), vv[u]);
+                st_pair(sA, I::A_BYTES / 2, mnmaj_off(D + cb, i, C), x);
             }
             // ---- M into the pack (64 x 64 K-major, zero above the diagonal)
             const int r = tid >> 3, c0 = 8 * (tid & 7);
@@ -779,12 +862,18 @@ intra_tc_kernel(const float *__restrict__ k, const float *__restrict__ q, const 
             *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + kmaj_off(r, c0, 64)) = hi;
             *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + PK::AM / 2 + kmaj_off(r, c0, 64)) = lo;
         }
-        // ---- the next item's inputs, fetched while this one finishes (Gamma's space and the
-        //      k, q registers are free; this item's beta is in sB)
-        if (item + static_cast<int>(gridDim.x) < total) fetch(item + gridDim.x);
+        // ---- the next item's inputs are fetched while this one finishes (v's space and the k, q
+        //      registers are free; this item's beta is in sB). A timed-out v box is waited for
+        //      once more, so that nothing still writes that space.
+        if (!ok && tid == 0) mbar_wait(vbar, par, kWaitCycles);
+        fence_async_smem();
+        __syncthreads();
+        const bool more = item + static_cast<int>(gridDim.x) < total;
         bool done = false;
+        if (!run && more) fetch(item + gridDim.x);
         if (run) {
             invert_unit_lower64(sL, sT, sTmp);
+            if (more) fetch(item + gridDim.x);  // after the inverse: its shared-memory traffic runs alone
             // ---- Tb = T diag(beta) as the A operand (64 x 64 K-major, zero above the diagonal)
             {
                 const int r = tid >> 3, c0 = 8 * (tid & 7);
@@ -900,7 +989,8 @@ struct State {
                          OFF_B2 = OFF_B1 + B1, OFF_U = OFF_B2 + B2, OFF_MISC = OFF_U + US;
     static constexpr int MISC = 1024;
     static constexpr int bytes = OFF_MISC + MISC + 1024;  // + alignment slack
-    static constexpr uint32_t TMEM_COLS = 2 * DVS <= 32 ? 32 : (2 * DVS <= 64 ? 64 : 128);
+    // D1 twice (chunk parity: a chunk's outputs are read while the next chunk's D1 is computed), D3
+    static constexpr uint32_t TMEM_COLS = 3 * DVS <= 32 ? 32 : (3 * DVS <= 64 ? 64 : (3 * DVS <= 128 ? 128 : 256));
 };
 
 // A bulk global -> shared copy completing on `bar`, whose expected bytes were already
@@ -974,7 +1064,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tD1 = tmem, tD3 = tmem + DVS;
+    const uint32_t tD3 = tmem + 2 * DVS;
     bool ok = true;
 
     // Epilogue roles: for an M = 128 accumulator warp w reads TMEM lanes 32(w%4)..+31 (rows),
@@ -1010,12 +1100,30 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // O = scale D1[64:128] of chunk c (quads 2 and 3: TMEM lanes 64..127 = the chunk's tokens),
+    // run while the tensor core computes chunk c + 1
+    auto out_epilogue = [&](int c) {
+        const int i = erow - 64, nn = min(C, T - c * C);
+        const size_t r0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(c) * C;
+        const uint32_t tD1c = tmem + (c & 1) * DVS;
+#pragma unroll
+        for (int j = 0; j < HALF; j += 8) {
+            float x[8];
+            tmem_ld8(tmem_lane_base(tD1c, warp) + ccol + j, x);
+            tmem_ld_wait();
+            if (i < nn) {
+                float *dst = core + (r0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
+                *reinterpret_cast<float4 *>(dst) = make_float4(scale * x[0], scale * x[1], scale * x[2], scale * x[3]);
+                *reinterpret_cast<float4 *>(dst + 4) =
+                    make_float4(scale * x[4], scale * x[5], scale * x[6], scale * x[7]);
+            }
+        }
+    };
 
 #pragma unroll 1
     for (int ch = 0; ch < nch; ++ch) {
-        const int n = min(C, T - ch * C);
-        const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
         const uint32_t par = ch & 1;
+        const uint32_t tD1 = tmem + par * DVS;
         const uint8_t *next = packs + static_cast<size_t>(ch + 1) * PK::bytes;
         const bool more = ch + 1 < nch;
         // e^{Gamma_C} of this thread's key row, read early (used in epilogue 2)
@@ -1037,6 +1145,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             }
             mma_commit(&bars[4]);
         }
+        if (ch > 0 && quad >= 2) out_epilogue(ch - 1);
         ok = ok && mbar_wait(&bars[4], par, kWaitCycles);
         ok = ok && mbar_wait(&bars[3], par, kWaitCycles);  // U~ of this chunk
         tc_fence_after();
@@ -1100,28 +1209,13 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             }
         }
         write_state_operand();
-        if (quad >= 2) {
-            const int i = erow - 64;
-#pragma unroll
-            for (int j = 0; j < HALF; j += 8) {
-                float x[8];
-                tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
-                tmem_ld_wait();
-                if (i < n) {
-                    float *dst = core + (row0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
-                    *reinterpret_cast<float4 *>(dst) =
-                        make_float4(scale * x[0], scale * x[1], scale * x[2], scale * x[3]);
-                    *reinterpret_cast<float4 *>(dst + 4) =
-                        make_float4(scale * x[4], scale * x[5], scale * x[6], scale * x[7]);
-                }
-            }
-        }
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
         tc_fence_after();
         if (!ok) break;  // block-uniform: every thread saw the same flag
     }
+    if (ok && quad >= 2) out_epilogue(nch - 1);
     if (!ok) {
         if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
     } else if (srow >= 0) {
@@ -1140,16 +1234,16 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
 template <int D>
 size_t packs_bytes(int B, int H, int nch) { return static_cast<size_t>(B) * H * nch * Pack<D>::bytes; }
 
-template <int D, int DVS>
-int launch_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
-              float *const *h_state, float *core, int B, int T, int H, float scale, void *scratch, cudaStream_t s) {
+template <int D, int DVS, bool FUSED>
+int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, int T, int H, float scale, void *scratch,
+              cudaStream_t s) {
     const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C));
     const int nch = T_pad / C;
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
     static std::atomic<unsigned long long> attr_intra{0}, attr_fix{0}, attr_state{0};
-    KDA_TRY(smem_opt_in(intra_tc_kernel<D>, IntraTC<D>::bytes, attr_intra));
-    KDA_TRY(smem_opt_in(intra_fix_kernel<D>, static_cast<int>(Intra<D>::bytes), attr_fix));
+    KDA_TRY(smem_opt_in(intra_tc_kernel<D, FUSED>, IntraTC<D>::bytes, attr_intra));
+    KDA_TRY(smem_opt_in(intra_fix_kernel<D, FUSED>, static_cast<int>(Intra<D>::bytes), attr_fix));
     KDA_TRY(smem_opt_in(state_kernel<D, DVS>, State<D, DVS>::bytes, attr_state));
     uint8_t *sc = static_cast<uint8_t *>(scratch);
     int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(B, H, nch));
@@ -1161,16 +1255,35 @@ int launch_tc(const float *q, const float *k, const float *v, const float *gate,
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
     const long long items = static_cast<long long>(B) * H * nch;
-    const int intra_grid = static_cast<int>(std::min<long long>(items, sms));
-    intra_tc_kernel<D><<<intra_grid, kIntraThreads, IntraTC<D>::bytes, s>>>(k, q, v, gate, beta, sc, list, B, T, T_pad,
-                                                                            H, status);
+    const int grid = static_cast<int>(std::min<long long>(items, sms));
+    CUtensorMap tmG, tmV;
+    if (FUSED) {
+        KDA_TRY(make_rows_map(&tmG, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, T, T_pad, B, D, C));
+        KDA_TRY(make_rows_map(&tmV, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, T, T_pad, B, D, C));
+    } else {
+        KDA_TRY(make_rows_map(&tmG, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, T, T_pad, B, D, C));
+        KDA_TRY(make_rows_map(&tmV, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, T, T_pad, B, D, C));
+    }
+    intra_tc_kernel<D, FUSED><<<grid, kIntraThreads, IntraTC<D>::bytes, s>>>(tmG, tmV, in, sc, list, B, T, T_pad, H,
+                                                                             status);
     KDA_TRY(launch_status());
-    const int fix_grid = intra_grid;
-    intra_fix_kernel<D><<<fix_grid, kIntraThreads, Intra<D>::bytes, s>>>(k, q, v, gate, beta, sc, list, T, T_pad, H);
+    intra_fix_kernel<D, FUSED><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, T, T_pad, H);
     KDA_TRY(launch_status());
-    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(
-        sc, h_state, core, T, T_pad, H, scale, status);
+    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, T, T_pad, H,
+                                                                                   scale, status);
     return launch_status();
+}
+
+// Value slice width: enough CTAs to cover the SMs (one state CTA per SM fits in shared memory).
+template <bool FUSED>
+int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
+               void *scratch, cudaStream_t s) {
+    const int H = dims->heads;
+    const float sc = dims->scale;
+    if (dims->head_dim == 64) return launch_tc<64, 32, FUSED>(in, h_state, core, B, T, H, sc, scratch, s);
+    const long long units = static_cast<long long>(B) * H;
+    if (units >= 60) return launch_tc<128, 64, FUSED>(in, h_state, core, B, T, H, sc, scratch, s);
+    return launch_tc<128, 32, FUSED>(in, h_state, core, B, T, H, sc, scratch, s);
 }
 
 }  // namespace
@@ -1186,13 +1299,15 @@ size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D) {
 int chunk_prefill_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                      float *const *h_state, float *core, int B, int T, const kda_dims *dims, void *scratch,
                      cudaStream_t s) {
-    const int H = dims->heads;
-    const float sc = dims->scale;
-    if (dims->head_dim == 64) return launch_tc<64, 32>(q, k, v, gate, beta, h_state, core, B, T, H, sc, scratch, s);
-    // value slice width: enough CTAs to cover the SMs (one CTA per SM fits in shared memory)
-    const long long units = static_cast<long long>(B) * H;
-    if (units >= 60) return launch_tc<128, 64>(q, k, v, gate, beta, h_state, core, B, T, H, sc, scratch, s);
-    return launch_tc<128, 32>(q, k, v, gate, beta, h_state, core, B, T, H, sc, scratch, s);
+    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta};
+    return launch_any<false>(in, h_state, core, B, T, dims, scratch, s);
+}
+
+int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
+                           const float *beta, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
+                           void *scratch, cudaStream_t s) {
+    const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta};
+    return launch_any<true>(in, h_state, core, B, T, dims, scratch, s);
 }
 
 }  // namespace kda

@@ -12,11 +12,10 @@
 //               then release the accumulator so the MMAs of the next tile overlap this one.
 // Every wait is bounded; a wait that gives up sets a shared abort flag so all roles leave
 // their loops, records KDA_ERR_TIMEOUT in the device status word, and TMEM is freed.
-#include <cuda.h>
-
 #include <algorithm>
 
 #include "common.cuh"
+#include "tma.cuh"
 #include "umma.cuh"
 
 namespace kda {
@@ -43,10 +42,6 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *t
             smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
 // Wait for a phase, giving up when another role aborted or the clock budget ran out.
@@ -190,23 +185,6 @@ done:
 }
 
 // ------------------------------------------------------------------ host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
 
 // 2-D BF16 tensor map over `rows` x `cols` (row stride ld elements), box 64 (K) x box_rows.
 int make_map(CUtensorMap *tm, const void *base, int rows, int cols, int ld, int box_rows) {

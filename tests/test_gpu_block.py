@@ -99,7 +99,7 @@ def _stages(ws, T, Wt):
     H, D, qkv = Wt.H, Wt.D, Wt.H * Wt.D
     v = lambda n, shp, dt: ws.view(n, shp, dt).clone()  # noqa: E731
     return dict(qkv_proj=v("qkv_proj", (T, 3 * qkv), torch.bfloat16), conv_out=v("conv_out", (T, 3 * qkv), torch.bfloat16),
-                g_raw=v("g_raw", (T, qkv), torch.bfloat16), gate=v("gate", (T, H, D), torch.float32),
+                g_raw=v("g_raw", (T, qkv), torch.bfloat16),
                 beta=v("beta", (T, H), torch.float32), core=v("core", (T, H, D), torch.float32),
                 out_gate=v("out_gate", (T, qkv), torch.bfloat16), o_norm_out=v("o_norm_out", (T, qkv), torch.bfloat16),
                 final_out=v("final_out", (T, Wt.hidden), torch.bfloat16))

@@ -7,7 +7,7 @@ import torch
 
 import kda_gated_delta_gate_b200 as kda
 import oracle
-from synth import core_inputs, t_pad
+from synth import core_inputs, pad_rows, t_pad
 from tests.gpu_harness import gpu_prefill, np64, oracle_prefill, rel_l2, worst_head_rel_l2
 
 pytestmark = pytest.mark.gpu
@@ -143,3 +143,47 @@ def test_long_prefill_poison_full_size(impl):
         assert rel_l2(got_s, S_ref[0, 0]) <= TOL
     del core_n, core_0
     torch.cuda.empty_cache()
+
+
+def _gpu_prefill_fused(ci, *, pad_fill=float("nan"), scale=1.0):
+    """kda_chunk_prefill_fused on BF16 q|k|v rows and BF16 g_raw; every tail row of qkv,
+    g_raw and beta holds pad_fill."""
+    B, T, H, D = ci.B, ci.T, ci.H, ci.D
+    Tp = t_pad(T)
+    d = kda.dims(H, D, scale=scale)
+    qkv = torch.cat([ci.q.reshape(B, T, H * D), ci.k.reshape(B, T, H * D), ci.v.reshape(B, T, H * D)], dim=-1)
+    qkv = pad_rows(qkv.to(torch.bfloat16), Tp, pad_fill).cuda()
+    g_raw = pad_rows(ci.g_raw, Tp, pad_fill).cuda()
+    beta = pad_rows(ci.b_logit, Tp, 0.0).cuda()
+    kda.kda_beta(beta, beta, beta.numel())
+    beta.view(B, Tp, H)[:, T:] = pad_fill
+    states = [ci.s0[b].cuda().clone() for b in range(B)]
+    core = torch.full((B * Tp, H, D), float("nan"), dtype=torch.float32, device="cuda")
+    kda.kda_chunk_prefill_fused(qkv, g_raw, ci.dt_bias.cuda(), ci.a_log.cuda(), beta, kda.ptr_array(states), core, B,
+                                T, d)
+    torch.cuda.synchronize()
+    return core.view(B, Tp, H, D)[:, :T], torch.stack(states)
+
+
+@pytest.mark.parametrize("B,T,H,D", [(1, 4096, 32, 128), (2, 150, 3, 128), (3, 1, 2, 64), (2, 257, 2, 64),
+                                     (1, 129, 1, 128)])
+def test_fused_prefill_matches_f32_path_and_oracle(B, T, H, D):
+    """The fused-input prefill (BF16 conv_out rows and g_raw, gate formed in-kernel) against
+    the FP32 path on the widened inputs (same operands: equal to within FP32 rounding) and
+    against the oracle; tails poisoned with NaN."""
+    ci = core_inputs(B, T, H, D, seed=40 + T, bf16_inputs=True, s0_std=0.1)
+    core_f, S_f = _gpu_prefill_fused(ci, scale=0.7)
+    core, S, _ = gpu_prefill(ci, scale=0.7)
+    assert rel_l2(np64(core_f), np64(core)) <= 1e-6 and rel_l2(np64(S_f), np64(S)) <= 1e-6
+    _check(ci, core_f, S_f, scale=0.7)
+
+
+def test_fused_prefill_extreme_decay_takes_exact_path():
+    """Strong decay on some channels sends chunks to the exact CUDA-core body, which forms the
+    gate from g_raw itself in this mode."""
+    ci = core_inputs(1, 200, 3, 128, seed=31, bf16_inputs=True, s0_std=0.1)
+    ci.a_log[1] = 3.0
+    ci.dt_bias[1 * 128 + 5] = 20.0
+    ci.dt_bias[1 * 128 + 9] = 6.0
+    core_f, S_f = _gpu_prefill_fused(ci)
+    _check(ci, core_f, S_f)
