@@ -5,104 +5,149 @@
 // those BF16 values (a second BF16 rounding, as l2_norm_bf16 does on prefill), and the
 // widening to FP32 with the pad rows set to pad_fill.
 //
-// Grid: (T_pad / 16 token tiles, heads). Block: D threads; thread d owns the head's three
-// channels q_d, k_d, v_d. The tile-0 block is the only reader of the carried conv state
-// and, after its reads, the only writer of the new one (the last three inputs).
+// Grid: (ceil(T_pad / 32) token tiles, column blocks of 256 x 8 channels). Thread j of
+// column block c owns the 8 consecutive channels [8 g, 8 g + 8), g = 256 c + j, of the
+// q|k|v row (16-byte loads and stores) and walks the tile's 32 tokens with a sliding
+// window of the 3 previous inputs. The D/8 threads of one head's q (or k) are adjacent
+// lanes and reduce the per-token sum of squares with shuffles. The tile-0 block of each
+// column block is the only reader of those channels' carried conv state and, after its
+// reads, the only writer of the new one (the last three inputs).
 #include "common.cuh"
 
 namespace kda {
 namespace {
 
-constexpr int kTile = 16;
+constexpr int kFrontThreads = 256, kTT = 32;
+
+__device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
+    x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    x[4] = __uint_as_float(u.z << 16); x[5] = __uint_as_float(u.z & 0xFFFF0000u);
+    x[6] = __uint_as_float(u.w << 16); x[7] = __uint_as_float(u.w & 0xFFFF0000u);
+}
+__device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) {
+    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
 
 template <int D>
-__global__ void __launch_bounds__(D) front_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ conv_state,
-                                                  const uint16_t *__restrict__ conv_w, uint16_t *__restrict__ conv_out,
-                                                  float *__restrict__ qf, float *__restrict__ kf, float *__restrict__ vf,
-                                                  float pad_fill, int T, int H, float eps) {
-    constexpr int NW = D / 32;
-    __shared__ float wsum[2][kTile][NW];
-    const int d = threadIdx.x, lane = d & 31, w = d >> 5;
-    const int h = blockIdx.y, t0 = blockIdx.x * kTile;
+__global__ void __launch_bounds__(kFrontThreads) front_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ conv_state,
+                                                              const uint16_t *__restrict__ conv_w,
+                                                              uint16_t *__restrict__ conv_out, float *__restrict__ qf,
+                                                              float *__restrict__ kf, float *__restrict__ vf,
+                                                              float pad_fill, int T, int T_pad, int H, float eps) {
+    constexpr int LG = D / 8;  // lanes per head part (q, k or v of one head)
     const int qkv = H * D, cd = 3 * qkv;
-    const int ch[3] = {h * D + d, qkv + h * D + d, 2 * qkv + h * D + d};
+    const int g = blockIdx.y * kFrontThreads + threadIdx.x;
+    const bool valid = 8 * g < cd;  // whole head groups are in or out (cd is a multiple of D)
+    const int c0 = valid ? 8 * g : 0;
+    const int part = c0 / qkv, pc = c0 - part * qkv;  // 0 = q, 1 = k, 2 = v; channel within the part
+    const int t0 = blockIdx.x * kTT;
+    float *wide = part == 0 ? qf : (part == 1 ? kf : vf);
 
-    float wt[3][4];
-    float xx[3][kTile + 3];
+    float w[4][8];  // w[tap][channel]
+    {
+        float wr[32];
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float tmp[8];
+            unpack8(reinterpret_cast<const uint4 *>(conv_w + static_cast<size_t>(c0) * 4)[q4], tmp);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) wt[m][j] = bf16_to_f32(conv_w[ch[m] * 4 + j]);
-#pragma unroll
-        for (int j = 0; j < kTile + 3; ++j) {
-            const int t = t0 - 3 + j;  // token index of xx[j]
-            float val = 0.f;
-            if (t < 0) val = bf16_to_f32(conv_state[ch[m] * 3 + (t + 3)]);
-            else if (t < T) val = bf16_to_f32(x[static_cast<size_t>(t) * cd + ch[m]]);
-            xx[m][j] = val;
+            for (int e = 0; e < 8; ++e) wr[8 * q4 + e] = tmp[e];
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j][e] = wr[4 * e + j];
     }
-    // conv + SiLU, rounded to BF16 (conv_out before the in-place L2)
-    float c[3][kTile];
-    float ssq[2][kTile];
+    // window: xm[0] = x_{t-3}, xm[1] = x_{t-2}, xm[2] = x_{t-1} (tiles at or past T read no x)
+    float xm[3][8];
+    if (t0 >= T) {
 #pragma unroll
-    for (int i = 0; i < kTile; ++i) {
+        for (int j = 0; j < 3; ++j)
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
-            float y = wt[m][0] * xx[m][i];
-            y = fmaf(wt[m][1], xx[m][i + 1], y);
-            y = fmaf(wt[m][2], xx[m][i + 2], y);
-            y = fmaf(wt[m][3], xx[m][i + 3], y);
+            for (int e = 0; e < 8; ++e) xm[j][e] = 0.f;
+    } else if (t0 == 0) {
+        float st[24];
+#pragma unroll
+        for (int q3 = 0; q3 < 3; ++q3) {
+            float tmp[8];
+            unpack8(reinterpret_cast<const uint4 *>(conv_state + static_cast<size_t>(c0) * 3)[q3], tmp);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) st[8 * q3 + e] = tmp[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int j = 0; j < 3; ++j) xm[j][e] = st[3 * e + j];
+    } else {
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+            unpack8(*reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t0 - 3 + j) * cd + c0), xm[j]);
+    }
+    const int tend = min(t0 + kTT, T);
+#pragma unroll 4
+    for (int t = t0; t < tend; ++t) {
+        float xc[8], c[8];
+        unpack8(*reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * cd + c0), xc);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float y = w[0][e] * xm[0][e];
+            y = fmaf(w[1][e], xm[1][e], y);
+            y = fmaf(w[2][e], xm[2][e], y);
+            y = fmaf(w[3][e], xc[e], y);
             y = y * sigmoid_f32(y);
-            c[m][i] = bf16_to_f32(f32_to_bf16(y));
+            c[e] = bf16_to_f32(f32_to_bf16(y));  // conv_out before the in-place L2
+            ss = fmaf(c[e], c[e], ss);
+            xm[0][e] = xm[1][e]; xm[1][e] = xm[2][e]; xm[2][e] = xc[e];
         }
-        ssq[0][i] = c[0][i] * c[0][i];
-        ssq[1][i] = c[1][i] * c[1][i];
-    }
 #pragma unroll
-    for (int i = 0; i < kTile; ++i) {
+        for (int o = 1; o < LG; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rs = part < 2 ? rsqrtf(ss + eps) : 1.f;
+        uint16_t ob[8];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            float s = ssq[m][i];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0) wsum[m][i][w] = s;
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kTile; ++i) {
-        const int t = t0 + i;
-        const size_t prow = static_cast<size_t>(t) * qkv + h * D + d;
-        if (t < T) {
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < NW; ++j) { s0 += wsum[0][i][j]; s1 += wsum[1][i][j]; }
-            const uint16_t qb = f32_to_bf16(c[0][i] * rsqrtf(s0 + eps));
-            const uint16_t kb = f32_to_bf16(c[1][i] * rsqrtf(s1 + eps));
-            const uint16_t vb = f32_to_bf16(c[2][i]);
-            uint16_t *orow = conv_out + static_cast<size_t>(t) * cd;
-            orow[ch[0]] = qb; orow[ch[1]] = kb; orow[ch[2]] = vb;
-            if (qf) { qf[prow] = bf16_to_f32(qb); kf[prow] = bf16_to_f32(kb); vf[prow] = bf16_to_f32(vb); }
-        } else if (qf) {
-            qf[prow] = pad_fill; kf[prow] = pad_fill; vf[prow] = pad_fill;
+        for (int e = 0; e < 8; ++e) ob[e] = f32_to_bf16(part < 2 ? c[e] * rs : c[e]);
+        if (valid) {
+            *reinterpret_cast<uint4 *>(conv_out + static_cast<size_t>(t) * cd + c0) =
+                make_uint4(pack2(ob[0], ob[1]), pack2(ob[2], ob[3]), pack2(ob[4], ob[5]), pack2(ob[6], ob[7]));
+            if (qf) {
+                float *dst = wide + static_cast<size_t>(t) * qkv + pc;
+                *reinterpret_cast<float4 *>(dst) =
+                    make_float4(bf16_to_f32(ob[0]), bf16_to_f32(ob[1]), bf16_to_f32(ob[2]), bf16_to_f32(ob[3]));
+                *reinterpret_cast<float4 *>(dst + 4) =
+                    make_float4(bf16_to_f32(ob[4]), bf16_to_f32(ob[5]), bf16_to_f32(ob[6]), bf16_to_f32(ob[7]));
+            }
         }
     }
-    if (blockIdx.x == 0) {
+    if (qf && valid) {  // pad rows of the widened copies
+        for (int t = max(t0, T); t < min(t0 + kTT, T_pad); ++t) {
+            float *dst = wide + static_cast<size_t>(t) * qkv + pc;
+            *reinterpret_cast<float4 *>(dst) = make_float4(pad_fill, pad_fill, pad_fill, pad_fill);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(pad_fill, pad_fill, pad_fill, pad_fill);
+        }
+    }
+    if (blockIdx.x == 0 && valid) {
         // new state = the last three inputs of (old state || x); only this block read the old state
-        float ns[3][3];
+        uint16_t ns[24];
 #pragma unroll
-        for (int m = 0; m < 3; ++m)
+        for (int j = 0; j < 3; ++j) {
+            const int idx = T + j;  // index into (state[0..2], x[0..T-1])
+            float v8[8];
+            if (idx < 3) {
 #pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                const int idx = T + j;  // index into (state[0..2], x[0..T-1])
-                ns[m][j] = idx < 3 ? bf16_to_f32(conv_state[ch[m] * 3 + idx])
-                                   : bf16_to_f32(x[static_cast<size_t>(idx - 3) * cd + ch[m]]);
+                for (int e = 0; e < 8; ++e) v8[e] = bf16_to_f32(conv_state[static_cast<size_t>(c0 + e) * 3 + idx]);
+            } else {
+                unpack8(*reinterpret_cast<const uint4 *>(x + static_cast<size_t>(idx - 3) * cd + c0), v8);
             }
 #pragma unroll
-        for (int m = 0; m < 3; ++m)
+            for (int e = 0; e < 8; ++e) ns[3 * e + j] = f32_to_bf16(v8[e]);
+        }
+        // only this thread reads or writes these 8 channels' state, and its reads come first
+        uint4 *dst = reinterpret_cast<uint4 *>(conv_state + static_cast<size_t>(c0) * 3);
 #pragma unroll
-            for (int j = 0; j < 3; ++j) conv_state[ch[m] * 3 + j] = f32_to_bf16(ns[m][j]);
+        for (int q3 = 0; q3 < 3; ++q3)
+            dst[q3] = make_uint4(pack2(ns[8 * q3], ns[8 * q3 + 1]), pack2(ns[8 * q3 + 2], ns[8 * q3 + 3]),
+                                 pack2(ns[8 * q3 + 4], ns[8 * q3 + 5]), pack2(ns[8 * q3 + 6], ns[8 * q3 + 7]));
     }
 }
 
@@ -117,14 +162,18 @@ extern "C" int kda_front_conv_silu_l2(const kda_bf16 *x, kda_bf16 *conv_state, c
     const bool any_f = q_f32 || k_f32 || v_f32, all_f = q_f32 && k_f32 && v_f32;
     if (any_f && !all_f) return KDA_ERR_INVALID_ARG;
     if (T == 0) return KDA_OK;
+    if (!kda::aligned16(x) || !kda::aligned16(conv_state) || !kda::aligned16(conv_w) || !kda::aligned16(conv_out) ||
+        (any_f && (!kda::aligned16(q_f32) || !kda::aligned16(k_f32) || !kda::aligned16(v_f32))))
+        return KDA_ERR_MISALIGNED;
     const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), kda::kChunk));
-    dim3 grid(T_pad / kda::kTile, dims->heads);
+    const int cd = 3 * dims->heads * dims->head_dim;
+    dim3 grid((T_pad + kda::kTT - 1) / kda::kTT, (cd / 8 + kda::kFrontThreads - 1) / kda::kFrontThreads);
     auto s = static_cast<cudaStream_t>(stream);
     if (dims->head_dim == 128)
-        kda::front_kernel<128><<<grid, 128, 0, s>>>(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32, pad_fill, T,
-                                                    dims->heads, dims->l2_eps);
+        kda::front_kernel<128><<<grid, kda::kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32,
+                                                                   pad_fill, T, T_pad, dims->heads, dims->l2_eps);
     else
-        kda::front_kernel<64><<<grid, 64, 0, s>>>(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32, pad_fill, T,
-                                                  dims->heads, dims->l2_eps);
+        kda::front_kernel<64><<<grid, kda::kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32,
+                                                                  pad_fill, T, T_pad, dims->heads, dims->l2_eps);
     return kda::launch_status();
 }
