@@ -337,6 +337,30 @@ KDA_API int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr,
 KDA_API int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T, float *h_state,
                               kda_bf16 *conv_state, float pad_fill, kda_workspace *ws, void *stream);
 
+/* kda_block_decode — N independent sequences, one token each, through the whole block
+ * (Glm5NextKdaLayer `decode`): the projections of the N hidden rows (each weight read once for
+ * all rows), kda_decode_fused's stateful row, then o_proj.
+ *   hidden      [N, hidden] BF16 (device)
+ *   h_state     DEVICE array of N pointers to [H, D, D] F32 states (as kda_decode_fused)
+ *   conv_state  DEVICE array of N pointers to [3*H*D, 3] BF16 conv states
+ * Results: KDA_BUF_FINAL_OUT rows 0..N-1 (block output), and the stage buffers QKV_PROJ,
+ * G_RAW, BETA (FP32 beta logits), OUT_GATE, CONV_OUT, CORE, O_NORM_OUT for those rows.
+ * KDA_ERR_CAPACITY if N > max_tokens. Allocates nothing. */
+KDA_API int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, float *const *h_state,
+                             kda_bf16 *const *conv_state, kda_workspace *ws, void *stream);
+
+/* kda_block_decode_k — K rows of ONE sequence through the whole block (Glm5NextKdaLayer
+ * `decode_k`: the K-token verify reads every weight once for all K rows). Projections of the
+ * K rows in one pass, kda_decode_k's stateful rows with snapshots, then o_proj.
+ * Bit-identical to K serial kda_block_decode calls with N = 1 on the same sequence (every
+ * projection of a row computes the same bits whatever the number of rows in the call).
+ *   hidden [K, hidden] BF16; h_state [H, D, D] F32 and conv_state [3*H*D, 3] BF16 (single
+ *   device pointers, updated in place); h_snap, conv_snap, n_snap as kda_decode_k.
+ * 1 <= K <= 32 (KDA_ERR_UNSUPPORTED beyond), K <= max_tokens (else KDA_ERR_CAPACITY). */
+KDA_API int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K, float *h_state,
+                               kda_bf16 *conv_state, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
+                               kda_workspace *ws, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,8 @@ _SIGS = {
     "kda_workspace_max_tokens": ([_VP], ctypes.c_size_t),
     "kda_workspace_buffer": ([_VP, _I, ctypes.POINTER(_VP), ctypes.POINTER(ctypes.c_size_t)], _I),
     "kda_block_prefill": ([_VP, _VP, _I, _VP, _VP, _F, _VP, _VP], _I),
+    "kda_block_decode": ([_VP, _VP, _I, _VP, _VP, _VP, _VP], _I),
+    "kda_block_decode_k": ([_VP, _VP, _I, _VP, _VP, _VP, _VP, _I, _VP, _VP], _I),
 }
 
 
@@ -307,3 +309,22 @@ def kda_block_prefill(weights: KdaBlockWeights, hidden, T: int, h_state, conv_st
                       ws: Workspace, stream=None):
     return _call("kda_block_prefill", ctypes.byref(weights), _p(hidden), T, _p(h_state), _p(conv_state),
                  float(pad_fill), ws.handle, _stream(stream))
+
+
+def kda_block_decode(weights: KdaBlockWeights, hidden, N: int, h_state_ptrs, conv_state_ptrs, ws: Workspace,
+                     stream=None):
+    """N sequences x 1 token through the whole block; h_state_ptrs / conv_state_ptrs are device
+    int64 arrays of N pointers (ptr_array). The output is in ws buffer "final_out"."""
+    return _call("kda_block_decode", ctypes.byref(weights), _p(hidden), N, _p(h_state_ptrs), _p(conv_state_ptrs),
+                 ws.handle, _stream(stream))
+
+
+def kda_block_decode_k(weights: KdaBlockWeights, hidden, K: int, h_state, conv_state, h_snaps: Sequence,
+                       conv_snaps: Sequence, ws: Workspace, stream=None):
+    """K rows of one sequence through the whole block (snapshots after every row but the last)."""
+    n = len(h_snaps)
+    hs = host_ptr_array(h_snaps) if n else None
+    cs = host_ptr_array(conv_snaps) if n else None
+    return _call("kda_block_decode_k", ctypes.byref(weights), _p(hidden), K, _p(h_state), _p(conv_state),
+                 ctypes.cast(hs, _VP) if hs is not None else None, ctypes.cast(cs, _VP) if cs is not None else None,
+                 n, ws.handle, _stream(stream))

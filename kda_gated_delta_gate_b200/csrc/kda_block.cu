@@ -9,6 +9,15 @@
 //   out_gate = g_b(g_a(h));  o_norm_out = gated RMSNorm(core, out_gate);  final_out = o_proj
 // The workspace is allocated once (kda_workspace_create) for at most max_tokens tokens; the
 // prefill call itself allocates nothing.
+//
+// Block decode (Glm5NextKdaLayer `decode`, `decode_k`): the same projections for the call's
+// rows (N sequences x 1 token, or K rows of one sequence), each weight read once for all
+// rows, then the fused stateful rows (kda_decode_fused / kda_decode_k: conv + SiLU + L2, gate,
+// beta, recurrence, gated RMSNorm) and o_proj. Every projection runs the tcgen05 GEMM with the
+// call's rows inside 128-row tiles and the column-tile width fixed by the weight's output
+// size, so each row's dot products take the same K-step order in the same tile shapes
+// whatever the number of rows: a row's projections are bit-identical in a call of K rows and
+// in a call of one (the batched-M matrix-vector product the decode_k identity needs).
 #include <cstring>
 #include <new>
 
@@ -32,6 +41,37 @@ struct kda_workspace {
     size_t bytes[KDA_BUF_COUNT];
     float **state_slot;  // device array holding the one state pointer of the call
 };
+
+namespace kda {
+namespace {
+// Projections of M rows of `hidden` into the workspace: qkv_proj (q|k|v packed), g_raw,
+// b_logit (FP32, in the BETA buffer), out_gate.
+int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M, kda_workspace *ws, cudaStream_t s) {
+    const kda_dims *d = &ws->dims;
+    const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
+    auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, M, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, M, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, M, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, M, R, Hd, 0, s));
+    KDA_TRY(gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, M, qkv, R, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, M, H, Hd, 1, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, M, R, Hd, 0, s));
+    KDA_TRY(gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, M, qkv, R, 0, s));
+    return KDA_OK;
+}
+
+int check_block_args(const kda_block_weights *w, const kda_bf16 *hidden, const kda_workspace *ws) {
+    if (!w || !hidden || !ws) return KDA_ERR_INVALID_ARG;
+    if (w->hidden != ws->hidden || w->rank != ws->rank) return KDA_ERR_INVALID_ARG;
+    if (!w->q_proj || !w->k_proj || !w->v_proj || !w->conv || !w->f_a || !w->f_b || !w->dt_bias || !w->a_log ||
+        !w->b_proj || !w->g_a || !w->g_b || !w->o_norm || !w->o_proj)
+        return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+}  // namespace
+}  // namespace kda
 
 extern "C" {
 
@@ -102,13 +142,10 @@ int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr, size_t 
 
 int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T, float *h_state,
                       kda_bf16 *conv_state, float pad_fill, kda_workspace *ws, void *stream) {
-    if (!w || !hidden || !h_state || !conv_state || !ws || T < 0) return KDA_ERR_INVALID_ARG;
+    KDA_TRY(kda::check_block_args(w, hidden, ws));
+    if (!h_state || !conv_state || T < 0) return KDA_ERR_INVALID_ARG;
     if (T == 0) return KDA_OK;
     if (static_cast<size_t>(T) > ws->max_tokens) return KDA_ERR_CAPACITY;
-    if (w->hidden != ws->hidden || w->rank != ws->rank) return KDA_ERR_INVALID_ARG;
-    if (!w->q_proj || !w->k_proj || !w->v_proj || !w->conv || !w->f_a || !w->f_b || !w->dt_bias || !w->a_log ||
-        !w->b_proj || !w->g_a || !w->g_b || !w->o_norm || !w->o_proj)
-        return KDA_ERR_INVALID_ARG;
     const kda_dims *d = &ws->dims;
     auto s = static_cast<cudaStream_t>(stream);
     const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
@@ -143,6 +180,45 @@ int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T,
     KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), Hd, T, Hd, qkv, 0, s));
     (void)Tp;
     return KDA_OK;
+}
+
+int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, float *const *h_state,
+                     kda_bf16 *const *conv_state, kda_workspace *ws, void *stream) {
+    KDA_TRY(kda::check_block_args(w, hidden, ws));
+    if (!h_state || !conv_state || N < 0) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    if (static_cast<size_t>(N) > ws->max_tokens) return KDA_ERR_CAPACITY;
+    auto s = static_cast<cudaStream_t>(stream);
+    const kda_dims *d = &ws->dims;
+    const int qkv = d->heads * d->head_dim;
+    auto bf = [&](int i) { return static_cast<kda_bf16 *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    KDA_TRY(kda::block_projections(w, hidden, N, ws, s));
+    KDA_TRY(kda_decode_fused(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
+                             f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
+                             bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), N, d, stream));
+    return kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, N, ws->hidden,
+                          qkv, 0, s);
+}
+
+int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K, float *h_state,
+                       kda_bf16 *conv_state, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
+                       kda_workspace *ws, void *stream) {
+    KDA_TRY(kda::check_block_args(w, hidden, ws));
+    if (!h_state || !conv_state || K < 1) return KDA_ERR_INVALID_ARG;
+    if (K > 32) return KDA_ERR_UNSUPPORTED;
+    if (static_cast<size_t>(K) > ws->max_tokens) return KDA_ERR_CAPACITY;
+    auto s = static_cast<cudaStream_t>(stream);
+    const kda_dims *d = &ws->dims;
+    const int qkv = d->heads * d->head_dim;
+    auto bf = [&](int i) { return static_cast<kda_bf16 *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    KDA_TRY(kda::block_projections(w, hidden, K, ws, s));
+    KDA_TRY(kda_decode_k(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
+                         f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
+                         bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), K, h_snap, conv_snap, n_snap, d, stream));
+    return kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, K, ws->hidden,
+                          qkv, 0, s);
 }
 
 }  // extern "C"

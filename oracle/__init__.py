@@ -284,3 +284,27 @@ def decode_rows(x_rows, conv_state, conv_w, g_raw, dt_bias, a_log, b_logit, out_
         snaps.append((S[0].copy(), cs.copy()))
     return dict(conv_out=conv_out, core=core, o_norm_out=onorm, h_state=S[0], conv_state=cs,
                 snapshots=snaps)
+
+
+def block_decode(W, hidden_rows, h_state, conv_state, *, scale: float = 1.0, l2_eps: float = 1e-6,
+                 rms_eps: float = 1e-6) -> dict:
+    """K rows of ONE sequence through the whole block, one token at a time.
+
+    Glm5NextKdaLayer `decode` / `decode_k` with the block's projections: every row's
+    q/k/v, f_b(f_a(h)), b_proj(h) and g_b(g_a(h)) (BF16 outputs, FP32 beta logits, as on
+    prefill), then decode_rows' stateful row (conv + SiLU + L2, gate, beta, recurrence,
+    o_norm), then o_proj -> BF16. hidden_rows [K, hidden]; h_state [H, D, D];
+    conv_state [3*H*D, 3]. Returns decode_rows' dict plus the projection stages and final_out.
+    """
+    H, D = W.H, W.D
+    h = _f64(hidden_rows)
+    x_rows = np.concatenate([bf16_round(linear(h, W.w_q)), bf16_round(linear(h, W.w_k)),
+                             bf16_round(linear(h, W.w_v))], axis=1)
+    g_raw = bf16_round(linear(bf16_round(linear(h, W.f_a)), W.f_b))
+    b_logit = linear(h, W.b_proj)
+    out_gate = bf16_round(linear(bf16_round(linear(h, W.g_a)), W.g_b))
+    r = decode_rows(x_rows, conv_state, W.conv_w, g_raw, W.dt_bias, W.a_log, b_logit, out_gate, W.o_norm,
+                    h_state, H, D, scale=scale, l2_eps=l2_eps, rms_eps=rms_eps)
+    r.update(qkv_proj=x_rows, g_raw=g_raw, b_logit=b_logit, out_gate=out_gate,
+             final_out=bf16_round(linear(r["o_norm_out"], W.o_proj)))
+    return r

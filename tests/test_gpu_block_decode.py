@@ -1,0 +1,102 @@
+"""GPU block decode (Glm5NextKdaLayer `decode`: N sequences x 1 token through the whole block)
+and block decode_k (`decode_k`: K rows of one sequence, projections read once for all rows)
+against the oracle, and the decode_k identity through the whole block: K rows in one call
+are bit-identical to K one-row calls, snapshots included."""
+import numpy as np
+import pytest
+import torch
+
+import kda_gated_delta_gate_b200 as kda
+import oracle
+from synth import block_hidden, block_weights
+from tests.gpu_harness import np64, rel_l2
+from tests.test_gpu_block import _device_weights
+
+pytestmark = pytest.mark.gpu
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(autouse=True)
+def _status(cuda_ok):
+    kda.device_status(clear=True)
+    yield
+    assert kda.device_status(clear=True) == 0
+
+
+def _states(n, H, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    hs = torch.randn((n, H, D, D), generator=g) * 0.1
+    cs = torch.randn((n, 3 * H * D, 3), generator=g).to(torch.bfloat16)
+    return hs, cs
+
+
+@pytest.mark.parametrize("hidden,H,D,rank,N,std", [(256, 2, 64, 64, 3, 0.05), (4096, 32, 128, 128, 4, 0.02)])
+def test_block_decode_matches_oracle(hidden, H, D, rank, N, std):
+    Wt = block_weights(hidden, H, D, rank, seed=7, std=std)
+    h = block_hidden(N, hidden, seed=7)
+    hs, cs = _states(N, H, D, seed=7)
+    dw = _device_weights(Wt)
+    st = kda.block_weights_struct(dw)
+    ws = kda.Workspace(kda.dims(H, D), hidden, rank, max_tokens=8)
+    hd = [hs[n].cuda().clone() for n in range(N)]
+    cd = [cs[n].cuda().clone() for n in range(N)]
+    kda.kda_block_decode(st, h.cuda(), N, kda.ptr_array(hd), kda.ptr_array(cd), ws)
+    torch.cuda.synchronize()
+    final = np64(ws.view("final_out", (N, hidden), torch.bfloat16))
+    for n in range(N):
+        ref = oracle.block_decode(Wt, h[n:n + 1], hs[n], cs[n])
+        assert rel_l2(final[n:n + 1], ref["final_out"]) <= TOL_BF16
+        assert rel_l2(np64(hd[n]), ref["h_state"]) <= TOL_BF16
+        assert rel_l2(np64(cd[n]), ref["conv_state"]) <= 4e-3
+    ws.close()
+
+
+@pytest.mark.parametrize("hidden,H,D,rank,K,std", [(256, 2, 64, 64, 5, 0.05), (4096, 32, 128, 128, 4, 0.02)])
+def test_block_decode_k_bit_identical_to_serial_block_decodes(hidden, H, D, rank, K, std):
+    Wt = block_weights(hidden, H, D, rank, seed=11, std=std)
+    h = block_hidden(K, hidden, seed=11).cuda()
+    hs, cs = _states(1, H, D, seed=11)
+    dw = _device_weights(Wt)
+    st = kda.block_weights_struct(dw)
+    ws = kda.Workspace(kda.dims(H, D), hidden, rank, max_tokens=K)
+    # one call of K rows, snapshots after rows 0..K-2
+    ha, ca = hs[0].cuda().clone(), cs[0].cuda().clone()
+    h_snaps = [torch.full_like(ha, float("nan")) for _ in range(K - 1)]
+    c_snaps = [torch.zeros_like(ca) for _ in range(K - 1)]
+    kda.kda_block_decode_k(st, h, K, ha, ca, h_snaps, c_snaps, ws)
+    torch.cuda.synchronize()
+    final_k = ws.view("final_out", (K, hidden), torch.bfloat16).clone()
+    onorm_k = ws.view("o_norm_out", (K, H * D), torch.bfloat16).clone()
+    # K serial one-row calls
+    hb, cb = hs[0].cuda().clone(), cs[0].cuda().clone()
+    rows, onorms = [], []
+    for t in range(K):
+        kda.kda_block_decode(st, h[t:t + 1].contiguous(), 1, kda.ptr_array([hb]), kda.ptr_array([cb]), ws)
+        torch.cuda.synchronize()
+        rows.append(ws.view("final_out", (1, hidden), torch.bfloat16).clone())
+        onorms.append(ws.view("o_norm_out", (1, H * D), torch.bfloat16).clone())
+        if t < K - 1:
+            assert torch.equal(hb, h_snaps[t]) and torch.equal(cb, c_snaps[t]), t
+    assert torch.equal(torch.cat(onorms), onorm_k)
+    assert torch.equal(torch.cat(rows), final_k)
+    assert torch.equal(ha, hb) and torch.equal(ca, cb)
+    ref = oracle.block_decode(Wt, h.cpu(), hs[0], cs[0])
+    assert rel_l2(np64(final_k), ref["final_out"]) <= TOL_BF16
+    assert rel_l2(np64(ha), ref["h_state"]) <= TOL_BF16
+    for t in range(K - 1):
+        assert rel_l2(np64(h_snaps[t]), ref["snapshots"][t][0]) <= TOL_BF16
+    ws.close()
+
+
+def test_block_decode_argument_checks():
+    Wt = block_weights(256, 2, 64, 64, seed=1, std=0.05)
+    st = kda.block_weights_struct(_device_weights(Wt))
+    ws = kda.Workspace(kda.dims(2, 64), 256, 64, max_tokens=4)
+    hs = torch.zeros((2, 64, 64), device="cuda")
+    cs = torch.zeros((384, 3), dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros((40, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kda.KdaError):  # more rows than the workspace holds
+        kda.kda_block_decode(st, h, 5, kda.ptr_array([hs] * 5), kda.ptr_array([cs] * 5), ws)
+    with pytest.raises(kda.KdaError):  # K > 32
+        kda.kda_block_decode_k(st, h, 33, hs, cs, [], [], ws)
+    ws.close()

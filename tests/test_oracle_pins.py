@@ -279,3 +279,31 @@ def test_block_prefill_split_equals_whole():
                                rtol=2 ** -7, atol=1e-6)
     np.testing.assert_allclose(b["h_state"], whole["h_state"], rtol=1e-9, atol=1e-12)
     np.testing.assert_array_equal(b["conv_state"], whole["conv_state"])
+
+
+def test_block_decode_rows_match_block_prefill():
+    """The block decode of K rows (one token at a time: Glm5NextKdaLayer decode / decode_k)
+    against the block prefill of the same K tokens: identical projections and conv state; the
+    conv output differs only by the prefill's second BF16 rounding of q|k (l2_norm_bf16 in
+    place), so the recurrent state and the block output agree to BF16 resolution."""
+    from synth import block_weights, block_hidden
+    Wt = block_weights(hidden=64, H=2, D=16, rank=8, seed=6, std=0.2)
+    h = block_hidden(5, 64, seed=6)
+    r = np.random.default_rng(6)
+    hs = r.standard_normal((2, 16, 16)) * 0.1
+    cs = oracle.bf16_round(r.standard_normal((96, 3)))
+    dec = oracle.block_decode(Wt, h, hs, cs)
+    pre = oracle.block_prefill(Wt, h, hs, cs)
+    for k_ in ("qkv_proj", "g_raw", "b_logit", "out_gate", "conv_state"):
+        np.testing.assert_array_equal(dec[k_], pre[k_])
+    assert np.all(np.abs(dec["conv_out"] - pre["conv_out"]) <= 2 * 2.0 ** -7 * np.abs(pre["conv_out"]) + 1e-30)
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)  # noqa: E731
+    assert rel(dec["h_state"], pre["h_state"]) <= 2e-2
+    assert rel(dec["final_out"], pre["final_out"]) <= 2e-2
+    # decode_k over K rows == K serial one-row decodes (bit for bit), snapshots included
+    S, c = hs, cs
+    for t in range(5):
+        one = oracle.block_decode(Wt, h[t:t + 1], S, c)
+        np.testing.assert_array_equal(one["final_out"][0], dec["final_out"][t])
+        np.testing.assert_array_equal(one["h_state"], dec["snapshots"][t][0])
+        S, c = one["h_state"], one["conv_state"]
