@@ -246,7 +246,7 @@ def main():
     e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch)
 
     # ---- the full block (projections + front end + core + back end) and its dominant GEMM
-    blk = None if args.no_block else _block_leg(kda, torch, dev, s, stream, flush, tc_peak)
+    blk = None if args.no_block else _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm)
 
     result = None
     if rank == 0:
@@ -312,9 +312,11 @@ def _decode_leg(kda, torch, dev, s, stream, flush, hbm):
             "frac_hbm": all_bytes / (ms * 1e-3) / 1e9 / hbm}
 
 
-def _block_leg(kda, torch, dev, s, stream, flush, tc_peak):
+def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
     """KDA block prefill, hidden 4096, H 32, D 128, rank 128, T 8192 (BF16 weights N(0, 0.02)),
-    and the q_proj-sized GEMM (8192 x 4096 x 4096) alone."""
+    the q_proj-sized GEMM (8192 x 4096 x 4096) alone, and the block decode on the same
+    weights: one token of one sequence, K = 4 rows of one sequence (decode_k), and 256
+    sequences x 1 token."""
     import types
     from synth import block_hidden, block_weights
     hidden, Hh, Dd, rank, Tb = 4096, 32, 128, 128, 8192
@@ -347,12 +349,35 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak):
     C = torch.empty((Tb, hidden), dtype=torch.bfloat16, device=dev)
     gms = timed(lambda: kda.kda_gemm_bf16(hid, Wt.w_q, C, Tb, hidden, hidden, stream=s))
     gflop = 2.0 * Tb * hidden * hidden
+    # block decode (L2 flushed before every call, so the weights stream from HBM)
+    wbytes = 2.0 * (3 * qkv * hidden + 2 * rank * hidden + 2 * qkv * rank + Hh * hidden + qkv * hidden)
+    sbytes = 2.0 * Hh * Dd * Dd * 4 + 2.0 * cd * 3 * 2  # one sequence's state + conv state, read + write
+    g = torch.Generator(device=dev).manual_seed(3)
+    n_b = 256
+    hs_b = torch.randn((n_b, Hh, Dd, Dd), generator=g, device=dev) * 0.1
+    cs_b = torch.randn((n_b, cd, 3), generator=g, device=dev).to(torch.bfloat16)
+    ph1, pc1 = kda.ptr_array([hs_b[0]], device=dev), kda.ptr_array([cs_b[0]], device=dev)
+    phn, pcn = kda.ptr_array(list(hs_b), device=dev), kda.ptr_array(list(cs_b), device=dev)
+    ms1 = timed(lambda: kda.kda_block_decode(st, hid[:1], 1, ph1, pc1, ws, s))
+    msk = timed(lambda: kda.kda_block_decode_k(st, hid[:4], 4, hs_b[1], cs_b[1], [], [], ws, s))
+    msn = timed(lambda: kda.kda_block_decode(st, hid[:n_b], n_b, phn, pcn, ws, s))
+    dec = {"one_token": {"ms": ms1, "tokens_per_s": 1 / (ms1 * 1e-3),
+                         "gbs": (wbytes + sbytes) / (ms1 * 1e-3) / 1e9,
+                         "frac_hbm": (wbytes + sbytes) / (ms1 * 1e-3) / 1e9 / hbm},
+           "decode_k4": {"ms": msk, "tokens_per_s": 4 / (msk * 1e-3),
+                         "gbs": (wbytes + sbytes) / (msk * 1e-3) / 1e9},
+           "batch256": {"ms": msn, "tokens_per_s": n_b / (msn * 1e-3),
+                        "gbs": (wbytes + n_b * sbytes) / (msn * 1e-3) / 1e9,
+                        "frac_hbm": (wbytes + n_b * sbytes) / (msn * 1e-3) / 1e9 / hbm},
+           "weights_bytes": wbytes, "state_bytes_per_seq": sbytes}
+    del hs_b, cs_b
     ws.close()
     return {"workload": "kda_block_prefill hidden 4096 H32 D128 rank 128 T8192 (9 GEMMs + conv + gate + core + o_norm)",
             "ms": ms, "tokens_per_s": Tb / (ms * 1e-3), "proj_flops": flops,
             "tflops_all": flops / (ms * 1e-3) / 1e12,
             "gemm": {"shape": "8192x4096x4096 bf16->bf16", "ms": gms, "tflops": gflop / (gms * 1e-3) / 1e12,
-                     "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak}}
+                     "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak},
+            "block_decode": dec}
 
 
 def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):

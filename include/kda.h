@@ -276,6 +276,16 @@ KDA_API int kda_back_gated_rmsnorm(const float *core, const kda_bf16 *out_gate, 
 KDA_API int kda_gemm_bf16(const kda_bf16 *A, int lda, const kda_bf16 *W, int ldw, void *C, int ldc, int M, int N,
                           int K, int out_f32, void *stream);
 
+/* kda_gemv_bf16 — y[m][n] = sum_k x[m][k] W[n][k] for a few rows (the decode / verify
+ * projections; the batched-M matrix-vector product of Glm5NextKdaLayer `decode_k`): W [N, K]
+ * BF16 (row stride ldw) is read once per group of 8 rows; FP32 accumulation; y BF16 (out_f32
+ * = 0) or F32, row stride ldy. Each output's arithmetic is fixed by K and its own row (lane-
+ * strided 8-element steps, then a fixed 32-lane butterfly), so a row gives the same bits
+ * whatever M is. K % 8 == 0, K <= 8192 (else KDA_ERR_UNSUPPORTED); x, W 16-byte aligned with
+ * ldx, ldw multiples of 8 (else KDA_ERR_MISALIGNED). */
+KDA_API int kda_gemv_bf16(const kda_bf16 *x, int ldx, const kda_bf16 *W, int ldw, void *y, int ldy, int M, int N,
+                          int K, int out_f32, void *stream);
+
 /* ---------------------------------------------------------------------------------
  * Block prefill: one KDA block over T tokens of one sequence (Glm5NextKdaLayer `prefill` /
  * `prefill_with_pad_fill`), stage by stage into a workspace (Glm5NextKdaWorkspace) that is

@@ -79,6 +79,7 @@ _SIGS = {
     "kda_workspace_buffer": ([_VP, _I, ctypes.POINTER(_VP), ctypes.POINTER(ctypes.c_size_t)], _I),
     "kda_block_prefill": ([_VP, _VP, _I, _VP, _VP, _F, _VP, _VP], _I),
     "kda_block_decode": ([_VP, _VP, _I, _VP, _VP, _VP, _VP], _I),
+    "kda_gemv_bf16": ([_VP, _I, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP], _I),
     "kda_block_decode_k": ([_VP, _VP, _I, _VP, _VP, _VP, _VP, _I, _VP, _VP], _I),
 }
 
@@ -328,3 +329,10 @@ def kda_block_decode_k(weights: KdaBlockWeights, hidden, K: int, h_state, conv_s
     return _call("kda_block_decode_k", ctypes.byref(weights), _p(hidden), K, _p(h_state), _p(conv_state),
                  ctypes.cast(hs, _VP) if hs is not None else None, ctypes.cast(cs, _VP) if cs is not None else None,
                  n, ws.handle, _stream(stream))
+
+
+def kda_gemv_bf16(x, W, y, M: int, N: int, K: int, ldx=None, ldw=None, ldy=None, stream=None):
+    """y[M, N] = x[M, K] . W[N, K]^T for a few rows (BF16 in; y's dtype picks BF16 or FP32)."""
+    import torch
+    return _call("kda_gemv_bf16", _p(x), ldx or K, _p(W), ldw or K, _p(y), ldy or N, M, N, K,
+                 1 if y.dtype == torch.float32 else 0, _stream(stream))

@@ -100,3 +100,23 @@ int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const flo
                            const float *beta, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
                            void *scratch, cudaStream_t s);
 }  // namespace kda
+
+namespace kda {
+// Projection GEMM and the batched-M matrix-vector products (kda_gemm.cu). Up to three weights
+// that read the same rows (q, k and v of one hidden row, say) go in one matrix-vector launch:
+// the column index runs over the concatenated outputs.
+struct GemvSeg {
+    const uint16_t *W;
+    void *y;
+    int N, ldw, ldy, out_f32;
+};
+struct GemvSegs {
+    GemvSeg s[3];
+    int count, total;
+};
+int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
+              int out_f32, cudaStream_t s);
+int gemv_bf16(const uint16_t *x, int ldx, const uint16_t *W, int ldw, void *y, int ldy, int M, int N, int K,
+              int out_f32, cudaStream_t s);
+int gemv_segs(const uint16_t *x, int ldx, const GemvSegs &segs, int M, int K, cudaStream_t s);
+}  // namespace kda

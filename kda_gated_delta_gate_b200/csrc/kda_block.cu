@@ -13,11 +13,11 @@
 // Block decode (Glm5NextKdaLayer `decode`, `decode_k`): the same projections for the call's
 // rows (N sequences x 1 token, or K rows of one sequence), each weight read once for all
 // rows, then the fused stateful rows (kda_decode_fused / kda_decode_k: conv + SiLU + L2, gate,
-// beta, recurrence, gated RMSNorm) and o_proj. Every projection runs the tcgen05 GEMM with the
-// call's rows inside 128-row tiles and the column-tile width fixed by the weight's output
-// size, so each row's dot products take the same K-step order in the same tile shapes
-// whatever the number of rows: a row's projections are bit-identical in a call of K rows and
-// in a call of one (the batched-M matrix-vector product the decode_k identity needs).
+// beta, recurrence, gated RMSNorm) and o_proj. Up to kRowsGemv rows the projections run the
+// batched-M matrix-vector kernel (kda_gemv_bf16), whose every output's arithmetic is fixed
+// by K and its own row: a row's projections are the same bits in a call of K rows and in a
+// call of one, which the decode_k identity needs. Larger batches (N independent sequences,
+// no such identity) run the tcgen05 GEMM.
 #include <cstring>
 #include <new>
 
@@ -29,8 +29,6 @@ namespace {
 // argument, so no host synchronisation is involved).
 __global__ void store_ptr_kernel(float **slot, float *p) { *slot = p; }
 }  // namespace
-int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
-              int out_f32, cudaStream_t s);
 }
 
 struct kda_workspace {
@@ -44,13 +42,42 @@ struct kda_workspace {
 
 namespace kda {
 namespace {
+constexpr int kRowsGemv = 32;
+
+// One projection of M decode rows: the batched-M matrix-vector kernel for up to kRowsGemv rows,
+// the tensor-core GEMM beyond.
+int proj(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *C, int ldc, int M, int N, int K, int out_f32,
+         cudaStream_t s) {
+    if (M <= kRowsGemv) return gemv_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
+    return gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
+}
+
 // Projections of M rows of `hidden` into the workspace: qkv_proj (q|k|v packed), g_raw,
-// b_logit (FP32, in the BETA buffer), out_gate.
+// b_logit (FP32, in the BETA buffer), out_gate. For the matrix-vector path the weights that
+// read the same rows share a launch: [q | k | v], [f_a | g_a | b_proj], then f_b and g_b.
 int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M, kda_workspace *ws, cudaStream_t s) {
     const kda_dims *d = &ws->dims;
     const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
     auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    if (M <= kRowsGemv) {
+        GemvSegs a{};
+        a.s[0] = GemvSeg{w->q_proj, bf(KDA_BUF_QKV_PROJ), qkv, Hd, cd, 0};
+        a.s[1] = GemvSeg{w->k_proj, bf(KDA_BUF_QKV_PROJ) + qkv, qkv, Hd, cd, 0};
+        a.s[2] = GemvSeg{w->v_proj, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, qkv, Hd, cd, 0};
+        a.count = 3;
+        a.total = 3 * qkv;
+        KDA_TRY(gemv_segs(hidden, Hd, a, M, Hd, s));
+        GemvSegs b{};
+        b.s[0] = GemvSeg{w->f_a, bf(KDA_BUF_F_A_OUT), R, Hd, R, 0};
+        b.s[1] = GemvSeg{w->g_a, bf(KDA_BUF_G_A_OUT), R, Hd, R, 0};
+        b.s[2] = GemvSeg{w->b_proj, f32(KDA_BUF_BETA), H, Hd, H, 1};
+        b.count = 3;
+        b.total = 2 * R + H;
+        KDA_TRY(gemv_segs(hidden, Hd, b, M, Hd, s));
+        KDA_TRY(gemv_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, M, qkv, R, 0, s));
+        return gemv_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, M, qkv, R, 0, s);
+    }
     KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, M, qkv, Hd, 0, s));
     KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, M, qkv, Hd, 0, s));
     KDA_TRY(gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, M, qkv, Hd, 0, s));
@@ -58,8 +85,7 @@ int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M,
     KDA_TRY(gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, M, qkv, R, 0, s));
     KDA_TRY(gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, M, H, Hd, 1, s));
     KDA_TRY(gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, M, R, Hd, 0, s));
-    KDA_TRY(gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, M, qkv, R, 0, s));
-    return KDA_OK;
+    return gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, M, qkv, R, 0, s);
 }
 
 int check_block_args(const kda_block_weights *w, const kda_bf16 *hidden, const kda_workspace *ws) {
@@ -197,8 +223,8 @@ int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, 
     KDA_TRY(kda_decode_fused(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                              f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                              bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), N, d, stream));
-    return kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, N, ws->hidden,
-                          qkv, 0, s);
+    return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, N, ws->hidden, qkv,
+                     0, s);
 }
 
 int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K, float *h_state,
@@ -217,8 +243,8 @@ int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K
     KDA_TRY(kda_decode_k(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                          f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                          bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), K, h_snap, conv_snap, n_snap, d, stream));
-    return kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, K, ws->hidden,
-                          qkv, 0, s);
+    return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, K, ws->hidden, qkv,
+                     0, s);
 }
 
 }  // extern "C"

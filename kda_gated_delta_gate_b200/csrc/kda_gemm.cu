@@ -240,6 +240,98 @@ int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout
     return launch_gemm<32>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
 }
 
+// ------------------------------------------------------------------ small-M matrix-vector products
+//
+// y[m][n] = sum_k x[m][k] W[n][k] for the M rows of a decode or verify step, W read once for
+// (up to) kGemvRows rows at a time. The warp that owns column n gives lane l the k in
+// {256 j + 8 l + e} (j, then e = 0..7 ascending, FP32 fma), then sums the 32 lanes by a fixed
+// butterfly: every output's arithmetic depends on K and its own row only, never on M, so a
+// row's result is the same bits in a call of one row and in a call of many (the identity the
+// K-token verify needs). x rows are staged in shared memory; W streams with 16-byte loads.
+constexpr int kGemvRows = 8, kGemvWarps = 8, kGemvMaxK = 8192;
+
+namespace {
+template <int MB>
+__global__ void __launch_bounds__(32 * kGemvWarps)
+gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M, int K) {
+    extern __shared__ __align__(16) uint16_t sx[];  // [mb][K]: this group's rows only
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int m0 = blockIdx.y * MB;
+    const int mb = min(MB, M - m0);
+    for (int e = tid; e < mb * (K / 8); e += 32 * kGemvWarps) {
+        const int r = e / (K / 8), c = 8 * (e % (K / 8));
+        *reinterpret_cast<uint4 *>(sx + r * K + c) = *reinterpret_cast<const uint4 *>(x + static_cast<size_t>(m0 + r) * ldx + c);
+    }
+    __syncthreads();
+    for (int col = blockIdx.x * kGemvWarps + warp; col < segs.total; col += gridDim.x * kGemvWarps) {
+        int si = 0, n = col;
+        while (si + 1 < segs.count && n >= segs.s[si].N) { n -= segs.s[si].N; ++si; }
+        const GemvSeg &sg = segs.s[si];
+        const uint16_t *wr = sg.W + static_cast<size_t>(n) * sg.ldw;
+        float acc[MB];
+#pragma unroll
+        for (int r = 0; r < MB; ++r) acc[r] = 0.f;
+#pragma unroll 4
+        for (int k = 8 * lane; k < K; k += 256) {
+            const uint4 wv = __ldcs(reinterpret_cast<const uint4 *>(wr + k));
+            float w8[8];
+            w8[0] = __uint_as_float(wv.x << 16); w8[1] = __uint_as_float(wv.x & 0xFFFF0000u);
+            w8[2] = __uint_as_float(wv.y << 16); w8[3] = __uint_as_float(wv.y & 0xFFFF0000u);
+            w8[4] = __uint_as_float(wv.z << 16); w8[5] = __uint_as_float(wv.z & 0xFFFF0000u);
+            w8[6] = __uint_as_float(wv.w << 16); w8[7] = __uint_as_float(wv.w & 0xFFFF0000u);
+#pragma unroll
+            for (int r = 0; r < MB; ++r) {
+                if (r < mb) {
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(sx + r * K + k);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.x << 16), w8[0], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.x & 0xFFFF0000u), w8[1], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.y << 16), w8[2], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.y & 0xFFFF0000u), w8[3], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.z << 16), w8[4], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.z & 0xFFFF0000u), w8[5], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.w << 16), w8[6], acc[r]);
+                    acc[r] = __fmaf_rn(__uint_as_float(xv.w & 0xFFFF0000u), w8[7], acc[r]);
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < MB; ++r) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[r] = __fadd_rn(acc[r], __shfl_xor_sync(0xffffffffu, acc[r], o));
+        }
+        if (lane < mb) {
+            float v = acc[0];
+#pragma unroll
+            for (int r = 1; r < MB; ++r)
+                if (lane == r) v = acc[r];
+            const size_t o = static_cast<size_t>(m0 + lane) * sg.ldy + n;
+            if (sg.out_f32) static_cast<float *>(sg.y)[o] = v;
+            else static_cast<uint16_t *>(sg.y)[o] = f32_to_bf16(v);
+        }
+    }
+}
+}  // namespace
+
+int gemv_segs(const uint16_t *x, int ldx, const GemvSegs &segs, int M, int K, cudaStream_t s) {
+    const int bytes = std::min(M, kGemvRows) * K * 2;  // the rows of one group
+    static std::atomic<unsigned long long> attr_done{0};  // opted in once, at the largest K
+    KDA_TRY(smem_opt_in(gemv_kernel<kGemvRows>, kGemvRows * kGemvMaxK * 2, attr_done));
+    const int col_blocks = (segs.total + kGemvWarps - 1) / kGemvWarps;
+    const int grid_x = std::min(col_blocks, 4 * sm_count());
+    gemv_kernel<kGemvRows><<<dim3(grid_x, (M + kGemvRows - 1) / kGemvRows), 32 * kGemvWarps, bytes, s>>>(x, ldx, segs,
+                                                                                                      M, K);
+    return launch_status();
+}
+
+int gemv_bf16(const uint16_t *x, int ldx, const uint16_t *W, int ldw, void *y, int ldy, int M, int N, int K,
+              int out_f32, cudaStream_t s) {
+    GemvSegs segs{};
+    segs.s[0] = GemvSeg{W, y, N, ldw, ldy, out_f32};
+    segs.count = 1;
+    segs.total = N;
+    return gemv_segs(x, ldx, segs, M, K, s);
+}
+
 }  // namespace kda
 
 extern "C" int kda_gemm_bf16(const kda_bf16 *A, int lda, const kda_bf16 *W, int ldw, void *C, int ldc, int M, int N,
@@ -250,4 +342,14 @@ extern "C" int kda_gemm_bf16(const kda_bf16 *A, int lda, const kda_bf16 *W, int 
     if (lda < K || ldw < K || ldc < N) return KDA_ERR_INVALID_ARG;
     if (!kda::aligned16(A) || !kda::aligned16(W) || (lda % 8) || (ldw % 8)) return KDA_ERR_MISALIGNED;
     return kda::gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int kda_gemv_bf16(const kda_bf16 *x, int ldx, const kda_bf16 *W, int ldw, void *y, int ldy, int M, int N,
+                             int K, int out_f32, void *stream) {
+    if (!x || !W || !y || M < 0 || N < 0 || K < 0) return KDA_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return KDA_OK;
+    if (K == 0 || K % 8 != 0 || K > kda::kGemvMaxK) return KDA_ERR_UNSUPPORTED;
+    if (ldx < K || ldw < K || ldy < N) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(x) || !kda::aligned16(W) || (ldx % 8) || (ldw % 8)) return KDA_ERR_MISALIGNED;
+    return kda::gemv_bf16(x, ldx, W, ldw, y, ldy, M, N, K, out_f32, static_cast<cudaStream_t>(stream));
 }

@@ -100,3 +100,26 @@ def test_block_decode_argument_checks():
     with pytest.raises(kda.KdaError):  # K > 32
         kda.kda_block_decode_k(st, h, 33, hs, cs, [], [], ws)
     ws.close()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (5, 4096, 128), (13, 96, 4096), (32, 32, 4096)])
+def test_gemv_matches_fp64_and_is_row_invariant(M, N, K):
+    """kda_gemv_bf16 against an FP64 product (FP32 output: accumulation error only; BF16 output:
+    one rounding), and every row's bits equal to a call with that row alone."""
+    g = torch.Generator().manual_seed(M * 7 + N)
+    x = torch.randn((M, K), generator=g).to(torch.bfloat16).cuda()
+    W = (torch.randn((N, K), generator=g) * 0.05).to(torch.bfloat16).cuda()
+    y32 = torch.empty((M, N), device="cuda")
+    y16 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    kda.kda_gemv_bf16(x, W, y32, M, N, K)
+    kda.kda_gemv_bf16(x, W, y16, M, N, K)
+    torch.cuda.synchronize()
+    ref = np64(x) @ np64(W).T
+    scale = np.abs(np64(x)) @ np.abs(np64(W)).T
+    assert np.all(np.abs(np64(y32) - ref) <= 1e-5 * scale + 1e-30)
+    assert np.all(np.abs(np64(y16) - np64(y32)) <= 2.0 ** -8 * np.abs(np64(y32)) + 1e-30)
+    for m in {0, M // 2, M - 1}:
+        one = torch.empty((1, N), device="cuda")
+        kda.kda_gemv_bf16(x[m:m + 1].contiguous(), W, one, 1, N, K)
+        torch.cuda.synchronize()
+        assert torch.equal(one[0], y32[m])
