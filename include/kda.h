@@ -129,6 +129,28 @@ KDA_API int kda_chunk_prefill(const float *q, const float *k, const float *v, co
 /* Scratch bytes kda_chunk_prefill needs for B streams of T tokens (0 if B or T is 0). */
 KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dims);
 
+/* kda_chunk_prefill_varlen — kda_chunk_prefill over B sequences of UNEQUAL lengths packed back
+ * to back (Glm5NextLayer varlen prefill: `cu_seqlens`, `max_num_chunks`): sequence b is rows
+ * [cu_seqlens[b], cu_seqlens[b+1]) of every token-major buffer, chunked from its own first
+ * row; the rows after a sequence's end (the next sequence's) never enter its chunks.
+ *   q, k, v, gate [total_tokens, H, D] F32;  beta [total_tokens, H] F32;  core likewise
+ *   cu_seqlens     DEVICE int32 [B + 1], cu_seqlens[0] = 0, non-decreasing, last = total_tokens
+ *   max_num_chunks at least ceil(len_b / 64) for every sequence (the scratch has that many
+ *                  chunk slots per sequence)
+ *   h_state        DEVICE array of B state pointers, read and overwritten (an empty sequence
+ *                  keeps its state)
+ *   scratch        at least kda_chunk_prefill_varlen_scratch_bytes(B, max_num_chunks, dims)
+ * A sequence whose bounds do not fit (negative, decreasing, past total_tokens, or longer than
+ * max_num_chunks * 64) is skipped, its state untouched, and KDA_ERR_INVALID_ARG is latched in
+ * kda_device_status. Each sequence's result equals kda_chunk_prefill on that sequence alone. */
+KDA_API int kda_chunk_prefill_varlen(const float *q, const float *k, const float *v, const float *gate,
+                                     const float *beta, const int *cu_seqlens, int B, int max_num_chunks,
+                                     int total_tokens, float *const *h_state, float *core, void *scratch,
+                                     size_t scratch_bytes, const kda_dims *dims, void *stream);
+
+/* Scratch bytes kda_chunk_prefill_varlen needs (0 if B or max_num_chunks is 0). */
+KDA_API size_t kda_chunk_prefill_varlen_scratch_bytes(int B, int max_num_chunks, const kda_dims *dims);
+
 /* kda_chunk_prefill_fused — kda_chunk_prefill reading the front end's BF16 output and the
  * raw gate directly (Glm5NextKdaWorkspace `conv_out` and `g_raw`: the fused-input mode, in
  * which the FP32 q/k/v/gate buffers are never written or read):

@@ -64,6 +64,8 @@ _SIGS = {
     "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_prefill_fused": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
+    "kda_chunk_prefill_varlen": ([_VP] * 6 + [_I, _I, _I, _VP, _VP, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
+    "kda_chunk_prefill_varlen_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_prefill_simt": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_chunk_prefill_noalloc": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_chunk_prefill_noalloc_max_scratch_bytes": ([], ctypes.c_size_t),
@@ -336,3 +338,15 @@ def kda_gemv_bf16(x, W, y, M: int, N: int, K: int, ldx=None, ldw=None, ldy=None,
     import torch
     return _call("kda_gemv_bf16", _p(x), ldx or K, _p(W), ldw or K, _p(y), ldy or N, M, N, K,
                  1 if y.dtype == torch.float32 else 0, _stream(stream))
+
+
+def kda_chunk_prefill_varlen(q, k, v, gate, beta, cu_seqlens, B: int, max_num_chunks: int, total_tokens: int,
+                             h_state_ptrs, core, d: KdaDims, stream=None, scratch=None):
+    """Chunked prefill over B packed sequences of unequal lengths (cu_seqlens: device int32 [B+1])."""
+    if scratch is None:
+        import torch
+        need = int(lib().kda_chunk_prefill_varlen_scratch_bytes(B, max_num_chunks, ctypes.byref(d)))
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+    return _call("kda_chunk_prefill_varlen", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(cu_seqlens), B,
+                 max_num_chunks, total_tokens, _p(h_state_ptrs), _p(core), _p(scratch),
+                 scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))

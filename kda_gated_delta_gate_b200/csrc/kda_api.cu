@@ -96,3 +96,30 @@ extern "C" int kda_chunk_prefill_fused(const kda_bf16 *qkv, const kda_bf16 *g_ra
     return kda::chunk_prefill_tc_fused(qkv, g_raw, dt_bias, a_log, beta, h_state, core, B, T, dims, scratch,
                                        static_cast<cudaStream_t>(stream));
 }
+
+extern "C" size_t kda_chunk_prefill_varlen_scratch_bytes(int B, int max_num_chunks, const kda_dims *dims) {
+    if (!dims || kda::check_dims(dims) != KDA_OK) return 0;
+    return kda::chunk_prefill_slots_scratch_bytes(B, max_num_chunks, dims->heads, dims->head_dim);
+}
+
+extern "C" int kda_chunk_prefill_varlen(const float *q, const float *k, const float *v, const float *gate,
+                                        const float *beta, const int *cu_seqlens, int B, int max_num_chunks,
+                                        int total_tokens, float *const *h_state, float *core, void *scratch,
+                                        size_t scratch_bytes, const kda_dims *dims, void *stream) {
+    KDA_TRY(kda::check_dims(dims));
+    if (!q || !k || !v || !gate || !beta || !cu_seqlens || !h_state || !core || B < 0 || max_num_chunks < 0 ||
+        total_tokens < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(q) || !kda::aligned16(k) || !kda::aligned16(v) || !kda::aligned16(gate) ||
+        !kda::aligned16(core))
+        return KDA_ERR_MISALIGNED;
+    if (B > 65535 || dims->heads > 65535) return KDA_ERR_UNSUPPORTED;
+    if (B == 0 || total_tokens == 0) return KDA_OK;  // every stream is empty: the states stay as they are
+    if (max_num_chunks == 0) return KDA_ERR_INVALID_ARG;
+    if (!scratch) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(scratch)) return KDA_ERR_MISALIGNED;
+    if (scratch_bytes < kda::chunk_prefill_slots_scratch_bytes(B, max_num_chunks, dims->heads, dims->head_dim))
+        return KDA_ERR_CAPACITY;
+    return kda::chunk_prefill_tc_varlen(q, k, v, gate, beta, cu_seqlens, B, max_num_chunks, total_tokens, h_state,
+                                        core, dims, scratch, static_cast<cudaStream_t>(stream));
+}

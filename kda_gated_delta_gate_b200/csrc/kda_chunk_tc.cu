@@ -120,6 +120,38 @@ __device__ __forceinline__ float4 load4_in(const PrefillIn &in, int part, size_t
     }
 }
 
+// Where the chunks of stream b live. Equal-length mode (cu == nullptr): B streams of T tokens
+// at a stride of T_pad rows (Glm5NextLayer `prefill_gdn_full_batched`). Varlen mode: stream b
+// is rows [cu[b], cu[b+1]) of the packed buffers (`cu_seqlens`, with `max_num_chunks` chunk
+// slots per stream); the rows after a stream's end belong to the next stream, and the chunk
+// guard keeps them out exactly as it keeps out the padding of equal-length streams.
+struct Seqs {
+    const int *cu;  // device [B + 1], or nullptr
+    int T, T_pad;   // equal-length mode
+    int nch;        // chunk slots per stream: T_pad / C, or max_num_chunks
+    int total;      // varlen mode: rows of the packed buffers
+};
+
+// Rows of chunk c of stream b: first row (row0) and count (n). False for an empty slot or (in
+// varlen mode) a stream whose bounds are not inside the buffers, which also latches
+// KDA_ERR_INVALID_ARG: nothing is addressed from a bad cu_seqlens entry.
+__device__ __forceinline__ bool seq_chunk(const Seqs &sq, int b, int c, size_t &row0, int &n, int *status) {
+    if (!sq.cu) {
+        row0 = static_cast<size_t>(b) * sq.T_pad + static_cast<size_t>(c) * C;
+        n = min(C, sq.T - c * C);
+        return n > 0;
+    }
+    const int s0 = sq.cu[b], s1 = sq.cu[b + 1];
+    if (s0 < 0 || s1 < s0 || s1 > sq.total || s1 - s0 > sq.nch * C) {
+        if (status) atomicExch(status, KDA_ERR_INVALID_ARG);
+        n = 0;
+        return false;
+    }
+    row0 = static_cast<size_t>(s0) + static_cast<size_t>(c) * C;
+    n = min(C, s1 - s0 - c * C);
+    return n > 0;
+}
+
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 1.9 GHz
 
 // Split 8 FP32 values into BF16 hi and lo, packed as two 16-byte chunks (paired conversions).
@@ -229,7 +261,7 @@ struct Intra {
 // factor is a product of per-token factors <= 1, whatever g holds. It writes the whole operand
 // pack. Used for the chunks whose in-block decay is too strong for the tensor-core path.
 template <int D, bool FUSED>
-__device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__restrict__ scratch, int T, int T_pad,
+__device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__restrict__ scratch, const Seqs &sq,
                                                 int H, int b, int h, int ch, float *smem) {
     using I = Intra<D>;
     constexpr int P = I::P, PC = I::PC, NT = kIntraThreads;
@@ -245,8 +277,9 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
     float *sTmp = sB + C;          // [1024]
 
     const int tid = threadIdx.x;
-    const int n = min(C, T - ch * C);
-    const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
+    int n = 0;
+    size_t row0 = 0;
+    seq_chunk(sq, b, ch, row0, n, nullptr);  // listed chunks are non-empty and in bounds
 
     // ---- load k, q and a = e^g (pad guard: rows >= n are k = q = 0, a = 1)
     for (int e = tid; e < C * D / 4; e += NT) {
@@ -403,7 +436,7 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
     //      K o e^{Gamma_C - Gamma} = Z S_a (pack), with P_a / S_a the decay of all blocks before /
     //      after block a; 16-byte chunks of 8 channels. v replaces a = e^g in sA (pad rows 0).
     using PK = Pack<D>;
-    uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * (T_pad / C) + ch) * PK::bytes;
+    uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * sq.nch + ch) * PK::bytes;
     for (int e = tid; e < C * (D / 8); e += NT) {
         const int i = e / (D / 8), cb = 8 * (e % (D / 8)), a = i >> 4;
         float xq[8], xb[8];
@@ -490,15 +523,15 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
 // Only the chunks the tensor-core kernel listed (count and packed (b, h, ch) entries in scratch).
 template <int D, bool FUSED>
 __global__ void __launch_bounds__(kIntraThreads, 1)
-intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *__restrict__ list, int T, int T_pad,
+intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *__restrict__ list, const Seqs sq,
                  int H) {
     extern __shared__ float smem[];
     const int count = list[0];
-    const int nch = T_pad / C;
+    const int nch = sq.nch;
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
         const int id = list[1 + e];
         const int ch = id % nch, h = (id / nch) % H, b = id / (nch * H);
-        intra_simt_body<D, FUSED>(in, scratch, T, T_pad, H, b, h, ch, smem);
+        intra_simt_body<D, FUSED>(in, scratch, sq, H, b, h, ch, smem);
         __syncthreads();
     }
 }
@@ -558,7 +591,7 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 template <int D, bool FUSED>
 __global__ void __launch_bounds__(kIntraThreads, 1)
 intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmV, const PrefillIn in,
-                uint8_t *__restrict__ scratch, int *__restrict__ list, int B, int T, int T_pad, int H,
+                uint8_t *__restrict__ scratch, int *__restrict__ list, int B, const Seqs sq, int H,
                 int *__restrict__ status) {
     using I = IntraTC<D>;
     using PK = Pack<D>;
@@ -583,7 +616,7 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
     // reference tables, [entry][D]: 0..3 e^{Gamma_{m_a}}, 4..7 e^{Gamma_C - Gamma_{m_a}},
     // 8..13 e^{Gamma_{m_a} - Gamma_{m_b}} for (a,b) = (1,0),(2,0),(2,1),(3,0),(3,1),(3,2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nch = T_pad / C;
+    const int nch = sq.nch;
     const int total = B * H * nch;
     constexpr uint32_t kBox = C * D * (FUSED ? 2 : 4);  // one g (g_raw) or v box
     // g's box: FP32 g at the start of its space, or BF16 g_raw in the upper half (the gate is
@@ -610,10 +643,26 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
     //      shared memory (thread 0; the caller made the space free); v only into L2; beta into
     //      a register of threads < C
     float kk[UPT][8], qq[UPT][8], bnext = 0.f;
+    // this CTA's items are blockIdx.x + j gridDim.x; empty chunk slots (varlen) are skipped
+    auto next_item = [&](int it) {
+        size_t r0;
+        int nn;
+        for (; it < total; it += gridDim.x) {
+            const int c = it % nch, bb = it / (nch * H);
+            if (seq_chunk(sq, bb, c, r0, nn, (it % (nch * H)) < nch && c == 0 ? status : nullptr)) break;
+        }
+        return it;
+    };
+    // TMA coordinates of a chunk's rows: (stream, row in stream) on the 3-D map, or the packed row
+    auto box_yz = [&](int ch, int b, size_t row0, int &y, int &z) {
+        if (sq.cu) { y = static_cast<int>(row0); z = 0; }
+        else { y = ch * C; z = b; }
+    };
     auto fetch = [&](int it) {
         const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
-        const int n = min(C, T - ch * C);
-        const size_t row0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(ch) * C;
+        int n;
+        size_t row0;
+        seq_chunk(sq, b, ch, row0, n, nullptr);
 #pragma unroll
         for (int u = 0; u < UPT; ++u) {
             const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
@@ -633,22 +682,32 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
             }
         }
         if (tid == 0) {
+            int y, z;
+            box_yz(ch, b, row0, y, z);
             mbar_expect_tx(gbar, kBox);
-            tma_load_3d(gdst, &tmG, h * D, ch * C, b, gbar);
+            tma_load_3d(gdst, &tmG, h * D, y, z, gbar);
         }
         if (tid < C) bnext = tid < n ? in.beta[(row0 + tid) * H + h] : 0.f;
     };
     tc_fence_before();
     __syncthreads();  // barriers initialised
     tc_fence_after();
-    if (blockIdx.x < total) fetch(blockIdx.x);
+    const int first = next_item(blockIdx.x);
+    if (first < total) fetch(first);
     const uint32_t tmem = *tmem_slot;
     bool dead = false;  // a wait timed out: hand every remaining item to the CUDA-core body
     uint32_t iter = 0;  // items done by this CTA: the parity of the g and v boxes
 
+    int following = total;
 #pragma unroll 1
-    for (int item = blockIdx.x; item < total; item += gridDim.x, ++iter) {
+    for (int item = first; item < total; item = following, ++iter) {
         const int ch = item % nch, h = (item / nch) % H, b = item / (nch * H);
+        following = next_item(item + gridDim.x);
+        int n;
+        size_t row0;
+        seq_chunk(sq, b, ch, row0, n, nullptr);
+        int boxy, boxz;
+        box_yz(ch, b, row0, boxy, boxz);
         uint8_t *pack = scratch + static_cast<size_t>(item) * PK::bytes;
         if (dead) {  // block-uniform
             if (tid == 0) list[1 + atomicAdd(list, 1)] = item;
@@ -677,7 +736,6 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
             if constexpr (FUSED) {
                 // g = -exp(a_log) softplus(g_raw + dt_bias) (0 past T), FP32 over g_raw's box
                 const uint16_t *gr = reinterpret_cast<const uint16_t *>(gdst);
-                const int n = min(C, T - ch * C);
                 float x[TPQ];
 #pragma unroll
                 for (int r = 0; r < TPQ; ++r) x[r] = bf16_to_f32(gr[(qr * TPQ + r) * D + c]);
@@ -690,7 +748,10 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
                 }
             }
             float acc = 0.f;
-            for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) { acc += sG[i * GP + c]; sG[i * GP + c] = acc; }
+            for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) {
+                acc += i < n ? sG[i * GP + c] : 0.f;  // rows past the chunk's end decay nothing
+                sG[i * GP + c] = acc;
+            }
             sTmp[qr * D + c] = acc;
             __syncthreads();
             float pre = 0.f;
@@ -788,7 +849,7 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         //      D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127)
         if (tid == 0) {
             mbar_expect_tx(vbar, kBox);
-            tma_load_3d(sG, &tmV, vx0 + h * D, ch * C, b, vbar);
+            tma_load_3d(sG, &tmV, vx0 + h * D, boxy, boxz, vbar);
             if (safe) {
                 constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
                 const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
@@ -849,6 +910,10 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
                 } else {
                     ld8(sG + i * GP + cb, x);
                 }
+                if (i >= n) {  // rows past the chunk's end: v = 0
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) x[w] = 0.f;
+                }
                 st_pair(sA, I::A_BYTES / 2, mnmaj_off(cb, i, C), kk[u]);
                 st_pair(sA, I::A_BYTES / 2, mnmaj_off(D + cb, i, C), x);
             }
@@ -868,12 +933,12 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         if (!ok && tid == 0) mbar_wait(vbar, par, kWaitCycles);
         fence_async_smem();
         __syncthreads();
-        const bool more = item + static_cast<int>(gridDim.x) < total;
+        const bool more = following < total;
         bool done = false;
-        if (!run && more) fetch(item + gridDim.x);
+        if (!run && more) fetch(following);
         if (run) {
             invert_unit_lower64(sL, sT, sTmp);
-            if (more) fetch(item + gridDim.x);  // after the inverse: its shared-memory traffic runs alone
+            if (more) fetch(following);  // after the inverse: its shared-memory traffic runs alone
             // ---- Tb = T diag(beta) as the A operand (64 x 64 K-major, zero above the diagonal)
             {
                 const int r = tid >> 3, c0 = 8 * (tid & 7);
@@ -1013,8 +1078,8 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
 
 template <int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
-state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core, int T,
-             int T_pad, int H, float scale, int *__restrict__ status) {
+state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core,
+             const Seqs sq, int H, float scale, int *__restrict__ status) {
     using S = State<D, DVS>;
     using PK = Pack<D>;
     constexpr int HALF = DVS / 2;  // value columns per thread in the epilogues
@@ -1031,8 +1096,18 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int c0 = slice * DVS;
     const size_t rs = static_cast<size_t>(H) * D;
+    const int nch = sq.nch;  // chunk slots per stream in the scratch
+    int nb = nch;            // this stream's chunks
+    if (sq.cu) {
+        const int s0 = sq.cu[b], s1 = sq.cu[b + 1];
+        if (s0 < 0 || s1 < s0 || s1 > sq.total || s1 - s0 > nch * C) {  // a bad cu_seqlens entry
+            if (tid == 0 && slice == 0 && h == 0) atomicExch(status, KDA_ERR_INVALID_ARG);
+            return;
+        }
+        nb = (s1 - s0 + C - 1) / C;
+    }
+    if (nb == 0) return;  // an empty stream keeps its state
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
-    const int nch = T_pad / C;
     const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
     const size_t u_off = PK::OFF_UT + static_cast<size_t>(c0 / 32) * PK::UG_BYTES;
 
@@ -1103,8 +1178,10 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     // O = scale D1[64:128] of chunk c (quads 2 and 3: TMEM lanes 64..127 = the chunk's tokens),
     // run while the tensor core computes chunk c + 1
     auto out_epilogue = [&](int c) {
-        const int i = erow - 64, nn = min(C, T - c * C);
-        const size_t r0 = static_cast<size_t>(b) * T_pad + static_cast<size_t>(c) * C;
+        const int i = erow - 64;
+        int nn;
+        size_t r0;
+        seq_chunk(sq, b, c, r0, nn, nullptr);
         const uint32_t tD1c = tmem + (c & 1) * DVS;
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
@@ -1121,11 +1198,11 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     };
 
 #pragma unroll 1
-    for (int ch = 0; ch < nch; ++ch) {
+    for (int ch = 0; ch < nb; ++ch) {
         const uint32_t par = ch & 1;
         const uint32_t tD1 = tmem + par * DVS;
         const uint8_t *next = packs + static_cast<size_t>(ch + 1) * PK::bytes;
-        const bool more = ch + 1 < nch;
+        const bool more = ch + 1 < nb;
         // e^{Gamma_C} of this thread's key row, read early (used in epilogue 2)
         const float ac = srow >= 0 ? reinterpret_cast<const float *>(packs + static_cast<size_t>(ch) * PK::bytes +
                                                                     PK::OFF_AC)[srow]
@@ -1215,7 +1292,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         tc_fence_after();
         if (!ok) break;  // block-uniform: every thread saw the same flag
     }
-    if (ok && quad >= 2) out_epilogue(nch - 1);
+    if (ok && quad >= 2) out_epilogue(nb - 1);
     if (!ok) {
         if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
     } else if (srow >= 0) {
@@ -1235,10 +1312,9 @@ template <int D>
 size_t packs_bytes(int B, int H, int nch) { return static_cast<size_t>(B) * H * nch * Pack<D>::bytes; }
 
 template <int D, int DVS, bool FUSED>
-int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, int T, int H, float scale, void *scratch,
-              cudaStream_t s) {
-    const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C));
-    const int nch = T_pad / C;
+int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, int H, float scale,
+              void *scratch, cudaStream_t s) {
+    const int nch = sq.nch;
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
     static std::atomic<unsigned long long> attr_intra{0}, attr_fix{0}, attr_state{0};
@@ -1256,41 +1332,51 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, in
     }
     const long long items = static_cast<long long>(B) * H * nch;
     const int grid = static_cast<int>(std::min<long long>(items, sms));
+    // box maps: (stream, row in stream) for equal-length streams; the packed rows in varlen mode
+    const int mT = sq.cu ? sq.total : sq.T, mTp = sq.cu ? sq.total : sq.T_pad, mB = sq.cu ? 1 : B;
     CUtensorMap tmG, tmV;
     if (FUSED) {
-        KDA_TRY(make_rows_map(&tmG, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, T, T_pad, B, D, C));
-        KDA_TRY(make_rows_map(&tmV, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, T, T_pad, B, D, C));
+        KDA_TRY(make_rows_map(&tmG, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, mT, mTp, mB, D, C));
+        KDA_TRY(make_rows_map(&tmV, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, mT, mTp, mB, D, C));
     } else {
-        KDA_TRY(make_rows_map(&tmG, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, T, T_pad, B, D, C));
-        KDA_TRY(make_rows_map(&tmV, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, T, T_pad, B, D, C));
+        KDA_TRY(make_rows_map(&tmG, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
+        KDA_TRY(make_rows_map(&tmV, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
     }
-    intra_tc_kernel<D, FUSED><<<grid, kIntraThreads, IntraTC<D>::bytes, s>>>(tmG, tmV, in, sc, list, B, T, T_pad, H,
-                                                                             status);
+    intra_tc_kernel<D, FUSED><<<grid, kIntraThreads, IntraTC<D>::bytes, s>>>(tmG, tmV, in, sc, list, B, sq, H, status);
     KDA_TRY(launch_status());
-    intra_fix_kernel<D, FUSED><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, T, T_pad, H);
+    intra_fix_kernel<D, FUSED><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
-    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, T, T_pad, H,
-                                                                                   scale, status);
+    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
+                                                                                   status);
     return launch_status();
 }
 
 // Value slice width: enough CTAs to cover the SMs (one state CTA per SM fits in shared memory).
 template <bool FUSED>
-int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
+int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, const kda_dims *dims,
                void *scratch, cudaStream_t s) {
     const int H = dims->heads;
     const float sc = dims->scale;
-    if (dims->head_dim == 64) return launch_tc<64, 32, FUSED>(in, h_state, core, B, T, H, sc, scratch, s);
+    if (dims->head_dim == 64) return launch_tc<64, 32, FUSED>(in, h_state, core, B, sq, H, sc, scratch, s);
     const long long units = static_cast<long long>(B) * H;
-    if (units >= 60) return launch_tc<128, 64, FUSED>(in, h_state, core, B, T, H, sc, scratch, s);
-    return launch_tc<128, 32, FUSED>(in, h_state, core, B, T, H, sc, scratch, s);
+    if (units >= 60) return launch_tc<128, 64, FUSED>(in, h_state, core, B, sq, H, sc, scratch, s);
+    return launch_tc<128, 32, FUSED>(in, h_state, core, B, sq, H, sc, scratch, s);
+}
+
+Seqs equal_seqs(int T) {
+    const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C));
+    return Seqs{nullptr, T, T_pad, T_pad / C, 0};
 }
 
 }  // namespace
 
 size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D) {
     if (B <= 0 || T <= 0 || H <= 0) return 0;
-    const int nch = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C) / C);
+    return chunk_prefill_slots_scratch_bytes(B, static_cast<int>(kda_t_pad(static_cast<size_t>(T), C) / C), H, D);
+}
+
+size_t chunk_prefill_slots_scratch_bytes(int B, int nch, int H, int D) {
+    if (B <= 0 || nch <= 0 || H <= 0) return 0;
     const size_t packs = D == 64 ? packs_bytes<64>(B, H, nch) : packs_bytes<128>(B, H, nch);
     const size_t list = (4 + 4 * static_cast<size_t>(B) * H * nch + 255) / 256 * 256;
     return packs + list;
@@ -1300,14 +1386,21 @@ int chunk_prefill_tc(const float *q, const float *k, const float *v, const float
                      float *const *h_state, float *core, int B, int T, const kda_dims *dims, void *scratch,
                      cudaStream_t s) {
     const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta};
-    return launch_any<false>(in, h_state, core, B, T, dims, scratch, s);
+    return launch_any<false>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
+}
+
+int chunk_prefill_tc_varlen(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                            const int *cu_seqlens, int B, int max_chunks, int total, float *const *h_state,
+                            float *core, const kda_dims *dims, void *scratch, cudaStream_t s) {
+    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta};
+    return launch_any<false>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, max_chunks, total}, dims, scratch, s);
 }
 
 int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
                            const float *beta, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
                            void *scratch, cudaStream_t s) {
     const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta};
-    return launch_any<true>(in, h_state, core, B, T, dims, scratch, s);
+    return launch_any<true>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
 }
 
 }  // namespace kda

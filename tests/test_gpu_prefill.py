@@ -187,3 +187,68 @@ def test_fused_prefill_extreme_decay_takes_exact_path():
     ci.dt_bias[1 * 128 + 9] = 6.0
     core_f, S_f = _gpu_prefill_fused(ci)
     _check(ci, core_f, S_f)
+
+
+def _varlen_case(lens, H, D, seed):
+    """Packed sequences of the given lengths: q, k, v [total, H, D], gate and beta formed on the
+    GPU from the packed g_raw / b_logit, per-sequence initial states, cu_seqlens on the device."""
+    total = sum(lens)
+    ci = core_inputs(1, max(total, 1), H, D, seed=seed, bf16_inputs=True, s0_std=0.0)
+    g = torch.Generator().manual_seed(seed + 1)
+    s0 = torch.randn((len(lens), H, D, D), generator=g) * 0.1
+    d = kda.dims(H, D)
+    dev = dict(q=ci.q[0, :total].cuda().contiguous(), k=ci.k[0, :total].cuda().contiguous(),
+               v=ci.v[0, :total].cuda().contiguous())
+    gate = torch.empty((total, H, D), device="cuda")
+    kda.kda_gate(ci.g_raw[0, :total].cuda().contiguous(), ci.dt_bias.cuda(), ci.a_log.cuda(), gate, total, d)
+    beta = ci.b_logit[0, :total].cuda().contiguous()
+    kda.kda_beta(beta, beta, beta.numel())
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    return ci, s0, dev, gate, beta, cu, d
+
+
+@pytest.mark.parametrize("lens,H,D", [([100, 0, 257, 64, 1], 2, 64), ([300, 129, 7], 4, 128)])
+def test_varlen_prefill_matches_per_sequence_path_and_oracle(lens, H, D):
+    """kda_chunk_prefill_varlen on back-to-back sequences: each sequence's outputs and final state
+    are the bits kda_chunk_prefill gives on that sequence alone, and match the oracle; an empty
+    sequence keeps its state."""
+    from synth.inputs import CoreInputs
+    ci, s0, dev, gate, beta, cu, d = _varlen_case(lens, H, D, seed=60 + len(lens))
+    total, B = sum(lens), len(lens)
+    states = [s0[b].cuda().clone() for b in range(B)]
+    core = torch.full((total, H, D), float("nan"), device="cuda")
+    max_chunks = max((L + 63) // 64 for L in lens) + 1  # one spare slot per sequence
+    kda.kda_chunk_prefill_varlen(dev["q"], dev["k"], dev["v"], gate, beta, cu, B, max_chunks, total,
+                                 kda.ptr_array(states), core, d)
+    torch.cuda.synchronize()
+    start = 0
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert torch.equal(states[b], s0[b].cuda())
+            continue
+        sl = slice(start, start + L)
+        one = CoreInputs(1, L, H, D, ci.q[:, sl], ci.k[:, sl], ci.v[:, sl], ci.g_raw[:, sl], ci.dt_bias, ci.a_log,
+                         ci.b_logit[:, sl], s0[b:b + 1])
+        c1, S1, _ = gpu_prefill(one)
+        assert torch.equal(core[sl], c1[0]), b
+        assert torch.equal(states[b], S1[0]), b
+        _check(one, core[sl].unsqueeze(0), states[b].unsqueeze(0))
+        start += L
+
+
+def test_varlen_prefill_rejects_a_sequence_longer_than_its_slots():
+    """With max_num_chunks = 1 a 100-token sequence does not fit: it is skipped, its state left
+    as it was, and KDA_ERR_INVALID_ARG is latched; the 50-token sequence beside it is exact."""
+    from synth.inputs import CoreInputs
+    lens, H, D = [100, 50], 2, 64
+    ci, s0, dev, gate, beta, cu, d = _varlen_case(lens, H, D, seed=77)
+    states = [s0[b].cuda().clone() for b in range(2)]
+    core = torch.zeros((150, H, D), device="cuda")
+    kda.kda_chunk_prefill_varlen(dev["q"], dev["k"], dev["v"], gate, beta, cu, 2, 1, 150, kda.ptr_array(states), core,
+                                 d)
+    torch.cuda.synchronize()
+    assert kda.device_status(clear=True) == 1  # KDA_ERR_INVALID_ARG
+    assert torch.equal(states[0], s0[0].cuda())
+    one = CoreInputs(1, 50, H, D, ci.q[:, 100:], ci.k[:, 100:], ci.v[:, 100:], ci.g_raw[:, 100:], ci.dt_bias,
+                     ci.a_log, ci.b_logit[:, 100:], s0[1:2])
+    _check(one, core[100:].unsqueeze(0), states[1].unsqueeze(0))
