@@ -381,12 +381,18 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
 
 
 def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
+    """The same prefill through the public C ABI from pinned host buffers, every step copying its
+    inputs in and its outputs out. The inputs travel as the serving path holds them: the BF16
+    q|k|v rows (the front end's conv_out layout; the workload's inputs are BF16-exact), the BF16
+    g_raw and the FP32 beta logits; kda_beta + kda_chunk_prefill_fused compute the step."""
     from synth import pad_rows
-    host = {n: pad_rows(getattr(ci, n), Tp, 0.0).pin_memory() for n in ("q", "k", "v", "g_raw", "b_logit")}
-    host["s0"] = ci.s0[0].clone().pin_memory()
+    qkv = torch.cat([ci.q.reshape(B, T, H * D), ci.k.reshape(B, T, H * D), ci.v.reshape(B, T, H * D)], dim=-1)
+    host = {"qkv": pad_rows(qkv.to(torch.bfloat16), Tp, 0.0).pin_memory(),
+            "g_raw": pad_rows(ci.g_raw, Tp, 0.0).pin_memory(),
+            "b_logit": pad_rows(ci.b_logit, Tp, 0.0).pin_memory(),
+            "s0": ci.s0[0].clone().pin_memory()}
     dv = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
     dt_bias, a_log = ci.dt_bias.to(dev), ci.a_log.to(dev)
-    gate = torch.empty((B * Tp, H, D), device=dev)
     beta = torch.empty((B * Tp, H), device=dev)
     core = torch.empty((B * Tp, H, D), device=dev)
     core_h = torch.empty_like(core, device="cpu").pin_memory()
@@ -398,10 +404,9 @@ def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
     def one():
         for n, t in host.items():
             dv[n].copy_(t, non_blocking=True)
-        kda.kda_gate(dv["g_raw"], dt_bias, a_log, gate, B * T, d, s)
         kda.kda_beta(dv["b_logit"], beta, B * T * H, s)
-        kda.kda_chunk_prefill(dv["q"], dv["k"], dv["v"], gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl,
-                              scratch=scratch)
+        kda.kda_chunk_prefill_fused(dv["qkv"], dv["g_raw"], dt_bias, a_log, beta, ptrs, core, B, T, d, s,
+                                    scratch=scratch)
         core_h.copy_(core, non_blocking=True)
         s_h.copy_(dv["s0"], non_blocking=True)
 
@@ -422,7 +427,9 @@ def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = t.item()
     return {"value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "call": "kda_beta + kda_chunk_prefill_fused (BF16 q|k|v rows, BF16 g_raw, FP32 beta logits in; FP32 core "
+                    "and state out)"}
 
 
 if __name__ == "__main__":

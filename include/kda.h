@@ -325,7 +325,9 @@ typedef struct kda_block_weights {
     const kda_bf16 *g_a;                      /* [rank, hidden]                          */
     const kda_bf16 *g_b;                      /* [H*D, rank]                             */
     const kda_bf16 *o_norm;                   /* [D]                                     */
-    const kda_bf16 *o_proj;                   /* [hidden, H*D]                           */
+    const kda_bf16 *o_proj;                   /* [hidden, H*D], or NULL: the block calls stop
+                                                 after o_norm_out (a tensor-parallel caller
+                                                 applies its o_proj slice and the all-reduce) */
     int hidden, rank;
 } kda_block_weights;
 

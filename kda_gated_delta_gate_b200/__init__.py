@@ -244,7 +244,8 @@ def kda_gemm_bf16(A, W, C, M: int, N: int, K: int, *, lda=None, ldw=None, ldc=No
 
 
 def block_weights_struct(w) -> KdaBlockWeights:
-    """KdaBlockWeights from an object with device tensors q_proj, ..., o_proj and ints hidden, rank."""
+    """KdaBlockWeights from an object with device tensors q_proj, ..., o_proj and ints hidden, rank.
+    The struct holds raw pointers only: keep `w` (and its tensors) alive while calls use it."""
     return KdaBlockWeights(*[_p(getattr(w, n)) for n in ("q_proj", "k_proj", "v_proj", "conv", "f_a", "f_b",
                                                           "dt_bias", "a_log", "b_proj", "g_a", "g_b", "o_norm",
                                                           "o_proj")], w.hidden, w.rank)

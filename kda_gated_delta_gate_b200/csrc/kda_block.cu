@@ -92,7 +92,7 @@ int check_block_args(const kda_block_weights *w, const kda_bf16 *hidden, const k
     if (!w || !hidden || !ws) return KDA_ERR_INVALID_ARG;
     if (w->hidden != ws->hidden || w->rank != ws->rank) return KDA_ERR_INVALID_ARG;
     if (!w->q_proj || !w->k_proj || !w->v_proj || !w->conv || !w->f_a || !w->f_b || !w->dt_bias || !w->a_log ||
-        !w->b_proj || !w->g_a || !w->g_b || !w->o_norm || !w->o_proj)
+        !w->b_proj || !w->g_a || !w->g_b || !w->o_norm)
         return KDA_ERR_INVALID_ARG;
     return KDA_OK;
 }
@@ -203,7 +203,8 @@ int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T,
     KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0, s));
     KDA_TRY(kda_back_gated_rmsnorm(f32(KDA_BUF_CORE), bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT), T, d,
                                    stream));
-    KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), Hd, T, Hd, qkv, 0, s));
+    if (w->o_proj)  // NULL: the caller applies its own o_proj (a tensor-parallel slice)
+        KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), Hd, T, Hd, qkv, 0, s));
     (void)Tp;
     return KDA_OK;
 }
@@ -223,6 +224,7 @@ int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, 
     KDA_TRY(kda_decode_fused(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                              f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                              bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), N, d, stream));
+    if (!w->o_proj) return KDA_OK;  // the caller applies its own o_proj (a tensor-parallel slice)
     return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, N, ws->hidden, qkv,
                      0, s);
 }
@@ -243,6 +245,7 @@ int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K
     KDA_TRY(kda_decode_k(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                          f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                          bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), K, h_snap, conv_snap, n_snap, d, stream));
+    if (!w->o_proj) return KDA_OK;
     return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, K, ws->hidden, qkv,
                      0, s);
 }

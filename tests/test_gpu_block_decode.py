@@ -90,7 +90,8 @@ def test_block_decode_k_bit_identical_to_serial_block_decodes(hidden, H, D, rank
 
 def test_block_decode_argument_checks():
     Wt = block_weights(256, 2, 64, 64, seed=1, std=0.05)
-    st = kda.block_weights_struct(_device_weights(Wt))
+    dw = _device_weights(Wt)  # held: the struct keeps only raw pointers
+    st = kda.block_weights_struct(dw)
     ws = kda.Workspace(kda.dims(2, 64), 256, 64, max_tokens=4)
     hs = torch.zeros((2, 64, 64), device="cuda")
     cs = torch.zeros((384, 3), dtype=torch.bfloat16, device="cuda")
