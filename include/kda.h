@@ -151,6 +151,33 @@ KDA_API int kda_chunk_prefill_varlen(const float *q, const float *k, const float
 /* Scratch bytes kda_chunk_prefill_varlen needs (0 if B or max_num_chunks is 0). */
 KDA_API size_t kda_chunk_prefill_varlen_scratch_bytes(int B, int max_num_chunks, const kda_dims *dims);
 
+/* kda_chunk_verify — batched verify under the WY tables (Glm5NextLayer speculative verify):
+ * the draft rows of B sequences, packed as for kda_chunk_prefill_varlen, each sequence at most
+ * 64 rows (one chunk), go through the chunked kernels from each sequence's state, which is NOT
+ * updated. Outputs `core` for every row (the same bits kda_chunk_prefill_varlen gives), and
+ * keeps in `tables` (kda_chunk_verify_tables_bytes(B, dims) bytes, 16-byte aligned) per
+ * (sequence, head): the rows' update vectors U [64][D] and the in-chunk cumulative log-decay
+ * Gamma [64][D], both FP32, for kda_chunk_verify_fold. scratch as kda_chunk_prefill_varlen with
+ * max_num_chunks = 1. A sequence longer than 64 rows is skipped and latches
+ * KDA_ERR_INVALID_ARG. */
+KDA_API int kda_chunk_verify(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                             const int *cu_seqlens, int B, int total_tokens, float *const *h_state, float *core,
+                             float *tables, size_t tables_bytes, void *scratch, size_t scratch_bytes,
+                             const kda_dims *dims, void *stream);
+
+/* Bytes of the tables kda_chunk_verify keeps for B sequences (B * heads * 2 * 64 * D * 4). */
+KDA_API size_t kda_chunk_verify_tables_bytes(int B, const kda_dims *dims);
+
+/* kda_chunk_verify_fold — accepted-row folding: sequence b's state becomes the state after its
+ * first accepted[b] verified rows (DEVICE int32 [B], 0 <= accepted[b] <= its row count):
+ *   S_r = diag(e^{Gamma_{r-1}}) S + sum_{t<r} (k_t o e^{Gamma_{r-1} - Gamma_t}) u_t^T
+ * from the verify tables and the same k rows; accepted[b] = 0 leaves the state. Run after
+ * kda_chunk_verify on the same states, before anything else changes them. Bad bounds latch
+ * KDA_ERR_INVALID_ARG and leave that state. */
+KDA_API int kda_chunk_verify_fold(const float *k, const int *cu_seqlens, const int *accepted, int B,
+                                  int total_tokens, const float *tables, float *const *h_state,
+                                  const kda_dims *dims, void *stream);
+
 /* kda_chunk_prefill_fused — kda_chunk_prefill reading the front end's BF16 output and the
  * raw gate directly (Glm5NextKdaWorkspace `conv_out` and `g_raw`: the fused-input mode, in
  * which the FP32 q/k/v/gate buffers are never written or read):

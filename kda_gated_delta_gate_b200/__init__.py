@@ -66,6 +66,9 @@ _SIGS = {
     "kda_chunk_prefill_fused": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_varlen": ([_VP] * 6 + [_I, _I, _I, _VP, _VP, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_varlen_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
+    "kda_chunk_verify": ([_VP] * 6 + [_I, _I, _VP, _VP, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
+    "kda_chunk_verify_tables_bytes": ([_I, _DIMS], ctypes.c_size_t),
+    "kda_chunk_verify_fold": ([_VP, _VP, _VP, _I, _I, _VP, _VP, _DIMS, _VP], _I),
     "kda_chunk_prefill_simt": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_chunk_prefill_noalloc": ([_VP] * 7 + [_I, _I, _DIMS, _VP], _I),
     "kda_chunk_prefill_noalloc_max_scratch_bytes": ([], ctypes.c_size_t),
@@ -351,3 +354,26 @@ def kda_chunk_prefill_varlen(q, k, v, gate, beta, cu_seqlens, B: int, max_num_ch
     return _call("kda_chunk_prefill_varlen", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(cu_seqlens), B,
                  max_num_chunks, total_tokens, _p(h_state_ptrs), _p(core), _p(scratch),
                  scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+
+
+def kda_chunk_verify(q, k, v, gate, beta, cu_seqlens, B: int, total_tokens: int, h_state_ptrs, core, tables,
+                     d: KdaDims, stream=None, scratch=None):
+    """Batched verify: outputs for every draft row, states unchanged, tables kept for the fold."""
+    if scratch is None:
+        import torch
+        need = int(lib().kda_chunk_prefill_varlen_scratch_bytes(B, 1, ctypes.byref(d)))
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+    return _call("kda_chunk_verify", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(cu_seqlens), B, total_tokens,
+                 _p(h_state_ptrs), _p(core), _p(tables), tables.numel() * tables.element_size(), _p(scratch),
+                 scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+
+
+def kda_chunk_verify_tables_bytes(B: int, d: KdaDims) -> int:
+    return int(lib().kda_chunk_verify_tables_bytes(B, ctypes.byref(d)))
+
+
+def kda_chunk_verify_fold(k, cu_seqlens, accepted, B: int, total_tokens: int, tables, h_state_ptrs, d: KdaDims,
+                          stream=None):
+    """Advance every state by its accepted rows (device int32 [B]) from the verify tables."""
+    return _call("kda_chunk_verify_fold", _p(k), _p(cu_seqlens), _p(accepted), B, total_tokens, _p(tables),
+                 _p(h_state_ptrs), ctypes.byref(d), _stream(stream))

@@ -94,6 +94,9 @@ int chunk_prefill_simt(const float *q, const float *k, const float *v, const flo
                        float *const *h_state, float *core, int B, int T, const kda_dims *dims, cudaStream_t s);
 size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D);
 size_t chunk_prefill_slots_scratch_bytes(int B, int nch, int H, int D);  // B streams x nch chunk slots
+int chunk_verify_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                    const int *cu_seqlens, int B, int total, float *const *h_state, float *core, float *tables,
+                    const kda_dims *dims, void *scratch, cudaStream_t s);
 int chunk_prefill_tc_varlen(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                             const int *cu_seqlens, int B, int max_chunks, int total, float *const *h_state,
                             float *core, const kda_dims *dims, void *scratch, cudaStream_t s);

@@ -68,6 +68,7 @@ struct PrefillIn {
     const float *q, *k, *v, *gate;
     const uint16_t *qkv, *g_raw;
     const float *dt_bias, *a_log, *beta;
+    float *tables;  // verify mode: per (stream, head) U [64][D] then Gamma [64][D] (FP32); else null
 };
 
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t u, float &lo, float &hi) {
@@ -518,6 +519,17 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
             *reinterpret_cast<float4 *>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
         }
     }
+    if (in.tables && tid < D) {  // verify mode: Gamma (in-chunk cumulative log-decay) for the fold
+        float *gt = in.tables + ((static_cast<size_t>(b) * H + h) * 2 + 1) * C * D;
+        float acc = 0.f;
+        for (int i = 0; i < C; ++i) {
+            if (i < n) {
+                const float4 g4 = load4_in<D, FUSED>(in, 3, row0 + i, H, h, tid & ~3);
+                acc += (tid & 3) == 0 ? g4.x : ((tid & 3) == 1 ? g4.y : ((tid & 3) == 2 ? g4.z : g4.w));
+            }
+            gt[i * D + tid] = acc;
+        }
+    }
 }
 
 // Only the chunks the tensor-core kernel listed (count and packed (b, h, ch) entries in scratch).
@@ -758,6 +770,10 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
             for (int r = 0; r < qr; ++r) pre += sTmp[r * D + c];
             if (qr > 0)
                 for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * GP + c] += pre;
+            if (in.tables) {  // verify mode: keep Gamma for the fold
+                float *gt = in.tables + ((static_cast<size_t>(b) * H + h) * 2 + 1) * C * D;
+                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) gt[i * D + c] = sG[i * GP + c];
+            }
             __syncthreads();
         }
         if (tid < D) {
@@ -1079,7 +1095,7 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
 template <int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
 state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core,
-             const Seqs sq, int H, float scale, int *__restrict__ status) {
+             const Seqs sq, int H, float scale, float *__restrict__ tables, int *__restrict__ status) {
     using S = State<D, DVS>;
     using PK = Pack<D>;
     constexpr int HALF = DVS / 2;  // value columns per thread in the epilogues
@@ -1240,6 +1256,11 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 const float4 u1 = *reinterpret_cast<const float4 *>(ur + 4);
                 x[0] = u0.x - x[0]; x[1] = u0.y - x[1]; x[2] = u0.z - x[2]; x[3] = u0.w - x[3];
                 x[4] = u1.x - x[4]; x[5] = u1.y - x[5]; x[6] = u1.z - x[6]; x[7] = u1.w - x[7];
+                if (tables) {  // verify mode: U of every row, for the fold
+                    float *ut = tables + (static_cast<size_t>(b) * H + h) * 2 * C * D + erow * D + c0 + c;
+                    *reinterpret_cast<float4 *>(ut) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4 *>(ut + 4) = make_float4(x[4], x[5], x[6], x[7]);
+                }
                 st_pair(sB2, S::B2 / 2, mnmaj_off(c, erow, C), x);
             }
         }
@@ -1295,7 +1316,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     if (ok && quad >= 2) out_epilogue(nb - 1);
     if (!ok) {
         if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
-    } else if (srow >= 0) {
+    } else if (srow >= 0 && !tables) {  // verify mode leaves the state as it was
 #pragma unroll
         for (int j = 0; j < HALF; j += 4)
             *reinterpret_cast<float4 *>(Sg + static_cast<size_t>(srow) * D + c0 + ccol + j) =
@@ -1347,7 +1368,7 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     intra_fix_kernel<D, FUSED><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
     state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
-                                                                                   status);
+                                                                                   in.tables, status);
     return launch_status();
 }
 
@@ -1385,21 +1406,28 @@ size_t chunk_prefill_slots_scratch_bytes(int B, int nch, int H, int D) {
 int chunk_prefill_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                      float *const *h_state, float *core, int B, int T, const kda_dims *dims, void *scratch,
                      cudaStream_t s) {
-    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta};
+    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, nullptr};
     return launch_any<false>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
 }
 
 int chunk_prefill_tc_varlen(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                             const int *cu_seqlens, int B, int max_chunks, int total, float *const *h_state,
                             float *core, const kda_dims *dims, void *scratch, cudaStream_t s) {
-    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta};
+    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, nullptr};
     return launch_any<false>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, max_chunks, total}, dims, scratch, s);
+}
+
+int chunk_verify_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
+                    const int *cu_seqlens, int B, int total, float *const *h_state, float *core, float *tables,
+                    const kda_dims *dims, void *scratch, cudaStream_t s) {
+    const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, tables};
+    return launch_any<false>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, 1, total}, dims, scratch, s);
 }
 
 int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
                            const float *beta, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
                            void *scratch, cudaStream_t s) {
-    const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta};
+    const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta, nullptr};
     return launch_any<true>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
 }
 

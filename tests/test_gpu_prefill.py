@@ -252,3 +252,45 @@ def test_varlen_prefill_rejects_a_sequence_longer_than_its_slots():
     one = CoreInputs(1, 50, H, D, ci.q[:, 100:], ci.k[:, 100:], ci.v[:, 100:], ci.g_raw[:, 100:], ci.dt_bias,
                      ci.a_log, ci.b_logit[:, 100:], s0[1:2])
     _check(one, core[100:].unsqueeze(0), states[1].unsqueeze(0))
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_verify_then_fold_accepted_rows(D):
+    """Batched verify under the WY tables: every draft row's output equals the varlen prefill's
+    (bit for bit) while the states stay; folding accepted[b] rows gives the state the prefill of
+    exactly those rows gives (and the oracle's); accepted = 0 leaves the state."""
+    from synth.inputs import CoreInputs
+    lens, H = [5, 64, 1, 17], 4
+    accepted = [3, 64, 0, 17]
+    ci, s0, dev, gate, beta, cu, d = _varlen_case(lens, H, D, seed=90 + D)
+    total, B = sum(lens), len(lens)
+    states = [s0[b].cuda().clone() for b in range(B)]
+    core = torch.full((total, H, D), float("nan"), device="cuda")
+    tables = torch.empty(kda.kda_chunk_verify_tables_bytes(B, d) // 4, device="cuda")
+    ptrs = kda.ptr_array(states)
+    kda.kda_chunk_verify(dev["q"], dev["k"], dev["v"], gate, beta, cu, B, total, ptrs, core, tables, d)
+    torch.cuda.synchronize()
+    for b in range(B):
+        assert torch.equal(states[b], s0[b].cuda())
+    fresh = [s0[b].cuda().clone() for b in range(B)]
+    core_p = torch.full((total, H, D), float("nan"), device="cuda")
+    kda.kda_chunk_prefill_varlen(dev["q"], dev["k"], dev["v"], gate, beta, cu, B, 1, total, kda.ptr_array(fresh),
+                                 core_p, d)
+    torch.cuda.synchronize()
+    assert torch.equal(core, core_p)
+    acc = torch.tensor(accepted, dtype=torch.int32, device="cuda")
+    kda.kda_chunk_verify_fold(dev["k"], cu, acc, B, total, tables, ptrs, d)
+    torch.cuda.synchronize()
+    start = 0
+    for b, (L, r) in enumerate(zip(lens, accepted)):
+        if r == 0:
+            assert torch.equal(states[b], s0[b].cuda())
+        else:
+            sl = slice(start, start + r)
+            one = CoreInputs(1, r, H, D, ci.q[:, sl], ci.k[:, sl], ci.v[:, sl], ci.g_raw[:, sl], ci.dt_bias,
+                             ci.a_log, ci.b_logit[:, sl], s0[b:b + 1])
+            _, S1, _ = gpu_prefill(one)
+            assert rel_l2(np64(states[b]), np64(S1[0])) <= 1e-5, b
+            o_ref, S_ref = oracle_prefill(one)
+            assert rel_l2(np64(states[b]), S_ref[0]) <= TOL, b
+        start += L
