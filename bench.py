@@ -4,8 +4,11 @@
 Workload (one step = one pass of the prefill hot path over one batch): B=1 sequence of
 T=4096 tokens, H=32 heads, head_dim 128, 64-token chunks, BF16-exact inputs widened to
 FP32, initial state N(0, 0.1): kda_gate (g_raw -> gate), kda_beta (b_logit -> beta) and
-kda_chunk_prefill (q, k, v, gate, beta, state -> core, state). Inputs are resident in
-HBM; L2 is flushed (a 512 MB write) before every timed step, outside the timed events.
+kda_chunk_prefill (q, k, v, gate, beta, state -> core, state). `--prefill-impl graw` runs
+kda_beta + kda_chunk_prefill_graw instead (the gate formed inside the chunked kernels from
+BF16 g_raw), `simt` the CUDA-core prefill.
+Inputs are resident in HBM; L2 is flushed (a 512 MB write) before every timed step,
+outside the timed events.
 Multi-GPU: each rank runs its own independent sequence (weak scaling, no collective).
 
 Also reported: the dominant kernel's roofline (CUDA events around each launch), a decode
@@ -33,8 +36,11 @@ B, T, H, D = 1, 4096, 32, 128
 CONFIG = {"workload": "kda_chunk_prefill B1 T4096 H32 D128 chunk64 (gate+beta+chunked core), FP32 I/O",
           "global_batch": B, "seq_len": T, "heads": H, "head_dim": D, "chunk": 64,
           "l2": "flushed before every timed step (512 MB write)"}
-# Algorithmic work per token-head: q, k, v, gate, core at D FP32 values each + beta.
-BYTES_PER_TOKEN_HEAD = 5 * D * 4 + 4
+# Algorithmic bytes per token-head of the timed chunked call: q, k, v, core at D FP32 values
+# each + beta, and the gate input: D BF16 g_raw values (graw) or D FP32 gate values (tc, simt).
+BYTES_PER_TOKEN_HEAD = {"graw": 4 * D * 4 + D * 2 + 4, "tc": 5 * D * 4 + 4, "simt": 5 * D * 4 + 4}
+# kernels one step launches: beta + intra, fix-up, state (graw); + gate (tc); gate, beta, one (simt)
+LAUNCHES_PER_STEP = {"graw": 4, "tc": 5, "simt": 3}
 FLOPS_PER_TOKEN_HEAD = 139_000  # L, M, WY/UT solve, W.S, Q.S, M.U, K^T.U at C=64, D=128 (triangles as half)
 
 
@@ -155,7 +161,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--prefill-impl", default="tc", choices=["tc", "simt"])
+    ap.add_argument("--prefill-impl", default="tc", choices=["tc", "graw", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-block", action="store_true", help="skip the block-prefill leg")
     args = ap.parse_args()
@@ -199,15 +205,22 @@ def main():
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
+    graw = args.prefill_impl == "graw"
+
     def step(kev=None):
-        kda.kda_gate(g_raw, dt_bias, a_log, gate, B * T, d, s)
+        if not graw:
+            kda.kda_gate(g_raw, dt_bias, a_log, gate, B * T, d, s)
         kda.kda_beta(b_logit, beta, B * T * H, s)
         if kev:
             kev[0].record(stream)
-        kda.kda_chunk_prefill(q, k, v, gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl, scratch=scratch)
+        if graw:
+            kda.kda_chunk_prefill_graw(q, k, v, g_raw, dt_bias, a_log, beta, ptrs, core, B, T, d, s, scratch=scratch)
+        else:
+            kda.kda_chunk_prefill(q, k, v, gate, beta, ptrs, core, B, T, d, s, impl=args.prefill_impl,
+                                  scratch=scratch)
         if kev:
             kev[1].record(stream)
-        return 3
+        return LAUNCHES_PER_STEP[args.prefill_impl]
 
     launches = 0
     with Clocks(local) as clk:
@@ -234,7 +247,7 @@ def main():
         step_ms, kern_ms = t.tolist()
 
     hbm, tc_peak, peak_kind = _peaks()
-    alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD + 2 * B * H * D * D * 4
+    alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD[args.prefill_impl] + 2 * B * H * D * D * 4
     alg_flops = B * T * H * FLOPS_PER_TOKEN_HEAD
     achieved_gbs = alg_bytes / (kern_ms * 1e-3) / 1e9
     achieved_tf = alg_flops / (kern_ms * 1e-3) / 1e12
@@ -262,7 +275,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": dict(CONFIG, parallelism=f"dp{world}",
                                                                                      prefill_impl=args.prefill_impl),
-            "roofline": {"kernel": "kda_chunk_prefill", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm,
+            "roofline": {"kernel": "kda_chunk_prefill_graw" if graw else "kda_chunk_prefill", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm,
                          "unit": "GB/s", "frac": achieved_gbs / hbm, "peak_kind": peak_kind,
                          "traffic": _traffic("chunk_prefill_" + args.prefill_impl),
                          "kernel_ms": kern_ms, "alg_bytes_per_launch": alg_bytes,

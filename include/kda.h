@@ -194,6 +194,21 @@ KDA_API int kda_chunk_prefill_fused(const kda_bf16 *qkv, const kda_bf16 *g_raw, 
                                     int B, int T, void *scratch, size_t scratch_bytes, const kda_dims *dims,
                                     void *stream);
 
+/* kda_chunk_prefill_graw — kda_chunk_prefill with the gate step folded in: FP32 q, k, v as
+ * kda_chunk_prefill, and the raw gate projection instead of kda_gate's output
+ * (Glm5NextKdaWorkspace `g_raw`; Glm5NextKdaWeights `dt_bias`, `a_log`):
+ *   g_raw     [B*T_pad, H*D] BF16; dt_bias [H*D] F32; a_log [H] F32: the kernel forms
+ *             g = -exp(a_log[h]) softplus(g_raw + dt_bias) exactly as kda_gate does; only rows
+ *             < T are read (the FP32 gate buffer is never written or read)
+ *   q, k, v, beta, h_state, core, B, T, scratch, scratch_bytes, dims: as kda_chunk_prefill
+ *             (same scratch size).
+ * Errors as kda_chunk_prefill (g_raw must be 16-byte aligned too). The result is bit-identical
+ * to kda_gate followed by kda_chunk_prefill on the same inputs. */
+KDA_API int kda_chunk_prefill_graw(const float *q, const float *k, const float *v, const kda_bf16 *g_raw,
+                                   const float *dt_bias, const float *a_log, const float *beta,
+                                   float *const *h_state, float *core, int B, int T, void *scratch,
+                                   size_t scratch_bytes, const kda_dims *dims, void *stream);
+
 /* kda_chunk_prefill_noalloc — kda_chunk_prefill for callers that cannot allocate device
  * memory (the pages have no counterpart: this is a deployment variant). Some callers cannot
  * call cudaMalloc at all: an engine that hands all free HBM to its KV-cache / state pools at

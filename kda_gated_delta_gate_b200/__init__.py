@@ -64,6 +64,7 @@ _SIGS = {
     "kda_chunk_prefill": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_prefill_fused": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
+    "kda_chunk_prefill_graw": ([_VP] * 9 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_varlen": ([_VP] * 6 + [_I, _I, _I, _VP, _VP, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_varlen_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_verify": ([_VP] * 6 + [_I, _I, _VP, _VP, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
@@ -194,6 +195,19 @@ def kda_chunk_prefill_fused(qkv, g_raw, dt_bias, a_log, beta, h_state_ptrs, core
     return _call("kda_chunk_prefill_fused", _p(qkv), _p(g_raw), _p(dt_bias), _p(a_log), _p(beta), _p(h_state_ptrs),
                  _p(core), B, T, _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d),
                  _stream(stream))
+
+
+def kda_chunk_prefill_graw(q, k, v, g_raw, dt_bias, a_log, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims,
+                           stream=None, scratch=None):
+    """kda_chunk_prefill on FP32 q, k, v with the gate formed in the kernel from the raw BF16
+    g_raw, dt_bias and a_log (bit-identical to kda_gate + kda_chunk_prefill)."""
+    if scratch is None:
+        import torch
+        need = kda_chunk_prefill_scratch_bytes(B, T, d)
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+    return _call("kda_chunk_prefill_graw", _p(q), _p(k), _p(v), _p(g_raw), _p(dt_bias), _p(a_log), _p(beta),
+                 _p(h_state_ptrs), _p(core), B, T, _p(scratch), scratch.numel() * scratch.element_size(),
+                 ctypes.byref(d), _stream(stream))
 
 
 def kda_chunk_prefill_noalloc(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None):

@@ -106,6 +106,9 @@ int chunk_prefill_tc(const float *q, const float *k, const float *v, const float
 int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
                            const float *beta, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
                            void *scratch, cudaStream_t s);
+int chunk_prefill_tc_graw(const float *q, const float *k, const float *v, const uint16_t *g_raw,
+                          const float *dt_bias, const float *a_log, const float *beta, float *const *h_state,
+                          float *core, int B, int T, const kda_dims *dims, void *scratch, cudaStream_t s);
 }  // namespace kda
 
 namespace kda {

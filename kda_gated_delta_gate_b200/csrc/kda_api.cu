@@ -97,6 +97,25 @@ extern "C" int kda_chunk_prefill_fused(const kda_bf16 *qkv, const kda_bf16 *g_ra
                                        static_cast<cudaStream_t>(stream));
 }
 
+extern "C" int kda_chunk_prefill_graw(const float *q, const float *k, const float *v, const kda_bf16 *g_raw,
+                                      const float *dt_bias, const float *a_log, const float *beta,
+                                      float *const *h_state, float *core, int B, int T, void *scratch,
+                                      size_t scratch_bytes, const kda_dims *dims, void *stream) {
+    KDA_TRY(kda::check_dims(dims));
+    if (!q || !k || !v || !g_raw || !dt_bias || !a_log || !beta || !h_state || !core || B < 0 || T < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(q) || !kda::aligned16(k) || !kda::aligned16(v) || !kda::aligned16(g_raw) ||
+        !kda::aligned16(core))
+        return KDA_ERR_MISALIGNED;
+    if (B > 65535 || dims->heads > 65535) return KDA_ERR_UNSUPPORTED;
+    if (B == 0 || T == 0) return KDA_OK;
+    if (!scratch) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(scratch)) return KDA_ERR_MISALIGNED;
+    if (scratch_bytes < kda::chunk_prefill_scratch_bytes(B, T, dims->heads, dims->head_dim)) return KDA_ERR_CAPACITY;
+    return kda::chunk_prefill_tc_graw(q, k, v, g_raw, dt_bias, a_log, beta, h_state, core, B, T, dims, scratch,
+                                      static_cast<cudaStream_t>(stream));
+}
+
 extern "C" size_t kda_chunk_prefill_varlen_scratch_bytes(int B, int max_num_chunks, const kda_dims *dims) {
     if (!dims || kda::check_dims(dims) != KDA_OK) return 0;
     return kda::chunk_prefill_slots_scratch_bytes(B, max_num_chunks, dims->heads, dims->head_dim);

@@ -71,16 +71,24 @@ struct PrefillIn {
     float *tables;  // verify mode: per (stream, head) U [64][D] then Gamma [64][D] (FP32); else null
 };
 
+// Input modes of the chunked kernels: where q, k, v and the log-decay come from.
+//   kInF32   FP32 q, k, v and FP32 gate (kda_gate's output)
+//   kInFused BF16 q|k|v rows (the front end's conv_out) and BF16 g_raw; the gate is formed in-kernel
+//   kInGraw  FP32 q, k, v and BF16 g_raw; the gate is formed in-kernel
+constexpr int kInF32 = 0, kInFused = 1, kInGraw = 2;
+template <int MODE> constexpr bool kQkv16 = MODE == kInFused;  // q|k|v in BF16 rows
+template <int MODE> constexpr bool kGraw = MODE != kInF32;      // gate formed from BF16 g_raw
+
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t u, float &lo, float &hi) {
     lo = __uint_as_float(u << 16);
     hi = __uint_as_float(u & 0xFFFF0000u);
 }
 
 // Channels [c, c + 8) of global token row `row`, head h: q (part 0), k (1) or v (2), as FP32.
-template <int D, bool FUSED>
+template <int D, bool QKV16>
 __device__ __forceinline__ void load8_in(const PrefillIn &in, int part, size_t row, int H, int h, int c,
                                          float (&x)[8]) {
-    if constexpr (FUSED) {
+    if constexpr (QKV16) {
         const uint4 u = *reinterpret_cast<const uint4 *>(in.qkv + row * (3 * static_cast<size_t>(H) * D) +
                                                          static_cast<size_t>(part * H + h) * D + c);
         bf16x2_to_f32(u.x, x[0], x[1]); bf16x2_to_f32(u.y, x[2], x[3]);
@@ -93,10 +101,11 @@ __device__ __forceinline__ void load8_in(const PrefillIn &in, int part, size_t r
     }
 }
 
-// Channels [c, c + 4): q / k / v as above, or the log-decay g (part 3; formed from g_raw in fused mode).
-template <int D, bool FUSED>
+// Channels [c, c + 4): q / k / v as above, or the log-decay g (part 3; formed from g_raw when
+// the mode says so).
+template <int D, int MODE>
 __device__ __forceinline__ float4 load4_in(const PrefillIn &in, int part, size_t row, int H, int h, int c) {
-    if constexpr (FUSED) {
+    if constexpr (kGraw<MODE>) {
         if (part == 3) {
             const uint2 u = *reinterpret_cast<const uint2 *>(in.g_raw + row * (static_cast<size_t>(H) * D) +
                                                              static_cast<size_t>(h) * D + c);
@@ -108,6 +117,8 @@ __device__ __forceinline__ float4 load4_in(const PrefillIn &in, int part, size_t
             return make_float4(kda_gate_f32(r0, dt[0], nea), kda_gate_f32(r1, dt[1], nea),
                                kda_gate_f32(r2, dt[2], nea), kda_gate_f32(r3, dt[3], nea));
         }
+    }
+    if constexpr (kQkv16<MODE>) {
         const uint2 u = *reinterpret_cast<const uint2 *>(in.qkv + row * (3 * static_cast<size_t>(H) * D) +
                                                          static_cast<size_t>(part * H + h) * D + c);
         float4 r;
@@ -261,7 +272,7 @@ struct Intra {
 // The exact CUDA-core intra-chunk computation of one (stream b, head h, chunk ch): every decay
 // factor is a product of per-token factors <= 1, whatever g holds. It writes the whole operand
 // pack. Used for the chunks whose in-block decay is too strong for the tensor-core path.
-template <int D, bool FUSED>
+template <int D, int MODE>
 __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__restrict__ scratch, const Seqs &sq,
                                                 int H, int b, int h, int ch, float *smem) {
     using I = Intra<D>;
@@ -287,9 +298,9 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
         const int i = e / (D / 4), c = 4 * (e % (D / 4));
         float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv, av = make_float4(1.f, 1.f, 1.f, 1.f);
         if (i < n) {
-            kv = load4_in<D, FUSED>(in, 1, row0 + i, H, h, c);
-            qv = load4_in<D, FUSED>(in, 0, row0 + i, H, h, c);
-            const float4 g = load4_in<D, FUSED>(in, 3, row0 + i, H, h, c);
+            kv = load4_in<D, MODE>(in, 1, row0 + i, H, h, c);
+            qv = load4_in<D, MODE>(in, 0, row0 + i, H, h, c);
+            const float4 g = load4_in<D, MODE>(in, 3, row0 + i, H, h, c);
             av = make_float4(expf(g.x), expf(g.y), expf(g.z), expf(g.w));
         }
         *reinterpret_cast<float4 *>(sK + i * P + c) = kv;
@@ -460,8 +471,8 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
         *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
         float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
         if (i < n) {
-            v0 = load4_in<D, FUSED>(in, 2, row0 + i, H, h, cb);
-            v1 = load4_in<D, FUSED>(in, 2, row0 + i, H, h, cb + 4);
+            v0 = load4_in<D, MODE>(in, 2, row0 + i, H, h, cb);
+            v1 = load4_in<D, MODE>(in, 2, row0 + i, H, h, cb + 4);
         }
         *reinterpret_cast<float4 *>(sA + i * P + cb) = v0;
         *reinterpret_cast<float4 *>(sA + i * P + cb + 4) = v1;
@@ -524,7 +535,7 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
         float acc = 0.f;
         for (int i = 0; i < C; ++i) {
             if (i < n) {
-                const float4 g4 = load4_in<D, FUSED>(in, 3, row0 + i, H, h, tid & ~3);
+                const float4 g4 = load4_in<D, MODE>(in, 3, row0 + i, H, h, tid & ~3);
                 acc += (tid & 3) == 0 ? g4.x : ((tid & 3) == 1 ? g4.y : ((tid & 3) == 2 ? g4.z : g4.w));
             }
             gt[i * D + tid] = acc;
@@ -533,7 +544,7 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
 }
 
 // Only the chunks the tensor-core kernel listed (count and packed (b, h, ch) entries in scratch).
-template <int D, bool FUSED>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kIntraThreads, 1)
 intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *__restrict__ list, const Seqs sq,
                  int H) {
@@ -543,7 +554,7 @@ intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *_
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
         const int id = list[1 + e];
         const int ch = id % nch, h = (id / nch) % H, b = id / (nch * H);
-        intra_simt_body<D, FUSED>(in, scratch, sq, H, b, h, ch, smem);
+        intra_simt_body<D, MODE>(in, scratch, sq, H, b, h, ch, smem);
         __syncthreads();
     }
 }
@@ -600,7 +611,7 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // k into registers, v into L2); v itself arrives by a TMA box once g's space is free again,
 // and the W | U~ results leave through shared memory in bulk copies. The g and v boxes come
 // from 3-D maps whose row extent is T, so rows past T arrive as zeros (the pad guard).
-template <int D, bool FUSED>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kIntraThreads, 1)
 intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmV, const PrefillIn in,
                 uint8_t *__restrict__ scratch, int *__restrict__ list, int B, const Seqs sq, int H,
@@ -630,11 +641,12 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nch = sq.nch;
     const int total = B * H * nch;
-    constexpr uint32_t kBox = C * D * (FUSED ? 2 : 4);  // one g (g_raw) or v box
+    constexpr bool QKV16 = kQkv16<MODE>, GRAW = kGraw<MODE>;
+    constexpr uint32_t kGBox = C * D * (GRAW ? 2 : 4), kVBox = C * D * (QKV16 ? 2 : 4);  // one g / v box
     // g's box: FP32 g at the start of its space, or BF16 g_raw in the upper half (the gate is
     // then formed in place, FP32, dense)
-    void *gdst = reinterpret_cast<uint8_t *>(sG) + (FUSED ? C * D * 2 : 0);
-    const int vx0 = FUSED ? 2 * H * D : 0;  // v's column in the box source
+    void *gdst = reinterpret_cast<uint8_t *>(sG) + (GRAW ? C * D * 2 : 0);
+    const int vx0 = QKV16 ? 2 * H * D : 0;  // v's column in the box source
     const size_t rs = static_cast<size_t>(H) * D;
 
     if (warp == 0) {
@@ -679,10 +691,10 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         for (int u = 0; u < UPT; ++u) {
             const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
             if (i < n) {
-                load8_in<D, FUSED>(in, 1, row0 + i, H, h, cb, kk[u]);
-                load8_in<D, FUSED>(in, 0, row0 + i, H, h, cb, qq[u]);
-                if ((cb & (FUSED ? 63 : 31)) == 0) {
-                    const void *vp = FUSED ? static_cast<const void *>(in.qkv + (row0 + i) * (3 * rs) + 2 * rs +
+                load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, kk[u]);
+                load8_in<D, QKV16>(in, 0, row0 + i, H, h, cb, qq[u]);
+                if ((cb & (QKV16 ? 63 : 31)) == 0) {
+                    const void *vp = QKV16 ? static_cast<const void *>(in.qkv + (row0 + i) * (3 * rs) + 2 * rs +
                                                                       static_cast<size_t>(h) * D + cb)
                                            : static_cast<const void *>(in.v + (row0 + i) * rs +
                                                                       static_cast<size_t>(h) * D + cb);
@@ -696,7 +708,7 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         if (tid == 0) {
             int y, z;
             box_yz(ch, b, row0, y, z);
-            mbar_expect_tx(gbar, kBox);
+            mbar_expect_tx(gbar, kGBox);
             tma_load_3d(gdst, &tmG, h * D, y, z, gbar);
         }
         if (tid < C) bnext = tid < n ? in.beta[(row0 + tid) * H + h] : 0.f;
@@ -745,7 +757,7 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
             constexpr int QT = NT / D;  // 4 (D=128) or 8 (D=64) token ranges
             constexpr int TPQ = C / QT;
             const int c = tid % D, qr = tid / D;
-            if constexpr (FUSED) {
+            if constexpr (GRAW) {
                 // g = -exp(a_log) softplus(g_raw + dt_bias) (0 past T), FP32 over g_raw's box
                 const uint16_t *gr = reinterpret_cast<const uint16_t *>(gdst);
                 float x[TPQ];
@@ -864,7 +876,7 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         // ---- v by one TMA box into g's space (Gamma is no longer read), for the W | U~ operand;
         //      D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127)
         if (tid == 0) {
-            mbar_expect_tx(vbar, kBox);
+            mbar_expect_tx(vbar, kVBox);
             tma_load_3d(sG, &tmV, vx0 + h * D, boxy, boxz, vbar);
             if (safe) {
                 constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
@@ -919,7 +931,7 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
             for (int u = 0; u < UPT; ++u) {
                 const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
                 float x[8];
-                if constexpr (FUSED) {
+                if constexpr (QKV16) {
                     const uint4 w4 = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(sG) + i * D + cb);
                     bf16x2_to_f32(w4.x, x[0], x[1]); bf16x2_to_f32(w4.y, x[2], x[3]);
                     bf16x2_to_f32(w4.z, x[4], x[5]); bf16x2_to_f32(w4.w, x[6], x[7]);
@@ -1332,15 +1344,15 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
 template <int D>
 size_t packs_bytes(int B, int H, int nch) { return static_cast<size_t>(B) * H * nch * Pack<D>::bytes; }
 
-template <int D, int DVS, bool FUSED>
+template <int D, int DVS, int MODE>
 int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, int H, float scale,
               void *scratch, cudaStream_t s) {
     const int nch = sq.nch;
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
     static std::atomic<unsigned long long> attr_intra{0}, attr_fix{0}, attr_state{0};
-    KDA_TRY(smem_opt_in(intra_tc_kernel<D, FUSED>, IntraTC<D>::bytes, attr_intra));
-    KDA_TRY(smem_opt_in(intra_fix_kernel<D, FUSED>, static_cast<int>(Intra<D>::bytes), attr_fix));
+    KDA_TRY(smem_opt_in(intra_tc_kernel<D, MODE>, IntraTC<D>::bytes, attr_intra));
+    KDA_TRY(smem_opt_in(intra_fix_kernel<D, MODE>, static_cast<int>(Intra<D>::bytes), attr_fix));
     KDA_TRY(smem_opt_in(state_kernel<D, DVS>, State<D, DVS>::bytes, attr_state));
     uint8_t *sc = static_cast<uint8_t *>(scratch);
     int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(B, H, nch));
@@ -1356,16 +1368,17 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     // box maps: (stream, row in stream) for equal-length streams; the packed rows in varlen mode
     const int mT = sq.cu ? sq.total : sq.T, mTp = sq.cu ? sq.total : sq.T_pad, mB = sq.cu ? 1 : B;
     CUtensorMap tmG, tmV;
-    if (FUSED) {
+    if (kGraw<MODE>)
         KDA_TRY(make_rows_map(&tmG, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, mT, mTp, mB, D, C));
-        KDA_TRY(make_rows_map(&tmV, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, mT, mTp, mB, D, C));
-    } else {
+    else
         KDA_TRY(make_rows_map(&tmG, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
+    if (kQkv16<MODE>)
+        KDA_TRY(make_rows_map(&tmV, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, mT, mTp, mB, D, C));
+    else
         KDA_TRY(make_rows_map(&tmV, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-    }
-    intra_tc_kernel<D, FUSED><<<grid, kIntraThreads, IntraTC<D>::bytes, s>>>(tmG, tmV, in, sc, list, B, sq, H, status);
+    intra_tc_kernel<D, MODE><<<grid, kIntraThreads, IntraTC<D>::bytes, s>>>(tmG, tmV, in, sc, list, B, sq, H, status);
     KDA_TRY(launch_status());
-    intra_fix_kernel<D, FUSED><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
+    intra_fix_kernel<D, MODE><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
     state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
                                                                                    in.tables, status);
@@ -1373,15 +1386,15 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
 }
 
 // Value slice width: enough CTAs to cover the SMs (one state CTA per SM fits in shared memory).
-template <bool FUSED>
+template <int MODE>
 int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, const kda_dims *dims,
                void *scratch, cudaStream_t s) {
     const int H = dims->heads;
     const float sc = dims->scale;
-    if (dims->head_dim == 64) return launch_tc<64, 32, FUSED>(in, h_state, core, B, sq, H, sc, scratch, s);
+    if (dims->head_dim == 64) return launch_tc<64, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
     const long long units = static_cast<long long>(B) * H;
-    if (units >= 60) return launch_tc<128, 64, FUSED>(in, h_state, core, B, sq, H, sc, scratch, s);
-    return launch_tc<128, 32, FUSED>(in, h_state, core, B, sq, H, sc, scratch, s);
+    if (units >= 60) return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    return launch_tc<128, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
 }
 
 Seqs equal_seqs(int T) {
@@ -1407,28 +1420,35 @@ int chunk_prefill_tc(const float *q, const float *k, const float *v, const float
                      float *const *h_state, float *core, int B, int T, const kda_dims *dims, void *scratch,
                      cudaStream_t s) {
     const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, nullptr};
-    return launch_any<false>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
+    return launch_any<kInF32>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
 }
 
 int chunk_prefill_tc_varlen(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                             const int *cu_seqlens, int B, int max_chunks, int total, float *const *h_state,
                             float *core, const kda_dims *dims, void *scratch, cudaStream_t s) {
     const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, nullptr};
-    return launch_any<false>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, max_chunks, total}, dims, scratch, s);
+    return launch_any<kInF32>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, max_chunks, total}, dims, scratch, s);
 }
 
 int chunk_verify_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                     const int *cu_seqlens, int B, int total, float *const *h_state, float *core, float *tables,
                     const kda_dims *dims, void *scratch, cudaStream_t s) {
     const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, tables};
-    return launch_any<false>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, 1, total}, dims, scratch, s);
+    return launch_any<kInF32>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, 1, total}, dims, scratch, s);
 }
 
 int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
                            const float *beta, float *const *h_state, float *core, int B, int T, const kda_dims *dims,
                            void *scratch, cudaStream_t s) {
     const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta, nullptr};
-    return launch_any<true>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
+    return launch_any<kInFused>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
+}
+
+int chunk_prefill_tc_graw(const float *q, const float *k, const float *v, const uint16_t *g_raw,
+                          const float *dt_bias, const float *a_log, const float *beta, float *const *h_state,
+                          float *core, int B, int T, const kda_dims *dims, void *scratch, cudaStream_t s) {
+    const PrefillIn in{q, k, v, nullptr, nullptr, g_raw, dt_bias, a_log, beta, nullptr};
+    return launch_any<kInGraw>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
 }
 
 }  // namespace kda

@@ -189,6 +189,44 @@ def test_fused_prefill_extreme_decay_takes_exact_path():
     _check(ci, core_f, S_f)
 
 
+@pytest.mark.parametrize("B,T,H,D,strong", [(1, 4096, 32, 128, False), (2, 150, 3, 128, False),
+                                            (3, 1, 2, 64, False), (2, 257, 2, 64, False), (1, 200, 3, 128, True)])
+def test_graw_prefill_bit_identical_to_gate_then_prefill(B, T, H, D, strong):
+    """kda_chunk_prefill_graw (the gate formed in the kernel from BF16 g_raw) gives the same
+    bits as kda_gate + kda_chunk_prefill on the same inputs, and matches the oracle; the tails
+    of q, k, v, g_raw and beta hold NaN. `strong`: decay strong enough on some channels to send
+    chunks to the exact CUDA-core body, which forms the gate itself in this mode."""
+    ci = core_inputs(B, T, H, D, seed=70 + T, s0_std=0.1)
+    if strong:
+        ci.a_log[1] = 3.0
+        ci.dt_bias[1 * D + 5] = 20.0
+        ci.dt_bias[1 * D + 9] = 6.0
+    Tp, nan = t_pad(T), float("nan")
+    d = kda.dims(H, D, scale=0.7)
+    q, k, v = (pad_rows(x, Tp, nan).cuda() for x in (ci.q, ci.k, ci.v))
+    g_raw = pad_rows(ci.g_raw, Tp, nan).cuda()
+    dt, al = ci.dt_bias.cuda(), ci.a_log.cuda()
+    beta = pad_rows(ci.b_logit, Tp, 0.0).cuda()
+    kda.kda_beta(beta, beta, beta.numel())
+    beta.view(B, Tp, H)[:, T:] = nan
+    gate = torch.full((B * Tp, H, D), nan, device="cuda")
+    for b in range(B):  # valid rows only: the gate of the tail stays NaN
+        kda.kda_gate(g_raw[b * Tp:b * Tp + T], dt, al, gate[b * Tp:b * Tp + T], T, d)
+    outs = []
+    for use_graw in (False, True):
+        states = [ci.s0[b].cuda().clone() for b in range(B)]
+        core = torch.full((B * Tp, H, D), nan, device="cuda")
+        if use_graw:
+            kda.kda_chunk_prefill_graw(q, k, v, g_raw, dt, al, beta, kda.ptr_array(states), core, B, T, d)
+        else:
+            kda.kda_chunk_prefill(q, k, v, gate, beta, kda.ptr_array(states), core, B, T, d)
+        torch.cuda.synchronize()
+        outs.append((core.view(B, Tp, H, D)[:, :T].clone(), torch.stack(states)))
+    (c0, s0), (c1, s1) = outs
+    assert torch.equal(c0, c1) and torch.equal(s0, s1)
+    _check(ci, c1, s1, scale=0.7)
+
+
 def _varlen_case(lens, H, D, seed):
     """Packed sequences of the given lengths: q, k, v [total, H, D], gate and beta formed on the
     GPU from the packed g_raw / b_logit, per-sequence initial states, cu_seqlens on the device."""
