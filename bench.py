@@ -13,7 +13,7 @@ Multi-GPU: each rank runs its own independent sequence (weak scaling, no collect
 
 Also reported: the dominant kernel's roofline (CUDA events around each launch), a decode
 leg (256 sequences x 1 token, kda_decode_fused, state GB/s), an end-to-end leg through
-the same C-ABI calls from pinned host buffers (copies inside the timed region), and the
+kda_chunk_prefill_host from pinned host buffers (copies inside the timed region), and the
 FP64 oracle timed on the host cores (`cpu_baseline`). `--impl reference` times the oracle
 alone (it is this project's reference implementation) and prints its own line.
 """
@@ -255,7 +255,7 @@ def main():
     # ---- decode leg: 256 sequences x 1 token, fused stateful row (state GB/s)
     dec = _decode_leg(kda, torch, dev, s, stream, flush, hbm)
 
-    # ---- end-to-end leg: the same C-ABI calls from pinned host buffers, copies timed
+    # ---- end-to-end leg: kda_chunk_prefill_host from pinned host buffers, copies timed
     e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch)
 
     # ---- the full block (projections + front end + core + back end) and its dominant GEMM
@@ -394,34 +394,28 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
 
 
 def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
-    """The same prefill through the public C ABI from pinned host buffers, every step copying its
-    inputs in and its outputs out. The inputs travel as the serving path holds them: the BF16
-    q|k|v rows (the front end's conv_out layout; the workload's inputs are BF16-exact), the BF16
-    g_raw and the FP32 beta logits; kda_beta + kda_chunk_prefill_fused compute the step."""
-    from synth import pad_rows
-    qkv = torch.cat([ci.q.reshape(B, T, H * D), ci.k.reshape(B, T, H * D), ci.v.reshape(B, T, H * D)], dim=-1)
-    host = {"qkv": pad_rows(qkv.to(torch.bfloat16), Tp, 0.0).pin_memory(),
-            "g_raw": pad_rows(ci.g_raw, Tp, 0.0).pin_memory(),
-            "b_logit": pad_rows(ci.b_logit, Tp, 0.0).pin_memory(),
-            "s0": ci.s0[0].clone().pin_memory()}
-    dv = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    """The same prefill through the public C ABI from pinned host buffers: kda_chunk_prefill_host
+    copies each step's inputs in and its outputs out, segment by segment (512 tokens), with the
+    copies of one segment overlapping the kernels of the next. The inputs travel as the serving
+    path holds them: the BF16 q|k|v rows (the front end's conv_out layout; the workload's inputs
+    are BF16-exact), the BF16 g_raw and the FP32 beta logits; the outputs are the FP32 core rows
+    and the final state."""
+    seg = 512
+    qkv = torch.cat([ci.q.reshape(T, H * D), ci.k.reshape(T, H * D), ci.v.reshape(T, H * D)], dim=-1)
+    host = {"qkv": qkv.to(torch.bfloat16).contiguous().pin_memory(),
+            "g_raw": ci.g_raw[0].contiguous().pin_memory(),
+            "b_logit": ci.b_logit[0].contiguous().pin_memory()}
+    s0 = ci.s0[0].clone()
+    state_h = s0.clone().pin_memory()
+    core_h = torch.empty((T, H, D)).pin_memory()
     dt_bias, a_log = ci.dt_bias.to(dev), ci.a_log.to(dev)
-    beta = torch.empty((B * Tp, H), device=dev)
-    core = torch.empty((B * Tp, H, D), device=dev)
-    core_h = torch.empty_like(core, device="cpu").pin_memory()
-    s_h = torch.empty_like(host["s0"]).pin_memory()
-    ptrs = kda.ptr_array([dv["s0"]], device=dev)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = core_h.numel() * 4 + s_h.numel() * 4
+    buf = torch.empty(kda.kda_chunk_prefill_host_bytes(T, seg, d), dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + state_h.numel() * 4
+    d2h = core_h.numel() * 4 + state_h.numel() * 4
 
     def one():
-        for n, t in host.items():
-            dv[n].copy_(t, non_blocking=True)
-        kda.kda_beta(dv["b_logit"], beta, B * T * H, s)
-        kda.kda_chunk_prefill_fused(dv["qkv"], dv["g_raw"], dt_bias, a_log, beta, ptrs, core, B, T, d, s,
-                                    scratch=scratch)
-        core_h.copy_(core, non_blocking=True)
-        s_h.copy_(dv["s0"], non_blocking=True)
+        kda.kda_chunk_prefill_host(host["qkv"], host["g_raw"], host["b_logit"], dt_bias, a_log, state_h, core_h, T,
+                                   seg, buf, d, s)
 
     for _ in range(3):
         one()
@@ -441,8 +435,8 @@ def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
         ms = t.item()
     return {"value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "call": "kda_beta + kda_chunk_prefill_fused (BF16 q|k|v rows, BF16 g_raw, FP32 beta logits in; FP32 core "
-                    "and state out)"}
+            "call": f"kda_chunk_prefill_host, {seg}-token segments (BF16 q|k|v rows, BF16 g_raw, FP32 beta logits "
+                    "and state in; FP32 core and state out; copies and kernels of consecutive segments overlapped)"}
 
 
 if __name__ == "__main__":

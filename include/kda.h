@@ -209,6 +209,36 @@ KDA_API int kda_chunk_prefill_graw(const float *q, const float *k, const float *
                                    float *const *h_state, float *core, int B, int T, void *scratch,
                                    size_t scratch_bytes, const kda_dims *dims, void *stream);
 
+/* kda_chunk_prefill_host — kda_beta + kda_chunk_prefill_fused for ONE sequence whose inputs
+ * and outputs are in HOST memory (a deployment variant; the pages keep everything on the device):
+ * the host->device copies, the kernels and the device->host copies of consecutive segments of
+ * segment_tokens tokens overlap on three streams (two copy streams the library keeps per device,
+ * and `stream`), so the call costs about the slower PCIe direction rather than the sum.
+ *   qkv      HOST [T, 3*H*D] BF16 rows q | k | v (the layout kda_chunk_prefill_fused reads)
+ *   g_raw    HOST [T, H*D] BF16;  b_logit HOST [T, H] F32 (beta = sigmoid(b_logit) is formed here)
+ *   dt_bias  DEVICE [H*D] F32;  a_log DEVICE [H] F32
+ *   h_state  HOST [H, D, D] F32: read as the carried state, overwritten with the state after T
+ *   core     HOST [T, H, D] F32 output
+ *   segment_tokens  a positive multiple of 64 (512 is a good size on PCIe 5)
+ *   device_buffer   DEVICE, 16-byte aligned, at least kda_chunk_prefill_host_bytes(T,
+ *                   segment_tokens, dims) bytes: the staging rows, beta, core, the state and one
+ *                   segment's prefill scratch; contents on entry do not matter
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for the copies to
+ * overlap; pageable ones work but serialise. The call only enqueues: host outputs are complete
+ * once `stream` has completed (it waits for the last copy out). Calls from several host threads
+ * are serialised while they enqueue. Because segments are whole chunks, core and the final state
+ * are the same bits as kda_beta + kda_chunk_prefill_fused over all T rows on the device.
+ * Errors: KDA_ERR_INVALID_ARG (NULL pointer, T < 0, bad segment_tokens), KDA_ERR_MISALIGNED,
+ * KDA_ERR_CAPACITY (device_bytes too small), KDA_ERR_CUDA. */
+KDA_API int kda_chunk_prefill_host(const kda_bf16 *qkv, const kda_bf16 *g_raw, const float *b_logit,
+                                   const float *dt_bias, const float *a_log, float *h_state, float *core, int T,
+                                   int segment_tokens, void *device_buffer, size_t device_bytes,
+                                   const kda_dims *dims, void *stream);
+
+/* Device bytes kda_chunk_prefill_host needs (0 if T <= 0 or segment_tokens is not a positive
+ * multiple of 64). */
+KDA_API size_t kda_chunk_prefill_host_bytes(int T, int segment_tokens, const kda_dims *dims);
+
 /* kda_chunk_prefill_noalloc — kda_chunk_prefill for callers that cannot allocate device
  * memory (the pages have no counterpart: this is a deployment variant). Some callers cannot
  * call cudaMalloc at all: an engine that hands all free HBM to its KV-cache / state pools at

@@ -89,6 +89,31 @@ def test_decode_alias_and_snapshot_checks(L):
     assert L.kda_recurrent_decode(*([BOGUS] * 7), -3, d, None) == 1
 
 
+def test_host_prefill_argument_checks(L):
+    d = ctypes.byref(_d())
+    # staging rows (T_pad = 128) for qkv, g_raw, beta, core, the state, the slot, one segment's scratch
+    hd, tp = 2 * 64, 128
+    r256 = lambda x: (x + 255) // 256 * 256
+    seg_scratch = L.kda_chunk_prefill_scratch_bytes(1, 64, d)
+    need = (r256(tp * 3 * hd * 2) + r256(tp * hd * 2) + r256(tp * 2 * 4) + r256(tp * hd * 4) + r256(hd * 64 * 4)
+            + 256 + r256(seg_scratch))
+    assert L.kda_chunk_prefill_host_bytes(100, 64, d) == need
+    assert L.kda_chunk_prefill_host_bytes(100, 96, d) == 0  # not whole chunks
+    assert L.kda_chunk_prefill_host_bytes(0, 64, d) == 0
+    args = [BOGUS] * 7
+    assert L.kda_chunk_prefill_host(*args, 0, 64, BOGUS, 0, d, None) == 0  # T = 0: nothing to do
+    assert L.kda_chunk_prefill_host(*args, 100, 0, BOGUS, need, d, None) == 1
+    assert L.kda_chunk_prefill_host(*args, 100, 100, BOGUS, need, d, None) == 1
+    assert L.kda_chunk_prefill_host(*args, -1, 64, BOGUS, need, d, None) == 1
+    assert L.kda_chunk_prefill_host(*args, 100, 64, None, need, d, None) == 1
+    assert L.kda_chunk_prefill_host(*args, 100, 64, BOGUS + 8, need, d, None) == 7
+    assert L.kda_chunk_prefill_host(*args, 100, 64, BOGUS, need - 16, d, None) == 3
+    bad = list(args)
+    bad[5] = None
+    assert L.kda_chunk_prefill_host(*bad, 100, 64, BOGUS, need, d, None) == 1
+    assert L.kda_chunk_prefill_host(*args, 100, 64, BOGUS, need, ctypes.byref(_d(head_dim=96)), None) == 4
+
+
 def test_front_back_argument_checks(L):
     d = ctypes.byref(_d())
     assert L.kda_front_conv_silu_l2(BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, None, None, 0.0, 8, d, None) == 1

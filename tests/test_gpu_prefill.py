@@ -227,6 +227,42 @@ def test_graw_prefill_bit_identical_to_gate_then_prefill(B, T, H, D, strong):
     _check(ci, c1, s1, scale=0.7)
 
 
+@pytest.mark.parametrize("T,H,D,seg", [(4096, 32, 128, 512), (1000, 4, 128, 256), (130, 3, 64, 64),
+                                      (70, 2, 128, 512)])
+def test_host_prefill_bit_identical_to_device_calls(T, H, D, seg):
+    """kda_chunk_prefill_host (pinned host inputs and outputs, segments of whole chunks with
+    copies and compute overlapped) gives the same bits as kda_beta + kda_chunk_prefill_fused over
+    all T rows on the device, and matches the oracle."""
+    ci = core_inputs(1, T, H, D, seed=90 + T, bf16_inputs=True, s0_std=0.1)
+    Tp = t_pad(T)
+    d = kda.dims(H, D, scale=0.7)
+    qkv = torch.cat([ci.q.reshape(T, H * D), ci.k.reshape(T, H * D), ci.v.reshape(T, H * D)], dim=-1)
+    qkv = qkv.to(torch.bfloat16).contiguous()
+    g_raw = ci.g_raw[0].contiguous()
+    b_logit = ci.b_logit[0].contiguous()
+    dt, al = ci.dt_bias.cuda(), ci.a_log.cuda()
+    # on the device, whole
+    qkv_d = pad_rows(qkv[None], Tp, 0.0).cuda()
+    g_d = pad_rows(g_raw[None], Tp, 0.0).cuda()
+    beta_d = pad_rows(b_logit[None], Tp, 0.0).cuda()
+    kda.kda_beta(beta_d, beta_d, beta_d.numel())
+    st_dev = ci.s0[0].cuda().clone()
+    core_dev = torch.zeros((Tp, H, D), device="cuda")
+    kda.kda_chunk_prefill_fused(qkv_d, g_d, dt, al, beta_d, kda.ptr_array([st_dev]), core_dev, 1, T, d)
+    # from host buffers, segmented
+    hq, hg, hb = qkv.pin_memory(), g_raw.pin_memory(), b_logit.pin_memory()
+    hs = ci.s0[0].clone().pin_memory()
+    hc = torch.full((T, H, D), float("nan")).pin_memory()
+    buf = torch.empty(kda.kda_chunk_prefill_host_bytes(T, seg, d), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream()
+    kda.kda_chunk_prefill_host(hq, hg, hb, dt, al, hs, hc, T, seg, buf, d, s.cuda_stream)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(hc, core_dev[:T].cpu()) and torch.equal(hs, st_dev.cpu())
+    if T <= 1000:
+        _check(ci, hc.reshape(1, T, H, D), hs.reshape(1, H, D, D), scale=0.7)
+
+
 def _varlen_case(lens, H, D, seed):
     """Packed sequences of the given lengths: q, k, v [total, H, D], gate and beta formed on the
     GPU from the packed g_raw / b_logit, per-sequence initial states, cu_seqlens on the device."""
