@@ -118,6 +118,17 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def _oracle_baseline(T_sample):
     """The FP64 oracle (as it stands) on the first T_sample tokens of the workload: gate,
     sigmoid and the token recurrence for all 32 heads, on all host cores."""
@@ -240,7 +251,9 @@ def main():
     if world > 1:
         dist.barrier()
     step_ms = sum(a.elapsed_time(b) for a, b in ev_s) / args.steps
-    kern_ms = sum(a.elapsed_time(b) for a, b in ev_k) / args.steps
+    kern_all = [a.elapsed_time(b) for a, b in ev_k]
+    kern_ms = sum(kern_all) / args.steps
+    kern_med, kern_min = statistics.median(kern_all), min(kern_all)
     if world > 1:
         t = torch.tensor([step_ms, kern_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -267,7 +280,7 @@ def main():
         cpu = None
         if not args.no_cpu_baseline:
             tps, dt, cores = _oracle_baseline(T)
-            cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu_model": _cpu_model(),
                    "sample": f"FP64 oracle (gate, sigmoid, token recurrence, 32 heads) over the whole {T}-token "
                              f"workload once; {dt:.2f} s wall on {cores} threads"}
         result = {
@@ -278,7 +291,8 @@ def main():
             "roofline": {"kernel": "kda_chunk_prefill_graw" if graw else "kda_chunk_prefill", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm,
                          "unit": "GB/s", "frac": achieved_gbs / hbm, "peak_kind": peak_kind,
                          "traffic": _traffic("chunk_prefill_" + args.prefill_impl),
-                         "kernel_ms": kern_ms, "alg_bytes_per_launch": alg_bytes,
+                         "kernel_ms": kern_ms, "kernel_ms_median": kern_med, "kernel_ms_min": kern_min,
+                         "alg_bytes_per_launch": alg_bytes,
                          "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                                     "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
             "decode": dec,
@@ -358,6 +372,7 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
 
     ms = timed(lambda: kda.kda_block_prefill(st, hid, Tb, hs, cs, 0.0, ws, s))
     qkv, cd = Hh * Dd, 3 * Hh * Dd
+    stages = _block_stages(kda, torch, dev, s, stream, flush, Wt, hid, ws, Tb, hidden, Hh, Dd, rank)
     flops = 2.0 * Tb * hidden * (3 * qkv + 2 * rank + Hh) + 2.0 * Tb * rank * 2 * qkv + 2.0 * Tb * qkv * hidden
     C = torch.empty((Tb, hidden), dtype=torch.bfloat16, device=dev)
     gms = timed(lambda: kda.kda_gemm_bf16(hid, Wt.w_q, C, Tb, hidden, hidden, stream=s))
@@ -388,9 +403,61 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
     return {"workload": "kda_block_prefill hidden 4096 H32 D128 rank 128 T8192 (9 GEMMs + conv + gate + core + o_norm)",
             "ms": ms, "tokens_per_s": Tb / (ms * 1e-3), "proj_flops": flops,
             "tflops_all": flops / (ms * 1e-3) / 1e12,
+            "stages_ms": stages,
             "gemm": {"shape": "8192x4096x4096 bf16->bf16", "ms": gms, "tflops": gflop / (gms * 1e-3) / 1e12,
                      "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak},
             "block_decode": dec}
+
+
+def _block_stages(kda, torch, dev, s, stream, flush, Wt, hid, ws, Tb, hidden, Hh, Dd, rank, reps=6):
+    """The block prefill's stages, run one after another through their own C-ABI calls on the
+    block's workspace (the order and arguments kda_block_prefill uses), with CUDA events between
+    them: median ms per stage over `reps` runs, L2 flushed before each run."""
+    bf = torch.bfloat16
+    qkv, cd = Hh * Dd, 3 * Hh * Dd
+    d = kda.dims(Hh, Dd)
+    qp = ws.view("qkv_proj", (Tb, cd), bf)
+    co = ws.view("conv_out", (Tb, cd), bf)
+    fa = ws.view("f_a_out", (Tb, rank), bf)
+    gr = ws.view("g_raw", (Tb, qkv), bf)
+    be = ws.view("beta", (Tb, Hh), torch.float32)
+    core = ws.view("core", (Tb, Hh, Dd), torch.float32)
+    ga = ws.view("g_a_out", (Tb, rank), bf)
+    og = ws.view("out_gate", (Tb, qkv), bf)
+    on = ws.view("o_norm_out", (Tb, qkv), bf)
+    fo = ws.view("final_out", (Tb, hidden), bf)
+    sc_ptr, sc_bytes = ws.buffer("prefill_scratch")
+    scratch = kda._device_view(sc_ptr, (sc_bytes,), torch.uint8)
+    hs = torch.zeros((Hh, Dd, Dd), device=dev)
+    cs = torch.zeros((cd, 3), dtype=bf, device=dev)
+    hp = kda.ptr_array([hs], device=dev)
+    gemm = lambda A, W, C, N, K: kda.kda_gemm_bf16(A, W, C, Tb, N, K, stream=s)
+    stages = (
+        ("proj_qkv", lambda: [gemm(hid, w, qp[:, i * qkv:(i + 1) * qkv], qkv, hidden)
+                              for i, w in enumerate((Wt.w_q, Wt.w_k, Wt.w_v))]),
+        ("front_conv_silu_l2", lambda: kda.kda_front_conv_silu_l2(qp, cs, Wt.conv_w, co, None, None, None, 0.0, Tb,
+                                                                   d, s)),
+        ("gate_beta_inputs", lambda: (gemm(hid, Wt.f_a, fa, rank, hidden), gemm(fa, Wt.f_b, gr, qkv, rank),
+                                      gemm(hid, Wt.b_proj, be, Hh, hidden), kda.kda_beta(be, be, Tb * Hh, s))),
+        ("core_prefill_fused", lambda: kda.kda_chunk_prefill_fused(co, gr, Wt.dt_bias, Wt.a_log, be, hp, core, 1, Tb,
+                                                                   d, s, scratch=scratch)),
+        ("out_gate_norm_oproj", lambda: (gemm(hid, Wt.g_a, ga, rank, hidden), gemm(ga, Wt.g_b, og, qkv, rank),
+                                         kda.kda_back_gated_rmsnorm(core, og, Wt.o_norm, on, Tb, d, s),
+                                         gemm(on, Wt.o_proj, fo, hidden, qkv))),
+    )
+    times = {name: [] for name, _ in stages}
+    for i in range(3 + reps):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        evs[0].record(stream)
+        for j, (_, fn) in enumerate(stages):
+            fn()
+            evs[j + 1].record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            for j, (name, _) in enumerate(stages):
+                times[name].append(evs[j].elapsed_time(evs[j + 1]))
+    return {name: statistics.median(t) for name, t in times.items()}
 
 
 def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
