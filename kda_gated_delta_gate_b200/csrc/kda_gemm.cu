@@ -254,6 +254,7 @@ namespace {
 template <int MB>
 __global__ void __launch_bounds__(32 * kGemvWarps)
 gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M, int K) {
+    constexpr int U = 8;  // weight loads in flight per lane (U x 16 bytes)
     extern __shared__ __align__(16) uint16_t sx[];  // [mb][K]: this group's rows only
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m0 = blockIdx.y * MB;
@@ -271,33 +272,45 @@ gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M,
         float acc[MB];
 #pragma unroll
         for (int r = 0; r < MB; ++r) acc[r] = 0.f;
-#pragma unroll 4
-        for (int k = 8 * lane; k < K; k += 256) {
-            const uint4 wv = __ldcs(reinterpret_cast<const uint4 *>(wr + k));
-            float w8[8];
-            w8[0] = __uint_as_float(wv.x << 16); w8[1] = __uint_as_float(wv.x & 0xFFFF0000u);
-            w8[2] = __uint_as_float(wv.y << 16); w8[3] = __uint_as_float(wv.y & 0xFFFF0000u);
-            w8[4] = __uint_as_float(wv.z << 16); w8[5] = __uint_as_float(wv.z & 0xFFFF0000u);
-            w8[6] = __uint_as_float(wv.w << 16); w8[7] = __uint_as_float(wv.w & 0xFFFF0000u);
+        // lane-strided K steps in ascending order (k = 8 lane + 256 j); the loads of U steps are
+        // issued together, the products then accumulate in the same order as one step at a time
+        for (int kb = 8 * lane; kb < K; kb += 256 * U) {
+            uint4 wv[U];
 #pragma unroll
-            for (int r = 0; r < MB; ++r) {
-                if (r < mb) {
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(sx + r * K + k);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.x << 16), w8[0], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.x & 0xFFFF0000u), w8[1], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.y << 16), w8[2], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.y & 0xFFFF0000u), w8[3], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.z << 16), w8[4], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.z & 0xFFFF0000u), w8[5], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.w << 16), w8[6], acc[r]);
-                    acc[r] = __fmaf_rn(__uint_as_float(xv.w & 0xFFFF0000u), w8[7], acc[r]);
+            for (int u = 0; u < U; ++u)
+                wv[u] = kb + 256 * u < K ? __ldcs(reinterpret_cast<const uint4 *>(wr + kb + 256 * u))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = kb + 256 * u;
+                if (k >= K) break;
+                float w8[8];
+                w8[0] = __uint_as_float(wv[u].x << 16); w8[1] = __uint_as_float(wv[u].x & 0xFFFF0000u);
+                w8[2] = __uint_as_float(wv[u].y << 16); w8[3] = __uint_as_float(wv[u].y & 0xFFFF0000u);
+                w8[4] = __uint_as_float(wv[u].z << 16); w8[5] = __uint_as_float(wv[u].z & 0xFFFF0000u);
+                w8[6] = __uint_as_float(wv[u].w << 16); w8[7] = __uint_as_float(wv[u].w & 0xFFFF0000u);
+#pragma unroll
+                for (int r = 0; r < MB; ++r) {
+                    if (r < mb) {
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(sx + r * K + k);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.x << 16), w8[0], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.x & 0xFFFF0000u), w8[1], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.y << 16), w8[2], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.y & 0xFFFF0000u), w8[3], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.z << 16), w8[4], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.z & 0xFFFF0000u), w8[5], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.w << 16), w8[6], acc[r]);
+                        acc[r] = __fmaf_rn(__uint_as_float(xv.w & 0xFFFF0000u), w8[7], acc[r]);
+                    }
                 }
             }
         }
 #pragma unroll
         for (int r = 0; r < MB; ++r) {
+            if (r < mb) {  // warp-uniform
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc[r] = __fadd_rn(acc[r], __shfl_xor_sync(0xffffffffu, acc[r], o));
+                for (int o = 16; o > 0; o >>= 1) acc[r] = __fadd_rn(acc[r], __shfl_xor_sync(0xffffffffu, acc[r], o));
+            }
         }
         if (lane < mb) {
             float v = acc[0];
@@ -314,10 +327,15 @@ gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M,
 
 int gemv_segs(const uint16_t *x, int ldx, const GemvSegs &segs, int M, int K, cudaStream_t s) {
     const int bytes = std::min(M, kGemvRows) * K * 2;  // the rows of one group
-    static std::atomic<unsigned long long> attr_done{0};  // opted in once, at the largest K
-    KDA_TRY(smem_opt_in(gemv_kernel<kGemvRows>, kGemvRows * kGemvMaxK * 2, attr_done));
+    static std::atomic<unsigned long long> attr_done{0}, attr1_done{0};  // opted in once, at the largest K
     const int col_blocks = (segs.total + kGemvWarps - 1) / kGemvWarps;
     const int grid_x = std::min(col_blocks, 4 * sm_count());
+    if (M == 1) {  // one row: the same per-output arithmetic without the other rows' registers
+        KDA_TRY(smem_opt_in(gemv_kernel<1>, kGemvMaxK * 2, attr1_done));
+        gemv_kernel<1><<<dim3(grid_x, 1), 32 * kGemvWarps, bytes, s>>>(x, ldx, segs, M, K);
+        return launch_status();
+    }
+    KDA_TRY(smem_opt_in(gemv_kernel<kGemvRows>, kGemvRows * kGemvMaxK * 2, attr_done));
     gemv_kernel<kGemvRows><<<dim3(grid_x, (M + kGemvRows - 1) / kGemvRows), 32 * kGemvWarps, bytes, s>>>(x, ldx, segs,
                                                                                                       M, K);
     return launch_status();
