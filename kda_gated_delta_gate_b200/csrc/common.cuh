@@ -28,8 +28,9 @@ __device__ __forceinline__ float softplus_f32(float x) {
     return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
 
+// 1 / (1 + e^-x), the reciprocal correctly rounded (the same value an IEEE division gives).
 __device__ __forceinline__ float sigmoid_f32(float x) {
-    return 1.0f / (1.0f + expf(-x));
+    return __frcp_rn(1.0f + expf(-x));
 }
 
 // The bounded log-decay gate: -exp(a_log[h]) * softplus(g_raw + dt_bias).

@@ -5,10 +5,12 @@
 // those BF16 values (a second BF16 rounding, as l2_norm_bf16 does on prefill), and the
 // widening to FP32 with the pad rows set to pad_fill.
 //
-// Grid: (ceil(T_pad / 32) token tiles, column blocks of 256 x 8 channels). Thread j of
+// Grid: (ceil(T_pad / 16) token tiles, column blocks of 256 x 8 channels). Thread j of
 // column block c owns the 8 consecutive channels [8 g, 8 g + 8), g = 256 c + j, of the
-// q|k|v row (16-byte loads and stores) and walks the tile's 32 tokens with a sliding
-// window of the 3 previous inputs. The D/8 threads of one head's q (or k) are adjacent
+// q|k|v row (16-byte loads and stores) and walks the tile's 16 tokens with a sliding
+// window of the 3 previous inputs. Short tiles and three CTAs per SM keep enough rows in
+// flight: the kernel is bound by latency and issue, not by the 2 x 16 bytes it moves per
+// token and thread. The D/8 threads of one head's q (or k) are adjacent
 // lanes and reduce the per-token sum of squares with shuffles. The tile-0 block of each
 // column block is the only reader of those channels' carried conv state and, after its
 // reads, the only writer of the new one (the last three inputs).
@@ -17,7 +19,7 @@
 namespace kda {
 namespace {
 
-constexpr int kFrontThreads = 256, kTT = 32;
+constexpr int kFrontThreads = 256, kTT = 16;
 
 __device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
     x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xFFFF0000u);
@@ -30,7 +32,7 @@ __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kFrontThreads) front_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ conv_state,
+__global__ void __launch_bounds__(kFrontThreads, 3) front_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ conv_state,
                                                               const uint16_t *__restrict__ conv_w,
                                                               uint16_t *__restrict__ conv_out, float *__restrict__ qf,
                                                               float *__restrict__ kf, float *__restrict__ vf,
