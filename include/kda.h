@@ -229,7 +229,9 @@ KDA_API int kda_chunk_prefill_graw(const float *q, const float *k, const float *
  * are serialised while they enqueue. Because segments are whole chunks, core and the final state
  * are the same bits as kda_beta + kda_chunk_prefill_fused over all T rows on the device.
  * Errors: KDA_ERR_INVALID_ARG (NULL pointer, T < 0, bad segment_tokens), KDA_ERR_MISALIGNED,
- * KDA_ERR_CAPACITY (device_bytes too small), KDA_ERR_CUDA. */
+ * KDA_ERR_CAPACITY (device_bytes too small), all found before anything is enqueued; KDA_ERR_CUDA
+ * (a runtime call failed part-way: some copies or kernels may be in flight, so synchronise the
+ * device before reading the outputs or reusing device_buffer). */
 KDA_API int kda_chunk_prefill_host(const kda_bf16 *qkv, const kda_bf16 *g_raw, const float *b_logit,
                                    const float *dt_bias, const float *a_log, float *h_state, float *core, int T,
                                    int segment_tokens, void *device_buffer, size_t device_bytes,

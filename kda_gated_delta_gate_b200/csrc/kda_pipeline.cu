@@ -31,15 +31,20 @@ int lanes(Lanes *&out) {
     Lanes &l = g_lanes[dev];
     if (!l.in) {
         const unsigned ef = cudaEventDisableTiming;
-        if (cudaStreamCreateWithFlags(&l.in, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaStreamCreateWithFlags(&l.out, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l.start, ef) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l.landed, ef) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l.computed, ef) != cudaSuccess ||
-            cudaEventCreateWithFlags(&l.drained, ef) != cudaSuccess) {
-            l = Lanes{};
+        Lanes n;
+        if (cudaStreamCreateWithFlags(&n.in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&n.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&n.start, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&n.landed, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&n.computed, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&n.drained, ef) != cudaSuccess) {
+            for (cudaEvent_t e : {n.start, n.landed, n.computed, n.drained})
+                if (e) cudaEventDestroy(e);
+            if (n.in) cudaStreamDestroy(n.in);
+            if (n.out) cudaStreamDestroy(n.out);
             return KDA_ERR_CUDA;
         }
+        l = n;
     }
     out = &l;
     return KDA_OK;
