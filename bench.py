@@ -13,7 +13,9 @@ Multi-GPU: each rank runs its own independent sequence (weak scaling, no collect
 
 Also reported: the dominant kernel's roofline (CUDA events around each launch), a decode
 leg (256 sequences x 1 token, kda_decode_fused, state GB/s), an end-to-end leg through
-kda_chunk_prefill_host from pinned host buffers (copies inside the timed region), and the
+kda_chunk_prefill_host from pinned host buffers (copies inside the timed region), the block
+(prefill with a per-stage split, its GEMM, block decode), 4 streams x 65500 tokens of prefill
+(inputs larger than L2), and the
 FP64 oracle timed on the host cores (`cpu_baseline`). `--impl reference` times the oracle
 alone (it is this project's reference implementation) and prints its own line.
 """
@@ -175,6 +177,7 @@ def main():
     ap.add_argument("--prefill-impl", default="tc", choices=["tc", "graw", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-block", action="store_true", help="skip the block-prefill leg")
+    ap.add_argument("--no-long", action="store_true", help="skip the 4 x 65500-token prefill leg")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -274,6 +277,11 @@ def main():
     # ---- the full block (projections + front end + core + back end) and its dominant GEMM
     blk = None if args.no_block else _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm)
 
+    # ---- long multi-stream prefill: 4 streams x 65500 tokens (T_pad 65536)
+    del q, k, v, g_raw, b_logit, gate, beta, core, scratch
+    torch.cuda.empty_cache()
+    long_leg = None if args.no_long else _long_leg(kda, torch, dev, s, stream, hbm, tc_peak, rank)
+
     result = None
     if rank == 0:
         tokens_per_s = world * B * T / (step_ms * 1e-3)
@@ -297,6 +305,7 @@ def main():
                                     "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
             "decode": dec,
             "block_prefill": blk,
+            "long_prefill": long_leg,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "gpu_launches": launches,
@@ -407,6 +416,50 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
             "gemm": {"shape": "8192x4096x4096 bf16->bf16", "ms": gms, "tflops": gflop / (gms * 1e-3) / 1e12,
                      "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak},
             "block_decode": dec}
+
+
+def _long_leg(kda, torch, dev, s, stream, hbm, tc_peak, rank):
+    """kda_gate + kda_beta + kda_chunk_prefill on 4 equal-length streams of 65500 tokens (T_pad
+    65536), H 32, D 128, FP32 I/O; the inputs (about 21 GB) are far larger than L2, so no flush."""
+    from synth import core_inputs, pad_rows, t_pad
+    Bl, Tl = 4, 65500
+    d = kda.dims(H, D)
+    Tp = t_pad(Tl)
+    ci = core_inputs(Bl, Tl, H, D, seed=4 + 1000 * rank, bf16_inputs=True, s0_std=0.1, device=dev)
+    q, k, v = (pad_rows(x, Tp, 0.0) for x in (ci.q, ci.k, ci.v))
+    g_raw = pad_rows(ci.g_raw, Tp, 0.0)
+    b_logit = pad_rows(ci.b_logit, Tp, 0.0)
+    dt_bias, a_log = ci.dt_bias, ci.a_log
+    states = [ci.s0[b].clone() for b in range(Bl)]
+    del ci
+    ptrs = kda.ptr_array(states, device=dev)
+    gate = torch.empty((Bl * Tp, H, D), device=dev)
+    beta = torch.empty((Bl * Tp, H), device=dev)
+    core = torch.empty((Bl * Tp, H, D), device=dev)
+    scratch = torch.empty(kda.kda_chunk_prefill_scratch_bytes(Bl, Tl, d), dtype=torch.uint8, device=dev)
+    steps, kms = [], []
+    for i in range(3 + 5):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        kda.kda_gate(g_raw, dt_bias, a_log, gate, Bl * Tp, d, s)
+        kda.kda_beta(b_logit, beta, Bl * Tp * H, s)
+        e[1].record(stream)
+        kda.kda_chunk_prefill(q, k, v, gate, beta, ptrs, core, Bl, Tl, d, s, scratch=scratch)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            steps.append(e[0].elapsed_time(e[2]))
+            kms.append(e[1].elapsed_time(e[2]))
+    ms, kern = statistics.median(steps), statistics.median(kms)
+    alg = Bl * Tl * H * BYTES_PER_TOKEN_HEAD["tc"] + 2 * Bl * H * D * D * 4
+    flops = Bl * Tl * H * FLOPS_PER_TOKEN_HEAD
+    del q, k, v, g_raw, b_logit, gate, beta, core, scratch, states
+    torch.cuda.empty_cache()
+    return {"workload": "kda_gate + kda_beta + kda_chunk_prefill, 4 streams x 65500 tokens (T_pad 65536), H32 D128, "
+                        "FP32 I/O; inputs larger than L2",
+            "ms_per_step": ms, "tokens_per_s": Bl * Tl / (ms * 1e-3), "kernel_ms": kern,
+            "hbm_frac": alg / (kern * 1e-3) / 1e9 / hbm, "tensor_frac": flops / (kern * 1e-3) / 1e12 / tc_peak,
+            "alg_bytes": alg}
 
 
 def _block_stages(kda, torch, dev, s, stream, flush, Wt, hid, ws, Tb, hidden, Hh, Dd, rank, reps=6):
