@@ -19,7 +19,7 @@ beta = sigmoid(b_proj(h)), and the core is the gated delta rule implemented in
 kda_recurrence.c. All accumulation is FP64; BF16 rounding (round-to-nearest-even) is
 applied exactly at the storage points the workspace page lists.
 
-Readings of points the pages leave open are listed in the design doc of the repository.
+Where the pages leave a point open, the function that depends on it states the reading taken.
 """
 from __future__ import annotations
 
