@@ -396,11 +396,17 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
     ph1, pc1 = kda.ptr_array([hs_b[0]], device=dev), kda.ptr_array([cs_b[0]], device=dev)
     phn, pcn = kda.ptr_array(list(hs_b), device=dev), kda.ptr_array(list(cs_b), device=dev)
     ms1 = timed(lambda: kda.kda_block_decode(st, hid[:1], 1, ph1, pc1, ws, s))
+    graph = kda.kda_block_decode_graph(st, hid[:1], 1, ph1, pc1, ws)  # the same call, replayed
+    ms1g = timed(lambda: graph.launch(s))
+    graph.close()
     msk = timed(lambda: kda.kda_block_decode_k(st, hid[:4], 4, hs_b[1], cs_b[1], [], [], ws, s))
     msn = timed(lambda: kda.kda_block_decode(st, hid[:n_b], n_b, phn, pcn, ws, s))
     dec = {"one_token": {"ms": ms1, "tokens_per_s": 1 / (ms1 * 1e-3),
                          "gbs": (wbytes + sbytes) / (ms1 * 1e-3) / 1e9,
                          "frac_hbm": (wbytes + sbytes) / (ms1 * 1e-3) / 1e9 / hbm},
+           "one_token_graph": {"ms": ms1g, "tokens_per_s": 1 / (ms1g * 1e-3),
+                               "frac_hbm": (wbytes + sbytes) / (ms1g * 1e-3) / 1e9 / hbm,
+                               "call": "kda_block_decode_graph once, kda_graph_launch per step"},
            "decode_k4": {"ms": msk, "tokens_per_s": 4 / (msk * 1e-3),
                          "gbs": (wbytes + sbytes) / (msk * 1e-3) / 1e9},
            "batch256": {"ms": msn, "tokens_per_s": n_b / (msn * 1e-3),

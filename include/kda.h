@@ -469,6 +469,26 @@ KDA_API int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidde
                                kda_bf16 *conv_state, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
                                kda_workspace *ws, void *stream);
 
+/* kda_block_decode_graph — kda_block_decode recorded once into a CUDA graph and instantiated,
+ * for a serving loop that decodes the same N sequences from the same buffers every step: each
+ * kda_graph_launch replays the call's kernels with one launch (the pages' engine has CUDA-graph
+ * hooks; this is the block-level one). Recording runs nothing: no state changes. The graph
+ * keeps the values the call would pass to its kernels: the pointers hidden, h_state,
+ * conv_state, the weights in *w and the workspace buffers, and N. Each replay reads the
+ * CURRENT contents of those buffers (new hidden rows, the advanced states), so they must stay
+ * allocated and in place while the graph lives; the workspace must not be destroyed first.
+ * Arguments and errors as kda_block_decode; KDA_ERR_CUDA if recording or instantiation fails.
+ * *out receives the graph (NULL on error); release it with kda_graph_destroy. */
+typedef struct kda_graph kda_graph;
+KDA_API int kda_block_decode_graph(const kda_block_weights *w, const kda_bf16 *hidden, int N, float *const *h_state,
+                                   kda_bf16 *const *conv_state, kda_workspace *ws, kda_graph **out);
+
+/* Replay a recorded graph on `stream` (asynchronous, like the call it replaces). */
+KDA_API int kda_graph_launch(kda_graph *g, void *stream);
+
+/* Release a graph (NULL is a no-op). Do not destroy a graph whose replay may still run. */
+KDA_API int kda_graph_destroy(kda_graph *g);
+
 #ifdef __cplusplus
 }
 #endif

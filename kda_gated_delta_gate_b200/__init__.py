@@ -89,6 +89,9 @@ _SIGS = {
     "kda_block_decode": ([_VP, _VP, _I, _VP, _VP, _VP, _VP], _I),
     "kda_gemv_bf16": ([_VP, _I, _VP, _I, _VP, _I, _I, _I, _I, _I, _VP], _I),
     "kda_block_decode_k": ([_VP, _VP, _I, _VP, _VP, _VP, _VP, _I, _VP, _VP], _I),
+    "kda_block_decode_graph": ([_VP, _VP, _I, _VP, _VP, _VP, ctypes.POINTER(_VP)], _I),
+    "kda_graph_launch": ([_VP, _VP], _I),
+    "kda_graph_destroy": ([_VP], _I),
 }
 
 
@@ -407,3 +410,35 @@ def kda_chunk_verify_fold(k, cu_seqlens, accepted, B: int, total_tokens: int, ta
     """Advance every state by its accepted rows (device int32 [B]) from the verify tables."""
     return _call("kda_chunk_verify_fold", _p(k), _p(cu_seqlens), _p(accepted), B, total_tokens, _p(tables),
                  _p(h_state_ptrs), ctypes.byref(d), _stream(stream))
+
+
+class Graph:
+    """A recorded kda_block_decode (kda_block_decode_graph); launch() replays it."""
+
+    def __init__(self, handle):
+        self._h = handle
+
+    def launch(self, stream=None):
+        _call("kda_graph_launch", self._h, _stream(stream))
+
+    def close(self):
+        if self._h:
+            lib().kda_graph_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def kda_block_decode_graph(weights: KdaBlockWeights, hidden, N: int, h_state_ptrs, conv_state_ptrs,
+                           ws: Workspace) -> Graph:
+    """Record kda_block_decode of N rows into a CUDA graph (nothing runs). The graph keeps the
+    buffers' addresses: keep `weights`' tensors, hidden, the states, the pointer arrays and `ws`
+    alive and in place while it is used."""
+    h = ctypes.c_void_p()
+    _call("kda_block_decode_graph", ctypes.byref(weights), _p(hidden), N, _p(h_state_ptrs), _p(conv_state_ptrs),
+          ws.handle, ctypes.byref(h))
+    return Graph(h)

@@ -114,6 +114,16 @@ def test_host_prefill_argument_checks(L):
     assert L.kda_chunk_prefill_host(*args, 100, 64, BOGUS, need, ctypes.byref(_d(head_dim=96)), None) == 4
 
 
+def test_graph_argument_checks(L):
+    out = ctypes.c_void_p(BOGUS)
+    assert L.kda_block_decode_graph(BOGUS, BOGUS, 1, BOGUS, BOGUS, BOGUS, None) == 1
+    assert L.kda_block_decode_graph(BOGUS, BOGUS, 0, BOGUS, BOGUS, BOGUS, ctypes.byref(out)) == 1
+    assert out.value is None  # cleared on error
+    assert L.kda_block_decode_graph(None, BOGUS, 1, BOGUS, BOGUS, BOGUS, ctypes.byref(out)) == 1
+    assert L.kda_graph_launch(None, None) == 1
+    assert L.kda_graph_destroy(None) == 0
+
+
 def test_front_back_argument_checks(L):
     d = ctypes.byref(_d())
     assert L.kda_front_conv_silu_l2(BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, None, None, 0.0, 8, d, None) == 1

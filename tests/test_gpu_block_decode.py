@@ -51,6 +51,48 @@ def test_block_decode_matches_oracle(hidden, H, D, rank, N, std):
     ws.close()
 
 
+@pytest.mark.parametrize("hidden,H,D,rank,N", [(256, 2, 64, 64, 3), (4096, 32, 128, 128, 1)])
+def test_block_decode_graph_replays_the_call(hidden, H, D, rank, N):
+    """kda_block_decode_graph records one kda_block_decode (recording runs nothing); three
+    replays with new hidden rows each time give the same bits as three direct calls on a copy
+    of the same states (outputs, states and conv states)."""
+    Wt = block_weights(hidden, H, D, rank, seed=13, std=0.02)
+    hs, cs = _states(N, H, D, seed=13)
+    dw = _device_weights(Wt)
+    st = kda.block_weights_struct(dw)
+    steps = [block_hidden(N, hidden, seed=20 + i).cuda() for i in range(3)]
+    # direct calls
+    ws_a = kda.Workspace(kda.dims(H, D), hidden, rank, max_tokens=8)
+    ha = [hs[n].cuda().clone() for n in range(N)]
+    ca = [cs[n].cuda().clone() for n in range(N)]
+    pa, pca = kda.ptr_array(ha), kda.ptr_array(ca)
+    outs_a = []
+    for x in steps:
+        kda.kda_block_decode(st, x, N, pa, pca, ws_a)
+        outs_a.append(ws_a.view("final_out", (N, hidden), torch.bfloat16).clone())
+    # recorded once, replayed with the hidden buffer refilled between replays
+    ws_b = kda.Workspace(kda.dims(H, D), hidden, rank, max_tokens=8)
+    hb = [hs[n].cuda().clone() for n in range(N)]
+    cb = [cs[n].cuda().clone() for n in range(N)]
+    pb, pcb = kda.ptr_array(hb), kda.ptr_array(cb)
+    xin = torch.empty_like(steps[0])
+    graph = kda.kda_block_decode_graph(st, xin, N, pb, pcb, ws_b)
+    torch.cuda.synchronize()
+    assert all(torch.equal(hb[n], hs[n].cuda()) for n in range(N)), "recording changed a state"
+    outs_b = []
+    for x in steps:
+        xin.copy_(x)
+        graph.launch()
+        outs_b.append(ws_b.view("final_out", (N, hidden), torch.bfloat16).clone())
+    torch.cuda.synchronize()
+    for a_, b_ in zip(outs_a, outs_b):
+        assert torch.equal(a_, b_)
+    assert all(torch.equal(ha[n], hb[n]) and torch.equal(ca[n], cb[n]) for n in range(N))
+    graph.close()
+    ws_a.close()
+    ws_b.close()
+
+
 @pytest.mark.parametrize("hidden,H,D,rank,K,std", [(256, 2, 64, 64, 5, 0.05), (4096, 32, 128, 128, 4, 0.02)])
 def test_block_decode_k_bit_identical_to_serial_block_decodes(hidden, H, D, rank, K, std):
     Wt = block_weights(hidden, H, D, rank, seed=11, std=std)
