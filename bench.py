@@ -12,7 +12,8 @@ outside the timed events.
 Multi-GPU: each rank runs its own independent sequence (weak scaling, no collective).
 
 Also reported: the dominant kernel's roofline (CUDA events around each launch), a decode
-leg (256 sequences x 1 token, kda_decode_fused, state GB/s), an end-to-end leg through
+leg (256 sequences x 1 token, kda_decode_fused, state GB/s), the same prefill in the
+fused-input mode (kda_chunk_prefill_fused on BF16 rows), an end-to-end leg through
 kda_chunk_prefill_host from pinned host buffers (copies inside the timed region), the block
 (prefill with a per-stage split, its GEMM, block decode), 4 streams x 65500 tokens of prefill
 (inputs larger than L2), and the
@@ -271,6 +272,9 @@ def main():
     # ---- decode leg: 256 sequences x 1 token, fused stateful row (state GB/s)
     dec = _decode_leg(kda, torch, dev, s, stream, flush, hbm)
 
+    # ---- the same workload in the fused-input mode (BF16 q|k|v rows + g_raw, gate in-kernel)
+    fused = _fused_leg(kda, torch, dev, s, stream, flush, d, ci, Tp, hbm, tc_peak, scratch)
+
     # ---- end-to-end leg: kda_chunk_prefill_host from pinned host buffers, copies timed
     e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch)
 
@@ -304,6 +308,7 @@ def main():
                          "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                                     "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
             "decode": dec,
+            "fused_input": fused,
             "block_prefill": blk,
             "long_prefill": long_leg,
             "e2e": e2e,
@@ -422,6 +427,39 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
             "gemm": {"shape": "8192x4096x4096 bf16->bf16", "ms": gms, "tflops": gflop / (gms * 1e-3) / 1e12,
                      "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak},
             "block_decode": dec}
+
+
+def _fused_leg(kda, torch, dev, s, stream, flush, d, ci, Tp, hbm, tc_peak, scratch):
+    """The headline workload through kda_chunk_prefill_fused: BF16 q|k|v rows (the front end's
+    conv_out layout) and BF16 g_raw in, the gate formed in the kernel, FP32 beta (kda_beta's
+    output), FP32 core and state out; L2 flushed before every call. Algorithmic bytes per
+    token-head: q, k, v and g_raw at D BF16 values each, beta 4 B, core D FP32 values."""
+    from synth import pad_rows
+    qkv = torch.cat([ci.q.reshape(B, T, H * D), ci.k.reshape(B, T, H * D), ci.v.reshape(B, T, H * D)], dim=-1)
+    qkv = pad_rows(qkv.to(torch.bfloat16), Tp, 0.0).to(dev)
+    g_raw = pad_rows(ci.g_raw, Tp, 0.0).to(dev)
+    beta = pad_rows(ci.b_logit, Tp, 0.0).to(dev)
+    kda.kda_beta(beta, beta, beta.numel(), s)
+    dt_bias, a_log = ci.dt_bias.to(dev), ci.a_log.to(dev)
+    state = ci.s0[0].to(dev).clone()
+    ptrs = kda.ptr_array([state], device=dev)
+    core = torch.empty((B * Tp, H, D), device=dev)
+    ts = []
+    for i in range(3 + 20):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        kda.kda_chunk_prefill_fused(qkv, g_raw, dt_bias, a_log, beta, ptrs, core, B, T, d, s, scratch=scratch)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(a.elapsed_time(b))
+    ms = statistics.median(ts)
+    alg = B * T * H * (3 * D * 2 + D * 2 + 4 + D * 4) + 2 * B * H * D * D * 4
+    flops = B * T * H * FLOPS_PER_TOKEN_HEAD
+    return {"workload": "kda_chunk_prefill_fused B1 T4096 H32 D128 (BF16 q|k|v rows and g_raw in, FP32 core out)",
+            "kernel_ms": ms, "tokens_per_s": B * T / (ms * 1e-3), "alg_bytes_per_launch": alg,
+            "hbm_frac": alg / (ms * 1e-3) / 1e9 / hbm, "tensor_frac": flops / (ms * 1e-3) / 1e12 / tc_peak}
 
 
 def _long_leg(kda, torch, dev, s, stream, hbm, tc_peak, rank):
