@@ -17,7 +17,10 @@
  *
  * Conventions for every entry point:
  *   - Pointers are DEVICE pointers owned by the caller unless a comment says "host".
- *     Nothing is allocated on these calls (the workspace is sized once, at creation).
+ *     No compute call allocates device memory: the workspace is sized once, at creation,
+ *     and scratch buffers are the caller's. The only other objects created are the graph
+ *     kda_block_decode_graph returns and, on the first kda_chunk_prefill_host call on a
+ *     device, that call's two copy streams and four events (kept for the process).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *     Calls are asynchronous: they enqueue kernels and return.
  *   - Return value: KDA_OK, or an error code from the list below. Argument errors are
