@@ -80,8 +80,11 @@ def test_decode_fused_matches_oracle(N, H, D):
     assert np.array_equal(np64(torch.stack(cs)), r_cs)
 
 
-def test_decode_k_bit_identical_to_serial_decodes():
-    H, D, K = 32, 128, 4
+@pytest.mark.parametrize("K", [4, 32])
+def test_decode_k_bit_identical_to_serial_decodes(K):
+    """K rows in one decode_k call (the largest K included: 31 snapshots) give the bits of K
+    serial one-row decodes."""
+    H, D = 32, 128
     di = decode_inputs(1, H, D, seed=3, K=K)
     d = kda.dims(H, D)
     dv = _dev(di)

@@ -310,6 +310,71 @@ def test_varlen_prefill_matches_per_sequence_path_and_oracle(lens, H, D):
         start += L
 
 
+def test_varlen_many_sequences_and_batched_verify_at_serving_shapes():
+    """64 packed sequences of mixed lengths (0..300 tokens) through the varlen prefill, then
+    256 sequences x 4 draft rows through the batched verify and fold (H 32, D 128): sampled
+    sequences bit-identical to the per-sequence path; every verify row equal to the varlen
+    prefill's; the folded states equal to the prefill of the accepted rows (sampled) and the
+    oracle's."""
+    from synth.inputs import CoreInputs
+    rng = np.random.default_rng(7)
+    lens = [int(x) for x in rng.integers(0, 301, size=64)]
+    lens[3] = 0
+    lens[10] = 300
+    H, D = 4, 128
+    ci, s0, dev, gate, beta, cu, d = _varlen_case(lens, H, D, seed=120)
+    total, B = sum(lens), len(lens)
+    states = [s0[b].cuda().clone() for b in range(B)]
+    core = torch.full((total, H, D), float("nan"), device="cuda")
+    kda.kda_chunk_prefill_varlen(dev["q"], dev["k"], dev["v"], gate, beta, cu, B, 5, total, kda.ptr_array(states),
+                                 core, d)
+    torch.cuda.synchronize()
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    for b in [0, 3, 10, 33, 63]:
+        L, st = lens[b], int(starts[b])
+        if L == 0:
+            assert torch.equal(states[b], s0[b].cuda())
+            continue
+        sl = slice(st, st + L)
+        one = CoreInputs(1, L, H, D, ci.q[:, sl], ci.k[:, sl], ci.v[:, sl], ci.g_raw[:, sl], ci.dt_bias, ci.a_log,
+                         ci.b_logit[:, sl], s0[b:b + 1])
+        c1, S1, _ = gpu_prefill(one)
+        assert torch.equal(core[sl], c1[0]) and torch.equal(states[b], S1[0]), b
+    # batched verify: 256 sequences x 4 rows, H 32
+    H, D, Bv, K = 32, 128, 256, 4
+    vlens = [K] * Bv
+    ci, s0, dev, gate, beta, cu, d = _varlen_case(vlens, H, D, seed=121)
+    total = Bv * K
+    states = [s0[b].cuda().clone() for b in range(Bv)]
+    ptrs = kda.ptr_array(states)
+    core = torch.full((total, H, D), float("nan"), device="cuda")
+    tables = torch.empty(kda.kda_chunk_verify_tables_bytes(Bv, d) // 4, device="cuda")
+    kda.kda_chunk_verify(dev["q"], dev["k"], dev["v"], gate, beta, cu, Bv, total, ptrs, core, tables, d)
+    fresh = [s0[b].cuda().clone() for b in range(Bv)]
+    core_p = torch.full((total, H, D), float("nan"), device="cuda")
+    kda.kda_chunk_prefill_varlen(dev["q"], dev["k"], dev["v"], gate, beta, cu, Bv, 1, total, kda.ptr_array(fresh),
+                                 core_p, d)
+    torch.cuda.synchronize()
+    assert torch.equal(core, core_p)
+    assert all(torch.equal(states[b], s0[b].cuda()) for b in range(0, Bv, 17))
+    accepted = [int(x) for x in rng.integers(0, K + 1, size=Bv)]
+    kda.kda_chunk_verify_fold(dev["k"], cu, torch.tensor(accepted, dtype=torch.int32, device="cuda"), Bv, total,
+                              tables, ptrs, d)
+    torch.cuda.synchronize()
+    for b in [0, 1, 100, 255]:
+        r, st = accepted[b], b * K
+        if r == 0:
+            assert torch.equal(states[b], s0[b].cuda())
+            continue
+        sl = slice(st, st + r)
+        one = CoreInputs(1, r, H, D, ci.q[:, sl], ci.k[:, sl], ci.v[:, sl], ci.g_raw[:, sl], ci.dt_bias, ci.a_log,
+                         ci.b_logit[:, sl], s0[b:b + 1])
+        _, S1, _ = gpu_prefill(one)
+        assert rel_l2(np64(states[b]), np64(S1[0])) <= 1e-5, b
+        _, S_ref = oracle_prefill(one)
+        assert rel_l2(np64(states[b]), S_ref[0]) <= TOL, b
+
+
 def test_varlen_prefill_rejects_a_sequence_longer_than_its_slots():
     """With max_num_chunks = 1 a 100-token sequence does not fit: it is skipped, its state left
     as it was, and KDA_ERR_INVALID_ARG is latched; the 50-token sequence beside it is exact."""
