@@ -60,3 +60,46 @@ def chunked_wy(q, k, v, g, beta, s0, scale=1.0, C=64):
         o[sl] = scale * ((Q * A) @ S + M @ U)
         S = np.exp(Gam[-1])[:, None] * S + (K * np.exp(Gam[-1][None, :] - Gam)).T @ U
     return o, S
+
+
+def _chunk_terms(Q, K, V, G, b):
+    """The per-chunk WY/UT quantities of chunked_wy: A = e^Gamma, a = e^{Gamma_C}, K-bar =
+    K o e^{Gamma_C - Gamma}, M, W, U~ (the state-independent part of a chunk)."""
+    n = Q.shape[0]
+    Gam = np.cumsum(G, axis=0)
+    diff = Gam[:, None, :] - Gam[None, :, :]
+    lower = np.tril(np.ones((n, n), dtype=bool))
+    E = np.where(lower[:, :, None], np.exp(np.where(lower[:, :, None], diff, 0.0)), 0.0)
+    L = np.tril(b[:, None] * np.einsum("ic,jc,ijc->ij", K, K, E), -1)
+    M = np.einsum("ic,jc,ijc->ij", Q, K, E)
+    A = np.exp(Gam)
+    Tinv = np.linalg.inv(np.eye(n) + L)
+    return dict(QA=Q * A, a=np.exp(Gam[-1]), Kbar=K * np.exp(Gam[-1][None, :] - Gam), M=M,
+                W=Tinv @ (b[:, None] * K * A), Ut=Tinv @ (b[:, None] * V))
+
+
+def chunked_lookahead(q, k, v, g, beta, s0, scale=1.0, C=64):
+    """One head, the chunked form with the inter-chunk chain carried by U instead of S:
+        U_{c+1} = U~_{c+1} - W_{c+1} (a_c o S_c) - Z_{c+1} U_c,   Z_{c+1} = W_{c+1} K-bar_c^T,
+    where the state update S_{c+1} = a_c o S_c + K-bar_c^T U_c and the product W_{c+1}(a_c o S_c)
+    both use S_c, one step behind the chain (a state pass built this way has one dependent
+    product and one epilogue per chunk on its critical path). Shapes as brute_force."""
+    T, D = q.shape
+    ch = [_chunk_terms(q[n0:n0 + C], k[n0:n0 + C], v[n0:n0 + C], g[n0:n0 + C], beta[n0:n0 + C])
+          for n0 in range(0, T, C)]
+    S = np.array(s0, dtype=np.float64, copy=True)
+    o = np.zeros((T, D))
+    U = ch[0]["Ut"] - ch[0]["W"] @ S
+    for c, t in enumerate(ch):
+        n0 = c * C
+        o[n0:n0 + t["M"].shape[0]] = scale * (t["QA"] @ S + t["M"] @ U)
+        aS = t["a"][:, None] * S
+        if c + 1 < len(ch):
+            nx = ch[c + 1]
+            Z = nx["W"] @ t["Kbar"].T
+            U_next = nx["Ut"] - nx["W"] @ aS - Z @ U
+        S = aS + t["Kbar"].T @ U
+        if c + 1 < len(ch):
+            U = U_next
+    return o, S
+

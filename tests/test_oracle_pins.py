@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from synth import core_inputs
-from tests.kda_forms import brute_force, chunked_wy
+from tests.kda_forms import brute_force, chunked_lookahead, chunked_wy
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -184,6 +184,18 @@ def test_chunked_equals_recurrent(T, D, C, seed):
     oc, Sc = chunked_wy(*args, scale=0.5, C=C)
     np.testing.assert_allclose(o, oc, rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(S, Sc, rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("T,D,C,seed", [(200, 32, 64, 4), (130, 16, 16, 5), (64, 8, 64, 6)])
+def test_lookahead_chain_equals_chunked_and_recurrent(T, D, C, seed):
+    """The U-carried inter-chunk chain (kda_forms.chunked_lookahead: U_{c+1} from U_c through
+    Z = W_{c+1} K-bar_c^T, the state one step behind) gives the chunked form's and the token
+    recurrence's outputs and final state to FP64 rounding, ragged last chunk included."""
+    args = _rand_head(T, D, seed, g_scale=1.5)
+    o, S = _oracle_head(*args, scale=0.7)
+    ol, Sl = chunked_lookahead(*args, scale=0.7, C=C)
+    np.testing.assert_allclose(ol, o, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(Sl, S, rtol=1e-9, atol=1e-11)
 
 
 def test_oracle_uses_heads_and_sequences_independently():
