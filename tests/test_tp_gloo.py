@@ -2,11 +2,12 @@
 processes each run the oracle block on their half of the heads (kda_gated_delta_gate_b200.tp
 shards the weights), multiply by their o_proj slice, and all-reduce the partial outputs; the
 sum equals the unsharded block's output. This covers the sharding and the collective on the
-host (world size 2); the GPU kernels on the shards are tested in test_gpu_tp.py."""
+host (world sizes 2 and 4); the GPU kernels on the shards are tested in test_gpu_tp.py."""
 import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -52,14 +53,15 @@ def _rank_main(rank: int, world: int, port: int, out_dir: str):
         dist.destroy_process_group()
 
 
-def test_head_sharded_block_all_reduce_matches_unsharded(tmp_path):
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_sharded_block_all_reduce_matches_unsharded(tmp_path, world):
+    """world = 4 leaves one head per rank."""
     port = _free_port()
-    mp.spawn(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    mp.spawn(_rank_main, args=(world, port, str(tmp_path)), nprocs=world, join=True)
     assert (tmp_path / "ok").exists()
 
 
 def test_shard_rejects_uneven_split():
-    import pytest
     from kda_gated_delta_gate_b200.tp import head_range
     with pytest.raises(ValueError):
         head_range(6, 0, 4)
