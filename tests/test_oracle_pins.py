@@ -9,6 +9,8 @@ import math
 import os
 
 import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import pytest
 import scipy.special
 import torch
@@ -196,6 +198,21 @@ def test_lookahead_chain_equals_chunked_and_recurrent(T, D, C, seed):
     ol, Sl = chunked_lookahead(*args, scale=0.7, C=C)
     np.testing.assert_allclose(ol, o, rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(Sl, S, rtol=1e-9, atol=1e-11)
+
+
+@settings(max_examples=25, deadline=None)
+@given(T=st.integers(1, 90), D=st.sampled_from([1, 2, 5, 8, 16]), C=st.sampled_from([4, 16, 64]),
+       seed=st.integers(0, 2 ** 31 - 1), g_scale=st.floats(0.0, 3.0), scale=st.floats(0.1, 2.0))
+def test_three_forms_agree_on_random_shapes(T, D, C, seed, g_scale, scale):
+    """Property: for any length (ragged chunks included), head size, chunk size, decay strength
+    and read-out scale, the token recurrence (the oracle), the chunked WY/UT form and the
+    U-carried chain give the same outputs and final state to FP64 rounding."""
+    args = _rand_head(T, D, seed, g_scale=g_scale)
+    o, S = _oracle_head(*args, scale=scale)
+    for form in (chunked_wy, chunked_lookahead):
+        of, Sf = form(*args, scale=scale, C=C)
+        np.testing.assert_allclose(of, o, rtol=1e-8, atol=1e-10)
+        np.testing.assert_allclose(Sf, S, rtol=1e-8, atol=1e-10)
 
 
 def test_oracle_uses_heads_and_sequences_independently():
