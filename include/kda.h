@@ -257,7 +257,13 @@ KDA_API size_t kda_chunk_prefill_host_bytes(int T, int segment_tokens, const kda
  *     above the maximum; for head_dim 128, B * heads * ceil(T / 64) > 219 chunks) are
  *     rejected with KDA_ERR_CAPACITY before anything runs.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *     with that device current; make that first call before any stream capture.
+ *     with that device current; make that first call before any stream capture. The lookup
+ *     loads the array's module, which is when its 32 MiB are taken from the device (modules
+ *     load lazily): a call with B == 0 or T == 0 does only this, so an engine that hands all
+ *     free memory to its pools makes one such call per device first (or runs with
+ *     CUDA_MODULE_LOADING=EAGER, which reserves the array when the library loads).
+ *   - The address is cached per device together with the CUDA context it belongs to; after
+ *     a cudaDeviceReset (a new context) the next call looks it up again.
  *   - Every call shares the one array and it keeps the last call's contents. Nothing in it
  *     needs to start at zero (each call writes every tile it later reads), but calls that
  *     overlap on the GPU (different streams, or different host threads) race on it:

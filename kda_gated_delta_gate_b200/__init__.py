@@ -153,6 +153,25 @@ def t_pad(T: int, chunk: int = 64) -> int:
     return int(lib().kda_t_pad(T, chunk))
 
 
+# One scratch buffer per (device, stream), grown on demand and kept: the chunked prefill, varlen
+# and verify wrappers take it when the caller passes no `scratch`, so a hot call allocates only
+# the first time it needs more bytes on that stream. Calls on one stream are ordered, so they may
+# share its buffer; calls on different streams never do.
+_SCRATCH = {}
+
+
+def scratch_buffer(nbytes: int, device, stream_handle: int):
+    """The cached scratch of (device, stream): a uint8 device tensor of at least nbytes."""
+    import torch
+    dev = torch.device(device)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(), int(stream_handle))
+    buf = _SCRATCH.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=dev)
+        _SCRATCH[key] = buf
+    return buf
+
+
 def device_status(clear: bool = True) -> int:
     out = ctypes.c_int(0)
     _call("kda_device_status", ctypes.byref(out), 1 if clear else 0)
@@ -176,43 +195,39 @@ def kda_chunk_prefill_scratch_bytes(B: int, T: int, d: KdaDims) -> int:
 def kda_chunk_prefill(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None,
                       impl: str = "tc", scratch=None):
     """impl "tc": the tensor-core path (needs `scratch`, a device buffer of at least
-    kda_chunk_prefill_scratch_bytes bytes; one is allocated here if None). impl "simt": the
-    CUDA-core path (no scratch)."""
+    kda_chunk_prefill_scratch_bytes bytes; the stream's cached buffer when None). impl "simt":
+    the CUDA-core path (no scratch)."""
     if impl == "simt":
         return _call("kda_chunk_prefill_simt", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core),
                      B, T, ctypes.byref(d), _stream(stream))
-    nbytes = kda_chunk_prefill_scratch_bytes(B, T, d)
+    st = _stream(stream)
     if scratch is None:
-        import torch
-        scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        scratch = scratch_buffer(kda_chunk_prefill_scratch_bytes(B, T, d), core.device, st)
     return _call("kda_chunk_prefill", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(h_state_ptrs), _p(core), B, T,
-                 _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+                 _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d), st)
 
 
 def kda_chunk_prefill_fused(qkv, g_raw, dt_bias, a_log, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims,
                             stream=None, scratch=None):
     """The chunked prefill on the front end's BF16 q|k|v rows and the raw BF16 gate input
     (the gate is formed in the kernel). `scratch` as for kda_chunk_prefill."""
+    st = _stream(stream)
     if scratch is None:
-        import torch
-        need = kda_chunk_prefill_scratch_bytes(B, T, d)
-        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+        scratch = scratch_buffer(kda_chunk_prefill_scratch_bytes(B, T, d), core.device, st)
     return _call("kda_chunk_prefill_fused", _p(qkv), _p(g_raw), _p(dt_bias), _p(a_log), _p(beta), _p(h_state_ptrs),
-                 _p(core), B, T, _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d),
-                 _stream(stream))
+                 _p(core), B, T, _p(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(d), st)
 
 
 def kda_chunk_prefill_graw(q, k, v, g_raw, dt_bias, a_log, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims,
                            stream=None, scratch=None):
     """kda_chunk_prefill on FP32 q, k, v with the gate formed in the kernel from the raw BF16
     g_raw, dt_bias and a_log (bit-identical to kda_gate + kda_chunk_prefill)."""
+    st = _stream(stream)
     if scratch is None:
-        import torch
-        need = kda_chunk_prefill_scratch_bytes(B, T, d)
-        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+        scratch = scratch_buffer(kda_chunk_prefill_scratch_bytes(B, T, d), core.device, st)
     return _call("kda_chunk_prefill_graw", _p(q), _p(k), _p(v), _p(g_raw), _p(dt_bias), _p(a_log), _p(beta),
                  _p(h_state_ptrs), _p(core), B, T, _p(scratch), scratch.numel() * scratch.element_size(),
-                 ctypes.byref(d), _stream(stream))
+                 ctypes.byref(d), st)
 
 
 def kda_chunk_prefill_host_bytes(T: int, segment_tokens: int, d: KdaDims) -> int:
@@ -380,25 +395,25 @@ def kda_gemv_bf16(x, W, y, M: int, N: int, K: int, ldx=None, ldw=None, ldy=None,
 def kda_chunk_prefill_varlen(q, k, v, gate, beta, cu_seqlens, B: int, max_num_chunks: int, total_tokens: int,
                              h_state_ptrs, core, d: KdaDims, stream=None, scratch=None):
     """Chunked prefill over B packed sequences of unequal lengths (cu_seqlens: device int32 [B+1])."""
+    st = _stream(stream)
     if scratch is None:
-        import torch
         need = int(lib().kda_chunk_prefill_varlen_scratch_bytes(B, max_num_chunks, ctypes.byref(d)))
-        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+        scratch = scratch_buffer(need, core.device, st)
     return _call("kda_chunk_prefill_varlen", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(cu_seqlens), B,
                  max_num_chunks, total_tokens, _p(h_state_ptrs), _p(core), _p(scratch),
-                 scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+                 scratch.numel() * scratch.element_size(), ctypes.byref(d), st)
 
 
 def kda_chunk_verify(q, k, v, gate, beta, cu_seqlens, B: int, total_tokens: int, h_state_ptrs, core, tables,
                      d: KdaDims, stream=None, scratch=None):
     """Batched verify: outputs for every draft row, states unchanged, tables kept for the fold."""
+    st = _stream(stream)
     if scratch is None:
-        import torch
         need = int(lib().kda_chunk_prefill_varlen_scratch_bytes(B, 1, ctypes.byref(d)))
-        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=core.device)
+        scratch = scratch_buffer(need, core.device, st)
     return _call("kda_chunk_verify", _p(q), _p(k), _p(v), _p(gate), _p(beta), _p(cu_seqlens), B, total_tokens,
                  _p(h_state_ptrs), _p(core), _p(tables), tables.numel() * tables.element_size(), _p(scratch),
-                 scratch.numel() * scratch.element_size(), ctypes.byref(d), _stream(stream))
+                 scratch.numel() * scratch.element_size(), ctypes.byref(d), st)
 
 
 def kda_chunk_verify_tables_bytes(B: int, d: KdaDims) -> int:

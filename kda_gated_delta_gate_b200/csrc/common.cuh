@@ -79,6 +79,12 @@ int smem_opt_in(K kernel, int bytes, std::atomic<unsigned long long> &done, bool
 // Device address of this device's latched status word (kda_api.cu).
 int *device_status_ptr();
 
+// The calling thread's current CUDA context (the driver's cuCtxGetCurrent, reached through the
+// runtime's entry-point query), or nullptr when there is none or the query fails. A device
+// address cached per device is only valid for the context it was looked up in: after a
+// cudaDeviceReset the device gets a new context and module-scope arrays new addresses.
+void *current_context();
+
 }  // namespace kda
 
 #define KDA_TRY(expr)                        \

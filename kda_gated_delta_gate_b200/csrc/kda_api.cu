@@ -1,5 +1,6 @@
 // Library-wide C-ABI entry points: version, status text, T_pad, latched device status.
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -9,18 +10,38 @@ namespace kda {
 // Kernels that run bounded waits write a KDA_ERR_* code here instead of trapping.
 __device__ int g_device_status;
 
-int *device_status_ptr() {
-    static std::atomic<int *> cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
-    if (dev < 64) {
-        int *p = cache[dev].load(std::memory_order_relaxed);
-        if (p) return p;
+void *current_context() {
+    typedef int (*GetCurrentFn)(void **);
+    static std::atomic<GetCurrentFn> fn{nullptr};
+    GetCurrentFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return nullptr;
+        f = reinterpret_cast<GetCurrentFn>(p);
+        fn.store(f, std::memory_order_release);
     }
+    void *ctx = nullptr;
+    return f(&ctx) == 0 ? ctx : nullptr;
+}
+
+int *device_status_ptr() {
+    // per device: the context the address was looked up in, and the address
+    static std::mutex lock;
+    static void *ctx_of[64] = {};
+    static int *addr_of[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    void *ctx = current_context();  // null before the runtime has made one current
+    std::lock_guard<std::mutex> g(lock);
+    if (addr_of[dev] && ctx && ctx == ctx_of[dev]) return addr_of[dev];
     void *addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return nullptr;
-    if (dev < 64) cache[dev].store(static_cast<int *>(addr), std::memory_order_relaxed);
-    return static_cast<int *>(addr);
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess || !addr) return nullptr;
+    ctx_of[dev] = current_context();  // the lookup made the device's context current
+    addr_of[dev] = static_cast<int *>(addr);
+    return addr_of[dev];
 }
 
 }  // namespace kda

@@ -194,10 +194,12 @@ constexpr int kTPC = C + 4;  // row stride of T (16-byte aligned rows for vector
 //   16 x 16 diagonal blocks by substitution (one thread per column);
 //   32 x 32 halves:  T_21 = -T_22 (L_21 T_11)  from their 16 x 16 blocks;
 //   the whole:       T_21 = -T_22 (L_21 T_11)  from the two 32 x 32 halves.
-// The products run 4 columns per thread (16-byte reads of the right operand). All
-// kIntraThreads threads call it; sTmp holds 1024 floats (16-byte aligned).
+// The products run 4 columns per thread (16-byte reads of the right operand). All NT (>= 256)
+// threads of the block call it; sTmp holds 1024 floats (16-byte aligned).
+template <int NT>
 __device__ __forceinline__ void invert_unit_lower64(const float *__restrict__ sL, float *__restrict__ sT,
                                                     float *__restrict__ sTmp) {
+    static_assert(NT >= 256, "the 32 x 32 products take 256 threads");
     constexpr int PC = kLPC, PT = kTPC;
     const int tid = threadIdx.x;
     auto fma4 = [](float a, const float4 &b, float4 &acc) {
@@ -235,9 +237,9 @@ __device__ __forceinline__ void invert_unit_lower64(const float *__restrict__ sL
         for (int m = 0; m < 16; ++m)
             fma4(sT[(b0 + 16 + i) * PT + b0 + 16 + m], *reinterpret_cast<const float4 *>(sTmp + hh * 256 + m * 16 + c4), x);
         *reinterpret_cast<float4 *>(sT + (b0 + 16 + i) * PT + b0 + c4) = make_float4(-x.x, -x.y, -x.z, -x.w);
-    } else if (tid < 384) {  // the upper-right 32 x 32 block
-        const int e = tid - 128;
-        *reinterpret_cast<float4 *>(sT + (e >> 3) * PT + 32 + 4 * (e & 7)) = zero4;
+    } else {  // the upper-right 32 x 32 block
+        for (int e = tid - 128; e < 256; e += NT - 128)
+            *reinterpret_cast<float4 *>(sT + (e >> 3) * PT + 32 + 4 * (e & 7)) = zero4;
     }
     __syncthreads();
     if (tid < 256) {  // Y = L_LU T_UU, row i, columns 4c..4c+3
@@ -499,7 +501,7 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
         if (i > j) sL[i * PC + j] *= sB[i];
     }
     __syncthreads();
-    invert_unit_lower64(sL, sT, sTmp);
+    invert_unit_lower64<NT>(sL, sT, sTmp);
     // ---- Tb = T diag(beta) in place (lower triangle and diagonal)
     for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, j = e % C;
@@ -561,8 +563,8 @@ intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *_
 
 // ---------------------------------------------------------------- intra-chunk on tensor cores
 //
-// L' and M for all pairs of the chunk in one tcgen05 MMA. Each 16-token block a gets the
-// reference point m_a = 16a + 7 (its middle). With Gamma the in-chunk cumulative decay,
+// L' and M for all pairs of the chunk in one tcgen05 contraction. Each 16-token block a gets
+// the reference point m_a = 16a + 7 (its middle). With Gamma the in-chunk cumulative decay,
 //   A rows  i (block a):      k_i e^{Gamma_i - Gamma_{m_a}}   (and q_i ... for rows 64 + i)
 //   B rows  (a', j), j <= 16a'+15:  k_j e^{Gamma_{m_a'} - Gamma_j}
 // so D[i][(a, j)] = sum_c k_ic k_jc e^{Gamma_ic - Gamma_jc} = L'[i][j] exactly for every j <= i
@@ -570,83 +572,82 @@ intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *_
 // 0, 16, 48, 96 (160 rows). Factors above 1 come only from decay inside one block (at most
 // 8 tokens); a chunk whose |Gamma_i - Gamma_{m_a}| exceeds kRefBound for some channel is
 // handed to the CUDA-core body instead (listed in scratch, run by intra_fix_kernel).
+//
+// Two 256-thread CTAs share an SM (113 KB of shared memory and 256 TMEM columns each), so one
+// CTA's MMA, barrier and load latencies run under the other's CUDA-core work. The L/M operands
+// are built and contracted 64 channels at a time through one 72 KB buffer; q, k and v come
+// straight from global memory (each item's rows are bulk-prefetched into L2 one item ahead);
+// W and U~ leave TMEM straight for the pack.
 
 constexpr float kRefBound = 80.0f;  // e^80 and e^-80 are comfortably inside BF16/FP32 range
+constexpr int kTcThreads = 256;
 
 template <int D>
 struct IntraTC {
-    static constexpr int NB = 160;                   // B rows of the L/M MMA
-    static constexpr int A_BYTES = 2 * 128 * D * 2;  // L/M A operand (hi + lo, K = D); then the
-                                                     // W | U~ B operand [K o A | V] (N = 2D, K = 64)
-    static constexpr int B_BYTES = 2 * NB * D * 2;   // L/M B operand; then L, M, T and the Tb operand;
-                                                     // then the staged W | U~ results
-    static constexpr int PC = kLPC, PT = kTPC;
-    static constexpr int LMT = (2 * C * PC + C * PT) * 4;
-    static constexpr int OFF_TB = (LMT + 1023) / 1024 * 1024;  // Tb, 64 x 64 K-major, hi + lo
-    static constexpr int W_STAGE = 2 * C * D * 2;              // W rows 0..63 of A1, hi + lo panels
-    static constexpr int STAGE = W_STAGE + Pack<D>::UT;
-    static constexpr int R2a = B_BYTES > OFF_TB + 2 * 8192 ? B_BYTES : OFF_TB + 2 * 8192;
-    static constexpr int R2 = R2a > STAGE ? R2a : STAGE;
-    static constexpr int GP = D;                     // g, then Gamma, then v: dense [C][D] rows (TMA boxes)
-    static constexpr int G_BYTES = C * GP * 4;
-    static constexpr int TAB = 14 * D * 4;           // per-channel reference factors
-    static constexpr int MISC = (C + 1024) * 4 + 256;  // beta[C], tmp[1024], barriers, tmem slot
-    static constexpr int OFF_A = 0, OFF_B = A_BYTES, OFF_G = OFF_B + R2, OFF_TAB = OFF_G + G_BYTES,
-                         OFF_MISC = OFF_TAB + TAB;
+    static constexpr int NH = D / 64;             // 64-channel parts of the L/M contraction
+    static constexpr int NB = 160;                // B rows of the L/M MMA
+    static constexpr int A_H = 2 * 128 * 64 * 2;  // L/M A part: 128 rows x 64 channels, hi + lo
+    static constexpr int B_H = 2 * NB * 64 * 2;   // L/M B part: 160 rows x 64 channels, hi + lo
+    static constexpr int R1 = A_H + B_H;          // 72 KB
+    static constexpr int R2 = C * D * 4;          // g / Gamma [C][D] FP32, then the V part of the W|U~ B operand
+    static constexpr int KA = 2 * C * D * 2;      // one [C tokens][D channels] MN-major operand, hi + lo
+    static constexpr int TAB = 14 * D * 4;        // per-channel reference factors
+    static constexpr int OFF_R2 = R1, OFF_TAB = OFF_R2 + R2, OFF_MISC = OFF_TAB + TAB;
+    static constexpr int MISC = C * 4 + 64;       // beta[C], two barriers, TMEM slot
     static constexpr int bytes = OFF_MISC + MISC + 1024;
+    // R1 once the L/M MMA has completed: L, T (FP32), scratch of the inverse, Tb (K-major hi + lo);
+    // then the K o A part of the W|U~ B operand at offset 0 (over the dead L and T)
+    static constexpr int OFF_L = 0, OFF_T = C * kLPC * 4, OFF_TMP = OFF_T + C * kTPC * 4;
+    static constexpr int OFF_TB = (OFF_TMP + 4096 + 1023) / 1024 * 1024;
+    static_assert(OFF_TB + 16384 <= R1, "R1 holds L, T, the inverse's scratch and Tb");
+    static_assert(KA <= OFF_TB, "the K o A operand part must not overlap Tb");
+    static_assert(KA == R2, "the V operand part fills R2");
+    static_assert(2 * (bytes + 1024) <= 233472, "two CTAs per SM");
 };
 
-// One thread: bulk shared -> global copy (bytes a multiple of 16), in this thread's bulk group.
-__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
-                 "r"(bytes)
-                 : "memory");
+__device__ __forceinline__ void ld8f(const float *p, float (&x)[8]) {
+    const float4 a0 = *reinterpret_cast<const float4 *>(p), a1 = *reinterpret_cast<const float4 *>(p + 4);
+    x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w; x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Persistent: gridDim.x CTAs walk the (stream, head, chunk) items; each item's q, k, g and
-// beta are fetched while the previous item finishes (g by a TMA box into shared memory, q and
-// k into registers, v into L2); v itself arrives by a TMA box once g's space is free again,
-// and the W | U~ results leave through shared memory in bulk copies. The g and v boxes come
-// from 3-D maps whose row extent is T, so rows past T arrive as zeros (the pad guard).
+// 16 BF16 hi + lo bytes of 8 values at `off` of a split tile in global memory (hi at dst, lo at dst + half)
+__device__ __forceinline__ void st_pair_g(uint8_t *dst, int half_bytes, uint32_t off, const float (&x)[8]) {
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4 *>(dst + off) = hi;
+    *reinterpret_cast<uint4 *>(dst + half_bytes + off) = lo;
+}
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(kIntraThreads, 1)
-intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmV, const PrefillIn in,
-                uint8_t *__restrict__ scratch, int *__restrict__ list, int B, const Seqs sq, int H,
-                int *__restrict__ status) {
+__global__ void __launch_bounds__(kTcThreads, 2)
+intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uint8_t *__restrict__ scratch,
+                int *__restrict__ list, int B, const Seqs sq, int H, int *__restrict__ status) {
     using I = IntraTC<D>;
     using PK = Pack<D>;
-    constexpr int NT = kIntraThreads, GP = I::GP, PC = I::PC, PT = I::PT;
-    constexpr int CG = D / 8;         // 8-channel groups
-    constexpr int UPT = C * CG / NT;  // (token, group) units per thread: 2 (D=128) or 1
+    constexpr int NT = kTcThreads, PC = kLPC, PT = kTPC, NH = I::NH;
+    constexpr int UB = C * (D / 8) / NT;  // (token, 8-channel group) units per thread over all D channels
+    constexpr bool QKV16 = kQkv16<MODE>, GRAW = kGraw<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = sm + I::OFF_A, *sBt = sm + I::OFF_B, *sTb = sm + I::OFF_B + I::OFF_TB;
-    float *sL = reinterpret_cast<float *>(sm + I::OFF_B);  // after the L/M MMA: L, M, T
-    float *sM = sL + C * PC;
-    float *sT = sM + C * PC;
-    uint8_t *sW = sm + I::OFF_B;                            // after the W | U~ MMA: staged results
-    float *sUt = reinterpret_cast<float *>(sm + I::OFF_B + I::W_STAGE);
-    float *sG = reinterpret_cast<float *>(sm + I::OFF_G);
+    uint8_t *sA = sm, *sBt = sm + I::A_H, *sR2 = sm + I::OFF_R2, *sTb = sm + I::OFF_TB, *sKA = sm;
+    float *sG = reinterpret_cast<float *>(sR2);
+    float *sL = reinterpret_cast<float *>(sm + I::OFF_L);
+    float *sT = reinterpret_cast<float *>(sm + I::OFF_T);
+    float *sTmp = reinterpret_cast<float *>(sm + I::OFF_TMP);
     float *sTab = reinterpret_cast<float *>(sm + I::OFF_TAB);
     float *sB = reinterpret_cast<float *>(sm + I::OFF_MISC);
-    float *sTmp = sB + C;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + (C + 1024) * 4);  // MMA commits
-    uint64_t *gbar = bar + 1, *vbar = bar + 2;                                          // g, v boxes
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 3);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + I::OFF_MISC + C * 4);  // MMA commits
+    uint64_t *gbar = bar + 1;                                                // the g box
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
     // reference tables, [entry][D]: 0..3 e^{Gamma_{m_a}}, 4..7 e^{Gamma_C - Gamma_{m_a}},
     // 8..13 e^{Gamma_{m_a} - Gamma_{m_b}} for (a,b) = (1,0),(2,0),(2,1),(3,0),(3,1),(3,2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nch = sq.nch;
     const int total = B * H * nch;
-    constexpr bool QKV16 = kQkv16<MODE>, GRAW = kGraw<MODE>;
-    constexpr uint32_t kGBox = C * D * (GRAW ? 2 : 4), kVBox = C * D * (QKV16 ? 2 : 4);  // one g / v box
-    // g's box: FP32 g at the start of its space, or BF16 g_raw in the upper half (the gate is
-    // then formed in place, FP32, dense)
-    void *gdst = reinterpret_cast<uint8_t *>(sG) + (GRAW ? C * D * 2 : 0);
-    const int vx0 = QKV16 ? 2 * H * D : 0;  // v's column in the box source
+    constexpr uint32_t kGBox = C * D * (GRAW ? 2 : 4);
+    // g's box: FP32 g at the start of R2, or BF16 g_raw in its upper half (the gate is then
+    // formed in place, FP32, dense)
+    void *gdst = sR2 + (GRAW ? C * D * 2 : 0);
     const size_t rs = static_cast<size_t>(H) * D;
 
     if (warp == 0) {
@@ -656,17 +657,8 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(gbar, 1);
-        mbar_init(vbar, 1);
         fence_mbar_init();
     }
-    auto ld8 = [](const float *p, float (&x)[8]) {
-        const float4 a0 = *reinterpret_cast<const float4 *>(p), a1 = *reinterpret_cast<const float4 *>(p + 4);
-        x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w; x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
-    };
-    // ---- fetch one item's inputs: k, q into registers (zeros past T); g by one TMA box into
-    //      shared memory (thread 0; the caller made the space free); v only into L2; beta into
-    //      a register of threads < C
-    float kk[UPT][8], qq[UPT][8], bnext = 0.f;
     // this CTA's items are blockIdx.x + j gridDim.x; empty chunk slots (varlen) are skipped
     auto next_item = [&](int it) {
         size_t r0;
@@ -682,29 +674,41 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         if (sq.cu) { y = static_cast<int>(row0); z = 0; }
         else { y = ch * C; z = b; }
     };
-    auto fetch = [&](int it) {
+    // an item's q, k, v and g rows into L2: thread (input tid / 64, row tid % 64), one bulk prefetch each
+    auto prefetch = [&](int it) {
         const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
         int n;
         size_t row0;
         seq_chunk(sq, b, ch, row0, n, nullptr);
-#pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
-            if (i < n) {
-                load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, kk[u]);
-                load8_in<D, QKV16>(in, 0, row0 + i, H, h, cb, qq[u]);
-                if ((cb & (QKV16 ? 63 : 31)) == 0) {
-                    const void *vp = QKV16 ? static_cast<const void *>(in.qkv + (row0 + i) * (3 * rs) + 2 * rs +
-                                                                      static_cast<size_t>(h) * D + cb)
-                                           : static_cast<const void *>(in.v + (row0 + i) * rs +
-                                                                      static_cast<size_t>(h) * D + cb);
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(vp));
+        const int part = tid >> 6, i = tid & 63;
+        if (i < n) {
+            const void *p;
+            uint32_t bytes;
+            if (part < 3) {
+                if constexpr (QKV16) {
+                    p = in.qkv + (row0 + i) * (3 * rs) + static_cast<size_t>(part * H + h) * D;
+                    bytes = D * 2;
+                } else {
+                    p = (part == 0 ? in.q : (part == 1 ? in.k : in.v)) + (row0 + i) * rs + static_cast<size_t>(h) * D;
+                    bytes = D * 4;
                 }
+            } else if constexpr (GRAW) {
+                p = in.g_raw + (row0 + i) * rs + static_cast<size_t>(h) * D;
+                bytes = D * 2;
             } else {
-#pragma unroll
-                for (int w = 0; w < 8; ++w) { kk[u][w] = 0.f; qq[u][w] = 0.f; }
+                p = in.gate + (row0 + i) * rs + static_cast<size_t>(h) * D;
+                bytes = D * 4;
             }
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
         }
+    };
+    // an item's g box into R2 (thread 0; the caller made R2 free) and its beta (threads < C)
+    float bnext = 0.f;
+    auto fetch_g = [&](int it) {
+        const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
+        int n;
+        size_t row0;
+        seq_chunk(sq, b, ch, row0, n, nullptr);
         if (tid == 0) {
             int y, z;
             box_yz(ch, b, row0, y, z);
@@ -714,13 +718,28 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         if (tid < C) bnext = tid < n ? in.beta[(row0 + tid) * H + h] : 0.f;
     };
     tc_fence_before();
-    __syncthreads();  // barriers initialised
+    __syncthreads();  // barriers initialised, TMEM allocated
     tc_fence_after();
     const int first = next_item(blockIdx.x);
-    if (first < total) fetch(first);
+    if (first < total) {
+        prefetch(first);
+        fetch_g(first);
+    }
     const uint32_t tmem = *tmem_slot;
-    bool dead = false;  // a wait timed out: hand every remaining item to the CUDA-core body
-    uint32_t iter = 0;  // items done by this CTA: the parity of the g and v boxes
+    bool dead = false;   // a wait timed out: hand every remaining item to the CUDA-core body
+    uint32_t iter = 0;   // items started by this CTA: the parity of the g box
+    uint32_t mph = 0;    // MMA commits waited for: the parity of `bar`
+    // a wait on `b` (phase `par`) gave up: latch the error, give the operation one more bounded
+    // wait (nothing may still write shared memory), list the item for the CUDA-core body
+    auto give_up = [&](uint64_t *b, uint32_t par, int it) {
+        if (tid == 0) {
+            atomicExch(status, KDA_ERR_TIMEOUT);
+            mbar_wait(b, par, kWaitCycles);
+            list[1 + atomicAdd(list, 1)] = it;
+        }
+        dead = true;
+        __syncthreads();
+    };
 
     int following = total;
 #pragma unroll 1
@@ -730,35 +749,25 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
         int n;
         size_t row0;
         seq_chunk(sq, b, ch, row0, n, nullptr);
-        int boxy, boxz;
-        box_yz(ch, b, row0, boxy, boxz);
         uint8_t *pack = scratch + static_cast<size_t>(item) * PK::bytes;
         if (dead) {  // block-uniform
             if (tid == 0) list[1 + atomicAdd(list, 1)] = item;
             continue;
         }
-        const uint32_t par = iter & 1;
-        bool okg = mbar_wait(gbar, par, kWaitCycles);
+        if (following < total) prefetch(following);
+        bool ok = mbar_wait(gbar, iter & 1, kWaitCycles);
         if (tid < C) sB[tid] = bnext;
-        if (tid == 0) bulk_wait_read();  // the previous item's staged results have left
-        okg = __syncthreads_and(okg) != 0;
-        if (!okg) {
-            if (tid == 0) {
-                atomicExch(status, KDA_ERR_TIMEOUT);
-                mbar_wait(gbar, par, kWaitCycles);
-                list[1 + atomicAdd(list, 1)] = item;
-            }
-            dead = true;
-            __syncthreads();
+        if (!__syncthreads_and(ok)) {
+            give_up(gbar, iter & 1, item);
             continue;
         }
         // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, range of tokens)
         {
-            constexpr int QT = NT / D;  // 4 (D=128) or 8 (D=64) token ranges
+            constexpr int QT = NT / D;  // 2 (D=128) or 4 (D=64) token ranges
             constexpr int TPQ = C / QT;
             const int c = tid % D, qr = tid / D;
             if constexpr (GRAW) {
-                // g = -exp(a_log) softplus(g_raw + dt_bias) (0 past T), FP32 over g_raw's box
+                // g = -exp(a_log) softplus(g_raw + dt_bias) (0 past the chunk's end), FP32 over g_raw's box
                 const uint16_t *gr = reinterpret_cast<const uint16_t *>(gdst);
                 float x[TPQ];
 #pragma unroll
@@ -768,30 +777,30 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
 #pragma unroll
                 for (int r = 0; r < TPQ; ++r) {
                     const int i = qr * TPQ + r;
-                    sG[i * GP + c] = i < n ? kda_gate_f32(x[r], dtb, nea) : 0.f;
+                    sG[i * D + c] = i < n ? kda_gate_f32(x[r], dtb, nea) : 0.f;
                 }
             }
             float acc = 0.f;
             for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) {
-                acc += i < n ? sG[i * GP + c] : 0.f;  // rows past the chunk's end decay nothing
-                sG[i * GP + c] = acc;
+                acc += i < n ? sG[i * D + c] : 0.f;  // rows past the chunk's end decay nothing
+                sG[i * D + c] = acc;
             }
             sTmp[qr * D + c] = acc;
             __syncthreads();
             float pre = 0.f;
             for (int r = 0; r < qr; ++r) pre += sTmp[r * D + c];
             if (qr > 0)
-                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * GP + c] += pre;
+                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * D + c] += pre;
             if (in.tables) {  // verify mode: keep Gamma for the fold
                 float *gt = in.tables + ((static_cast<size_t>(b) * H + h) * 2 + 1) * C * D;
-                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) gt[i * D + c] = sG[i * GP + c];
+                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) gt[i * D + c] = sG[i * D + c];
             }
             __syncthreads();
         }
         if (tid < D) {
             const int c = tid;
-            const float gm[4] = {sG[7 * GP + c], sG[23 * GP + c], sG[39 * GP + c], sG[55 * GP + c]};
-            const float gc = sG[63 * GP + c];
+            const float gm[4] = {sG[7 * D + c], sG[23 * D + c], sG[39 * D + c], sG[55 * D + c]};
+            const float gc = sG[63 * D + c];
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
                 sTab[a * D + c] = __expf(gm[a]);
@@ -803,267 +812,250 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__
             sTab[11 * D + c] = __expf(gm[3] - gm[0]);
             sTab[12 * D + c] = __expf(gm[3] - gm[1]);
             sTab[13 * D + c] = __expf(gm[3] - gm[2]);
+            reinterpret_cast<float *>(pack + PK::OFF_AC)[c] = __expf(gc);
         }
         __syncthreads();
-        // ---- one pass over this thread's (token, 8-channel group) units builds the operands of
-        //      the L/M MMA in shared memory, A (mid-block reference) and B (all references),
-        //      and writes the state-independent pack operands: Q o e^Gamma (A1 rows 64..127) and
-        //      K o e^{Gamma_C - Gamma} (A3); K o e^Gamma stays in registers (kk) for W | U~.
-        //      (The pack is written for unsafe chunks too; the CUDA-core body then rewrites it.)
+        // ---- the L/M operands, 64 channels at a time: thread units (token i, 8-channel group),
+        //      A (mid-block reference) and B (all references) in shared memory, and the pack's
+        //      state-independent operands Q o e^Gamma (A1 rows 64..127) and K o e^{Gamma_C - Gamma}
+        //      (A3) written out. (The pack is written for unsafe chunks too; the CUDA-core body
+        //      then rewrites it.)
         bool safe = true;
-#pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG), a = i >> 4;
-            float gi[8], gm[8], ef[8], ei[8], x[8];
-            ld8(sG + i * GP + cb, gi);
-            ld8(sG + (16 * a + 7) * GP + cb, gm);
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                const float r = gi[w] - gm[w];
-                safe = safe && fabsf(r) <= kRefBound;
-                ef[w] = __expf(r);
-                ei[w] = __expf(-r);
+#pragma unroll 1
+        for (int hf = 0; hf < NH; ++hf) {
+            if (hf > 0) {  // the previous part's MMA has finished reading the operand buffer
+                ok = mbar_wait(bar, mph & 1, kWaitCycles);
+                tc_fence_after();
+                ok = __syncthreads_and(ok) != 0;
+                if (!ok) break;
+                ++mph;
             }
 #pragma unroll
-            for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ef[w];
-            st_pair(sA, I::A_BYTES / 2, kmaj_off(i, cb, 128), x);
-#pragma unroll
-            for (int w = 0; w < 8; ++w) x[w] = qq[u][w] * ef[w];
-            st_pair(sA, I::A_BYTES / 2, kmaj_off(64 + i, cb, 128), x);
-            // B rows for every reference block a2 >= a (column offsets 0, 16, 48, 96)
-#pragma unroll
-            for (int a2 = 0; a2 < 4; ++a2) {
-                if (a2 < a) continue;
-                const int off2 = 8 * a2 * (a2 + 1);
-                if (a2 == a) {
-#pragma unroll
-                    for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w];
+            for (int j = 0; j < 2; ++j) {
+                const int u = tid + NT * j, i = u >> 3, cl = 8 * (u & 7), cb = 64 * hf + cl, a = i >> 4;
+                float k8[8], q8[8], gi[8], gm[8], ef[8], ei[8], x[8];
+                if (i < n) {
+                    load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, k8);
+                    load8_in<D, QKV16>(in, 0, row0 + i, H, h, cb, q8);
                 } else {
-                    const int tix = a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13)));
-                    float tb[8];
-                    ld8(sTab + tix * D + cb, tb);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) x[w] = kk[u][w] * ei[w] * tb[w];
+                    for (int w = 0; w < 8; ++w) { k8[w] = 0.f; q8[w] = 0.f; }
                 }
-                st_pair(sBt, I::B_BYTES / 2, kmaj_off(off2 + i, cb, I::NB), x);
-            }
-            // pack operands: e^{Gamma_i} = ef e^{Gamma_m}, e^{Gamma_C - Gamma_i} = ei e^{Gamma_C - Gamma_m}
-            float em[8];
-            ld8(sTab + a * D + cb, em);
+                ld8f(sG + i * D + cb, gi);
+                ld8f(sG + (16 * a + 7) * D + cb, gm);
 #pragma unroll
-            for (int w = 0; w < 8; ++w) ef[w] *= em[w];
-            ld8(sTab + (4 + a) * D + cb, em);
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                ei[w] *= em[w];
-                x[w] = qq[u][w] * ef[w];
-                qq[u][w] = kk[u][w] * ei[w];
-                kk[u][w] *= ef[w];
-            }
-            uint4 hi, lo;
-            split8(x, hi, lo);
-            *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + kmaj_off(64 + i, cb, 128)) = hi;
-            *reinterpret_cast<uint4 *>(pack + PK::OFF_A1 + PK::A1 / 2 + kmaj_off(64 + i, cb, 128)) = lo;
-            split8(qq[u], hi, lo);
-            *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + mnmaj_off(cb, i, C)) = hi;
-            *reinterpret_cast<uint4 *>(pack + PK::OFF_A3 + PK::A3 / 2 + mnmaj_off(cb, i, C)) = lo;
-        }
-        if (tid < D) reinterpret_cast<float *>(pack + PK::OFF_AC)[tid] = sTab[3 * D + tid] * sTab[7 * D + tid];
-        fence_async_smem();
-        tc_fence_before();
-        safe = __syncthreads_and(safe) != 0;
-        tc_fence_after();
-        // ---- v by one TMA box into g's space (Gamma is no longer read), for the W | U~ operand;
-        //      D[128 x 160] = A . B^T (L' in rows 0..63, M in rows 64..127)
-        if (tid == 0) {
-            mbar_expect_tx(vbar, kVBox);
-            tma_load_3d(sG, &tmV, vx0 + h * D, boxy, boxz, vbar);
-            if (safe) {
-                constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
-                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_BYTES / 2, 128, 0, ks);
-                    const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_BYTES / 2, I::NB, 0, ks);
-                    mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
-                    mma_bf16(tmem, ah, bl, id, 1);
-                    mma_bf16(tmem, al, bh, id, 1);
+                for (int w = 0; w < 8; ++w) {
+                    const float r = gi[w] - gm[w];
+                    safe = safe && fabsf(r) <= kRefBound;
+                    ef[w] = __expf(r);
+                    ei[w] = __expf(-r);
                 }
-                mma_commit(bar);
-            }
-        }
-        bool ok = true;
-        if (safe) {
-            ok = mbar_wait(bar, 0, kWaitCycles);
-            tc_fence_after();
-            // ---- read back: warp (quad, part); row r = 32 quad + lane (i = r % 64, block a = i / 16)
-            //      needs columns [off_a, off_a + 16(a+1)); the quad's window is [0, 48) for rows in
-            //      blocks 0-1 and [48, 160) for blocks 2-3, split over the 4 warps of the quad.
-            //      L = diag(beta) L' (strictly lower) and M (lower with diagonal) go to shared memory.
-            if (ok) {
-                const int quad = warp & 3, part = warp >> 2;
-                const int r = 32 * quad + lane, i = r & 63, a = i >> 4;
-                const int off_a = 8 * a * (a + 1);
-                const int w0 = (quad & 1) ? 48 : 0, wlen = (quad & 1) ? 112 : 48;
-                const bool is_l = r < 64;
-                float *dstm = is_l ? sL : sM;
-                const float bi = is_l ? sB[i] : 1.f;
-                for (int c8 = part * 8; c8 < wlen; c8 += 32) {
-                    float x[8];
-                    tmem_ld8(tmem_lane_base(tmem, warp) + w0 + c8, x);
-                    tmem_ld_wait();
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        const int j = w0 + c8 + w - off_a;
-                        if (j >= 0 && (is_l ? j < i : j <= i)) dstm[i * PC + j] = x[w] * bi;
+                for (int w = 0; w < 8; ++w) x[w] = k8[w] * ef[w];
+                st_pair(sA, I::A_H / 2, kmaj_off(i, cl, 128), x);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) x[w] = q8[w] * ef[w];
+                st_pair(sA, I::A_H / 2, kmaj_off(64 + i, cl, 128), x);
+                // B rows for every reference block a2 >= a (column offsets 0, 16, 48, 96)
+#pragma unroll
+                for (int a2 = 0; a2 < 4; ++a2) {
+                    if (a2 < a) continue;
+                    const int off2 = 8 * a2 * (a2 + 1);
+                    if (a2 == a) {
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) x[w] = k8[w] * ei[w];
+                    } else {
+                        const int tix = a2 == 1 ? 8 : (a2 == 2 ? (a == 0 ? 9 : 10) : (a == 0 ? 11 : (a == 1 ? 12 : 13)));
+                        float tb[8];
+                        ld8f(sTab + tix * D + cb, tb);
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) x[w] = k8[w] * ei[w] * tb[w];
                     }
+                    st_pair(sBt, I::B_H / 2, kmaj_off(off2 + i, cl, I::NB), x);
                 }
-            }
-            tc_fence_before();
-        }
-        ok = ok && mbar_wait(vbar, par, kWaitCycles);
-        ok = __syncthreads_and(ok) != 0;
-        const bool run = safe && ok;
-        if (run) {
-            // ---- the W | U~ B operand in the (now free) A region: [K o A | V], MN-major (n = channel
-            //      0..D-1 for K o A, D..2D-1 for V; k = token)
+                // pack operands: e^{Gamma_i} = ef e^{Gamma_m}, e^{Gamma_C - Gamma_i} = ei e^{Gamma_C - Gamma_m}
+                float em[8];
+                ld8f(sTab + a * D + cb, em);
 #pragma unroll
-            for (int u = 0; u < UPT; ++u) {
-                const int e = tid + u * NT, i = e / CG, cb = 8 * (e % CG);
-                float x[8];
-                if constexpr (QKV16) {
-                    const uint4 w4 = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(sG) + i * D + cb);
-                    bf16x2_to_f32(w4.x, x[0], x[1]); bf16x2_to_f32(w4.y, x[2], x[3]);
-                    bf16x2_to_f32(w4.z, x[4], x[5]); bf16x2_to_f32(w4.w, x[6], x[7]);
-                } else {
-                    ld8(sG + i * GP + cb, x);
-                }
-                if (i >= n) {  // rows past the chunk's end: v = 0
+                for (int w = 0; w < 8; ++w) x[w] = q8[w] * (ef[w] * em[w]);
+                st_pair_g(pack + PK::OFF_A1, PK::A1 / 2, kmaj_off(64 + i, cb, 128), x);
+                ld8f(sTab + (4 + a) * D + cb, em);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) x[w] = 0.f;
-                }
-                st_pair(sA, I::A_BYTES / 2, mnmaj_off(cb, i, C), kk[u]);
-                st_pair(sA, I::A_BYTES / 2, mnmaj_off(D + cb, i, C), x);
-            }
-            // ---- M into the pack (64 x 64 K-major, zero above the diagonal)
-            const int r = tid >> 3, c0 = 8 * (tid & 7);
-            float x[8];
-#pragma unroll
-            for (int w = 0; w < 8; ++w) x[w] = c0 + w <= r ? sM[r * PC + c0 + w] : 0.f;
-            uint4 hi, lo;
-            split8(x, hi, lo);
-            *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + kmaj_off(r, c0, 64)) = hi;
-            *reinterpret_cast<uint4 *>(pack + PK::OFF_AM + PK::AM / 2 + kmaj_off(r, c0, 64)) = lo;
-        }
-        // ---- the next item's inputs are fetched while this one finishes (v's space and the k, q
-        //      registers are free; this item's beta is in sB). A timed-out v box is waited for
-        //      once more, so that nothing still writes that space.
-        if (!ok && tid == 0) mbar_wait(vbar, par, kWaitCycles);
-        fence_async_smem();
-        __syncthreads();
-        const bool more = following < total;
-        bool done = false;
-        if (!run && more) fetch(following);
-        if (run) {
-            invert_unit_lower64(sL, sT, sTmp);
-            if (more) fetch(following);  // after the inverse: its shared-memory traffic runs alone
-            // ---- Tb = T diag(beta) as the A operand (64 x 64 K-major, zero above the diagonal)
-            {
-                const int r = tid >> 3, c0 = 8 * (tid & 7);
-                float tr[8], bc[8], x[8];
-                ld8(sT + r * PT + c0, tr);
-                ld8(sB + c0, bc);
-#pragma unroll
-                for (int w = 0; w < 8; ++w) x[w] = c0 + w <= r ? tr[w] * bc[w] : 0.f;
-                st_pair(sTb, 8192, kmaj_off(r, c0, 64), x);
+                for (int w = 0; w < 8; ++w) x[w] = k8[w] * (ei[w] * em[w]);
+                st_pair_g(pack + PK::OFF_A3, PK::A3 / 2, mnmaj_off(cb, i, C), x);
             }
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            // ---- [W | U~] = Tb . [K o A | V]  (M = 64, N = 2D, K = 64) into TMEM columns 0..2D-1
+            // D[128 x 160] (+)= A . B^T over this part's 64 channels (L' in rows 0..63, M in 64..127)
             if (tid == 0) {
-                constexpr uint32_t id = idesc_bf16(64, 2 * D, false, true);
-                const uint32_t a0 = smem_u32(sTb), b0 = smem_u32(sA);
+                constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
+                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks) {
-                    const uint64_t ah = kmaj_desc(a0, 64, 0, ks), al = kmaj_desc(a0 + 8192, 64, 0, ks);
-                    const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + I::A_BYTES / 2, C, 0, ks);
-                    mma_bf16(tmem, ah, bh, id, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_H / 2, 128, 0, ks);
+                    const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_H / 2, I::NB, 0, ks);
+                    mma_bf16(tmem, ah, bh, id, (hf > 0 || ks > 0) ? 1u : 0u);
                     mma_bf16(tmem, ah, bl, id, 1);
                     mma_bf16(tmem, al, bh, id, 1);
                 }
                 mma_commit(bar);
             }
-            bool ok2 = mbar_wait(bar, 1, kWaitCycles);
-            tc_fence_after();
-            ok2 = __syncthreads_and(ok2) != 0;
-            if (ok2) {
-                // M = 64 layout: row 16 quad + lane in lanes < 16 of the quad; warp part p takes
-                // columns [p 2D/4, (p+1) 2D/4): W for columns < D, U~ above. Staged in shared
-                // memory (the B region: L, M, T and Tb are dead) in the pack's own layout.
-                const int quad = warp & 3, part = warp >> 2;
-                const int row = 16 * quad + lane;
-                constexpr int CW = 2 * D / 4;
+        }
+        if (!ok) {  // a part's wait gave up (block-uniform)
+            give_up(bar, mph & 1, item);
+            continue;
+        }
+        safe = __syncthreads_and(safe) != 0;
+        ok = mbar_wait(bar, mph & 1, kWaitCycles);  // the last part's MMA
+        tc_fence_after();
+        if (!__syncthreads_and(ok)) {
+            give_up(bar, mph & 1, item);
+            continue;
+        }
+        ++mph;
+        if (!safe) {  // the CUDA-core body redoes this chunk (it rewrites the whole pack)
+            if (tid == 0) list[1 + atomicAdd(list, 1)] = item;
+            if (following < total) fetch_g(following);  // R2 (Gamma) is free
+            continue;
+        }
+        // ---- read back: warp (quad, part); row r = 32 quad + lane (i = r % 64, block a = i / 16)
+        //      needs columns [off_a, off_a + 16(a+1)); the quad's window is [0, 48) for rows in
+        //      blocks 0-1 and [48, 160) for blocks 2-3, its 8-column chunks split over two warps.
+        //      L = diag(beta) L' (strictly lower) to shared memory; M (lower with diagonal, zero
+        //      above) straight into the pack.
+        {
+            const int quad = warp & 3, part = warp >> 2;
+            const int r = 32 * quad + lane, i = r & 63, a = i >> 4;
+            const int off_a = 8 * a * (a + 1), seg = 16 * (a + 1);
+            const int w0 = (quad & 1) ? 48 : 0, wlen = (quad & 1) ? 112 : 48;
+            const bool is_l = r < 64;
+            const float bi = sB[i];
+#pragma unroll 1
+            for (int c8 = part * 8; c8 < wlen; c8 += 16) {
+                float x[8];
+                tmem_ld8(tmem_lane_base(tmem, warp) + w0 + c8, x);
+                tmem_ld_wait();
+                const int j0 = w0 + c8 - off_a;
+                if (j0 >= 0 && j0 < seg) {
+                    if (is_l) {
 #pragma unroll
-                for (int c16 = 0; c16 < CW; c16 += 16) {
-                    const int col = part * CW + c16;
-                    float x[16];
-                    tmem_ld16(tmem_lane_base(tmem, warp) + col, x);
-                    tmem_ld_wait();
-                    if (lane < 16) {
+                        for (int w = 0; w < 8; ++w)
+                            if (j0 + w < i) sL[i * PC + j0 + w] = x[w] * bi;
+                    } else {
 #pragma unroll
-                        for (int hlf = 0; hlf < 2; ++hlf) {
-                            const int cc = col + 8 * hlf;
-                            const float(&x8)[8] = *reinterpret_cast<const float(*)[8]>(x + 8 * hlf);
-                            if (cc < D) {
-                                // rows 0..63 of A1 panel p = cc / 64: the first 8 KB of the panel
-                                const uint32_t off = (cc >> 6) * 8192 + kmaj_off(row, cc & 63, 64);
-                                uint4 hi, lo;
-                                split8(x8, hi, lo);
-                                *reinterpret_cast<uint4 *>(sW + off) = hi;
-                                *reinterpret_cast<uint4 *>(sW + I::W_STAGE / 2 + off) = lo;
-                            } else {
-                                const int c = cc - D;
-                                float *dst = sUt + (c >> 5) * (PK::UG_BYTES / 4) + row * PK::UP + (c & 31);
-                                *reinterpret_cast<float4 *>(dst) = make_float4(x8[0], x8[1], x8[2], x8[3]);
-                                *reinterpret_cast<float4 *>(dst + 4) = make_float4(x8[4], x8[5], x8[6], x8[7]);
-                            }
+                        for (int w = 0; w < 8; ++w) x[w] = j0 + w <= i ? x[w] : 0.f;
+                        st_pair_g(pack + PK::OFF_AM, PK::AM / 2, kmaj_off(i, j0, 64), x);
+                    }
+                }
+            }
+            if (!is_l) {
+                const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int jc = seg / 8 + part; jc < 8; jc += 2) st_pair_g(pack + PK::OFF_AM, PK::AM / 2, kmaj_off(i, 8 * jc, 64), z);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        invert_unit_lower64<NT>(sL, sT, sTmp);
+        // ---- Tb = T diag(beta) as the A operand (64 x 64 K-major, zero above the diagonal)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int u = tid + NT * j, r = u >> 3, c0 = 8 * (u & 7);
+            float tr[8], bc[8], x[8];
+            ld8f(sT + r * PT + c0, tr);
+            ld8f(sB + c0, bc);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = c0 + w <= r ? tr[w] * bc[w] : 0.f;
+            st_pair(sTb, 8192, kmaj_off(r, c0, 64), x);
+        }
+        __syncthreads();  // T is dead: the K o A operand part may overwrite it
+        // ---- the W|U~ B operand, MN-major (n = channel, k = token): K o A = K o e^Gamma over the
+        //      dead L and T, then V over Gamma (v held in registers across the barrier)
+        float vv[UB][8];
+#pragma unroll
+        for (int j = 0; j < UB; ++j) {
+            const int u = tid + NT * j, i = u / (D / 8), cb = 8 * (u % (D / 8));
+            float k8[8], gi[8], x[8];
+            if (i < n) {
+                load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, k8);
+                load8_in<D, QKV16>(in, 2, row0 + i, H, h, cb, vv[j]);
+            } else {
+#pragma unroll
+                for (int w = 0; w < 8; ++w) { k8[w] = 0.f; vv[j][w] = 0.f; }
+            }
+            ld8f(sG + i * D + cb, gi);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x[w] = k8[w] * __expf(gi[w]);
+            st_pair(sKA, I::KA / 2, mnmaj_off(cb, i, C), x);
+        }
+        __syncthreads();  // Gamma is dead
+#pragma unroll
+        for (int j = 0; j < UB; ++j) {
+            const int u = tid + NT * j, i = u / (D / 8), cb = 8 * (u % (D / 8));
+            st_pair(sR2, I::KA / 2, mnmaj_off(cb, i, C), vv[j]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ---- [W | U~] = Tb . [K o A | V]  (M = 64, N = D each, K = 64) into TMEM columns 0..2D-1
+        if (tid == 0) {
+            constexpr uint32_t id = idesc_bf16(64, D, false, true);
+            const uint32_t a0 = smem_u32(sTb), bk = smem_u32(sKA), bv = smem_u32(sR2);
+#pragma unroll
+            for (int ks = 0; ks < C / 16; ++ks) {
+                const uint64_t ah = kmaj_desc(a0, 64, 0, ks), al = kmaj_desc(a0 + 8192, 64, 0, ks);
+                const uint64_t kh = mnmaj_desc(bk, C, 0, ks), kl = mnmaj_desc(bk + I::KA / 2, C, 0, ks);
+                const uint64_t vh = mnmaj_desc(bv, C, 0, ks), vl = mnmaj_desc(bv + I::KA / 2, C, 0, ks);
+                const uint32_t acc = ks > 0 ? 1u : 0u;
+                mma_bf16(tmem, ah, kh, id, acc);
+                mma_bf16(tmem, ah, kl, id, 1);
+                mma_bf16(tmem, al, kh, id, 1);
+                mma_bf16(tmem + D, ah, vh, id, acc);
+                mma_bf16(tmem + D, ah, vl, id, 1);
+                mma_bf16(tmem + D, al, vh, id, 1);
+            }
+            mma_commit(bar);
+        }
+        ok = mbar_wait(bar, mph & 1, kWaitCycles);
+        tc_fence_after();
+        if (!__syncthreads_and(ok)) {
+            give_up(bar, mph & 1, item);
+            continue;
+        }
+        ++mph;
+        if (following < total) fetch_g(following);  // R2 is free: the next item's g box comes in
+        // ---- read back (M = 64 layout: row 16 quad + lane in lanes < 16 of the quad); warp part 0
+        //      takes W (columns 0..D-1, into A1 rows 0..63 as BF16 hi + lo), part 1 U~ (FP32)
+        {
+            const int quad = warp & 3, part = warp >> 2, row = 16 * quad + lane;
+#pragma unroll 1
+            for (int c16 = 0; c16 < D; c16 += 16) {
+                float x[16];
+                tmem_ld16(tmem_lane_base(tmem, warp) + part * D + c16, x);
+                tmem_ld_wait();
+                if (lane < 16) {
+#pragma unroll
+                    for (int hl = 0; hl < 2; ++hl) {
+                        const int cc = c16 + 8 * hl;
+                        const float(&x8)[8] = *reinterpret_cast<const float(*)[8]>(x + 8 * hl);
+                        if (part == 0) {
+                            st_pair_g(pack + PK::OFF_A1, PK::A1 / 2, kmaj_off(row, cc, 128), x8);
+                        } else {
+                            float *dst = reinterpret_cast<float *>(pack + PK::OFF_UT + (cc >> 5) * PK::UG_BYTES) +
+                                         row * PK::UP + (cc & 31);
+                            *reinterpret_cast<float4 *>(dst) = make_float4(x8[0], x8[1], x8[2], x8[3]);
+                            *reinterpret_cast<float4 *>(dst + 4) = make_float4(x8[4], x8[5], x8[6], x8[7]);
                         }
                     }
                 }
-                fence_async_smem();
-                __syncthreads();
-                if (tid == 0) {
-                    // W hi and lo: rows 0..63 of each 64-column panel of A1 (8 KB each); U~ whole
-#pragma unroll
-                    for (int p = 0; p < D / 64; ++p) {
-                        bulk_store(pack + PK::OFF_A1 + p * 16384, sW + p * 8192, 8192);
-                        bulk_store(pack + PK::OFF_A1 + PK::A1 / 2 + p * 16384, sW + I::W_STAGE / 2 + p * 8192, 8192);
-                    }
-                    bulk_store(pack + PK::OFF_UT, sUt, PK::UT);
-                    bulk_commit();
-                }
-                done = true;
-            } else {
-                if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
-                mbar_wait(bar, 1, kWaitCycles);  // bounded: the MMA may still be reading shared memory
-                dead = true;
             }
-            tc_fence_before();
-        } else if (safe && !ok) {
-            if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
-            mbar_wait(bar, 0, kWaitCycles);
-            dead = true;
         }
-        if (!done && tid == 0) {
-            // the CUDA-core body redoes this chunk (it rewrites the whole pack)
-            const int slot = atomicAdd(list, 1);
-            list[1 + slot] = item;
-        }
-        __syncthreads();
+        tc_fence_before();
+        __syncthreads();  // TMEM is read: the next item's MMAs may overwrite it
     }
-    if (tid == 0) bulk_wait_all();  // every staged result is in global memory
+    tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
@@ -1077,13 +1069,14 @@ struct State {
     static constexpr int A2 = 2 * kTileBytes;       // [0; M]: 128 x 64 K-major hi + lo, rows 0..63 zero
     static constexpr int B1 = 2 * NB * D * 2;       // S0 hi + lo, MN-major (N = value columns, K = D keys)
     static constexpr int B2 = 2 * NB * C * 2;       // U hi + lo, MN-major (N = value columns, K = 64)
-    static constexpr int US = (DVS / 32) * PK::UG_BYTES;  // the slice's U~ groups
     static constexpr int OFF_A1 = 0, OFF_A2 = PK::A1, OFF_A3 = OFF_A2 + A2, OFF_B1 = OFF_A3 + PK::A3,
-                         OFF_B2 = OFF_B1 + B1, OFF_U = OFF_B2 + B2, OFF_MISC = OFF_U + US;
+                         OFF_B2 = OFF_B1 + B1, OFF_MISC = OFF_B2 + B2;
     static constexpr int MISC = 1024;
     static constexpr int bytes = OFF_MISC + MISC + 1024;  // + alignment slack
+    static_assert(bytes <= 232448, "one CTA per SM");
     // D1 twice (chunk parity: a chunk's outputs are read while the next chunk's D1 is computed), D3
-    static constexpr uint32_t TMEM_COLS = 3 * DVS <= 32 ? 32 : (3 * DVS <= 64 ? 64 : (3 * DVS <= 128 ? 128 : 256));
+    static constexpr uint32_t TMEM_COLS =
+        3 * DVS <= 32 ? 32 : (3 * DVS <= 64 ? 64 : (3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512)));
 };
 
 // A bulk global -> shared copy completing on `bar`, whose expected bytes were already
@@ -1104,6 +1097,15 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
                  : "memory");
 }
 
+// The chain of one (stream, head, value slice of DVS columns) over its chunks. Per chunk:
+//   MMA group 1   D1 = [W; Q o A] . S0                       (M = 128, N = DVS, K = D)
+//   epilogue 1    U = U~ - D1[0:64] into shared memory (U~ read from the pack into registers
+//                 while group 1 runs)
+//   MMA group 2   D3 = (K o e^{Gamma_C - Gamma})^T . U        (M = D, N = DVS, K = 64), committed alone
+//   MMA group 3   D1 += [0; M] . U                            (so D1[64:128] = (Q o A) S0 + M U)
+//   epilogue 2    S = A_C o S0 + D3 (FP32 master copy in registers) into the S operand
+// Groups 1 and 2 and the two epilogues are the critical path; group 3 and the output rows
+// O = scale D1[64:128] run beside the next chunk.
 template <int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
 state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core,
@@ -1115,8 +1117,8 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = sm + S::OFF_A1, *sA2 = sm + S::OFF_A2, *sA3 = sm + S::OFF_A3, *sB1 = sm + S::OFF_B1,
             *sB2 = sm + S::OFF_B2;
-    const float *sU = reinterpret_cast<const float *>(sm + S::OFF_U);  // [DVS/32][64][UP]
-    // barriers: copies 0 A1, 1 M, 2 A3, 3 U~; MMA groups 4 (D1), 5 (D3 and D1 += [0; M] U)
+    // barriers: copies 0 A1, 1 M, 2 A3; MMA groups 4 (D1), 5 (D3), 6 (D1 += [0; M] U); 7 the
+    // final drain after a timeout
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 64);
 
@@ -1137,7 +1139,6 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     if (nb == 0) return;  // an empty stream keeps its state
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
     const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
-    const size_t u_off = PK::OFF_UT + static_cast<size_t>(c0 / 32) * PK::UG_BYTES;
 
     auto copy_m = [&](const uint8_t *pk) {  // M's hi and lo halves into rows 64..127 of A2
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bars[1])),
@@ -1146,13 +1147,21 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         bulk_copy_nx(sA2 + 8192, pk + PK::OFF_AM, PK::AM / 2, &bars[1]);
         bulk_copy_nx(sA2 + kTileBytes + 8192, pk + PK::OFF_AM + PK::AM / 2, PK::AM / 2, &bars[1]);
     };
+    // thread 0 issues every copy and counts, per copy barrier, the copies issued and the phases
+    // it has waited for (so that a timed-out CTA can drain what is still in flight)
+    uint32_t issued[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
+    auto wait_copy = [&](int k) {
+        const bool r = mbar_wait(&bars[k], waited[k] & 1, kWaitCycles);
+        if (r) ++waited[k];
+        return r;
+    };
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         bulk_copy(sA1, packs + PK::OFF_A1, PK::A1, &bars[0]);
         copy_m(packs);
         bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[2]);
-        bulk_copy(const_cast<float *>(sU), packs + u_off, S::US, &bars[3]);
+        issued[0] = issued[1] = issued[2] = 1;
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -1177,7 +1186,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     const int ccol = colh * HALF;
     const int srow = (D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1);
 
-    // FP32 master state slice: key row srow, value columns [ccol, ccol + HALF)
+    // FP32 master state slice: key row srow, value columns [c0 + ccol, + HALF)
     float st[HALF];
     if (srow >= 0) {
 #pragma unroll
@@ -1204,8 +1213,10 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     __syncthreads();
     tc_fence_after();
     // O = scale D1[64:128] of chunk c (quads 2 and 3: TMEM lanes 64..127 = the chunk's tokens),
-    // run while the tensor core computes chunk c + 1
+    // once group 3 of chunk c has completed; run while the tensor core computes chunk c + 1
     auto out_epilogue = [&](int c) {
+        ok = ok && mbar_wait(&bars[6], c & 1, kWaitCycles);
+        tc_fence_after();
         const int i = erow - 64;
         int nn;
         size_t r0;
@@ -1216,7 +1227,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             float x[8];
             tmem_ld8(tmem_lane_base(tD1c, warp) + ccol + j, x);
             tmem_ld_wait();
-            if (i < nn) {
+            if (i < nn && ok) {
                 float *dst = core + (r0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
                 *reinterpret_cast<float4 *>(dst) = make_float4(scale * x[0], scale * x[1], scale * x[2], scale * x[3]);
                 *reinterpret_cast<float4 *>(dst + 4) =
@@ -1229,14 +1240,24 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     for (int ch = 0; ch < nb; ++ch) {
         const uint32_t par = ch & 1;
         const uint32_t tD1 = tmem + par * DVS;
-        const uint8_t *next = packs + static_cast<size_t>(ch + 1) * PK::bytes;
+        const uint8_t *cur = packs + static_cast<size_t>(ch) * PK::bytes;
+        const uint8_t *next = cur + PK::bytes;
         const bool more = ch + 1 < nb;
-        // e^{Gamma_C} of this thread's key row, read early (used in epilogue 2)
-        const float ac = srow >= 0 ? reinterpret_cast<const float *>(packs + static_cast<size_t>(ch) * PK::bytes +
-                                                                    PK::OFF_AC)[srow]
-                                   : 0.f;
+        // e^{Gamma_C} of this thread's key row (epilogue 2) and U~ of its row (epilogue 1), read
+        // from the pack while group 1 runs
+        const float ac = srow >= 0 ? reinterpret_cast<const float *>(cur + PK::OFF_AC)[srow] : 0.f;
+        float ut[HALF];
+        if (quad < 2) {
+#pragma unroll
+            for (int j = 0; j < HALF; j += 4) {
+                const int c = c0 + ccol + j;
+                const float4 u4 = *reinterpret_cast<const float4 *>(
+                    reinterpret_cast<const float *>(cur + PK::OFF_UT + (c >> 5) * PK::UG_BYTES) + erow * PK::UP + (c & 31));
+                ut[j] = u4.x; ut[j + 1] = u4.y; ut[j + 2] = u4.z; ut[j + 3] = u4.w;
+            }
+        }
         // ---- MMA group 1: D1 = [W; Q o A] . S0
-        if (tid == 0 && ok) ok = mbar_wait(&bars[0], par, kWaitCycles);
+        if (tid == 0 && ok) ok = wait_copy(0);
         if (tid == 0 && ok) {
             constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
             const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
@@ -1249,12 +1270,22 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 mma_bf16(tD1, al, bh, id, 1);
             }
             mma_commit(&bars[4]);
+            // group 3 of the previous chunk has read M: the next M may come in
+            if (ch > 0) {
+                ok = mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles);
+                if (ok) {
+                    copy_m(cur);
+                    ++issued[1];
+                }
+            }
         }
         if (ch > 0 && quad >= 2) out_epilogue(ch - 1);
         ok = ok && mbar_wait(&bars[4], par, kWaitCycles);
-        ok = ok && mbar_wait(&bars[3], par, kWaitCycles);  // U~ of this chunk
         tc_fence_after();
-        if (tid == 0 && ok && more) bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);  // A1 is free again
+        if (tid == 0 && ok && more) {  // A1 is free again
+            bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);
+            ++issued[0];
+        }
         // ---- epilogue 1: U = U~ - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
         if (quad < 2) {
 #pragma unroll
@@ -1262,31 +1293,26 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 float x[8];
                 tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
                 tmem_ld_wait();
-                const int c = ccol + j;  // column within the slice
-                const float *ur = sU + (c >> 5) * (PK::UG_BYTES / 4) + erow * PK::UP + (c & 31);
-                const float4 u0 = *reinterpret_cast<const float4 *>(ur);
-                const float4 u1 = *reinterpret_cast<const float4 *>(ur + 4);
-                x[0] = u0.x - x[0]; x[1] = u0.y - x[1]; x[2] = u0.z - x[2]; x[3] = u0.w - x[3];
-                x[4] = u1.x - x[4]; x[5] = u1.y - x[5]; x[6] = u1.z - x[6]; x[7] = u1.w - x[7];
-                if (tables) {  // verify mode: U of every row, for the fold
-                    float *ut = tables + (static_cast<size_t>(b) * H + h) * 2 * C * D + erow * D + c0 + c;
-                    *reinterpret_cast<float4 *>(ut) = make_float4(x[0], x[1], x[2], x[3]);
-                    *reinterpret_cast<float4 *>(ut + 4) = make_float4(x[4], x[5], x[6], x[7]);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) x[u] = ut[j + u] - x[u];
+                if (tables && ok) {  // verify mode: U of every row, for the fold
+                    float *utab = tables + (static_cast<size_t>(b) * H + h) * 2 * C * D + erow * D + c0 + ccol + j;
+                    *reinterpret_cast<float4 *>(utab) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4 *>(utab + 4) = make_float4(x[4], x[5], x[6], x[7]);
                 }
-                st_pair(sB2, S::B2 / 2, mnmaj_off(c, erow, C), x);
+                st_pair(sB2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
             }
         }
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
         tc_fence_after();
-        if (tid == 0 && ok && more) bulk_copy(const_cast<float *>(sU), next + u_off, S::US, &bars[3]);
-        // ---- MMA group 2: D3 = (K o e^{Gamma_C - Gamma})^T . U;  D1 += [0; M] . U
-        if (tid == 0 && ok) ok = mbar_wait(&bars[1], par, kWaitCycles) && mbar_wait(&bars[2], par, kWaitCycles);
+        // ---- MMA group 2: D3 = (K o e^{Gamma_C - Gamma})^T . U (the chain), then group 3:
+        //      D1 += [0; M] . U (the output rows), each committed on its own
+        if (tid == 0 && ok) ok = wait_copy(2);
         if (tid == 0 && ok) {
             constexpr uint32_t id3 = idesc_bf16(D, DVS, true, true);
-            constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
-            const uint32_t a3 = smem_u32(sA3), a2 = smem_u32(sA2), b0 = smem_u32(sB2);
+            const uint32_t a3 = smem_u32(sA3), b0 = smem_u32(sB2);
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
                 const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
@@ -1294,20 +1320,30 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 mma_bf16(tD3, ah, bh, id3, ks > 0 ? 1u : 0u);
                 mma_bf16(tD3, ah, bl, id3, 1);
                 mma_bf16(tD3, al, bh, id3, 1);
-                const uint64_t mh = kmaj_desc(a2, 128, 0, ks), ml = kmaj_desc(a2 + kTileBytes, 128, 0, ks);
-                mma_bf16(tD1, mh, bh, idm, 1);
-                mma_bf16(tD1, mh, bl, idm, 1);
-                mma_bf16(tD1, ml, bh, idm, 1);
             }
             mma_commit(&bars[5]);
+            ok = wait_copy(1);
+            if (ok) {
+                constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
+                const uint32_t a2 = smem_u32(sA2);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks) {
+                    const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
+                    const uint64_t mh = kmaj_desc(a2, 128, 0, ks), ml = kmaj_desc(a2 + kTileBytes, 128, 0, ks);
+                    mma_bf16(tD1, mh, bh, idm, 1);
+                    mma_bf16(tD1, mh, bl, idm, 1);
+                    mma_bf16(tD1, ml, bh, idm, 1);
+                }
+                mma_commit(&bars[6]);
+            }
         }
         ok = ok && mbar_wait(&bars[5], par, kWaitCycles);
         tc_fence_after();
-        if (tid == 0 && ok && more) {  // M and A3 are free again
-            copy_m(next);
+        if (tid == 0 && ok && more) {  // A3 is free again
             bulk_copy(sA3, next + PK::OFF_A3, PK::A3, &bars[2]);
+            ++issued[2];
         }
-        // ---- epilogue 2: S = A_C o S0 + D3 (FP32 in registers), S into B1;  O = scale D1[64:128]
+        // ---- epilogue 2: S = A_C o S0 + D3 (FP32 in registers), S into B1
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
             float x[8];
@@ -1326,8 +1362,18 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         if (!ok) break;  // block-uniform: every thread saw the same flag
     }
     if (ok && quad >= 2) out_epilogue(nb - 1);
+    ok = __syncthreads_and(ok) != 0;
     if (!ok) {
-        if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
+        if (tid == 0) {
+            atomicExch(status, KDA_ERR_TIMEOUT);
+            // drain (bounded): every MMA this thread issued, then every copy still in flight, so that
+            // nothing reads or writes shared memory or TMEM once they are released
+            mma_commit(&bars[7]);
+            mbar_wait(&bars[7], 0, kWaitCycles);
+            for (int k = 0; k < 3; ++k)
+                while (waited[k] < issued[k] && wait_copy(k)) {
+                }
+        }
     } else if (srow >= 0 && !tables) {  // verify mode leaves the state as it was
 #pragma unroll
         for (int j = 0; j < HALF; j += 4)
@@ -1351,7 +1397,7 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
     static std::atomic<unsigned long long> attr_intra{0}, attr_fix{0}, attr_state{0};
-    KDA_TRY(smem_opt_in(intra_tc_kernel<D, MODE>, IntraTC<D>::bytes, attr_intra));
+    KDA_TRY(smem_opt_in(intra_tc_kernel<D, MODE>, IntraTC<D>::bytes, attr_intra, true));
     KDA_TRY(smem_opt_in(intra_fix_kernel<D, MODE>, static_cast<int>(Intra<D>::bytes), attr_fix));
     KDA_TRY(smem_opt_in(state_kernel<D, DVS>, State<D, DVS>::bytes, attr_state));
     uint8_t *sc = static_cast<uint8_t *>(scratch);
@@ -1364,21 +1410,19 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
     const long long items = static_cast<long long>(B) * H * nch;
-    const int grid = static_cast<int>(std::min<long long>(items, sms));
-    // box maps: (stream, row in stream) for equal-length streams; the packed rows in varlen mode
+    // two tensor-core intra CTAs per SM; the CUDA-core fix-up runs one per SM
+    const int grid = static_cast<int>(std::min<long long>(items, 2LL * sms));
+    const int grid_fix = static_cast<int>(std::min<long long>(items, sms));
+    // g box map: (stream, row in stream) for equal-length streams; the packed rows in varlen mode
     const int mT = sq.cu ? sq.total : sq.T, mTp = sq.cu ? sq.total : sq.T_pad, mB = sq.cu ? 1 : B;
-    CUtensorMap tmG, tmV;
+    CUtensorMap tmG;
     if (kGraw<MODE>)
         KDA_TRY(make_rows_map(&tmG, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, mT, mTp, mB, D, C));
     else
         KDA_TRY(make_rows_map(&tmG, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-    if (kQkv16<MODE>)
-        KDA_TRY(make_rows_map(&tmV, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, mT, mTp, mB, D, C));
-    else
-        KDA_TRY(make_rows_map(&tmV, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-    intra_tc_kernel<D, MODE><<<grid, kIntraThreads, IntraTC<D>::bytes, s>>>(tmG, tmV, in, sc, list, B, sq, H, status);
+    intra_tc_kernel<D, MODE><<<grid, kTcThreads, IntraTC<D>::bytes, s>>>(tmG, in, sc, list, B, sq, H, status);
     KDA_TRY(launch_status());
-    intra_fix_kernel<D, MODE><<<grid, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
+    intra_fix_kernel<D, MODE><<<grid_fix, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
     state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
                                                                                    in.tables, status);
@@ -1393,7 +1437,8 @@ int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, c
     const float sc = dims->scale;
     if (dims->head_dim == 64) return launch_tc<64, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
     const long long units = static_cast<long long>(B) * H;
-    if (units >= 60) return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    if (units >= 100) return launch_tc<128, 128, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    if (units >= 50) return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
     return launch_tc<128, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
 }
 

@@ -1,6 +1,8 @@
 """GPU parity of the projection GEMM and of the whole block prefill (Glm5NextKdaLayer `prefill`)
 with the FP64 oracle. BF16 block outputs: relative L2 <= 2e-2 (the block path rounds to BF16 at
-every stage the workspace page lists, on both sides, from FP32 vs FP64 arithmetic)."""
+every stage the workspace page lists, on both sides, from FP32 vs FP64 arithmetic). The block's
+FP32 core and state are held to 1e-4: the block's core stage is the fused-input chunked prefill
+bit for bit, and that call on the oracle's own stage values matches the oracle's core."""
 import types
 
 import numpy as np
@@ -105,6 +107,40 @@ def _stages(ws, T, Wt):
                 final_out=v("final_out", (T, Wt.hidden), torch.bfloat16))
 
 
+def _fused_core(conv_out, g_raw, beta, Wt, T, s0):
+    """kda_chunk_prefill_fused on given BF16 conv_out rows [T, 3HD], BF16 g_raw [T, HD] and FP32
+    beta [T, H] (rows past T zero), from state s0: (core [T, H, D], final state)."""
+    H, D = Wt.H, Wt.D
+    Tp = t_pad(T)
+    qkv = torch.zeros((Tp, 3 * H * D), dtype=torch.bfloat16, device="cuda")
+    qkv[:T] = torch.as_tensor(conv_out).to("cuda", torch.bfloat16)
+    gr = torch.zeros((Tp, H * D), dtype=torch.bfloat16, device="cuda")
+    gr[:T] = torch.as_tensor(g_raw).to("cuda", torch.bfloat16)
+    be = torch.zeros((Tp, H), dtype=torch.float32, device="cuda")
+    be[:T] = torch.as_tensor(beta).reshape(T, H).to("cuda", torch.float32)
+    hs = torch.as_tensor(s0).to("cuda", torch.float32).clone()
+    core = torch.full((Tp, H, D), float("nan"), device="cuda")
+    kda.kda_chunk_prefill_fused(qkv, gr, Wt.dt_bias.cuda(), Wt.a_log.cuda(), be, kda.ptr_array([hs]), core, 1, T,
+                                kda.dims(H, D))
+    torch.cuda.synchronize()
+    return core[:T], hs
+
+
+def _check_block_core(ws, hs, Wt, T, ref):
+    """The block's FP32 core and state at the FP32 tolerance, in two steps that never feed a GPU
+    value to the oracle: (a) the block's core stage is kda_chunk_prefill_fused on the block's own
+    stage buffers, bit for bit; (b) kda_chunk_prefill_fused on the oracle's stage values (its
+    BF16 conv_out and g_raw, its beta) matches the oracle's core and state to 1e-4."""
+    H, D, qkv = Wt.H, Wt.D, Wt.H * Wt.D
+    core_b = ws.view("core", (T, H, D), torch.float32)
+    c_a, s_a = _fused_core(ws.view("conv_out", (T, 3 * qkv), torch.bfloat16), ws.view("g_raw", (T, qkv), torch.bfloat16),
+                           ws.view("beta", (T, H), torch.float32), Wt, T, torch.zeros((H, D, D)))
+    assert torch.equal(c_a, core_b) and torch.equal(s_a, hs)
+    c_b, s_b = _fused_core(ref["conv_out"], ref["g_raw"], ref["beta"], Wt, T, np.zeros((H, D, D)))
+    assert rel_l2(np64(c_b), ref["core"]) <= 1e-4
+    assert rel_l2(np64(s_b), ref["h_state"]) <= 1e-4
+
+
 @pytest.mark.parametrize("hidden,H,D,rank,T", [(256, 2, 64, 64, 200), (512, 4, 128, 128, 130)])
 def test_block_prefill_stages_match_oracle(hidden, H, D, rank, T):
     Wt = block_weights(hidden, H, D, rank, seed=2, std=0.05)
@@ -120,6 +156,7 @@ def test_block_prefill_stages_match_oracle(hidden, H, D, rank, T):
     errs["conv_state"] = rel_l2(np64(cs), ref["conv_state"])
     assert errs["qkv_proj"] <= 4e-3 and errs["conv_state"] <= 4e-3, errs
     assert all(e <= TOL_BF16 for e in errs.values()), errs
+    _check_block_core(ws, hs, Wt, T, ref)
     ws.close()
 
 
@@ -160,4 +197,5 @@ def test_block_prefill_full_size():
     ref = oracle.block_prefill(Wt, h, np.zeros((H, D, D)), np.zeros((3 * H * D, 3)))
     assert rel_l2(final, ref["final_out"]) <= TOL_BF16
     assert rel_l2(np64(hs), ref["h_state"]) <= TOL_BF16
+    _check_block_core(ws, hs, Wt, T, ref)
     ws.close()

@@ -1,7 +1,9 @@
 """GPU block decode (Glm5NextKdaLayer `decode`: N sequences x 1 token through the whole block)
 and block decode_k (`decode_k`: K rows of one sequence, projections read once for all rows)
 against the oracle, and the decode_k identity through the whole block: K rows in one call
-are bit-identical to K one-row calls, snapshots included."""
+are bit-identical to K one-row calls, snapshots included. BF16 block outputs at 2e-2; the FP32
+core and states at 1e-4 through the stateful row's own entry point (never feeding a GPU value
+to the oracle)."""
 import numpy as np
 import pytest
 import torch
@@ -30,6 +32,26 @@ def _states(n, H, D, seed):
     return hs, cs
 
 
+def _decode_fused(x_rows, g_raw, b_logit, out_gate, hs, cs, Wt):
+    """kda_decode_fused on given stage rows (one token for each of N sequences) from copies of
+    the states hs [N, H, D, D] and conv states cs [N, 3HD, 3]: (core, states, conv states, o_norm_out)."""
+    H, D = Wt.H, Wt.D
+    N = len(hs)
+    dev = "cuda"
+    x = torch.as_tensor(x_rows).to(dev, torch.bfloat16).contiguous()
+    gr = torch.as_tensor(g_raw).to(dev, torch.bfloat16).contiguous()
+    bl = torch.as_tensor(b_logit).to(dev, torch.float32).contiguous()
+    og = torch.as_tensor(out_gate).to(dev, torch.bfloat16).contiguous()
+    hd = [torch.as_tensor(hs[n]).to(dev, torch.float32).clone() for n in range(N)]
+    cd = [torch.as_tensor(cs[n]).to(dev, torch.bfloat16).clone() for n in range(N)]
+    out = torch.empty((N, H * D), dtype=torch.bfloat16, device=dev)
+    core = torch.empty((N, H, D), device=dev)
+    kda.kda_decode_fused(x, kda.ptr_array(cd), Wt.conv_w.cuda(), gr, Wt.dt_bias.cuda(), Wt.a_log.cuda(), bl,
+                         kda.ptr_array(hd), og, Wt.o_norm.cuda(), out, None, core, N, kda.dims(H, D))
+    torch.cuda.synchronize()
+    return core, hd, cd, out
+
+
 @pytest.mark.parametrize("hidden,H,D,rank,N,std", [(256, 2, 64, 64, 3, 0.05), (4096, 32, 128, 128, 4, 0.02)])
 def test_block_decode_matches_oracle(hidden, H, D, rank, N, std):
     Wt = block_weights(hidden, H, D, rank, seed=7, std=std)
@@ -43,11 +65,27 @@ def test_block_decode_matches_oracle(hidden, H, D, rank, N, std):
     kda.kda_block_decode(st, h.cuda(), N, kda.ptr_array(hd), kda.ptr_array(cd), ws)
     torch.cuda.synchronize()
     final = np64(ws.view("final_out", (N, hidden), torch.bfloat16))
-    for n in range(N):
-        ref = oracle.block_decode(Wt, h[n:n + 1], hs[n], cs[n])
+    refs = [oracle.block_decode(Wt, h[n:n + 1], hs[n], cs[n]) for n in range(N)]
+    for n, ref in enumerate(refs):
         assert rel_l2(final[n:n + 1], ref["final_out"]) <= TOL_BF16
         assert rel_l2(np64(hd[n]), ref["h_state"]) <= TOL_BF16
         assert rel_l2(np64(cd[n]), ref["conv_state"]) <= 4e-3
+    # the FP32 core and state at 1e-4, with no GPU value fed to the oracle: (a) the block's
+    # stateful row is kda_decode_fused on the block's own stage buffers, bit for bit; (b) that
+    # call on the oracle's stage values matches the oracle's core and state
+    qkv = H * D
+    c_a, h_a, c_sa, o_a = _decode_fused(ws.view("qkv_proj", (N, 3 * qkv), torch.bfloat16),
+                                        ws.view("g_raw", (N, qkv), torch.bfloat16),
+                                        ws.view("beta", (N, H), torch.float32),
+                                        ws.view("out_gate", (N, qkv), torch.bfloat16), hs, cs, Wt)
+    assert torch.equal(c_a, ws.view("core", (N, H, D), torch.float32))
+    assert torch.equal(o_a, ws.view("o_norm_out", (N, qkv), torch.bfloat16))
+    assert all(torch.equal(h_a[n], hd[n]) and torch.equal(c_sa[n], cd[n]) for n in range(N))
+    stack = lambda key: np.concatenate([r[key] for r in refs])  # noqa: E731
+    c_b, h_b, _, _ = _decode_fused(stack("qkv_proj"), stack("g_raw"), stack("b_logit"), stack("out_gate"), hs, cs, Wt)
+    for n, ref in enumerate(refs):
+        assert rel_l2(np64(c_b[n]), ref["core"][0]) <= 1e-4
+        assert rel_l2(np64(h_b[n]), ref["h_state"]) <= 1e-4
     ws.close()
 
 

@@ -127,7 +127,8 @@ def test_tc_and_simt_agree():
 @pytest.mark.parametrize("impl", ["tc"])
 def test_long_prefill_poison_full_size(impl):
     """B=4 streams of T=65500 (T_pad 65536), H=32, D=128, pad_fill NaN vs 0: full final states
-    bit-identical; sampled (stream, head) pairs within tolerance of the oracle."""
+    bit-identical; 16 (stream, head) pairs, four heads of every stream, within tolerance of the
+    oracle (outputs of every token and final state)."""
     B, T, H, D = 4, 65500, 32, 128
     ci = core_inputs(B, T, H, D, seed=4, bf16_inputs=True, s0_std=0.1, device="cuda")
     core_n, S_n, _ = gpu_prefill(ci, impl=impl, pad_fill=float("nan"))
@@ -135,12 +136,12 @@ def test_long_prefill_poison_full_size(impl):
     core_0, S_0, _ = gpu_prefill(ci, impl=impl, pad_fill=0.0)
     assert torch.equal(S_n, S_0)
     assert torch.equal(core_n, core_0)
-    for b, h in [(0, 0), (1, 17), (2, 31), (3, 5)]:
-        o_ref, S_ref = oracle_prefill(ci, seqs=[b], heads=[h])
-        got_o = np64(core_n[b, :, h])
-        got_s = np64(S_n[b, h])
-        assert rel_l2(got_o, o_ref[0, :, 0]) <= TOL
-        assert rel_l2(got_s, S_ref[0, 0]) <= TOL
+    heads = {0: [0, 9, 17, 31], 1: [3, 12, 20, 28], 2: [5, 14, 22, 30], 3: [1, 7, 19, 26]}
+    for b, hs in heads.items():
+        o_ref, S_ref = oracle_prefill(ci, seqs=[b], heads=hs)  # the four heads in parallel
+        for j, h in enumerate(hs):
+            assert rel_l2(np64(core_n[b, :, h]), o_ref[0, :, j]) <= TOL, (b, h)
+            assert rel_l2(np64(S_n[b, h]), S_ref[0, j]) <= TOL, (b, h)
     del core_n, core_0
     torch.cuda.empty_cache()
 
@@ -357,6 +358,12 @@ def test_varlen_many_sequences_and_batched_verify_at_serving_shapes():
     torch.cuda.synchronize()
     assert torch.equal(core, core_p)
     assert all(torch.equal(states[b], s0[b].cuda()) for b in range(0, Bv, 17))
+    for b in [0, 77, 128, 255]:  # sampled sequences' draft rows against the oracle
+        sl = slice(b * K, b * K + K)
+        one = CoreInputs(1, K, H, D, ci.q[:, sl], ci.k[:, sl], ci.v[:, sl], ci.g_raw[:, sl], ci.dt_bias, ci.a_log,
+                         ci.b_logit[:, sl], s0[b:b + 1])
+        o_ref, _ = oracle_prefill(one)
+        assert rel_l2(np64(core[sl]), o_ref[0]) <= TOL, b
     accepted = [int(x) for x in rng.integers(0, K + 1, size=Bv)]
     kda.kda_chunk_verify_fold(dev["k"], cu, torch.tensor(accepted, dtype=torch.int32, device="cuda"), Bv, total,
                               tables, ptrs, d)
@@ -417,6 +424,14 @@ def test_verify_then_fold_accepted_rows(D):
                                  core_p, d)
     torch.cuda.synchronize()
     assert torch.equal(core, core_p)
+    start = 0
+    for b, L in enumerate(lens):  # every draft row against the oracle from the unchanged state
+        sl = slice(start, start + L)
+        one = CoreInputs(1, L, H, D, ci.q[:, sl], ci.k[:, sl], ci.v[:, sl], ci.g_raw[:, sl], ci.dt_bias, ci.a_log,
+                         ci.b_logit[:, sl], s0[b:b + 1])
+        o_ref, _ = oracle_prefill(one)
+        assert rel_l2(np64(core[sl]), o_ref[0]) <= TOL, b
+        start += L
     acc = torch.tensor(accepted, dtype=torch.int32, device="cuda")
     kda.kda_chunk_verify_fold(dev["k"], cu, acc, B, total, tables, ptrs, d)
     torch.cuda.synchronize()
