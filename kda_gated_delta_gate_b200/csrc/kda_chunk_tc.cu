@@ -36,7 +36,6 @@ namespace {
 using namespace umma;
 
 constexpr int C = kChunk;          // 64
-constexpr int kThreads = 256;
 constexpr int kTileBytes = 16384;  // one 128 x 64 BF16 K-major tile
 
 // Per (stream, head, chunk) the intra kernel writes one pack of state-independent operands,
@@ -602,6 +601,8 @@ struct IntraTC {
     static_assert(OFF_TB + 16384 <= R1, "R1 holds L, T, the inverse's scratch and Tb");
     static_assert(KA <= OFF_TB, "the K o A operand part must not overlap Tb");
     static_assert(KA == R2, "the V operand part fills R2");
+    static constexpr int W_STAGE = 2 * C * D * 2;  // W rows 0..63 of A1 (hi + lo), staged in R1 for the bulk stores
+    static_assert(W_STAGE + Pack<D>::UT <= R1, "the staged W and U~ fit in R1");
     static_assert(2 * (bytes + 1024) <= 233472, "two CTAs per SM");
 };
 
@@ -618,10 +619,36 @@ __device__ __forceinline__ void st_pair_g(uint8_t *dst, int half_bytes, uint32_t
     *reinterpret_cast<uint4 *>(dst + half_bytes + off) = lo;
 }
 
+// One thread: prefetch the box at (x, y, z) of a 3-D tensor map into L2 (no shared memory).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *tm, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+// One thread: bulk shared -> global copy (bytes a multiple of 16), in this thread's bulk group.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Maps over the rows of the chunked path's inputs (3-D: columns, row in stream, stream): the g box
+// of an item is loaded from tmG; every input's box of the next item is prefetched into L2 through
+// tmG, tmQ, tmK, tmV (in the fused-input mode tmQ = tmK = tmV map the q|k|v rows).
+struct InMaps {
+    CUtensorMap g, q, k, v;
+};
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 2)
-intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uint8_t *__restrict__ scratch,
+intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t *__restrict__ scratch,
                 int *__restrict__ list, int B, const Seqs sq, int H, int *__restrict__ status) {
+    const CUtensorMap &tmG = maps.g;
     using I = IntraTC<D>;
     using PK = Pack<D>;
     constexpr int NT = kTcThreads, PC = kLPC, PT = kTPC, NH = I::NH;
@@ -648,7 +675,6 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
     // g's box: FP32 g at the start of R2, or BF16 g_raw in its upper half (the gate is then
     // formed in place, FP32, dense)
     void *gdst = sR2 + (GRAW ? C * D * 2 : 0);
-    const size_t rs = static_cast<size_t>(H) * D;
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
@@ -674,32 +700,21 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
         if (sq.cu) { y = static_cast<int>(row0); z = 0; }
         else { y = ch * C; z = b; }
     };
-    // an item's q, k, v and g rows into L2: thread (input tid / 64, row tid % 64), one bulk prefetch each
+    // an item's q, k, v and g boxes into L2 (thread 0, one tensor prefetch each)
     auto prefetch = [&](int it) {
+        if (tid != 0) return;
         const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
-        int n;
+        int n, y, z;
         size_t row0;
         seq_chunk(sq, b, ch, row0, n, nullptr);
-        const int part = tid >> 6, i = tid & 63;
-        if (i < n) {
-            const void *p;
-            uint32_t bytes;
-            if (part < 3) {
-                if constexpr (QKV16) {
-                    p = in.qkv + (row0 + i) * (3 * rs) + static_cast<size_t>(part * H + h) * D;
-                    bytes = D * 2;
-                } else {
-                    p = (part == 0 ? in.q : (part == 1 ? in.k : in.v)) + (row0 + i) * rs + static_cast<size_t>(h) * D;
-                    bytes = D * 4;
-                }
-            } else if constexpr (GRAW) {
-                p = in.g_raw + (row0 + i) * rs + static_cast<size_t>(h) * D;
-                bytes = D * 2;
-            } else {
-                p = in.gate + (row0 + i) * rs + static_cast<size_t>(h) * D;
-                bytes = D * 4;
-            }
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+        box_yz(ch, b, row0, y, z);
+        tma_prefetch_3d(&maps.g, h * D, y, z);
+        if constexpr (QKV16) {
+            for (int part = 0; part < 3; ++part) tma_prefetch_3d(&maps.q, (part * H + h) * D, y, z);
+        } else {
+            tma_prefetch_3d(&maps.q, h * D, y, z);
+            tma_prefetch_3d(&maps.k, h * D, y, z);
+            tma_prefetch_3d(&maps.v, h * D, y, z);
         }
     };
     // an item's g box into R2 (thread 0; the caller made R2 free) and its beta (threads < C)
@@ -757,11 +772,13 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
         if (following < total) prefetch(following);
         bool ok = mbar_wait(gbar, iter & 1, kWaitCycles);
         if (tid < C) sB[tid] = bnext;
+        if (tid == 0) bulk_wait_read();  // the previous item's staged results have left R1
         if (!__syncthreads_and(ok)) {
             give_up(gbar, iter & 1, item);
             continue;
         }
         // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, range of tokens)
+        bool safe = true;
         {
             constexpr int QT = NT / D;  // 2 (D=128) or 4 (D=64) token ranges
             constexpr int TPQ = C / QT;
@@ -795,7 +812,14 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
                 float *gt = in.tables + ((static_cast<size_t>(b) * H + h) * 2 + 1) * C * D;
                 for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) gt[i * D + c] = sG[i * D + c];
             }
-            __syncthreads();
+            // the reference bound of the 16-token blocks in this thread's range: every factor
+            // e^{+-(Gamma_i - Gamma_m)} of the L/M operands stays within e^{kRefBound}
+            for (int a = qr * TPQ / 16; a < (qr + 1) * TPQ / 16; ++a) {
+                const float gm = sG[(16 * a + 7) * D + c];
+#pragma unroll 4
+                for (int i = 16 * a; i < 16 * a + 16; ++i) safe = safe && fabsf(sG[i * D + c] - gm) <= kRefBound;
+            }
+            safe = __syncthreads_and(safe) != 0;
         }
         if (tid < D) {
             const int c = tid;
@@ -820,7 +844,6 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
         //      state-independent operands Q o e^Gamma (A1 rows 64..127) and K o e^{Gamma_C - Gamma}
         //      (A3) written out. (The pack is written for unsafe chunks too; the CUDA-core body
         //      then rewrites it.)
-        bool safe = true;
 #pragma unroll 1
         for (int hf = 0; hf < NH; ++hf) {
             if (hf > 0) {  // the previous part's MMA has finished reading the operand buffer
@@ -846,7 +869,6 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
 #pragma unroll
                 for (int w = 0; w < 8; ++w) {
                     const float r = gi[w] - gm[w];
-                    safe = safe && fabsf(r) <= kRefBound;
                     ef[w] = __expf(r);
                     ei[w] = __expf(-r);
                 }
@@ -891,11 +913,13 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
             // D[128 x 160] (+)= A . B^T over this part's 64 channels (L' in rows 0..63, M in 64..127)
             if (tid == 0) {
                 constexpr uint32_t id = idesc_bf16(128, I::NB, false, false);
-                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sBt);
+                const uint64_t dah = kmaj_desc(smem_u32(sA), 128, 0, 0), dal = kmaj_desc(smem_u32(sA) + I::A_H / 2, 128, 0, 0);
+                const uint64_t dbh = kmaj_desc(smem_u32(sBt), I::NB, 0, 0);
+                const uint64_t dbl = kmaj_desc(smem_u32(sBt) + I::B_H / 2, I::NB, 0, 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + I::A_H / 2, 128, 0, ks);
-                    const uint64_t bh = kmaj_desc(b0, I::NB, 0, ks), bl = kmaj_desc(b0 + I::B_H / 2, I::NB, 0, ks);
+                    const uint64_t ah = dah + kmaj_step(128, ks), al = dal + kmaj_step(128, ks);
+                    const uint64_t bh = dbh + kmaj_step(I::NB, ks), bl = dbl + kmaj_step(I::NB, ks);
                     mma_bf16(tmem, ah, bh, id, (hf > 0 || ks > 0) ? 1u : 0u);
                     mma_bf16(tmem, ah, bl, id, 1);
                     mma_bf16(tmem, al, bh, id, 1);
@@ -907,7 +931,6 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
             give_up(bar, mph & 1, item);
             continue;
         }
-        safe = __syncthreads_and(safe) != 0;
         ok = mbar_wait(bar, mph & 1, kWaitCycles);  // the last part's MMA
         tc_fence_after();
         if (!__syncthreads_and(ok)) {
@@ -1002,12 +1025,14 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
         // ---- [W | U~] = Tb . [K o A | V]  (M = 64, N = D each, K = 64) into TMEM columns 0..2D-1
         if (tid == 0) {
             constexpr uint32_t id = idesc_bf16(64, D, false, true);
-            const uint32_t a0 = smem_u32(sTb), bk = smem_u32(sKA), bv = smem_u32(sR2);
+            const uint64_t dah = kmaj_desc(smem_u32(sTb), 64, 0, 0), dal = kmaj_desc(smem_u32(sTb) + 8192, 64, 0, 0);
+            const uint64_t dkh = mnmaj_desc(smem_u32(sKA), C, 0, 0), dkl = mnmaj_desc(smem_u32(sKA) + I::KA / 2, C, 0, 0);
+            const uint64_t dvh = mnmaj_desc(smem_u32(sR2), C, 0, 0), dvl = mnmaj_desc(smem_u32(sR2) + I::KA / 2, C, 0, 0);
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 64, 0, ks), al = kmaj_desc(a0 + 8192, 64, 0, ks);
-                const uint64_t kh = mnmaj_desc(bk, C, 0, ks), kl = mnmaj_desc(bk + I::KA / 2, C, 0, ks);
-                const uint64_t vh = mnmaj_desc(bv, C, 0, ks), vl = mnmaj_desc(bv + I::KA / 2, C, 0, ks);
+                const uint64_t ah = dah + kmaj_step(64, ks), al = dal + kmaj_step(64, ks);
+                const uint64_t kh = dkh + mnmaj_step(ks), kl = dkl + mnmaj_step(ks);
+                const uint64_t vh = dvh + mnmaj_step(ks), vl = dvl + mnmaj_step(ks);
                 const uint32_t acc = ks > 0 ? 1u : 0u;
                 mma_bf16(tmem, ah, kh, id, acc);
                 mma_bf16(tmem, ah, kl, id, 1);
@@ -1027,34 +1052,48 @@ intra_tc_kernel(const __grid_constant__ CUtensorMap tmG, const PrefillIn in, uin
         ++mph;
         if (following < total) fetch_g(following);  // R2 is free: the next item's g box comes in
         // ---- read back (M = 64 layout: row 16 quad + lane in lanes < 16 of the quad); warp part 0
-        //      takes W (columns 0..D-1, into A1 rows 0..63 as BF16 hi + lo), part 1 U~ (FP32)
+        //      takes W (columns 0..D-1: rows 0..63 of A1, BF16 hi + lo), part 1 U~ (FP32), staged in
+        //      R1 in the pack's own layout (the operands there are dead) and written out by bulk copies
         {
+            uint8_t *sWs = sm;                                          // W: [hi|lo][D/64 panels][64 rows x 128 B]
+            float *sUs = reinterpret_cast<float *>(sm + I::W_STAGE);  // U~: the pack's UT layout
             const int quad = warp & 3, part = warp >> 2, row = 16 * quad + lane;
 #pragma unroll 1
-            for (int c16 = 0; c16 < D; c16 += 16) {
-                float x[16];
-                tmem_ld16(tmem_lane_base(tmem, warp) + part * D + c16, x);
+            for (int c32 = 0; c32 < D; c32 += 32) {
+                float x[2][16];
+                tmem_ld16(tmem_lane_base(tmem, warp) + part * D + c32, x[0]);
+                tmem_ld16(tmem_lane_base(tmem, warp) + part * D + c32 + 16, x[1]);
                 tmem_ld_wait();
                 if (lane < 16) {
 #pragma unroll
-                    for (int hl = 0; hl < 2; ++hl) {
-                        const int cc = c16 + 8 * hl;
-                        const float(&x8)[8] = *reinterpret_cast<const float(*)[8]>(x + 8 * hl);
+                    for (int hl = 0; hl < 4; ++hl) {
+                        const int cc = c32 + 8 * hl;
+                        const float(&x8)[8] = *reinterpret_cast<const float(*)[8]>(&x[hl >> 1][8 * (hl & 1)]);
                         if (part == 0) {
-                            st_pair_g(pack + PK::OFF_A1, PK::A1 / 2, kmaj_off(row, cc, 128), x8);
+                            st_pair(sWs, I::W_STAGE / 2, (cc >> 6) * 8192 + kmaj_off(row, cc & 63, 64), x8);
                         } else {
-                            float *dst = reinterpret_cast<float *>(pack + PK::OFF_UT + (cc >> 5) * PK::UG_BYTES) +
-                                         row * PK::UP + (cc & 31);
+                            float *dst = sUs + (cc >> 5) * (PK::UG_BYTES / 4) + row * PK::UP + (cc & 31);
                             *reinterpret_cast<float4 *>(dst) = make_float4(x8[0], x8[1], x8[2], x8[3]);
                             *reinterpret_cast<float4 *>(dst + 4) = make_float4(x8[4], x8[5], x8[6], x8[7]);
                         }
                     }
                 }
             }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();  // TMEM is read: the next item's MMAs may overwrite it
+            if (tid == 0) {
+#pragma unroll
+                for (int p = 0; p < D / 64; ++p) {
+                    bulk_store(pack + PK::OFF_A1 + p * 16384, sWs + p * 8192, 8192);
+                    bulk_store(pack + PK::OFF_A1 + PK::A1 / 2 + p * 16384, sWs + I::W_STAGE / 2 + p * 8192, 8192);
+                }
+                bulk_store(pack + PK::OFF_UT, sUs, PK::UT);
+                bulk_commit();
+            }
         }
-        tc_fence_before();
-        __syncthreads();  // TMEM is read: the next item's MMAs may overwrite it
     }
+    if (tid == 0) bulk_wait_all();  // every staged result is in global memory
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
@@ -1069,14 +1108,18 @@ struct State {
     static constexpr int A2 = 2 * kTileBytes;       // [0; M]: 128 x 64 K-major hi + lo, rows 0..63 zero
     static constexpr int B1 = 2 * NB * D * 2;       // S0 hi + lo, MN-major (N = value columns, K = D keys)
     static constexpr int B2 = 2 * NB * C * 2;       // U hi + lo, MN-major (N = value columns, K = 64)
+    // two U operands where they fit: a chunk's output group (D1 += [0; M] U) then runs after the
+    // next chunk's D1, beside its epilogue, instead of ahead of it in the tensor pipe
+    static constexpr int NU = PK::A1 + 2 * kTileBytes + PK::A3 + B1 + 2 * B2 + 2048 <= 232448 ? 2 : 1;
     static constexpr int OFF_A1 = 0, OFF_A2 = PK::A1, OFF_A3 = OFF_A2 + A2, OFF_B1 = OFF_A3 + PK::A3,
-                         OFF_B2 = OFF_B1 + B1, OFF_MISC = OFF_B2 + B2;
+                         OFF_B2 = OFF_B1 + B1, OFF_MISC = OFF_B2 + NU * B2;
     static constexpr int MISC = 1024;
     static constexpr int bytes = OFF_MISC + MISC + 1024;  // + alignment slack
     static_assert(bytes <= 232448, "one CTA per SM");
-    // D1 twice (chunk parity: a chunk's outputs are read while the next chunk's D1 is computed), D3
-    static constexpr uint32_t TMEM_COLS =
-        3 * DVS <= 32 ? 32 : (3 * DVS <= 64 ? 64 : (3 * DVS <= 128 ? 128 : (3 * DVS <= 256 ? 256 : 512)));
+    // D1 twice (chunk parity: a chunk's outputs are read while the next chunk's D1 is computed), D3,
+    // and the FP32 master copy of the state slice (key row = lane, value column = column)
+    static constexpr uint32_t TMEM_COLS = 4 * DVS;
+    static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512, "TMEM columns");
 };
 
 // A bulk global -> shared copy completing on `bar`, whose expected bytes were already
@@ -1099,28 +1142,39 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
 
 // The chain of one (stream, head, value slice of DVS columns) over its chunks. Per chunk:
 //   MMA group 1   D1 = [W; Q o A] . S0                       (M = 128, N = DVS, K = D)
-//   epilogue 1    U = U~ - D1[0:64] into shared memory (U~ read from the pack into registers
-//                 while group 1 runs)
-//   MMA group 2   D3 = (K o e^{Gamma_C - Gamma})^T . U        (M = D, N = DVS, K = 64), committed alone
+//   epilogue 1    U = U~ - D1[0:64] into shared memory
+//   MMA group 2   D3 = (K o e^{Gamma_C - Gamma})^T . U        (M = D, N = DVS, K = 64)
 //   MMA group 3   D1 += [0; M] . U                            (so D1[64:128] = (Q o A) S0 + M U)
 //   epilogue 2    S = A_C o S0 + D3 (FP32 master copy in registers) into the S operand
-// Groups 1 and 2 and the two epilogues are the critical path; group 3 and the output rows
-// O = scale D1[64:128] run beside the next chunk.
+// Groups 1 and 2 and the two epilogues are the critical path. Warp kEpiWarps (the control warp)
+// issues every copy and every MMA, so that the epilogue warps never stall behind the tensor
+// pipe's back-pressure on MMA issue. Group 3 of chunk c is issued right after group 1 of chunk
+// c + 1 (with two U operands in shared memory), so it runs while epilogue 1 of c + 1 does instead
+// of delaying that group 1; the output rows O = scale D1[64:128] of chunk c are read while group
+// 2 of chunk c + 1 runs. Epilogue and control warps hand over through mbarriers.
+constexpr int kEpiWarps = 8;
+constexpr int kStateThreads = 32 * (kEpiWarps + 1);
+
 template <int D, int DVS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core,
              const Seqs sq, int H, float scale, float *__restrict__ tables, int *__restrict__ status) {
     using S = State<D, DVS>;
     using PK = Pack<D>;
-    constexpr int HALF = DVS / 2;  // value columns per thread in the epilogues
+    constexpr int HALF = DVS / 2;         // value columns per epilogue thread
+    // U~ read into registers while group 1 runs (slices up to 64 columns; wider slices read it one
+    // 8-column group ahead: with 9 warps one scheduler holds three, so a thread has about 168 registers)
+    constexpr bool kPreU = HALF <= 32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = sm + S::OFF_A1, *sA2 = sm + S::OFF_A2, *sA3 = sm + S::OFF_A3, *sB1 = sm + S::OFF_B1,
             *sB2 = sm + S::OFF_B2;
-    // barriers: copies 0 A1, 1 M, 2 A3; MMA groups 4 (D1), 5 (D3), 6 (D1 += [0; M] U); 7 the
-    // final drain after a timeout
+    // barriers: copies 0 A1, 1 M, 2 A3; MMA groups 4 (D1), 5 (D3), 6 (D1 += [0; M] U); 7 the final
+    // drain after a timeout; 8 "U is in B2" and 9 "S is in B1, D3 read" (one arrival per epilogue
+    // warp, after the warp's own writes and TMEM reads)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 64);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 128);
+    int *fail = reinterpret_cast<int *>(sm + S::OFF_MISC + 136);  // a role gave up waiting
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -1139,6 +1193,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     if (nb == 0) return;  // an empty stream keeps its state
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
     const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
+    const bool ctl = warp == kEpiWarps && lane == 0;  // the control thread
 
     auto copy_m = [&](const uint8_t *pk) {  // M's hi and lo halves into rows 64..127 of A2
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bars[1])),
@@ -1147,238 +1202,302 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         bulk_copy_nx(sA2 + 8192, pk + PK::OFF_AM, PK::AM / 2, &bars[1]);
         bulk_copy_nx(sA2 + kTileBytes + 8192, pk + PK::OFF_AM + PK::AM / 2, PK::AM / 2, &bars[1]);
     };
-    // thread 0 issues every copy and counts, per copy barrier, the copies issued and the phases
-    // it has waited for (so that a timed-out CTA can drain what is still in flight)
-    uint32_t issued[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
-    auto wait_copy = [&](int k) {
-        const bool r = mbar_wait(&bars[k], waited[k] & 1, kWaitCycles);
-        if (r) ++waited[k];
-        return r;
-    };
-    if (tid == 0) {
+    if (ctl) {
         for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&bars[8], kEpiWarps);  // one arrival per epilogue warp
+        mbar_init(&bars[9], kEpiWarps);
+        *fail = 0;
         fence_mbar_init();
         bulk_copy(sA1, packs + PK::OFF_A1, PK::A1, &bars[0]);
         copy_m(packs);
         bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[2]);
-        issued[0] = issued[1] = issued[2] = 1;
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
         tmem_relinquish();
     }
     // rows 0..63 of both halves of A2 stay zero: D1 += [0; M] U adds nothing to rows 0..63
-    for (int e = tid; e < 2 * 8192 / 16; e += kThreads) {
+    for (int e = tid; e < 2 * 8192 / 16; e += kStateThreads) {
         const int half = e / (8192 / 16), off = (e % (8192 / 16)) * 16;
         *reinterpret_cast<uint4 *>(sA2 + half * kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tD3 = tmem + 2 * DVS;
-    bool ok = true;
-
     // Epilogue roles: for an M = 128 accumulator warp w reads TMEM lanes 32(w%4)..+31 (rows),
     // value columns [(w/4) HALF, + HALF). D3 with D = 64 (M = 64) has rows 16 (w%4) + lane, lane < 16.
     const int quad = warp & 3, colh = warp >> 2;
     const int erow = 32 * quad + lane;
     const int ccol = colh * HALF;
-    const int srow = (D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1);
-
-    // FP32 master state slice: key row srow, value columns [c0 + ccol, + HALF)
-    float st[HALF];
-    if (srow >= 0) {
+    const int srow = warp >= kEpiWarps ? -1 : ((D == 128) ? erow : ((lane < 16) ? 16 * quad + lane : -1));
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tD3 = tmem + 2 * DVS;
+    // the FP32 master state slice lives in TMEM: key row srow in this thread's own lane, value
+    // columns [ccol, ccol + HALF) of the slice at tS (lanes of rows that do not exist hold zeros)
+    const uint32_t tS = tmem_lane_base(tmem + 3 * DVS, warp) + ccol;
+    if (warp < kEpiWarps) {
 #pragma unroll
-        for (int j = 0; j < HALF; j += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(Sg + static_cast<size_t>(srow) * D + c0 + ccol + j);
-            st[j] = x.x; st[j + 1] = x.y; st[j + 2] = x.z; st[j + 3] = x.w;
-        }
-    }
-    // S0 into B1 (MN-major: element (n = value column, k = key row)), 16-byte chunks
-    auto write_state_operand = [&]() {
-        if (srow >= 0) {
-#pragma unroll
-            for (int j = 0; j < HALF; j += 8) {
-                float x[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) x[u] = st[j + u];
+        for (int j = 0; j < HALF; j += 8) {
+            float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (srow >= 0) {
+                const float *src = Sg + static_cast<size_t>(srow) * D + c0 + ccol + j;
+                const float4 a = *reinterpret_cast<const float4 *>(src), c = *reinterpret_cast<const float4 *>(src + 4);
+                x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+                // S0 into B1 (MN-major: element (n = value column, k = key row)), 16-byte chunks
                 st_pair(sB1, S::B1 / 2, mnmaj_off(ccol + j, srow, D), x);
             }
+            tmem_st8(tS + j, x);
         }
-    };
-    write_state_operand();
+        tmem_st_wait();
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // O = scale D1[64:128] of chunk c (quads 2 and 3: TMEM lanes 64..127 = the chunk's tokens),
-    // once group 3 of chunk c has completed; run while the tensor core computes chunk c + 1
-    auto out_epilogue = [&](int c) {
-        ok = ok && mbar_wait(&bars[6], c & 1, kWaitCycles);
-        tc_fence_after();
-        const int i = erow - 64;
-        int nn;
-        size_t r0;
-        seq_chunk(sq, b, c, r0, nn, nullptr);
-        const uint32_t tD1c = tmem + (c & 1) * DVS;
-#pragma unroll
-        for (int j = 0; j < HALF; j += 8) {
-            float x[8];
-            tmem_ld8(tmem_lane_base(tD1c, warp) + ccol + j, x);
-            tmem_ld_wait();
-            if (i < nn && ok) {
-                float *dst = core + (r0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
-                *reinterpret_cast<float4 *>(dst) = make_float4(scale * x[0], scale * x[1], scale * x[2], scale * x[3]);
-                *reinterpret_cast<float4 *>(dst + 4) =
-                    make_float4(scale * x[4], scale * x[5], scale * x[6], scale * x[7]);
-            }
-        }
-    };
+    bool ok = true;
 
+    if (warp == kEpiWarps) {
+        // ================================================= control warp (lane 0 works)
+        if (ctl) {
+            uint32_t issued[3] = {1, 1, 1}, waited[3] = {0, 0, 0};
+            auto wait_copy = [&](int k) {
+                const bool r = mbar_wait(&bars[k], waited[k] & 1, kWaitCycles);
+                if (r) ++waited[k];
+                return r;
+            };
+            auto give_up = [&]() {
+                ok = false;
+                atomicExch(fail, 1);
+            };
+            // K-step-0 descriptors of every operand (the buffers never move)
+            const uint64_t dA1h = kmaj_desc(smem_u32(sA1), 128, 0, 0), dA1l = kmaj_desc(smem_u32(sA1) + PK::A1 / 2, 128, 0, 0);
+            const uint64_t dB1h = mnmaj_desc(smem_u32(sB1), D, 0, 0), dB1l = mnmaj_desc(smem_u32(sB1) + S::B1 / 2, D, 0, 0);
+            const uint64_t dA3h = mnmaj_desc(smem_u32(sA3), C, 0, 0), dA3l = mnmaj_desc(smem_u32(sA3) + PK::A3 / 2, C, 0, 0);
+            const uint64_t dA2h = kmaj_desc(smem_u32(sA2), 128, 0, 0), dA2l = kmaj_desc(smem_u32(sA2) + kTileBytes, 128, 0, 0);
+            const uint64_t dB2h = mnmaj_desc(smem_u32(sB2), C, 0, 0), dB2l = mnmaj_desc(smem_u32(sB2) + S::B2 / 2, C, 0, 0);
+            constexpr uint64_t kB2Buf = static_cast<uint64_t>(S::B2 >> 4);  // one U buffer, in descriptor units
+            // the output group (D1 += [0; M] U) of chunk c: U from B2 buffer c % NU, M from A2
+            auto issue_out_group = [&](int c) {
+                constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
+                const uint64_t ub = (c % S::NU) * kB2Buf;
+                const uint32_t tD1c = tmem + (c & 1) * DVS;
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks) {
+                    const uint64_t bh = dB2h + ub + mnmaj_step(ks), bl = dB2l + ub + mnmaj_step(ks);
+                    const uint64_t mh = dA2h + kmaj_step(128, ks), ml = dA2l + kmaj_step(128, ks);
+                    mma_bf16(tD1c, mh, bh, idm, 1);
+                    mma_bf16(tD1c, mh, bl, idm, 1);
+                    mma_bf16(tD1c, ml, bh, idm, 1);
+                }
+                mma_commit(&bars[6]);
+            };
 #pragma unroll 1
-    for (int ch = 0; ch < nb; ++ch) {
-        const uint32_t par = ch & 1;
-        const uint32_t tD1 = tmem + par * DVS;
-        const uint8_t *cur = packs + static_cast<size_t>(ch) * PK::bytes;
-        const uint8_t *next = cur + PK::bytes;
-        const bool more = ch + 1 < nb;
-        // e^{Gamma_C} of this thread's key row (epilogue 2) and U~ of its row (epilogue 1), read
-        // from the pack while group 1 runs
-        const float ac = srow >= 0 ? reinterpret_cast<const float *>(cur + PK::OFF_AC)[srow] : 0.f;
-        float ut[HALF];
-        if (quad < 2) {
+            for (int ch = 0; ch < nb && ok; ++ch) {
+                const uint32_t par = ch & 1;
+                const uint32_t tD1 = tmem + par * DVS;
+                const uint8_t *cur = packs + static_cast<size_t>(ch) * PK::bytes;
+                const uint8_t *next = cur + PK::bytes;
+                const bool more = ch + 1 < nb;
+                // S of this chunk is in B1 (the epilogue's previous round), A1 has landed
+                if (ch > 0 && !mbar_wait(&bars[9], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
+                if (!wait_copy(0)) { give_up(); break; }
+                tc_fence_after();
+                {
+                    constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
 #pragma unroll
-            for (int j = 0; j < HALF; j += 4) {
-                const int c = c0 + ccol + j;
-                const float4 u4 = *reinterpret_cast<const float4 *>(
-                    reinterpret_cast<const float *>(cur + PK::OFF_UT + (c >> 5) * PK::UG_BYTES) + erow * PK::UP + (c & 31));
-                ut[j] = u4.x; ut[j + 1] = u4.y; ut[j + 2] = u4.z; ut[j + 3] = u4.w;
-            }
-        }
-        // ---- MMA group 1: D1 = [W; Q o A] . S0
-        if (tid == 0 && ok) ok = wait_copy(0);
-        if (tid == 0 && ok) {
-            constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
-            const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t ah = kmaj_desc(a0, 128, 0, ks), al = kmaj_desc(a0 + PK::A1 / 2, 128, 0, ks);
-                const uint64_t bh = mnmaj_desc(b0, D, 0, ks), bl = mnmaj_desc(b0 + S::B1 / 2, D, 0, ks);
-                mma_bf16(tD1, ah, bh, id, ks > 0 ? 1u : 0u);
-                mma_bf16(tD1, ah, bl, id, 1);
-                mma_bf16(tD1, al, bh, id, 1);
-            }
-            mma_commit(&bars[4]);
-            // group 3 of the previous chunk has read M: the next M may come in
-            if (ch > 0) {
-                ok = mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles);
-                if (ok) {
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t ah = dA1h + kmaj_step(128, ks), al = dA1l + kmaj_step(128, ks);
+                        const uint64_t bh = dB1h + mnmaj_step(ks), bl = dB1l + mnmaj_step(ks);
+                        mma_bf16(tD1, ah, bh, id, ks > 0 ? 1u : 0u);
+                        mma_bf16(tD1, ah, bl, id, 1);
+                        mma_bf16(tD1, al, bh, id, 1);
+                    }
+                    mma_commit(&bars[4]);
+                }
+                if (S::NU == 2 && ch > 0) {  // the previous chunk's output group, behind this D1
+                    if (!wait_copy(1)) { give_up(); break; }
+                    issue_out_group(ch - 1);
+                }
+                if (S::NU == 1 && ch > 0) {  // the previous output group has read M: this chunk's M
+                    if (!mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
                     copy_m(cur);
                     ++issued[1];
                 }
+                if (!mbar_wait(&bars[4], par, kWaitCycles)) { give_up(); break; }
+                if (more) {  // A1 is free again
+                    bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);
+                    ++issued[0];
+                }
+                // U is in B2
+                if (!mbar_wait(&bars[8], par, kWaitCycles)) { give_up(); break; }
+                if (!wait_copy(2)) { give_up(); break; }
+                tc_fence_after();
+                {
+                    constexpr uint32_t id3 = idesc_bf16(D, DVS, true, true);
+                    const uint64_t ub = (ch % S::NU) * kB2Buf;
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks) {
+                        const uint64_t bh = dB2h + ub + mnmaj_step(ks), bl = dB2l + ub + mnmaj_step(ks);
+                        const uint64_t ah = dA3h + mnmaj_step(ks), al = dA3l + mnmaj_step(ks);
+                        mma_bf16(tD3, ah, bh, id3, ks > 0 ? 1u : 0u);
+                        mma_bf16(tD3, ah, bl, id3, 1);
+                        mma_bf16(tD3, al, bh, id3, 1);
+                    }
+                    mma_commit(&bars[5]);
+                }
+                if (S::NU == 2 && ch > 0) {  // the previous output group has read M (it ran ahead of group 2)
+                    if (!mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
+                    copy_m(cur);
+                    ++issued[1];
+                }
+                if (S::NU == 1 || !more) {  // one U buffer (or the last chunk): the output group now
+                    if (!wait_copy(1)) { give_up(); break; }
+                    issue_out_group(ch);
+                }
+                if (more) {  // A3 is free once group 2 has completed
+                    if (!mbar_wait(&bars[5], par, kWaitCycles)) { give_up(); break; }
+                    bulk_copy(sA3, next + PK::OFF_A3, PK::A3, &bars[2]);
+                    ++issued[2];
+                }
+            }
+            if (!ok) {
+                // drain (bounded): every MMA issued, then every copy still in flight
+                mma_commit(&bars[7]);
+                mbar_wait(&bars[7], 0, kWaitCycles);
+                for (int k = 0; k < 3; ++k)
+                    while (waited[k] < issued[k] && wait_copy(k)) {
+                    }
             }
         }
-        if (ch > 0 && quad >= 2) out_epilogue(ch - 1);
-        ok = ok && mbar_wait(&bars[4], par, kWaitCycles);
-        tc_fence_after();
-        if (tid == 0 && ok && more) {  // A1 is free again
-            bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);
-            ++issued[0];
-        }
-        // ---- epilogue 1: U = U~ - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
-        if (quad < 2) {
+    } else {
+        // ================================================= epilogue warps
+        // O = scale D1[64:128] of chunk c (quads 2 and 3: TMEM lanes 64..127 = the chunk's tokens),
+        // once group 3 of chunk c has completed
+        auto out_epilogue = [&](int c) {
+            ok = ok && mbar_wait(&bars[6], c & 1, kWaitCycles);
+            tc_fence_after();
+            const int i = erow - 64;
+            int nn;
+            size_t r0;
+            seq_chunk(sq, b, c, r0, nn, nullptr);
+            const uint32_t tD1c = tmem + (c & 1) * DVS;
 #pragma unroll
             for (int j = 0; j < HALF; j += 8) {
                 float x[8];
-                tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
+                tmem_ld8(tmem_lane_base(tD1c, warp) + ccol + j, x);
+                tmem_ld_wait();
+                if (i < nn && ok) {
+                    float *dst = core + (r0 + i) * rs + static_cast<size_t>(h) * D + c0 + ccol + j;
+                    *reinterpret_cast<float4 *>(dst) =
+                        make_float4(scale * x[0], scale * x[1], scale * x[2], scale * x[3]);
+                    *reinterpret_cast<float4 *>(dst + 4) =
+                        make_float4(scale * x[4], scale * x[5], scale * x[6], scale * x[7]);
+                }
+            }
+        };
+#pragma unroll 1
+        for (int ch = 0; ch < nb; ++ch) {
+            const uint32_t par = ch & 1;
+            const uint32_t tD1 = tmem + par * DVS;
+            const uint8_t *cur = packs + static_cast<size_t>(ch) * PK::bytes;
+            const float ac = srow >= 0 ? reinterpret_cast<const float *>(cur + PK::OFF_AC)[srow] : 0.f;
+            auto ut_ptr = [&](int j) {  // U~ of this thread's row, value columns c0 + ccol + j ..
+                const int c = c0 + ccol + j;
+                return reinterpret_cast<const float *>(cur + PK::OFF_UT + (c >> 5) * PK::UG_BYTES) + erow * PK::UP +
+                       (c & 31);
+            };
+            float ut[kPreU ? HALF : 1];
+            if (kPreU && quad < 2) {
+#pragma unroll
+                for (int j = 0; j < (kPreU ? HALF : 0); j += 4) {
+                    const float4 u4 = *reinterpret_cast<const float4 *>(ut_ptr(j));
+                    ut[j] = u4.x; ut[j + 1] = u4.y; ut[j + 2] = u4.z; ut[j + 3] = u4.w;
+                }
+            }
+            ok = ok && mbar_wait(&bars[4], par, kWaitCycles);
+            tc_fence_after();
+            // ---- epilogue 1: U = U~ - D1[0:64] -> B2 (MN-major: element (n = value column, k = token))
+            if (quad < 2) {
+                float4 un0 = make_float4(0.f, 0.f, 0.f, 0.f), un1 = un0;  // the next group of U~ (wide slices)
+                if (!kPreU) {
+                    un0 = *reinterpret_cast<const float4 *>(ut_ptr(0));
+                    un1 = *reinterpret_cast<const float4 *>(ut_ptr(0) + 4);
+                }
+#pragma unroll
+                for (int j = 0; j < HALF; j += 8) {
+                    float x[8];
+                    tmem_ld8(tmem_lane_base(tD1, warp) + ccol + j, x);
+                    float u8[8];
+                    if constexpr (kPreU) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) u8[u] = ut[j + u];
+                    } else {
+                        u8[0] = un0.x; u8[1] = un0.y; u8[2] = un0.z; u8[3] = un0.w;
+                        u8[4] = un1.x; u8[5] = un1.y; u8[6] = un1.z; u8[7] = un1.w;
+                        if (j + 8 < HALF) {
+                            un0 = *reinterpret_cast<const float4 *>(ut_ptr(j + 8));
+                            un1 = *reinterpret_cast<const float4 *>(ut_ptr(j + 8) + 4);
+                        }
+                    }
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) x[u] = u8[u] - x[u];
+                    if (tables && ok) {  // verify mode: U of every row, for the fold
+                        float *utab = tables + (static_cast<size_t>(b) * H + h) * 2 * C * D + erow * D + c0 + ccol + j;
+                        *reinterpret_cast<float4 *>(utab) = make_float4(x[0], x[1], x[2], x[3]);
+                        *reinterpret_cast<float4 *>(utab + 4) = make_float4(x[4], x[5], x[6], x[7]);
+                    }
+                    st_pair(sB2 + (ch % S::NU) * S::B2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[8]);
+            // the previous chunk's output rows, while group 2 runs
+            if (ch > 0 && quad >= 2) out_epilogue(ch - 1);
+            // ---- epilogue 2: S = A_C o S0 + D3 (the FP32 master copy in TMEM), S into B1
+            ok = ok && mbar_wait(&bars[5], par, kWaitCycles);
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < HALF; j += 8) {
+                float x[8], sv[8];
+                tmem_ld8(tmem_lane_base(tD3, warp) + ccol + j, x);
+                tmem_ld8(tS + j, sv);
                 tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 8; ++u) x[u] = ut[j + u] - x[u];
-                if (tables && ok) {  // verify mode: U of every row, for the fold
-                    float *utab = tables + (static_cast<size_t>(b) * H + h) * 2 * C * D + erow * D + c0 + ccol + j;
-                    *reinterpret_cast<float4 *>(utab) = make_float4(x[0], x[1], x[2], x[3]);
-                    *reinterpret_cast<float4 *>(utab + 4) = make_float4(x[4], x[5], x[6], x[7]);
-                }
-                st_pair(sB2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
+                for (int u = 0; u < 8; ++u) sv[u] = fmaf(ac, sv[u], x[u]);
+                tmem_st8(tS + j, sv);
+                if (srow >= 0) st_pair(sB1, S::B1 / 2, mnmaj_off(ccol + j, srow, D), sv);
+            }
+            tmem_st_wait();
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[9]);
+            if (!ok || *reinterpret_cast<volatile int *>(fail)) {
+                ok = false;
+                break;
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;
+        if (ok && quad >= 2) out_epilogue(nb - 1);
+    }
+    ok = __syncthreads_and(ok && *reinterpret_cast<volatile int *>(fail) == 0) != 0;
+    if (!ok) {
+        if (tid == 0) atomicExch(status, KDA_ERR_TIMEOUT);
+    } else if (warp < kEpiWarps && !tables) {  // verify mode leaves the state as it was
         tc_fence_after();
-        // ---- MMA group 2: D3 = (K o e^{Gamma_C - Gamma})^T . U (the chain), then group 3:
-        //      D1 += [0; M] . U (the output rows), each committed on its own
-        if (tid == 0 && ok) ok = wait_copy(2);
-        if (tid == 0 && ok) {
-            constexpr uint32_t id3 = idesc_bf16(D, DVS, true, true);
-            const uint32_t a3 = smem_u32(sA3), b0 = smem_u32(sB2);
-#pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
-                const uint64_t ah = mnmaj_desc(a3, C, 0, ks), al = mnmaj_desc(a3 + PK::A3 / 2, C, 0, ks);
-                mma_bf16(tD3, ah, bh, id3, ks > 0 ? 1u : 0u);
-                mma_bf16(tD3, ah, bl, id3, 1);
-                mma_bf16(tD3, al, bh, id3, 1);
-            }
-            mma_commit(&bars[5]);
-            ok = wait_copy(1);
-            if (ok) {
-                constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
-                const uint32_t a2 = smem_u32(sA2);
-#pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks) {
-                    const uint64_t bh = mnmaj_desc(b0, C, 0, ks), bl = mnmaj_desc(b0 + S::B2 / 2, C, 0, ks);
-                    const uint64_t mh = kmaj_desc(a2, 128, 0, ks), ml = kmaj_desc(a2 + kTileBytes, 128, 0, ks);
-                    mma_bf16(tD1, mh, bh, idm, 1);
-                    mma_bf16(tD1, mh, bl, idm, 1);
-                    mma_bf16(tD1, ml, bh, idm, 1);
-                }
-                mma_commit(&bars[6]);
-            }
-        }
-        ok = ok && mbar_wait(&bars[5], par, kWaitCycles);
-        tc_fence_after();
-        if (tid == 0 && ok && more) {  // A3 is free again
-            bulk_copy(sA3, next + PK::OFF_A3, PK::A3, &bars[2]);
-            ++issued[2];
-        }
-        // ---- epilogue 2: S = A_C o S0 + D3 (FP32 in registers), S into B1
 #pragma unroll
         for (int j = 0; j < HALF; j += 8) {
-            float x[8];
-            tmem_ld8(tmem_lane_base(tD3, warp) + ccol + j, x);
+            float sv[8];
+            tmem_ld8(tS + j, sv);
             tmem_ld_wait();
             if (srow >= 0) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) st[j + u] = fmaf(ac, st[j + u], x[u]);
+                float *dst = Sg + static_cast<size_t>(srow) * D + c0 + ccol + j;
+                *reinterpret_cast<float4 *>(dst) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+                *reinterpret_cast<float4 *>(dst + 4) = make_float4(sv[4], sv[5], sv[6], sv[7]);
             }
         }
-        write_state_operand();
-        fence_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;
-        tc_fence_after();
-        if (!ok) break;  // block-uniform: every thread saw the same flag
-    }
-    if (ok && quad >= 2) out_epilogue(nb - 1);
-    ok = __syncthreads_and(ok) != 0;
-    if (!ok) {
-        if (tid == 0) {
-            atomicExch(status, KDA_ERR_TIMEOUT);
-            // drain (bounded): every MMA this thread issued, then every copy still in flight, so that
-            // nothing reads or writes shared memory or TMEM once they are released
-            mma_commit(&bars[7]);
-            mbar_wait(&bars[7], 0, kWaitCycles);
-            for (int k = 0; k < 3; ++k)
-                while (waited[k] < issued[k] && wait_copy(k)) {
-                }
-        }
-    } else if (srow >= 0 && !tables) {  // verify mode leaves the state as it was
-#pragma unroll
-        for (int j = 0; j < HALF; j += 4)
-            *reinterpret_cast<float4 *>(Sg + static_cast<size_t>(srow) * D + c0 + ccol + j) =
-                make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
     }
     tc_fence_before();
     __syncthreads();
@@ -1413,18 +1532,27 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     // two tensor-core intra CTAs per SM; the CUDA-core fix-up runs one per SM
     const int grid = static_cast<int>(std::min<long long>(items, 2LL * sms));
     const int grid_fix = static_cast<int>(std::min<long long>(items, sms));
-    // g box map: (stream, row in stream) for equal-length streams; the packed rows in varlen mode
+    // row maps: (stream, row in stream) for equal-length streams; the packed rows in varlen mode
     const int mT = sq.cu ? sq.total : sq.T, mTp = sq.cu ? sq.total : sq.T_pad, mB = sq.cu ? 1 : B;
-    CUtensorMap tmG;
+    InMaps maps;
     if (kGraw<MODE>)
-        KDA_TRY(make_rows_map(&tmG, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, mT, mTp, mB, D, C));
+        KDA_TRY(make_rows_map(&maps.g, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, mT, mTp, mB, D, C));
     else
-        KDA_TRY(make_rows_map(&tmG, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-    intra_tc_kernel<D, MODE><<<grid, kTcThreads, IntraTC<D>::bytes, s>>>(tmG, in, sc, list, B, sq, H, status);
+        KDA_TRY(make_rows_map(&maps.g, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
+    if (kQkv16<MODE>) {
+        KDA_TRY(make_rows_map(&maps.q, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, mT, mTp, mB, D, C));
+        maps.k = maps.q;
+        maps.v = maps.q;
+    } else {
+        KDA_TRY(make_rows_map(&maps.q, in.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
+        KDA_TRY(make_rows_map(&maps.k, in.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
+        KDA_TRY(make_rows_map(&maps.v, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
+    }
+    intra_tc_kernel<D, MODE><<<grid, kTcThreads, IntraTC<D>::bytes, s>>>(maps, in, sc, list, B, sq, H, status);
     KDA_TRY(launch_status());
     intra_fix_kernel<D, MODE><<<grid_fix, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
-    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
+    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kStateThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
                                                                                    in.tables, status);
     return launch_status();
 }

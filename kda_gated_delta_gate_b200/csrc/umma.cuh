@@ -59,6 +59,15 @@ __device__ __forceinline__ uint64_t mnmaj_desc(uint32_t base, int Kx, int mn0, i
     return sdesc(base + (mn0 >> 6) * (Kx * 128) + ks * 2048, Kx * 128, 1024);
 }
 
+// The descriptor of K-step ks minus that of K-step 0, for kmaj_desc (R rows) and mnmaj_desc: the
+// start-address field counts 16-byte units, and a tile ends below 256 KB of shared memory, so the
+// offset never carries into the other fields. An issuing thread keeps the K-step-0 descriptors
+// and adds these constants (an unrolled K loop folds them into immediates).
+__host__ __device__ constexpr uint64_t kmaj_step(int R, int ks) {
+    return static_cast<uint64_t>(((ks >> 2) * (R * 128) + (ks & 3) * 32) >> 4);
+}
+__host__ __device__ constexpr uint64_t mnmaj_step(int ks) { return static_cast<uint64_t>((ks * 2048) >> 4); }
+
 // Instruction descriptor, kind::f16: BF16 A and B, FP32 D, dense, no negation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
@@ -79,14 +88,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One try: true once phase `parity` of the barrier has completed. The thread may be suspended
+// inside the instruction until the phase completes or up to kSuspendNs nanoseconds pass, so a
+// waiting warp does not spin and take issue slots from the warps that are working.
+constexpr uint32_t kSuspendNs = 100000;
 __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t addr, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(done)
-        : "r"(addr), "r"(parity)
+        : "r"(addr), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return done;
 }

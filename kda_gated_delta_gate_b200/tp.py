@@ -5,10 +5,12 @@ each take H / world heads: the output channels of those heads in q/k/v, f_b, g_b
 rows of their q, k and v channels, their dt_bias and a_log entries, their b_proj rows, and
 the matching input columns of o_proj; f_a, g_a and o_norm are replicated. Each rank runs the
 block on its heads (kda_block_prefill / kda_block_decode with o_proj = NULL, so the calls stop
-at o_norm_out), multiplies by its o_proj slice into an FP32 [rows, hidden] partial, and the
-partials are summed across ranks by one all-reduce (torch.distributed: NCCL over NVLink on
-GPUs, gloo on CPU); the sum is rounded to BF16 once, as the unsharded o_proj rounds its
-FP32 accumulation once.
+at o_norm_out), multiplies by its o_proj slice into a [rows, hidden] partial, and the partials
+are summed across ranks by one all-reduce (torch.distributed: NCCL over NVLink on GPUs, gloo on
+CPU). By default the partial is the BF16 block output of this rank's heads and the all-reduce
+runs on BF16, as the mixer all-reduce of the pages moves the block output (2 bytes per value);
+reduce_dtype="fp32" keeps the partials in FP32 and rounds the sum once, as the unsharded o_proj
+rounds its FP32 accumulation once, at twice the bytes on the links.
 
 This module is plumbing around the C ABI: every step of the block runs in libkda's kernels.
 """
@@ -58,11 +60,14 @@ class TPBlock:
 
     shard: the output of shard_block_weights with device tensors. max_tokens sizes the
     workspace. group: a torch.distributed process group (None: the default group if
-    torch.distributed is initialised, else no reduction: the caller sums the partials)."""
+    torch.distributed is initialised, else no reduction: the caller sums the partials).
+    reduce_dtype: "bf16" (the partials and the all-reduce in BF16) or "fp32"."""
 
     def __init__(self, shard, max_tokens: int, group=None, l2_eps: float = 1e-6, rms_eps: float = 1e-6,
-                 scale: float = 1.0):
+                 scale: float = 1.0, reduce_dtype: str = "bf16"):
         import torch
+        if reduce_dtype not in ("bf16", "fp32"):
+            raise ValueError(f"reduce_dtype must be bf16 or fp32, not {reduce_dtype}")
         self.w = shard
         self.H, self.D, self.hidden = shard.H, shard.D, shard.hidden
         self.dw = types.SimpleNamespace(
@@ -72,7 +77,8 @@ class TPBlock:
         self.st = kda.block_weights_struct(self.dw)
         self.ws = kda.Workspace(kda.dims(self.H, self.D, scale=scale, l2_eps=l2_eps, rms_eps=rms_eps), shard.hidden,
                                 shard.rank, max_tokens)
-        self.partial = torch.empty((max_tokens, shard.hidden), dtype=torch.float32, device=shard.w_q.device)
+        dt = torch.bfloat16 if reduce_dtype == "bf16" else torch.float32
+        self.partial = torch.empty((max_tokens, shard.hidden), dtype=dt, device=shard.w_q.device)
         self.group = group
 
     def _reduce(self, rows: int):
@@ -86,13 +92,13 @@ class TPBlock:
         return part
 
     def prefill(self, hidden, T: int, h_state, conv_state, pad_fill: float = 0.0):
-        """The block prefill of T rows on this rank's heads; returns the FP32 [T, hidden] output
-        summed over the group (round it to BF16 for the block output)."""
+        """The block prefill of T rows on this rank's heads; returns the [T, hidden] output summed
+        over the group (BF16; with reduce_dtype "fp32" the FP32 sum, to be rounded to BF16)."""
         kda.kda_block_prefill(self.st, hidden, T, h_state, conv_state, pad_fill, self.ws)
         return self._reduce(T)
 
     def decode(self, hidden, N: int, h_state_ptrs, conv_state_ptrs):
-        """N sequences x 1 token on this rank's heads (kda_block_decode); FP32 [N, hidden] summed."""
+        """N sequences x 1 token on this rank's heads (kda_block_decode); [N, hidden] summed."""
         kda.kda_block_decode(self.st, hidden, N, h_state_ptrs, conv_state_ptrs, self.ws)
         return self._reduce(N)
 

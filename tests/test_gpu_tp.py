@@ -1,8 +1,9 @@
 """Tensor-parallel head sharding on the GPU kernels: the two halves of the heads run one after
-the other on one device (no inter-rank waiting; the sum of their FP32 partials stands in for
-the all-reduce, which test_tp_gloo.py checks across processes). Each shard's recurrent state
-is bit-identical to the unsharded block's state for those heads; the summed output matches
-the unsharded block and the oracle."""
+the other on one device (no inter-rank waiting; the sum of their partials stands in for the
+all-reduce, which test_tp_gloo.py checks across processes). Each shard's recurrent state is
+bit-identical to the unsharded block's state for those heads; the summed output matches the
+unsharded block and the oracle, with the partials in FP32 and in BF16 (the default: the block
+output is reduced in BF16)."""
 import numpy as np
 import pytest
 import torch
@@ -31,8 +32,10 @@ def _to_device(W):
                                      if isinstance(getattr(W, f.name), torch.Tensor)})
 
 
-@pytest.mark.parametrize("hidden,H,D,rank,T,world", [(256, 4, 64, 64, 130, 2), (4096, 32, 128, 128, 256, 2)])
-def test_tp_prefill_shards_sum_to_unsharded_block(hidden, H, D, rank, T, world):
+@pytest.mark.parametrize("hidden,H,D,rank,T,world,rd", [(256, 4, 64, 64, 130, 2, "fp32"),
+                                                        (4096, 32, 128, 128, 256, 2, "fp32"),
+                                                        (4096, 32, 128, 128, 256, 2, "bf16")])
+def test_tp_prefill_shards_sum_to_unsharded_block(hidden, H, D, rank, T, world, rd):
     Wt = block_weights(hidden, H, D, rank, seed=21, std=0.05 if hidden < 4096 else 0.02)
     h = block_hidden(T, hidden, seed=21).cuda()
     # unsharded block
@@ -49,10 +52,10 @@ def test_tp_prefill_shards_sum_to_unsharded_block(hidden, H, D, rank, T, world):
     total = torch.zeros((T, hidden), device="cuda")
     for r in range(world):
         sh = shard_block_weights(Wd, r, world)
-        blk = TPBlock(sh, max_tokens=T)
+        blk = TPBlock(sh, max_tokens=T, reduce_dtype=rd)
         hs_r = torch.zeros((sh.H, D, D), device="cuda")
         cs_r = torch.zeros((3 * sh.H * D, 3), dtype=torch.bfloat16, device="cuda")
-        total += blk.prefill(h, T, hs_r, cs_r)
+        total += blk.prefill(h, T, hs_r, cs_r).float()
         torch.cuda.synchronize()
         h0 = r * sh.H
         assert torch.equal(hs_r, hs[h0:h0 + sh.H]), r
@@ -85,7 +88,7 @@ def test_tp_decode_shards_sum_to_unsharded_block():
     for r in range(world):
         sh = shard_block_weights(Wd, r, world)
         h0, c0, c1 = r * sh.H, r * sh.H * D, (r + 1) * sh.H * D
-        blk = TPBlock(sh, max_tokens=8)
+        blk = TPBlock(sh, max_tokens=8, reduce_dtype="fp32")
         hs_r = [hs0[n, h0:h0 + sh.H].cuda().contiguous() for n in range(N)]
         cs_r = [torch.cat([cs0[n, c0:c1], cs0[n, qkv + c0:qkv + c1], cs0[n, 2 * qkv + c0:2 * qkv + c1]]).cuda()
                 for n in range(N)]

@@ -1,7 +1,8 @@
 """Tensor-parallel head sharding (Glm5NextLayer `mixer_all_reduce`) on CPU ranks: two gloo
 processes each run the oracle block on their half of the heads (kda_gated_delta_gate_b200.tp
 shards the weights), multiply by their o_proj slice, and all-reduce the partial outputs; the
-sum equals the unsharded block's output. This covers the sharding and the collective on the
+FP64 sum equals the unsharded block's output, and the BF16 reduction (the default of TPBlock)
+stays within its rounding bound of it. This covers the sharding and the collective on the
 host (world sizes 2 and 4); the GPU kernels on the shards are tested in test_gpu_tp.py."""
 import os
 import socket
@@ -48,6 +49,20 @@ def _rank_main(rank: int, world: int, port: int, out_dir: str):
             got = oracle.bf16_round(part.numpy())
             assert np.all(np.abs(got - full["final_out"]) <= 2.0 ** -8 * np.abs(full["final_out"]) + 1e-30)
             np.testing.assert_allclose(torch.cat(states).numpy(), full["h_state"], rtol=1e-12, atol=1e-14)
+        # the default reduction of the block output in BF16: each rank's partial rounded to BF16,
+        # summed by the collective in BF16; within a few BF16 steps of the unsharded output
+        p64 = torch.from_numpy(oracle.linear(mine["o_norm_out"], sh.o_proj))
+        part16 = p64.to(torch.bfloat16)
+        mag = p64.abs()  # sum over ranks of |partial|: each BF16 rounding is relative to its operands
+        dist.all_reduce(part16, op=dist.ReduceOp.SUM)
+        dist.all_reduce(mag, op=dist.ReduceOp.SUM)
+        if rank == 0:
+            full = oracle.block_prefill(W, h, hs_full, cs_full)
+            ref = oracle.linear(full["o_norm_out"], W.o_proj)
+            got16 = part16.double().numpy()
+            # one rounding of each partial and one per addition, each at most half a BF16 step
+            bound = world * 2.0 ** -8 * (mag.numpy() + np.abs(ref)) + 1e-30
+            assert np.all(np.abs(got16 - ref) <= bound)
             open(os.path.join(out_dir, "ok"), "w").write("ok")
     finally:
         dist.destroy_process_group()
