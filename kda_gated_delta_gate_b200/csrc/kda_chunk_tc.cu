@@ -1146,14 +1146,16 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
 //   MMA group 2   D3 = (K o e^{Gamma_C - Gamma})^T . U        (M = D, N = DVS, K = 64)
 //   MMA group 3   D1 += [0; M] . U                            (so D1[64:128] = (Q o A) S0 + M U)
 //   epilogue 2    S = A_C o S0 + D3 (FP32 master copy in registers) into the S operand
-// Groups 1 and 2 and the two epilogues are the critical path. Warp kEpiWarps (the control warp)
-// issues every copy and every MMA, so that the epilogue warps never stall behind the tensor
-// pipe's back-pressure on MMA issue. Group 3 of chunk c is issued right after group 1 of chunk
-// c + 1 (with two U operands in shared memory), so it runs while epilogue 1 of c + 1 does instead
-// of delaying that group 1; the output rows O = scale D1[64:128] of chunk c are read while group
-// 2 of chunk c + 1 runs. Epilogue and control warps hand over through mbarriers.
+// Groups 1 and 2 and the two epilogues are the critical path. Two control threads issue every
+// copy and every MMA, so that the epilogue warps never wait behind MMA issue: the chain thread
+// (warp kEpiWarps) issues groups 1 and 2 and the copies of their operands; with two U operands in
+// shared memory the output thread (warp kEpiWarps + 1) issues group 3 of a chunk once its group 2
+// has completed (it then runs while epilogue 2 does) and copies the next M; with one U operand the
+// chain thread issues group 3 right after group 2. The output rows O = scale D1[64:128] of chunk c
+// are read while group 2 of chunk c + 1 runs. Every chunk's operand pack two chunks ahead is
+// prefetched into L2. Epilogue and control warps hand over through mbarriers.
 constexpr int kEpiWarps = 8;
-constexpr int kStateThreads = 32 * (kEpiWarps + 1);
+constexpr int kStateThreads = 32 * (kEpiWarps + 2);  // + the two control warps
 
 template <int D, int DVS>
 __global__ void __launch_bounds__(kStateThreads, 1)
@@ -1169,9 +1171,9 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = sm + S::OFF_A1, *sA2 = sm + S::OFF_A2, *sA3 = sm + S::OFF_A3, *sB1 = sm + S::OFF_B1,
             *sB2 = sm + S::OFF_B2;
-    // barriers: copies 0 A1, 1 M, 2 A3; MMA groups 4 (D1), 5 (D3), 6 (D1 += [0; M] U); 7 the final
-    // drain after a timeout; 8 "U is in B2" and 9 "S is in B1, D3 read" (one arrival per epilogue
-    // warp, after the warp's own writes and TMEM reads)
+    // barriers: copies 0 A1, 1 M, 2 A3; MMA groups 4 (D1), 5 (D3), 6 (D1 += [0; M] U); 7 and 10 the
+    // final drains after a timeout (chain and output threads); 8 "U is in B2" and 9 "S is in B1, D3
+    // read" (one arrival per epilogue warp, after the warp's own writes and TMEM reads)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::OFF_MISC);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::OFF_MISC + 128);
     int *fail = reinterpret_cast<int *>(sm + S::OFF_MISC + 136);  // a role gave up waiting
@@ -1193,7 +1195,8 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     if (nb == 0) return;  // an empty stream keeps its state
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
     const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
-    const bool ctl = warp == kEpiWarps && lane == 0;  // the control thread
+    const bool ctl = warp == kEpiWarps && lane == 0;      // the chain thread
+    const bool ctl2 = warp == kEpiWarps + 1 && lane == 0;  // the output thread
 
     auto copy_m = [&](const uint8_t *pk) {  // M's hi and lo halves into rows 64..127 of A2
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bars[1])),
@@ -1206,6 +1209,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_init(&bars[8], kEpiWarps);  // one arrival per epilogue warp
         mbar_init(&bars[9], kEpiWarps);
+        mbar_init(&bars[10], 1);
         *fail = 0;
         fence_mbar_init();
         bulk_copy(sA1, packs + PK::OFF_A1, PK::A1, &bars[0]);
@@ -1256,41 +1260,46 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     tc_fence_after();
     bool ok = true;
 
-    if (warp == kEpiWarps) {
-        // ================================================= control warp (lane 0 works)
+    if (warp >= kEpiWarps) {
+        // ================================================= control warps (lane 0 of each works)
+        // K-step-0 descriptors of every operand (the buffers never move)
+        const uint64_t dA2h = kmaj_desc(smem_u32(sA2), 128, 0, 0), dA2l = kmaj_desc(smem_u32(sA2) + kTileBytes, 128, 0, 0);
+        const uint64_t dB2h = mnmaj_desc(smem_u32(sB2), C, 0, 0), dB2l = mnmaj_desc(smem_u32(sB2) + S::B2 / 2, C, 0, 0);
+        constexpr uint64_t kB2Buf = static_cast<uint64_t>(S::B2 >> 4);  // one U buffer, in descriptor units
+        // the output group (D1 += [0; M] U) of chunk c: U from B2 buffer c % NU, M from A2
+        auto issue_out_group = [&](int c) {
+            constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
+            const uint64_t ub = (c % S::NU) * kB2Buf;
+            const uint32_t tD1c = tmem + (c & 1) * DVS;
+#pragma unroll
+            for (int ks = 0; ks < C / 16; ++ks) {
+                const uint64_t bh = dB2h + ub + mnmaj_step(ks), bl = dB2l + ub + mnmaj_step(ks);
+                const uint64_t mh = dA2h + kmaj_step(128, ks), ml = dA2l + kmaj_step(128, ks);
+                mma_bf16(tD1c, mh, bh, idm, 1);
+                mma_bf16(tD1c, mh, bl, idm, 1);
+                mma_bf16(tD1c, ml, bh, idm, 1);
+            }
+            mma_commit(&bars[6]);
+        };
+        // copy barriers this thread issues on: copies issued and phases waited for (so that a
+        // timed-out thread can drain what is still in flight)
+        uint32_t issued[3] = {1, 1, 1}, waited[3] = {0, 0, 0};
+        auto wait_copy = [&](int k) {
+            const bool r = mbar_wait(&bars[k], waited[k] & 1, kWaitCycles);
+            if (r) ++waited[k];
+            return r;
+        };
+        auto give_up = [&]() {
+            ok = false;
+            atomicExch(fail, 1);
+        };
         if (ctl) {
-            uint32_t issued[3] = {1, 1, 1}, waited[3] = {0, 0, 0};
-            auto wait_copy = [&](int k) {
-                const bool r = mbar_wait(&bars[k], waited[k] & 1, kWaitCycles);
-                if (r) ++waited[k];
-                return r;
-            };
-            auto give_up = [&]() {
-                ok = false;
-                atomicExch(fail, 1);
-            };
-            // K-step-0 descriptors of every operand (the buffers never move)
             const uint64_t dA1h = kmaj_desc(smem_u32(sA1), 128, 0, 0), dA1l = kmaj_desc(smem_u32(sA1) + PK::A1 / 2, 128, 0, 0);
             const uint64_t dB1h = mnmaj_desc(smem_u32(sB1), D, 0, 0), dB1l = mnmaj_desc(smem_u32(sB1) + S::B1 / 2, D, 0, 0);
             const uint64_t dA3h = mnmaj_desc(smem_u32(sA3), C, 0, 0), dA3l = mnmaj_desc(smem_u32(sA3) + PK::A3 / 2, C, 0, 0);
-            const uint64_t dA2h = kmaj_desc(smem_u32(sA2), 128, 0, 0), dA2l = kmaj_desc(smem_u32(sA2) + kTileBytes, 128, 0, 0);
-            const uint64_t dB2h = mnmaj_desc(smem_u32(sB2), C, 0, 0), dB2l = mnmaj_desc(smem_u32(sB2) + S::B2 / 2, C, 0, 0);
-            constexpr uint64_t kB2Buf = static_cast<uint64_t>(S::B2 >> 4);  // one U buffer, in descriptor units
-            // the output group (D1 += [0; M] U) of chunk c: U from B2 buffer c % NU, M from A2
-            auto issue_out_group = [&](int c) {
-                constexpr uint32_t idm = idesc_bf16(128, DVS, false, true);
-                const uint64_t ub = (c % S::NU) * kB2Buf;
-                const uint32_t tD1c = tmem + (c & 1) * DVS;
-#pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks) {
-                    const uint64_t bh = dB2h + ub + mnmaj_step(ks), bl = dB2l + ub + mnmaj_step(ks);
-                    const uint64_t mh = dA2h + kmaj_step(128, ks), ml = dA2l + kmaj_step(128, ks);
-                    mma_bf16(tD1c, mh, bh, idm, 1);
-                    mma_bf16(tD1c, mh, bl, idm, 1);
-                    mma_bf16(tD1c, ml, bh, idm, 1);
-                }
-                mma_commit(&bars[6]);
-            };
+            if (S::NU == 2) issued[1] = 0;  // the output thread owns the M copies
+            if (nb > 1) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(packs + PK::bytes),
+                                     "r"(static_cast<uint32_t>(PK::bytes)) : "memory");
 #pragma unroll 1
             for (int ch = 0; ch < nb && ok; ++ch) {
                 const uint32_t par = ch & 1;
@@ -1314,10 +1323,9 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                     }
                     mma_commit(&bars[4]);
                 }
-                if (S::NU == 2 && ch > 0) {  // the previous chunk's output group, behind this D1
-                    if (!wait_copy(1)) { give_up(); break; }
-                    issue_out_group(ch - 1);
-                }
+                if (ch + 2 < nb)  // the pack two chunks ahead into L2
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(cur + 2 * PK::bytes),
+                                 "r"(static_cast<uint32_t>(PK::bytes)) : "memory");
                 if (S::NU == 1 && ch > 0) {  // the previous output group has read M: this chunk's M
                     if (!mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
                     copy_m(cur);
@@ -1345,12 +1353,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                     }
                     mma_commit(&bars[5]);
                 }
-                if (S::NU == 2 && ch > 0) {  // the previous output group has read M (it ran ahead of group 2)
-                    if (!mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
-                    copy_m(cur);
-                    ++issued[1];
-                }
-                if (S::NU == 1 || !more) {  // one U buffer (or the last chunk): the output group now
+                if (S::NU == 1) {  // one U buffer: the output group now, behind group 2
                     if (!wait_copy(1)) { give_up(); break; }
                     issue_out_group(ch);
                 }
@@ -1368,13 +1371,33 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                     while (waited[k] < issued[k] && wait_copy(k)) {
                     }
             }
+        } else if (ctl2 && S::NU == 2) {
+            issued[0] = issued[2] = 0;  // the chain thread owns the A1 and A3 copies
+#pragma unroll 1
+            for (int ch = 0; ch < nb && ok; ++ch) {
+                // group 2 of this chunk has completed: its output group runs while epilogue 2 does
+                if (!mbar_wait(&bars[5], ch & 1, kWaitCycles)) { give_up(); break; }
+                if (!wait_copy(1)) { give_up(); break; }
+                tc_fence_after();
+                issue_out_group(ch);
+                if (ch + 1 < nb) {  // the output group has read M: the next chunk's M may come in
+                    if (!mbar_wait(&bars[6], ch & 1, kWaitCycles)) { give_up(); break; }
+                    copy_m(packs + static_cast<size_t>(ch + 1) * PK::bytes);
+                    ++issued[1];
+                }
+            }
+            if (!ok) {
+                mma_commit(&bars[10]);
+                mbar_wait(&bars[10], 0, kWaitCycles);
+                while (waited[1] < issued[1] && wait_copy(1)) {
+                }
+            }
         }
     } else {
         // ================================================= epilogue warps
         // O = scale D1[64:128] of chunk c (quads 2 and 3: TMEM lanes 64..127 = the chunk's tokens),
         // once group 3 of chunk c has completed
-        auto out_epilogue = [&](int c) {
-            ok = ok && mbar_wait(&bars[6], c & 1, kWaitCycles);
+        auto out_epilogue = [&](int c) {  // the caller has waited for the output group of chunk c
             tc_fence_after();
             const int i = erow - 64;
             int nn;
@@ -1450,6 +1473,9 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                     st_pair(sB2 + (ch % S::NU) * S::B2, S::B2 / 2, mnmaj_off(ccol + j, erow, C), x);
                 }
             }
+            // the previous chunk's output group has completed (waited for before this warp's arrival:
+            // the next output group cannot complete before that arrival, so the phase is unambiguous)
+            if (ch > 0 && quad >= 2) ok = ok && mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles);
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -1480,6 +1506,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 break;
             }
         }
+        if (quad >= 2) ok = ok && mbar_wait(&bars[6], (nb - 1) & 1, kWaitCycles);
         if (ok && quad >= 2) out_epilogue(nb - 1);
     }
     ok = __syncthreads_and(ok && *reinterpret_cast<volatile int *>(fail) == 0) != 0;
