@@ -126,6 +126,7 @@ struct GemvSeg {
     const uint16_t *W;
     void *y;
     int N, ldw, ldy, out_f32;
+    const uint16_t *x;  // this segment's input rows (same row stride), or null: the call's x
 };
 struct GemvSegs {
     GemvSeg s[3];

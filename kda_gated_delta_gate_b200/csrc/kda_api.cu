@@ -28,19 +28,29 @@ void *current_context() {
 }
 
 int *device_status_ptr() {
-    // per device: the context the address was looked up in, and the address
+    // per device: the context the address was looked up in, and the address (a per-thread copy
+    // answers the common case without the lock)
     static std::mutex lock;
     static void *ctx_of[64] = {};
     static int *addr_of[64] = {};
+    thread_local void *tl_ctx[64] = {};
+    thread_local int *tl_addr[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     void *ctx = current_context();  // null before the runtime has made one current
+    if (ctx && tl_addr[dev] && ctx == tl_ctx[dev]) return tl_addr[dev];
     std::lock_guard<std::mutex> g(lock);
-    if (addr_of[dev] && ctx && ctx == ctx_of[dev]) return addr_of[dev];
+    if (addr_of[dev] && ctx && ctx == ctx_of[dev]) {
+        tl_ctx[dev] = ctx;
+        tl_addr[dev] = addr_of[dev];
+        return addr_of[dev];
+    }
     void *addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess || !addr) return nullptr;
     ctx_of[dev] = current_context();  // the lookup made the device's context current
     addr_of[dev] = static_cast<int *>(addr);
+    tl_ctx[dev] = ctx_of[dev];
+    tl_addr[dev] = addr_of[dev];
     return addr_of[dev];
 }
 

@@ -75,8 +75,13 @@ int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M,
         b.count = 3;
         b.total = 2 * R + H;
         KDA_TRY(gemv_segs(hidden, Hd, b, M, Hd, s));
-        KDA_TRY(gemv_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, M, qkv, R, 0, s));
-        return gemv_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, M, qkv, R, 0, s);
+        // f_b and g_b read different rows (f_a_out, g_a_out) with one width: one launch
+        GemvSegs c{};
+        c.s[0] = GemvSeg{w->f_b, bf(KDA_BUF_G_RAW), qkv, R, qkv, 0, bf(KDA_BUF_F_A_OUT)};
+        c.s[1] = GemvSeg{w->g_b, bf(KDA_BUF_OUT_GATE), qkv, R, qkv, 0, bf(KDA_BUF_G_A_OUT)};
+        c.count = 2;
+        c.total = 2 * qkv;
+        return gemv_segs(bf(KDA_BUF_F_A_OUT), R, c, M, R, s);
     }
     KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, M, qkv, Hd, 0, s));
     KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, M, qkv, Hd, 0, s));

@@ -248,20 +248,28 @@ int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout
 // butterfly: every output's arithmetic depends on K and its own row only, never on M, so a
 // row's result is the same bits in a call of one row and in a call of many (the identity the
 // K-token verify needs). x rows are staged in shared memory; W streams with 16-byte loads.
+// Segments may bring their own input rows (two products of one step that read different rows
+// share a launch); their rows are staged side by side.
 constexpr int kGemvRows = 8, kGemvWarps = 8, kGemvMaxK = 8192;
 
 namespace {
 template <int MB>
 __global__ void __launch_bounds__(32 * kGemvWarps)
 gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M, int K) {
-    constexpr int U = 8;  // weight loads in flight per lane (U x 16 bytes)
-    extern __shared__ __align__(16) uint16_t sx[];  // [mb][K]: this group's rows only
+    // weight loads in flight per lane (U x 16 bytes): a whole 4096-wide row for one-row calls
+    constexpr int U = MB == 1 ? 16 : 8;
+    extern __shared__ __align__(16) uint16_t sx[];  // [set][mb][K]: this group's rows of each input
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int m0 = blockIdx.y * MB;
     const int mb = min(MB, M - m0);
-    for (int e = tid; e < mb * (K / 8); e += 32 * kGemvWarps) {
-        const int r = e / (K / 8), c = 8 * (e % (K / 8));
-        *reinterpret_cast<uint4 *>(sx + r * K + c) = *reinterpret_cast<const uint4 *>(x + static_cast<size_t>(m0 + r) * ldx + c);
+    const int nx = segs.s[0].x ? segs.count : 1;  // input sets: one per segment, or the call's x
+    for (int q = 0; q < nx; ++q) {
+        const uint16_t *xs = segs.s[0].x ? segs.s[q].x : x;
+        for (int e = tid; e < mb * (K / 8); e += 32 * kGemvWarps) {
+            const int r = e / (K / 8), c = 8 * (e % (K / 8));
+            *reinterpret_cast<uint4 *>(sx + (q * mb + r) * K + c) =
+                *reinterpret_cast<const uint4 *>(xs + static_cast<size_t>(m0 + r) * ldx + c);
+        }
     }
     __syncthreads();
     for (int col = blockIdx.x * kGemvWarps + warp; col < segs.total; col += gridDim.x * kGemvWarps) {
@@ -269,6 +277,7 @@ gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M,
         while (si + 1 < segs.count && n >= segs.s[si].N) { n -= segs.s[si].N; ++si; }
         const GemvSeg &sg = segs.s[si];
         const uint16_t *wr = sg.W + static_cast<size_t>(n) * sg.ldw;
+        const uint16_t *sxs = sx + (nx > 1 ? si * mb * K : 0);  // this segment's input rows
         float acc[MB];
 #pragma unroll
         for (int r = 0; r < MB; ++r) acc[r] = 0.f;
@@ -292,7 +301,7 @@ gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M,
 #pragma unroll
                 for (int r = 0; r < MB; ++r) {
                     if (r < mb) {
-                        const uint4 xv = *reinterpret_cast<const uint4 *>(sx + r * K + k);
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(sxs + r * K + k);
                         acc[r] = __fmaf_rn(__uint_as_float(xv.x << 16), w8[0], acc[r]);
                         acc[r] = __fmaf_rn(__uint_as_float(xv.x & 0xFFFF0000u), w8[1], acc[r]);
                         acc[r] = __fmaf_rn(__uint_as_float(xv.y << 16), w8[2], acc[r]);
@@ -323,10 +332,23 @@ gemv_kernel(const uint16_t *__restrict__ x, int ldx, const GemvSegs segs, int M,
         }
     }
 }
+
 }  // namespace
 
 int gemv_segs(const uint16_t *x, int ldx, const GemvSegs &segs, int M, int K, cudaStream_t s) {
-    const int bytes = std::min(M, kGemvRows) * K * 2;  // the rows of one group
+    const int nx = segs.s[0].x ? segs.count : 1;
+    const int bytes = nx * std::min(M, kGemvRows) * K * 2;  // the rows of one group, per input
+    if (bytes > (M == 1 ? 1 : kGemvRows) * kGemvMaxK * 2) {  // the inputs do not fit side by side: one launch each
+        for (int i = 0; i < segs.count; ++i) {
+            GemvSegs one{};
+            one.s[0] = segs.s[i];
+            one.s[0].x = nullptr;
+            one.count = 1;
+            one.total = segs.s[i].N;
+            KDA_TRY(gemv_segs(segs.s[0].x ? segs.s[i].x : x, ldx, one, M, K, s));
+        }
+        return KDA_OK;
+    }
     static std::atomic<unsigned long long> attr_done{0}, attr1_done{0};  // opted in once, at the largest K
     const int col_blocks = (segs.total + kGemvWarps - 1) / kGemvWarps;
     const int grid_x = std::min(col_blocks, 4 * sm_count());
