@@ -142,7 +142,10 @@ KDA_API size_t kda_chunk_prefill_scratch_bytes(int B, int T, const kda_dims *dim
  *                  chunk slots per sequence)
  *   h_state        DEVICE array of B state pointers, read and overwritten (an empty sequence
  *                  keeps its state)
- *   scratch        at least kda_chunk_prefill_varlen_scratch_bytes(B, max_num_chunks, dims)
+ *   scratch        at least kda_chunk_prefill_varlen_scratch_bytes(B, max_num_chunks, dims), or
+ *                  kda_chunk_prefill_packed_scratch_bytes(m, t, dims) for any m >= B, t >= total_tokens
+ *                  (the call takes the smaller of the two chunk-slot layouts; KDA_ERR_CAPACITY if the
+ *                  scratch holds neither)
  * A sequence whose bounds do not fit (negative, decreasing, past total_tokens, or longer than
  * max_num_chunks * 64) is skipped, its state untouched, and KDA_ERR_INVALID_ARG is latched in
  * kda_device_status. Each sequence's result equals kda_chunk_prefill on that sequence alone. */
@@ -151,8 +154,15 @@ KDA_API int kda_chunk_prefill_varlen(const float *q, const float *k, const float
                                      int total_tokens, float *const *h_state, float *core, void *scratch,
                                      size_t scratch_bytes, const kda_dims *dims, void *stream);
 
-/* Scratch bytes kda_chunk_prefill_varlen needs (0 if B or max_num_chunks is 0). */
+/* Scratch bytes kda_chunk_prefill_varlen needs (0 if B or max_num_chunks is 0): one operand
+ * pack per (sequence, head, chunk slot). */
 KDA_API size_t kda_chunk_prefill_varlen_scratch_bytes(int B, int max_num_chunks, const kda_dims *dims);
+
+/* Scratch bytes enough for every kda_chunk_prefill_varlen call of at most max_seqs sequences and
+ * max_total_tokens rows, whatever the mix of lengths (0 if either is 0): the compact layout, in
+ * which sequence b's chunks take consecutive pack slots from floor(cu_seqlens[b] / 64) + b, so
+ * a head needs ceil(max_total_tokens / 64) + max_seqs - 1 slots. */
+KDA_API size_t kda_chunk_prefill_packed_scratch_bytes(int max_seqs, int max_total_tokens, const kda_dims *dims);
 
 /* kda_chunk_verify — batched verify under the WY tables (Glm5NextLayer speculative verify):
  * the draft rows of B sequences, packed as for kda_chunk_prefill_varlen, each sequence at most
@@ -334,7 +344,9 @@ KDA_API int kda_decode_fused(const kda_bf16 *x, kda_bf16 *const *conv_state, con
  *   h_snap     HOST array of n_snap device pointers to [H, D, D] F32, or NULL if n_snap = 0
  *   conv_snap  HOST array of n_snap device pointers to [3*H*D, 3] BF16, or NULL
  * snapshot t receives the (recurrent, conv) state AFTER row t, t = 0..K-2.
- * 1 <= K <= 32 (KDA_ERR_UNSUPPORTED beyond).
+ * K >= 1. One launch carries at most 32 rows; a longer call runs as launches of up to 32 rows,
+ * each continuing from the state the previous one left in place (the FP32 state and the BF16
+ * conv inputs round-trip exactly, so the result is still bit-identical to K serial decodes).
  */
 KDA_API int kda_decode_k(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w,
                  const kda_bf16 *g_raw, const float *dt_bias, const float *a_log,
@@ -342,6 +354,31 @@ KDA_API int kda_decode_k(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16
                  const kda_bf16 *o_norm_w, kda_bf16 *o_norm_out, kda_bf16 *conv_out, float *core,
                  int K, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
                  const kda_dims *dims, void *stream);
+
+/* kda_front_conv_silu_l2_varlen — the front end of kda_front_conv_silu_l2 (the same per-row
+ * arithmetic) over B sequences packed back to back (Glm5NextLayer varlen prefill): row t of
+ * sequence b (rows [cu_seqlens[b], cu_seqlens[b+1])) takes its conv window from that sequence
+ * only, reaching into sequence b's carried conv state before its first row.
+ *   x           [total_tokens, 3*H*D] BF16 (qkv_proj rows);  conv_out likewise (output)
+ *   conv_state  DEVICE array of B device pointers to [3*H*D, 3] BF16 conv states (16-byte aligned;
+ *               a misaligned one latches KDA_ERR_MISALIGNED and its rows are skipped)
+ *   cu_seqlens  DEVICE int32 [B + 1] as kda_chunk_prefill_varlen
+ *   advance_state  0: the conv states are only read (a verify); else each is then replaced by
+ *               the last three inputs of (state || its rows), as kda_front_conv_silu_l2 does
+ * No FP32 widening (the packed block core reads conv_out). Bad cu_seqlens bounds latch
+ * KDA_ERR_INVALID_ARG; the rows of the tile that met them are skipped. */
+KDA_API int kda_front_conv_silu_l2_varlen(const kda_bf16 *x, kda_bf16 *const *conv_state, const kda_bf16 *conv_w,
+                                          kda_bf16 *conv_out, const int *cu_seqlens, int B, int total_tokens,
+                                          int advance_state, const kda_dims *dims, void *stream);
+
+/* kda_conv_state_fold — the conv half of accepted-row folding (Glm5NextLayer `gdn_fold_accepted`):
+ * sequence b's conv state becomes the last three inputs of (state || its first accepted[b] rows
+ * of x), x the qkv_proj rows the verify's front end read; accepted = NULL takes every row.
+ * accepted DEVICE int32 [B], 0 <= accepted[b] <= the sequence's rows (else KDA_ERR_INVALID_ARG is
+ * latched and that state left); 0 leaves the state. Other arguments as
+ * kda_front_conv_silu_l2_varlen. */
+KDA_API int kda_conv_state_fold(const kda_bf16 *x, kda_bf16 *const *conv_state, const int *cu_seqlens,
+                                const int *accepted, int B, int total_tokens, const kda_dims *dims, void *stream);
 
 /* ---------------------------------------------------------------------------------
  * kda_front_conv_silu_l2 — prefill front end for one sequence of T tokens
@@ -436,11 +473,19 @@ enum {
 
 typedef struct kda_workspace kda_workspace;
 
-/* Allocate the workspace for up to max_tokens tokens (the only allocating call). */
+/* Allocate the workspace for up to max_tokens tokens (the only allocating call); single-sequence
+ * calls and packed calls of one sequence. */
 KDA_API int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_tokens,
                                  kda_workspace **out);
+/* The same for packed calls (kda_block_prefill_varlen / _batched, kda_block_verify) of up to
+ * max_seqs sequences and max_tokens rows in all: the chunked-prefill scratch is sized by
+ * kda_chunk_prefill_packed_scratch_bytes(max_seqs, max_tokens), which fits any mix of lengths.
+ * max_seqs = 1 is kda_workspace_create. */
+KDA_API int kda_workspace_create_batched(const kda_dims *dims, int hidden, int rank, size_t max_tokens,
+                                         int max_seqs, kda_workspace **out);
 KDA_API int kda_workspace_destroy(kda_workspace *ws);
 KDA_API size_t kda_workspace_max_tokens(const kda_workspace *ws);
+KDA_API int kda_workspace_max_seqs(const kda_workspace *ws);
 /* Device pointer and size of one stage buffer (the buffers are public so each stage can be
  * compared on its own, as the workspace page intends). */
 KDA_API int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr, size_t *bytes);
@@ -453,6 +498,30 @@ KDA_API int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr,
  * KDA_ERR_CAPACITY if T > max_tokens. Allocates nothing. */
 KDA_API int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T, float *h_state,
                               kda_bf16 *conv_state, float pad_fill, kda_workspace *ws, void *stream);
+
+/* kda_block_prefill_varlen — B sequences packed back to back through one block call
+ * (Glm5NextLayer `prefill_gdn_full_batched` in its varlen form): the projections, beta, o_norm
+ * and o_proj run once over all total_tokens rows; the conv (kda_front_conv_silu_l2_varlen) and
+ * the chunked core (the fused-input mode of kda_chunk_prefill_varlen) keep the sequences apart.
+ *   hidden      [total_tokens, hidden] BF16 (device), sequence b = rows [cu_seqlens[b], cu_seqlens[b+1])
+ *   cu_seqlens  DEVICE int32 [B + 1];  max_num_chunks >= ceil(len_b / 64) for every sequence
+ *   h_state     DEVICE array of B pointers to [H, D, D] F32 states, carried and updated in place
+ *   conv_state  DEVICE array of B pointers to [3*H*D, 3] BF16 conv states, likewise
+ * Each sequence's rows and states equal kda_block_prefill on that sequence alone, up to the
+ * projection GEMM (the same kernel on more rows). An empty sequence keeps its states.
+ * Results in the workspace rows 0..total_tokens-1 (KDA_BUF_FINAL_OUT and the stage buffers).
+ * KDA_ERR_CAPACITY if total_tokens > max_tokens or B > max_seqs. Allocates nothing. */
+KDA_API int kda_block_prefill_varlen(const kda_block_weights *w, const kda_bf16 *hidden, const int *cu_seqlens, int B,
+                                     int max_num_chunks, int total_tokens, float *const *h_state,
+                                     kda_bf16 *const *conv_state, kda_workspace *ws, void *stream);
+
+/* kda_block_prefill_batched — B sequences of T rows each (Glm5NextLayer
+ * `prefill_gdn_full_batched`): hidden [B*T, hidden] BF16, sequence b = rows [b T, (b+1) T);
+ * the call writes the cu_seqlens into the workspace and runs kda_block_prefill_varlen.
+ * KDA_ERR_CAPACITY if B*T > max_tokens or B > max_seqs. */
+KDA_API int kda_block_prefill_batched(const kda_block_weights *w, const kda_bf16 *hidden, int B, int T,
+                                      float *const *h_state, kda_bf16 *const *conv_state, kda_workspace *ws,
+                                      void *stream);
 
 /* kda_block_decode — N independent sequences, one token each, through the whole block
  * (Glm5NextKdaLayer `decode`): the projections of the N hidden rows (each weight read once for
@@ -473,10 +542,42 @@ KDA_API int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden,
  * projection of a row computes the same bits whatever the number of rows in the call).
  *   hidden [K, hidden] BF16; h_state [H, D, D] F32 and conv_state [3*H*D, 3] BF16 (single
  *   device pointers, updated in place); h_snap, conv_snap, n_snap as kda_decode_k.
- * 1 <= K <= 32 (KDA_ERR_UNSUPPORTED beyond), K <= max_tokens (else KDA_ERR_CAPACITY). */
+ * 1 <= K <= max_tokens (else KDA_ERR_CAPACITY). The projections and o_proj run on groups of
+ * at most 32 rows (the matrix-vector kernel, whose per-row bits the identity needs), so a
+ * call past 32 rows reads the weights once per group. */
 KDA_API int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K, float *h_state,
                                kda_bf16 *conv_state, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
                                kda_workspace *ws, void *stream);
+
+/* kda_block_verify — batched speculative verify through the whole block (Glm5NextLayer verify:
+ * N sequences x K draft rows; Glm5NextKdaLayer `decode_k` at layer level): the projections of all
+ * draft rows of all sequences in one pass (each weight read once for all rows), the packed conv
+ * from each sequence's conv state, then the chunked core in verify mode (kda_chunk_verify, fused
+ * input) from each sequence's recurrent state, o_norm and o_proj. NO state changes: the
+ * recurrent and conv states stay as they were, and `tables` (kda_chunk_verify_tables_bytes(B),
+ * 16-byte aligned) receives what kda_block_verify_fold needs.
+ *   hidden      [total_tokens, hidden] BF16, sequence b = rows [cu_seqlens[b], cu_seqlens[b+1]),
+ *               at most 64 rows each (a longer one latches KDA_ERR_INVALID_ARG and is skipped)
+ *   cu_seqlens  DEVICE int32 [B + 1];  h_state, conv_state: DEVICE pointer arrays as
+ *               kda_block_prefill_varlen (read only here)
+ * Each row's output equals what kda_block_prefill_varlen on that sequence's first rows gives
+ * for it (the same core arithmetic), up to the projection kernel: up to 32 rows in all the
+ * matrix-vector kernel, beyond that the GEMM. The workspace keeps the rows' qkv_proj and
+ * conv_out for the fold. KDA_ERR_CAPACITY if total_tokens > max_tokens or B > max_seqs. */
+KDA_API int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const int *cu_seqlens, int B,
+                             int total_tokens, float *const *h_state, kda_bf16 *const *conv_state, float *tables,
+                             size_t tables_bytes, kda_workspace *ws, void *stream);
+
+/* kda_block_verify_fold — accepted-row folding after kda_block_verify (Glm5NextLayer
+ * `gdn_fold_accepted`): sequence b's recurrent state becomes its state after its first
+ * accepted[b] verified rows (kda_chunk_verify_fold's formula on the verify's tables and the BF16
+ * k rows its core read) and its conv state the last three inputs of (state || those rows'
+ * qkv_proj). accepted DEVICE int32 [B], 0 <= accepted[b] <= its rows; 0 leaves both states.
+ * Run on the same workspace, cu_seqlens, tables and states right after kda_block_verify, before
+ * any other call on that workspace. */
+KDA_API int kda_block_verify_fold(const int *cu_seqlens, const int *accepted, int B, int total_tokens,
+                                  const float *tables, float *const *h_state, kda_bf16 *const *conv_state,
+                                  kda_workspace *ws, void *stream);
 
 /* kda_block_decode_graph — kda_block_decode recorded once into a CUDA graph and instantiated,
  * for a serving loop that decodes the same N sequences from the same buffers every step: each

@@ -92,6 +92,15 @@ _SIGS = {
     "kda_block_decode_graph": ([_VP, _VP, _I, _VP, _VP, _VP, ctypes.POINTER(_VP)], _I),
     "kda_graph_launch": ([_VP, _VP], _I),
     "kda_graph_destroy": ([_VP], _I),
+    "kda_chunk_prefill_packed_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
+    "kda_front_conv_silu_l2_varlen": ([_VP] * 5 + [_I, _I, _I, _DIMS, _VP], _I),
+    "kda_conv_state_fold": ([_VP] * 4 + [_I, _I, _DIMS, _VP], _I),
+    "kda_workspace_create_batched": ([_DIMS, _I, _I, ctypes.c_size_t, _I, ctypes.POINTER(_VP)], _I),
+    "kda_workspace_max_seqs": ([_VP], _I),
+    "kda_block_prefill_varlen": ([_VP, _VP, _VP, _I, _I, _I, _VP, _VP, _VP, _VP], _I),
+    "kda_block_prefill_batched": ([_VP, _VP, _I, _I, _VP, _VP, _VP, _VP], _I),
+    "kda_block_verify": ([_VP, _VP, _VP, _I, _I, _VP, _VP, _VP, ctypes.c_size_t, _VP, _VP], _I),
+    "kda_block_verify_fold": ([_VP, _VP, _I, _I, _VP, _VP, _VP, _VP, _VP], _I),
 }
 
 
@@ -303,12 +312,15 @@ def block_weights_struct(w) -> KdaBlockWeights:
 
 
 class Workspace:
-    """The block prefill's stage buffers, allocated once for max_tokens (kda_workspace_create)."""
+    """The block's stage buffers, allocated once for max_tokens rows and, for packed calls
+    (kda_block_prefill_varlen / _batched, kda_block_verify), max_seqs sequences
+    (kda_workspace_create_batched; max_seqs = 1 is kda_workspace_create)."""
 
-    def __init__(self, d: KdaDims, hidden: int, rank: int, max_tokens: int):
+    def __init__(self, d: KdaDims, hidden: int, rank: int, max_tokens: int, max_seqs: int = 1):
         self.dims = d
         self._h = ctypes.c_void_p()
-        _call("kda_workspace_create", ctypes.byref(d), hidden, rank, max_tokens, ctypes.byref(self._h))
+        _call("kda_workspace_create_batched", ctypes.byref(d), hidden, rank, max_tokens, max_seqs,
+              ctypes.byref(self._h))
 
     @property
     def handle(self):
@@ -383,6 +395,53 @@ def kda_block_decode_k(weights: KdaBlockWeights, hidden, K: int, h_state, conv_s
     return _call("kda_block_decode_k", ctypes.byref(weights), _p(hidden), K, _p(h_state), _p(conv_state),
                  ctypes.cast(hs, _VP) if hs is not None else None, ctypes.cast(cs, _VP) if cs is not None else None,
                  n, ws.handle, _stream(stream))
+
+
+def kda_block_prefill_varlen(weights: KdaBlockWeights, hidden, cu_seqlens, B: int, max_num_chunks: int,
+                             total_tokens: int, h_state_ptrs, conv_state_ptrs, ws: Workspace, stream=None):
+    """B packed sequences (cu_seqlens: device int32 [B+1]) through the whole block; the states are
+    device pointer arrays (ptr_array), carried and updated. Output in ws buffer "final_out"."""
+    return _call("kda_block_prefill_varlen", ctypes.byref(weights), _p(hidden), _p(cu_seqlens), B, max_num_chunks,
+                 total_tokens, _p(h_state_ptrs), _p(conv_state_ptrs), ws.handle, _stream(stream))
+
+
+def kda_block_prefill_batched(weights: KdaBlockWeights, hidden, B: int, T: int, h_state_ptrs, conv_state_ptrs,
+                              ws: Workspace, stream=None):
+    """B sequences of T rows each (hidden [B*T, hidden]) through the whole block."""
+    return _call("kda_block_prefill_batched", ctypes.byref(weights), _p(hidden), B, T, _p(h_state_ptrs),
+                 _p(conv_state_ptrs), ws.handle, _stream(stream))
+
+
+def kda_block_verify(weights: KdaBlockWeights, hidden, cu_seqlens, B: int, total_tokens: int, h_state_ptrs,
+                     conv_state_ptrs, tables, ws: Workspace, stream=None):
+    """Draft rows of B sequences (at most 64 each) through the whole block; no state changes;
+    tables (kda_chunk_verify_tables_bytes(B) bytes) kept for kda_block_verify_fold."""
+    return _call("kda_block_verify", ctypes.byref(weights), _p(hidden), _p(cu_seqlens), B, total_tokens,
+                 _p(h_state_ptrs), _p(conv_state_ptrs), _p(tables), tables.numel() * tables.element_size(),
+                 ws.handle, _stream(stream))
+
+
+def kda_block_verify_fold(cu_seqlens, accepted, B: int, total_tokens: int, tables, h_state_ptrs, conv_state_ptrs,
+                          ws: Workspace, stream=None):
+    """Advance each sequence's recurrent and conv state past its accepted rows (device int32 [B])."""
+    return _call("kda_block_verify_fold", _p(cu_seqlens), _p(accepted), B, total_tokens, _p(tables),
+                 _p(h_state_ptrs), _p(conv_state_ptrs), ws.handle, _stream(stream))
+
+
+def kda_front_conv_silu_l2_varlen(x, conv_state_ptrs, conv_w, conv_out, cu_seqlens, B: int, total_tokens: int,
+                                  advance_state: bool, d: KdaDims, stream=None):
+    return _call("kda_front_conv_silu_l2_varlen", _p(x), _p(conv_state_ptrs), _p(conv_w), _p(conv_out),
+                 _p(cu_seqlens), B, total_tokens, 1 if advance_state else 0, ctypes.byref(d), _stream(stream))
+
+
+def kda_conv_state_fold(x, conv_state_ptrs, cu_seqlens, accepted, B: int, total_tokens: int, d: KdaDims,
+                        stream=None):
+    return _call("kda_conv_state_fold", _p(x), _p(conv_state_ptrs), _p(cu_seqlens), _p(accepted), B, total_tokens,
+                 ctypes.byref(d), _stream(stream))
+
+
+def kda_chunk_prefill_packed_scratch_bytes(max_seqs: int, max_total_tokens: int, d: KdaDims) -> int:
+    return int(lib().kda_chunk_prefill_packed_scratch_bytes(max_seqs, max_total_tokens, ctypes.byref(d)))
 
 
 def kda_gemv_bf16(x, W, y, M: int, N: int, K: int, ldx=None, ldw=None, ldy=None, stream=None):

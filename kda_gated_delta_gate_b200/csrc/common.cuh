@@ -101,6 +101,28 @@ int chunk_prefill_simt(const float *q, const float *k, const float *v, const flo
                        float *const *h_state, float *core, int B, int T, const kda_dims *dims, cudaStream_t s);
 size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D);
 size_t chunk_prefill_slots_scratch_bytes(int B, int nch, int H, int D);  // B streams x nch chunk slots
+// Scratch a packed (varlen) call of B streams, max_chunks chunks each at most, total rows needs.
+size_t chunk_prefill_varlen_need_bytes(int B, int max_chunks, int total, int H, int D);
+// Scratch enough for any packed call of at most max_seqs streams and max_total rows.
+size_t chunk_prefill_packed_bytes(int max_seqs, int max_total, int H, int D);
+int chunk_prefill_tc_fused_varlen(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
+                                  const float *beta, const int *cu_seqlens, int B, int max_chunks, int total,
+                                  float *const *h_state, float *core, const kda_dims *dims, void *scratch,
+                                  cudaStream_t s);
+int chunk_verify_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
+                          const float *beta, const int *cu_seqlens, int B, int total, float *const *h_state,
+                          float *core, float *tables, const kda_dims *dims, void *scratch, cudaStream_t s);
+// Accepted-row folding (kda_verify.cu): k as FP32 rows [total, H*D] (kf) or BF16 rows of
+// stride ldk elements (kb, pointing at head 0's channel 0 of row 0).
+int verify_fold(const float *kf, const uint16_t *kb, size_t ldk, const int *cu_seqlens, const int *accepted, int B,
+                int total, const float *tables, float *const *h_state, const kda_dims *dims, cudaStream_t s);
+// Packed-sequence front end (kda_front.cu): conv + SiLU + q|k L2 of every row from its own
+// sequence's conv state (read only), and the conv-state advance over each sequence's first
+// `accepted[b]` rows (all rows if accepted is null).
+int front_varlen(const uint16_t *x, uint16_t *const *conv_state, const uint16_t *conv_w, uint16_t *conv_out,
+                 const int *cu_seqlens, int B, int total, const kda_dims *dims, cudaStream_t s);
+int conv_state_advance(const uint16_t *x, uint16_t *const *conv_state, const int *cu_seqlens, const int *accepted,
+                       int B, int total, const kda_dims *dims, cudaStream_t s);
 int chunk_verify_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                     const int *cu_seqlens, int B, int total, float *const *h_state, float *core, float *tables,
                     const kda_dims *dims, void *scratch, cudaStream_t s);

@@ -152,6 +152,11 @@ extern "C" size_t kda_chunk_prefill_varlen_scratch_bytes(int B, int max_num_chun
     return kda::chunk_prefill_slots_scratch_bytes(B, max_num_chunks, dims->heads, dims->head_dim);
 }
 
+extern "C" size_t kda_chunk_prefill_packed_scratch_bytes(int max_seqs, int max_total_tokens, const kda_dims *dims) {
+    if (!dims || kda::check_dims(dims) != KDA_OK) return 0;
+    return kda::chunk_prefill_packed_bytes(max_seqs, max_total_tokens, dims->heads, dims->head_dim);
+}
+
 extern "C" int kda_chunk_prefill_varlen(const float *q, const float *k, const float *v, const float *gate,
                                         const float *beta, const int *cu_seqlens, int B, int max_num_chunks,
                                         int total_tokens, float *const *h_state, float *core, void *scratch,
@@ -168,7 +173,8 @@ extern "C" int kda_chunk_prefill_varlen(const float *q, const float *k, const fl
     if (max_num_chunks == 0) return KDA_ERR_INVALID_ARG;
     if (!scratch) return KDA_ERR_INVALID_ARG;
     if (!kda::aligned16(scratch)) return KDA_ERR_MISALIGNED;
-    if (scratch_bytes < kda::chunk_prefill_slots_scratch_bytes(B, max_num_chunks, dims->heads, dims->head_dim))
+    if (scratch_bytes <
+        kda::chunk_prefill_varlen_need_bytes(B, max_num_chunks, total_tokens, dims->heads, dims->head_dim))
         return KDA_ERR_CAPACITY;
     return kda::chunk_prefill_tc_varlen(q, k, v, gate, beta, cu_seqlens, B, max_num_chunks, total_tokens, h_state,
                                         core, dims, scratch, static_cast<cudaStream_t>(stream));

@@ -7,8 +7,19 @@
 //   chunked core, fused-input mode: reads conv_out and g_raw directly (the gate is formed in
 //   the kernel; rows past T are never read)  -> core [T_pad, H, D], recurrent state in place
 //   out_gate = g_b(g_a(h));  o_norm_out = gated RMSNorm(core, out_gate);  final_out = o_proj
-// The workspace is allocated once (kda_workspace_create) for at most max_tokens tokens; the
-// prefill call itself allocates nothing.
+// The workspace is allocated once (kda_workspace_create) for at most max_tokens tokens (and, for
+// packed calls, max_seqs sequences); the prefill call itself allocates nothing.
+//
+// Packed sequences (Glm5NextLayer batched prefill and its varlen form): the row-wise stages
+// (projections, gate, beta, o_norm, o_proj) run once over all rows of all sequences; the conv
+// takes each row's window from its own sequence and conv state, and the chunked core runs the
+// packed-sequence (cu_seqlens) layout, so no stage mixes two sequences.
+//
+// Batched verify (Glm5NextLayer speculative verify; Glm5NextKdaLayer `decode_k`): the draft rows
+// of N sequences, at most 64 each, through the same stages with every weight read once for all
+// rows; the core runs in verify mode from each sequence's states, which stay as they were, and
+// keeps the tables the fold needs. The fold then moves each sequence's recurrent state and conv
+// state past its accepted rows without rerunning anything.
 //
 // Block decode (Glm5NextKdaLayer `decode`, `decode_k`): the same projections for the call's
 // rows (N sequences x 1 token, or K rows of one sequence), each weight read once for all
@@ -18,6 +29,7 @@
 // by K and its own row: a row's projections are the same bits in a call of K rows and in a
 // call of one, which the decode_k identity needs. Larger batches (N independent sequences,
 // no such identity) run the tcgen05 GEMM.
+#include <algorithm>
 #include <cstring>
 #include <new>
 
@@ -28,6 +40,11 @@ namespace {
 // Writes the call's state pointer into the workspace's one-entry device pointer array (a kernel
 // argument, so no host synchronisation is involved).
 __global__ void store_ptr_kernel(float **slot, float *p) { *slot = p; }
+
+// cu_seqlens of B sequences of T rows each: cu[b] = b T.
+__global__ void equal_cu_kernel(int *cu, int B, int T) {
+    for (int b = threadIdx.x; b <= B; b += blockDim.x) cu[b] = b * T;
+}
 }  // namespace
 }
 
@@ -35,9 +52,11 @@ struct kda_workspace {
     kda_dims dims;
     int hidden, rank;
     size_t max_tokens, t_pad_max;
+    int max_seqs;
     void *buf[KDA_BUF_COUNT];
     size_t bytes[KDA_BUF_COUNT];
     float **state_slot;  // device array holding the one state pointer of the call
+    int *cu_equal;       // device [max_seqs + 1]: cu_seqlens of an equal-length batched call
 };
 
 namespace kda {
@@ -52,45 +71,84 @@ int proj(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *C, int ld
     return gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
 }
 
-// Projections of M rows of `hidden` into the workspace: qkv_proj (q|k|v packed), g_raw,
-// b_logit (FP32, in the BETA buffer), out_gate. For the matrix-vector path the weights that
-// read the same rows share a launch: [q | k | v], [f_a | g_a | b_proj], then f_b and g_b.
-int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M, kda_workspace *ws, cudaStream_t s) {
+// Projections of M rows of `hidden` into the workspace rows [r0, r0 + M): qkv_proj (q|k|v
+// packed), g_raw, b_logit (FP32, in the BETA buffer), out_gate. For the matrix-vector path the
+// weights that read the same rows share a launch: [q | k | v], [f_a | g_a | b_proj], then f_b
+// and g_b.
+int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M, kda_workspace *ws, cudaStream_t s,
+                      int r0 = 0) {
     const kda_dims *d = &ws->dims;
     const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
+    const size_t o = static_cast<size_t>(r0);
     auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    uint16_t *qkv_p = bf(KDA_BUF_QKV_PROJ) + o * cd, *fa = bf(KDA_BUF_F_A_OUT) + o * R, *ga = bf(KDA_BUF_G_A_OUT) + o * R;
+    uint16_t *graw = bf(KDA_BUF_G_RAW) + o * qkv, *og = bf(KDA_BUF_OUT_GATE) + o * qkv;
+    float *blog = f32(KDA_BUF_BETA) + o * H;
+    hidden += o * Hd;
     if (M <= kRowsGemv) {
         GemvSegs a{};
-        a.s[0] = GemvSeg{w->q_proj, bf(KDA_BUF_QKV_PROJ), qkv, Hd, cd, 0};
-        a.s[1] = GemvSeg{w->k_proj, bf(KDA_BUF_QKV_PROJ) + qkv, qkv, Hd, cd, 0};
-        a.s[2] = GemvSeg{w->v_proj, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, qkv, Hd, cd, 0};
+        a.s[0] = GemvSeg{w->q_proj, qkv_p, qkv, Hd, cd, 0};
+        a.s[1] = GemvSeg{w->k_proj, qkv_p + qkv, qkv, Hd, cd, 0};
+        a.s[2] = GemvSeg{w->v_proj, qkv_p + 2 * qkv, qkv, Hd, cd, 0};
         a.count = 3;
         a.total = 3 * qkv;
         KDA_TRY(gemv_segs(hidden, Hd, a, M, Hd, s));
         GemvSegs b{};
-        b.s[0] = GemvSeg{w->f_a, bf(KDA_BUF_F_A_OUT), R, Hd, R, 0};
-        b.s[1] = GemvSeg{w->g_a, bf(KDA_BUF_G_A_OUT), R, Hd, R, 0};
-        b.s[2] = GemvSeg{w->b_proj, f32(KDA_BUF_BETA), H, Hd, H, 1};
+        b.s[0] = GemvSeg{w->f_a, fa, R, Hd, R, 0};
+        b.s[1] = GemvSeg{w->g_a, ga, R, Hd, R, 0};
+        b.s[2] = GemvSeg{w->b_proj, blog, H, Hd, H, 1};
         b.count = 3;
         b.total = 2 * R + H;
         KDA_TRY(gemv_segs(hidden, Hd, b, M, Hd, s));
         // f_b and g_b read different rows (f_a_out, g_a_out) with one width: one launch
         GemvSegs c{};
-        c.s[0] = GemvSeg{w->f_b, bf(KDA_BUF_G_RAW), qkv, R, qkv, 0, bf(KDA_BUF_F_A_OUT)};
-        c.s[1] = GemvSeg{w->g_b, bf(KDA_BUF_OUT_GATE), qkv, R, qkv, 0, bf(KDA_BUF_G_A_OUT)};
+        c.s[0] = GemvSeg{w->f_b, graw, qkv, R, qkv, 0, fa};
+        c.s[1] = GemvSeg{w->g_b, og, qkv, R, qkv, 0, ga};
         c.count = 2;
         c.total = 2 * qkv;
-        return gemv_segs(bf(KDA_BUF_F_A_OUT), R, c, M, R, s);
+        return gemv_segs(fa, R, c, M, R, s);
     }
-    KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, M, qkv, Hd, 0, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, M, qkv, Hd, 0, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, M, qkv, Hd, 0, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, M, R, Hd, 0, s));
-    KDA_TRY(gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, M, qkv, R, 0, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, M, H, Hd, 1, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, M, R, Hd, 0, s));
-    return gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, M, qkv, R, 0, s);
+    KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, qkv_p, cd, M, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, qkv_p + qkv, cd, M, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->v_proj, Hd, qkv_p + 2 * qkv, cd, M, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->f_a, Hd, fa, R, M, R, Hd, 0, s));
+    KDA_TRY(gemm_bf16(fa, R, w->f_b, R, graw, qkv, M, qkv, R, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->b_proj, Hd, blog, H, M, H, Hd, 1, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->g_a, Hd, ga, R, M, R, Hd, 0, s));
+    return gemm_bf16(ga, R, w->g_b, R, og, qkv, M, qkv, R, 0, s);
+}
+
+// The prefill projections of T rows (always the tensor-core GEMM).
+int prefill_projections(const kda_block_weights *w, const kda_bf16 *hidden, int T, kda_workspace *ws,
+                        cudaStream_t s) {
+    const kda_dims *d = &ws->dims;
+    const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
+    auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    // q | k | v projections straight into the packed qkv_proj rows
+    KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, T, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, T, qkv, Hd, 0, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, T, qkv, Hd, 0, s));
+    // forget-gate input: g_raw = f_b(f_a(h)) (the gate itself is formed inside the chunked core)
+    KDA_TRY(gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, T, R, Hd, 0, s));
+    KDA_TRY(gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, T, qkv, R, 0, s));
+    // beta logits (FP32), the output gate's low-rank pair
+    KDA_TRY(gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, T, H, Hd, 1, s));
+    KDA_TRY(gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, T, R, Hd, 0, s));
+    return gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0, s);
+}
+
+// gated RMSNorm of `rows` core rows, then o_proj (GEMM) unless the caller applies its own.
+int prefill_back(const kda_block_weights *w, int rows, kda_workspace *ws, void *stream) {
+    const kda_dims *d = &ws->dims;
+    const int Hd = ws->hidden, qkv = d->heads * d->head_dim;
+    auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
+    KDA_TRY(kda_back_gated_rmsnorm(static_cast<float *>(ws->buf[KDA_BUF_CORE]), bf(KDA_BUF_OUT_GATE), w->o_norm,
+                                   bf(KDA_BUF_O_NORM_OUT), rows, d, stream));
+    if (!w->o_proj) return KDA_OK;  // the caller applies its own o_proj (a tensor-parallel slice)
+    return gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), Hd, rows, Hd, qkv, 0,
+                     static_cast<cudaStream_t>(stream));
 }
 
 int check_block_args(const kda_block_weights *w, const kda_bf16 *hidden, const kda_workspace *ws) {
@@ -106,18 +164,21 @@ int check_block_args(const kda_block_weights *w, const kda_bf16 *hidden, const k
 
 extern "C" {
 
-int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_tokens, kda_workspace **out) {
+int kda_workspace_create_batched(const kda_dims *dims, int hidden, int rank, size_t max_tokens, int max_seqs,
+                                 kda_workspace **out) {
     if (!out) return KDA_ERR_INVALID_ARG;
     *out = nullptr;
     KDA_TRY(kda::check_dims(dims));
-    if (hidden <= 0 || rank <= 0 || max_tokens == 0) return KDA_ERR_INVALID_ARG;
+    if (hidden <= 0 || rank <= 0 || max_tokens == 0 || max_seqs <= 0) return KDA_ERR_INVALID_ARG;
     if (hidden % 64 || rank % 64 || (dims->heads * dims->head_dim) % 64) return KDA_ERR_UNSUPPORTED;
+    if (max_tokens > 0x7fffffffULL || max_seqs > 65535) return KDA_ERR_UNSUPPORTED;
     kda_workspace *ws = new (std::nothrow) kda_workspace();
     if (!ws) return KDA_ERR_CUDA;
     ws->dims = *dims;
     ws->hidden = hidden;
     ws->rank = rank;
     ws->max_tokens = max_tokens;
+    ws->max_seqs = max_seqs;
     ws->t_pad_max = kda_t_pad(max_tokens, dims->chunk);
     const size_t T = max_tokens, Tp = ws->t_pad_max;
     const size_t qkv = static_cast<size_t>(dims->heads) * dims->head_dim, H = dims->heads;
@@ -136,7 +197,9 @@ int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_
         T * hidden * 2,    // FINAL_OUT
         T * rank * 2,      // F_A_OUT
         T * rank * 2,      // G_A_OUT
-        kda_chunk_prefill_scratch_bytes(1, static_cast<int>(T), dims),  // PREFILL_SCRATCH
+        // PREFILL_SCRATCH: one sequence of T rows, or any packed call of max_seqs sequences and
+        // T rows in all (the same size when max_seqs = 1)
+        kda::chunk_prefill_packed_bytes(max_seqs, static_cast<int>(T), dims->heads, dims->head_dim),
     };
     for (int i = 0; i < KDA_BUF_COUNT; ++i) {
         ws->bytes[i] = sizes[i];
@@ -145,7 +208,9 @@ int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_
             return KDA_ERR_CUDA;
         }
     }
-    if (cudaMalloc(reinterpret_cast<void **>(&ws->state_slot), sizeof(float *)) != cudaSuccess) {
+    if (cudaMalloc(reinterpret_cast<void **>(&ws->state_slot), sizeof(float *)) != cudaSuccess ||
+        cudaMalloc(reinterpret_cast<void **>(&ws->cu_equal), (static_cast<size_t>(max_seqs) + 1) * sizeof(int)) !=
+            cudaSuccess) {
         kda_workspace_destroy(ws);
         return KDA_ERR_CUDA;
     }
@@ -153,16 +218,23 @@ int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_
     return KDA_OK;
 }
 
+int kda_workspace_create(const kda_dims *dims, int hidden, int rank, size_t max_tokens, kda_workspace **out) {
+    return kda_workspace_create_batched(dims, hidden, rank, max_tokens, 1, out);
+}
+
 int kda_workspace_destroy(kda_workspace *ws) {
     if (!ws) return KDA_OK;
     for (int i = 0; i < KDA_BUF_COUNT; ++i)
         if (ws->buf[i]) cudaFree(ws->buf[i]);
     if (ws->state_slot) cudaFree(ws->state_slot);
+    if (ws->cu_equal) cudaFree(ws->cu_equal);
     delete ws;
     return KDA_OK;
 }
 
 size_t kda_workspace_max_tokens(const kda_workspace *ws) { return ws ? ws->max_tokens : 0; }
+
+int kda_workspace_max_seqs(const kda_workspace *ws) { return ws ? ws->max_seqs : 0; }
 
 int kda_workspace_buffer(const kda_workspace *ws, int which, void **ptr, size_t *bytes) {
     if (!ws || !ptr || which < 0 || which >= KDA_BUF_COUNT) return KDA_ERR_INVALID_ARG;
@@ -179,39 +251,60 @@ int kda_block_prefill(const kda_block_weights *w, const kda_bf16 *hidden, int T,
     if (static_cast<size_t>(T) > ws->max_tokens) return KDA_ERR_CAPACITY;
     const kda_dims *d = &ws->dims;
     auto s = static_cast<cudaStream_t>(stream);
-    const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
-    const int Tp = static_cast<int>(kda_t_pad(static_cast<size_t>(T), d->chunk));
-    auto B = [&](int i) { return ws->buf[i]; };
     auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
-
-    // q | k | v projections straight into the packed qkv_proj rows
-    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, T, qkv, Hd, 0, s));
-    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, T, qkv, Hd, 0, s));
-    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, T, qkv, Hd, 0, s));
+    KDA_TRY(kda::prefill_projections(w, hidden, T, ws, s));
     KDA_TRY(kda_front_conv_silu_l2(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), nullptr, nullptr,
                                    nullptr, pad_fill, T, d, stream));
-    // forget-gate input: g_raw = f_b(f_a(h)) (the gate itself is formed inside the chunked core)
-    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, T, R, Hd, 0, s));
-    KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, T, qkv, R, 0, s));
-    // beta = sigmoid(b_proj(h)), FP32 logits
-    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, T, H, Hd, 1, s));
-    KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), T * H, stream));
+    KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), T * d->heads, stream));
     // chunked core from the carried state, on the BF16 conv_out rows and g_raw
     kda::store_ptr_kernel<<<1, 1, 0, s>>>(ws->state_slot, h_state);
     KDA_TRY(kda::launch_status());
     KDA_TRY(kda_chunk_prefill_fused(bf(KDA_BUF_CONV_OUT), bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log, f32(KDA_BUF_BETA),
-                                    ws->state_slot, f32(KDA_BUF_CORE), 1, T, B(KDA_BUF_PREFILL_SCRATCH),
+                                    ws->state_slot, f32(KDA_BUF_CORE), 1, T, ws->buf[KDA_BUF_PREFILL_SCRATCH],
                                     ws->bytes[KDA_BUF_PREFILL_SCRATCH], d, stream));
-    // output gate, gated RMSNorm, output projection
-    KDA_TRY(kda::gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, T, R, Hd, 0, s));
-    KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0, s));
-    KDA_TRY(kda_back_gated_rmsnorm(f32(KDA_BUF_CORE), bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT), T, d,
-                                   stream));
-    if (w->o_proj)  // NULL: the caller applies its own o_proj (a tensor-parallel slice)
-        KDA_TRY(kda::gemm_bf16(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), Hd, T, Hd, qkv, 0, s));
-    (void)Tp;
-    return KDA_OK;
+    return kda::prefill_back(w, T, ws, stream);
+}
+
+int kda_block_prefill_varlen(const kda_block_weights *w, const kda_bf16 *hidden, const int *cu_seqlens, int B,
+                             int max_num_chunks, int total_tokens, float *const *h_state,
+                             kda_bf16 *const *conv_state, kda_workspace *ws, void *stream) {
+    KDA_TRY(kda::check_block_args(w, hidden, ws));
+    if (!cu_seqlens || !h_state || !conv_state || B < 0 || total_tokens < 0 || max_num_chunks < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (B == 0 || total_tokens == 0) return KDA_OK;
+    if (max_num_chunks == 0) return KDA_ERR_INVALID_ARG;
+    if (static_cast<size_t>(total_tokens) > ws->max_tokens || B > ws->max_seqs) return KDA_ERR_CAPACITY;
+    const kda_dims *d = &ws->dims;
+    if (ws->bytes[KDA_BUF_PREFILL_SCRATCH] <
+        kda::chunk_prefill_varlen_need_bytes(B, max_num_chunks, total_tokens, d->heads, d->head_dim))
+        return KDA_ERR_CAPACITY;
+    auto s = static_cast<cudaStream_t>(stream);
+    auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    KDA_TRY(kda::prefill_projections(w, hidden, total_tokens, ws, s));
+    KDA_TRY(kda::front_varlen(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), cu_seqlens, B,
+                              total_tokens, d, s));
+    KDA_TRY(kda::conv_state_advance(bf(KDA_BUF_QKV_PROJ), conv_state, cu_seqlens, nullptr, B, total_tokens, d, s));
+    KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), total_tokens * d->heads, stream));
+    KDA_TRY(kda::chunk_prefill_tc_fused_varlen(bf(KDA_BUF_CONV_OUT), bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
+                                               f32(KDA_BUF_BETA), cu_seqlens, B, max_num_chunks, total_tokens,
+                                               h_state, f32(KDA_BUF_CORE), d, ws->buf[KDA_BUF_PREFILL_SCRATCH], s));
+    return kda::prefill_back(w, total_tokens, ws, stream);
+}
+
+int kda_block_prefill_batched(const kda_block_weights *w, const kda_bf16 *hidden, int B, int T,
+                              float *const *h_state, kda_bf16 *const *conv_state, kda_workspace *ws, void *stream) {
+    KDA_TRY(kda::check_block_args(w, hidden, ws));
+    if (!h_state || !conv_state || B < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return KDA_OK;
+    if (B > ws->max_seqs || static_cast<long long>(B) * T > static_cast<long long>(ws->max_tokens))
+        return KDA_ERR_CAPACITY;
+    auto s = static_cast<cudaStream_t>(stream);
+    kda::equal_cu_kernel<<<1, 256, 0, s>>>(ws->cu_equal, B, T);
+    KDA_TRY(kda::launch_status());
+    const int nch = static_cast<int>(kda_t_pad(static_cast<size_t>(T), kda::kChunk) / kda::kChunk);
+    return kda_block_prefill_varlen(w, hidden, ws->cu_equal, B, nch, B * T, h_state, conv_state, ws, stream);
 }
 
 int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, float *const *h_state,
@@ -239,20 +332,74 @@ int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K
                        kda_workspace *ws, void *stream) {
     KDA_TRY(kda::check_block_args(w, hidden, ws));
     if (!h_state || !conv_state || K < 1) return KDA_ERR_INVALID_ARG;
-    if (K > 32) return KDA_ERR_UNSUPPORTED;
     if (static_cast<size_t>(K) > ws->max_tokens) return KDA_ERR_CAPACITY;
     auto s = static_cast<cudaStream_t>(stream);
     const kda_dims *d = &ws->dims;
-    const int qkv = d->heads * d->head_dim;
+    const int qkv = d->heads * d->head_dim, Hd = ws->hidden;
     auto bf = [&](int i) { return static_cast<kda_bf16 *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
-    KDA_TRY(kda::block_projections(w, hidden, K, ws, s));
+    // projections and o_proj in groups of at most kRowsGemv rows: the matrix-vector kernel gives
+    // each row the bits it gets alone, which the identity with serial decodes needs
+    for (int r0 = 0; r0 < K; r0 += kda::kRowsGemv)
+        KDA_TRY(kda::block_projections(w, hidden, std::min(kda::kRowsGemv, K - r0), ws, s, r0));
     KDA_TRY(kda_decode_k(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                          f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                          bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), K, h_snap, conv_snap, n_snap, d, stream));
     if (!w->o_proj) return KDA_OK;
-    return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, K, ws->hidden, qkv,
-                     0, s);
+    for (int r0 = 0; r0 < K; r0 += kda::kRowsGemv) {
+        const size_t o = static_cast<size_t>(r0);
+        KDA_TRY(kda::proj(bf(KDA_BUF_O_NORM_OUT) + o * qkv, qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT) + o * Hd, Hd,
+                          std::min(kda::kRowsGemv, K - r0), Hd, qkv, 0, s));
+    }
+    return KDA_OK;
+}
+
+int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const int *cu_seqlens, int B,
+                     int total_tokens, float *const *h_state, kda_bf16 *const *conv_state, float *tables,
+                     size_t tables_bytes, kda_workspace *ws, void *stream) {
+    KDA_TRY(kda::check_block_args(w, hidden, ws));
+    if (!cu_seqlens || !h_state || !conv_state || !tables || B < 0 || total_tokens < 0) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(tables)) return KDA_ERR_MISALIGNED;
+    if (B == 0 || total_tokens == 0) return KDA_OK;
+    if (static_cast<size_t>(total_tokens) > ws->max_tokens || B > ws->max_seqs) return KDA_ERR_CAPACITY;
+    const kda_dims *d = &ws->dims;
+    if (tables_bytes < kda_chunk_verify_tables_bytes(B, d)) return KDA_ERR_CAPACITY;
+    if (ws->bytes[KDA_BUF_PREFILL_SCRATCH] < kda::chunk_prefill_slots_scratch_bytes(B, 1, d->heads, d->head_dim))
+        return KDA_ERR_CAPACITY;
+    auto s = static_cast<cudaStream_t>(stream);
+    const int qkv = d->heads * d->head_dim;
+    auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
+    auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
+    // every weight read once for all draft rows of all sequences
+    KDA_TRY(kda::block_projections(w, hidden, total_tokens, ws, s));
+    KDA_TRY(kda::front_varlen(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), cu_seqlens, B,
+                              total_tokens, d, s));
+    KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), total_tokens * d->heads, stream));
+    KDA_TRY(kda::chunk_verify_tc_fused(bf(KDA_BUF_CONV_OUT), bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
+                                       f32(KDA_BUF_BETA), cu_seqlens, B, total_tokens, h_state, f32(KDA_BUF_CORE),
+                                       tables, d, ws->buf[KDA_BUF_PREFILL_SCRATCH], s));
+    KDA_TRY(kda_back_gated_rmsnorm(f32(KDA_BUF_CORE), bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
+                                   total_tokens, d, stream));
+    if (!w->o_proj) return KDA_OK;
+    return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, total_tokens,
+                     ws->hidden, qkv, 0, s);
+}
+
+int kda_block_verify_fold(const int *cu_seqlens, const int *accepted, int B, int total_tokens, const float *tables,
+                          float *const *h_state, kda_bf16 *const *conv_state, kda_workspace *ws, void *stream) {
+    if (!ws || !cu_seqlens || !accepted || !tables || !h_state || !conv_state || B < 0 || total_tokens < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (B == 0) return KDA_OK;
+    if (static_cast<size_t>(total_tokens) > ws->max_tokens || B > ws->max_seqs) return KDA_ERR_CAPACITY;
+    auto s = static_cast<cudaStream_t>(stream);
+    const kda_dims *d = &ws->dims;
+    const size_t qkv = static_cast<size_t>(d->heads) * d->head_dim;
+    const auto *conv_out = static_cast<const uint16_t *>(ws->buf[KDA_BUF_CONV_OUT]);
+    // k: the BF16 k channels of the verify's conv_out rows (what its core read)
+    KDA_TRY(kda::verify_fold(nullptr, conv_out + qkv, 3 * qkv, cu_seqlens, accepted, B, total_tokens, tables, h_state,
+                             d, s));
+    return kda::conv_state_advance(static_cast<const uint16_t *>(ws->buf[KDA_BUF_QKV_PROJ]), conv_state, cu_seqlens,
+                                   accepted, B, total_tokens, d, s);
 }
 
 }  // extern "C"

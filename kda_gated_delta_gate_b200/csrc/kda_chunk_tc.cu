@@ -139,9 +139,24 @@ __device__ __forceinline__ float4 load4_in(const PrefillIn &in, int part, size_t
 struct Seqs {
     const int *cu;  // device [B + 1], or nullptr
     int T, T_pad;   // equal-length mode
-    int nch;        // chunk slots per stream: T_pad / C, or max_num_chunks
+    int nch;        // chunks a stream may have: T_pad / C, or max_num_chunks
     int total;      // varlen mode: rows of the packed buffers
+    int slots;      // varlen mode, compact pack layout: pack slots per head; 0 = one slot per
+                    // (stream, head, chunk)
 };
+
+// The operand pack of chunk c of stream b, head h (row0: the chunk's first row, from seq_chunk).
+// Rectangular layout: slot (b H + h) nch + c. Compact layout (varlen mode, sq.slots > 0): head h
+// owns slots [h slots, (h + 1) slots) and stream b's chunks take the consecutive slots from
+// floor(cu[b] / C) + b. Consecutive streams cannot collide: the next stream starts at
+// floor(cu[b+1] / C) + b + 1, at least this one's start plus its ceil(len / C) chunks. The last
+// slot any stream with 0 <= cu[b] <= cu[b+1] <= total uses is below ceil(total / C) + B - 1,
+// the per-head slot count the host sizes the scratch for.
+__device__ __forceinline__ size_t pack_slot(const Seqs &sq, int b, int h, int c, size_t row0, int H) {
+    if (sq.slots)
+        return static_cast<size_t>(h) * sq.slots + (row0 - static_cast<size_t>(c) * C) / C + b + c;
+    return (static_cast<size_t>(b) * H + h) * sq.nch + c;
+}
 
 // Rows of chunk c of stream b: first row (row0) and count (n). False for an empty slot or (in
 // varlen mode) a stream whose bounds are not inside the buffers, which also latches
@@ -449,7 +464,7 @@ __device__ __forceinline__ void intra_simt_body(const PrefillIn &in, uint8_t *__
     //      K o e^{Gamma_C - Gamma} = Z S_a (pack), with P_a / S_a the decay of all blocks before /
     //      after block a; 16-byte chunks of 8 channels. v replaces a = e^g in sA (pad rows 0).
     using PK = Pack<D>;
-    uint8_t *pack = scratch + ((static_cast<size_t>(b) * H + h) * sq.nch + ch) * PK::bytes;
+    uint8_t *pack = scratch + pack_slot(sq, b, h, ch, row0, H) * PK::bytes;
     for (int e = tid; e < C * (D / 8); e += NT) {
         const int i = e / (D / 8), cb = 8 * (e % (D / 8)), a = i >> 4;
         float xq[8], xb[8];
@@ -764,7 +779,7 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
         int n;
         size_t row0;
         seq_chunk(sq, b, ch, row0, n, nullptr);
-        uint8_t *pack = scratch + static_cast<size_t>(item) * PK::bytes;
+        uint8_t *pack = scratch + pack_slot(sq, b, h, ch, row0, H) * PK::bytes;
         if (dead) {  // block-uniform
             if (tid == 0) list[1 + atomicAdd(list, 1)] = item;
             continue;
@@ -1184,6 +1199,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     const size_t rs = static_cast<size_t>(H) * D;
     const int nch = sq.nch;  // chunk slots per stream in the scratch
     int nb = nch;            // this stream's chunks
+    size_t first_row = 0;    // its first row (varlen mode)
     if (sq.cu) {
         const int s0 = sq.cu[b], s1 = sq.cu[b + 1];
         if (s0 < 0 || s1 < s0 || s1 > sq.total || s1 - s0 > nch * C) {  // a bad cu_seqlens entry
@@ -1191,10 +1207,11 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             return;
         }
         nb = (s1 - s0 + C - 1) / C;
+        first_row = static_cast<size_t>(s0);
     }
     if (nb == 0) return;  // an empty stream keeps its state
     float *Sg = h_state[b] + static_cast<size_t>(h) * D * D;
-    const uint8_t *packs = scratch + (static_cast<size_t>(b) * H + h) * nch * PK::bytes;
+    const uint8_t *packs = scratch + pack_slot(sq, b, h, 0, first_row, H) * PK::bytes;  // chunks follow
     const bool ctl = warp == kEpiWarps && lane == 0;      // the chain thread
     const bool ctl2 = warp == kEpiWarps + 1 && lane == 0;  // the output thread
 
@@ -1534,7 +1551,12 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
 // Scratch layout: the operand packs, then a 256-byte slot with the count of chunks the
 // tensor-core intra kernel handed to the CUDA-core body, then their (b, h, chunk) ids.
 template <int D>
-size_t packs_bytes(int B, int H, int nch) { return static_cast<size_t>(B) * H * nch * Pack<D>::bytes; }
+size_t packs_bytes(long long npacks) { return static_cast<size_t>(npacks) * Pack<D>::bytes; }
+
+// Packs the call's layout holds: one per (stream, head, chunk slot), or H x slots (compact).
+long long pack_count(int B, int H, const Seqs &sq) {
+    return static_cast<long long>(H) * (sq.slots ? sq.slots : static_cast<long long>(B) * sq.nch);
+}
 
 template <int D, int DVS, int MODE>
 int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, int H, float scale,
@@ -1547,7 +1569,7 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     KDA_TRY(smem_opt_in(intra_fix_kernel<D, MODE>, static_cast<int>(Intra<D>::bytes), attr_fix));
     KDA_TRY(smem_opt_in(state_kernel<D, DVS>, State<D, DVS>::bytes, attr_state));
     uint8_t *sc = static_cast<uint8_t *>(scratch);
-    int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(B, H, nch));
+    int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(pack_count(B, H, sq)));
     if (cudaMemsetAsync(list, 0, sizeof(int), s) != cudaSuccess) return KDA_ERR_CUDA;
     int sms = 148;
     {
@@ -1556,6 +1578,7 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
     const long long items = static_cast<long long>(B) * H * nch;
+    if (items > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;  // item ids are int
     // two tensor-core intra CTAs per SM; the CUDA-core fix-up runs one per SM
     const int grid = static_cast<int>(std::min<long long>(items, 2LL * sms));
     const int grid_fix = static_cast<int>(std::min<long long>(items, sms));
@@ -1599,7 +1622,21 @@ int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, c
 
 Seqs equal_seqs(int T) {
     const int T_pad = static_cast<int>(kda_t_pad(static_cast<size_t>(T), C));
-    return Seqs{nullptr, T, T_pad, T_pad / C, 0};
+    return Seqs{nullptr, T, T_pad, T_pad / C, 0, 0};
+}
+
+size_t scratch_for_packs(long long npacks, int D) {
+    const size_t packs = D == 64 ? packs_bytes<64>(npacks) : packs_bytes<128>(npacks);
+    const size_t list = (4 + 4 * static_cast<size_t>(npacks) + 255) / 256 * 256;
+    return packs + list;
+}
+
+// Packed streams: the compact layout when it takes fewer slots than one per (stream, chunk).
+Seqs varlen_seqs(const int *cu, int B, int max_chunks, int total) {
+    const long long rect = static_cast<long long>(B) * max_chunks;
+    const long long compact = (static_cast<long long>(total) + C - 1) / C + B - 1;
+    const int slots = compact < rect ? static_cast<int>(compact) : 0;
+    return Seqs{cu, 0, 0, max_chunks, total, slots};
 }
 
 }  // namespace
@@ -1611,9 +1648,18 @@ size_t chunk_prefill_scratch_bytes(int B, int T, int H, int D) {
 
 size_t chunk_prefill_slots_scratch_bytes(int B, int nch, int H, int D) {
     if (B <= 0 || nch <= 0 || H <= 0) return 0;
-    const size_t packs = D == 64 ? packs_bytes<64>(B, H, nch) : packs_bytes<128>(B, H, nch);
-    const size_t list = (4 + 4 * static_cast<size_t>(B) * H * nch + 255) / 256 * 256;
-    return packs + list;
+    return scratch_for_packs(static_cast<long long>(B) * H * nch, D);
+}
+
+size_t chunk_prefill_varlen_need_bytes(int B, int max_chunks, int total, int H, int D) {
+    if (B <= 0 || max_chunks <= 0 || H <= 0) return 0;
+    return scratch_for_packs(pack_count(B, H, varlen_seqs(nullptr, B, max_chunks, total)), D);
+}
+
+size_t chunk_prefill_packed_bytes(int max_seqs, int max_total, int H, int D) {
+    if (max_seqs <= 0 || max_total <= 0 || H <= 0) return 0;
+    return scratch_for_packs(static_cast<long long>(H) * ((static_cast<long long>(max_total) + C - 1) / C + max_seqs - 1),
+                             D);
 }
 
 int chunk_prefill_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
@@ -1627,14 +1673,14 @@ int chunk_prefill_tc_varlen(const float *q, const float *k, const float *v, cons
                             const int *cu_seqlens, int B, int max_chunks, int total, float *const *h_state,
                             float *core, const kda_dims *dims, void *scratch, cudaStream_t s) {
     const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, nullptr};
-    return launch_any<kInF32>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, max_chunks, total}, dims, scratch, s);
+    return launch_any<kInF32>(in, h_state, core, B, varlen_seqs(cu_seqlens, B, max_chunks, total), dims, scratch, s);
 }
 
 int chunk_verify_tc(const float *q, const float *k, const float *v, const float *gate, const float *beta,
                     const int *cu_seqlens, int B, int total, float *const *h_state, float *core, float *tables,
                     const kda_dims *dims, void *scratch, cudaStream_t s) {
     const PrefillIn in{q, k, v, gate, nullptr, nullptr, nullptr, nullptr, beta, tables};
-    return launch_any<kInF32>(in, h_state, core, B, Seqs{cu_seqlens, 0, 0, 1, total}, dims, scratch, s);
+    return launch_any<kInF32>(in, h_state, core, B, varlen_seqs(cu_seqlens, B, 1, total), dims, scratch, s);
 }
 
 int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
@@ -1642,6 +1688,22 @@ int chunk_prefill_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const flo
                            void *scratch, cudaStream_t s) {
     const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta, nullptr};
     return launch_any<kInFused>(in, h_state, core, B, equal_seqs(T), dims, scratch, s);
+}
+
+int chunk_prefill_tc_fused_varlen(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
+                                  const float *beta, const int *cu_seqlens, int B, int max_chunks, int total,
+                                  float *const *h_state, float *core, const kda_dims *dims, void *scratch,
+                                  cudaStream_t s) {
+    const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta, nullptr};
+    return launch_any<kInFused>(in, h_state, core, B, varlen_seqs(cu_seqlens, B, max_chunks, total), dims, scratch,
+                                s);
+}
+
+int chunk_verify_tc_fused(const uint16_t *qkv, const uint16_t *g_raw, const float *dt_bias, const float *a_log,
+                          const float *beta, const int *cu_seqlens, int B, int total, float *const *h_state,
+                          float *core, float *tables, const kda_dims *dims, void *scratch, cudaStream_t s) {
+    const PrefillIn in{nullptr, nullptr, nullptr, nullptr, qkv, g_raw, dt_bias, a_log, beta, tables};
+    return launch_any<kInFused>(in, h_state, core, B, varlen_seqs(cu_seqlens, B, 1, total), dims, scratch, s);
 }
 
 int chunk_prefill_tc_graw(const float *q, const float *k, const float *v, const uint16_t *g_raw,

@@ -5,7 +5,8 @@
 //   kda_decode_fused     : the whole stateful row (conv + SiLU + L2, gate, beta, recurrence,
 //                          sigmoid-gated RMSNorm) for N sequences, one token each.
 //   kda_decode_k         : the same row K times for one sequence, state kept on chip,
-//                          snapshots after each row but the last.
+//                          snapshots after each row but the last (groups of up to 32 rows
+//                          per launch, chained through the state in place).
 // decode_fused and decode_k launch the SAME kernel (N sequences x K rows), so every row
 // executes identical device code; all arithmetic on the row uses explicitly rounded
 // intrinsics (__fmul_rn / __fadd_rn / __fmaf_rn), which the compiler may not re-associate
@@ -434,7 +435,6 @@ int kda_decode_k(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w
                  float *core, int K, float *const *h_snap, kda_bf16 *const *conv_snap, int n_snap,
                  const kda_dims *dims, void *stream) {
     if (K < 1 || !conv_state || !h_state) return KDA_ERR_INVALID_ARG;
-    if (K > kda::kMaxSnap + 1) return KDA_ERR_UNSUPPORTED;
     if (n_snap != 0 && n_snap != K - 1) return KDA_ERR_INVALID_ARG;
     if (n_snap > 0 && (!h_snap || !conv_snap)) return KDA_ERR_INVALID_ARG;
     kda::RowParams p;
@@ -444,11 +444,38 @@ int kda_decode_k(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w
     for (int t = 0; t < n_snap; ++t) {
         if (!h_snap[t] || !conv_snap[t]) return KDA_ERR_INVALID_ARG;
         if (!kda::aligned16(h_snap[t])) return KDA_ERR_MISALIGNED;
-        p.h_snap[t] = h_snap[t];
-        p.conv_snap[t] = conv_snap[t];
     }
-    p.conv_one = conv_state; p.h_one = h_state; p.K = K; p.n_snap = n_snap;
-    return kda::launch_rows(p, 1, dims->head_dim, static_cast<cudaStream_t>(stream));
+    // One launch takes at most kMaxSnap + 1 rows (its snapshot pointers travel in the kernel
+    // parameters). Longer calls run in groups, each continuing from the state the previous one
+    // left in place: the FP32 state and the BF16 conv inputs round-trip exactly, so every row
+    // sees the bits it would in one launch. A group that is not the last also snapshots its
+    // own last row: the conv state from the kernel, the recurrent state (which the kernel
+    // streams to h_state) by a copy.
+    const size_t qkv = static_cast<size_t>(dims->heads) * dims->head_dim;
+    const size_t h_bytes = qkv * dims->head_dim * sizeof(float);
+    auto s = static_cast<cudaStream_t>(stream);
+    const kda::RowParams base = p;
+    for (int r0 = 0; r0 < K;) {
+        const bool final_group = K - r0 <= kda::kMaxSnap + 1;
+        const int rows = final_group ? K - r0 : (n_snap ? kda::kMaxSnap : kda::kMaxSnap + 1);
+        p = base;
+        p.x = base.x + r0 * 3 * qkv; p.g_raw = base.g_raw + r0 * qkv; p.b_logit = base.b_logit + r0 * dims->heads;
+        p.out_gate = base.out_gate + r0 * qkv; p.o_norm_out = base.o_norm_out + r0 * qkv;
+        if (base.conv_out) p.conv_out = base.conv_out + r0 * 3 * qkv;
+        if (base.core) p.core = base.core + r0 * qkv;
+        p.conv_one = conv_state; p.h_one = h_state; p.K = rows;
+        p.n_snap = n_snap ? (final_group ? rows - 1 : rows) : 0;
+        for (int t = 0; t < p.n_snap; ++t) {
+            p.h_snap[t] = h_snap[r0 + t];
+            p.conv_snap[t] = conv_snap[r0 + t];
+        }
+        KDA_TRY(kda::launch_rows(p, 1, dims->head_dim, s));
+        if (n_snap && !final_group &&
+            cudaMemcpyAsync(h_snap[r0 + rows - 1], h_state, h_bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        r0 += rows;
+    }
+    return KDA_OK;
 }
 
 }  // extern "C"

@@ -153,7 +153,205 @@ __global__ void __launch_bounds__(kFrontThreads, 3) front_kernel(const uint16_t 
     }
 }
 
+// ---- packed sequences (cu_seqlens): the same per-row arithmetic as front_kernel, each row's
+// window taken from its own sequence (the carried conv state before the sequence's first row).
+// A token tile may hold the end of one sequence and the start of the next; the window is
+// rebuilt at each sequence start. The conv states are only read here: conv_advance_kernel
+// moves them on afterwards, so no reader of a state can race its writer.
+
+// Row r of sequence [s0, s1) (r < s0 reaches into the carried state, 3 inputs deep); st holds
+// the state's 8 channels x 3 inputs once loaded.
+__device__ __forceinline__ void window_input(const uint16_t *x, const float (&st)[24], int r, int s0, int cd,
+                                             int c0, float (&out)[8]) {
+    if (r >= s0) {
+        unpack8(*reinterpret_cast<const uint4 *>(x + static_cast<size_t>(r) * cd + c0), out);
+    } else {
+        const int m = r - s0 + 3;  // 0..2: oldest .. newest carried input
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[e] = m == 0 ? st[3 * e] : (m == 1 ? st[3 * e + 1] : st[3 * e + 2]);
+    }
+}
+
+__device__ __forceinline__ void load_state8(const uint16_t *cst, int c0, float (&st)[24]) {
+#pragma unroll
+    for (int q3 = 0; q3 < 3; ++q3) {
+        float tmp[8];
+        unpack8(reinterpret_cast<const uint4 *>(cst + static_cast<size_t>(c0) * 3)[q3], tmp);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) st[8 * q3 + e] = tmp[e];
+    }
+}
+
+// Sequence bounds [s0, s1) of stream b, false (and the error latched) when they do not fit.
+__device__ __forceinline__ bool seq_bounds(const int *cu, int b, int total, int &s0, int &s1, int *status) {
+    s0 = cu[b];
+    s1 = cu[b + 1];
+    if (s0 < 0 || s1 < s0 || s1 > total) {
+        atomicExch(status, KDA_ERR_INVALID_ARG);
+        return false;
+    }
+    return true;
+}
+
+// Row t starts (or resumes) sequence b: its bounds, and the window x_{t-3} .. x_{t-1} from its
+// rows and carried state. False (the error latched) if t is not in the sequence or the state
+// pointer is misaligned. Every thread of a block reads the same cu entries: block-uniform.
+__device__ __forceinline__ bool enter_seq(const uint16_t *x, uint16_t *const *conv_state, const int *cu, int b, int t,
+                                          int total, int cd, int c0, int &s0, int &s1, float (&xm)[3][8],
+                                          int *status) {
+    if (!seq_bounds(cu, b, total, s0, s1, status) || t < s0 || t >= s1) {
+        atomicExch(status, KDA_ERR_INVALID_ARG);
+        return false;
+    }
+    const uint16_t *cst = conv_state[b];
+    if (reinterpret_cast<uintptr_t>(cst) & 15) {
+        atomicExch(status, KDA_ERR_MISALIGNED);
+        return false;
+    }
+    float st[24];
+    if (t - s0 < 3) load_state8(cst, c0, st);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) window_input(x, st, t - 3 + j, s0, cd, c0, xm[j]);
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFrontThreads, 2)
+front_varlen_kernel(const uint16_t *__restrict__ x, uint16_t *const *__restrict__ conv_state,
+                    const uint16_t *__restrict__ conv_w, uint16_t *__restrict__ conv_out, const int *__restrict__ cu,
+                    int B, int total, int H, float eps, int *__restrict__ status) {
+    constexpr int LG = D / 8;
+    const int qkv = H * D, cd = 3 * qkv;
+    const int g = blockIdx.y * kFrontThreads + threadIdx.x;
+    const bool valid = 8 * g < cd;
+    const int c0 = valid ? 8 * g : 0;
+    const int part = c0 / qkv;
+    const int t0 = blockIdx.x * kTT, tend = min(t0 + kTT, total);
+    float w[4][8];
+    {
+        float wr[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float tmp[8];
+            unpack8(reinterpret_cast<const uint4 *>(conv_w + static_cast<size_t>(c0) * 4)[q4], tmp);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) wr[8 * q4 + e] = tmp[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j][e] = wr[4 * e + j];
+    }
+    // the sequence holding row t0: the last b with cu[b] <= t0 (empty sequences are passed over)
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cu[mid] <= t0) lo = mid;
+        else hi = mid - 1;
+    }
+    int b = lo, s0 = 0, s1 = 0;
+    float xm[3][8];
+    if (t0 >= tend || !enter_seq(x, conv_state, cu, b, t0, total, cd, c0, s0, s1, xm, status)) return;
+    for (int t = t0; t < tend; ++t) {
+        if (t == s1) {  // the next non-empty sequence starts here
+            while (b < B - 1 && cu[b + 1] <= t) ++b;
+            if (!enter_seq(x, conv_state, cu, b, t, total, cd, c0, s0, s1, xm, status)) return;
+        }
+        float xc[8], c[8];
+        unpack8(*reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * cd + c0), xc);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float y = w[0][e] * xm[0][e];
+            y = fmaf(w[1][e], xm[1][e], y);
+            y = fmaf(w[2][e], xm[2][e], y);
+            y = fmaf(w[3][e], xc[e], y);
+            y = y * sigmoid_f32(y);
+            c[e] = bf16_to_f32(f32_to_bf16(y));
+            ss = fmaf(c[e], c[e], ss);
+            xm[0][e] = xm[1][e]; xm[1][e] = xm[2][e]; xm[2][e] = xc[e];
+        }
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rs = part < 2 ? rsqrtf(ss + eps) : 1.f;
+        uint16_t ob[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ob[e] = f32_to_bf16(part < 2 ? c[e] * rs : c[e]);
+        if (valid)
+            *reinterpret_cast<uint4 *>(conv_out + static_cast<size_t>(t) * cd + c0) =
+                make_uint4(pack2(ob[0], ob[1]), pack2(ob[2], ob[3]), pack2(ob[4], ob[5]), pack2(ob[6], ob[7]));
+    }
+}
+
+// Conv state of sequence b after its first r rows (r = accepted[b], or all of them): the last
+// three inputs of (state || x rows s0 .. s0 + r - 1). One thread per 8 channels of a sequence
+// reads its state before it writes it.
+__global__ void __launch_bounds__(kFrontThreads)
+conv_advance_kernel(const uint16_t *__restrict__ x, uint16_t *const *__restrict__ conv_state,
+                    const int *__restrict__ cu, const int *__restrict__ accepted, int total, int cd,
+                    int *__restrict__ status) {
+    const int b = blockIdx.x, g = blockIdx.y * kFrontThreads + threadIdx.x;
+    if (8 * g >= cd) return;
+    const int c0 = 8 * g;
+    int s0, s1;
+    if (!seq_bounds(cu, b, total, s0, s1, status)) return;
+    const int r = accepted ? accepted[b] : s1 - s0;
+    if (r < 0 || r > s1 - s0) {
+        atomicExch(status, KDA_ERR_INVALID_ARG);
+        return;
+    }
+    if (r == 0) return;  // nothing taken: the state stays
+    uint16_t *cst = conv_state[b];
+    if (reinterpret_cast<uintptr_t>(cst) & 15) {
+        atomicExch(status, KDA_ERR_MISALIGNED);
+        return;
+    }
+    float st[24];
+    load_state8(cst, c0, st);
+    uint16_t ns[24];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        float v8[8];
+        window_input(x, st, s0 + r - 3 + j, s0, cd, c0, v8);  // input r + j of (state || x)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ns[3 * e + j] = f32_to_bf16(v8[e]);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(cst + static_cast<size_t>(c0) * 3);
+#pragma unroll
+    for (int q3 = 0; q3 < 3; ++q3)
+        dst[q3] = make_uint4(pack2(ns[8 * q3], ns[8 * q3 + 1]), pack2(ns[8 * q3 + 2], ns[8 * q3 + 3]),
+                             pack2(ns[8 * q3 + 4], ns[8 * q3 + 5]), pack2(ns[8 * q3 + 6], ns[8 * q3 + 7]));
+}
+
 }  // namespace
+
+int front_varlen(const uint16_t *x, uint16_t *const *conv_state, const uint16_t *conv_w, uint16_t *conv_out,
+                 const int *cu_seqlens, int B, int total, const kda_dims *dims, cudaStream_t s) {
+    if (B == 0 || total == 0) return KDA_OK;
+    int *status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
+    const int cd = 3 * dims->heads * dims->head_dim;
+    dim3 grid((total + kTT - 1) / kTT, (cd / 8 + kFrontThreads - 1) / kFrontThreads);
+    if (dims->head_dim == 128)
+        front_varlen_kernel<128><<<grid, kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, cu_seqlens, B, total,
+                                                                dims->heads, dims->l2_eps, status);
+    else
+        front_varlen_kernel<64><<<grid, kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, cu_seqlens, B, total,
+                                                               dims->heads, dims->l2_eps, status);
+    return launch_status();
+}
+
+int conv_state_advance(const uint16_t *x, uint16_t *const *conv_state, const int *cu_seqlens, const int *accepted,
+                       int B, int total, const kda_dims *dims, cudaStream_t s) {
+    if (B == 0) return KDA_OK;
+    int *status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
+    const int cd = 3 * dims->heads * dims->head_dim;
+    dim3 grid(B, (cd / 8 + kFrontThreads - 1) / kFrontThreads);
+    conv_advance_kernel<<<grid, kFrontThreads, 0, s>>>(x, conv_state, cu_seqlens, accepted, total, cd, status);
+    return launch_status();
+}
+
 }  // namespace kda
 
 extern "C" int kda_front_conv_silu_l2(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w,
@@ -178,4 +376,29 @@ extern "C" int kda_front_conv_silu_l2(const kda_bf16 *x, kda_bf16 *conv_state, c
         kda::front_kernel<64><<<grid, kda::kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, q_f32, k_f32, v_f32,
                                                                   pad_fill, T, T_pad, dims->heads, dims->l2_eps);
     return kda::launch_status();
+}
+
+extern "C" int kda_front_conv_silu_l2_varlen(const kda_bf16 *x, kda_bf16 *const *conv_state, const kda_bf16 *conv_w,
+                                             kda_bf16 *conv_out, const int *cu_seqlens, int B, int total_tokens,
+                                             int advance_state, const kda_dims *dims, void *stream) {
+    KDA_TRY(kda::check_dims(dims));
+    if (!x || !conv_state || !conv_w || !conv_out || !cu_seqlens || B < 0 || total_tokens < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(x) || !kda::aligned16(conv_w) || !kda::aligned16(conv_out)) return KDA_ERR_MISALIGNED;
+    if (B > 65535) return KDA_ERR_UNSUPPORTED;
+    if (B == 0 || total_tokens == 0) return KDA_OK;
+    auto s = static_cast<cudaStream_t>(stream);
+    KDA_TRY(kda::front_varlen(x, conv_state, conv_w, conv_out, cu_seqlens, B, total_tokens, dims, s));
+    if (!advance_state) return KDA_OK;
+    return kda::conv_state_advance(x, conv_state, cu_seqlens, nullptr, B, total_tokens, dims, s);
+}
+
+extern "C" int kda_conv_state_fold(const kda_bf16 *x, kda_bf16 *const *conv_state, const int *cu_seqlens,
+                                   const int *accepted, int B, int total_tokens, const kda_dims *dims, void *stream) {
+    KDA_TRY(kda::check_dims(dims));
+    if (!x || !conv_state || !cu_seqlens || B < 0 || total_tokens < 0) return KDA_ERR_INVALID_ARG;
+    if (!kda::aligned16(x)) return KDA_ERR_MISALIGNED;
+    if (B > 65535) return KDA_ERR_UNSUPPORTED;
+    return kda::conv_state_advance(x, conv_state, cu_seqlens, accepted, B, total_tokens, dims,
+                                   static_cast<cudaStream_t>(stream));
 }

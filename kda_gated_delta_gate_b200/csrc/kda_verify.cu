@@ -14,11 +14,13 @@
 namespace kda {
 namespace {
 
+// k rows: FP32 [total, H*D] (kf), or BF16 rows of ldk elements (kb: the block's conv_out, whose
+// k channels the verify read the same way, widened exactly).
 template <int D>
 __global__ void __launch_bounds__(256)
-fold_kernel(const float *__restrict__ k, const int *__restrict__ cu, const int *__restrict__ accepted,
-            const float *__restrict__ tables, float *const *__restrict__ h_state, int H, int total,
-            int *__restrict__ status) {
+fold_kernel(const float *__restrict__ kf, const uint16_t *__restrict__ kb, size_t ldk, const int *__restrict__ cu,
+            const int *__restrict__ accepted, const float *__restrict__ tables, float *const *__restrict__ h_state,
+            int H, int total, int *__restrict__ status) {
     extern __shared__ __align__(16) float fs[];
     float *w = fs;               // [64][D]: k_t o e^{Gamma_{r-1} - Gamma_t}
     float *u = fs + kChunk * D;  // [64][D]: u_t
@@ -32,11 +34,11 @@ fold_kernel(const float *__restrict__ k, const int *__restrict__ cu, const int *
     if (r == 0) return;  // nothing accepted: the state stays
     const float *U = tables + (static_cast<size_t>(b) * H + h) * 2 * kChunk * D;
     const float *G = U + kChunk * D;
-    const size_t rs = static_cast<size_t>(H) * D;
     for (int e = tid; e < r * D; e += 256) {
         const int t = e / D, i = e % D;
-        w[e] = k[(static_cast<size_t>(s0) + t) * rs + static_cast<size_t>(h) * D + i] *
-               expf(G[(r - 1) * D + i] - G[t * D + i]);
+        const size_t at = (static_cast<size_t>(s0) + t) * ldk + static_cast<size_t>(h) * D + i;
+        const float kv = kf ? kf[at] : bf16_to_f32(kb[at]);
+        w[e] = kv * expf(G[(r - 1) * D + i] - G[t * D + i]);
         u[e] = U[e];
     }
     for (int i = tid; i < D; i += 256) dcy[i] = expf(G[(r - 1) * D + i]);
@@ -53,6 +55,29 @@ fold_kernel(const float *__restrict__ k, const int *__restrict__ cu, const int *
 }
 
 }  // namespace
+
+int verify_fold(const float *kf, const uint16_t *kb, size_t ldk, const int *cu_seqlens, const int *accepted, int B,
+                int total, const float *tables, float *const *h_state, const kda_dims *dims, cudaStream_t s) {
+    if (B == 0) return KDA_OK;
+    int *status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
+    const int D = dims->head_dim;
+    const int bytes = (2 * kChunk * D + D) * static_cast<int>(sizeof(float));
+    dim3 grid(dims->heads, B);
+    if (D == 128) {
+        static std::atomic<unsigned long long> attr{0};
+        KDA_TRY(smem_opt_in(fold_kernel<128>, bytes, attr));
+        fold_kernel<128><<<grid, 256, bytes, s>>>(kf, kb, ldk, cu_seqlens, accepted, tables, h_state, dims->heads,
+                                                   total, status);
+    } else {
+        static std::atomic<unsigned long long> attr{0};
+        KDA_TRY(smem_opt_in(fold_kernel<64>, bytes, attr));
+        fold_kernel<64><<<grid, 256, bytes, s>>>(kf, kb, ldk, cu_seqlens, accepted, tables, h_state, dims->heads,
+                                                  total, status);
+    }
+    return launch_status();
+}
+
 }  // namespace kda
 
 extern "C" {
@@ -89,25 +114,8 @@ int kda_chunk_verify_fold(const float *k, const int *cu_seqlens, const int *acce
     KDA_TRY(kda::check_dims(dims));
     if (!k || !cu_seqlens || !accepted || !tables || !h_state || B < 0 || total_tokens < 0) return KDA_ERR_INVALID_ARG;
     if (B > 65535 || dims->heads > 65535) return KDA_ERR_UNSUPPORTED;
-    if (B == 0) return KDA_OK;
-    int *status = kda::device_status_ptr();
-    if (!status) return KDA_ERR_CUDA;
-    auto s = static_cast<cudaStream_t>(stream);
-    const int D = dims->head_dim;
-    const int bytes = (2 * kda::kChunk * D + D) * static_cast<int>(sizeof(float));
-    dim3 grid(dims->heads, B);
-    if (D == 128) {
-        static std::atomic<unsigned long long> attr{0};
-        KDA_TRY(kda::smem_opt_in(kda::fold_kernel<128>, bytes, attr));
-        kda::fold_kernel<128><<<grid, 256, bytes, s>>>(k, cu_seqlens, accepted, tables, h_state, dims->heads,
-                                                       total_tokens, status);
-    } else {
-        static std::atomic<unsigned long long> attr{0};
-        KDA_TRY(kda::smem_opt_in(kda::fold_kernel<64>, bytes, attr));
-        kda::fold_kernel<64><<<grid, 256, bytes, s>>>(k, cu_seqlens, accepted, tables, h_state, dims->heads,
-                                                      total_tokens, status);
-    }
-    return kda::launch_status();
+    return kda::verify_fold(k, nullptr, static_cast<size_t>(dims->heads) * dims->head_dim, cu_seqlens, accepted, B,
+                            total_tokens, tables, h_state, dims, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

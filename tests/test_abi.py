@@ -83,7 +83,7 @@ def test_decode_alias_and_snapshot_checks(L):
     far = BOGUS + (1 << 20)
     common = [BOGUS, BOGUS, BOGUS, g_raw, BOGUS, BOGUS, BOGUS, BOGUS, far, BOGUS, BOGUS, None, None]
     assert L.kda_decode_k(*common, 0, None, None, 0, d, None) == 1          # K < 1
-    assert L.kda_decode_k(*common, 40, None, None, 0, d, None) == 4         # K > 32
+    assert L.kda_decode_k(*common, 40, None, None, 39, d, None) == 1       # K > 32 is taken; snapshots missing
     assert L.kda_decode_k(*common, 4, None, None, 2, d, None) == 1          # n_snap not 0 or K-1
     assert L.kda_decode_k(*common, 4, None, None, 3, d, None) == 1          # snapshots missing
     assert L.kda_recurrent_decode(*([BOGUS] * 7), -3, d, None) == 1
@@ -137,3 +137,39 @@ def test_binding_raises_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "libkda.so"))
     with pytest.raises(ImportError):
         kda.lib()
+
+
+def test_packed_block_argument_checks(L):
+    """The packed-sequence block calls, the batched verify and the fold refuse bad arguments
+    before any launch (no device memory is touched)."""
+    d = _d()
+    dp = ctypes.byref(d)
+    ws = ctypes.c_void_p()
+    assert L.kda_workspace_create_batched(dp, 256, 64, 128, 0, ctypes.byref(ws)) == 1       # max_seqs 0
+    assert L.kda_workspace_create_batched(dp, 256, 64, 0, 2, ctypes.byref(ws)) == 1         # max_tokens 0
+    assert L.kda_workspace_create_batched(dp, 200, 64, 128, 2, ctypes.byref(ws)) == 4       # hidden % 64
+    assert L.kda_workspace_max_seqs(None) == 0
+    assert L.kda_block_prefill_varlen(None, BOGUS, BOGUS, 2, 1, 100, BOGUS, BOGUS, None, None) == 1
+    assert L.kda_block_prefill_batched(None, BOGUS, 2, 50, BOGUS, BOGUS, None, None) == 1
+    assert L.kda_block_verify(None, BOGUS, BOGUS, 2, 10, BOGUS, BOGUS, BOGUS, 1 << 20, None, None) == 1
+    assert L.kda_block_verify_fold(BOGUS, BOGUS, 2, 10, BOGUS, BOGUS, BOGUS, None, None) == 1   # no workspace
+    assert L.kda_front_conv_silu_l2_varlen(BOGUS, BOGUS, BOGUS, BOGUS, None, 2, 10, 1, dp, None) == 1
+    assert L.kda_front_conv_silu_l2_varlen(BOGUS + 8, BOGUS, BOGUS, BOGUS, BOGUS, 2, 10, 1, dp, None) == 7
+    assert L.kda_front_conv_silu_l2_varlen(BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, 0, 0, 1, dp, None) == 0
+    assert L.kda_conv_state_fold(BOGUS, BOGUS, BOGUS, BOGUS, -1, 10, dp, None) == 1
+    assert L.kda_conv_state_fold(BOGUS, BOGUS, BOGUS, BOGUS, 0, 10, dp, None) == 0
+
+
+def test_packed_scratch_bounds(L):
+    """The compact chunk-slot layout: a head needs ceil(total / 64) + B - 1 pack slots, never more
+    than the one-slot-per-(sequence, chunk) layout asks for a long enough max_num_chunks."""
+    d = ctypes.byref(_d())
+    one = L.kda_chunk_prefill_scratch_bytes(1, 64, d)          # one chunk per head, plus the list
+    for seqs, total in [(1, 64), (1, 4096), (8, 4096), (64, 100), (3, 1)]:
+        slots = -(-total // 64) + seqs - 1
+        got = L.kda_chunk_prefill_packed_scratch_bytes(seqs, total, d)
+        assert got == L.kda_chunk_prefill_varlen_scratch_bytes(1, slots, d), (seqs, total)
+        assert got >= one
+    # a single sequence: the same bytes as the equal-length call of that length
+    assert L.kda_chunk_prefill_packed_scratch_bytes(1, 1000, d) == L.kda_chunk_prefill_scratch_bytes(1, 1000, d)
+    assert L.kda_chunk_prefill_packed_scratch_bytes(0, 10, d) == 0

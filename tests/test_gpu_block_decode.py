@@ -131,8 +131,11 @@ def test_block_decode_graph_replays_the_call(hidden, H, D, rank, N):
     ws_b.close()
 
 
-@pytest.mark.parametrize("hidden,H,D,rank,K,std", [(256, 2, 64, 64, 5, 0.05), (4096, 32, 128, 128, 4, 0.02)])
+@pytest.mark.parametrize("hidden,H,D,rank,K,std", [(256, 2, 64, 64, 5, 0.05), (4096, 32, 128, 128, 4, 0.02),
+                                                   (256, 2, 64, 64, 40, 0.05)])
 def test_block_decode_k_bit_identical_to_serial_block_decodes(hidden, H, D, rank, K, std):
+    """K rows in one call are the bits of K one-row calls; at K = 40 the projections and o_proj
+    run on groups of 32 and 8 rows and the stateful rows on launches of 31 and 9."""
     Wt = block_weights(hidden, H, D, rank, seed=11, std=std)
     h = block_hidden(K, hidden, seed=11).cuda()
     hs, cs = _states(1, H, D, seed=11)
@@ -178,8 +181,8 @@ def test_block_decode_argument_checks():
     h = torch.zeros((40, 256), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(kda.KdaError):  # more rows than the workspace holds
         kda.kda_block_decode(st, h, 5, kda.ptr_array([hs] * 5), kda.ptr_array([cs] * 5), ws)
-    with pytest.raises(kda.KdaError):  # K > 32
-        kda.kda_block_decode_k(st, h, 33, hs, cs, [], [], ws)
+    with pytest.raises(kda.KdaError):  # K > max_tokens
+        kda.kda_block_decode_k(st, h, 5, hs, cs, [], [], ws)
     ws.close()
 
 

@@ -80,10 +80,11 @@ def test_decode_fused_matches_oracle(N, H, D):
     assert np.array_equal(np64(torch.stack(cs)), r_cs)
 
 
-@pytest.mark.parametrize("K", [4, 32])
+@pytest.mark.parametrize("K", [4, 32, 33, 70])
 def test_decode_k_bit_identical_to_serial_decodes(K):
-    """K rows in one decode_k call (the largest K included: 31 snapshots) give the bits of K
-    serial one-row decodes."""
+    """K rows in one decode_k call give the bits of K serial one-row decodes, snapshots included:
+    32 rows fill one launch (31 snapshots); 33 and 70 rows run as chained launches of 31 rows
+    plus the rest, each group's last snapshot copied from the state it leaves."""
     H, D = 32, 128
     di = decode_inputs(1, H, D, seed=3, K=K)
     d = kda.dims(H, D)
@@ -167,3 +168,25 @@ def test_misaligned_state_pointer_is_skipped():
     o_ref, S_ref = oracle_prefill(ci)
     assert rel_l2(np64(o[0]), o_ref[0, 0]) <= TOL
     assert rel_l2(np64(good), S_ref[0]) <= TOL
+
+
+def test_decode_k_groups_without_snapshots():
+    """70 rows without snapshots (launches of 32, 32, 6 rows) equal 70 rows with snapshots
+    (launches of 31, 31, 8): the grouping never changes a bit."""
+    H, D, K = 4, 64, 70
+    di = decode_inputs(1, H, D, seed=9, K=K)
+    d = kda.dims(H, D)
+    dv = _dev(di)
+    res = []
+    for snaps in (False, True):
+        h_, c_ = di.s0[0].cuda().clone(), di.conv_state[0].cuda().clone()
+        out = torch.empty((K, H * D), dtype=torch.bfloat16, device="cuda")
+        core = torch.empty((K, H, D), device="cuda")
+        hsn = [torch.empty_like(h_) for _ in range(K - 1)] if snaps else []
+        csn = [torch.empty_like(c_) for _ in range(K - 1)] if snaps else []
+        kda.kda_decode_k(dv["x"], c_, dv["conv_w"], dv["g_raw"], dv["dt_bias"], dv["a_log"], dv["b_logit"], h_,
+                         dv["out_gate"], dv["o_norm"], out, None, core, K, hsn, csn, d)
+        torch.cuda.synchronize()
+        res.append((out, core, h_, c_))
+    for a_, b_ in zip(*res):
+        assert torch.equal(a_, b_)
