@@ -276,8 +276,10 @@ def main():
     # ---- the same workload in the fused-input mode (BF16 q|k|v rows + g_raw, gate in-kernel)
     fused = _fused_leg(kda, torch, dev, s, stream, flush, d, ci, Tp, hbm, tc_peak, scratch)
 
-    # ---- end-to-end leg: kda_chunk_prefill_host from pinned host buffers, copies timed
-    e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch)
+    # ---- end-to-end legs from pinned host buffers, copies timed: the headline call (FP32 I/O)
+    # and the serving layout (BF16 q|k|v rows)
+    e2e = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch, "f32")
+    e2e_bf16 = _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch, "bf16", seg=512)
 
     # ---- the full block (projections + front end + core + back end) and its dominant GEMM
     blk = None if args.no_block else _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm)
@@ -313,6 +315,7 @@ def main():
             "block_prefill": blk,
             "long_prefill": long_leg,
             "e2e": e2e,
+            "e2e_bf16_host": e2e_bf16,
             "cpu_baseline": cpu,
             "gpu_launches": launches,
             "clocks": clk.summary(),
@@ -558,29 +561,58 @@ def _block_stages(kda, torch, dev, s, stream, flush, Wt, hid, ws, Tb, hidden, Hh
     return {name: statistics.median(t) for name, t in times.items()}
 
 
-def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
-    """The same prefill through the public C ABI from pinned host buffers: kda_chunk_prefill_host
-    copies each step's inputs in and its outputs out, segment by segment (512 tokens), with the
-    copies of one segment overlapping the kernels of the next. The inputs travel as the serving
-    path holds them: the BF16 q|k|v rows (the front end's conv_out layout; the workload's inputs
-    are BF16-exact), the BF16 g_raw and the FP32 beta logits; the outputs are the FP32 core rows
-    and the final state."""
-    seg = 512
-    qkv = torch.cat([ci.q.reshape(T, H * D), ci.k.reshape(T, H * D), ci.v.reshape(T, H * D)], dim=-1)
-    host = {"qkv": qkv.to(torch.bfloat16).contiguous().pin_memory(),
-            "g_raw": ci.g_raw[0].contiguous().pin_memory(),
-            "b_logit": ci.b_logit[0].contiguous().pin_memory()}
-    s0 = ci.s0[0].clone()
-    state_h = s0.clone().pin_memory()
+def _pcie(torch, dev, stream, nbytes=256 << 20):
+    """Measured pinned-host <-> device copy bandwidth (GB/s), each direction alone: the floor
+    of an end-to-end call is its larger direction's bytes over these."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    g = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, fn in (("h2d_gbs", lambda: g.copy_(h, non_blocking=True)),
+                     ("d2h_gbs", lambda: h.copy_(g, non_blocking=True))):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(3):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out[name] = 3 * nbytes / (a.elapsed_time(b) * 1e-3) / 1e9
+    return out
+
+
+def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch, mode="f32", seg=1024):
+    """The headline prefill through the public C ABI from pinned host buffers, the copies inside
+    the timed region, segment by segment with the copies of one segment overlapping the kernels
+    of the next.
+    mode "f32": kda_chunk_prefill_host_f32, the same kernels and inputs as the timed step (FP32
+    q, k, v; BF16 g_raw; FP32 beta logits; kda_gate + kda_beta + kda_chunk_prefill).
+    mode "bf16": kda_chunk_prefill_host, the serving layout (BF16 q|k|v rows as the front end
+    writes them, the gate formed in the core). Both return the FP32 core rows and final state."""
+    pcie = _pcie(torch, dev, stream)
+    qf, kf, vf = (x[0].reshape(T, H * D).contiguous() for x in (ci.q, ci.k, ci.v))
+    if mode == "f32":
+        host = {"q": qf.pin_memory(), "k": kf.pin_memory(), "v": vf.pin_memory()}
+        nbytes = kda.kda_chunk_prefill_host_f32_bytes(T, seg, d)
+    else:
+        host = {"qkv": torch.cat([qf, kf, vf], dim=-1).to(torch.bfloat16).contiguous().pin_memory()}
+        nbytes = kda.kda_chunk_prefill_host_bytes(T, seg, d)
+    host["g_raw"] = ci.g_raw[0].contiguous().pin_memory()
+    host["b_logit"] = ci.b_logit[0].contiguous().pin_memory()
+    state_h = ci.s0[0].clone().pin_memory()
     core_h = torch.empty((T, H, D)).pin_memory()
     dt_bias, a_log = ci.dt_bias.to(dev), ci.a_log.to(dev)
-    buf = torch.empty(kda.kda_chunk_prefill_host_bytes(T, seg, d), dtype=torch.uint8, device=dev)
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host.values()) + state_h.numel() * 4
     d2h = core_h.numel() * 4 + state_h.numel() * 4
 
     def one():
-        kda.kda_chunk_prefill_host(host["qkv"], host["g_raw"], host["b_logit"], dt_bias, a_log, state_h, core_h, T,
-                                   seg, buf, d, s)
+        if mode == "f32":
+            kda.kda_chunk_prefill_host_f32(host["q"], host["k"], host["v"], host["g_raw"], host["b_logit"], dt_bias,
+                                           a_log, state_h, core_h, T, seg, buf, d, s)
+        else:
+            kda.kda_chunk_prefill_host(host["qkv"], host["g_raw"], host["b_logit"], dt_bias, a_log, state_h, core_h,
+                                       T, seg, buf, d, s)
 
     for _ in range(3):
         one()
@@ -598,10 +630,15 @@ def _e2e_leg(kda, torch, dev, s, stream, d, args, ci, Tp, world, scratch):
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = t.item()
+    ins = ("FP32 q, k, v, BF16 g_raw, FP32 beta logits and state in" if mode == "f32" else
+           "BF16 q|k|v rows, BF16 g_raw, FP32 beta logits and state in")
+    call = "kda_chunk_prefill_host_f32" if mode == "f32" else "kda_chunk_prefill_host"
     return {"value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "call": f"kda_chunk_prefill_host, {seg}-token segments (BF16 q|k|v rows, BF16 g_raw, FP32 beta logits "
-                    "and state in; FP32 core and state out; copies and kernels of consecutive segments overlapped)"}
+            "pcie_floor_ms": max(h2d / pcie["h2d_gbs"], d2h / pcie["d2h_gbs"]) / 1e6,
+            "pcie": pcie,
+            "call": f"{call}, {seg}-token segments ({ins}; FP32 core and state out; copies and kernels of "
+                    "consecutive segments overlapped)"}
 
 
 if __name__ == "__main__":

@@ -254,6 +254,22 @@ KDA_API int kda_chunk_prefill_host(const kda_bf16 *qkv, const kda_bf16 *g_raw, c
  * multiple of 64). */
 KDA_API size_t kda_chunk_prefill_host_bytes(int T, int segment_tokens, const kda_dims *dims);
 
+/* kda_chunk_prefill_host_f32 — the FP32-input form of kda_chunk_prefill_host: the device call it
+ * stands for is kda_gate + kda_beta + kda_chunk_prefill on FP32 q, k, v (the workload of the
+ * chunked-prefill benchmark), run segment by segment with the same three-stream overlap.
+ *   q, k, v  HOST [T, H*D] F32 each;  g_raw HOST [T, H*D] BF16 (the gate is formed by kda_gate);
+ *   b_logit, dt_bias, a_log, h_state, core, segment_tokens, stream: as kda_chunk_prefill_host
+ *   device_buffer   at least kda_chunk_prefill_host_f32_bytes(T, segment_tokens, dims) bytes
+ * core and the final state are the same bits as kda_gate + kda_beta + kda_chunk_prefill over all
+ * T rows on the device. Errors as kda_chunk_prefill_host. */
+KDA_API int kda_chunk_prefill_host_f32(const float *q, const float *k, const float *v, const kda_bf16 *g_raw,
+                                       const float *b_logit, const float *dt_bias, const float *a_log,
+                                       float *h_state, float *core, int T, int segment_tokens, void *device_buffer,
+                                       size_t device_bytes, const kda_dims *dims, void *stream);
+
+/* Device bytes kda_chunk_prefill_host_f32 needs (0 as kda_chunk_prefill_host_bytes). */
+KDA_API size_t kda_chunk_prefill_host_f32_bytes(int T, int segment_tokens, const kda_dims *dims);
+
 /* kda_chunk_prefill_noalloc — kda_chunk_prefill for callers that cannot allocate device
  * memory (the pages have no counterpart: this is a deployment variant). Some callers cannot
  * call cudaMalloc at all: an engine that hands all free HBM to its KV-cache / state pools at

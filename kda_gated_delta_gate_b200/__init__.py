@@ -67,6 +67,8 @@ _SIGS = {
     "kda_chunk_prefill_graw": ([_VP] * 9 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_host": ([_VP] * 7 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_host_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
+    "kda_chunk_prefill_host_f32": ([_VP] * 9 + [_I, _I, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
+    "kda_chunk_prefill_host_f32_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_prefill_varlen": ([_VP] * 6 + [_I, _I, _I, _VP, _VP, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
     "kda_chunk_prefill_varlen_scratch_bytes": ([_I, _I, _DIMS], ctypes.c_size_t),
     "kda_chunk_verify": ([_VP] * 6 + [_I, _I, _VP, _VP, _VP, ctypes.c_size_t, _VP, ctypes.c_size_t, _DIMS, _VP], _I),
@@ -251,6 +253,20 @@ def kda_chunk_prefill_host(qkv, g_raw, b_logit, dt_bias, a_log, h_state, core, T
     return _call("kda_chunk_prefill_host", _p(qkv), _p(g_raw), _p(b_logit), _p(dt_bias), _p(a_log), _p(h_state),
                  _p(core), T, segment_tokens, _p(device_buffer), device_buffer.numel() * device_buffer.element_size(),
                  ctypes.byref(d), _stream(stream))
+
+
+def kda_chunk_prefill_host_f32_bytes(T: int, segment_tokens: int, d: KdaDims) -> int:
+    return int(lib().kda_chunk_prefill_host_f32_bytes(T, segment_tokens, ctypes.byref(d)))
+
+
+def kda_chunk_prefill_host_f32(q, k, v, g_raw, b_logit, dt_bias, a_log, h_state, core, T: int, segment_tokens: int,
+                               device_buffer, d: KdaDims, stream=None):
+    """kda_gate + kda_beta + kda_chunk_prefill on HOST (pinned) FP32 q, k, v, BF16 g_raw, FP32
+    b_logit, h_state and core, copies and compute of consecutive segments overlapped.
+    `device_buffer`: a device tensor of kda_chunk_prefill_host_f32_bytes bytes."""
+    return _call("kda_chunk_prefill_host_f32", _p(q), _p(k), _p(v), _p(g_raw), _p(b_logit), _p(dt_bias), _p(a_log),
+                 _p(h_state), _p(core), T, segment_tokens, _p(device_buffer),
+                 device_buffer.numel() * device_buffer.element_size(), ctypes.byref(d), _stream(stream))
 
 
 def kda_chunk_prefill_noalloc(q, k, v, gate, beta, h_state_ptrs, core, B: int, T: int, d: KdaDims, stream=None):

@@ -264,6 +264,41 @@ def test_host_prefill_bit_identical_to_device_calls(T, H, D, seg):
         _check(ci, hc.reshape(1, T, H, D), hs.reshape(1, H, D, D), scale=0.7)
 
 
+@pytest.mark.parametrize("T,H,D,seg", [(4096, 32, 128, 1024), (1000, 4, 128, 256), (70, 2, 64, 512)])
+def test_host_f32_prefill_bit_identical_to_device_calls(T, H, D, seg):
+    """kda_chunk_prefill_host_f32 (pinned FP32 q, k, v, BF16 g_raw and FP32 beta logits in; core
+    and state out; segments overlapped) gives the bits of kda_gate + kda_beta +
+    kda_chunk_prefill over all T rows on the device, and matches the oracle."""
+    ci = core_inputs(1, T, H, D, seed=95 + T, bf16_inputs=False, s0_std=0.1)
+    Tp = t_pad(T)
+    d = kda.dims(H, D)
+    q, k, v = (x[0].reshape(T, H * D).contiguous() for x in (ci.q, ci.k, ci.v))
+    g_raw, b_logit = ci.g_raw[0].contiguous(), ci.b_logit[0].contiguous()
+    dt, al = ci.dt_bias.cuda(), ci.a_log.cuda()
+    # on the device, whole
+    dq, dk, dv = (pad_rows(x[None], Tp, 0.0).cuda() for x in (q, k, v))
+    gate = torch.zeros((Tp, H * D), device="cuda")
+    kda.kda_gate(pad_rows(g_raw[None], Tp, 0.0).cuda(), dt, al, gate, T, d)
+    beta = pad_rows(b_logit[None], Tp, 0.0).cuda()
+    kda.kda_beta(beta, beta, beta.numel())
+    st_dev = ci.s0[0].cuda().clone()
+    core_dev = torch.zeros((Tp, H, D), device="cuda")
+    kda.kda_chunk_prefill(dq, dk, dv, gate, beta, kda.ptr_array([st_dev]), core_dev, 1, T, d)
+    # from host buffers, segmented
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    hg, hb = g_raw.pin_memory(), b_logit.pin_memory()
+    hs = ci.s0[0].clone().pin_memory()
+    hc = torch.full((T, H, D), float("nan")).pin_memory()
+    buf = torch.empty(kda.kda_chunk_prefill_host_f32_bytes(T, seg, d), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream()
+    kda.kda_chunk_prefill_host_f32(hq, hk, hv, hg, hb, dt, al, hs, hc, T, seg, buf, d, s.cuda_stream)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(hc, core_dev[:T].cpu()) and torch.equal(hs, st_dev.cpu())
+    if T <= 1000:
+        _check(ci, hc.reshape(1, T, H, D), hs.reshape(1, H, D, D))
+
+
 def _varlen_case(lens, H, D, seed):
     """Packed sequences of the given lengths: q, k, v [total, H, D], gate and beta formed on the
     GPU from the packed g_raw / b_logit, per-sequence initial states, cu_seqlens on the device."""
