@@ -68,7 +68,29 @@ struct PrefillIn {
     const uint16_t *qkv, *g_raw;
     const float *dt_bias, *a_log, *beta;
     float *tables;  // verify mode: per (stream, head) U [64][D] then Gamma [64][D] (FP32); else null
+    int stream_pack;  // the call's operand packs overflow L2: store them evict-first
 };
+
+// L2 eviction policies (createpolicy): evict-first for data read or written for the last time
+// in this pass, so that the inputs prefetched for the coming items keep their place in L2.
+__device__ __forceinline__ uint64_t l2_policy(bool evict_first) {
+    uint64_t p;
+    if (evict_first) asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    else asm("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint4 ld16_hint(const void *p, uint64_t pol) {
+    uint4 r;
+    asm("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p), "l"(pol));
+    return r;
+}
+__device__ __forceinline__ void st16_hint(void *p, const uint4 &v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w), "l"(pol)
+                 : "memory");
+}
 
 // Input modes of the chunked kernels: where q, k, v and the log-decay come from.
 //   kInF32   FP32 q, k, v and FP32 gate (kda_gate's output)
@@ -85,18 +107,28 @@ __device__ __forceinline__ void bf16x2_to_f32(uint32_t u, float &lo, float &hi) 
 
 // Channels [c, c + 8) of global token row `row`, head h: q (part 0), k (1) or v (2), as FP32.
 template <int D, bool QKV16>
+// last: the kernel's last read of these values (loaded evict-first with policy `pol`).
 __device__ __forceinline__ void load8_in(const PrefillIn &in, int part, size_t row, int H, int h, int c,
-                                         float (&x)[8]) {
+                                         float (&x)[8], bool last = false, uint64_t pol = 0) {
     if constexpr (QKV16) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(in.qkv + row * (3 * static_cast<size_t>(H) * D) +
-                                                         static_cast<size_t>(part * H + h) * D + c);
+        const uint16_t *p = in.qkv + row * (3 * static_cast<size_t>(H) * D) + static_cast<size_t>(part * H + h) * D + c;
+        const uint4 u = last ? ld16_hint(p, pol) : *reinterpret_cast<const uint4 *>(p);
         bf16x2_to_f32(u.x, x[0], x[1]); bf16x2_to_f32(u.y, x[2], x[3]);
         bf16x2_to_f32(u.z, x[4], x[5]); bf16x2_to_f32(u.w, x[6], x[7]);
     } else {
         const float *p = (part == 0 ? in.q : (part == 1 ? in.k : in.v)) + row * (static_cast<size_t>(H) * D) +
                          static_cast<size_t>(h) * D + c;
-        const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+        uint4 a, b;
+        if (last) {
+            a = ld16_hint(p, pol);
+            b = ld16_hint(p + 4, pol);
+        } else {
+            a = *reinterpret_cast<const uint4 *>(p);
+            b = *reinterpret_cast<const uint4 *>(p + 4);
+        }
+        x[0] = __uint_as_float(a.x); x[1] = __uint_as_float(a.y); x[2] = __uint_as_float(a.z);
+        x[3] = __uint_as_float(a.w); x[4] = __uint_as_float(b.x); x[5] = __uint_as_float(b.y);
+        x[6] = __uint_as_float(b.z); x[7] = __uint_as_float(b.w);
     }
 }
 
@@ -590,8 +622,9 @@ intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *_
 // Two 256-thread CTAs share an SM (113 KB of shared memory and 256 TMEM columns each), so one
 // CTA's MMA, barrier and load latencies run under the other's CUDA-core work. The L/M operands
 // are built and contracted 64 channels at a time through one 72 KB buffer; q, k and v come
-// straight from global memory (each item's rows are bulk-prefetched into L2 one item ahead);
-// W and U~ leave TMEM straight for the pack.
+// straight from global memory, read evict-first where an item reads them for the last time (an
+// L2 prefetch of the next item's rows measured slower: it competes with the current item's
+// misses); W and U~ leave TMEM straight for the pack.
 
 constexpr float kRefBound = 80.0f;  // e^80 and e^-80 are comfortably inside BF16/FP32 range
 constexpr int kTcThreads = 256;
@@ -627,36 +660,28 @@ __device__ __forceinline__ void ld8f(const float *p, float (&x)[8]) {
 }
 
 // 16 BF16 hi + lo bytes of 8 values at `off` of a split tile in global memory (hi at dst, lo at dst + half)
-__device__ __forceinline__ void st_pair_g(uint8_t *dst, int half_bytes, uint32_t off, const float (&x)[8]) {
+__device__ __forceinline__ void st_pair_g(uint8_t *dst, int half_bytes, uint32_t off, const float (&x)[8],
+                                          uint64_t pol) {
     uint4 hi, lo;
     split8(x, hi, lo);
-    *reinterpret_cast<uint4 *>(dst + off) = hi;
-    *reinterpret_cast<uint4 *>(dst + half_bytes + off) = lo;
-}
-
-// One thread: prefetch the box at (x, y, z) of a 3-D tensor map into L2 (no shared memory).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *tm, int x, int y, int z) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tm)),
-                 "r"(x), "r"(y), "r"(z)
-                 : "memory");
+    st16_hint(dst + off, hi, pol);
+    st16_hint(dst + half_bytes + off, lo, pol);
 }
 
 // One thread: bulk shared -> global copy (bytes a multiple of 16), in this thread's bulk group.
-__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
-                 "r"(bytes)
+__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(gdst),
+                 "r"(smem_u32(smem_src)), "r"(bytes), "l"(pol)
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Maps over the rows of the chunked path's inputs (3-D: columns, row in stream, stream): the g box
-// of an item is loaded from tmG; every input's box of the next item is prefetched into L2 through
-// tmG, tmQ, tmK, tmV (in the fused-input mode tmQ = tmK = tmV map the q|k|v rows).
+// The map over the rows of the log-decay input (3-D: columns, row in stream, stream): the g box
+// (FP32 gate, or BF16 g_raw) of an item is loaded through it.
 struct InMaps {
-    CUtensorMap g, q, k, v;
+    CUtensorMap g;
 };
 
 template <int D, int MODE>
@@ -686,6 +711,7 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nch = sq.nch;
     const int total = B * H * nch;
+    const uint64_t pol_first = l2_policy(true), pol_pack = l2_policy(in.stream_pack != 0);
     constexpr uint32_t kGBox = C * D * (GRAW ? 2 : 4);
     // g's box: FP32 g at the start of R2, or BF16 g_raw in its upper half (the gate is then
     // formed in place, FP32, dense)
@@ -715,23 +741,6 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
         if (sq.cu) { y = static_cast<int>(row0); z = 0; }
         else { y = ch * C; z = b; }
     };
-    // an item's q, k, v and g boxes into L2 (thread 0, one tensor prefetch each)
-    auto prefetch = [&](int it) {
-        if (tid != 0) return;
-        const int ch = it % nch, h = (it / nch) % H, b = it / (nch * H);
-        int n, y, z;
-        size_t row0;
-        seq_chunk(sq, b, ch, row0, n, nullptr);
-        box_yz(ch, b, row0, y, z);
-        tma_prefetch_3d(&maps.g, h * D, y, z);
-        if constexpr (QKV16) {
-            for (int part = 0; part < 3; ++part) tma_prefetch_3d(&maps.q, (part * H + h) * D, y, z);
-        } else {
-            tma_prefetch_3d(&maps.q, h * D, y, z);
-            tma_prefetch_3d(&maps.k, h * D, y, z);
-            tma_prefetch_3d(&maps.v, h * D, y, z);
-        }
-    };
     // an item's g box into R2 (thread 0; the caller made R2 free) and its beta (threads < C)
     float bnext = 0.f;
     auto fetch_g = [&](int it) {
@@ -751,10 +760,7 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
     __syncthreads();  // barriers initialised, TMEM allocated
     tc_fence_after();
     const int first = next_item(blockIdx.x);
-    if (first < total) {
-        prefetch(first);
-        fetch_g(first);
-    }
+    if (first < total) fetch_g(first);
     const uint32_t tmem = *tmem_slot;
     bool dead = false;   // a wait timed out: hand every remaining item to the CUDA-core body
     uint32_t iter = 0;   // items started by this CTA: the parity of the g box
@@ -784,7 +790,6 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
             if (tid == 0) list[1 + atomicAdd(list, 1)] = item;
             continue;
         }
-        if (following < total) prefetch(following);
         bool ok = mbar_wait(gbar, iter & 1, kWaitCycles);
         if (tid < C) sB[tid] = bnext;
         if (tid == 0) bulk_wait_read();  // the previous item's staged results have left R1
@@ -874,7 +879,7 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
                 float k8[8], q8[8], gi[8], gm[8], ef[8], ei[8], x[8];
                 if (i < n) {
                     load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, k8);
-                    load8_in<D, QKV16>(in, 0, row0 + i, H, h, cb, q8);
+                    load8_in<D, QKV16>(in, 0, row0 + i, H, h, cb, q8, true, pol_first);
                 } else {
 #pragma unroll
                     for (int w = 0; w < 8; ++w) { k8[w] = 0.f; q8[w] = 0.f; }
@@ -915,11 +920,11 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
                 ld8f(sTab + a * D + cb, em);
 #pragma unroll
                 for (int w = 0; w < 8; ++w) x[w] = q8[w] * (ef[w] * em[w]);
-                st_pair_g(pack + PK::OFF_A1, PK::A1 / 2, kmaj_off(64 + i, cb, 128), x);
+                st_pair_g(pack + PK::OFF_A1, PK::A1 / 2, kmaj_off(64 + i, cb, 128), x, pol_pack);
                 ld8f(sTab + (4 + a) * D + cb, em);
 #pragma unroll
                 for (int w = 0; w < 8; ++w) x[w] = k8[w] * (ei[w] * em[w]);
-                st_pair_g(pack + PK::OFF_A3, PK::A3 / 2, mnmaj_off(cb, i, C), x);
+                st_pair_g(pack + PK::OFF_A3, PK::A3 / 2, mnmaj_off(cb, i, C), x, pol_pack);
             }
             fence_async_smem();
             tc_fence_before();
@@ -984,13 +989,13 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
                     } else {
 #pragma unroll
                         for (int w = 0; w < 8; ++w) x[w] = j0 + w <= i ? x[w] : 0.f;
-                        st_pair_g(pack + PK::OFF_AM, PK::AM / 2, kmaj_off(i, j0, 64), x);
+                        st_pair_g(pack + PK::OFF_AM, PK::AM / 2, kmaj_off(i, j0, 64), x, pol_pack);
                     }
                 }
             }
             if (!is_l) {
                 const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                for (int jc = seg / 8 + part; jc < 8; jc += 2) st_pair_g(pack + PK::OFF_AM, PK::AM / 2, kmaj_off(i, 8 * jc, 64), z);
+                for (int jc = seg / 8 + part; jc < 8; jc += 2) st_pair_g(pack + PK::OFF_AM, PK::AM / 2, kmaj_off(i, 8 * jc, 64), z, pol_pack);
             }
         }
         tc_fence_before();
@@ -1016,8 +1021,8 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
             const int u = tid + NT * j, i = u / (D / 8), cb = 8 * (u % (D / 8));
             float k8[8], gi[8], x[8];
             if (i < n) {
-                load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, k8);
-                load8_in<D, QKV16>(in, 2, row0 + i, H, h, cb, vv[j]);
+                load8_in<D, QKV16>(in, 1, row0 + i, H, h, cb, k8, true, pol_first);
+                load8_in<D, QKV16>(in, 2, row0 + i, H, h, cb, vv[j], true, pol_first);
             } else {
 #pragma unroll
                 for (int w = 0; w < 8; ++w) { k8[w] = 0.f; vv[j][w] = 0.f; }
@@ -1100,10 +1105,10 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
             if (tid == 0) {
 #pragma unroll
                 for (int p = 0; p < D / 64; ++p) {
-                    bulk_store(pack + PK::OFF_A1 + p * 16384, sWs + p * 8192, 8192);
-                    bulk_store(pack + PK::OFF_A1 + PK::A1 / 2 + p * 16384, sWs + I::W_STAGE / 2 + p * 8192, 8192);
+                    bulk_store(pack + PK::OFF_A1 + p * 16384, sWs + p * 8192, 8192, pol_pack);
+                    bulk_store(pack + PK::OFF_A1 + PK::A1 / 2 + p * 16384, sWs + I::W_STAGE / 2 + p * 8192, 8192, pol_pack);
                 }
-                bulk_store(pack + PK::OFF_UT, sUs, PK::UT);
+                bulk_store(pack + PK::OFF_UT, sUs, PK::UT, pol_pack);
                 bulk_commit();
             }
         }
@@ -1222,14 +1227,28 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         bulk_copy_nx(sA2 + 8192, pk + PK::OFF_AM, PK::AM / 2, &bars[1]);
         bulk_copy_nx(sA2 + kTileBytes + 8192, pk + PK::OFF_AM + PK::AM / 2, PK::AM / 2, &bars[1]);
     };
+    // A1 ([W; Q o A], hi then lo) in k-parts of 64 channels: a part is one 64-channel atom column
+    // of the hi half and of the lo half, so group 1 can start on part 0 while part 1 lands, and
+    // part 0 of the next chunk can come in once the MMAs of part 0 have completed
+    constexpr int kA1Parts = D / 64, kA1Part = PK::A1 / 2 / kA1Parts;
+    auto copy_a1 = [&](const uint8_t *pk, int part) {  // part 0 completes on bars[0], part 1 on bars[11]
+        uint64_t *bar = part ? &bars[11] : &bars[0];
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                     "r"(static_cast<uint32_t>(2 * kA1Part))
+                     : "memory");
+        bulk_copy_nx(sA1 + part * kA1Part, pk + PK::OFF_A1 + part * kA1Part, kA1Part, bar);
+        bulk_copy_nx(sA1 + PK::A1 / 2 + part * kA1Part, pk + PK::OFF_A1 + PK::A1 / 2 + part * kA1Part, kA1Part, bar);
+    };
     if (ctl) {
         for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
         mbar_init(&bars[8], kEpiWarps);  // one arrival per epilogue warp
         mbar_init(&bars[9], kEpiWarps);
         mbar_init(&bars[10], 1);
+        mbar_init(&bars[11], 1);
+        mbar_init(&bars[12], 1);
         *fail = 0;
         fence_mbar_init();
-        bulk_copy(sA1, packs + PK::OFF_A1, PK::A1, &bars[0]);
+        for (int part = 0; part < kA1Parts; ++part) copy_a1(packs, part);
         copy_m(packs);
         bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[2]);
     }
@@ -1298,11 +1317,12 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             }
             mma_commit(&bars[6]);
         };
-        // copy barriers this thread issues on: copies issued and phases waited for (so that a
-        // timed-out thread can drain what is still in flight)
-        uint32_t issued[3] = {1, 1, 1}, waited[3] = {0, 0, 0};
+        // copy barriers this thread issues on (A1 part 0, M, A3, A1 part 1): copies issued and
+        // phases waited for (so that a timed-out thread can drain what is still in flight)
+        constexpr int kCopyBar[4] = {0, 1, 2, 11};
+        uint32_t issued[4] = {1, 1, 1, kA1Parts > 1 ? 1u : 0u}, waited[4] = {0, 0, 0, 0};
         auto wait_copy = [&](int k) {
-            const bool r = mbar_wait(&bars[k], waited[k] & 1, kWaitCycles);
+            const bool r = mbar_wait(&bars[kCopyBar[k]], waited[k] & 1, kWaitCycles);
             if (r) ++waited[k];
             return r;
         };
@@ -1315,8 +1335,6 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             const uint64_t dB1h = mnmaj_desc(smem_u32(sB1), D, 0, 0), dB1l = mnmaj_desc(smem_u32(sB1) + S::B1 / 2, D, 0, 0);
             const uint64_t dA3h = mnmaj_desc(smem_u32(sA3), C, 0, 0), dA3l = mnmaj_desc(smem_u32(sA3) + PK::A3 / 2, C, 0, 0);
             if (S::NU == 2) issued[1] = 0;  // the output thread owns the M copies
-            if (nb > 1) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(packs + PK::bytes),
-                                     "r"(static_cast<uint32_t>(PK::bytes)) : "memory");
 #pragma unroll 1
             for (int ch = 0; ch < nb && ok; ++ch) {
                 const uint32_t par = ch & 1;
@@ -1326,32 +1344,41 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 const bool more = ch + 1 < nb;
                 // S of this chunk is in B1 (the epilogue's previous round), A1 has landed
                 if (ch > 0 && !mbar_wait(&bars[9], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
-                if (!wait_copy(0)) { give_up(); break; }
-                tc_fence_after();
                 {
                     constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
+                    bool got = true;
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint64_t ah = dA1h + kmaj_step(128, ks), al = dA1l + kmaj_step(128, ks);
-                        const uint64_t bh = dB1h + mnmaj_step(ks), bl = dB1l + mnmaj_step(ks);
-                        mma_bf16(tD1, ah, bh, id, ks > 0 ? 1u : 0u);
-                        mma_bf16(tD1, ah, bl, id, 1);
-                        mma_bf16(tD1, al, bh, id, 1);
+                    for (int part = 0; part < kA1Parts; ++part) {
+                        if (!wait_copy(part ? 3 : 0)) { got = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const int ks = 4 * part + kk;
+                            const uint64_t ah = dA1h + kmaj_step(128, ks), al = dA1l + kmaj_step(128, ks);
+                            const uint64_t bh = dB1h + mnmaj_step(ks), bl = dB1l + mnmaj_step(ks);
+                            mma_bf16(tD1, ah, bh, id, ks > 0 ? 1u : 0u);
+                            mma_bf16(tD1, ah, bl, id, 1);
+                            mma_bf16(tD1, al, bh, id, 1);
+                        }
+                        if (part + 1 < kA1Parts) mma_commit(&bars[12]);  // part 0 has been read
                     }
+                    if (!got) { give_up(); break; }
                     mma_commit(&bars[4]);
                 }
-                if (ch + 2 < nb)  // the pack two chunks ahead into L2
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(cur + 2 * PK::bytes),
-                                 "r"(static_cast<uint32_t>(PK::bytes)) : "memory");
                 if (S::NU == 1 && ch > 0) {  // the previous output group has read M: this chunk's M
                     if (!mbar_wait(&bars[6], (ch - 1) & 1, kWaitCycles)) { give_up(); break; }
                     copy_m(cur);
                     ++issued[1];
                 }
-                if (!mbar_wait(&bars[4], par, kWaitCycles)) { give_up(); break; }
-                if (more) {  // A1 is free again
-                    bulk_copy(sA1, next + PK::OFF_A1, PK::A1, &bars[0]);
+                if (kA1Parts > 1 && more) {  // A1 part 0 is free again
+                    if (!mbar_wait(&bars[12], par, kWaitCycles)) { give_up(); break; }
+                    copy_a1(next, 0);
                     ++issued[0];
+                }
+                if (!mbar_wait(&bars[4], par, kWaitCycles)) { give_up(); break; }
+                if (more) {  // the rest of A1 is free again
+                    copy_a1(next, kA1Parts - 1);
+                    ++issued[kA1Parts > 1 ? 3 : 0];
                 }
                 // U is in B2
                 if (!mbar_wait(&bars[8], par, kWaitCycles)) { give_up(); break; }
@@ -1384,12 +1411,12 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
                 // drain (bounded): every MMA issued, then every copy still in flight
                 mma_commit(&bars[7]);
                 mbar_wait(&bars[7], 0, kWaitCycles);
-                for (int k = 0; k < 3; ++k)
+                for (int k = 0; k < 4; ++k)
                     while (waited[k] < issued[k] && wait_copy(k)) {
                     }
             }
         } else if (ctl2 && S::NU == 2) {
-            issued[0] = issued[2] = 0;  // the chain thread owns the A1 and A3 copies
+            issued[0] = issued[2] = issued[3] = 0;  // the chain thread owns the A1 and A3 copies
 #pragma unroll 1
             for (int ch = 0; ch < nb && ok; ++ch) {
                 // group 2 of this chunk has completed: its output group runs while epilogue 2 does
@@ -1558,6 +1585,13 @@ long long pack_count(int B, int H, const Seqs &sq) {
     return static_cast<long long>(H) * (sq.slots ? sq.slots : static_cast<long long>(B) * sq.nch);
 }
 
+int sm_count() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
 template <int D, int DVS, int MODE>
 int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, int H, float scale,
               void *scratch, cudaStream_t s) {
@@ -1571,12 +1605,7 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     uint8_t *sc = static_cast<uint8_t *>(scratch);
     int *list = reinterpret_cast<int *>(sc + packs_bytes<D>(pack_count(B, H, sq)));
     if (cudaMemsetAsync(list, 0, sizeof(int), s) != cudaSuccess) return KDA_ERR_CUDA;
-    int sms = 148;
-    {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = sm_count();
     const long long items = static_cast<long long>(B) * H * nch;
     if (items > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;  // item ids are int
     // two tensor-core intra CTAs per SM; the CUDA-core fix-up runs one per SM
@@ -1589,16 +1618,11 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
         KDA_TRY(make_rows_map(&maps.g, in.g_raw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H * D, mT, mTp, mB, D, C));
     else
         KDA_TRY(make_rows_map(&maps.g, in.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-    if (kQkv16<MODE>) {
-        KDA_TRY(make_rows_map(&maps.q, in.qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3 * H * D, mT, mTp, mB, D, C));
-        maps.k = maps.q;
-        maps.v = maps.q;
-    } else {
-        KDA_TRY(make_rows_map(&maps.q, in.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-        KDA_TRY(make_rows_map(&maps.k, in.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-        KDA_TRY(make_rows_map(&maps.v, in.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H * D, mT, mTp, mB, D, C));
-    }
-    intra_tc_kernel<D, MODE><<<grid, kTcThreads, IntraTC<D>::bytes, s>>>(maps, in, sc, list, B, sq, H, status);
+    // packs that overflow half of L2 go out evict-first: they are read back only by the state
+    // pass, and the inputs prefetched for the coming items need the room
+    PrefillIn inp = in;
+    inp.stream_pack = packs_bytes<D>(pack_count(B, H, sq)) > (size_t{64} << 20) ? 1 : 0;
+    intra_tc_kernel<D, MODE><<<grid, kTcThreads, IntraTC<D>::bytes, s>>>(maps, inp, sc, list, B, sq, H, status);
     KDA_TRY(launch_status());
     intra_fix_kernel<D, MODE><<<grid_fix, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
@@ -1607,7 +1631,11 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     return launch_status();
 }
 
-// Value slice width: enough CTAs to cover the SMs (one state CTA per SM fits in shared memory).
+// Value slice width. One state CTA fills an SM and walks its (stream, head)'s chunks in order,
+// so the pass takes (waves of CTAs) x (chunks) x (one chunk's chain). Measured chains: about
+// 4.9 K cycles per chunk with 32 value columns, 6 K with 64 and 13.5 K with 128 (the MMAs cost
+// the same up to N = 64, and the epilogues grow with the columns). So 32 columns while four
+// slices per unit fit on the SMs in one wave, else 64: two 64-column waves beat one of 128.
 template <int MODE>
 int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, const kda_dims *dims,
                void *scratch, cudaStream_t s) {
@@ -1615,9 +1643,8 @@ int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, c
     const float sc = dims->scale;
     if (dims->head_dim == 64) return launch_tc<64, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
     const long long units = static_cast<long long>(B) * H;
-    if (units >= 100) return launch_tc<128, 128, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
-    if (units >= 50) return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
-    return launch_tc<128, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    if (4 * units <= sm_count()) return launch_tc<128, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
 }
 
 Seqs equal_seqs(int T) {
