@@ -797,47 +797,54 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
             give_up(gbar, iter & 1, item);
             continue;
         }
-        // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, range of tokens)
+        // ---- Gamma: inclusive cumulative sum over tokens, thread (channel, range of TPQ tokens).
+        //      The range lives in registers: one pass of loads, the prefix sum, the other ranges'
+        //      totals added, the reference-bound check, one pass of stores.
         bool safe = true;
         {
             constexpr int QT = NT / D;  // 2 (D=128) or 4 (D=64) token ranges
             constexpr int TPQ = C / QT;
-            const int c = tid % D, qr = tid / D;
+            const int c = tid % D, qr = tid / D, i0 = qr * TPQ;
+            float gv[TPQ];
             if constexpr (GRAW) {
                 // g = -exp(a_log) softplus(g_raw + dt_bias) (0 past the chunk's end), FP32 over g_raw's box
                 const uint16_t *gr = reinterpret_cast<const uint16_t *>(gdst);
-                float x[TPQ];
 #pragma unroll
-                for (int r = 0; r < TPQ; ++r) x[r] = bf16_to_f32(gr[(qr * TPQ + r) * D + c]);
+                for (int r = 0; r < TPQ; ++r) gv[r] = bf16_to_f32(gr[(i0 + r) * D + c]);
                 const float nea = -expf(in.a_log[h]), dtb = in.dt_bias[static_cast<size_t>(h) * D + c];
-                __syncthreads();
 #pragma unroll
-                for (int r = 0; r < TPQ; ++r) {
-                    const int i = qr * TPQ + r;
-                    sG[i * D + c] = i < n ? kda_gate_f32(x[r], dtb, nea) : 0.f;
-                }
+                for (int r = 0; r < TPQ; ++r) gv[r] = i0 + r < n ? kda_gate_f32(gv[r], dtb, nea) : 0.f;
+            } else {
+#pragma unroll
+                for (int r = 0; r < TPQ; ++r) gv[r] = i0 + r < n ? sG[(i0 + r) * D + c] : 0.f;  // rows past the end decay nothing
             }
             float acc = 0.f;
-            for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) {
-                acc += i < n ? sG[i * D + c] : 0.f;  // rows past the chunk's end decay nothing
-                sG[i * D + c] = acc;
+#pragma unroll
+            for (int r = 0; r < TPQ; ++r) {
+                acc += gv[r];
+                gv[r] = acc;
             }
             sTmp[qr * D + c] = acc;
-            __syncthreads();
+            __syncthreads();  // every range's total is in sTmp; g_raw's box has been read
             float pre = 0.f;
             for (int r = 0; r < qr; ++r) pre += sTmp[r * D + c];
-            if (qr > 0)
-                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) sG[i * D + c] += pre;
+#pragma unroll
+            for (int r = 0; r < TPQ; ++r) {
+                gv[r] += pre;
+                sG[(i0 + r) * D + c] = gv[r];
+            }
             if (in.tables) {  // verify mode: keep Gamma for the fold
                 float *gt = in.tables + ((static_cast<size_t>(b) * H + h) * 2 + 1) * C * D;
-                for (int i = qr * TPQ; i < (qr + 1) * TPQ; ++i) gt[i * D + c] = sG[i * D + c];
+#pragma unroll
+                for (int r = 0; r < TPQ; ++r) gt[(i0 + r) * D + c] = gv[r];
             }
             // the reference bound of the 16-token blocks in this thread's range: every factor
             // e^{+-(Gamma_i - Gamma_m)} of the L/M operands stays within e^{kRefBound}
-            for (int a = qr * TPQ / 16; a < (qr + 1) * TPQ / 16; ++a) {
-                const float gm = sG[(16 * a + 7) * D + c];
-#pragma unroll 4
-                for (int i = 16 * a; i < 16 * a + 16; ++i) safe = safe && fabsf(sG[i * D + c] - gm) <= kRefBound;
+#pragma unroll
+            for (int a = 0; a < TPQ / 16; ++a) {
+                const float gm = gv[16 * a + 7];
+#pragma unroll
+                for (int r = 16 * a; r < 16 * a + 16; ++r) safe = safe && fabsf(gv[r] - gm) <= kRefBound;
             }
             safe = __syncthreads_and(safe) != 0;
         }
