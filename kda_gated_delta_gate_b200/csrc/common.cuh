@@ -151,7 +151,7 @@ struct GemvSeg {
     const uint16_t *x;  // this segment's input rows (same row stride), or null: the call's x
 };
 struct GemvSegs {
-    GemvSeg s[3];
+    GemvSeg s[6];
     int count, total;
 };
 int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,

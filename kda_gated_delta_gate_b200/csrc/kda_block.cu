@@ -73,8 +73,8 @@ int proj(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *C, int ld
 
 // Projections of M rows of `hidden` into the workspace rows [r0, r0 + M): qkv_proj (q|k|v
 // packed), g_raw, b_logit (FP32, in the BETA buffer), out_gate. For the matrix-vector path the
-// weights that read the same rows share a launch: [q | k | v], [f_a | g_a | b_proj], then f_b
-// and g_b.
+// weights that read the hidden rows share one launch ([q | k | v | f_a | g_a | b_proj]), then
+// f_b and g_b share another.
 int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M, kda_workspace *ws, cudaStream_t s,
                       int r0 = 0) {
     const kda_dims *d = &ws->dims;
@@ -87,20 +87,18 @@ int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M,
     float *blog = f32(KDA_BUF_BETA) + o * H;
     hidden += o * Hd;
     if (M <= kRowsGemv) {
+        // every weight that reads the hidden rows: q, k, v, then the small f_a, g_a, b_proj
+        // products ride in the tail of the same launch
         GemvSegs a{};
         a.s[0] = GemvSeg{w->q_proj, qkv_p, qkv, Hd, cd, 0};
         a.s[1] = GemvSeg{w->k_proj, qkv_p + qkv, qkv, Hd, cd, 0};
         a.s[2] = GemvSeg{w->v_proj, qkv_p + 2 * qkv, qkv, Hd, cd, 0};
-        a.count = 3;
-        a.total = 3 * qkv;
+        a.s[3] = GemvSeg{w->f_a, fa, R, Hd, R, 0};
+        a.s[4] = GemvSeg{w->g_a, ga, R, Hd, R, 0};
+        a.s[5] = GemvSeg{w->b_proj, blog, H, Hd, H, 1};
+        a.count = 6;
+        a.total = 3 * qkv + 2 * R + H;
         KDA_TRY(gemv_segs(hidden, Hd, a, M, Hd, s));
-        GemvSegs b{};
-        b.s[0] = GemvSeg{w->f_a, fa, R, Hd, R, 0};
-        b.s[1] = GemvSeg{w->g_a, ga, R, Hd, R, 0};
-        b.s[2] = GemvSeg{w->b_proj, blog, H, Hd, H, 1};
-        b.count = 3;
-        b.total = 2 * R + H;
-        KDA_TRY(gemv_segs(hidden, Hd, b, M, Hd, s));
         // f_b and g_b read different rows (f_a_out, g_a_out) with one width: one launch
         GemvSegs c{};
         c.s[0] = GemvSeg{w->f_b, graw, qkv, R, qkv, 0, fa};
