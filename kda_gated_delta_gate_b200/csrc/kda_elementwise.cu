@@ -4,6 +4,8 @@
 //   kda_back_gated_rmsnorm (Glm5NextKdaWorkspace, field `o_norm_out`; Glm5NextKdaWeights `o_norm`)
 // Each thread moves 16-byte vectors; grids are sized in multiples of the SM count and
 // walk the tensor with a grid-stride loop.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace kda {
@@ -25,27 +27,42 @@ int grid_for(long long work_items, int threads) {
 
 // 8 gate values per thread: one 16-byte BF16 load of g_raw, two float4 of dt_bias, two
 // float4 stores. groups = n_rows * H*D / 8; hd8 = H*D/8; d8 = D/8 (all 8 in one head).
+// Thread (x) owns one 8-channel group of the H*D columns and walks rows (y): its dt_bias and
+// -exp(a_log) are loaded once; each row is one 16-byte load and two 16-byte stores, four rows'
+// loads in flight at a time.
 __global__ void __launch_bounds__(256) gate_kernel(const uint4 *__restrict__ g_raw,
                                                    const float4 *__restrict__ dt_bias,
                                                    const float *__restrict__ a_log,
-                                                   float4 *__restrict__ gate, long long groups,
-                                                   int hd8, int d8) {
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < groups;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int c8 = static_cast<int>(i % hd8);
-        const float nea = -expf(__ldg(a_log + c8 / d8));
-        const uint4 raw = g_raw[i];
-        const float4 b0 = __ldg(dt_bias + 2 * c8), b1 = __ldg(dt_bias + 2 * c8 + 1);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        float g[8];
+                                                   float4 *__restrict__ gate, int rows, int hd8, int d8) {
+    const int c8 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c8 >= hd8) return;
+    const float nea = -expf(__ldg(a_log + c8 / d8));
+    const float4 b0 = __ldg(dt_bias + 2 * c8), b1 = __ldg(dt_bias + 2 * c8 + 1);
+    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    // kRows rows per step, their loads issued together (bytes in flight, not issue, bound this)
+    constexpr int kRows = 4;
+    for (int r0 = blockIdx.y; r0 < rows; r0 += kRows * gridDim.y) {
+        uint4 raw[kRows];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint16_t bits = static_cast<uint16_t>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu));
-            g[e] = kda_gate_f32(bf16_to_f32(bits), bb[e], nea);
+        for (int q = 0; q < kRows; ++q) {
+            const int r = r0 + q * gridDim.y;
+            raw[q] = r < rows ? g_raw[static_cast<size_t>(r) * hd8 + c8] : make_uint4(0u, 0u, 0u, 0u);
         }
-        gate[2 * i] = make_float4(g[0], g[1], g[2], g[3]);
-        gate[2 * i + 1] = make_float4(g[4], g[5], g[6], g[7]);
+#pragma unroll
+        for (int q = 0; q < kRows; ++q) {
+            const int r = r0 + q * gridDim.y;
+            if (r >= rows) break;
+            const size_t i = static_cast<size_t>(r) * hd8 + c8;
+            const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+            float g[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint16_t bits = static_cast<uint16_t>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu));
+                g[e] = kda_gate_f32(bf16_to_f32(bits), bb[e], nea);
+            }
+            gate[2 * i] = make_float4(g[0], g[1], g[2], g[3]);
+            gate[2 * i + 1] = make_float4(g[4], g[5], g[6], g[7]);
+        }
     }
 }
 
@@ -112,11 +129,13 @@ int kda_gate(const kda_bf16 *g_raw, const float *dt_bias, const float *a_log, fl
     if (!g_raw || !dt_bias || !a_log || !gate || n_rows < 0) return KDA_ERR_INVALID_ARG;
     if (!kda::aligned16(g_raw) || !kda::aligned16(dt_bias) || !kda::aligned16(gate)) return KDA_ERR_MISALIGNED;
     if (n_rows == 0) return KDA_OK;
-    const int hd = dims->heads * dims->head_dim;
-    const long long groups = static_cast<long long>(n_rows) * hd / 8;
-    kda::gate_kernel<<<kda::grid_for(groups, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    const int hd8 = dims->heads * dims->head_dim / 8;
+    const int gx = (hd8 + 255) / 256;
+    // one wave of 256-thread blocks (8 per SM), each walking rows four at a time
+    const int gy = static_cast<int>(std::min<long long>((n_rows + 3) / 4, std::max(1, 8 * kda::num_sms() / gx)));
+    kda::gate_kernel<<<dim3(gx, gy), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const uint4 *>(g_raw), reinterpret_cast<const float4 *>(dt_bias), a_log,
-        reinterpret_cast<float4 *>(gate), groups, hd / 8, dims->head_dim / 8);
+        reinterpret_cast<float4 *>(gate), n_rows, hd8, dims->head_dim / 8);
     return kda::launch_status();
 }
 

@@ -50,6 +50,28 @@ def test_gate_and_beta_match_oracle():
     np.testing.assert_allclose(np64(beta), oracle.sigmoid(ci.b_logit[0].reshape(-1)), rtol=1e-6)
 
 
+def test_gate_softplus_sweep_against_fp64():
+    """The kernels' softplus (SFU exponential, atanh series below y = 1/8, SFU logarithm above)
+    over x in [-40, 40] on a fine grid, x = g_raw + dt_bias with g_raw in {0, +-1/8} and a_log = 0,
+    so that g = -softplus(x): relative error within 2e-6 + 1.2e-7 |x| of the FP64 oracle
+    everywhere, both branches and the switch between them included. The |x| term is the FP32
+    rounding of x itself (and of the exponential's scaled argument): for x << 0 softplus is
+    about e^x, whose relative error is the absolute error of x. It changes e^g by less than
+    one FP32 step."""
+    H, D, T = 32, 128, 3
+    d = kda.dims(H, D)
+    dt = torch.linspace(-40.0, 40.0, H * D, dtype=torch.float64).float()
+    g_raw = torch.tensor([0.0, 0.125, -0.125]).repeat_interleave(H * D).reshape(T, H * D).to(torch.bfloat16)
+    a_log = torch.zeros(H)
+    gate = torch.empty((T, H, D), device="cuda")
+    kda.kda_gate(g_raw.cuda(), dt.cuda(), a_log.cuda(), gate, T, d)
+    torch.cuda.synchronize()
+    ref = oracle.gate(g_raw.float(), dt, a_log, H, D).reshape(T, H * D)
+    x = np64(g_raw) + np64(dt)[None, :]
+    rel = np.abs(np64(gate).reshape(T, H * D) - ref) / np.abs(ref)
+    assert np.all(rel <= 2e-6 + 1.2e-7 * np.abs(x)), float(np.max(rel / (2e-6 + 1.2e-7 * np.abs(x))))
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_prefill_small_config(impl):
     """B=1, T=64, H=2, D=64, zero initial state, FP32 inputs (the CPU-checkable workload)."""
