@@ -27,6 +27,11 @@ __device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
     x[4] = __uint_as_float(u.z << 16); x[5] = __uint_as_float(u.z & 0xFFFF0000u);
     x[6] = __uint_as_float(u.w << 16); x[7] = __uint_as_float(u.w & 0xFFFF0000u);
 }
+// SiLU y / (1 + e^-y) from the SFU exponential and the fast divide (a few ulp of FP32; the
+// result is rounded to BF16 next). For y << 0 the denominator overflows to inf and the result
+// is -0, as the exact value rounds.
+__device__ __forceinline__ float silu_fast(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
+
 __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) {
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kFrontThreads, 3) front_kernel(const uint16_t 
             y = fmaf(w[1][e], xm[1][e], y);
             y = fmaf(w[2][e], xm[2][e], y);
             y = fmaf(w[3][e], xc[e], y);
-            y = y * sigmoid_f32(y);
+            y = silu_fast(y);
             c[e] = bf16_to_f32(f32_to_bf16(y));  // conv_out before the in-place L2
             ss = fmaf(c[e], c[e], ss);
             xm[0][e] = xm[1][e]; xm[1][e] = xm[2][e]; xm[2][e] = xc[e];
@@ -266,7 +271,7 @@ front_varlen_kernel(const uint16_t *__restrict__ x, uint16_t *const *__restrict_
             y = fmaf(w[1][e], xm[1][e], y);
             y = fmaf(w[2][e], xm[2][e], y);
             y = fmaf(w[3][e], xc[e], y);
-            y = y * sigmoid_f32(y);
+            y = silu_fast(y);
             c[e] = bf16_to_f32(f32_to_bf16(y));
             ss = fmaf(c[e], c[e], ss);
             xm[0][e] = xm[1][e]; xm[1][e] = xm[2][e]; xm[2][e] = xc[e];
