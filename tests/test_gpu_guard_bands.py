@@ -206,3 +206,105 @@ def test_host_prefill_writes_only_its_outputs():
     torch.cuda.synchronize()
     assert hs.margins_intact() and hc.margins_intact() and buf.margins_intact()
     assert torch.all(torch.isfinite(hc.t))
+
+
+def test_packed_scratch_is_enough_for_the_compact_layout():
+    """Packed sequences whose chunks start mid-chunk everywhere, with scratch sized exactly by
+    kda_chunk_prefill_packed_scratch_bytes (ceil(total/64) + B - 1 pack slots per head): the
+    compact layout stays inside it, and the results are the bits of the one-slot-per-chunk
+    layout (a larger scratch)."""
+    lens, H, D = [63, 1, 65, 130, 2], 2, 128
+    total, nb = sum(lens), len(lens)
+    ci, d, q, k, v, _, gate, beta = _prefill_inputs(1, total, H, D, seed=12)
+    q, k, v, gate, beta = (x[:total].contiguous() for x in (q, k, v, gate, beta))
+    cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32, device="cuda")
+    s0 = torch.randn((nb, H, D, D), generator=torch.Generator().manual_seed(12)) * 0.1
+    out = []
+    for sb in (kda.kda_chunk_prefill_packed_scratch_bytes(nb, total, d), _varlen_scratch_bytes(nb, 3, d)):
+        core = Guarded((total, H, D), torch.float32)
+        states = [Guarded((H, D, D), torch.float32) for _ in range(nb)]
+        for b in range(nb):
+            states[b].t.copy_(s0[b])
+        scratch = Guarded((sb,), torch.uint8)
+        kda.kda_chunk_prefill_varlen(q, k, v, gate, beta, cu, nb, 3, total, kda.ptr_array([s.t for s in states]),
+                                     core.t, d, scratch=scratch.t)
+        torch.cuda.synchronize()
+        assert core.margins_intact() and scratch.margins_intact() and all(s.margins_intact() for s in states)
+        out.append((core.t.clone(), [s.t.clone() for s in states]))
+    (c0, s0_), (c1, s1_) = out
+    assert torch.equal(c0, c1) and all(torch.equal(a, b) for a, b in zip(s0_, s1_))
+    assert (kda.kda_chunk_prefill_packed_scratch_bytes(nb, total, d) < _varlen_scratch_bytes(nb, 3, d))
+
+
+def test_packed_front_end_and_conv_fold_write_only_their_outputs():
+    """kda_front_conv_silu_l2_varlen (reading and advancing B conv states) and kda_conv_state_fold
+    keep to conv_out and the states; sequences start inside 16-token tiles, one is empty."""
+    H, D = 2, 64
+    lens = [5, 0, 30, 1, 19]
+    total, nb, cd = sum(lens), len(lens), 3 * H * D
+    g = torch.Generator().manual_seed(13)
+    x = (torch.randn((total, cd), generator=g)).to(torch.bfloat16).cuda()
+    cw = (torch.randn((cd, 4), generator=g) * 0.5).to(torch.bfloat16).cuda()
+    cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32, device="cuda")
+    states = [Guarded((cd, 3), torch.bfloat16) for _ in range(nb)]
+    for s in states:
+        s.t.copy_(torch.randn((cd, 3), generator=g).to(torch.bfloat16))
+    out = Guarded((total, cd), torch.bfloat16)
+    d = kda.dims(H, D)
+    kda.kda_front_conv_silu_l2_varlen(x, kda.ptr_array([s.t for s in states]), cw, out.t, cu, nb, total, True, d)
+    acc = torch.tensor([3, 0, 30, 1, 0], dtype=torch.int32, device="cuda")
+    kda.kda_conv_state_fold(x, kda.ptr_array([s.t for s in states]), cu, acc, nb, total, d)
+    torch.cuda.synchronize()
+    assert out.margins_intact() and all(s.margins_intact() for s in states)
+
+
+def test_host_f32_prefill_writes_only_its_outputs():
+    T, H, D, seg = 200, 2, 128, 128
+    ci = core_inputs(1, T, H, D, seed=14, s0_std=0.1)
+    d = kda.dims(H, D)
+    hq, hk, hv = (x[0].reshape(T, H * D).contiguous().pin_memory() for x in (ci.q, ci.k, ci.v))
+    hg, hb = ci.g_raw[0].contiguous().pin_memory(), ci.b_logit[0].contiguous().pin_memory()
+    hs = Guarded((H, D, D), torch.float32, pin=True)
+    hs.t.copy_(ci.s0[0])
+    hc = Guarded((T, H, D), torch.float32, pin=True)
+    buf = Guarded((kda.kda_chunk_prefill_host_f32_bytes(T, seg, d),), torch.uint8)
+    s = torch.cuda.current_stream()
+    kda.kda_chunk_prefill_host_f32(hq, hk, hv, hg, hb, ci.dt_bias.cuda(), ci.a_log.cuda(), hs.t, hc.t, T, seg, buf.t,
+                                   d, s.cuda_stream)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert hs.margins_intact() and hc.margins_intact() and buf.margins_intact()
+    assert torch.all(torch.isfinite(hc.t))
+
+
+def test_block_verify_and_fold_write_only_their_outputs():
+    """kda_block_verify reads the guarded recurrent and conv states and leaves them as they were;
+    kda_block_verify_fold writes only inside them; the tables stay inside their allocation."""
+    from synth import block_hidden, block_weights
+    from tests.test_gpu_block import _device_weights
+    hidden, H, D, rank, lens, acc = 256, 2, 64, 64, [7, 64, 1], [7, 10, 0]
+    total, nb = sum(lens), len(lens)
+    Wt = block_weights(hidden, H, D, rank, seed=15, std=0.05)
+    h = block_hidden(total, hidden, seed=15).cuda()
+    d = kda.dims(H, D)
+    ws = kda.Workspace(d, hidden, rank, max_tokens=total, max_seqs=nb)
+    g = torch.Generator().manual_seed(15)
+    hs = [Guarded((H, D, D), torch.float32) for _ in range(nb)]
+    cs = [Guarded((3 * H * D, 3), torch.bfloat16) for _ in range(nb)]
+    for a, c in zip(hs, cs):
+        a.t.copy_(torch.randn((H, D, D), generator=g) * 0.1)
+        c.t.copy_(torch.randn((3 * H * D, 3), generator=g).to(torch.bfloat16))
+    before = [(a.t.clone(), c.t.clone()) for a, c in zip(hs, cs)]
+    tables = Guarded((kda.kda_chunk_verify_tables_bytes(nb, d) // 4,), torch.float32)
+    cu = torch.tensor([0, 7, 71, 72], dtype=torch.int32, device="cuda")
+    dw = _device_weights(Wt)
+    st = kda.block_weights_struct(dw)
+    hp, cp = kda.ptr_array([a.t for a in hs]), kda.ptr_array([c.t for c in cs])
+    kda.kda_block_verify(st, h, cu, nb, total, hp, cp, tables.t, ws)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a.t, b0) and torch.equal(c.t, b1) for (a, c), (b0, b1) in zip(zip(hs, cs), before))
+    kda.kda_block_verify_fold(cu, torch.tensor(acc, dtype=torch.int32, device="cuda"), nb, total, tables.t, hp, cp, ws)
+    torch.cuda.synchronize()
+    assert tables.margins_intact() and all(a.margins_intact() and c.margins_intact() for a, c in zip(hs, cs))
+    assert torch.equal(hs[2].t, before[2][0]) and torch.equal(cs[2].t, before[2][1])  # accepted 0
+    ws.close()
