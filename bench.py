@@ -422,6 +422,33 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
                         "gbs": (wbytes + n_b * sbytes) / (msn * 1e-3) / 1e9,
                         "frac_hbm": (wbytes + n_b * sbytes) / (msn * 1e-3) / 1e9 / hbm},
            "weights_bytes": wbytes, "state_bytes_per_seq": sbytes}
+    # packed sequences through one block call, the same 8192 rows: 8 x 1024 (batched) and a ragged mix (varlen)
+    ws2 = kda.Workspace(kda.dims(Hh, Dd), hidden, rank, max_tokens=Tb, max_seqs=64)
+    lens = [3000, 2000, 1500, 1000, 500, 192]
+    cu = torch.tensor([0] + [sum(lens[:i + 1]) for i in range(len(lens))], dtype=torch.int32, device=dev)
+    p8h, p8c = kda.ptr_array(list(hs_b[:8]), device=dev), kda.ptr_array(list(cs_b[:8]), device=dev)
+    msb = timed(lambda: kda.kda_block_prefill_batched(st, hid, 8, Tb // 8, p8h, p8c, ws2, s))
+    msv = timed(lambda: kda.kda_block_prefill_varlen(st, hid, cu, len(lens), (max(lens) + 63) // 64, Tb, p8h, p8c,
+                                                     ws2, s))
+    # batched speculative verify + accepted-row fold: N sequences x 4 draft rows, states left in place by the
+    # verify (the fold then advances them)
+    ver = {}
+    for n_v in (8, 64):
+        rows = 4 * n_v
+        cu_v = torch.arange(0, rows + 1, 4, dtype=torch.int32, device=dev)
+        acc_v = torch.full((n_v,), 2, dtype=torch.int32, device=dev)
+        tabs = torch.empty(kda.kda_chunk_verify_tables_bytes(n_v, kda.dims(Hh, Dd)) // 4, device=dev)
+        pvh, pvc = kda.ptr_array(list(hs_b[:n_v]), device=dev), kda.ptr_array(list(cs_b[:n_v]), device=dev)
+        msv1 = timed(lambda: kda.kda_block_verify(st, hid[:rows], cu_v, n_v, rows, pvh, pvc, tabs, ws2, s))
+        msf = timed(lambda: (kda.kda_block_verify(st, hid[:rows], cu_v, n_v, rows, pvh, pvc, tabs, ws2, s),
+                             kda.kda_block_verify_fold(cu_v, acc_v, n_v, rows, tabs, pvh, pvc, ws2, s)))
+        ver[f"n{n_v}_k4"] = {"verify_ms": msv1, "verify_and_fold_ms": msf, "draft_rows_per_s": rows / (msv1 * 1e-3),
+                             "call": "kda_block_verify (+ kda_block_verify_fold, 2 rows accepted per sequence)"}
+        del tabs
+    ws2.close()
+    packed = {"batched_8x1024": {"ms": msb, "tokens_per_s": Tb / (msb * 1e-3), "call": "kda_block_prefill_batched"},
+              "varlen_ragged": {"ms": msv, "tokens_per_s": Tb / (msv * 1e-3), "lens": lens,
+                                "call": "kda_block_prefill_varlen"}}
     del hs_b, cs_b
     ws.close()
     return {"workload": "kda_block_prefill hidden 4096 H32 D128 rank 128 T8192 (9 GEMMs + conv + gate + core + o_norm)",
@@ -430,7 +457,7 @@ def _block_leg(kda, torch, dev, s, stream, flush, tc_peak, hbm):
             "stages_ms": stages,
             "gemm": {"shape": "8192x4096x4096 bf16->bf16", "ms": gms, "tflops": gflop / (gms * 1e-3) / 1e12,
                      "peak": tc_peak, "frac": gflop / (gms * 1e-3) / 1e12 / tc_peak},
-            "block_decode": dec}
+            "block_decode": dec, "packed_prefill": packed, "verify": ver}
 
 
 def _fused_leg(kda, torch, dev, s, stream, flush, d, ci, Tp, hbm, tc_peak, scratch):

@@ -577,8 +577,8 @@ KDA_API int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidde
  *   cu_seqlens  DEVICE int32 [B + 1];  h_state, conv_state: DEVICE pointer arrays as
  *               kda_block_prefill_varlen (read only here)
  * Each row's output equals what kda_block_prefill_varlen on that sequence's first rows gives
- * for it (the same core arithmetic), up to the projection kernel: up to 32 rows in all the
- * matrix-vector kernel, beyond that the GEMM. The workspace keeps the rows' qkv_proj and
+ * for it (the same core arithmetic), up to the projection kernel: up to 8 rows in all the
+ * matrix-vector kernel, up to 256 the small-M tensor-core form, beyond that the GEMM. The workspace keeps the rows' qkv_proj and
  * conv_out for the fold. KDA_ERR_CAPACITY if total_tokens > max_tokens or B > max_seqs. */
 KDA_API int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const int *cu_seqlens, int B,
                              int total_tokens, float *const *h_state, kda_bf16 *const *conv_state, float *tables,

@@ -176,6 +176,16 @@ struct GemvSegs {
 };
 int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
               int out_f32, cudaStream_t s);
+// A few input rows (at most 256) against up to six weights in one launch, each weight read
+// once: y[m][n] = x[m] . W[n] for m < rows, n < N (rows of y at stride ldy), on the tensor
+// cores with the weights' rows as the 128-row tiles. Not the matrix-vector kernel's bits.
+struct GemmTSeg {
+    const uint16_t *W;  // [N, K], row stride ldw
+    const uint16_t *x;  // [rows, K], row stride ldx
+    void *y;
+    int N, ldw, ldx, ldy, out_f32;
+};
+int gemm_bf16_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s);
 int gemv_bf16(const uint16_t *x, int ldx, const uint16_t *W, int ldw, void *y, int ldy, int M, int N, int K,
               int out_f32, cudaStream_t s);
 int gemv_segs(const uint16_t *x, int ldx, const GemvSegs &segs, int M, int K, cudaStream_t s);

@@ -24,11 +24,14 @@
 // Block decode (Glm5NextKdaLayer `decode`, `decode_k`): the same projections for the call's
 // rows (N sequences x 1 token, or K rows of one sequence), each weight read once for all
 // rows, then the fused stateful rows (kda_decode_fused / kda_decode_k: conv + SiLU + L2, gate,
-// beta, recurrence, gated RMSNorm) and o_proj. Up to kRowsGemv rows the projections run the
-// batched-M matrix-vector kernel (kda_gemv_bf16), whose every output's arithmetic is fixed
-// by K and its own row: a row's projections are the same bits in a call of K rows and in a
-// call of one, which the decode_k identity needs. Larger batches (N independent sequences,
-// no such identity) run the tcgen05 GEMM.
+// beta, recurrence, gated RMSNorm) and o_proj. decode_k's projections run the batched-M
+// matrix-vector kernel (kda_gemv_bf16) on groups of up to 32 rows: its every output's
+// arithmetic is fixed by K and its own row, so a row's projections are the same bits in a call
+// of K rows and in a call of one, which the decode_k identity needs. Calls without that
+// identity (N independent sequences, the batched verify) take the matrix-vector kernel up to 8
+// rows (one pass over the weights), the small-M tensor-core form up to 256 rows (the weights'
+// output rows as the 128-row tiles, so each weight is read once by many CTAs), and the GEMM
+// beyond.
 #include <algorithm>
 #include <cstring>
 #include <new>
@@ -61,14 +64,29 @@ struct kda_workspace {
 
 namespace kda {
 namespace {
-constexpr int kRowsGemv = 32;
+constexpr int kRowsGemv = 32;   // exact calls: the matrix-vector kernel up to this many rows
+constexpr int kRowsGemvFree = 8; // other calls: the matrix-vector kernel up to one row group
+constexpr int kRowsSmallM = 256; // then the small-M tensor-core form, then the GEMM
 
-// One projection of M decode rows: the batched-M matrix-vector kernel for up to kRowsGemv rows,
-// the tensor-core GEMM beyond.
+// Which kernel takes M rows. `exact`: every row must get the bits it gets alone (decode_k's
+// identity with serial one-row decodes), which only the matrix-vector kernel gives.
+enum class ProjKind { Gemv, SmallM, Gemm };
+ProjKind proj_kind(int M, bool exact) {
+    if (M <= (exact ? kRowsGemv : kRowsGemvFree)) return ProjKind::Gemv;
+    return M <= kRowsSmallM ? ProjKind::SmallM : ProjKind::Gemm;
+}
+
+// One projection of M rows.
 int proj(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *C, int ldc, int M, int N, int K, int out_f32,
-         cudaStream_t s) {
-    if (M <= kRowsGemv) return gemv_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
-    return gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
+         cudaStream_t s, bool exact) {
+    switch (proj_kind(M, exact)) {
+    case ProjKind::Gemv: return gemv_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
+    case ProjKind::SmallM: {
+        const GemmTSeg t{W, A, C, N, ldw, lda, ldc, out_f32};
+        return gemm_bf16_small_m(&t, 1, M, K, s);
+    }
+    default: return gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
+    }
 }
 
 // Projections of M rows of `hidden` into the workspace rows [r0, r0 + M): qkv_proj (q|k|v
@@ -76,7 +94,7 @@ int proj(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *C, int ld
 // weights that read the hidden rows share one launch ([q | k | v | f_a | g_a | b_proj]), then
 // f_b and g_b share another.
 int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M, kda_workspace *ws, cudaStream_t s,
-                      int r0 = 0) {
+                      bool exact, int r0 = 0) {
     const kda_dims *d = &ws->dims;
     const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
     const size_t o = static_cast<size_t>(r0);
@@ -86,7 +104,19 @@ int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M,
     uint16_t *graw = bf(KDA_BUF_G_RAW) + o * qkv, *og = bf(KDA_BUF_OUT_GATE) + o * qkv;
     float *blog = f32(KDA_BUF_BETA) + o * H;
     hidden += o * Hd;
-    if (M <= kRowsGemv) {
+    const ProjKind kind = proj_kind(M, exact);
+    if (kind == ProjKind::SmallM) {  // two launches, each weight read once by many CTAs
+        const GemmTSeg a[6] = {{w->q_proj, hidden, qkv_p, qkv, Hd, Hd, cd, 0},
+                               {w->k_proj, hidden, qkv_p + qkv, qkv, Hd, Hd, cd, 0},
+                               {w->v_proj, hidden, qkv_p + 2 * qkv, qkv, Hd, Hd, cd, 0},
+                               {w->f_a, hidden, fa, R, Hd, Hd, R, 0},
+                               {w->g_a, hidden, ga, R, Hd, Hd, R, 0},
+                               {w->b_proj, hidden, blog, H, Hd, Hd, H, 1}};
+        KDA_TRY(gemm_bf16_small_m(a, 6, M, Hd, s));
+        const GemmTSeg c[2] = {{w->f_b, fa, graw, qkv, R, R, qkv, 0}, {w->g_b, ga, og, qkv, R, R, qkv, 0}};
+        return gemm_bf16_small_m(c, 2, M, R, s);
+    }
+    if (kind == ProjKind::Gemv) {
         // every weight that reads the hidden rows: q, k, v, then the small f_a, g_a, b_proj
         // products ride in the tail of the same launch
         GemvSegs a{};
@@ -316,13 +346,13 @@ int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, 
     const int qkv = d->heads * d->head_dim;
     auto bf = [&](int i) { return static_cast<kda_bf16 *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
-    KDA_TRY(kda::block_projections(w, hidden, N, ws, s));
+    KDA_TRY(kda::block_projections(w, hidden, N, ws, s, false));
     KDA_TRY(kda_decode_fused(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                              f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                              bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), N, d, stream));
     if (!w->o_proj) return KDA_OK;  // the caller applies its own o_proj (a tensor-parallel slice)
     return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, N, ws->hidden, qkv,
-                     0, s);
+                     0, s, false);
 }
 
 int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K, float *h_state,
@@ -339,7 +369,7 @@ int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K
     // projections and o_proj in groups of at most kRowsGemv rows: the matrix-vector kernel gives
     // each row the bits it gets alone, which the identity with serial decodes needs
     for (int r0 = 0; r0 < K; r0 += kda::kRowsGemv)
-        KDA_TRY(kda::block_projections(w, hidden, std::min(kda::kRowsGemv, K - r0), ws, s, r0));
+        KDA_TRY(kda::block_projections(w, hidden, std::min(kda::kRowsGemv, K - r0), ws, s, true, r0));
     KDA_TRY(kda_decode_k(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias, w->a_log,
                          f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm, bf(KDA_BUF_O_NORM_OUT),
                          bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), K, h_snap, conv_snap, n_snap, d, stream));
@@ -347,7 +377,7 @@ int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K
     for (int r0 = 0; r0 < K; r0 += kda::kRowsGemv) {
         const size_t o = static_cast<size_t>(r0);
         KDA_TRY(kda::proj(bf(KDA_BUF_O_NORM_OUT) + o * qkv, qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT) + o * Hd, Hd,
-                          std::min(kda::kRowsGemv, K - r0), Hd, qkv, 0, s));
+                          std::min(kda::kRowsGemv, K - r0), Hd, qkv, 0, s, true));
     }
     return KDA_OK;
 }
@@ -369,7 +399,7 @@ int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const i
     auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
     // every weight read once for all draft rows of all sequences
-    KDA_TRY(kda::block_projections(w, hidden, total_tokens, ws, s));
+    KDA_TRY(kda::block_projections(w, hidden, total_tokens, ws, s, false));
     KDA_TRY(kda::front_varlen(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), cu_seqlens, B,
                               total_tokens, d, s));
     KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), total_tokens * d->heads, stream));
@@ -380,7 +410,7 @@ int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const i
                                    total_tokens, d, stream));
     if (!w->o_proj) return KDA_OK;
     return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, total_tokens,
-                     ws->hidden, qkv, 0, s);
+                     ws->hidden, qkv, 0, s, false);
 }
 
 int kda_block_verify_fold(const int *cu_seqlens, const int *accepted, int B, int total_tokens, const float *tables,

@@ -14,6 +14,8 @@
 // lanes and reduce the per-token sum of squares with shuffles. The tile-0 block of each
 // column block is the only reader of those channels' carried conv state and, after its
 // reads, the only writer of the new one (the last three inputs).
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace kda {
@@ -224,14 +226,14 @@ template <int D>
 __global__ void __launch_bounds__(kFrontThreads, 2)
 front_varlen_kernel(const uint16_t *__restrict__ x, uint16_t *const *__restrict__ conv_state,
                     const uint16_t *__restrict__ conv_w, uint16_t *__restrict__ conv_out, const int *__restrict__ cu,
-                    int B, int total, int H, float eps, int *__restrict__ status) {
+                    int B, int total, int tt, int H, float eps, int *__restrict__ status) {
     constexpr int LG = D / 8;
     const int qkv = H * D, cd = 3 * qkv;
     const int g = blockIdx.y * kFrontThreads + threadIdx.x;
     const bool valid = 8 * g < cd;
     const int c0 = valid ? 8 * g : 0;
     const int part = c0 / qkv;
-    const int t0 = blockIdx.x * kTT, tend = min(t0 + kTT, total);
+    const int t0 = blockIdx.x * tt, tend = min(t0 + tt, total);
     float w[4][8];
     {
         float wr[32];
@@ -336,13 +338,16 @@ int front_varlen(const uint16_t *x, uint16_t *const *conv_state, const uint16_t 
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
     const int cd = 3 * dims->heads * dims->head_dim;
-    dim3 grid((total + kTT - 1) / kTT, (cd / 8 + kFrontThreads - 1) / kFrontThreads);
+    const int colb = (cd / 8 + kFrontThreads - 1) / kFrontThreads;
+    // token tiles of up to 16 rows, shorter when the call has too few rows for two blocks per SM
+    const int tt = std::max(1, std::min(kTT, total / std::max(1, 2 * num_sms() / colb)));
+    dim3 grid((total + tt - 1) / tt, colb);
     if (dims->head_dim == 128)
         front_varlen_kernel<128><<<grid, kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, cu_seqlens, B, total,
-                                                                dims->heads, dims->l2_eps, status);
+                                                                tt, dims->heads, dims->l2_eps, status);
     else
         front_varlen_kernel<64><<<grid, kFrontThreads, 0, s>>>(x, conv_state, conv_w, conv_out, cu_seqlens, B, total,
-                                                               dims->heads, dims->l2_eps, status);
+                                                               tt, dims->heads, dims->l2_eps, status);
     return launch_status();
 }
 

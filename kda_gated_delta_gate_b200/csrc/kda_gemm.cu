@@ -4,8 +4,8 @@
 // the packed q|k|v rows of Glm5NextKdaWorkspace `qkv_proj`).
 //
 // Persistent, warp-specialised kernel (192 threads, one CTA per SM):
-//   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 W tiles, 128-byte swizzle, 4-stage
-//               ring of shared-memory buffers (full / empty mbarriers). No multicast.
+//   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 W tiles, 128-byte swizzle, a ring of
+//               4 to 10 shared-memory stages by tile width (full / empty mbarriers). No multicast.
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128, N = BN, K = 16) into
 //               one of two accumulators and commits to the stage's `empty` barrier.
 //   warps 2..5  epilogue: tcgen05.ld the accumulator rows (TMEM lanes = rows), convert, store;
@@ -23,7 +23,7 @@ namespace {
 
 using namespace umma;
 
-constexpr int BM = 128, BK = 64, STAGES = 4, kGemmThreads = 192;
+constexpr int BM = 128, BK = 64, kGemmThreads = 192;
 constexpr long long kGemmWait = 4000000000LL;
 
 template <int BN>
@@ -31,7 +31,11 @@ struct GemmCfg {
     static constexpr int A_STAGE = BM * BK * 2;
     static constexpr int B_STAGE = BN * BK * 2;
     static constexpr int STAGE = A_STAGE + B_STAGE;
+    // as many stages as about 200 KB holds: narrow tiles (the small-M form, few CTAs) then keep
+    // as many bytes in flight per SM as wide ones
+    static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 8 : 10));
     static constexpr int OFF_BARS = STAGES * STAGE;
+    static_assert(OFF_BARS + 256 + 1024 <= 232448, "shared memory");
     static constexpr int bytes = OFF_BARS + 256 + 1024;
     static constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
 };
@@ -59,26 +63,58 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     return true;
 }
 
+// Up to three products in one launch, each its own A (M rows) and W (the shared N rows), its own
+// output: a segment's tiles follow the previous segment's in the tile order. trans: element
+// (m, n) of a product is stored at C[n ldc + m] (the small-M form below computes C^T).
+constexpr int kMaxGemmSegs = 6;
+struct GemmSeg {
+    void *C;
+    int ldc, M, out_f32, vec;
+};
+struct GemmArgs {
+    CUtensorMap tmA[kMaxGemmSegs];
+    CUtensorMap tmW[kMaxGemmSegs];
+    GemmSeg seg[kMaxGemmSegs];
+    int nseg, N, K, trans;
+};
+
+// The segment and the tile origin of tile `t`.
+template <int BN>
+__device__ __forceinline__ int gemm_tile(const GemmArgs &g, int tiles_n, int t, int &m0, int &n0) {
+    int s = 0;
+    for (;;) {
+        const int nt = (g.seg[s].M + BM - 1) / BM * tiles_n;
+        if (t < nt || s + 1 == g.nseg) break;
+        t -= nt;
+        ++s;
+    }
+    m0 = (t / tiles_n) * BM;
+    n0 = (t % tiles_n) * BN;
+    return s;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, void *__restrict__ Cout,
-            int ldc, int M, int N, int K, int out_f32, int vec, int *__restrict__ status) {
+gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
+    const int N = g.N, K = g.K;
     using G = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + G::OFF_BARS);
-    uint64_t *empty = full + STAGES;
-    uint64_t *accf = empty + STAGES;
+    uint64_t *empty = full + G::STAGES;
+    uint64_t *accf = empty + G::STAGES;
     uint64_t *acce = accf + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN, ntiles = tiles_m * tiles_n;
+    const int tiles_n = (N + BN - 1) / BN;
+    int ntiles = 0;
+    for (int i = 0; i < g.nseg; ++i) ntiles += (g.seg[i].M + BM - 1) / BM * tiles_n;
     const int nk = K / BK;
 
     if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < G::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 4); }
         *abort = 0;
         fence_mbar_init();
@@ -96,15 +132,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (lane == 0) {  // ---- TMA producer
             int it = 0;
             for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-                const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+                int m0, n0;
+                const int sg = gemm_tile<BN>(g, tiles_n, tile, m0, n0);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
+                    const int s = it % G::STAGES;
+                    const uint32_t ph = (it / G::STAGES) & 1;
                     if (!wait_or_abort(&empty[s], ph ^ 1, abort, status)) goto done;
                     uint8_t *sa = sm + s * G::STAGE;
                     mbar_expect_tx(&full[s], G::STAGE);
-                    tma_load_2d(sa, &tmA, kb * BK, m0, &full[s]);
-                    tma_load_2d(sa + G::A_STAGE, &tmW, kb * BK, n0, &full[s]);
+                    tma_load_2d(sa, &g.tmA[sg], kb * BK, m0, &full[s]);
+                    tma_load_2d(sa + G::A_STAGE, &g.tmW[sg], kb * BK, n0, &full[s]);
                 }
             }
         }
@@ -119,8 +156,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 tc_fence_after();
                 const uint32_t dcol = tmem + acc * BN;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
+                    const int s = it % G::STAGES;
+                    const uint32_t ph = (it / G::STAGES) & 1;
                     if (!wait_or_abort(&full[s], ph, abort, status)) goto done;
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sm + s * G::STAGE), b0 = a0 + G::A_STAGE;
@@ -137,7 +174,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const int quad = warp & 3;
         int tc = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
-            const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+            int m0, n0;
+            const GemmSeg &sgm = g.seg[gemm_tile<BN>(g, tiles_n, tile, m0, n0)];
+            void *const Cout = sgm.C;
+            const int ldc = sgm.ldc, M = sgm.M, out_f32 = sgm.out_f32, vec = sgm.vec;
             const int acc = tc & 1;
             const uint32_t aph = (tc >> 1) & 1;
             if (!wait_or_abort(&accf[acc], aph, abort, status)) goto done;
@@ -149,9 +189,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 float x[16];
                 tmem_ld16(src + c, x);
                 tmem_ld_wait();
-                if (row < M && n0 + c < N && !(vec && n0 + c + 16 <= N)) {
+                if (g.trans) {  // C^T: for each column, the warp's 32 rows are 32 consecutive elements
+                    if (row < M) {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            if (n0 + c + u >= N) break;
+                            const size_t o = static_cast<size_t>(n0 + c + u) * ldc + row;
+                            if (out_f32) static_cast<float *>(Cout)[o] = x[u];
+                            else static_cast<__nv_bfloat16 *>(Cout)[o] = __float2bfloat16_rn(x[u]);
+                        }
+                    }
+                } else if (row < M && n0 + c < N && !(vec && n0 + c + 16 <= N)) {
                     // ragged column tail or unaligned rows: element stores
-                    for (int u = 0; u < 16 && n0 + c + u < N; ++u) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        if (n0 + c + u >= N) break;
                         if (out_f32) static_cast<float *>(Cout)[static_cast<size_t>(row) * ldc + n0 + c + u] = x[u];
                         else static_cast<__nv_bfloat16 *>(Cout)[static_cast<size_t>(row) * ldc + n0 + c + u] = __float2bfloat16_rn(x[u]);
                     }
@@ -212,32 +264,70 @@ int sm_count() {
 }
 
 template <int BN>
-int launch_gemm(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
-                int out_f32, cudaStream_t s) {
+int launch_gemm(GemmArgs &g, cudaStream_t s) {
     using G = GemmCfg<BN>;
     static std::atomic<unsigned long long> attr_done{0};
     KDA_TRY(smem_opt_in(gemm_kernel<BN>, G::bytes, attr_done));
-    CUtensorMap ta, tw;
-    KDA_TRY(make_map(&ta, A, M, K, lda, BM));
-    KDA_TRY(make_map(&tw, W, N, K, ldw, BN));
     int *status = device_status_ptr();
     if (!status) return KDA_ERR_CUDA;
-    const long long ntiles = static_cast<long long>((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    long long ntiles = 0;
+    for (int i = 0; i < g.nseg; ++i) ntiles += static_cast<long long>((g.seg[i].M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+    if (ntiles == 0) return KDA_OK;
     const int grid = static_cast<int>(std::min<long long>(ntiles, sm_count()));
-    // 16-element vector stores need 16-byte aligned rows
-    const int vec = aligned16(Cout) && (ldc % (out_f32 ? 4 : 8)) == 0;
-    gemm_kernel<BN><<<grid, kGemmThreads, G::bytes, s>>>(ta, tw, Cout, ldc, M, N, K, out_f32, vec, status);
+    gemm_kernel<BN><<<grid, kGemmThreads, G::bytes, s>>>(g, status);
     return launch_status();
+}
+
+template <int BN>
+int gemm_one(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
+             int out_f32, cudaStream_t s) {
+    GemmArgs g{};
+    KDA_TRY(make_map(&g.tmA[0], A, M, K, lda, BM));
+    KDA_TRY(make_map(&g.tmW[0], W, N, K, ldw, BN));
+    // 16-element vector stores need 16-byte aligned rows
+    g.seg[0] = GemmSeg{Cout, ldc, M, out_f32, aligned16(Cout) && (ldc % (out_f32 ? 4 : 8)) == 0};
+    g.nseg = 1;
+    g.N = N;
+    g.K = K;
+    g.trans = 0;
+    return launch_gemm<BN>(g, s);
+}
+
+// The small-M form: y_s[m][n] = x_s[m] . W_s[n] for a few rows m of each segment's input, as
+// the transposed product W_s . x_s^T, so that the 128-row tiles run over the weights' output
+// rows (every weight is read once, by many CTAs) and the few input rows are the N side.
+template <int BN>
+int gemm_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s) {
+    GemmArgs g{};
+    for (int i = 0; i < nseg; ++i) {
+        const GemmTSeg &t = segs[i];
+        KDA_TRY(make_map(&g.tmA[i], t.W, t.N, K, t.ldw, BM));
+        KDA_TRY(make_map(&g.tmW[i], t.x, rows, K, t.ldx, BN));
+        g.seg[i] = GemmSeg{t.y, t.ldy, t.N, t.out_f32, 0};
+    }
+    g.nseg = nseg;
+    g.N = rows;
+    g.K = K;
+    g.trans = 1;
+    return launch_gemm<BN>(g, s);
 }
 
 }  // namespace
 
 int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
               int out_f32, cudaStream_t s) {
-    if (N > 128) return launch_gemm<256>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
-    if (N > 64) return launch_gemm<128>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
-    if (N > 32) return launch_gemm<64>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
-    return launch_gemm<32>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    if (N > 128) return gemm_one<256>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    if (N > 64) return gemm_one<128>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    if (N > 32) return gemm_one<64>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+    return gemm_one<32>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
+}
+
+int gemm_bf16_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s) {
+    if (nseg < 1 || nseg > kMaxGemmSegs || rows <= 0) return KDA_ERR_INVALID_ARG;
+    if (rows > 128) return gemm_small_m<256>(segs, nseg, rows, K, s);
+    if (rows > 64) return gemm_small_m<128>(segs, nseg, rows, K, s);
+    if (rows > 32) return gemm_small_m<64>(segs, nseg, rows, K, s);
+    return gemm_small_m<32>(segs, nseg, rows, K, s);
 }
 
 // ------------------------------------------------------------------ small-M matrix-vector products
