@@ -1172,25 +1172,29 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *gsrc, uint
 //   epilogue 1    U = U~ - D1[0:64] into shared memory
 //   MMA group 2   D3 = (K o e^{Gamma_C - Gamma})^T . U        (M = D, N = DVS, K = 64)
 //   MMA group 3   D1 += [0; M] . U                            (so D1[64:128] = (Q o A) S0 + M U)
-//   epilogue 2    S = A_C o S0 + D3 (FP32 master copy in registers) into the S operand
+//   epilogue 2    S = A_C o S0 + D3 (the FP32 master copy lives in TMEM) into the S operand
 // Groups 1 and 2 and the two epilogues are the critical path. Two control threads issue every
 // copy and every MMA, so that the epilogue warps never wait behind MMA issue: the chain thread
 // (warp kEpiWarps) issues groups 1 and 2 and the copies of their operands; with two U operands in
 // shared memory the output thread (warp kEpiWarps + 1) issues group 3 of a chunk once its group 2
 // has completed (it then runs while epilogue 2 does) and copies the next M; with one U operand the
 // chain thread issues group 3 right after group 2. The output rows O = scale D1[64:128] of chunk c
-// are read while group 2 of chunk c + 1 runs. Every chunk's operand pack two chunks ahead is
-// prefetched into L2. Epilogue and control warps hand over through mbarriers.
-constexpr int kEpiWarps = 8;
-constexpr int kStateThreads = 32 * (kEpiWarps + 2);  // + the two control warps
+// are read while group 2 of chunk c + 1 runs. Epilogue and control warps hand over through
+// mbarriers. Epilogue warps: 8 (4 TMEM lane quarters x 2 column groups), 16 for 128-column
+// slices (x 4), so that a thread's share of an epilogue stays at 32 columns or fewer.
+template <int DVS>
+constexpr int kEpiWarpsFor = DVS >= 128 ? 16 : 8;
+template <int DVS>
+constexpr int kStateThreadsFor = 32 * (kEpiWarpsFor<DVS> + 2);  // + the two control warps
 
 template <int D, int DVS>
-__global__ void __launch_bounds__(kStateThreads, 1)
+__global__ void __launch_bounds__(kStateThreadsFor<DVS>, 1)
 state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_state, float *__restrict__ core,
              const Seqs sq, int H, float scale, float *__restrict__ tables, int *__restrict__ status) {
     using S = State<D, DVS>;
     using PK = Pack<D>;
-    constexpr int HALF = DVS / 2;         // value columns per epilogue thread
+    constexpr int kEpiWarps = kEpiWarpsFor<DVS>, kStateThreads = kStateThreadsFor<DVS>;
+    constexpr int HALF = DVS / (kEpiWarps / 4);  // value columns per epilogue thread
     // U~ read into registers while group 1 runs (slices up to 64 columns; wider slices read it one
     // 8-column group ahead: with 9 warps one scheduler holds three, so a thread has about 168 registers)
     constexpr bool kPreU = HALF <= 32;
@@ -1270,6 +1274,7 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
     }
     // Epilogue roles: for an M = 128 accumulator warp w reads TMEM lanes 32(w%4)..+31 (rows),
     // value columns [(w/4) HALF, + HALF). D3 with D = 64 (M = 64) has rows 16 (w%4) + lane, lane < 16.
+    static_assert(DVS % (kEpiWarps / 4) == 0 && HALF % 8 == 0, "epilogue column groups");
     const int quad = warp & 3, colh = warp >> 2;
     const int erow = 32 * quad + lane;
     const int ccol = colh * HALF;
@@ -1633,25 +1638,29 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     KDA_TRY(launch_status());
     intra_fix_kernel<D, MODE><<<grid_fix, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
     KDA_TRY(launch_status());
-    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kStateThreads, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
+    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kStateThreadsFor<DVS>, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
                                                                                    in.tables, status);
     return launch_status();
 }
 
 // Value slice width. One state CTA fills an SM and walks its (stream, head)'s chunks in order,
-// so the pass takes (waves of CTAs) x (chunks) x (one chunk's chain). Measured chains: about
-// 4.9 K cycles per chunk with 32 value columns, 6 K with 64 and 13.5 K with 128 (the MMAs cost
-// the same up to N = 64, and the epilogues grow with the columns). So 32 columns while four
-// slices per unit fit on the SMs in one wave, else 64: two 64-column waves beat one of 128.
+// so the pass takes (waves of CTAs) x (chunks) x (one chunk's chain). Measured chains per chunk:
+// about 4.9 K cycles with 32 value columns, 6 K with 64, 10 K with 128 (16 epilogue warps; the
+// MMAs cost the same up to N = 64 and the epilogues grow with the columns). The width with the
+// smallest waves x chain is taken: 32 columns while four slices per unit fit in one wave, 64
+// while two do, 128 for one wave of whole heads beyond that.
 template <int MODE>
 int launch_any(const PrefillIn &in, float *const *h_state, float *core, int B, const Seqs &sq, const kda_dims *dims,
                void *scratch, cudaStream_t s) {
     const int H = dims->heads;
     const float sc = dims->scale;
     if (dims->head_dim == 64) return launch_tc<64, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
-    const long long units = static_cast<long long>(B) * H;
-    if (4 * units <= sm_count()) return launch_tc<128, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
-    return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    const long long units = static_cast<long long>(B) * H, sms = sm_count();
+    auto cost = [&](long long slices, long long chain) { return (units * slices + sms - 1) / sms * chain; };
+    const long long c32 = cost(4, 49), c64 = cost(2, 60), c128 = cost(1, 100);
+    if (c32 <= c64 && c32 <= c128) return launch_tc<128, 32, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    if (c64 <= c128) return launch_tc<128, 64, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
+    return launch_tc<128, 128, MODE>(in, h_state, core, B, sq, H, sc, scratch, s);
 }
 
 Seqs equal_seqs(int T) {
