@@ -496,7 +496,10 @@ KDA_API int kda_workspace_create(const kda_dims *dims, int hidden, int rank, siz
 /* The same for packed calls (kda_block_prefill_varlen / _batched, kda_block_verify) of up to
  * max_seqs sequences and max_tokens rows in all: the chunked-prefill scratch is sized by
  * kda_chunk_prefill_packed_scratch_bytes(max_seqs, max_tokens), which fits any mix of lengths.
- * max_seqs = 1 is kda_workspace_create. */
+ * max_seqs = 1 is kda_workspace_create. Besides the stage buffers, the workspace holds an FP32
+ * buffer for the split-K partial sums of projections over at most 256 rows (one 128 x BN tile
+ * per SM; BN the smallest of 32, 64, 128, 256 covering min(max_tokens, 256) rows: 19 MB on a
+ * 148-SM GPU at BN 256). */
 KDA_API int kda_workspace_create_batched(const kda_dims *dims, int hidden, int rank, size_t max_tokens,
                                          int max_seqs, kda_workspace **out);
 KDA_API int kda_workspace_destroy(kda_workspace *ws);

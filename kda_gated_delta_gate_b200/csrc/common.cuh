@@ -185,7 +185,11 @@ struct GemmTSeg {
     void *y;
     int N, ldw, ldx, ldy, out_f32;
 };
-int gemm_bf16_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s);
+// part: FP32 buffer for split-K partial sums (null: no split); a launch splits only as far as
+// part_bytes holds. small_m_part_bytes(rows) holds any split of a call of that many rows.
+int gemm_bf16_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s, float *part = nullptr,
+                      size_t part_bytes = 0);
+size_t small_m_part_bytes(int rows);
 int gemv_bf16(const uint16_t *x, int ldx, const uint16_t *W, int ldw, void *y, int ldy, int M, int N, int K,
               int out_f32, cudaStream_t s);
 int gemv_segs(const uint16_t *x, int ldx, const GemvSegs &segs, int M, int K, cudaStream_t s);

@@ -60,6 +60,8 @@ struct kda_workspace {
     size_t bytes[KDA_BUF_COUNT];
     float **state_slot;  // device array holding the one state pointer of the call
     int *cu_equal;       // device [max_seqs + 1]: cu_seqlens of an equal-length batched call
+    float *splitk;       // FP32 split-K partial sums of the small-M projections
+    size_t splitk_bytes;
 };
 
 namespace kda {
@@ -78,12 +80,12 @@ ProjKind proj_kind(int M, bool exact) {
 
 // One projection of M rows.
 int proj(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *C, int ldc, int M, int N, int K, int out_f32,
-         cudaStream_t s, bool exact) {
+         cudaStream_t s, bool exact, const kda_workspace *ws) {
     switch (proj_kind(M, exact)) {
     case ProjKind::Gemv: return gemv_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
     case ProjKind::SmallM: {
         const GemmTSeg t{W, A, C, N, ldw, lda, ldc, out_f32};
-        return gemm_bf16_small_m(&t, 1, M, K, s);
+        return gemm_bf16_small_m(&t, 1, M, K, s, ws->splitk, ws->splitk_bytes);
     }
     default: return gemm_bf16(A, lda, W, ldw, C, ldc, M, N, K, out_f32, s);
     }
@@ -112,9 +114,9 @@ int block_projections(const kda_block_weights *w, const kda_bf16 *hidden, int M,
                                {w->f_a, hidden, fa, R, Hd, Hd, R, 0},
                                {w->g_a, hidden, ga, R, Hd, Hd, R, 0},
                                {w->b_proj, hidden, blog, H, Hd, Hd, H, 1}};
-        KDA_TRY(gemm_bf16_small_m(a, 6, M, Hd, s));
+        KDA_TRY(gemm_bf16_small_m(a, 6, M, Hd, s, ws->splitk, ws->splitk_bytes));
         const GemmTSeg c[2] = {{w->f_b, fa, graw, qkv, R, R, qkv, 0}, {w->g_b, ga, og, qkv, R, R, qkv, 0}};
-        return gemm_bf16_small_m(c, 2, M, R, s);
+        return gemm_bf16_small_m(c, 2, M, R, s, ws->splitk, ws->splitk_bytes);
     }
     if (kind == ProjKind::Gemv) {
         // every weight that reads the hidden rows: q, k, v, then the small f_a, g_a, b_proj
@@ -236,6 +238,11 @@ int kda_workspace_create_batched(const kda_dims *dims, int hidden, int rank, siz
             return KDA_ERR_CUDA;
         }
     }
+    ws->splitk_bytes = kda::small_m_part_bytes(static_cast<int>(std::min<size_t>(T, 256)));
+    if (cudaMalloc(reinterpret_cast<void **>(&ws->splitk), ws->splitk_bytes) != cudaSuccess) {
+        kda_workspace_destroy(ws);
+        return KDA_ERR_CUDA;
+    }
     if (cudaMalloc(reinterpret_cast<void **>(&ws->state_slot), sizeof(float *)) != cudaSuccess ||
         cudaMalloc(reinterpret_cast<void **>(&ws->cu_equal), (static_cast<size_t>(max_seqs) + 1) * sizeof(int)) !=
             cudaSuccess) {
@@ -255,6 +262,7 @@ int kda_workspace_destroy(kda_workspace *ws) {
     for (int i = 0; i < KDA_BUF_COUNT; ++i)
         if (ws->buf[i]) cudaFree(ws->buf[i]);
     if (ws->state_slot) cudaFree(ws->state_slot);
+    if (ws->splitk) cudaFree(ws->splitk);
     if (ws->cu_equal) cudaFree(ws->cu_equal);
     delete ws;
     return KDA_OK;
@@ -352,7 +360,7 @@ int kda_block_decode(const kda_block_weights *w, const kda_bf16 *hidden, int N, 
                              bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), N, d, stream));
     if (!w->o_proj) return KDA_OK;  // the caller applies its own o_proj (a tensor-parallel slice)
     return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, N, ws->hidden, qkv,
-                     0, s, false);
+                     0, s, false, ws);
 }
 
 int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K, float *h_state,
@@ -377,7 +385,7 @@ int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidden, int K
     for (int r0 = 0; r0 < K; r0 += kda::kRowsGemv) {
         const size_t o = static_cast<size_t>(r0);
         KDA_TRY(kda::proj(bf(KDA_BUF_O_NORM_OUT) + o * qkv, qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT) + o * Hd, Hd,
-                          std::min(kda::kRowsGemv, K - r0), Hd, qkv, 0, s, true));
+                          std::min(kda::kRowsGemv, K - r0), Hd, qkv, 0, s, true, ws));
     }
     return KDA_OK;
 }
@@ -410,7 +418,7 @@ int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const i
                                    total_tokens, d, stream));
     if (!w->o_proj) return KDA_OK;
     return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, total_tokens,
-                     ws->hidden, qkv, 0, s, false);
+                     ws->hidden, qkv, 0, s, false, ws);
 }
 
 int kda_block_verify_fold(const int *cu_seqlens, const int *accepted, int B, int total_tokens, const float *tables,

@@ -76,7 +76,26 @@ struct GemmArgs {
     CUtensorMap tmW[kMaxGemmSegs];
     GemmSeg seg[kMaxGemmSegs];
     int nseg, N, K, trans;
+    // split-K (small-M form): each tile's K loop in ksplit consecutive parts, one work unit each;
+    // a unit stores its FP32 sums to part[unit][BN][BM] and splitk_reduce_kernel adds the parts
+    int ksplit;
+    float *part;
 };
+
+// First k-block of a tile's K loop. In the small-M form every tile reads the same few input rows,
+// so tiles that started together would read the same k-block of them from the same L2 lines at
+// the same time; each tile starts its (wrapping) K loop at its own k-block instead.
+__device__ __forceinline__ int k_start(const GemmArgs &g, int tile, int nk) {
+    return g.trans && g.ksplit <= 1 ? static_cast<int>((static_cast<unsigned>(tile) * 37u) % static_cast<unsigned>(nk))
+                                    : 0;
+}
+
+// The k-blocks [kb0, kb1) of work unit u (tile u / ks, part u % ks).
+__device__ __forceinline__ void unit_k(int u, int ks, int nk, int &kb0, int &kb1) {
+    const int kp = u % ks;
+    kb0 = kp * nk / ks;
+    kb1 = (kp + 1) * nk / ks;
+}
 
 // The segment and the tile origin of tile `t`.
 template <int BN>
@@ -112,6 +131,8 @@ gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
     int ntiles = 0;
     for (int i = 0; i < g.nseg; ++i) ntiles += (g.seg[i].M + BM - 1) / BM * tiles_n;
     const int nk = K / BK;
+    const int ksp = g.ksplit > 1 ? g.ksplit : 1;
+    const int nunits = ntiles * ksp;
 
     if (tid == 0) {
         for (int s = 0; s < G::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -131,17 +152,21 @@ gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
     if (warp == 0) {
         if (lane == 0) {  // ---- TMA producer
             int it = 0;
-            for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-                int m0, n0;
+            for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+                const int tile = u / ksp;
+                int m0, n0, kb0, kb1;
                 const int sg = gemm_tile<BN>(g, tiles_n, tile, m0, n0);
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                unit_k(u, ksp, nk, kb0, kb1);
+                const int k0 = k_start(g, tile, nk);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % G::STAGES;
                     const uint32_t ph = (it / G::STAGES) & 1;
                     if (!wait_or_abort(&empty[s], ph ^ 1, abort, status)) goto done;
                     uint8_t *sa = sm + s * G::STAGE;
+                    const int kx = (k0 + kb < nk ? k0 + kb : k0 + kb - nk) * BK;
                     mbar_expect_tx(&full[s], G::STAGE);
-                    tma_load_2d(sa, &g.tmA[sg], kb * BK, m0, &full[s]);
-                    tma_load_2d(sa + G::A_STAGE, &g.tmW[sg], kb * BK, n0, &full[s]);
+                    tma_load_2d(sa, &g.tmA[sg], kx, m0, &full[s]);
+                    tma_load_2d(sa + G::A_STAGE, &g.tmW[sg], kx, n0, &full[s]);
                 }
             }
         }
@@ -149,13 +174,15 @@ gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
         if (lane == 0) {  // ---- MMA issuer
             constexpr uint32_t id = idesc_bf16(BM, BN, false, false);
             int it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+            for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++tc) {
+                int kb0, kb1;
+                unit_k(u, ksp, nk, kb0, kb1);
                 const int acc = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
                 if (!wait_or_abort(&acce[acc], aph ^ 1, abort, status)) goto done;
                 tc_fence_after();
                 const uint32_t dcol = tmem + acc * BN;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % G::STAGES;
                     const uint32_t ph = (it / G::STAGES) & 1;
                     if (!wait_or_abort(&full[s], ph, abort, status)) goto done;
@@ -164,7 +191,7 @@ gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks)
                         mma_bf16(dcol, kmaj_desc(a0, BM, 0, ks), kmaj_desc(b0, BN, 0, ks), id,
-                                 (kb > 0 || ks > 0) ? 1u : 0u);
+                                 (kb > kb0 || ks > 0) ? 1u : 0u);
                     mma_commit(&empty[s]);
                 }
                 mma_commit(&accf[acc]);
@@ -173,7 +200,8 @@ gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
     } else {  // ---- epilogue warps 2..5: TMEM lanes 32 (warp % 4) .. + 31
         const int quad = warp & 3;
         int tc = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++tc) {
+            const int tile = u / ksp;
             int m0, n0;
             const GemmSeg &sgm = g.seg[gemm_tile<BN>(g, tiles_n, tile, m0, n0)];
             void *const Cout = sgm.C;
@@ -189,7 +217,14 @@ gemm_kernel(const __grid_constant__ GemmArgs g, int *__restrict__ status) {
                 float x[16];
                 tmem_ld16(src + c, x);
                 tmem_ld_wait();
-                if (g.trans) {  // C^T: for each column, the warp's 32 rows are 32 consecutive elements
+                if (ksp > 1) {  // this unit's FP32 sums: part[u][column][row], the warp's 32 rows contiguous
+                    float *pu = g.part + static_cast<size_t>(u) * BN * BM + 32 * quad + lane;
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) {
+                        if (n0 + c + v >= N) break;
+                        pu[static_cast<size_t>(c + v) * BM] = x[v];
+                    }
+                } else if (g.trans) {  // C^T: for each column, the warp's 32 rows are 32 consecutive elements
                     if (row < M) {
 #pragma unroll
                         for (int u = 0; u < 16; ++u) {
@@ -236,6 +271,34 @@ done:
     if (warp == 1) tmem_dealloc(tmem, G::TMEM_COLS);
 }
 
+// The parts of a split-K launch added in part order (a fixed order: the same bits on every
+// call with the same split), each element stored as the unsplit epilogue stores it. Block
+// (tile, group of 8 columns), one thread per 4 consecutive rows of a column (16-byte reads).
+template <int BN>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ GemmArgs g) {
+    const int tile = blockIdx.x, N = g.N, ksp = g.ksplit;
+    const int tiles_n = (N + BN - 1) / BN;
+    int m0, n0;
+    const GemmSeg &sg = g.seg[gemm_tile<BN>(g, tiles_n, tile, m0, n0)];
+    const int c = 8 * blockIdx.y + threadIdx.x / (BM / 4), r = 4 * (threadIdx.x % (BM / 4));
+    if (n0 + c >= N || m0 + r >= sg.M) return;
+    const float *p = g.part + static_cast<size_t>(tile) * ksp * BN * BM + static_cast<size_t>(c) * BM + r;
+    float4 t = *reinterpret_cast<const float4 *>(p);
+    for (int kp = 1; kp < ksp; ++kp) {
+        const float4 v = *reinterpret_cast<const float4 *>(p + static_cast<size_t>(kp) * BN * BM);
+        t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+    }
+    const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (m0 + r + j >= sg.M) break;
+        const size_t o = g.trans ? static_cast<size_t>(n0 + c) * sg.ldc + m0 + r + j
+                                 : static_cast<size_t>(m0 + r + j) * sg.ldc + n0 + c;
+        if (sg.out_f32) static_cast<float *>(sg.C)[o] = tv[j];
+        else static_cast<__nv_bfloat16 *>(sg.C)[o] = __float2bfloat16_rn(tv[j]);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 // 2-D BF16 tensor map over `rows` x `cols` (row stride ld elements), box 64 (K) x box_rows.
@@ -273,7 +336,7 @@ int launch_gemm(GemmArgs &g, cudaStream_t s) {
     long long ntiles = 0;
     for (int i = 0; i < g.nseg; ++i) ntiles += static_cast<long long>((g.seg[i].M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
     if (ntiles == 0) return KDA_OK;
-    const int grid = static_cast<int>(std::min<long long>(ntiles, sm_count()));
+    const int grid = static_cast<int>(std::min<long long>(ntiles * std::max(g.ksplit, 1), sm_count()));
     gemm_kernel<BN><<<grid, kGemmThreads, G::bytes, s>>>(g, status);
     return launch_status();
 }
@@ -296,20 +359,40 @@ int gemm_one(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout,
 // The small-M form: y_s[m][n] = x_s[m] . W_s[n] for a few rows m of each segment's input, as
 // the transposed product W_s . x_s^T, so that the 128-row tiles run over the weights' output
 // rows (every weight is read once, by many CTAs) and the few input rows are the N side.
+// A CTA streams only so many bytes per second, so a launch with at most one tile per two SMs
+// splits each tile's K loop over several CTAs, as many as one wave holds (at least 4 k-blocks
+// each, at most 8 parts, as many as the part buffer holds), and adds the parts in a second, short
+// launch. Launches with more tiles gain nothing from it: every tile re-reads all input rows, and
+// that L2 traffic, not the CTA count, sets their time.
 template <int BN>
-int gemm_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s) {
+int gemm_small_m(const GemmTSeg *segs, int nseg, int rows, int K, float *part, size_t part_bytes, cudaStream_t s) {
     GemmArgs g{};
+    long long ntiles = 0;
     for (int i = 0; i < nseg; ++i) {
         const GemmTSeg &t = segs[i];
         KDA_TRY(make_map(&g.tmA[i], t.W, t.N, K, t.ldw, BM));
         KDA_TRY(make_map(&g.tmW[i], t.x, rows, K, t.ldx, BN));
         g.seg[i] = GemmSeg{t.y, t.ldy, t.N, t.out_f32, 0};
+        ntiles += static_cast<long long>((t.N + BM - 1) / BM) * ((rows + BN - 1) / BN);
     }
     g.nseg = nseg;
     g.N = rows;
     g.K = K;
     g.trans = 1;
-    return launch_gemm<BN>(g, s);
+    g.ksplit = 1;
+    const long long sms = sm_count();
+    if (part && ntiles > 0 && 2 * ntiles <= sms) {
+        long long ksp = std::min<long long>({sms / ntiles, 8, K / BK / 4});
+        ksp = std::min<long long>(ksp, static_cast<long long>(part_bytes / (static_cast<size_t>(ntiles) * BN * BM * 4)));
+        if (ksp >= 2) {
+            g.ksplit = static_cast<int>(ksp);
+            g.part = part;
+        }
+    }
+    KDA_TRY(launch_gemm<BN>(g, s));
+    if (g.ksplit == 1 || ntiles == 0) return KDA_OK;
+    splitk_reduce_kernel<BN><<<dim3(static_cast<unsigned>(ntiles), BN / 8), 256, 0, s>>>(g);
+    return launch_status();
 }
 
 }  // namespace
@@ -322,12 +405,18 @@ int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout
     return gemm_one<32>(A, lda, W, ldw, Cout, ldc, M, N, K, out_f32, s);
 }
 
-int gemm_bf16_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s) {
+size_t small_m_part_bytes(int rows) {
+    const int bn = rows > 128 ? 256 : (rows > 64 ? 128 : (rows > 32 ? 64 : 32));
+    return static_cast<size_t>(sm_count()) * bn * BM * 4;  // one wave of units
+}
+
+int gemm_bf16_small_m(const GemmTSeg *segs, int nseg, int rows, int K, cudaStream_t s, float *part,
+                      size_t part_bytes) {
     if (nseg < 1 || nseg > kMaxGemmSegs || rows <= 0) return KDA_ERR_INVALID_ARG;
-    if (rows > 128) return gemm_small_m<256>(segs, nseg, rows, K, s);
-    if (rows > 64) return gemm_small_m<128>(segs, nseg, rows, K, s);
-    if (rows > 32) return gemm_small_m<64>(segs, nseg, rows, K, s);
-    return gemm_small_m<32>(segs, nseg, rows, K, s);
+    if (rows > 128) return gemm_small_m<256>(segs, nseg, rows, K, part, part_bytes, s);
+    if (rows > 64) return gemm_small_m<128>(segs, nseg, rows, K, part, part_bytes, s);
+    if (rows > 32) return gemm_small_m<64>(segs, nseg, rows, K, part, part_bytes, s);
+    return gemm_small_m<32>(segs, nseg, rows, K, part, part_bytes, s);
 }
 
 // ------------------------------------------------------------------ small-M matrix-vector products
