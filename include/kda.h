@@ -570,30 +570,43 @@ KDA_API int kda_block_decode_k(const kda_block_weights *w, const kda_bf16 *hidde
 
 /* kda_block_verify — batched speculative verify through the whole block (Glm5NextLayer verify:
  * N sequences x K draft rows; Glm5NextKdaLayer `decode_k` at layer level): the projections of all
- * draft rows of all sequences in one pass (each weight read once for all rows), the packed conv
- * from each sequence's conv state, then the chunked core in verify mode (kda_chunk_verify, fused
- * input) from each sequence's recurrent state, o_norm and o_proj. NO state changes: the
- * recurrent and conv states stay as they were, and `tables` (kda_chunk_verify_tables_bytes(B),
- * 16-byte aligned) receives what kda_block_verify_fold needs.
+ * draft rows of all sequences in one pass (each weight read once for all rows), then one of two
+ * routes, chosen from (B, total_tokens) alone:
+ *   - short drafts (total_tokens <= 16 B): each (sequence, head) runs its rows in the stateful
+ *     decode row (conv + SiLU + L2, gate, beta, recurrence, o_norm; the state in shared memory
+ *     and written back nowhere), then o_proj. Every row's outputs are bit for bit what
+ *     kda_decode_k gives on that sequence's stage rows. KDA_BUF_BETA then holds the beta LOGITS.
+ *   - longer drafts: the packed conv from each conv state, the chunked core in verify mode
+ *     (kda_chunk_verify, fused input) from each recurrent state, o_norm and o_proj; `tables`
+ *     receives what the fold needs. Each row's output equals what kda_block_prefill_varlen on
+ *     that sequence's first rows gives for it (the same core arithmetic), up to the projection
+ *     kernel.
+ * NO state changes on either route: the recurrent and conv states stay as they were. `tables`
+ * (kda_chunk_verify_tables_bytes(B), 16-byte aligned) is required on both.
  *   hidden      [total_tokens, hidden] BF16, sequence b = rows [cu_seqlens[b], cu_seqlens[b+1]),
  *               at most 64 rows each (a longer one latches KDA_ERR_INVALID_ARG and is skipped)
  *   cu_seqlens  DEVICE int32 [B + 1];  h_state, conv_state: DEVICE pointer arrays as
  *               kda_block_prefill_varlen (read only here)
- * Each row's output equals what kda_block_prefill_varlen on that sequence's first rows gives
- * for it (the same core arithmetic), up to the projection kernel: up to 8 rows in all the
- * matrix-vector kernel, up to 256 the small-M tensor-core form, beyond that the GEMM. The workspace keeps the rows' qkv_proj and
- * conv_out for the fold. KDA_ERR_CAPACITY if total_tokens > max_tokens or B > max_seqs. */
+ * Projections: up to 8 rows in all the matrix-vector kernel, up to 256 the small-M tensor-core
+ * form, beyond that the GEMM. The workspace keeps the rows' stage buffers (and, on the row route,
+ * a copy of *w: the weights must stay valid until the fold) for the fold. KDA_ERR_CAPACITY if
+ * total_tokens > max_tokens or B > max_seqs. */
 KDA_API int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const int *cu_seqlens, int B,
                              int total_tokens, float *const *h_state, kda_bf16 *const *conv_state, float *tables,
                              size_t tables_bytes, kda_workspace *ws, void *stream);
 
 /* kda_block_verify_fold — accepted-row folding after kda_block_verify (Glm5NextLayer
  * `gdn_fold_accepted`): sequence b's recurrent state becomes its state after its first
- * accepted[b] verified rows (kda_chunk_verify_fold's formula on the verify's tables and the BF16
- * k rows its core read) and its conv state the last three inputs of (state || those rows'
- * qkv_proj). accepted DEVICE int32 [B], 0 <= accepted[b] <= its rows; 0 leaves both states.
- * Run on the same workspace, cu_seqlens, tables and states right after kda_block_verify, before
- * any other call on that workspace. */
+ * accepted[b] verified rows and its conv state the last three inputs of (state || those rows'
+ * qkv_proj). The route is the verify's (the same rule on B and total_tokens):
+ *   - row route: the accepted rows run again through the stateful decode row with the verify's
+ *     weights and stage buffers, now advancing both states: bit for bit the states kda_decode_k
+ *     leaves after those rows (KDA_ERR_INVALID_ARG if no row-route verify ran on this workspace);
+ *   - chunked route: kda_chunk_verify_fold's formula on the verify's tables and the BF16 k rows
+ *     its core read.
+ * accepted DEVICE int32 [B], 0 <= accepted[b] <= its rows; 0 leaves both states. Run on the same
+ * workspace, cu_seqlens, tables and states right after kda_block_verify, before any other call
+ * on that workspace. */
 KDA_API int kda_block_verify_fold(const int *cu_seqlens, const int *accepted, int B, int total_tokens,
                                   const float *tables, float *const *h_state, kda_bf16 *const *conv_state,
                                   kda_workspace *ws, void *stream);

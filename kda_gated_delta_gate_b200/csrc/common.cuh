@@ -164,6 +164,14 @@ namespace kda {
 // Projection GEMM and the batched-M matrix-vector products (kda_gemm.cu). Up to three weights
 // that read the same rows (q, k and v of one hidden row, say) go in one matrix-vector launch:
 // the column index runs over the concatenated outputs.
+// The stateful decode row over packed draft rows: a verify (acc null: every row, states kept) or
+// a fold (each sequence's first acc[n] rows, states advanced). kda_decode.cu.
+int decode_rows_packed(const uint16_t *x, uint16_t *const *conv_state, const uint16_t *conv_w, const uint16_t *g_raw,
+                       const float *dt_bias, const float *a_log, const float *b_logit, float *const *h_state,
+                       const uint16_t *out_gate, const uint16_t *o_norm_w, uint16_t *o_norm_out, uint16_t *conv_out,
+                       float *core, const int *cu, const int *acc, int B, int total, const kda_dims *dims,
+                       cudaStream_t s);
+
 struct GemvSeg {
     const uint16_t *W;
     void *y;

@@ -62,6 +62,10 @@ struct kda_workspace {
     int *cu_equal;       // device [max_seqs + 1]: cu_seqlens of an equal-length batched call
     float *splitk;       // FP32 split-K partial sums of the small-M projections
     size_t splitk_bytes;
+    // the weights of the last kda_block_verify that ran row by row: its fold re-runs the accepted
+    // rows through the same stateful row, which needs the conv, gate and beta weights
+    kda_block_weights verify_w;
+    int verify_w_set;
 };
 
 namespace kda {
@@ -69,6 +73,11 @@ namespace {
 constexpr int kRowsGemv = 32;   // exact calls: the matrix-vector kernel up to this many rows
 constexpr int kRowsGemvFree = 8; // other calls: the matrix-vector kernel up to one row group
 constexpr int kRowsSmallM = 256; // then the small-M tensor-core form, then the GEMM
+// A batched verify of at most this many draft rows per sequence on average runs row by row in the
+// stateful decode row (K steps per (sequence, head), the state in shared memory); longer drafts
+// take the chunked verify. Its fold follows the same rule on the same (B, total_tokens).
+constexpr int kVerifyRowsByRow = 16;
+bool verify_by_rows(int B, int total) { return static_cast<long long>(total) <= static_cast<long long>(kVerifyRowsByRow) * B; }
 
 // Which kernel takes M rows. `exact`: every row must get the bits it gets alone (decode_k's
 // identity with serial one-row decodes), which only the matrix-vector kernel gives.
@@ -408,6 +417,19 @@ int kda_block_verify(const kda_block_weights *w, const kda_bf16 *hidden, const i
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
     // every weight read once for all draft rows of all sequences
     KDA_TRY(kda::block_projections(w, hidden, total_tokens, ws, s, false));
+    if (kda::verify_by_rows(B, total_tokens)) {
+        // short drafts: each (sequence, head) runs its rows in the stateful decode row, with the
+        // state in shared memory and written back nowhere (the beta buffer keeps its logits)
+        ws->verify_w = *w;
+        ws->verify_w_set = 1;
+        KDA_TRY(kda::decode_rows_packed(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_G_RAW), w->dt_bias,
+                                        w->a_log, f32(KDA_BUF_BETA), h_state, bf(KDA_BUF_OUT_GATE), w->o_norm,
+                                        bf(KDA_BUF_O_NORM_OUT), bf(KDA_BUF_CONV_OUT), f32(KDA_BUF_CORE), cu_seqlens,
+                                        nullptr, B, total_tokens, d, s));
+        if (!w->o_proj) return KDA_OK;
+        return kda::proj(bf(KDA_BUF_O_NORM_OUT), qkv, w->o_proj, qkv, bf(KDA_BUF_FINAL_OUT), ws->hidden, total_tokens,
+                         ws->hidden, qkv, 0, s, false, ws);
+    }
     KDA_TRY(kda::front_varlen(bf(KDA_BUF_QKV_PROJ), conv_state, w->conv, bf(KDA_BUF_CONV_OUT), cu_seqlens, B,
                               total_tokens, d, s));
     KDA_TRY(kda_beta(f32(KDA_BUF_BETA), f32(KDA_BUF_BETA), total_tokens * d->heads, stream));
@@ -430,6 +452,17 @@ int kda_block_verify_fold(const int *cu_seqlens, const int *accepted, int B, int
     auto s = static_cast<cudaStream_t>(stream);
     const kda_dims *d = &ws->dims;
     const size_t qkv = static_cast<size_t>(d->heads) * d->head_dim;
+    if (kda::verify_by_rows(B, total_tokens)) {
+        // the verify ran row by row: the accepted rows run again through the same stateful row,
+        // now advancing both states (bits as the verify computed them)
+        if (!ws->verify_w_set) return KDA_ERR_INVALID_ARG;
+        const kda_block_weights &vw = ws->verify_w;
+        auto bfc = [&](int i) { return static_cast<const uint16_t *>(ws->buf[i]); };
+        return kda::decode_rows_packed(bfc(KDA_BUF_QKV_PROJ), conv_state, vw.conv, bfc(KDA_BUF_G_RAW), vw.dt_bias,
+                                       vw.a_log, static_cast<const float *>(ws->buf[KDA_BUF_BETA]), h_state,
+                                       bfc(KDA_BUF_OUT_GATE), nullptr, nullptr, nullptr, nullptr, cu_seqlens, accepted, B,
+                                       total_tokens, d, s);
+    }
     const auto *conv_out = static_cast<const uint16_t *>(ws->buf[KDA_BUF_CONV_OUT]);
     // k: the BF16 k channels of the verify's conv_out rows (what its core read)
     KDA_TRY(kda::verify_fold(nullptr, conv_out + qkv, 3 * qkv, cu_seqlens, accepted, B, total_tokens, tables, h_state,

@@ -216,6 +216,7 @@ recurrent_decode_kernel(const float *__restrict__ q, const float *__restrict__ k
 // ----------------------------------------------------------------------------- fused stateful row
 
 constexpr int kMaxSnap = 31;
+constexpr int kMaxPackedRows = 64;  // rows of one packed sequence (one chunk, as the chunked verify)
 
 struct RowParams {
     const uint16_t *x;          // [rows, 3*H*D]
@@ -234,6 +235,11 @@ struct RowParams {
     float scale, l2_eps, rms_eps;
     float *h_snap[kMaxSnap];
     uint16_t *conv_snap[kMaxSnap];
+    // packed rows (cu non-null): sequence n owns rows cu[n] .. cu[n+1]-1 of the call's total;
+    // verify runs them all and writes neither state; with acc, only the first acc[n] rows run and
+    // both states are advanced (outputs may then be null: the o_norm step is skipped)
+    const int *cu, *acc;
+    int total, verify;
 };
 
 template <int D>
@@ -247,6 +253,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
         if (tid == 0) atomicExch(p.status, KDA_ERR_MISALIGNED);
         return;
     }
+    // this CTA's rows: K rows from n K, or the packed sequence's (the first acc[n] of them)
+    int nrows = p.K;
+    size_t rbase = static_cast<size_t>(n) * p.K;
+    if (p.cu) {
+        const int s0 = p.cu[n], s1 = p.cu[n + 1];
+        const int lim = p.acc ? p.acc[n] : s1 - s0;
+        if (s0 < 0 || s1 < s0 || s1 > p.total || s1 - s0 > kMaxPackedRows || lim < 0 || lim > s1 - s0) {
+            if (tid == 0 && h == 0) atomicExch(p.status, KDA_ERR_INVALID_ARG);  // this sequence is skipped
+            return;
+        }
+        rbase = static_cast<size_t>(s0);
+        nrows = lim;
+    }
+    if (nrows == 0) return;  // nothing to run: both states stay (no copy was issued)
     state_begin<D>(sm, S);
     uint16_t *cst = p.conv_one ? p.conv_one : p.conv_arr[n];
 
@@ -270,11 +290,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
     }
     const float nea = -expf(p.a_log[h]);
     const float dtb = qk_thread ? p.dt_bias[h * D + d] : 0.f;
-    const float ow = qk_thread ? bf16_to_f32(p.o_norm_w[d]) : 0.f;
+    const float ow = qk_thread && p.o_norm_w ? bf16_to_f32(p.o_norm_w[d]) : 0.f;
     bool ok = true;
 
-    for (int t = 0; t < p.K; ++t) {
-        const size_t row = static_cast<size_t>(n) * p.K + t;
+    for (int t = 0; t < nrows; ++t) {
+        const size_t row = rbase + t;
         // every global input of the row, loaded up front (they do not depend on the state)
         float x0 = 0.f, x1 = 0.f, graw = 0.f, og = 0.f;
         if (qk_thread || v_thread) x0 = bf16_to_f32(p.x[row * 3 * qkv + c0]);
@@ -318,14 +338,15 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
             ok = state_ready<D>(sm, p.status);
             if (!ok) break;  // block-uniform
         }
-        // the last row streams the state out; earlier rows keep it (and write their snapshot)
-        const bool last = t == p.K - 1;
+        // the last row streams the state out; earlier rows keep it (and write their snapshot);
+        // a verify keeps it in shared memory throughout
+        const bool last = t == nrows - 1;
         float *snap = !last && t < p.n_snap ? p.h_snap[t] + static_cast<size_t>(h) * D * D : nullptr;
-        state_step<D>(sm, beta, kq, p.scale, !last, S, snap);  // sm.o is complete when it returns
-        // o_norm: sigmoid-gated RMSNorm over the head's D outputs
+        state_step<D>(sm, beta, kq, p.scale, p.verify || !last, S, snap);  // sm.o is complete when it returns
+        // o_norm: sigmoid-gated RMSNorm over the head's D outputs (skipped by a fold)
         const float ov = qk_thread ? sm.o[d] : 0.f;
-        const float ms = sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm).x;
-        if (qk_thread) {
+        const float ms = p.o_norm_out ? sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm).x : 0.f;
+        if (qk_thread && p.o_norm_out) {
             const float rs = rsqrtf(__fadd_rn(__fmul_rn(ms, 1.0f / D), p.rms_eps));
             const float yv = __fmul_rn(__fmul_rn(__fmul_rn(ov, rs), ow), sigmoid_rn(og));
             p.o_norm_out[row * qkv + h * D + d] = f32_to_bf16(yv);
@@ -343,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
             }
         }
     }
-    if (!ok) return;
+    if (!ok || p.verify) return;  // a verify leaves the conv state too
     if (qk_thread || v_thread) {
 #pragma unroll
         for (int j = 0; j < 3; ++j) cst[c0 * 3 + j] = f32_to_bf16(s0[j]);
@@ -479,3 +500,35 @@ int kda_decode_k(const kda_bf16 *x, kda_bf16 *conv_state, const kda_bf16 *conv_w
 }
 
 }  // extern "C"
+
+namespace kda {
+
+// The stateful row over packed sequences: rows cu[n] .. cu[n+1]-1 belong to sequence n (at most
+// kMaxPackedRows). Without acc (a verify) every row runs and neither state is written; with acc
+// (a fold) only each sequence's first acc[n] rows run, both states are advanced as decode_k's
+// rows would advance them, and the outputs may be null.
+int decode_rows_packed(const uint16_t *x, uint16_t *const *conv_state, const uint16_t *conv_w, const uint16_t *g_raw,
+                       const float *dt_bias, const float *a_log, const float *b_logit, float *const *h_state,
+                       const uint16_t *out_gate, const uint16_t *o_norm_w, uint16_t *o_norm_out, uint16_t *conv_out,
+                       float *core, const int *cu, const int *acc, int B, int total, const kda_dims *dims,
+                       cudaStream_t s) {
+    KDA_TRY(check_dims(dims));
+    if (!x || !conv_state || !conv_w || !g_raw || !dt_bias || !a_log || !b_logit || !h_state || !out_gate || !cu ||
+        B < 0 || total < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (!acc && (!o_norm_w || !o_norm_out)) return KDA_ERR_INVALID_ARG;
+    if (B == 0) return KDA_OK;
+    if (B > 65535) return KDA_ERR_UNSUPPORTED;
+    RowParams p{};
+    p.x = x; p.conv_arr = conv_state; p.conv_w = conv_w; p.g_raw = g_raw; p.dt_bias = dt_bias; p.a_log = a_log;
+    p.b_logit = b_logit; p.h_arr = h_state; p.out_gate = out_gate; p.o_norm_w = o_norm_w;
+    p.o_norm_out = acc ? nullptr : o_norm_out;
+    p.conv_out = acc ? nullptr : conv_out;
+    p.core = acc ? nullptr : core;
+    p.H = dims->heads; p.scale = dims->scale; p.l2_eps = dims->l2_eps; p.rms_eps = dims->rms_eps;
+    p.K = 0; p.n_snap = 0;
+    p.cu = cu; p.acc = acc; p.total = total; p.verify = acc ? 0 : 1;
+    return launch_rows(p, B, dims->head_dim, s);
+}
+
+}  // namespace kda

@@ -2,6 +2,11 @@
 form) and of the block-level batched verify and accepted-row fold (Glm5NextLayer speculative
 verify and `gdn_fold_accepted`; Glm5NextKdaLayer `decode_k` at layer level).
 
+A verify of at most 16 draft rows per sequence on average runs row by row in the stateful decode
+row. Its exact check is decode_k's: every draft row's outputs, and the states its fold leaves,
+equal kda_decode_k run on that sequence's own stage rows, bit for bit. Longer drafts take the
+chunked verify, checked as the prefill is below.
+
 Each sequence is checked on its own against the FP64 oracle run on that sequence alone:
 - the BF16 stage buffers at 2e-2 (BF16 rounding at every stage, on both sides);
 - the conv state bit for bit against the last three inputs of (old state || the sequence's
@@ -42,6 +47,21 @@ def _states(n, H, D, seed):
     hs = torch.randn((n, H, D, D), generator=g) * 0.1
     cs = torch.randn((n, 3 * H * D, 3), generator=g).to(torch.bfloat16)
     return hs, cs
+
+
+def _decode_k_rows(dw, got, sl, hs0_b, cs0_b, d):
+    """kda_decode_k over the stage rows sl (pre-conv qkv_proj rows, g_raw, beta logits, out_gate)
+    from copies of one sequence's states: (o_norm_out, core, conv_out, state, conv state)."""
+    K, qkv = sl.stop - sl.start, d.heads * d.head_dim
+    hs, cs = hs0_b.cuda().clone(), cs0_b.cuda().clone()
+    on = torch.empty((K, qkv), dtype=torch.bfloat16, device="cuda")
+    co = torch.empty((K, 3 * qkv), dtype=torch.bfloat16, device="cuda")
+    core = torch.empty((K, d.heads, d.head_dim), dtype=torch.float32, device="cuda")
+    kda.kda_decode_k(got["qkv_proj"][sl].contiguous(), cs, dw.conv, got["g_raw"][sl].contiguous(), dw.dt_bias,
+                     dw.a_log, got["beta"][sl].contiguous(), hs, got["out_gate"][sl].contiguous(), dw.o_norm, on, co,
+                     core, K, [], [], d)
+    torch.cuda.synchronize()
+    return on, core, co, hs, cs
 
 
 def _conv_after(cs0, qkv_rows):
@@ -148,9 +168,10 @@ def test_block_prefill_batched_equals_varlen_and_single_calls():
 def test_block_verify_then_fold(hidden, H, D, rank, lens, acc):
     """kda_block_verify leaves every state as it was and gives each draft row the output of the
     block prefill of that sequence's rows (oracle); kda_block_verify_fold then moves each
-    recurrent state to the state after its accepted rows (the chunked prefill of those rows on
-    the same stage values, and the oracle) and each conv state to the last three accepted
-    inputs, bit for bit; accepted = 0 leaves both states."""
+    recurrent state to the state after its accepted rows (oracle; and bit for bit decode_k's on
+    the same stage rows for a row-by-row verify, within 1e-5 of the chunked prefill of those
+    rows for a chunked one) and each conv state to the last three accepted inputs, bit for bit;
+    accepted = 0 leaves both states."""
     Wt = block_weights(hidden, H, D, rank, seed=41, std=0.05)
     B, total, cu = len(lens), sum(lens), _cu(lens)
     d = kda.dims(H, D)
@@ -168,6 +189,7 @@ def test_block_verify_then_fold(hidden, H, D, rank, lens, acc):
     torch.cuda.synchronize()
     assert all(torch.equal(hs[b], hs0[b].cuda()) and torch.equal(cs[b], cs0[b].cuda()) for b in range(B))
     got = _stages(ws, total, Wt)
+    by_rows = total <= 16 * B  # kda_block_verify's rule: short drafts run row by row
     for b in range(B):
         r0, L = cu[b], lens[b]
         if L == 0:
@@ -176,7 +198,12 @@ def test_block_verify_then_fold(hidden, H, D, rank, lens, acc):
         ref = oracle.block_prefill(Wt, h[sl], np64(hs0[b]), np64(cs0[b]))
         errs = {k_: rel_l2(np64(got[k_][sl]), ref[k_]) for k_ in ("conv_out", "g_raw", "o_norm_out", "final_out")}
         assert all(e <= TOL_BF16 for e in errs.values()), (b, errs)
-        _check_core(got, r0, L, Wt, hs0[b], got["core"][sl], None, ref)
+        if by_rows:
+            on, core, co, _, _ = _decode_k_rows(dw, got, sl, hs0[b], cs0[b], d)
+            assert torch.equal(on, got["o_norm_out"][sl]) and torch.equal(co, got["conv_out"][sl]), b
+            assert torch.equal(core, got["core"][sl]), b
+        else:
+            _check_core(got, r0, L, Wt, hs0[b], got["core"][sl], None, ref)
     kda.kda_block_verify_fold(cu_d, torch.tensor(acc, dtype=torch.int32, device="cuda"), B, total, tables, hp, cp,
                               ws)
     torch.cuda.synchronize()
@@ -187,8 +214,12 @@ def test_block_verify_then_fold(hidden, H, D, rank, lens, acc):
             continue
         sl = slice(r0, r0 + r)
         assert torch.equal(cs[b], _conv_after(cs0[b].cuda(), got["qkv_proj"][sl])), b
-        _, s_r = _fused_core(got["conv_out"][sl], got["g_raw"][sl], got["beta"][sl], Wt, r, hs0[b])
-        assert rel_l2(np64(hs[b]), np64(s_r)) <= 1e-5, b
+        if by_rows:
+            _, _, _, s_r, c_r = _decode_k_rows(dw, got, sl, hs0[b], cs0[b], d)
+            assert torch.equal(hs[b], s_r) and torch.equal(cs[b], c_r), b
+        else:
+            _, s_r = _fused_core(got["conv_out"][sl], got["g_raw"][sl], got["beta"][sl], Wt, r, hs0[b])
+            assert rel_l2(np64(hs[b]), np64(s_r)) <= 1e-5, b
         ref = oracle.block_prefill(Wt, h[sl], np64(hs0[b]), np64(cs0[b]))
         assert rel_l2(np64(hs[b]), ref["h_state"]) <= TOL_BF16, b
         assert rel_l2(np64(cs[b]), ref["conv_state"]) <= 4e-3, b

@@ -6,6 +6,7 @@ write past a buffer's end, before its start, or into rows the contract leaves al
 import ctypes
 import math
 
+import numpy as np
 import pytest
 import torch
 
@@ -277,12 +278,15 @@ def test_host_f32_prefill_writes_only_its_outputs():
     assert torch.all(torch.isfinite(hc.t))
 
 
-def test_block_verify_and_fold_write_only_their_outputs():
+@pytest.mark.parametrize("lens,acc", [([7, 64, 1], [7, 10, 0]),   # 72 rows: the chunked verify
+                                      ([7, 16, 1], [7, 10, 0])])  # 24 rows: row by row
+def test_block_verify_and_fold_write_only_their_outputs(lens, acc):
     """kda_block_verify reads the guarded recurrent and conv states and leaves them as they were;
-    kda_block_verify_fold writes only inside them; the tables stay inside their allocation."""
+    kda_block_verify_fold writes only inside them; the tables stay inside their allocation. Both
+    routes: the chunked verify and the row-by-row one of short drafts."""
     from synth import block_hidden, block_weights
     from tests.test_gpu_block import _device_weights
-    hidden, H, D, rank, lens, acc = 256, 2, 64, 64, [7, 64, 1], [7, 10, 0]
+    hidden, H, D, rank = 256, 2, 64, 64
     total, nb = sum(lens), len(lens)
     Wt = block_weights(hidden, H, D, rank, seed=15, std=0.05)
     h = block_hidden(total, hidden, seed=15).cuda()
@@ -296,7 +300,7 @@ def test_block_verify_and_fold_write_only_their_outputs():
         c.t.copy_(torch.randn((3 * H * D, 3), generator=g).to(torch.bfloat16))
     before = [(a.t.clone(), c.t.clone()) for a, c in zip(hs, cs)]
     tables = Guarded((kda.kda_chunk_verify_tables_bytes(nb, d) // 4,), torch.float32)
-    cu = torch.tensor([0, 7, 71, 72], dtype=torch.int32, device="cuda")
+    cu = torch.tensor([0] + [int(x) for x in np.cumsum(lens)], dtype=torch.int32, device="cuda")
     dw = _device_weights(Wt)
     st = kda.block_weights_struct(dw)
     hp, cp = kda.ptr_array([a.t for a in hs]), kda.ptr_array([c.t for c in cs])
