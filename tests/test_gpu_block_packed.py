@@ -249,3 +249,35 @@ def test_block_verify_refuses_a_draft_longer_than_a_chunk():
     ref = oracle.block_prefill(Wt, h[65:69], np64(hs0[1]), np64(cs0[1]))
     assert rel_l2(np64(got["final_out"][65:69]), ref["final_out"]) <= TOL_BF16
     ws.close()
+
+
+def test_block_verify_full_size_short_drafts():
+    """hidden 4096, H 32, D 128, rank 128: 16 sequences x 4 draft rows run row by row, with
+    o_proj's 32 weight tiles each splitting K = 4096 over four CTAs. Sampled sequences' stage
+    buffers and block outputs against the oracle (2e-2), every sampled row's o_norm_out and core
+    bit for bit kda_decode_k's on its stage rows, and both states untouched."""
+    hidden, H, D, rank, B, K = 4096, 32, 128, 128, 16, 4
+    Wt = block_weights(hidden, H, D, rank, seed=47, std=0.02)
+    lens = [K] * B
+    total, cu = B * K, _cu(lens)
+    d = kda.dims(H, D)
+    h = block_hidden(total, hidden, seed=47)
+    hs0, cs0 = _states(B, H, D, seed=47)
+    ws = kda.Workspace(d, hidden, rank, max_tokens=total, max_seqs=B)
+    hs = [hs0[b].cuda().clone() for b in range(B)]
+    cs = [cs0[b].cuda().clone() for b in range(B)]
+    tables = torch.empty(kda.kda_chunk_verify_tables_bytes(B, d) // 4, device="cuda")
+    dw = _device_weights(Wt)
+    kda.kda_block_verify(kda.block_weights_struct(dw), h.cuda(), torch.tensor(cu, dtype=torch.int32, device="cuda"), B,
+                         total, kda.ptr_array(hs), kda.ptr_array(cs), tables, ws)
+    torch.cuda.synchronize()
+    assert all(torch.equal(hs[b], hs0[b].cuda()) and torch.equal(cs[b], cs0[b].cuda()) for b in range(B))
+    got = _stages(ws, total, Wt)
+    for b in (0, 7, 15):
+        sl = slice(cu[b], cu[b] + K)
+        ref = oracle.block_prefill(Wt, h[sl], np64(hs0[b]), np64(cs0[b]))
+        errs = {k_: rel_l2(np64(got[k_][sl]), ref[k_]) for k_ in ("conv_out", "g_raw", "o_norm_out", "final_out")}
+        assert all(e <= TOL_BF16 for e in errs.values()), (b, errs)
+        on, core, _, _, _ = _decode_k_rows(dw, got, sl, hs0[b], cs0[b], d)
+        assert torch.equal(on, got["o_norm_out"][sl]) and torch.equal(core, got["core"][sl]), b
+    ws.close()
