@@ -45,25 +45,29 @@ struct __align__(16) Smem {
     float S[D * D];  // the head's state, row i = key channel i
     float q[D], k[D], v[D], a[D], u[D], o[D];
     float red[2][Lay<D>::RG][D];
-    float wsum[2][8];
+    float wsum[2][2][8];  // two buffers: consecutive sums alternate (see sum2_first_d)
     uint64_t bar;
 };
 
-// Sum of (x, y) over threads 0..D-1 in a fixed tree (same order on every call).
+// Sum of (x, y) over threads 0..D-1 in a fixed tree (same order on every call). Consecutive calls
+// alternate between the two wsum buffers (the caller's parity `par`, flipped here), so one barrier
+// per call suffices: a buffer is written again two calls later, and every thread has finished
+// reading it before it arrives at the barrier of the call in between.
 template <int D>
-__device__ __forceinline__ float2 sum2_first_d(float x, float y, Smem<D> &sm) {
+__device__ __forceinline__ float2 sum2_first_d(float x, float y, Smem<D> &sm, int &par) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, o));
         y = __fadd_rn(y, __shfl_xor_sync(0xffffffffu, y, o));
     }
-    if (lane == 0 && w < Lay<D>::NW) { sm.wsum[0][w] = x; sm.wsum[1][w] = y; }
+    float(&ws)[2][8] = sm.wsum[par];
+    par ^= 1;
+    if (lane == 0 && w < Lay<D>::NW) { ws[0][w] = x; ws[1][w] = y; }
     __syncthreads();
-    float sx = sm.wsum[0][0], sy = sm.wsum[1][0];
+    float sx = ws[0][0], sy = ws[1][0];
 #pragma unroll
-    for (int i = 1; i < Lay<D>::NW; ++i) { sx = __fadd_rn(sx, sm.wsum[0][i]); sy = __fadd_rn(sy, sm.wsum[1][i]); }
-    __syncthreads();
+    for (int i = 1; i < Lay<D>::NW; ++i) { sx = __fadd_rn(sx, ws[0][i]); sy = __fadd_rn(sy, ws[1][i]); }
     return make_float2(sx, sy);
 }
 
@@ -207,7 +211,8 @@ recurrent_decode_kernel(const float *__restrict__ q, const float *__restrict__ k
         sm.a[tid] = expf(gate[row + tid]);
         qk = __fmul_rn(qd, kd);
     }
-    const float kq = sum2_first_d<D>(tid < D ? qk : 0.f, 0.f, sm).x;
+    int spar = 0;
+    const float kq = sum2_first_d<D>(tid < D ? qk : 0.f, 0.f, sm, spar).x;
     if (!state_ready<D>(sm, status)) return;
     state_step<D>(sm, bt, kq, scale, false, S, nullptr);
     if (tid < D) o[row + tid] = sm.o[tid];
@@ -292,18 +297,27 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
     const float dtb = qk_thread ? p.dt_bias[h * D + d] : 0.f;
     const float ow = qk_thread && p.o_norm_w ? bf16_to_f32(p.o_norm_w[d]) : 0.f;
     bool ok = true;
+    int spar = 0;  // wsum buffer parity of the next block sum
 
+    // every global input of a row (none depends on the state): the next row's are requested while
+    // the current one runs
+    uint16_t nx0 = 0, nx1 = 0, ngr = 0, nog = 0;
+    float nbl = 0.f;
+    auto load_row = [&](size_t row) {
+        if (qk_thread || v_thread) nx0 = p.x[row * 3 * qkv + c0];
+        if (qk_thread) {
+            nx1 = p.x[row * 3 * qkv + c1];
+            ngr = p.g_raw[row * qkv + h * D + d];
+            nog = p.out_gate[row * qkv + h * D + d];
+        }
+        nbl = p.b_logit[row * H + h];
+    };
+    load_row(rbase);
     for (int t = 0; t < nrows; ++t) {
         const size_t row = rbase + t;
-        // every global input of the row, loaded up front (they do not depend on the state)
-        float x0 = 0.f, x1 = 0.f, graw = 0.f, og = 0.f;
-        if (qk_thread || v_thread) x0 = bf16_to_f32(p.x[row * 3 * qkv + c0]);
-        if (qk_thread) {
-            x1 = bf16_to_f32(p.x[row * 3 * qkv + c1]);
-            graw = bf16_to_f32(p.g_raw[row * qkv + h * D + d]);
-            og = bf16_to_f32(p.out_gate[row * qkv + h * D + d]);
-        }
-        const float blog = p.b_logit[row * H + h];
+        const float x0 = bf16_to_f32(nx0), x1 = bf16_to_f32(nx1), graw = bf16_to_f32(ngr), og = bf16_to_f32(nog);
+        const float blog = nbl;
+        if (t + 1 < nrows) load_row(row + 1);
         // conv step + SiLU (fixed-order FP32), new conv state in registers
         float y0 = 0.f, y1 = 0.f;
         if (qk_thread || v_thread) {
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
             }
         }
         // per-head L2 of q and k (one BF16 rounding after the norm), v rounded as is
-        const float2 ss = sum2_first_d<D>(qk_thread ? __fmul_rn(y0, y0) : 0.f, qk_thread ? __fmul_rn(y1, y1) : 0.f, sm);
+        const float2 ss = sum2_first_d<D>(qk_thread ? __fmul_rn(y0, y0) : 0.f, qk_thread ? __fmul_rn(y1, y1) : 0.f, sm, spar);
         float qv = 0.f, kv = 0.f;
         if (qk_thread) {
             const uint16_t qb = f32_to_bf16(__fmul_rn(y0, rsqrtf(__fadd_rn(ss.x, p.l2_eps))));
@@ -333,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
             if (p.conv_out) p.conv_out[row * 3 * qkv + c0] = vb;
         }
         const float beta = sigmoid_rn(blog);
-        const float kq = sum2_first_d<D>(qk_thread ? __fmul_rn(qv, kv) : 0.f, 0.f, sm).x;
+        const float kq = sum2_first_d<D>(qk_thread ? __fmul_rn(qv, kv) : 0.f, 0.f, sm, spar).x;
         if (t == 0) {
             ok = state_ready<D>(sm, p.status);
             if (!ok) break;  // block-uniform
@@ -345,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
         state_step<D>(sm, beta, kq, p.scale, p.verify || !last, S, snap);  // sm.o is complete when it returns
         // o_norm: sigmoid-gated RMSNorm over the head's D outputs (skipped by a fold)
         const float ov = qk_thread ? sm.o[d] : 0.f;
-        const float ms = p.o_norm_out ? sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm).x : 0.f;
+        const float ms = p.o_norm_out ? sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm, spar).x : 0.f;
         if (qk_thread && p.o_norm_out) {
             const float rs = rsqrtf(__fadd_rn(__fmul_rn(ms, 1.0f / D), p.rms_eps));
             const float yv = __fmul_rn(__fmul_rn(__fmul_rn(ov, rs), ow), sigmoid_rn(og));
