@@ -43,7 +43,7 @@ struct Lay {
 template <int D>
 struct __align__(16) Smem {
     float S[D * D];  // the head's state, row i = key channel i
-    float q[D], k[D], v[D], a[D], u[D], o[D];
+    float q[D], k[D], v[D], a[D], o[D];
     float red[2][Lay<D>::RG][D];
     float wsum[2][2][8];  // two buffers: consecutive sums alternate (see sum2_first_d)
     uint64_t bar;
@@ -99,7 +99,7 @@ __device__ __forceinline__ bool state_load_wait(Smem<D> &sm) {
 
 // One recurrence step on the shared-memory state, with q,k,v,a(=exp g) in shared memory:
 //   S' = diag(a) S;  y_k = S'^T k, y_q = S'^T q;  u = beta (v - y_k);  S = S' + k u^T;
-//   o = scale (y_q + (k.q) u)   (= scale S^T q after the update).   o lands in sm.o.
+//   o = scale (y_q + (k.q) u)   (= scale S^T q after the update): thread j < D stores o[j] to sm.o[j].
 // The decayed value S'[i][j] is formed twice (once per pass) by the same rounded product.
 // Pass 2 writes the new state to shared memory (keep), to global memory (g, streaming), to
 // a snapshot (snap, plain stores), in any combination.
@@ -119,16 +119,13 @@ __device__ __forceinline__ void state_step(Smem<D> &sm, float beta, float kq, fl
     sm.red[0][grp][j] = pk;
     sm.red[1][grp][j] = pq;
     __syncthreads();
-    if (tid < D) {
-        float yk = sm.red[0][0][tid], yq = sm.red[1][0][tid];
+    // every thread of column j forms u[j] itself, by the same fixed-order sums, so pass 2 needs no
+    // second barrier; thread j < D also publishes o[j]
+    float yk = sm.red[0][0][j], yq = sm.red[1][0][j];
 #pragma unroll
-        for (int gg = 1; gg < L::RG; ++gg) { yk = __fadd_rn(yk, sm.red[0][gg][tid]); yq = __fadd_rn(yq, sm.red[1][gg][tid]); }
-        const float u = __fmul_rn(beta, __fsub_rn(sm.v[tid], yk));
-        sm.u[tid] = u;
-        sm.o[tid] = __fmul_rn(scale, __fmaf_rn(kq, u, yq));
-    }
-    __syncthreads();
-    const float u = sm.u[j];
+    for (int gg = 1; gg < L::RG; ++gg) { yk = __fadd_rn(yk, sm.red[0][gg][j]); yq = __fadd_rn(yq, sm.red[1][gg][j]); }
+    const float u = __fmul_rn(beta, __fsub_rn(sm.v[j], yk));
+    if (tid < D) sm.o[tid] = __fmul_rn(scale, __fmaf_rn(kq, u, yq));
     if (!keep) {
 #pragma unroll 16
         for (int r = 0; r < L::RPG; ++r) {
@@ -356,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
         // a verify keeps it in shared memory throughout
         const bool last = t == nrows - 1;
         float *snap = !last && t < p.n_snap ? p.h_snap[t] + static_cast<size_t>(h) * D * D : nullptr;
-        state_step<D>(sm, beta, kq, p.scale, p.verify || !last, S, snap);  // sm.o is complete when it returns
+        state_step<D>(sm, beta, kq, p.scale, p.verify || !last, S, snap);  // sm.o[d] (this thread's) is set
         // o_norm: sigmoid-gated RMSNorm over the head's D outputs (skipped by a fold)
         const float ov = qk_thread ? sm.o[d] : 0.f;
         const float ms = p.o_norm_out ? sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm, spar).x : 0.f;
