@@ -43,7 +43,7 @@ struct Lay {
 template <int D>
 struct __align__(16) Smem {
     float S[D * D];  // the head's state, row i = key channel i
-    float q[D], k[D], v[D], a[D], o[D];
+    float q[2][D], k[2][D], v[2][D], a[2][D], o[D];  // a row's vectors, in two slots (rows alternate)
     float red[2][Lay<D>::RG][D];
     float wsum[2][2][8];  // two buffers: consecutive sums alternate (see sum2_first_d)
     uint64_t bar;
@@ -112,9 +112,9 @@ __device__ __forceinline__ void state_step(Smem<D> &sm, float beta, float kq, fl
 #pragma unroll 16
     for (int r = 0; r < L::RPG; ++r) {
         const int i = r0 + r;
-        const float s = __fmul_rn(sm.S[i * D + j], sm.a[i]);
-        pk = __fmaf_rn(s, sm.k[i], pk);
-        pq = __fmaf_rn(s, sm.q[i], pq);
+        const float s = __fmul_rn(sm.S[i * D + j], sm.a[0][i]);
+        pk = __fmaf_rn(s, sm.k[0][i], pk);
+        pq = __fmaf_rn(s, sm.q[0][i], pq);
     }
     sm.red[0][grp][j] = pk;
     sm.red[1][grp][j] = pq;
@@ -124,19 +124,19 @@ __device__ __forceinline__ void state_step(Smem<D> &sm, float beta, float kq, fl
     float yk = sm.red[0][0][j], yq = sm.red[1][0][j];
 #pragma unroll
     for (int gg = 1; gg < L::RG; ++gg) { yk = __fadd_rn(yk, sm.red[0][gg][j]); yq = __fadd_rn(yq, sm.red[1][gg][j]); }
-    const float u = __fmul_rn(beta, __fsub_rn(sm.v[j], yk));
+    const float u = __fmul_rn(beta, __fsub_rn(sm.v[0][j], yk));
     if (tid < D) sm.o[tid] = __fmul_rn(scale, __fmaf_rn(kq, u, yq));
     if (!keep) {
 #pragma unroll 16
         for (int r = 0; r < L::RPG; ++r) {
             const int i = r0 + r;
-            __stcs(g + i * D + j, __fmaf_rn(sm.k[i], u, __fmul_rn(sm.S[i * D + j], sm.a[i])));
+            __stcs(g + i * D + j, __fmaf_rn(sm.k[0][i], u, __fmul_rn(sm.S[i * D + j], sm.a[0][i])));
         }
     } else if (snap) {
 #pragma unroll 16
         for (int r = 0; r < L::RPG; ++r) {
             const int i = r0 + r;
-            const float x = __fmaf_rn(sm.k[i], u, __fmul_rn(sm.S[i * D + j], sm.a[i]));
+            const float x = __fmaf_rn(sm.k[0][i], u, __fmul_rn(sm.S[i * D + j], sm.a[0][i]));
             sm.S[i * D + j] = x;
             snap[i * D + j] = x;
         }
@@ -144,9 +144,106 @@ __device__ __forceinline__ void state_step(Smem<D> &sm, float beta, float kq, fl
 #pragma unroll 16
         for (int r = 0; r < L::RPG; ++r) {
             const int i = r0 + r;
-            sm.S[i * D + j] = __fmaf_rn(sm.k[i], u, __fmul_rn(sm.S[i * D + j], sm.a[i]));
+            sm.S[i * D + j] = __fmaf_rn(sm.k[0][i], u, __fmul_rn(sm.S[i * D + j], sm.a[0][i]));
         }
     }
+}
+
+// The stateful rows' two passes over the shared-memory state, with a row's q, k, v, a in slot b:
+//   row_reduce   pass 1 of a row: y_k = S'^T k, y_q = S'^T q (S' = diag(a) S), then this thread's
+//                column's u and, for thread j < D, o[j] (returned in o);
+//   row_update   pass 2 of a row: S = S' + k u^T, to shared memory (keep; and snap), or streamed
+//                to g; fused, when `next`, with pass 1 of the following row (slot nb) on the new
+//                values, so a row reads the state once and writes it once.
+// The same rounded operations, in the same order, as state_step: the bits do not depend on the
+// fusion.
+template <int D>
+__device__ __forceinline__ float row_finish(Smem<D> &sm, int b, float pk, float pq, float beta, float kq, float scale,
+                                            float &o) {
+    using L = Lay<D>;
+    const int tid = threadIdx.x, j = tid % D, grp = tid / D;
+    sm.red[0][grp][j] = pk;
+    sm.red[1][grp][j] = pq;
+    __syncthreads();
+    float yk = sm.red[0][0][j], yq = sm.red[1][0][j];
+#pragma unroll
+    for (int gg = 1; gg < L::RG; ++gg) { yk = __fadd_rn(yk, sm.red[0][gg][j]); yq = __fadd_rn(yq, sm.red[1][gg][j]); }
+    const float u = __fmul_rn(beta, __fsub_rn(sm.v[b][j], yk));
+    o = __fmul_rn(scale, __fmaf_rn(kq, u, yq));
+    return u;
+}
+
+// Four consecutive entries of a row vector (every lane reads the same ones: one broadcast).
+__device__ __forceinline__ void ld4(const float *p, float (&x)[4]) {
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+
+template <int D>
+__device__ __forceinline__ float row_reduce(Smem<D> &sm, int b, float beta, float kq, float scale, float &o) {
+    using L = Lay<D>;
+    const int tid = threadIdx.x, j = tid % D, r0 = (tid / D) * L::RPG;
+    float pk = 0.f, pq = 0.f;
+#pragma unroll 4
+    for (int r = 0; r < L::RPG; r += 4) {
+        float a4[4], k4[4], q4[4];
+        ld4(&sm.a[b][r0 + r], a4);
+        ld4(&sm.k[b][r0 + r], k4);
+        ld4(&sm.q[b][r0 + r], q4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float s = __fmul_rn(sm.S[(r0 + r + e) * D + j], a4[e]);
+            pk = __fmaf_rn(s, k4[e], pk);
+            pq = __fmaf_rn(s, q4[e], pq);
+        }
+    }
+    return row_finish<D>(sm, b, pk, pq, beta, kq, scale, o);
+}
+
+template <int D>
+__device__ __forceinline__ float row_update(Smem<D> &sm, int b, float u, bool keep, float *g, float *snap, bool next,
+                                            int nb, float beta_n, float kq_n, float scale, float &o_n) {
+    using L = Lay<D>;
+    const int tid = threadIdx.x, j = tid % D, r0 = (tid / D) * L::RPG;
+    float pk = 0.f, pq = 0.f;
+    if (!keep) {
+#pragma unroll 4
+        for (int r = 0; r < L::RPG; r += 4) {
+            float a4[4], k4[4];
+            ld4(&sm.a[b][r0 + r], a4);
+            ld4(&sm.k[b][r0 + r], k4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = r0 + r + e;
+                __stcs(g + i * D + j, __fmaf_rn(k4[e], u, __fmul_rn(sm.S[i * D + j], a4[e])));
+            }
+        }
+        return 0.f;
+    }
+#pragma unroll 4
+    for (int r = 0; r < L::RPG; r += 4) {
+        float a4[4], k4[4], an[4], kn[4], qn[4];
+        ld4(&sm.a[b][r0 + r], a4);
+        ld4(&sm.k[b][r0 + r], k4);
+        if (next) {
+            ld4(&sm.a[nb][r0 + r], an);
+            ld4(&sm.k[nb][r0 + r], kn);
+            ld4(&sm.q[nb][r0 + r], qn);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = r0 + r + e;
+            const float x = __fmaf_rn(k4[e], u, __fmul_rn(sm.S[i * D + j], a4[e]));
+            sm.S[i * D + j] = x;
+            if (snap) snap[i * D + j] = x;
+            if (next) {
+                const float s = __fmul_rn(x, an[e]);
+                pk = __fmaf_rn(s, kn[e], pk);
+                pq = __fmaf_rn(s, qn[e], pq);
+            }
+        }
+    }
+    return next ? row_finish<D>(sm, nb, pk, pq, beta_n, kq_n, scale, o_n) : 0.f;
 }
 
 __device__ __forceinline__ float sigmoid_rn(float x) {
@@ -204,8 +301,8 @@ recurrent_decode_kernel(const float *__restrict__ q, const float *__restrict__ k
     float qk = 0.f;
     if (tid < D) {
         const float qd = q[row + tid], kd = k[row + tid];
-        sm.q[tid] = qd; sm.k[tid] = kd; sm.v[tid] = v[row + tid];
-        sm.a[tid] = expf(gate[row + tid]);
+        sm.q[0][tid] = qd; sm.k[0][tid] = kd; sm.v[0][tid] = v[row + tid];
+        sm.a[0][tid] = expf(gate[row + tid]);
         qk = __fmul_rn(qd, kd);
     }
     int spar = 0;
@@ -310,9 +407,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
         nbl = p.b_logit[row * H + h];
     };
     load_row(rbase);
-    for (int t = 0; t < nrows; ++t) {
+    // The front of a row (conv step, SiLU, q|k L2, gate, beta, k.q) into slot t & 1, its conv_out
+    // and conv snapshot; returns the row's beta and k.q, and its output gate for the o_norm.
+    float og_t = 0.f;
+    auto front = [&](int t, float &beta, float &kq, float &og) {
         const size_t row = rbase + t;
-        const float x0 = bf16_to_f32(nx0), x1 = bf16_to_f32(nx1), graw = bf16_to_f32(ngr), og = bf16_to_f32(nog);
+        const int b = t & 1;
+        const float x0 = bf16_to_f32(nx0), x1 = bf16_to_f32(nx1), graw = bf16_to_f32(ngr);
+        og = bf16_to_f32(nog);
         const float blog = nbl;
         if (t + 1 < nrows) load_row(row + 1);
         // conv step + SiLU (fixed-order FP32), new conv state in registers
@@ -334,35 +436,17 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
             const uint16_t qb = f32_to_bf16(__fmul_rn(y0, rsqrtf(__fadd_rn(ss.x, p.l2_eps))));
             const uint16_t kb = f32_to_bf16(__fmul_rn(y1, rsqrtf(__fadd_rn(ss.y, p.l2_eps))));
             qv = bf16_to_f32(qb); kv = bf16_to_f32(kb);
-            sm.q[d] = qv; sm.k[d] = kv;
+            sm.q[b][d] = qv; sm.k[b][d] = kv;
             if (p.conv_out) { p.conv_out[row * 3 * qkv + c0] = qb; p.conv_out[row * 3 * qkv + c1] = kb; }
             // gate for key channel d
-            sm.a[d] = expf(kda_gate_f32(graw, dtb, nea));
+            sm.a[b][d] = expf(kda_gate_f32(graw, dtb, nea));
         } else if (v_thread) {
             const uint16_t vb = f32_to_bf16(y0);
-            sm.v[d] = bf16_to_f32(vb);
+            sm.v[b][d] = bf16_to_f32(vb);
             if (p.conv_out) p.conv_out[row * 3 * qkv + c0] = vb;
         }
-        const float beta = sigmoid_rn(blog);
-        const float kq = sum2_first_d<D>(qk_thread ? __fmul_rn(qv, kv) : 0.f, 0.f, sm, spar).x;
-        if (t == 0) {
-            ok = state_ready<D>(sm, p.status);
-            if (!ok) break;  // block-uniform
-        }
-        // the last row streams the state out; earlier rows keep it (and write their snapshot);
-        // a verify keeps it in shared memory throughout
-        const bool last = t == nrows - 1;
-        float *snap = !last && t < p.n_snap ? p.h_snap[t] + static_cast<size_t>(h) * D * D : nullptr;
-        state_step<D>(sm, beta, kq, p.scale, p.verify || !last, S, snap);  // sm.o[d] (this thread's) is set
-        // o_norm: sigmoid-gated RMSNorm over the head's D outputs (skipped by a fold)
-        const float ov = qk_thread ? sm.o[d] : 0.f;
-        const float ms = p.o_norm_out ? sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm, spar).x : 0.f;
-        if (qk_thread && p.o_norm_out) {
-            const float rs = rsqrtf(__fadd_rn(__fmul_rn(ms, 1.0f / D), p.rms_eps));
-            const float yv = __fmul_rn(__fmul_rn(__fmul_rn(ov, rs), ow), sigmoid_rn(og));
-            p.o_norm_out[row * qkv + h * D + d] = f32_to_bf16(yv);
-            if (p.core) p.core[row * qkv + h * D + d] = ov;
-        }
+        beta = sigmoid_rn(blog);
+        kq = sum2_first_d<D>(qk_thread ? __fmul_rn(qv, kv) : 0.f, 0.f, sm, spar).x;
         if (t < p.n_snap) {
             uint16_t *cs = p.conv_snap[t];
             if (qk_thread || v_thread) {
@@ -374,6 +458,37 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rows_kernel(const RowParam
                 }
             }
         }
+    };
+    float beta_t, kq_t, o_t = 0.f;
+    front(0, beta_t, kq_t, og_t);
+    ok = state_ready<D>(sm, p.status);
+    float u_t = 0.f;
+    if (ok) u_t = row_reduce<D>(sm, 0, beta_t, kq_t, p.scale, o_t);
+    for (int t = 0; t < nrows && ok; ++t) {
+        const size_t row = rbase + t;
+        const bool next = t + 1 < nrows;
+        // the next row's front: its slot is free (the pass that last read it has finished)
+        float beta_n = 0.f, kq_n = 0.f, og_n = 0.f;
+        if (next) front(t + 1, beta_n, kq_n, og_n);
+        // o_norm of this row: sigmoid-gated RMSNorm over the head's D outputs (skipped by a fold)
+        const float ov = qk_thread ? o_t : 0.f;
+        const float ms = p.o_norm_out ? sum2_first_d<D>(qk_thread ? __fmul_rn(ov, ov) : 0.f, 0.f, sm, spar).x : 0.f;
+        if (qk_thread && p.o_norm_out) {
+            const float rs = rsqrtf(__fadd_rn(__fmul_rn(ms, 1.0f / D), p.rms_eps));
+            const float yv = __fmul_rn(__fmul_rn(__fmul_rn(ov, rs), ow), sigmoid_rn(og_t));
+            p.o_norm_out[row * qkv + h * D + d] = f32_to_bf16(yv);
+            if (p.core) p.core[row * qkv + h * D + d] = ov;
+        }
+        // this row's update, fused with the next row's first pass. The last row streams the state
+        // out; earlier rows keep it (and write their snapshot); a verify leaves it (its last row
+        // is not even applied)
+        if (next || !p.verify) {
+            float *snap = next && t < p.n_snap ? p.h_snap[t] + static_cast<size_t>(h) * D * D : nullptr;
+            float o_n = 0.f;
+            u_t = row_update<D>(sm, t & 1, u_t, next, S, snap, next, (t + 1) & 1, beta_n, kq_n, p.scale, o_n);
+            o_t = o_n;
+        }
+        og_t = og_n;
     }
     if (!ok || p.verify) return;  // a verify leaves the conv state too
     if (qk_thread || v_thread) {
