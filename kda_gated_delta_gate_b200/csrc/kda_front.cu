@@ -259,13 +259,24 @@ front_varlen_kernel(const uint16_t *__restrict__ x, uint16_t *const *__restrict_
     int b = lo, s0 = 0, s1 = 0;
     float xm[3][8];
     if (t0 >= tend || !enter_seq(x, conv_state, cu, b, t0, total, cd, c0, s0, s1, xm, status)) return;
-    for (int t = t0; t < tend; ++t) {
+    // rows four at a time: their loads go out together (the sequence switch inside would keep
+    // the compiler from hoisting them)
+    for (int t4 = t0; t4 < tend; t4 += 4) {
+      uint4 raw[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+          raw[q] = t4 + q < tend ? *reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t4 + q) * cd + c0)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = t4 + q;
+        if (t >= tend) break;
         if (t == s1) {  // the next non-empty sequence starts here
             while (b < B - 1 && cu[b + 1] <= t) ++b;
             if (!enter_seq(x, conv_state, cu, b, t, total, cd, c0, s0, s1, xm, status)) return;
         }
         float xc[8], c[8];
-        unpack8(*reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * cd + c0), xc);
+        unpack8(raw[q], xc);
         float ss = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -287,6 +298,7 @@ front_varlen_kernel(const uint16_t *__restrict__ x, uint16_t *const *__restrict_
         if (valid)
             *reinterpret_cast<uint4 *>(conv_out + static_cast<size_t>(t) * cd + c0) =
                 make_uint4(pack2(ob[0], ob[1]), pack2(ob[2], ob[3]), pack2(ob[4], ob[5]), pack2(ob[6], ob[7]));
+      }
     }
 }
 
