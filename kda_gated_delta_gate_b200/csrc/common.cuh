@@ -184,6 +184,16 @@ struct GemvSegs {
 };
 int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
               int out_f32, cudaStream_t s);
+// Up to six products C_i = A_i . W_i^T of one width N and depth K (M may differ) in one launch.
+struct GemmProd {
+    const uint16_t *A;
+    int lda;
+    const uint16_t *W;
+    int ldw;
+    void *C;
+    int ldc, M, N, K, out_f32;
+};
+int gemm_bf16_multi(const GemmProd *prods, int n, cudaStream_t s);
 // A few input rows (at most 256) against up to six weights in one launch, each weight read
 // once: y[m][n] = x[m] . W[n] for m < rows, n < N (rows of y at stride ldy), on the tensor
 // cores with the weights' rows as the 128-row tiles. Not the matrix-vector kernel's bits.

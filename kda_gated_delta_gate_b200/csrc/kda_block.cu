@@ -165,17 +165,21 @@ int prefill_projections(const kda_block_weights *w, const kda_bf16 *hidden, int 
     const int Hd = ws->hidden, R = ws->rank, H = d->heads, qkv = d->heads * d->head_dim, cd = 3 * qkv;
     auto bf = [&](int i) { return static_cast<uint16_t *>(ws->buf[i]); };
     auto f32 = [&](int i) { return static_cast<float *>(ws->buf[i]); };
-    // q | k | v projections straight into the packed qkv_proj rows
-    KDA_TRY(gemm_bf16(hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, T, qkv, Hd, 0, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, T, qkv, Hd, 0, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, T, qkv, Hd, 0, s));
-    // forget-gate input: g_raw = f_b(f_a(h)) (the gate itself is formed inside the chunked core)
-    KDA_TRY(gemm_bf16(hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, T, R, Hd, 0, s));
-    KDA_TRY(gemm_bf16(bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, T, qkv, R, 0, s));
-    // beta logits (FP32), the output gate's low-rank pair
-    KDA_TRY(gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, T, H, Hd, 1, s));
-    KDA_TRY(gemm_bf16(hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, T, R, Hd, 0, s));
-    return gemm_bf16(bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0, s);
+    // q | k | v projections straight into the packed qkv_proj rows, one launch
+    const GemmProd p_qkv[3] = {{hidden, Hd, w->q_proj, Hd, bf(KDA_BUF_QKV_PROJ), cd, T, qkv, Hd, 0},
+                               {hidden, Hd, w->k_proj, Hd, bf(KDA_BUF_QKV_PROJ) + qkv, cd, T, qkv, Hd, 0},
+                               {hidden, Hd, w->v_proj, Hd, bf(KDA_BUF_QKV_PROJ) + 2 * qkv, cd, T, qkv, Hd, 0}};
+    KDA_TRY(gemm_bf16_multi(p_qkv, 3, s));
+    // the two low-rank pairs: forget-gate input g_raw = f_b(f_a(h)) (the gate itself is formed
+    // inside the chunked core) and the output gate g_b(g_a(h)), each stage of both in one launch
+    const GemmProd p_a[2] = {{hidden, Hd, w->f_a, Hd, bf(KDA_BUF_F_A_OUT), R, T, R, Hd, 0},
+                             {hidden, Hd, w->g_a, Hd, bf(KDA_BUF_G_A_OUT), R, T, R, Hd, 0}};
+    KDA_TRY(gemm_bf16_multi(p_a, 2, s));
+    const GemmProd p_b[2] = {{bf(KDA_BUF_F_A_OUT), R, w->f_b, R, bf(KDA_BUF_G_RAW), qkv, T, qkv, R, 0},
+                             {bf(KDA_BUF_G_A_OUT), R, w->g_b, R, bf(KDA_BUF_OUT_GATE), qkv, T, qkv, R, 0}};
+    KDA_TRY(gemm_bf16_multi(p_b, 2, s));
+    // beta logits (FP32)
+    return gemm_bf16(hidden, Hd, w->b_proj, Hd, f32(KDA_BUF_BETA), H, T, H, Hd, 1, s);
 }
 
 // gated RMSNorm of `rows` core rows, then o_proj (GEMM) unless the caller applies its own.

@@ -356,6 +356,26 @@ int gemm_one(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout,
     return launch_gemm<BN>(g, s);
 }
 
+// Several products of one width N and depth K in one launch: their tiles follow one another in the
+// tile order, so the launch fills the machine where each alone would leave SMs idle or a ragged
+// last wave. Each tile runs exactly as it would in its own launch.
+template <int BN>
+int gemm_multi(const GemmProd *prods, int n, cudaStream_t s) {
+    GemmArgs g{};
+    for (int i = 0; i < n; ++i) {
+        const GemmProd &p = prods[i];
+        KDA_TRY(make_map(&g.tmA[i], p.A, p.M, p.K, p.lda, BM));
+        KDA_TRY(make_map(&g.tmW[i], p.W, p.N, p.K, p.ldw, BN));
+        g.seg[i] = GemmSeg{p.C, p.ldc, p.M, p.out_f32, aligned16(p.C) && (p.ldc % (p.out_f32 ? 4 : 8)) == 0};
+    }
+    g.nseg = n;
+    g.N = prods[0].N;
+    g.K = prods[0].K;
+    g.trans = 0;
+    g.ksplit = 1;
+    return launch_gemm<BN>(g, s);
+}
+
 // The small-M form: y_s[m][n] = x_s[m] . W_s[n] for a few rows m of each segment's input, as
 // the transposed product W_s . x_s^T, so that the 128-row tiles run over the weights' output
 // rows (every weight is read once, by many CTAs) and the few input rows are the N side.
@@ -396,6 +416,17 @@ int gemm_small_m(const GemmTSeg *segs, int nseg, int rows, int K, float *part, s
 }
 
 }  // namespace
+
+int gemm_bf16_multi(const GemmProd *prods, int n, cudaStream_t s) {
+    if (n < 1 || n > kMaxGemmSegs) return KDA_ERR_INVALID_ARG;
+    for (int i = 1; i < n; ++i)
+        if (prods[i].N != prods[0].N || prods[i].K != prods[0].K) return KDA_ERR_INVALID_ARG;
+    const int N = prods[0].N;
+    if (N > 128) return gemm_multi<256>(prods, n, s);
+    if (N > 64) return gemm_multi<128>(prods, n, s);
+    if (N > 32) return gemm_multi<64>(prods, n, s);
+    return gemm_multi<32>(prods, n, s);
+}
 
 int gemm_bf16(const uint16_t *A, int lda, const uint16_t *W, int ldw, void *Cout, int ldc, int M, int N, int K,
               int out_f32, cudaStream_t s) {
