@@ -63,7 +63,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     return true;
 }
 
-// Up to three products in one launch, each its own A (M rows) and W (the shared N rows), its own
+// Up to six products in one launch, each its own A (M rows) and W (the shared N rows), its own
 // output: a segment's tiles follow the previous segment's in the tile order. trans: element
 // (m, n) of a product is stored at C[n ldc + m] (the small-M form below computes C^T).
 constexpr int kMaxGemmSegs = 6;
