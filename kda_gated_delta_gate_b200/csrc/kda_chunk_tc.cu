@@ -71,6 +71,14 @@ struct PrefillIn {
     int stream_pack;  // the call's operand packs overflow L2: store them evict-first
 };
 
+// Programmatic dependent launch: the kernels of a call run back to back with the next one
+// launched as soon as every CTA of the current one has started (pdl_release at the start), so
+// its launch and its set-up that reads nothing the current one writes overlap the current
+// one's tail; pdl_acquire waits until the previous kernel has completed and its memory is
+// visible. A kernel launched without the attribute passes both at once.
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_acquire() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // L2 eviction policies (createpolicy): evict-first for data read or written for the last time
 // in this pass, so that the inputs prefetched for the coming items keep their place in L2.
 __device__ __forceinline__ uint64_t l2_policy(bool evict_first) {
@@ -597,6 +605,8 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
 intra_fix_kernel(const PrefillIn in, uint8_t *__restrict__ scratch, const int *__restrict__ list, const Seqs sq,
                  int H) {
     extern __shared__ float smem[];
+    pdl_release();
+    pdl_acquire();  // the tensor-core pass has listed its chunks
     const int count = list[0];
     const int nch = sq.nch;
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
@@ -695,6 +705,7 @@ intra_tc_kernel(const __grid_constant__ InMaps maps, const PrefillIn in, uint8_t
     constexpr int UB = C * (D / 8) / NT;  // (token, 8-channel group) units per thread over all D channels
     constexpr bool QKV16 = kQkv16<MODE>, GRAW = kGraw<MODE>;
     extern __shared__ uint8_t smem_raw[];
+    pdl_release();  // the fix-up pass may launch (it waits for this pass to complete)
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = sm, *sBt = sm + I::A_H, *sR2 = sm + I::OFF_R2, *sTb = sm + I::OFF_TB, *sKA = sm;
     float *sG = reinterpret_cast<float *>(sR2);
@@ -1259,9 +1270,6 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
         mbar_init(&bars[12], 1);
         *fail = 0;
         fence_mbar_init();
-        for (int part = 0; part < kA1Parts; ++part) copy_a1(packs, part);
-        copy_m(packs);
-        bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[2]);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -1301,6 +1309,13 @@ state_kernel(const uint8_t *__restrict__ scratch, float *const *__restrict__ h_s
             tmem_st8(tS + j, x);
         }
         tmem_st_wait();
+    }
+    // the packs: written by the passes before this one (everything above reads none of them)
+    pdl_acquire();
+    if (ctl) {
+        for (int part = 0; part < kA1Parts; ++part) copy_a1(packs, part);
+        copy_m(packs);
+        bulk_copy(sA3, packs + PK::OFF_A3, PK::A3, &bars[2]);
     }
     fence_async_smem();
     tc_fence_before();
@@ -1636,10 +1651,25 @@ int launch_tc(const PrefillIn &in, float *const *h_state, float *core, int B, co
     inp.stream_pack = packs_bytes<D>(pack_count(B, H, sq)) > (size_t{64} << 20) ? 1 : 0;
     intra_tc_kernel<D, MODE><<<grid, kTcThreads, IntraTC<D>::bytes, s>>>(maps, inp, sc, list, B, sq, H, status);
     KDA_TRY(launch_status());
-    intra_fix_kernel<D, MODE><<<grid_fix, kIntraThreads, Intra<D>::bytes, s>>>(in, sc, list, sq, H);
-    KDA_TRY(launch_status());
-    state_kernel<D, DVS><<<dim3(D / DVS, H, B), kStateThreadsFor<DVS>, State<D, DVS>::bytes, s>>>(sc, h_state, core, sq, H, scale,
-                                                                                   in.tables, status);
+    // the fix-up and state passes launch programmatically: each waits in-kernel for its predecessor
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(kIntraThreads);
+    cfg.gridDim = dim3(grid_fix);
+    cfg.dynamicSmemBytes = Intra<D>::bytes;
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, intra_fix_kernel<D, MODE>, in, sc, static_cast<const int *>(list), sq, H) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    cfg.blockDim = dim3(kStateThreadsFor<DVS>);
+    cfg.gridDim = dim3(D / DVS, H, B);
+    cfg.dynamicSmemBytes = State<D, DVS>::bytes;
+    if (cudaLaunchKernelEx(&cfg, state_kernel<D, DVS>, static_cast<const uint8_t *>(sc), h_state, core, sq, H, scale,
+                           in.tables, status) != cudaSuccess)
+        return KDA_ERR_CUDA;
     return launch_status();
 }
 
