@@ -281,3 +281,24 @@ def test_block_verify_full_size_short_drafts():
         on, core, _, _, _ = _decode_k_rows(dw, got, sl, hs0[b], cs0[b], d)
         assert torch.equal(on, got["o_norm_out"][sl]) and torch.equal(core, got["core"][sl]), b
     ws.close()
+
+
+def test_block_fold_without_a_row_route_verify_refuses():
+    """A fold whose (B, total) picks the row-by-row route, on a workspace where no such verify ran,
+    is refused (KDA_ERR_INVALID_ARG) before any launch: both states stay."""
+    hidden, H, D, rank, lens = 256, 2, 64, 64, [3, 2]
+    B, total, cu = len(lens), sum(lens), _cu(lens)
+    d = kda.dims(H, D)
+    hs0, cs0 = _states(B, H, D, seed=49)
+    ws = kda.Workspace(d, hidden, rank, max_tokens=total, max_seqs=B)
+    hs = [hs0[b].cuda().clone() for b in range(B)]
+    cs = [cs0[b].cuda().clone() for b in range(B)]
+    tables = torch.empty(kda.kda_chunk_verify_tables_bytes(B, d) // 4, device="cuda")
+    with pytest.raises(kda.KdaError) as err:
+        kda.kda_block_verify_fold(torch.tensor(cu, dtype=torch.int32, device="cuda"),
+                                  torch.tensor([1, 1], dtype=torch.int32, device="cuda"), B, total, tables,
+                                  kda.ptr_array(hs), kda.ptr_array(cs), ws)
+    assert err.value.status == KDA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert all(torch.equal(hs[b], hs0[b].cuda()) and torch.equal(cs[b], cs0[b].cuda()) for b in range(B))
+    ws.close()
